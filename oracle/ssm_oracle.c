@@ -1,0 +1,395 @@
+/*
+ * CPU oracle for the Mamba-1 selective-SSM layer core — TEST INFRASTRUCTURE.
+ *
+ * Plain, slow, obviously-correct fp64 C. Only the tests, the smoke check and
+ * the benchmark's CPU-baseline leg may load it; the product library never
+ * does, and this file shares no code, header or table with the CUDA path.
+ *
+ * What is computed, and where the pages define it:
+ *   conv   "hung-phan ml-skills mamba", section "Mamba: Selective State
+ *          Spaces (S6)" (the SelectiveSSM sketch: depthwise Conv1d with
+ *          padding d_conv-1, output cut to the first L steps, then SiLU) and
+ *          section "Mamba Block Architecture" (Conv1d(k=4) -> SiLU).
+ *   delta  same sketch: delta = softplus(dt) "to keep the step positive";
+ *          the per-channel bias is the dt_bias of "Key Training Tips" 1.
+ *   scan   same page, "Architecture Diagram" (S6 block): A_bar = exp(delta*A),
+ *          B_bar = delta*B, h_t = A_bar*h_{t-1} + B_bar*x_t, y_t = C_t*h_t;
+ *          section "Core Concept" adds the D*x feed-through; the sketch gates
+ *          y * silu(z).
+ *   resets "FLA Mamba and Mamba2" (Axolotl), packing paragraph: convolution
+ *          and recurrent state start independently for every document.
+ *
+ * Readings taken where the pages are silent (each is listed in the design doc):
+ *   - A is passed directly (negative for the S4D-real init), not A_log.exp().
+ *   - conv taps are cross-correlation: w[d][W-1] multiplies x_t and w[d][0]
+ *     multiplies x_{t-W+1} (PyTorch Conv1d with left padding W-1).
+ *   - a document boundary is any t with seq_idx[t] != seq_idx[t-1]; a conv tap
+ *     counts only when its token is in the same segment as the output token.
+ *   - u (the conv+SiLU output) feeds both B_bar*x and D*x.
+ *   - the backward is hand-derived reverse mode of the definitions above.
+ *
+ * Threading: every core routine works on one (batch, channel) row; the *_mt
+ * drivers only hand rows to pthreads and add per-thread partial sums in a
+ * fixed order. Nothing is blocked, fused or reordered inside a row.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "ssm_oracle.h"
+
+/* ---------------------------------------------------------------- helpers */
+static double sigm(double v) { return 1.0 / (1.0 + exp(-v)); }
+
+/* softplus(v) = log(1 + exp(v)), written so that neither branch overflows. */
+static double softplus(double v) {
+    if (v > 0.0) return v + log1p(exp(-v));
+    return log1p(exp(v));
+}
+
+static int seg_of(const int32_t* seq, int L, int b, int t) {
+    return seq ? seq[(size_t)b * L + t] : 0;
+}
+
+/* Round one double to the nearest bfloat16 value (8 significant bits,
+ * ties to even). Used only to mirror where the GPU path stores bf16. */
+static double round_bf16_one(double v) {
+    if (v == 0.0 || !isfinite(v)) return v;
+    int e;
+    double m = frexp(v, &e);               /* v = m * 2^e, 0.5 <= |m| < 1 */
+    if (e < -125) {                        /* below the bf16 normal range */
+        double q = ldexp(1.0, -133);       /* bf16 subnormal spacing */
+        return nearbyint(v / q) * q;
+    }
+    double r = ldexp(nearbyint(ldexp(m, 8)), e - 8);
+    return r;
+}
+
+void oracle_round_bf16(const double* in, double* out, size_t n) {
+    for (size_t i = 0; i < n; ++i) out[i] = round_bf16_one(in[i]);
+}
+
+/* ------------------------------------------------------------- conv1d fwd */
+/* One row (b, d): c_t = bias + sum_k w[k] x_{t-W+1+k} over taps inside the
+ * sequence and the output token's segment; u_t = silu(c_t) or c_t. */
+static void conv_fwd_row(const double* x, const double* w, double bias,
+                         const int32_t* seq, int b, int L, int W, int silu,
+                         double* c, double* u) {
+    for (int t = 0; t < L; ++t) {
+        int st = seg_of(seq, L, b, t);
+        double acc = bias;
+        for (int k = 0; k < W; ++k) {
+            int s = t - (W - 1) + k;
+            if (s < 0) continue;
+            if (seg_of(seq, L, b, s) != st) continue;
+            acc += w[k] * x[s];
+        }
+        if (c) c[t] = acc;
+        u[t] = silu ? acc * sigm(acc) : acc;
+    }
+}
+
+void oracle_conv1d_fwd(const double* x, const double* w, const double* bias,
+                       const int32_t* seq, double* c, double* u,
+                       int B, int D, int L, int W, int silu) {
+    for (int b = 0; b < B; ++b)
+        for (int d = 0; d < D; ++d) {
+            size_t row = ((size_t)b * D + d) * L;
+            conv_fwd_row(x + row, w + (size_t)d * W, bias ? bias[d] : 0.0, seq,
+                         b, L, W, silu, c ? c + row : NULL, u + row);
+        }
+}
+
+/* ------------------------------------------------------------- conv1d bwd */
+/* Transpose of conv_fwd_row under the same masks. dw/dbias accumulate. */
+static void conv_bwd_row(const double* x, const double* w, double bias,
+                         const int32_t* seq, int b, int L, int W, int silu,
+                         const double* du, double* dx, double* dw, double* dbias) {
+    for (int s = 0; s < L; ++s) dx[s] = 0.0;
+    for (int t = 0; t < L; ++t) {
+        int st = seg_of(seq, L, b, t);
+        double c = bias;
+        for (int k = 0; k < W; ++k) {
+            int s = t - (W - 1) + k;
+            if (s < 0 || seg_of(seq, L, b, s) != st) continue;
+            c += w[k] * x[s];
+        }
+        double dc = du[t];
+        if (silu) {
+            double sg = sigm(c);
+            dc *= sg * (1.0 + c * (1.0 - sg));
+        }
+        *dbias += dc;
+        for (int k = 0; k < W; ++k) {
+            int s = t - (W - 1) + k;
+            if (s < 0 || seg_of(seq, L, b, s) != st) continue;
+            dx[s] += w[k] * dc;
+            dw[k] += x[s] * dc;
+        }
+    }
+}
+
+void oracle_conv1d_bwd(const double* x, const double* w, const double* bias,
+                       const int32_t* seq, const double* du, double* dx,
+                       double* dw, double* dbias, int B, int D, int L, int W,
+                       int silu) {
+    memset(dw, 0, sizeof(double) * (size_t)D * W);
+    memset(dbias, 0, sizeof(double) * (size_t)D);
+    for (int b = 0; b < B; ++b)
+        for (int d = 0; d < D; ++d) {
+            size_t row = ((size_t)b * D + d) * L;
+            conv_bwd_row(x + row, w + (size_t)d * W, bias ? bias[d] : 0.0, seq, b,
+                         L, W, silu, du + row, dx + row, dw + (size_t)d * W,
+                         dbias + d);
+        }
+}
+
+/* --------------------------------------------------------------- scan fwd */
+typedef struct {
+    const double *u, *delta, *z, *A, *Dskip, *delta_bias, *Bm, *Cm;
+    const int32_t* seq;
+    int B, D, L, N, softplus_on;
+} scan_in_t;
+
+/* delta_t for row (b, d), token t (softplus of raw + bias, or raw + bias). */
+static double delta_at(const scan_in_t* p, int d, size_t row, int t) {
+    double v = p->delta[row + t] + (p->delta_bias ? p->delta_bias[d] : 0.0);
+    return p->softplus_on ? softplus(v) : v;
+}
+
+/* One row: sequential recurrence over t, all N states. Writes out (gated),
+ * y (before the gate, optional) and the state after the last token. */
+static void scan_fwd_row(const scan_in_t* p, int b, int d, double* out,
+                         double* y_out, double* final_state) {
+    const int L = p->L, N = p->N;
+    size_t row = ((size_t)b * p->D + d) * L;
+    double* h = (double*)calloc((size_t)N, sizeof(double));
+    for (int t = 0; t < L; ++t) {
+        double dt = delta_at(p, d, row, t);
+        double ut = p->u[row + t];
+        int reset = (t > 0) && seg_of(p->seq, L, b, t) != seg_of(p->seq, L, b, t - 1);
+        double y = 0.0;
+        for (int n = 0; n < N; ++n) {
+            double abar = exp(dt * p->A[(size_t)d * N + n]);
+            double bt = p->Bm[((size_t)b * N + n) * L + t];
+            double ct = p->Cm[((size_t)b * N + n) * L + t];
+            double hprev = reset ? 0.0 : h[n];
+            h[n] = abar * hprev + dt * bt * ut;
+            y += ct * h[n];
+        }
+        if (p->Dskip) y += p->Dskip[d] * ut;
+        if (y_out) y_out[row + t] = y;
+        if (p->z) {
+            double zt = p->z[row + t];
+            out[row + t] = y * zt * sigm(zt);
+        } else {
+            out[row + t] = y;
+        }
+    }
+    if (final_state)
+        for (int n = 0; n < N; ++n) final_state[((size_t)b * p->D + d) * N + n] = h[n];
+    free(h);
+}
+
+void oracle_scan_fwd(const double* u, const double* delta, const double* z,
+                     const double* A, const double* Dskip, const double* delta_bias,
+                     const double* Bm, const double* Cm, int softplus_on,
+                     const int32_t* seq, double* out, double* y_out,
+                     double* final_state, int B, int D, int L, int N) {
+    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on};
+    for (int b = 0; b < B; ++b)
+        for (int d = 0; d < D; ++d) scan_fwd_row(&p, b, d, out, y_out, final_state);
+}
+
+/* --------------------------------------------------------------- scan bwd */
+typedef struct {
+    const double* dout;
+    double *du, *ddelta, *dz;          /* per row, overwritten */
+    double *dA, *dB, *dC, *dD, *ddb;   /* accumulated */
+} scan_grad_t;
+
+/* One row. Re-runs the forward keeping every h_t and A_bar_t, then walks t
+ * backwards with g_t = dL/dh_t:
+ *   g_t = dy_t C_t + r_{t+1} A_bar_{t+1} g_{t+1}
+ * and collects every input / parameter gradient from it. */
+static void scan_bwd_row(const scan_in_t* p, const scan_grad_t* g, int b, int d) {
+    const int L = p->L, N = p->N;
+    size_t row = ((size_t)b * p->D + d) * L;
+    double* hs = (double*)malloc(sizeof(double) * (size_t)L * N);
+    double* ab = (double*)malloc(sizeof(double) * (size_t)L * N);
+    double* dts = (double*)malloc(sizeof(double) * (size_t)L);
+    double* ys = (double*)malloc(sizeof(double) * (size_t)L);
+    int* rs = (int*)malloc(sizeof(int) * (size_t)L);
+    double* carry = (double*)calloc((size_t)N, sizeof(double));
+    double Dd = p->Dskip ? p->Dskip[d] : 0.0;
+
+    for (int t = 0; t < L; ++t) {
+        double dt = delta_at(p, d, row, t);
+        double ut = p->u[row + t];
+        int reset = (t > 0) && seg_of(p->seq, L, b, t) != seg_of(p->seq, L, b, t - 1);
+        double y = 0.0;
+        dts[t] = dt;
+        rs[t] = reset ? 0 : 1;
+        for (int n = 0; n < N; ++n) {
+            double abar = exp(dt * p->A[(size_t)d * N + n]);
+            double bt = p->Bm[((size_t)b * N + n) * L + t];
+            double ct = p->Cm[((size_t)b * N + n) * L + t];
+            double hprev = (t == 0 || reset) ? 0.0 : hs[(size_t)(t - 1) * N + n];
+            double h = abar * hprev + dt * bt * ut;
+            hs[(size_t)t * N + n] = h;
+            ab[(size_t)t * N + n] = abar;
+            y += ct * h;
+        }
+        ys[t] = y + Dd * ut;
+    }
+
+    for (int t = L - 1; t >= 0; --t) {
+        double ut = p->u[row + t];
+        double dt = dts[t];
+        double go = g->dout[row + t];
+        double dy;
+        if (p->z) {
+            double zt = p->z[row + t];
+            double sg = sigm(zt);
+            dy = go * zt * sg;
+            g->dz[row + t] = go * ys[t] * sg * (1.0 + zt * (1.0 - sg));
+        } else {
+            dy = go;
+            if (g->dz) g->dz[row + t] = 0.0;
+        }
+        if (g->dD) g->dD[d] += dy * ut;
+        double sgB = 0.0, sAq = 0.0;
+        for (int n = 0; n < N; ++n) {
+            size_t bn = ((size_t)b * N + n) * L + t;
+            double An = p->A[(size_t)d * N + n];
+            double gt = dy * p->Cm[bn] + carry[n];
+            double hprev = (t == 0) ? 0.0 : hs[(size_t)(t - 1) * N + n];
+            double q = gt * rs[t] * ab[(size_t)t * N + n] * hprev; /* g * dh/d(A_bar) * A_bar */
+            g->dC[bn] += dy * hs[(size_t)t * N + n];
+            g->dB[bn] += gt * dt * ut;
+            g->dA[(size_t)d * N + n] += q * dt;
+            sgB += gt * p->Bm[bn];
+            sAq += An * q;
+            carry[n] = rs[t] * ab[(size_t)t * N + n] * gt;
+        }
+        g->du[row + t] = dy * Dd + dt * sgB;
+        double ddt = ut * sgB + sAq;
+        double dv = ddt;
+        if (p->softplus_on) {
+            double v = p->delta[row + t] + (p->delta_bias ? p->delta_bias[d] : 0.0);
+            dv = ddt * sigm(v);
+        }
+        g->ddelta[row + t] = dv;
+        if (g->ddb) g->ddb[d] += dv;
+    }
+    free(hs); free(ab); free(dts); free(ys); free(rs); free(carry);
+}
+
+void oracle_scan_bwd(const double* u, const double* delta, const double* z,
+                     const double* A, const double* Dskip, const double* delta_bias,
+                     const double* Bm, const double* Cm, int softplus_on,
+                     const int32_t* seq, const double* dout, double* du,
+                     double* ddelta, double* dz, double* dA, double* dB,
+                     double* dC, double* dD, double* ddelta_bias,
+                     int B, int D, int L, int N) {
+    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on};
+    memset(dA, 0, sizeof(double) * (size_t)D * N);
+    memset(dB, 0, sizeof(double) * (size_t)B * N * L);
+    memset(dC, 0, sizeof(double) * (size_t)B * N * L);
+    if (dD) memset(dD, 0, sizeof(double) * (size_t)D);
+    if (ddelta_bias) memset(ddelta_bias, 0, sizeof(double) * (size_t)D);
+    scan_grad_t g = {dout, du, ddelta, dz, dA, dB, dC, dD, ddelta_bias};
+    for (int b = 0; b < B; ++b)
+        for (int d = 0; d < D; ++d) scan_bwd_row(&p, &g, b, d);
+}
+
+/* ------------------------------------------------- threaded row drivers */
+/* Rows are independent; only the reductions over rows (dA, dB, dC, dD,
+ * ddelta_bias) need per-thread partials, added afterwards in thread order. */
+typedef struct {
+    const scan_in_t* p;
+    scan_grad_t g;      /* per-thread accumulators for the reductions */
+    double *out, *y_out, *final_state;
+    int row_begin, row_end, bwd;
+} job_t;
+
+static void* run_job(void* arg) {
+    job_t* j = (job_t*)arg;
+    for (int r = j->row_begin; r < j->row_end; ++r) {
+        int b = r / j->p->D, d = r % j->p->D;
+        if (j->bwd) scan_bwd_row(j->p, &j->g, b, d);
+        else scan_fwd_row(j->p, b, d, j->out, j->y_out, j->final_state);
+    }
+    return NULL;
+}
+
+void oracle_scan_fwd_mt(const double* u, const double* delta, const double* z,
+                        const double* A, const double* Dskip, const double* delta_bias,
+                        const double* Bm, const double* Cm, int softplus_on,
+                        const int32_t* seq, double* out, double* y_out,
+                        double* final_state, int B, int D, int L, int N, int nthreads) {
+    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on};
+    int rows = B * D;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > rows) nthreads = rows;
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * nthreads);
+    job_t* jobs = (job_t*)calloc((size_t)nthreads, sizeof(job_t));
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i].p = &p;
+        jobs[i].out = out; jobs[i].y_out = y_out; jobs[i].final_state = final_state;
+        jobs[i].row_begin = (int)((long)rows * i / nthreads);
+        jobs[i].row_end = (int)((long)rows * (i + 1) / nthreads);
+        pthread_create(&th[i], NULL, run_job, &jobs[i]);
+    }
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    free(th); free(jobs);
+}
+
+void oracle_scan_bwd_mt(const double* u, const double* delta, const double* z,
+                        const double* A, const double* Dskip, const double* delta_bias,
+                        const double* Bm, const double* Cm, int softplus_on,
+                        const int32_t* seq, const double* dout, double* du,
+                        double* ddelta, double* dz, double* dA, double* dB,
+                        double* dC, double* dD, double* ddelta_bias,
+                        int B, int D, int L, int N, int nthreads) {
+    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on};
+    int rows = B * D;
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > rows) nthreads = rows;
+    size_t nA = (size_t)D * N, nBC = (size_t)B * N * L;
+    pthread_t* th = (pthread_t*)malloc(sizeof(pthread_t) * nthreads);
+    job_t* jobs = (job_t*)calloc((size_t)nthreads, sizeof(job_t));
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i].p = &p;
+        jobs[i].bwd = 1;
+        jobs[i].g.dout = dout;
+        jobs[i].g.du = du; jobs[i].g.ddelta = ddelta; jobs[i].g.dz = dz;
+        jobs[i].g.dA = (double*)calloc(nA, sizeof(double));
+        jobs[i].g.dB = (double*)calloc(nBC, sizeof(double));
+        jobs[i].g.dC = (double*)calloc(nBC, sizeof(double));
+        jobs[i].g.dD = (double*)calloc((size_t)D, sizeof(double));
+        jobs[i].g.ddb = (double*)calloc((size_t)D, sizeof(double));
+        jobs[i].row_begin = (int)((long)rows * i / nthreads);
+        jobs[i].row_end = (int)((long)rows * (i + 1) / nthreads);
+        pthread_create(&th[i], NULL, run_job, &jobs[i]);
+    }
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    memset(dA, 0, sizeof(double) * nA);
+    memset(dB, 0, sizeof(double) * nBC);
+    memset(dC, 0, sizeof(double) * nBC);
+    if (dD) memset(dD, 0, sizeof(double) * (size_t)D);
+    if (ddelta_bias) memset(ddelta_bias, 0, sizeof(double) * (size_t)D);
+    for (int i = 0; i < nthreads; ++i) {
+        for (size_t k = 0; k < nA; ++k) dA[k] += jobs[i].g.dA[k];
+        for (size_t k = 0; k < nBC; ++k) { dB[k] += jobs[i].g.dB[k]; dC[k] += jobs[i].g.dC[k]; }
+        for (int k = 0; k < D; ++k) {
+            if (dD) dD[k] += jobs[i].g.dD[k];
+            if (ddelta_bias) ddelta_bias[k] += jobs[i].g.ddb[k];
+        }
+        free(jobs[i].g.dA); free(jobs[i].g.dB); free(jobs[i].g.dC);
+        free(jobs[i].g.dD); free(jobs[i].g.ddb);
+    }
+    free(th); free(jobs);
+}

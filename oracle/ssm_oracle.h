@@ -1,0 +1,49 @@
+/*
+ * CPU oracle for the Mamba-1 selective-SSM layer core — TEST INFRASTRUCTURE.
+ * fp64 throughout. Only tests, the smoke check and the benchmark's CPU
+ * baseline use it; the product library never includes or links it.
+ *
+ * Layouts (all contiguous): activations [B][D][L]; B/C [B][N][L];
+ * A [D][N]; conv weight [D][W]; per-channel vectors [D]; seq_idx [B][L]
+ * (NULL = one segment per row); final state [B][D][N].
+ */
+#ifndef SSM_ORACLE_H
+#define SSM_ORACLE_H
+#include <stddef.h>
+#include <stdint.h>
+
+void oracle_round_bf16(const double* in, double* out, size_t n);
+
+void oracle_conv1d_fwd(const double* x, const double* w, const double* bias,
+                       const int32_t* seq, double* c, double* u,
+                       int B, int D, int L, int W, int silu);
+void oracle_conv1d_bwd(const double* x, const double* w, const double* bias,
+                       const int32_t* seq, const double* du, double* dx,
+                       double* dw, double* dbias, int B, int D, int L, int W, int silu);
+
+void oracle_scan_fwd(const double* u, const double* delta, const double* z,
+                     const double* A, const double* Dskip, const double* delta_bias,
+                     const double* Bm, const double* Cm, int softplus_on,
+                     const int32_t* seq, double* out, double* y_out,
+                     double* final_state, int B, int D, int L, int N);
+void oracle_scan_bwd(const double* u, const double* delta, const double* z,
+                     const double* A, const double* Dskip, const double* delta_bias,
+                     const double* Bm, const double* Cm, int softplus_on,
+                     const int32_t* seq, const double* dout, double* du,
+                     double* ddelta, double* dz, double* dA, double* dB,
+                     double* dC, double* dD, double* ddelta_bias,
+                     int B, int D, int L, int N);
+
+void oracle_scan_fwd_mt(const double* u, const double* delta, const double* z,
+                        const double* A, const double* Dskip, const double* delta_bias,
+                        const double* Bm, const double* Cm, int softplus_on,
+                        const int32_t* seq, double* out, double* y_out,
+                        double* final_state, int B, int D, int L, int N, int nthreads);
+void oracle_scan_bwd_mt(const double* u, const double* delta, const double* z,
+                        const double* A, const double* Dskip, const double* delta_bias,
+                        const double* Bm, const double* Cm, int softplus_on,
+                        const int32_t* seq, const double* dout, double* du,
+                        double* ddelta, double* dz, double* dA, double* dB,
+                        double* dC, double* dD, double* ddelta_bias,
+                        int B, int D, int L, int N, int nthreads);
+#endif

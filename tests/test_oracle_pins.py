@@ -1,0 +1,425 @@
+"""Pins for the fp64 CPU oracle: checks that do not go through the oracle's
+own formulas (closed forms, special cases, brute force, a library conv, the
+associative split, packing invariance, finite differences, hand-worked
+values). Every check here runs on CPU."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed=1234):
+    return np.random.Generator(np.random.PCG64(seed))
+
+
+def _sig(v):
+    return 1.0 / (1.0 + np.exp(-v))
+
+
+def _problem(rng, B=1, D=3, N=4, L=40, seq=None):
+    u = rng.standard_normal((B, D, L))
+    delta = 0.5 * rng.standard_normal((B, D, L))
+    z = rng.standard_normal((B, D, L))
+    A = -rng.uniform(0.2, 2.0, size=(D, N))
+    Bm = rng.standard_normal((B, N, L))
+    Cm = rng.standard_normal((B, N, L))
+    Dskip = rng.uniform(0.5, 1.5, size=D)
+    dbias = rng.uniform(-3, -1, size=D)
+    return dict(u=u, delta=delta, z=z, A=A, Bm=Bm, Cm=Cm, Dskip=Dskip,
+                delta_bias=dbias, seq_idx=seq)
+
+
+# --------------------------------------------------------------------------
+# bf16 rounding used at the storage points
+# --------------------------------------------------------------------------
+def test_round_bf16_hand_values():
+    # spacing of bf16 at 1.0 is 2^-7; ties go to the even mantissa
+    vals = np.array([1.0 + 2**-8, 1.0 + 3 * 2**-8, 1.0 + 2**-8 + 2**-20, -3.0, 0.0,
+                     2**-130])
+    want = np.array([1.0, 1.0 + 2**-6, 1.0 + 2**-7, -3.0, 0.0, 2**-130])
+    np.testing.assert_array_equal(oracle.round_bf16(vals), want)
+
+
+def test_round_bf16_matches_fp32_rne_bits():
+    x = _rng(7).standard_normal(10000).astype(np.float32) * 37.0
+    bits = synth.f32_to_bf16_bits(x)
+    np.testing.assert_array_equal(oracle.round_bf16(x.astype(np.float64)),
+                                  synth.bf16_bits_to_f32(bits).astype(np.float64))
+
+
+# --------------------------------------------------------------------------
+# conv1d
+# --------------------------------------------------------------------------
+def test_conv_identity_tap():
+    rng = _rng()
+    x = rng.standard_normal((2, 3, 50))
+    w = np.zeros((3, 4))
+    w[:, 3] = 1.0  # the newest tap multiplies x_t
+    c, u = oracle.conv1d_fwd(x, w, None, None, silu=False)
+    np.testing.assert_array_equal(u, x)
+    np.testing.assert_array_equal(c, x)
+
+
+def test_conv_matches_torch_conv1d():
+    torch = pytest.importorskip("torch")
+    rng = _rng(3)
+    B, D, L = 2, 5, 37
+    x = rng.standard_normal((B, D, L))
+    w = rng.uniform(-0.5, 0.5, size=(D, 4))
+    b = rng.standard_normal(D)
+    ref = torch.nn.functional.conv1d(torch.from_numpy(x), torch.from_numpy(w)[:, None, :],
+                                     torch.from_numpy(b), padding=3, groups=D)[..., :L].numpy()
+    c, u = oracle.conv1d_fwd(x, w, b, None, silu=True)
+    np.testing.assert_allclose(c, ref, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(u, ref * _sig(ref), rtol=1e-13, atol=1e-13)
+
+
+def test_conv_packed_equals_separate():
+    rng = _rng(5)
+    D, L = 3, 60
+    seq = np.zeros((1, L), dtype=np.int32)
+    cuts = [0, 1, 2, 17, 18, 40, L]
+    for i in range(len(cuts) - 1):
+        seq[0, cuts[i]:cuts[i + 1]] = i
+    x = rng.standard_normal((1, D, L))
+    w = rng.uniform(-0.5, 0.5, size=(D, 4))
+    b = rng.standard_normal(D)
+    du = rng.standard_normal((1, D, L))
+    _, u = oracle.conv1d_fwd(x, w, b, seq)
+    dx, dw, db = oracle.conv1d_bwd(x, w, b, seq, du)
+    dw_sum = np.zeros_like(dw)
+    db_sum = np.zeros_like(db)
+    for i in range(len(cuts) - 1):
+        s, e = cuts[i], cuts[i + 1]
+        _, ui = oracle.conv1d_fwd(x[:, :, s:e].copy(), w, b, None)
+        np.testing.assert_array_equal(u[:, :, s:e], ui)
+        dxi, dwi, dbi = oracle.conv1d_bwd(x[:, :, s:e].copy(), w, b, None, du[:, :, s:e].copy())
+        np.testing.assert_array_equal(dx[:, :, s:e], dxi)
+        dw_sum += dwi
+        db_sum += dbi
+    np.testing.assert_allclose(dw, dw_sum, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(db, db_sum, rtol=1e-13, atol=1e-13)
+
+
+def _fd(f, arr, h_rel=1e-6):
+    g = np.zeros_like(arr)
+    it = np.nditer(arr, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        old = arr[i]
+        h = h_rel * max(1.0, abs(old))
+        arr[i] = old + h
+        fp = f()
+        arr[i] = old - h
+        fm = f()
+        arr[i] = old
+        g[i] = (fp - fm) / (2 * h)
+    return g
+
+
+def _close(fd, an, tol=1e-6):
+    scale = max(1.0, float(np.abs(an).max()))
+    err = np.abs(fd - an).max() / scale
+    assert err < tol, err
+
+
+def test_conv_bwd_finite_differences():
+    rng = _rng(11)
+    B, D, L = 1, 3, 20
+    seq = np.zeros((B, L), dtype=np.int32)
+    seq[:, 9:] = 1
+    x = rng.standard_normal((B, D, L))
+    w = rng.uniform(-0.5, 0.5, size=(D, 4))
+    b = rng.standard_normal(D)
+    gu = rng.standard_normal((B, D, L))
+
+    def loss():
+        return float(np.sum(oracle.conv1d_fwd(x, w, b, seq)[1] * gu))
+
+    dx, dw, db = oracle.conv1d_bwd(x, w, b, seq, gu)
+    _close(_fd(loss, x), dx)
+    _close(_fd(loss, w), dw)
+    _close(_fd(loss, b), db)
+
+
+# --------------------------------------------------------------------------
+# scan forward: closed forms and special cases
+# --------------------------------------------------------------------------
+def test_scan_L1_closed_form():
+    rng = _rng(13)
+    p = _problem(rng, B=2, D=3, N=5, L=1)
+    r = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], z=p["z"],
+                        Dskip=p["Dskip"], delta_bias=p["delta_bias"])
+    v = p["delta"] + p["delta_bias"][None, :, None]
+    dt = np.log1p(np.exp(v))
+    # y_0 = sum_n C_n * (delta_0 B_n u_0) + D u_0   (h_{-1} = 0)
+    y = np.einsum("bnl,bnl->bl", p["Cm"], p["Bm"])[:, None, :] * dt * p["u"] \
+        + p["Dskip"][None, :, None] * p["u"]
+    np.testing.assert_allclose(r["y"], y, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(r["out"], y * p["z"] * _sig(p["z"]), rtol=1e-13, atol=1e-14)
+
+
+def test_scan_zero_step_gives_skip_only():
+    rng = _rng(17)
+    p = _problem(rng, L=33)
+    zero = np.zeros_like(p["delta"])
+    r = oracle.scan_fwd(p["u"], zero, p["A"], p["Bm"], p["Cm"], Dskip=p["Dskip"],
+                        softplus=False)
+    np.testing.assert_array_equal(r["y"], p["Dskip"][None, :, None] * p["u"])
+    np.testing.assert_array_equal(r["final_state"], 0.0)
+    # the same limit through softplus: delta_raw -> -inf makes delta underflow to 0
+    r2 = oracle.scan_fwd(p["u"], np.full_like(p["delta"], -1000.0), p["A"], p["Bm"],
+                         p["Cm"], Dskip=p["Dskip"], softplus=True)
+    np.testing.assert_array_equal(r2["y"], p["Dskip"][None, :, None] * p["u"])
+
+
+def test_scan_A_zero_is_prefix_sum():
+    rng = _rng(19)
+    p = _problem(rng, B=2, D=2, N=3, L=45)
+    A0 = np.zeros_like(p["A"])
+    r = oracle.scan_fwd(p["u"], p["delta"], A0, p["Bm"], p["Cm"], Dskip=None,
+                        delta_bias=p["delta_bias"])
+    dt = np.log1p(np.exp(p["delta"] + p["delta_bias"][None, :, None]))
+    contrib = dt[:, :, None, :] * p["Bm"][:, None, :, :] * p["u"][:, :, None, :]  # [B,D,N,L]
+    h = np.cumsum(contrib, axis=-1)
+    y = np.einsum("bdnl,bnl->bdl", h, p["Cm"])
+    np.testing.assert_allclose(r["y"], y, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(r["final_state"], h[..., -1], rtol=1e-12, atol=1e-12)
+
+
+def _brute_force_y(u, dt, A, Bm, Cm, Dskip, seq):
+    """h_t = sum_{s<=t, same doc} exp(A * sum_{s<r<=t} dt_r) dt_s B_s u_s."""
+    B_, D, L = u.shape
+    N = A.shape[1]
+    y = np.zeros_like(u)
+    for b in range(B_):
+        for d in range(D):
+            for t in range(L):
+                acc = Dskip[d] * u[b, d, t]
+                for s in range(t + 1):
+                    if seq is not None and np.any(seq[b, s:t + 1] != seq[b, t]):
+                        continue
+                    decay = np.exp(A[d] * dt[b, d, s + 1:t + 1].sum())
+                    acc += np.sum(Cm[b, :, t] * decay * dt[b, d, s] * Bm[b, :, s]) * u[b, d, s]
+                y[b, d, t] = acc
+    assert N == Bm.shape[1]
+    return y
+
+
+@pytest.mark.parametrize("packed", [False, True])
+def test_scan_unrolled_sum_brute_force(packed):
+    rng = _rng(23)
+    L = 48
+    seq = None
+    if packed:
+        seq = np.zeros((2, L), dtype=np.int32)
+        seq[0, 10:] = 1
+        seq[0, 11:] = 2
+        seq[0, 30:] = 3
+        seq[1, 47:] = 5
+    p = _problem(rng, B=2, D=2, N=3, L=L, seq=seq)
+    r = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], Dskip=p["Dskip"],
+                        delta_bias=p["delta_bias"], seq_idx=seq)
+    dt = np.log1p(np.exp(p["delta"] + p["delta_bias"][None, :, None]))
+    y = _brute_force_y(p["u"], dt, p["A"], p["Bm"], p["Cm"], p["Dskip"], seq)
+    np.testing.assert_allclose(r["y"], y, rtol=1e-11, atol=1e-12)
+
+
+def test_scan_lti_is_causal_convolution():
+    # delta, B, C constant in t: y = u * K + D u with K_k = sum_n C_n e^{k dt A_n} dt B_n
+    rng = _rng(29)
+    D, N, L = 2, 4, 64
+    u = rng.standard_normal((1, D, L))
+    A = -rng.uniform(0.1, 1.0, size=(D, N))
+    dt = np.array([0.3, 0.07])
+    bv = rng.standard_normal(N)
+    cv = rng.standard_normal(N)
+    Bm = np.repeat(bv[None, :, None], L, axis=2)
+    Cm = np.repeat(cv[None, :, None], L, axis=2)
+    delta = np.repeat(dt[None, :, None], L, axis=2)
+    Dskip = np.array([0.7, -0.2])
+    r = oracle.scan_fwd(u, delta, A, Bm, Cm, Dskip=Dskip, softplus=False)
+    for d in range(D):
+        k = np.arange(L)
+        K = (cv[None, :] * np.exp(k[:, None] * dt[d] * A[d][None, :]) * dt[d] * bv[None, :]).sum(1)
+        y = np.convolve(u[0, d], K)[:L] + Dskip[d] * u[0, d]
+        np.testing.assert_allclose(r["y"][0, d], y, rtol=1e-11, atol=1e-12)
+
+
+def test_scan_associative_split():
+    # (a1,b1) (+) (a2,b2) = (a1 a2, a2 b1 + b2): pieces from zero state, combined.
+    rng = _rng(31)
+    p = _problem(rng, B=1, D=2, N=3, L=70)
+    cuts = [0, 23, 24, 70]
+    full = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"],
+                           delta_bias=p["delta_bias"])["final_state"]
+    dt = np.log1p(np.exp(p["delta"] + p["delta_bias"][None, :, None]))
+    P = np.ones_like(full)
+    H = np.zeros_like(full)
+    for s, e in zip(cuts[:-1], cuts[1:]):
+        sl = np.s_[:, :, s:e]
+        Hi = oracle.scan_fwd(p["u"][sl].copy(), p["delta"][sl].copy(), p["A"],
+                             p["Bm"][sl].copy(), p["Cm"][sl].copy(),
+                             delta_bias=p["delta_bias"])["final_state"]
+        Pi = np.exp(p["A"][None] * dt[sl].sum(-1)[..., None])
+        H = Pi * H + Hi
+        P = P * Pi
+    np.testing.assert_allclose(H, full, rtol=1e-12, atol=1e-13)
+
+
+def test_scan_linear_in_u():
+    rng = _rng(37)
+    p = _problem(rng, L=30)
+    u2 = rng.standard_normal(p["u"].shape)
+    kw = dict(Dskip=p["Dskip"], delta_bias=p["delta_bias"])
+    y1 = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], **kw)["out"]
+    y2 = oracle.scan_fwd(u2, p["delta"], p["A"], p["Bm"], p["Cm"], **kw)["out"]
+    y3 = oracle.scan_fwd(2.5 * p["u"] - 0.5 * u2, p["delta"], p["A"], p["Bm"], p["Cm"], **kw)["out"]
+    np.testing.assert_allclose(y3, 2.5 * y1 - 0.5 * y2, rtol=1e-11, atol=1e-12)
+
+
+def test_scan_hand_worked_golden():
+    with open(os.path.join(GOLDEN, "hand_worked_s6.json")) as f:
+        g = json.load(f)
+    for c in g["cases"]:
+        L = len(c["u"])
+        u = np.array(c["u"], dtype=np.float64).reshape(1, 1, L)
+        dl = np.array(c["delta"], dtype=np.float64).reshape(1, 1, L)
+        A = np.array(c["A"], dtype=np.float64).reshape(1, -1)
+        Bm = np.array(c["Bm"], dtype=np.float64)[None]
+        Cm = np.array(c["Cm"], dtype=np.float64)[None]
+        seq = None if c["seq_idx"] is None else np.array(c["seq_idx"], dtype=np.int32)[None]
+        r = oracle.scan_fwd(u, dl, A, Bm, Cm, Dskip=np.array([c["D"]]), softplus=False,
+                            seq_idx=seq)
+        np.testing.assert_allclose(r["y"][0, 0], c["y"], rtol=1e-14, atol=1e-14, err_msg=c["name"])
+        np.testing.assert_allclose(r["final_state"][0, 0], c["final_state"], rtol=1e-14,
+                                   atol=1e-14, err_msg=c["name"])
+
+
+# --------------------------------------------------------------------------
+# packing: a packed batch equals its documents run separately
+# --------------------------------------------------------------------------
+def test_scan_packed_equals_separate():
+    rng = _rng(41)
+    L = 57
+    cuts = [0, 1, 2, 20, 21, 50, L]
+    seq = np.zeros((1, L), dtype=np.int32)
+    for i in range(len(cuts) - 1):
+        seq[0, cuts[i]:cuts[i + 1]] = 10 - i  # ids need not increase
+    p = _problem(rng, B=1, D=2, N=3, L=L, seq=seq)
+    dout = rng.standard_normal(p["u"].shape)
+    kw = dict(z=p["z"], Dskip=p["Dskip"], delta_bias=p["delta_bias"])
+    f = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], seq_idx=seq, **kw)
+    g = oracle.scan_bwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], dout, seq_idx=seq, **kw)
+    acc = {k: np.zeros_like(g[k]) for k in ("dA", "dD", "ddelta_bias")}
+    for s, e in zip(cuts[:-1], cuts[1:]):
+        sl = np.s_[:, :, s:e]
+        kw_i = dict(z=p["z"][sl].copy(), Dskip=p["Dskip"], delta_bias=p["delta_bias"])
+        fi = oracle.scan_fwd(p["u"][sl].copy(), p["delta"][sl].copy(), p["A"],
+                             p["Bm"][sl].copy(), p["Cm"][sl].copy(), **kw_i)
+        gi = oracle.scan_bwd(p["u"][sl].copy(), p["delta"][sl].copy(), p["A"],
+                             p["Bm"][sl].copy(), p["Cm"][sl].copy(), dout[sl].copy(), **kw_i)
+        np.testing.assert_array_equal(f["out"][sl], fi["out"])
+        for k in ("du", "ddelta", "dz", "dB", "dC"):
+            np.testing.assert_array_equal(g[k][sl], gi[k], err_msg=k)
+        for k in acc:
+            acc[k] += gi[k]
+        if e == L:
+            np.testing.assert_array_equal(f["final_state"], fi["final_state"])
+    for k in acc:
+        np.testing.assert_allclose(g[k], acc[k], rtol=1e-12, atol=1e-13, err_msg=k)
+
+
+# --------------------------------------------------------------------------
+# backward: finite differences and closed forms
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("softplus", [True, False])
+def test_scan_bwd_finite_differences(softplus):
+    inp = synth.make_inputs(synth.CONFIGS[1], synth.seed_for(1), dskip_random=True)
+    rng = _rng(43)
+    p = dict(u=rng.standard_normal((1, 4, 64)), delta=inp.delta.f64.copy(), z=inp.z.f64.copy(),
+             A=inp.A.astype(np.float64), Bm=inp.Bm.f64.copy(), Cm=inp.Cm.f64.copy(),
+             Dskip=inp.Dskip.astype(np.float64), delta_bias=inp.delta_bias.astype(np.float64))
+    if not softplus:
+        p["delta"] = np.abs(p["delta"]) * 0.2
+        p["delta_bias"] = np.zeros_like(p["delta_bias"])
+    seq = inp.seq_idx
+    dout = inp.dout.f64
+
+    def loss():
+        r = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], z=p["z"],
+                            Dskip=p["Dskip"], delta_bias=p["delta_bias"], softplus=softplus,
+                            seq_idx=seq)
+        return float(np.sum(r["out"] * dout))
+
+    g = oracle.scan_bwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], dout, z=p["z"],
+                        Dskip=p["Dskip"], delta_bias=p["delta_bias"], softplus=softplus,
+                        seq_idx=seq)
+    pairs = [("u", "du"), ("delta", "ddelta"), ("z", "dz"), ("A", "dA"), ("Bm", "dB"),
+             ("Cm", "dC"), ("Dskip", "dD"), ("delta_bias", "ddelta_bias")]
+    for name, gname in pairs:
+        _close(_fd(loss, p[name]), g[gname])
+
+
+def test_scan_dD_closed_form():
+    rng = _rng(47)
+    p = _problem(rng, B=2, D=3, N=2, L=25)
+    dout = rng.standard_normal(p["u"].shape)
+    g = oracle.scan_bwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], dout, z=p["z"],
+                        Dskip=p["Dskip"], delta_bias=p["delta_bias"])
+    dy = dout * p["z"] * _sig(p["z"])
+    np.testing.assert_allclose(g["dD"], (dy * p["u"]).sum(axis=(0, 2)), rtol=1e-12)
+
+
+def test_layer_chain_finite_differences():
+    """conv -> scan -> gate, end to end, against finite differences in x, w, bias."""
+    inp = synth.make_inputs(synth.CONFIGS[1], synth.seed_for(1), conv_bias_scale=0.3)
+    x = inp.x.f64.copy()
+    w = inp.conv_w.astype(np.float64)
+    cb = inp.conv_b.astype(np.float64)
+    seq = inp.seq_idx
+
+    def loss():
+        _, u = oracle.conv1d_fwd(x, w, cb, seq)
+        r = oracle.scan_fwd(u, inp.delta.f64, inp.A, inp.Bm.f64, inp.Cm.f64, z=inp.z.f64,
+                            Dskip=inp.Dskip, delta_bias=inp.delta_bias, seq_idx=seq)
+        return float(np.sum(r["out"] * inp.dout.f64))
+
+    r = oracle.layer_fwd_bwd(inp, bf16_points=False)
+    _close(_fd(loss, x), r["dx"])
+    _close(_fd(loss, w), r["dconv_w"])
+    _close(_fd(loss, cb), r["dconv_b"])
+
+
+def test_threaded_driver_matches_single_thread():
+    rng = _rng(53)
+    p = _problem(rng, B=2, D=5, N=4, L=31)
+    dout = rng.standard_normal(p["u"].shape)
+    kw = dict(z=p["z"], Dskip=p["Dskip"], delta_bias=p["delta_bias"])
+    f1 = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], **kw)
+    f4 = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], nthreads=4, **kw)
+    np.testing.assert_array_equal(f1["out"], f4["out"])
+    g1 = oracle.scan_bwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], dout, **kw)
+    g4 = oracle.scan_bwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], dout, nthreads=4, **kw)
+    for k in g1:
+        np.testing.assert_allclose(g1[k], g4[k], rtol=1e-12, atol=1e-13, err_msg=k)
+
+
+def test_softplus_reading_is_exact_log1p_exp():
+    # delta = log(1 + e^v): check the oracle's step against a direct evaluation
+    u = np.ones((1, 1, 5))
+    v = np.array([-30.0, -1.0, 0.0, 1.0, 30.0]).reshape(1, 1, 5)
+    A = np.zeros((1, 1))
+    Bm = np.zeros((1, 1, 5))
+    Bm[0, 0, :] = 1.0
+    Cm = np.ones((1, 1, 5))
+    y = oracle.scan_fwd(u, v, A, Bm, Cm, softplus=True)["y"][0, 0]
+    want = np.cumsum([math.log1p(math.exp(t)) for t in v.ravel()])
+    np.testing.assert_allclose(y, want, rtol=1e-14)

@@ -1,0 +1,471 @@
+#!/usr/bin/env python
+"""Benchmark of the Mamba-1 selective-SSM layer core on B200.
+
+One step = the whole hot path over one batch, for every layer of the
+workload: causal conv1d + SiLU forward, selective scan forward, selective
+scan backward, conv1d backward. Default workload: the long-context shape,
+4 independent layers of B=2, d_inner=1536, d_state=16, L=32768, bf16
+activations with fp32 state (inputs of each layer ~0.8 GB, larger than L2,
+layers rotated, so no L2 flush is needed).
+
+Prints one JSON line (rank 0). `value` is layer-tokens/s of the whole step
+with inputs resident in HBM; `e2e` is the same metric through the same C-ABI
+calls with host buffers (pinned host -> device copies of every input and
+device -> host copies of every output inside the timed region).
+
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same
+workload (the reference arm for this project); the oracle is also timed as
+`cpu_baseline` on rank 0 at N=1.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "scan fwd+bwd tokens/s (B2×1536ch×32K, N=16); achieved HBM GB/s % of roofline"
+UNIT = "layer-tokens/s"
+SFU_EX2_PER_CLK_PER_SM = 16  # MUFU ex2 throughput per SM per clock
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": float(pk["hbm_gbs"]), "sm_max_mhz": float(pk.get("sm_max_mhz", 1965.0)),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+_REASONS = ["gpu_idle", "applications_clocks_setting", "sw_power_cap", "hw_slowdown", "sync_boost",
+            "sw_thermal_slowdown", "hw_thermal_slowdown", "hw_power_brake_slowdown",
+            "display_clock_setting"]
+
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.th = threading.Thread(target=self._read, daemon=True)
+        self.th.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.th.join(timeout=2)
+        mhz, mx, reasons = [], [], set()
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                mhz.append(float(f[0]))
+                mx.append(float(f[1]))
+                act = int(f[3], 16) if f[3].startswith("0x") else int(f[3])
+            except ValueError:
+                continue
+            for bit, name in enumerate(_REASONS):
+                if act & (1 << bit) and name != "gpu_idle":
+                    reasons.add(name)
+        if not mhz:
+            return None
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ----------------------------------------------------------------------------
+# one layer on the device
+# ----------------------------------------------------------------------------
+class Layer:
+    """Device buffers of one layer and the four C-ABI calls of a step."""
+
+    def __init__(self, inp, device, n_splits):
+        import torch
+        import selective_state_space_35_b200 as ssm
+        self.ssm = ssm
+        self.shape = inp.shape
+        B, D, N, L = inp.shape.B, inp.shape.D, inp.shape.N, inp.shape.L
+        bf = torch.bfloat16
+
+        def act(t):
+            return torch.from_numpy(t.bits.view(np.int16)).view(bf).to(device)
+
+        self.host = {k: getattr(inp, k) for k in ("x", "z", "delta", "Bm", "Cm", "dout")}
+        self.x, self.z, self.delta = act(inp.x), act(inp.z), act(inp.delta)
+        self.Bm, self.Cm, self.dout = act(inp.Bm), act(inp.Cm), act(inp.dout)
+        f32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device)  # noqa: E731
+        self.A, self.Dskip, self.dbias = f32(inp.A), f32(inp.Dskip), f32(inp.delta_bias)
+        self.w, self.cb = f32(inp.conv_w), f32(inp.conv_b)
+        self.seq = (torch.from_numpy(inp.seq_idx).to(device) if inp.seq_idx is not None else None)
+        e = lambda: torch.empty((B, D, L), dtype=bf, device=device)  # noqa: E731
+        self.u, self.out, self.dx = e(), e(), e()
+        self.final_state = torch.empty((B, D, N), dtype=torch.float32, device=device)
+        self.g = {"du": e(), "ddelta": e(), "dz": e(),
+                  "dA": torch.empty((D, N), dtype=torch.float32, device=device),
+                  "dB": torch.empty((B, N, L), dtype=torch.float32, device=device),
+                  "dC": torch.empty((B, N, L), dtype=torch.float32, device=device),
+                  "dD": torch.empty((D,), dtype=torch.float32, device=device),
+                  "ddelta_bias": torch.empty((D,), dtype=torch.float32, device=device)}
+        self.dw = torch.empty((D, 4), dtype=torch.float32, device=device)
+        self.dcb = torch.empty((D,), dtype=torch.float32, device=device)
+        p = ssm.scan_params(self.u, self.delta, self.A, self.Bm, self.Cm, z=self.z, Dskip=self.Dskip,
+                            delta_bias=self.dbias, seq_idx=self.seq, n_splits=n_splits,
+                            out=self.out, final_state=self.final_state)
+        self.ws = torch.empty(ssm.scan_workspace_size(p), dtype=torch.uint8, device=device)
+        self.cws = torch.empty(ssm.ssm_conv1d_bwd_workspace_size(B, D, L, 4), dtype=torch.uint8,
+                               device=device)
+        self.n_splits = n_splits
+        self.kw = dict(z=self.z, Dskip=self.Dskip, delta_bias=self.dbias, seq_idx=self.seq,
+                       n_splits=n_splits)
+
+    def launches(self) -> int:
+        """Kernels of this library one step of this layer launches."""
+        nch = (self.shape.L + 255) // 256
+        P = self.n_splits
+        if P == 0:  # mirror the library's automatic choice
+            rows = self.shape.B * self.shape.D
+            P = 1 if rows >= 148 * 8 else -(-148 * 8 // rows)
+        P = max(1, min(P, nch))
+        cps = -(-nch // P)
+        P = -(-nch // cps)
+        extra = 2 if P > 1 else 0
+        return 1 + (1 + extra) + (2 + extra) + 2
+
+    def step(self, ev=None):
+        ssm = self.ssm
+        if ev is not None:
+            ev[0].record()
+        ssm.conv1d_fwd(self.x, self.w, self.cb, self.seq, out=self.u)
+        if ev is not None:
+            ev[1].record()
+        ssm.scan_fwd(self.u, self.delta, self.A, self.Bm, self.Cm, out=self.out,
+                     workspace=self.ws, return_final_state=False, **self.kw)
+        if ev is not None:
+            ev[2].record()
+        ssm.scan_bwd(self.u, self.delta, self.A, self.Bm, self.Cm, self.dout, self.ws,
+                     grads=self.g, **self.kw)
+        if ev is not None:
+            ev[3].record()
+        ssm.conv1d_bwd(self.x, self.w, self.cb, self.seq, self.g["du"], dx=self.dx, dw=self.dw,
+                       dbias=self.dcb, workspace=self.cws)
+        if ev is not None:
+            ev[4].record()
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle timing (bounded sample of the same workload)
+# ----------------------------------------------------------------------------
+def oracle_sample(inp, seconds: float, threads: int):
+    """Run the fp64 oracle on channel rows of batch row 0 until `seconds` pass.
+
+    Returns (layer-tokens/s equivalent, rows done, seconds, threads)."""
+    import oracle
+    sh = inp.shape
+    D, L = sh.D, sh.L
+    rows_per = max(1, threads)
+    done, t_total, d0 = 0, 0.0, 0
+    f64 = lambda t, sl: synth.bf16_bits_to_f32(t.bits[sl]).astype(np.float64)  # noqa: E731
+    while t_total < seconds and d0 < D:
+        d1 = min(D, d0 + rows_per)
+        sl = np.s_[0:1, d0:d1, :]
+        x, z, dl, go = f64(inp.x, sl), f64(inp.z, sl), f64(inp.delta, sl), f64(inp.dout, sl)
+        Bm, Cm = f64(inp.Bm, np.s_[0:1]), f64(inp.Cm, np.s_[0:1])
+        seq = None if inp.seq_idx is None else np.ascontiguousarray(inp.seq_idx[0:1])
+        A, Dk, db = inp.A[d0:d1], inp.Dskip[d0:d1], inp.delta_bias[d0:d1]
+        w, cb = inp.conv_w[d0:d1], inp.conv_b[d0:d1]
+        t0 = time.perf_counter()
+        _, u = oracle.conv1d_fwd(x, w, cb, seq)
+        u = oracle.round_bf16(u)
+        kw = dict(z=z, Dskip=Dk, delta_bias=db, seq_idx=seq, nthreads=threads)
+        oracle.scan_fwd(u, dl, A, Bm, Cm, **kw)
+        g = oracle.scan_bwd(u, dl, A, Bm, Cm, go, **kw)
+        oracle.conv1d_bwd(x, w, cb, seq, oracle.round_bf16(g["du"]))
+        t_total += time.perf_counter() - t0
+        done += d1 - d0
+        d0 = d1
+    # a full layer is B*D such rows and carries B*L tokens
+    tok_s = (done * L) / (D * t_total) if t_total > 0 else 0.0
+    return tok_s, done, t_total
+
+
+def cpu_count() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, cfg, rank):
+    if rank != 0:
+        return 0
+    sh = synth.CONFIGS[cfg]
+    sh1 = synth.Shape(sh.name, sh.B, sh.D, sh.N, sh.L, sh.dtype, packed=sh.packed)
+    inp = synth.make_inputs(sh1, synth.seed_for(cfg, 0), want_f64=False)
+    threads = cpu_count()
+    budget = max(1.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample(inp, budget * 0.25, threads)
+    vals, secs, rows = [], 0.0, 0
+    for _ in range(args.steps):
+        v, r, s = oracle_sample(inp, budget, threads)
+        vals.append(v)
+        secs += s
+        rows += r
+    val = float(np.mean(vals)) if vals else 0.0
+    sample = (f"{rows} channel rows x {sh.L} tokens of layer 0 ({sh.name}), conv+scan fwd+bwd in "
+              f"fp64, over {args.steps} steps of ~{budget:.1f} s")
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs / max(1, args.steps), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(sh, cfg),
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(sh, cfg):
+    return {"workload": f"{sh.name} bf16, conv1d+SiLU -> selective scan fwd+bwd -> conv1d bwd",
+            "config_index": cfg, "layers": sh.layers, "B": sh.B, "D": sh.D, "N": sh.N, "L": sh.L,
+            "conv_width": 4, "storage": sh.dtype, "state": "f32", "packed": sh.packed,
+            "l2": "inputs larger than L2 (each layer's inputs > 126 MB, layers rotated); no flush"}
+
+
+# ----------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", type=int, default=3)
+    ap.add_argument("--n-splits", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = args.config
+    if args.impl == "reference":
+        return run_reference(args, cfg, rank)
+
+    import torch
+    import torch.distributed as dist
+    from selective_state_space_35_b200 import build
+    build.build()
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    sh = synth.CONFIGS[cfg]
+    inps = [synth.make_inputs(sh, synth.seed_for(cfg, l), want_f64=False) for l in range(sh.layers)]
+    layers = [Layer(inp, device, args.n_splits) for inp in inps]
+    stream = torch.cuda.current_stream(device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        for ly in layers:
+            ly.step()
+    torch.cuda.synchronize()
+
+    nlay = len(layers)
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(nlay)]
+           for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local_rank]))
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for s in range(args.steps):
+        for i, ly in enumerate(layers):
+            ly.step(evs[s][i])
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ck = clocks.stop()
+    ms = start.elapsed_time(stop)
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    tokens_step = nlay * sh.B * sh.L
+    value = world * tokens_step / (ms_step * 1e-3)
+
+    # per-call durations (events bracket each C-ABI call on the launching stream)
+    names = ["conv1d_fwd", "scan_fwd", "scan_bwd", "conv1d_bwd"]
+    per = {n: [] for n in names}
+    for s in range(args.steps):
+        for i in range(nlay):
+            e = evs[s][i]
+            for k, n in enumerate(names):
+                per[n].append(e[k].elapsed_time(e[k + 1]))
+    avg = {n: float(np.mean(v)) for n, v in per.items()}
+    scan_ms = avg["scan_fwd"] + avg["scan_bwd"]
+    B, D, N, L = sh.B, sh.D, sh.N, sh.L
+    pk = _peaks()
+    e_sz = 2
+    bytes_tok = {"scan_fwd": 4 * D * e_sz + 2 * N * e_sz,
+                 "scan_bwd": 7 * D * e_sz + 2 * N * e_sz + 2 * N * 4,
+                 "conv1d_fwd": 2 * D * e_sz, "conv1d_bwd": 3 * D * e_sz}
+    hbm = {n: bytes_tok[n] * B * L / (avg[n] * 1e-3) / 1e9 for n in names}
+    dom = max(names, key=lambda n: avg[n])
+    exps = B * D * L * N
+    ex2_peak = SFU_EX2_PER_CLK_PER_SM * 148 * pk["sm_max_mhz"] * 1e6 / 1e12  # T ex2/s
+    if dom.startswith("scan"):
+        achieved = exps / (avg[dom] * 1e-3) / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": ex2_peak, "unit": "Tex2/s",
+                "frac": achieved / ex2_peak, "traffic": None, "kernel": f"ssm_{dom}",
+                "peak_source": "derived: 16 ex2/clk/SM x 148 SMs x max SM clock (of measured "
+                               "clock)", "work_per_launch": f"{exps} ex2 (B*D*L*N)"}
+    else:
+        achieved = hbm[dom]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": None, "kernel": f"ssm_{dom}"}
+    t_sfu = 2 * exps / (ex2_peak * 1e12) * 1e3
+    t_hbm = (bytes_tok["scan_fwd"] + bytes_tok["scan_bwd"]) * B * L / (pk["hbm_gbs"] * 1e9) * 1e3
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(workload_config(sh, cfg), parallelism=f"replicas x{world}"),
+        "roofline": roof,
+        "scan": {"tokens_per_s": world * nlay * B * L / (scan_ms * 1e-3),
+                 "ms_per_layer": {n: avg[n] for n in names},
+                 "hbm_gbs": hbm, "hbm_frac_of_measured": {n: hbm[n] / pk["hbm_gbs"] for n in names},
+                 "roofline_ms_per_layer": {"sfu_2BDLN": t_sfu, "hbm_alg_bytes": t_hbm},
+                 "frac_of_roofline": max(t_sfu, t_hbm) / scan_ms},
+        "gpu_launches": args.steps * sum(ly.launches() for ly in layers),
+        "clocks": ck,
+    }
+
+    # e2e: host buffers in, host buffers out, through the same calls
+    if not args.no_e2e:
+        line["e2e"] = e2e(layers, device, args, world)
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = cpu_count()
+        v, rows, secs = oracle_sample(inps[0], args.cpu_seconds, threads)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": f"{rows} channel rows x {L} tokens of layer 0, conv+scan "
+                                          f"fwd+bwd in fp64, {secs:.1f} s"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def e2e(layers, device, args, world):
+    import torch
+    import torch.distributed as dist
+    bf = torch.bfloat16
+    pinned_in = []
+    for ly in layers:
+        d = {}
+        for k in ("x", "z", "delta", "Bm", "Cm", "dout"):
+            t = torch.from_numpy(ly.host[k].bits.view(np.int16)).view(bf)
+            d[k] = t.pin_memory()
+        pinned_in.append(d)
+    ly0 = layers[0]
+    outs = {"out": ly0.out, "dx": ly0.dx, "ddelta": ly0.g["ddelta"], "dz": ly0.g["dz"],
+            "dB": ly0.g["dB"], "dC": ly0.g["dC"], "dA": ly0.g["dA"], "dD": ly0.g["dD"],
+            "ddelta_bias": ly0.g["ddelta_bias"], "dconv_w": ly0.dw, "dconv_b": ly0.dcb}
+    pinned_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outs.items()}
+    h2d = sum(t.numel() * t.element_size() for d in pinned_in for t in d.values())
+    d2h = len(layers) * sum(t.numel() * t.element_size() for t in pinned_out.values())
+
+    def step():
+        for ly, hin in zip(layers, pinned_in):
+            for k, t in hin.items():
+                getattr(ly, k).copy_(t, non_blocking=True)
+            ly.step()
+            o = {"out": ly.out, "dx": ly.dx, "ddelta": ly.g["ddelta"], "dz": ly.g["dz"],
+                 "dB": ly.g["dB"], "dC": ly.g["dC"], "dA": ly.g["dA"], "dD": ly.g["dD"],
+                 "ddelta_bias": ly.g["ddelta_bias"], "dconv_w": ly.dw, "dconv_b": ly.dcb}
+            for k, t in o.items():
+                pinned_out[k].copy_(t, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    n = max(1, args.e2e_steps)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    a.record()
+    for _ in range(n):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    if world > 1:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    sh = layers[0].shape
+    tokens = world * len(layers) * sh.B * sh.L
+    return {"value": tokens / (ms / n * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": ms / n}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

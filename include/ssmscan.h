@@ -1,0 +1,173 @@
+/*
+ * libssmscan — C ABI for the Mamba-1 selective-SSM layer core on NVIDIA B200
+ * (sm_100a): depthwise causal conv1d + SiLU, and the selective scan with
+ * softplus step, D skip and SiLU(z) gate, forward and backward, with state
+ * and conv resets at packed-document boundaries.
+ *
+ * Where each operation is defined (page title, section):
+ *   conv1d   "hung-phan ml-skills mamba", "Mamba: Selective State Spaces
+ *            (S6)" (depthwise Conv1d, padding d_conv-1, first L outputs, then
+ *            SiLU) and "Mamba Block Architecture" (Conv1d(k=4) -> SiLU).
+ *   scan     same page, "Architecture Diagram" (S6 block: A_bar = exp(dt*A),
+ *            B_bar = dt*B, h_t = A_bar h_{t-1} + B_bar x_t, y_t = C_t h_t),
+ *            "Core Concept" (y += D x), the S6 sketch (dt = softplus(dt),
+ *            y * silu(z)) and "Hardware-Aware Parallel Scan" (the operator
+ *            (a1,b1)+(a2,b2) = (a1 a2, a2 b1 + b2) used to combine pieces).
+ *   resets   "FLA Mamba and Mamba2" (Axolotl), packing paragraph: conv and
+ *            recurrent state start independently for every document.
+ *   recompute in backward: "hung-phan ml-skills mamba", "Hardware-Aware
+ *            Parallel Scan", memory-optimisation note.
+ *
+ * Conventions for every call:
+ *   - All array pointers are caller-owned DEVICE memory, C-contiguous, in the
+ *     layouts stated per argument. The library allocates nothing; scratch is
+ *     a caller-provided workspace whose size the *_workspace_size calls give.
+ *   - Activations ([B][D][L], L fastest) and B/C ([B][N][L]) have dtype
+ *     `dtype` (bf16 or fp32); A, D, biases, conv weights, gradients of
+ *     parameters and of B/C are fp32; segment ids are int32.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns without synchronising.
+ *   - Gradient outputs are overwritten, never accumulated into.
+ *   - On any non-OK status nothing has been launched (argument errors) or the
+ *     launch itself failed (SSM_ERR_CUDA); ssm_last_error() then returns a
+ *     thread-local, human-readable message. No call throws or aborts.
+ *   - Sizes: B, D, L >= 1, 1 <= N <= 16, W == 4. Any L is accepted; when L is
+ *     a multiple of 8 and every activation pointer is 16-byte aligned the
+ *     kernels use 16-byte vector accesses, otherwise a scalar path.
+ *   - A segment id array seq_idx [B][L] (nullable) marks documents: token t
+ *     starts a new document when seq_idx[b][t] != seq_idx[b][t-1]. Ids need
+ *     not be increasing; padding may carry any id of its own (e.g. -1).
+ */
+#ifndef SSMSCAN_H
+#define SSMSCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* ssm_stream_t;
+
+typedef enum {
+    SSM_OK = 0,
+    SSM_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad alignment, bad struct_size */
+    SSM_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. N > 16, W != 4) */
+    SSM_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed */
+    SSM_ERR_TIMEOUT = 4,     /* reserved: a bounded device-side wait gave up */
+    SSM_ERR_INJECTED = 5     /* host-side fault injection (env SSM_INJECT_FAIL) */
+} ssm_status_t;
+
+typedef enum { SSM_DTYPE_F32 = 0, SSM_DTYPE_BF16 = 1 } ssm_dtype_t;
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char* ssm_last_error(void);
+
+/* ABI version of this header (bumped on any incompatible change). */
+#define SSM_ABI_VERSION 1
+int ssm_abi_version(void);
+
+/* ---------------------------------------------------------------------------
+ * ssm_conv1d_fwd — depthwise causal conv1d, width W = 4, optional SiLU.
+ *   c[b][d][t] = bias[d] + sum_{k=0..3} w[d][k] * x[b][d][t-3+k]
+ * where a tap counts only if t-3+k >= 0 and, when seq_idx is given,
+ * seq_idx[b][t-3+k] == seq_idx[b][t]. u = silu(c) if silu != 0, else c.
+ *   x        [B][D][L] dtype          input
+ *   w        [D][W]    fp32           w[d][W-1] multiplies x_t (cross-correlation)
+ *   bias     [D]       fp32, nullable (0)
+ *   seq_idx  [B][L]    int32, nullable (one document per row)
+ *   u        [B][D][L] dtype          output (may not alias x)
+ * ------------------------------------------------------------------------ */
+ssm_status_t ssm_conv1d_fwd(const void* x, const float* w, const float* bias,
+                            const int32_t* seq_idx, void* u, int B, int D, int L,
+                            int W, ssm_dtype_t dtype, int silu, ssm_stream_t stream);
+
+/* Bytes of workspace ssm_conv1d_bwd needs for these sizes (per-tile partial
+ * sums of dw and dbias, reduced in a fixed order: results are deterministic). */
+ssm_status_t ssm_conv1d_bwd_workspace_size(int B, int D, int L, int W, size_t* bytes);
+
+/* ---------------------------------------------------------------------------
+ * ssm_conv1d_bwd — gradients of ssm_conv1d_fwd's output u.
+ *   du       [B][D][L] dtype   upstream gradient dL/du
+ *   dx       [B][D][L] dtype   output dL/dx
+ *   dw       [D][W]    fp32    output dL/dw (summed over batch and time)
+ *   dbias    [D]       fp32, nullable   output dL/dbias
+ *   workspace            device scratch of ssm_conv1d_bwd_workspace_size bytes
+ * The pre-activation is recomputed from x, w, bias (nothing is saved by fwd).
+ * ------------------------------------------------------------------------ */
+ssm_status_t ssm_conv1d_bwd(const void* x, const float* w, const float* bias,
+                            const int32_t* seq_idx, const void* du, void* dx,
+                            float* dw, float* dbias, int B, int D, int L, int W,
+                            ssm_dtype_t dtype, int silu, void* workspace,
+                            size_t workspace_bytes, ssm_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Selective scan. For each row (b, d) and state n < N, with
+ *   dt_t = softplus(delta[b][d][t] + delta_bias[d])   (or without softplus)
+ *   a_t  = exp(dt_t * A[d][n])      (0 at the first token of a document)
+ *   h_t  = a_t * h_{t-1} + dt_t * Bm[b][n][t] * u[b][d][t],   h_{-1} = 0
+ *   y_t  = sum_n Cm[b][n][t] * h_t + Dskip[d] * u[b][d][t]
+ *   out  = y_t * silu(z[b][d][t])   (or y_t when z is NULL)
+ * final_state[b][d][n] = h_{L-1}.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    size_t struct_size;        /* = sizeof(ssm_scan_params) */
+    int B, D, L, N;
+    ssm_dtype_t dtype;         /* dtype of u, delta, z, Bm, Cm, out */
+    const void* u;             /* [B][D][L] scan input x (the conv+SiLU output) */
+    const void* delta;         /* [B][D][L] raw step, before bias and softplus */
+    const void* z;             /* [B][D][L] gate input, nullable (no gate) */
+    const float* A;            /* [D][N] state matrix diagonal (negative for decay) */
+    const float* Dskip;        /* [D] nullable (0) */
+    const float* delta_bias;   /* [D] nullable (0) */
+    const void* Bm;            /* [B][N][L] */
+    const void* Cm;            /* [B][N][L] */
+    int delta_softplus;        /* 1: dt = softplus(delta + bias); 0: dt = delta + bias */
+    const int32_t* seq_idx;    /* [B][L] nullable */
+    const int32_t* cu_seqlens; /* [n_docs + 1] nullable, B == 1 only, exclusive with seq_idx;
+                                  cu_seqlens[0] = 0, increasing, cu_seqlens[n_docs] == L */
+    int n_docs;
+    int n_splits;              /* 0: automatic. P >= 1: split each row's L into P ranges
+                                  run on different CTAs and joined by a carry pass */
+    void* out;                 /* [B][D][L] output */
+    float* final_state;        /* [B][D][N] nullable */
+    void* workspace;           /* device scratch, >= ssm_scan_workspace_size bytes, 256-B aligned */
+    size_t workspace_bytes;
+} ssm_scan_params;
+
+/* Workspace bytes for these params: per-chunk state checkpoints (read by the
+ * backward), split carries, segment ids built from cu_seqlens, and partial
+ * sums of the backward's parameter reductions. */
+ssm_status_t ssm_scan_workspace_size(const ssm_scan_params* p, size_t* bytes);
+
+/* Forward. Also writes the checkpoints the backward reads into p->workspace:
+ * keep the workspace unchanged between ssm_scan_fwd and ssm_scan_bwd. */
+ssm_status_t ssm_scan_fwd(const ssm_scan_params* p, ssm_stream_t stream);
+
+typedef struct {
+    size_t struct_size;        /* = sizeof(ssm_scan_grads) */
+    const void* dout;          /* [B][D][L] dtype, dL/dout */
+    void* du;                  /* [B][D][L] dtype, output dL/du */
+    void* ddelta;              /* [B][D][L] dtype, output dL/d(raw delta) */
+    void* dz;                  /* [B][D][L] dtype, output dL/dz; required iff z != NULL */
+    float* dA;                 /* [D][N] output */
+    float* dB;                 /* [B][N][L] fp32 output */
+    float* dC;                 /* [B][N][L] fp32 output */
+    float* dD;                 /* [D] nullable output */
+    float* ddelta_bias;        /* [D] nullable output */
+    int deterministic;         /* reserved; dA, dD, ddelta_bias are always reduced in a fixed
+                                  order, dB and dC are summed over channels with fp32 atomics */
+} ssm_scan_grads;
+
+/* Backward. Recomputes states from the checkpoints in p->workspace, so the
+ * same params (inputs and workspace) as the forward must be passed. The final
+ * state is not differentiated (it has no incoming gradient). */
+ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
+                          ssm_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SSMSCAN_H */

@@ -1,0 +1,210 @@
+"""B200 (sm_100a) Mamba-1 selective-SSM layer core: torch-facing binding.
+
+Each function marshals torch CUDA tensors to the C ABI of libssmscan
+(include/ssmscan.h) and returns torch tensors; every step of the layer core
+runs in the library's kernels. Tensors must be CUDA and C-contiguous; layouts
+are activations [B, D, L], B/C [B, N, L], A [D, N], per-channel vectors [D],
+conv weight [D, 4], seq_idx int32 [B, L]. Activations are bf16 or fp32;
+parameters and the gradients of parameters, B and C are fp32.
+"""
+from __future__ import annotations
+
+import ctypes
+
+from . import _lib
+from ._lib import (SsmError, ssm_abi_version, ssm_conv1d_bwd, ssm_conv1d_bwd_workspace_size,
+                   ssm_conv1d_fwd, ssm_last_error, ssm_scan_bwd, ssm_scan_fwd,
+                   ssm_scan_grads, ssm_scan_params, ssm_scan_workspace_size)
+
+__all__ = [
+    "SsmError", "ssm_abi_version", "ssm_last_error", "ssm_conv1d_fwd", "ssm_conv1d_bwd",
+    "ssm_conv1d_bwd_workspace_size", "ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_scan_bwd",
+    "ssm_scan_params", "ssm_scan_grads", "conv1d_fwd", "conv1d_bwd", "scan_params",
+    "scan_workspace_size", "scan_fwd", "scan_bwd", "load",
+]
+
+load = _lib.load
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t):
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return _lib.SSM_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return _lib.SSM_DTYPE_F32
+    raise TypeError(f"activations must be bf16 or fp32, got {t.dtype}")
+
+
+def _need(t, name, dtype=None, shape=None):
+    torch = _torch()
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _stream(stream, device):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def conv1d_fwd(x, w, bias=None, seq_idx=None, *, silu=True, out=None, stream=None):
+    """u = silu(causal depthwise conv1d(x)) (width 4, segment-masked taps)."""
+    torch = _torch()
+    B, D, L = x.shape
+    _need(x, "x", shape=(B, D, L))
+    _need(w, "w", torch.float32, (D, 4))
+    _need(bias, "bias", torch.float32, (D,))
+    _need(seq_idx, "seq_idx", torch.int32, (B, L))
+    if out is None:
+        out = torch.empty_like(x)
+    _need(out, "out", x.dtype, (B, D, L))
+    _lib.check(ssm_conv1d_fwd(_ptr(x), _ptr(w), _ptr(bias), _ptr(seq_idx), _ptr(out), B, D, L, 4,
+                              _dtype_code(x), int(silu), _stream(stream, x.device)))
+    return out
+
+
+def conv1d_bwd(x, w, bias, seq_idx, du, *, silu=True, dx=None, dw=None, dbias=None,
+               workspace=None, stream=None):
+    """Gradients of conv1d_fwd: returns (dx, dw, dbias)."""
+    torch = _torch()
+    B, D, L = x.shape
+    _need(x, "x", shape=(B, D, L))
+    _need(du, "du", x.dtype, (B, D, L))
+    _need(w, "w", torch.float32, (D, 4))
+    _need(bias, "bias", torch.float32, (D,))
+    _need(seq_idx, "seq_idx", torch.int32, (B, L))
+    dx = torch.empty_like(x) if dx is None else dx
+    dw = torch.empty((D, 4), dtype=torch.float32, device=x.device) if dw is None else dw
+    if dbias is None:
+        dbias = torch.empty((D,), dtype=torch.float32, device=x.device)
+    ws_bytes = ssm_conv1d_bwd_workspace_size(B, D, L, 4)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
+    _lib.check(ssm_conv1d_bwd(_ptr(x), _ptr(w), _ptr(bias), _ptr(seq_idx), _ptr(du), _ptr(dx),
+                              _ptr(dw), _ptr(dbias), B, D, L, 4, _dtype_code(x), int(silu),
+                              _ptr(workspace), workspace.numel(), _stream(stream, x.device)))
+    return dx, dw, dbias
+
+
+def scan_params(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softplus=True,
+                seq_idx=None, cu_seqlens=None, n_splits=0, out=None, final_state=None,
+                workspace=None) -> ssm_scan_params:
+    """Fill an ssm_scan_params from tensors (validating shapes and dtypes)."""
+    torch = _torch()
+    B, D, L = u.shape
+    N = A.shape[1]
+    _need(u, "u", shape=(B, D, L))
+    _need(delta, "delta", u.dtype, (B, D, L))
+    _need(z, "z", u.dtype, (B, D, L))
+    _need(A, "A", torch.float32, (D, N))
+    _need(Dskip, "Dskip", torch.float32, (D,))
+    _need(delta_bias, "delta_bias", torch.float32, (D,))
+    _need(Bm, "Bm", u.dtype, (B, N, L))
+    _need(Cm, "Cm", u.dtype, (B, N, L))
+    _need(seq_idx, "seq_idx", torch.int32, (B, L))
+    _need(cu_seqlens, "cu_seqlens", torch.int32)
+    _need(out, "out", u.dtype, (B, D, L))
+    _need(final_state, "final_state", torch.float32, (B, D, N))
+    p = ssm_scan_params()
+    p.struct_size = ctypes.sizeof(ssm_scan_params)
+    p.B, p.D, p.L, p.N = B, D, L, N
+    p.dtype = _dtype_code(u)
+    p.u, p.delta, p.z = u.data_ptr(), delta.data_ptr(), (z.data_ptr() if z is not None else None)
+    p.A = A.data_ptr()
+    p.Dskip = Dskip.data_ptr() if Dskip is not None else None
+    p.delta_bias = delta_bias.data_ptr() if delta_bias is not None else None
+    p.Bm, p.Cm = Bm.data_ptr(), Cm.data_ptr()
+    p.delta_softplus = int(softplus)
+    p.seq_idx = seq_idx.data_ptr() if seq_idx is not None else None
+    p.cu_seqlens = cu_seqlens.data_ptr() if cu_seqlens is not None else None
+    p.n_docs = (cu_seqlens.numel() - 1) if cu_seqlens is not None else 0
+    p.n_splits = int(n_splits)
+    p.out = out.data_ptr() if out is not None else None
+    p.final_state = final_state.data_ptr() if final_state is not None else None
+    p.workspace = workspace.data_ptr() if workspace is not None else None
+    p.workspace_bytes = workspace.numel() if workspace is not None else 0
+    return p
+
+
+def scan_workspace_size(p: ssm_scan_params) -> int:
+    return ssm_scan_workspace_size(p)
+
+
+def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softplus=True,
+             seq_idx=None, cu_seqlens=None, n_splits=0, return_final_state=False, out=None,
+             workspace=None, stream=None):
+    """Selective scan forward.
+
+    Returns (out, final_state or None, workspace). Keep `workspace` (it holds
+    the per-chunk state checkpoints) and pass it to scan_bwd unchanged.
+    """
+    torch = _torch()
+    B, D, L = u.shape
+    N = A.shape[1]
+    out = torch.empty_like(u) if out is None else out
+    fs = torch.empty((B, D, N), dtype=torch.float32, device=u.device) if return_final_state else None
+    p = scan_params(u, delta, A, Bm, Cm, z=z, Dskip=Dskip, delta_bias=delta_bias, softplus=softplus,
+                    seq_idx=seq_idx, cu_seqlens=cu_seqlens, n_splits=n_splits, out=out,
+                    final_state=fs)
+    need = ssm_scan_workspace_size(p)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=u.device)
+    p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    _lib.check(ssm_scan_fwd(p, _stream(stream, u.device)))
+    return out, fs, workspace
+
+
+def scan_bwd(u, delta, A, Bm, Cm, dout, workspace, *, z=None, Dskip=None, delta_bias=None,
+             softplus=True, seq_idx=None, cu_seqlens=None, n_splits=0, grads=None, stream=None):
+    """Selective scan backward; `workspace` must come from the matching scan_fwd.
+
+    Returns a dict: du, ddelta (w.r.t. the raw delta), dz (or None), dA, dB,
+    dC, dD, ddelta_bias. Preallocated outputs may be passed in `grads`.
+    """
+    torch = _torch()
+    B, D, L = u.shape
+    N = A.shape[1]
+    _need(dout, "dout", u.dtype, (B, D, L))
+    g = dict(grads or {})
+    dev = u.device
+    g.setdefault("du", torch.empty_like(u))
+    g.setdefault("ddelta", torch.empty_like(u))
+    g.setdefault("dz", torch.empty_like(u) if z is not None else None)
+    g.setdefault("dA", torch.empty((D, N), dtype=torch.float32, device=dev))
+    g.setdefault("dB", torch.empty((B, N, L), dtype=torch.float32, device=dev))
+    g.setdefault("dC", torch.empty((B, N, L), dtype=torch.float32, device=dev))
+    g.setdefault("dD", torch.empty((D,), dtype=torch.float32, device=dev))
+    g.setdefault("ddelta_bias", torch.empty((D,), dtype=torch.float32, device=dev))
+    p = scan_params(u, delta, A, Bm, Cm, z=z, Dskip=Dskip, delta_bias=delta_bias, softplus=softplus,
+                    seq_idx=seq_idx, cu_seqlens=cu_seqlens, n_splits=n_splits, out=None,
+                    workspace=workspace)
+    p.out = dout.data_ptr()  # not written by the backward; any valid activation pointer
+    gr = ssm_scan_grads()
+    gr.struct_size = ctypes.sizeof(ssm_scan_grads)
+    gr.dout = dout.data_ptr()
+    gr.du, gr.ddelta = g["du"].data_ptr(), g["ddelta"].data_ptr()
+    gr.dz = g["dz"].data_ptr() if g["dz"] is not None else None
+    gr.dA, gr.dB, gr.dC = g["dA"].data_ptr(), g["dB"].data_ptr(), g["dC"].data_ptr()
+    gr.dD = g["dD"].data_ptr() if g["dD"] is not None else None
+    gr.ddelta_bias = g["ddelta_bias"].data_ptr() if g["ddelta_bias"] is not None else None
+    _lib.check(ssm_scan_bwd(p, gr, _stream(stream, u.device)))
+    return g

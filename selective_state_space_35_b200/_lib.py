@@ -1,0 +1,141 @@
+"""ctypes binding of libssmscan (include/ssmscan.h).
+
+Argument marshalling only: every step of the layer core runs in the
+library's CUDA kernels. PyTorch supplies device memory and the stream. There
+is no CPU fallback: a missing library or a CPU tensor raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libssmscan.so")
+
+SSM_OK = 0
+SSM_ERR_INVALID_ARG = 1
+SSM_ERR_UNSUPPORTED = 2
+SSM_ERR_CUDA = 3
+SSM_ERR_TIMEOUT = 4
+SSM_ERR_INJECTED = 5
+SSM_DTYPE_F32 = 0
+SSM_DTYPE_BF16 = 1
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_sz = ctypes.c_size_t
+
+
+class SsmError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"libssmscan status {status}: {msg}")
+        self.status = status
+
+
+class ssm_scan_params(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", _sz),
+        ("B", _i), ("D", _i), ("L", _i), ("N", _i),
+        ("dtype", _i),
+        ("u", _vp), ("delta", _vp), ("z", _vp),
+        ("A", _vp), ("Dskip", _vp), ("delta_bias", _vp),
+        ("Bm", _vp), ("Cm", _vp),
+        ("delta_softplus", _i),
+        ("seq_idx", _vp), ("cu_seqlens", _vp), ("n_docs", _i),
+        ("n_splits", _i),
+        ("out", _vp), ("final_state", _vp),
+        ("workspace", _vp), ("workspace_bytes", _sz),
+    ]
+
+
+class ssm_scan_grads(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", _sz),
+        ("dout", _vp), ("du", _vp), ("ddelta", _vp), ("dz", _vp),
+        ("dA", _vp), ("dB", _vp), ("dC", _vp), ("dD", _vp), ("ddelta_bias", _vp),
+        ("deterministic", _i),
+    ]
+
+
+_lib = None
+
+EXPORTS = ("ssm_last_error", "ssm_abi_version", "ssm_conv1d_fwd", "ssm_conv1d_bwd_workspace_size",
+           "ssm_conv1d_bwd", "ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_scan_bwd")
+
+
+def load(path: str | None = None):
+    """Load libssmscan.so (built in-tree by build.py); raises if it is missing."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError(f"{p} is missing: build it with `python -m selective_state_space_35_b200.build`"
+                          " (the package has no CPU fallback)")
+    L = ctypes.CDLL(p)
+    L.ssm_last_error.restype = ctypes.c_char_p
+    L.ssm_last_error.argtypes = []
+    L.ssm_abi_version.restype = _i
+    L.ssm_abi_version.argtypes = []
+    L.ssm_conv1d_fwd.restype = _i
+    L.ssm_conv1d_fwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
+    L.ssm_conv1d_bwd_workspace_size.restype = _i
+    L.ssm_conv1d_bwd_workspace_size.argtypes = [_i, _i, _i, _i, ctypes.POINTER(_sz)]
+    L.ssm_conv1d_bwd.restype = _i
+    L.ssm_conv1d_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                 _vp, _sz, _vp]
+    L.ssm_scan_workspace_size.restype = _i
+    L.ssm_scan_workspace_size.argtypes = [ctypes.POINTER(ssm_scan_params), ctypes.POINTER(_sz)]
+    L.ssm_scan_fwd.restype = _i
+    L.ssm_scan_fwd.argtypes = [ctypes.POINTER(ssm_scan_params), _vp]
+    L.ssm_scan_bwd.restype = _i
+    L.ssm_scan_bwd.argtypes = [ctypes.POINTER(ssm_scan_params), ctypes.POINTER(ssm_scan_grads), _vp]
+    if path is None:
+        _lib = L
+    return L
+
+
+def check(status: int) -> None:
+    if status != SSM_OK:
+        raise SsmError(status, load().ssm_last_error().decode(errors="replace"))
+
+
+# Raw entry points with the ABI's own names (pointer-level).
+def ssm_last_error() -> str:
+    return load().ssm_last_error().decode(errors="replace")
+
+
+def ssm_abi_version() -> int:
+    return load().ssm_abi_version()
+
+
+def ssm_conv1d_fwd(*args) -> int:
+    return load().ssm_conv1d_fwd(*args)
+
+
+def ssm_conv1d_bwd_workspace_size(B, D, L, W) -> int:
+    n = _sz(0)
+    check(load().ssm_conv1d_bwd_workspace_size(B, D, L, W, ctypes.byref(n)))
+    return n.value
+
+
+def ssm_conv1d_bwd(*args) -> int:
+    return load().ssm_conv1d_bwd(*args)
+
+
+def ssm_scan_workspace_size(params: ssm_scan_params) -> int:
+    n = _sz(0)
+    check(load().ssm_scan_workspace_size(ctypes.byref(params), ctypes.byref(n)))
+    return n.value
+
+
+def _ref(x):
+    return None if x is None else ctypes.byref(x)
+
+
+def ssm_scan_fwd(params: ssm_scan_params, stream) -> int:
+    return load().ssm_scan_fwd(_ref(params), stream)
+
+
+def ssm_scan_bwd(params: ssm_scan_params, grads: ssm_scan_grads, stream) -> int:
+    return load().ssm_scan_bwd(_ref(params), _ref(grads), stream)

@@ -1,0 +1,337 @@
+// C ABI entry points (include/ssmscan.h): argument validation, workspace
+// layout, launch-shape choice, error reporting. No allocation happens here.
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+
+#include "../../include/ssmscan.h"
+#include "internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+ssm_status_t fail(ssm_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+ssm_status_t ok() {
+  g_err[0] = '\0';
+  return SSM_OK;
+}
+
+// Host-side fault injection: SSM_INJECT_FAIL="ssm_scan_fwd,ssm_conv1d_bwd"
+// makes the named calls fail before any launch. Never touches the device.
+bool injected(const char* name) {
+  const char* e = getenv("SSM_INJECT_FAIL");
+  if (!e || !*e) return false;
+  const size_t n = strlen(name);
+  for (const char* p = strstr(e, name); p; p = strstr(p + 1, name)) {
+    const bool start = p == e || p[-1] == ',';
+    const bool end = p[n] == '\0' || p[n] == ',';
+    if (start && end) return true;
+  }
+  return false;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t elem_size(ssm_dtype_t dt) { return dt == SSM_DTYPE_BF16 ? 2 : 4; }
+
+ssm_status_t cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return ok();
+  return fail(SSM_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr size_t kAlign = 256;
+size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+struct ScanPlan {
+  int nchunks, nsplits, chunks_per_split;
+  size_t off_seq, off_ckpt, off_sP, off_sH, off_sIn, off_pA, off_pD, off_pB, total;
+};
+
+ssm_status_t check_params(const ssm_scan_params* p) {
+  if (!p) return fail(SSM_ERR_INVALID_ARG, "params is NULL");
+  if (p->struct_size != sizeof(ssm_scan_params))
+    return fail(SSM_ERR_INVALID_ARG, "params.struct_size %zu != %zu", p->struct_size,
+                sizeof(ssm_scan_params));
+  if (p->B < 1 || p->D < 1 || p->L < 1 || p->N < 1)
+    return fail(SSM_ERR_INVALID_ARG, "sizes must be >= 1 (B=%d D=%d L=%d N=%d)", p->B, p->D,
+                p->L, p->N);
+  if (p->N > ssm::kNMax) return fail(SSM_ERR_UNSUPPORTED, "N=%d > %d", p->N, ssm::kNMax);
+  if (p->B > 65535) return fail(SSM_ERR_UNSUPPORTED, "B=%d > 65535", p->B);
+  if (p->dtype != SSM_DTYPE_F32 && p->dtype != SSM_DTYPE_BF16)
+    return fail(SSM_ERR_INVALID_ARG, "unknown dtype %d", (int)p->dtype);
+  if (p->n_splits < 0) return fail(SSM_ERR_INVALID_ARG, "n_splits=%d < 0", p->n_splits);
+  if (p->seq_idx && p->cu_seqlens)
+    return fail(SSM_ERR_INVALID_ARG, "seq_idx and cu_seqlens are mutually exclusive");
+  if (p->cu_seqlens && p->B != 1)
+    return fail(SSM_ERR_INVALID_ARG, "cu_seqlens requires B == 1 (B=%d)", p->B);
+  if (p->cu_seqlens && p->n_docs < 1)
+    return fail(SSM_ERR_INVALID_ARG, "cu_seqlens needs n_docs >= 1 (n_docs=%d)", p->n_docs);
+  return ok();
+}
+
+ScanPlan plan_scan(const ssm_scan_params* p) {
+  ScanPlan s{};
+  s.nchunks = (p->L + ssm::kChunk - 1) / ssm::kChunk;
+  int P = p->n_splits;
+  if (P == 0) {
+    // enough warps to keep every SM busy without splitting? (a split costs a
+    // second pass over all but the last range)
+    const long target = (long)sm_count() * 8;
+    const long rows = (long)p->B * p->D;
+    P = rows >= target ? 1 : (int)((target + rows - 1) / rows);
+  }
+  if (P > s.nchunks) P = s.nchunks;
+  if (P > 65535) P = 65535;
+  if (P < 1) P = 1;
+  s.chunks_per_split = (s.nchunks + P - 1) / P;
+  s.nsplits = (s.nchunks + s.chunks_per_split - 1) / s.chunks_per_split;
+  const size_t rows = (size_t)p->B * p->D;
+  size_t off = 0;
+  s.off_seq = off;
+  off += p->cu_seqlens ? up((size_t)p->B * p->L * sizeof(int32_t)) : 0;
+  s.off_ckpt = off;
+  off += up(rows * s.nchunks * p->N * sizeof(float));
+  const size_t per_split = up(rows * s.nsplits * p->N * sizeof(float));
+  s.off_sP = off;
+  off += s.nsplits > 1 ? per_split : 0;
+  s.off_sH = off;
+  off += s.nsplits > 1 ? per_split : 0;
+  s.off_sIn = off;
+  off += s.nsplits > 1 ? per_split : 0;
+  s.off_pA = off;
+  off += per_split;
+  s.off_pD = off;
+  off += up(rows * s.nsplits * sizeof(float));
+  s.off_pB = off;
+  off += up(rows * s.nsplits * sizeof(float));
+  s.total = off;
+  return s;
+}
+
+ssm_status_t build_args(const ssm_scan_params* p, const ScanPlan& pl, ssm::ScanArgs* a) {
+  char* ws = static_cast<char*>(p->workspace);
+  memset(a, 0, sizeof(*a));
+  a->u = p->u;
+  a->delta = p->delta;
+  a->z = p->z;
+  a->A = p->A;
+  a->Dskip = p->Dskip;
+  a->delta_bias = p->delta_bias;
+  a->Bm = p->Bm;
+  a->Cm = p->Cm;
+  a->seq = p->cu_seqlens ? reinterpret_cast<int32_t*>(ws + pl.off_seq) : p->seq_idx;
+  a->softplus = p->delta_softplus ? 1 : 0;
+  a->out = p->out;
+  a->final_state = p->final_state;
+  a->ckpt = reinterpret_cast<float*>(ws + pl.off_ckpt);
+  a->split_P = pl.nsplits > 1 ? reinterpret_cast<float*>(ws + pl.off_sP) : nullptr;
+  a->split_H = pl.nsplits > 1 ? reinterpret_cast<float*>(ws + pl.off_sH) : nullptr;
+  a->split_in = pl.nsplits > 1 ? reinterpret_cast<float*>(ws + pl.off_sIn) : nullptr;
+  a->part_dA = reinterpret_cast<float*>(ws + pl.off_pA);
+  a->part_dD = reinterpret_cast<float*>(ws + pl.off_pD);
+  a->part_ddb = reinterpret_cast<float*>(ws + pl.off_pB);
+  a->B = p->B;
+  a->D = p->D;
+  a->L = p->L;
+  a->N = p->N;
+  a->nchunks = pl.nchunks;
+  a->nsplits = pl.nsplits;
+  a->chunks_per_split = pl.chunks_per_split;
+  a->bf16 = p->dtype == SSM_DTYPE_BF16;
+  return ok();
+}
+
+ssm_status_t check_scan_buffers(const ssm_scan_params* p, const ScanPlan& pl) {
+  if (!p->u || !p->delta || !p->A || !p->Bm || !p->Cm || !p->out)
+    return fail(SSM_ERR_INVALID_ARG, "u, delta, A, Bm, Cm and out must be non-NULL");
+  if (!p->workspace) return fail(SSM_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned(p->workspace, kAlign))
+    return fail(SSM_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if (p->workspace_bytes < pl.total)
+    return fail(SSM_ERR_INVALID_ARG, "workspace_bytes %zu < required %zu", p->workspace_bytes,
+                pl.total);
+  const size_t es = elem_size(p->dtype);
+  const void* acts[] = {p->u, p->delta, p->z, p->Bm, p->Cm, p->out};
+  for (const void* q : acts)
+    if (q && !aligned(q, es)) return fail(SSM_ERR_INVALID_ARG, "activation pointer misaligned");
+  const void* f32s[] = {p->A, p->Dskip, p->delta_bias, p->final_state, p->seq_idx, p->cu_seqlens};
+  for (const void* q : f32s)
+    if (q && !aligned(q, 4)) return fail(SSM_ERR_INVALID_ARG, "fp32/int32 pointer misaligned");
+  return ok();
+}
+
+bool vec_ok(int L, std::initializer_list<const void*> ptrs) {
+  if (L % 8) return false;
+  for (const void* q : ptrs)
+    if (q && !aligned(q, 16)) return false;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ssm_last_error(void) { return g_err; }
+
+int ssm_abi_version(void) { return SSM_ABI_VERSION; }
+
+ssm_status_t ssm_conv1d_fwd(const void* x, const float* w, const float* bias,
+                            const int32_t* seq_idx, void* u, int B, int D, int L, int W,
+                            ssm_dtype_t dtype, int silu, ssm_stream_t stream) {
+  if (injected("ssm_conv1d_fwd")) return fail(SSM_ERR_INJECTED, "ssm_conv1d_fwd: injected failure");
+  if (!x || !w || !u) return fail(SSM_ERR_INVALID_ARG, "x, w and u must be non-NULL");
+  if (B < 1 || D < 1 || L < 1) return fail(SSM_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (W != 4) return fail(SSM_ERR_UNSUPPORTED, "conv width W=%d (only 4)", W);
+  if (B > 65535 || D > 65535) return fail(SSM_ERR_UNSUPPORTED, "B and D must be <= 65535");
+  if (dtype != SSM_DTYPE_F32 && dtype != SSM_DTYPE_BF16)
+    return fail(SSM_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (x == u) return fail(SSM_ERR_INVALID_ARG, "u may not alias x");
+  const size_t es = elem_size(dtype);
+  if (!aligned(x, es) || !aligned(u, es) || !aligned(w, 4) || (bias && !aligned(bias, 4)) ||
+      (seq_idx && !aligned(seq_idx, 4)))
+    return fail(SSM_ERR_INVALID_ARG, "misaligned pointer");
+  ssm::ConvArgs a{};
+  a.x = x; a.w = w; a.bias = bias; a.seq = seq_idx; a.out = u;
+  a.B = B; a.D = D; a.L = L; a.silu = silu ? 1 : 0;
+  a.bf16 = dtype == SSM_DTYPE_BF16;
+  a.vec = vec_ok(L, {x, u, seq_idx});
+  return cuda_status(ssm::launch_conv1d_fwd(a, reinterpret_cast<cudaStream_t>(stream)),
+                     "ssm_conv1d_fwd launch");
+}
+
+ssm_status_t ssm_conv1d_bwd_workspace_size(int B, int D, int L, int W, size_t* bytes) {
+  if (!bytes) return fail(SSM_ERR_INVALID_ARG, "bytes is NULL");
+  if (B < 1 || D < 1 || L < 1) return fail(SSM_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (W != 4) return fail(SSM_ERR_UNSUPPORTED, "conv width W=%d (only 4)", W);
+  *bytes = up((size_t)B * ssm::conv_tiles(L) * D * 5 * sizeof(float));
+  return ok();
+}
+
+ssm_status_t ssm_conv1d_bwd(const void* x, const float* w, const float* bias,
+                            const int32_t* seq_idx, const void* du, void* dx, float* dw,
+                            float* dbias, int B, int D, int L, int W, ssm_dtype_t dtype,
+                            int silu, void* workspace, size_t workspace_bytes,
+                            ssm_stream_t stream) {
+  if (injected("ssm_conv1d_bwd")) return fail(SSM_ERR_INJECTED, "ssm_conv1d_bwd: injected failure");
+  if (!x || !w || !du || !dx || !dw)
+    return fail(SSM_ERR_INVALID_ARG, "x, w, du, dx and dw must be non-NULL");
+  size_t need = 0;
+  ssm_status_t st = ssm_conv1d_bwd_workspace_size(B, D, L, W, &need);
+  if (st != SSM_OK) return st;
+  if (B > 65535 || D > 65535) return fail(SSM_ERR_UNSUPPORTED, "B and D must be <= 65535");
+  if (dtype != SSM_DTYPE_F32 && dtype != SSM_DTYPE_BF16)
+    return fail(SSM_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (!workspace || workspace_bytes < need)
+    return fail(SSM_ERR_INVALID_ARG, "workspace too small (%zu < %zu)", workspace_bytes, need);
+  if (!aligned(workspace, 16)) return fail(SSM_ERR_INVALID_ARG, "workspace misaligned");
+  if (dx == x || dx == du) return fail(SSM_ERR_INVALID_ARG, "dx may not alias x or du");
+  const size_t es = elem_size(dtype);
+  if (!aligned(x, es) || !aligned(du, es) || !aligned(dx, es) || !aligned(w, 4) ||
+      !aligned(dw, 4) || (bias && !aligned(bias, 4)) || (dbias && !aligned(dbias, 4)) ||
+      (seq_idx && !aligned(seq_idx, 4)))
+    return fail(SSM_ERR_INVALID_ARG, "misaligned pointer");
+  ssm::ConvArgs a{};
+  a.x = x; a.w = w; a.bias = bias; a.seq = seq_idx; a.du = du; a.out = dx;
+  a.dw = dw; a.dbias = dbias; a.partial = static_cast<float*>(workspace);
+  a.B = B; a.D = D; a.L = L; a.silu = silu ? 1 : 0;
+  a.bf16 = dtype == SSM_DTYPE_BF16;
+  a.vec = vec_ok(L, {x, du, dx, seq_idx});
+  return cuda_status(ssm::launch_conv1d_bwd(a, reinterpret_cast<cudaStream_t>(stream)),
+                     "ssm_conv1d_bwd launch");
+}
+
+ssm_status_t ssm_scan_workspace_size(const ssm_scan_params* p, size_t* bytes) {
+  if (!bytes) return fail(SSM_ERR_INVALID_ARG, "bytes is NULL");
+  ssm_status_t st = check_params(p);
+  if (st != SSM_OK) return st;
+  *bytes = plan_scan(p).total;
+  return ok();
+}
+
+ssm_status_t ssm_scan_fwd(const ssm_scan_params* p, ssm_stream_t stream) {
+  if (injected("ssm_scan_fwd")) return fail(SSM_ERR_INJECTED, "ssm_scan_fwd: injected failure");
+  ssm_status_t st = check_params(p);
+  if (st != SSM_OK) return st;
+  const ScanPlan pl = plan_scan(p);
+  st = check_scan_buffers(p, pl);
+  if (st != SSM_OK) return st;
+  ssm::ScanArgs a;
+  build_args(p, pl, &a);
+  a.vec = vec_ok(p->L, {p->u, p->delta, p->z, p->Bm, p->Cm, p->out, a.seq});
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (p->cu_seqlens) {
+    cudaError_t e = ssm::launch_cu_seqlens_to_seq(p->cu_seqlens, p->n_docs, p->L,
+                                                  const_cast<int32_t*>(a.seq), s);
+    if (e != cudaSuccess) return cuda_status(e, "cu_seqlens conversion");
+  }
+  return cuda_status(ssm::launch_scan_fwd(a, s), "ssm_scan_fwd launch");
+}
+
+ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
+                          ssm_stream_t stream) {
+  if (injected("ssm_scan_bwd")) return fail(SSM_ERR_INJECTED, "ssm_scan_bwd: injected failure");
+  ssm_status_t st = check_params(p);
+  if (st != SSM_OK) return st;
+  if (!g) return fail(SSM_ERR_INVALID_ARG, "grads is NULL");
+  if (g->struct_size != sizeof(ssm_scan_grads))
+    return fail(SSM_ERR_INVALID_ARG, "grads.struct_size %zu != %zu", g->struct_size,
+                sizeof(ssm_scan_grads));
+  const ScanPlan pl = plan_scan(p);
+  st = check_scan_buffers(p, pl);
+  if (st != SSM_OK) return st;
+  if (!g->dout || !g->du || !g->ddelta || !g->dA || !g->dB || !g->dC)
+    return fail(SSM_ERR_INVALID_ARG, "dout, du, ddelta, dA, dB and dC must be non-NULL");
+  if (p->z && !g->dz) return fail(SSM_ERR_INVALID_ARG, "dz must be non-NULL when z is given");
+  const size_t es = elem_size(p->dtype);
+  const void* acts[] = {g->dout, g->du, g->ddelta, g->dz};
+  for (const void* q : acts)
+    if (q && !aligned(q, es)) return fail(SSM_ERR_INVALID_ARG, "gradient pointer misaligned");
+  const void* f32s[] = {g->dA, g->dB, g->dC, g->dD, g->ddelta_bias};
+  for (const void* q : f32s)
+    if (q && !aligned(q, 4)) return fail(SSM_ERR_INVALID_ARG, "fp32 gradient pointer misaligned");
+  ssm::ScanArgs a;
+  build_args(p, pl, &a);
+  a.dout = g->dout;
+  a.du = g->du;
+  a.ddelta = g->ddelta;
+  a.dz = p->z ? g->dz : nullptr;
+  a.dA = g->dA;
+  a.dB = g->dB;
+  a.dC = g->dC;
+  a.dD = g->dD;
+  a.ddelta_bias = g->ddelta_bias;
+  a.vec = vec_ok(p->L, {p->u, p->delta, p->z, p->Bm, p->Cm, g->dout, g->du, g->ddelta, a.dz, a.seq});
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (p->cu_seqlens) {
+    cudaError_t e = ssm::launch_cu_seqlens_to_seq(p->cu_seqlens, p->n_docs, p->L,
+                                                  const_cast<int32_t*>(a.seq), s);
+    if (e != cudaSuccess) return cuda_status(e, "cu_seqlens conversion");
+  }
+  const size_t bc = (size_t)p->B * p->N * p->L * sizeof(float);
+  cudaError_t e = cudaMemsetAsync(g->dB, 0, bc, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(g->dC, 0, bc, s);
+  if (e != cudaSuccess) return cuda_status(e, "ssm_scan_bwd memset");
+  return cuda_status(ssm::launch_scan_bwd(a, s), "ssm_scan_bwd launch");
+}
+
+}  // extern "C"

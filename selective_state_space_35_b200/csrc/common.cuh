@@ -1,0 +1,111 @@
+// Device-side helpers shared by the conv and scan kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssm {
+
+constexpr unsigned kFull = 0xffffffffu;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// 2^x on the special-function unit (PTX ex2.approx.ftz.f32).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float sigmoidf_(float v) { return 1.0f / (1.0f + expf(-v)); }
+
+// softplus(v) = log(1 + e^v); for v > 20 it equals v to within 2.1e-9.
+__device__ __forceinline__ float softplusf_(float v) {
+  return v > 20.0f ? v : log1pf(expf(v));
+}
+
+// ---------------------------------------------------------------------------
+// Element I/O: 8 consecutive elements per thread, fp32 in registers.
+// ---------------------------------------------------------------------------
+template <typename T>
+struct Io;
+
+template <>
+struct Io<float> {
+  static __device__ __forceinline__ float ld(const float* p) { return __ldg(p); }
+  static __device__ __forceinline__ void st(float* p, float v) { *p = v; }
+  // p must be 16-byte aligned
+  static __device__ __forceinline__ void ld8(const float* p, float v[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+  static __device__ __forceinline__ void st8(float* p, const float v[8]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+};
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+template <>
+struct Io<__nv_bfloat16> {
+  static __device__ __forceinline__ float ld(const __nv_bfloat16* p) {
+    return __bfloat162float(p[0]);
+  }
+  static __device__ __forceinline__ void st(__nv_bfloat16* p, float v) {
+    *p = __float2bfloat16_rn(v);
+  }
+  static __device__ __forceinline__ void ld8(const __nv_bfloat16* p, float v[8]) {
+    const uint4 r = __ldg(reinterpret_cast<const uint4*>(p));
+    v[0] = bf16lo(r.x); v[1] = bf16hi(r.x);
+    v[2] = bf16lo(r.y); v[3] = bf16hi(r.y);
+    v[4] = bf16lo(r.z); v[5] = bf16hi(r.z);
+    v[6] = bf16lo(r.w); v[7] = bf16hi(r.w);
+  }
+  static __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  }
+  static __device__ __forceinline__ void st8(__nv_bfloat16* p, const float v[8]) {
+    uint4 r;
+    r.x = pack2(v[0], v[1]);
+    r.y = pack2(v[2], v[3]);
+    r.z = pack2(v[4], v[5]);
+    r.w = pack2(v[6], v[7]);
+    *reinterpret_cast<uint4*>(p) = r;
+  }
+};
+
+// Load 8 elements starting at token t of a row of length L. VEC: L is a
+// multiple of 8 and the row is 16-byte aligned, so t < L means all 8 are in
+// range. Out-of-range elements read as 0.
+template <typename T, bool VEC>
+__device__ __forceinline__ void load_row8(const T* row, int t, int L, float v[8]) {
+  if (VEC) {
+    if (t < L) {
+      Io<T>::ld8(row + t, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.0f;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = (t + i < L) ? Io<T>::ld(row + t + i) : 0.0f;
+  }
+}
+
+template <typename T, bool VEC>
+__device__ __forceinline__ void store_row8(T* row, int t, int L, const float v[8]) {
+  if (VEC) {
+    if (t < L) Io<T>::st8(row + t, v);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (t + i < L) Io<T>::st(row + t + i, v[i]);
+  }
+}
+
+}  // namespace ssm

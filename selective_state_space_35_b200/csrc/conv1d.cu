@@ -1,0 +1,240 @@
+// Depthwise causal conv1d (width 4) + SiLU, forward and backward.
+//
+// Defined on "hung-phan ml-skills mamba", section "Mamba: Selective State
+// Spaces (S6)": Conv1d(d_inner, d_inner, d_conv, padding=d_conv-1,
+// groups=d_inner) on the channel-major activation, first L outputs kept, then
+// SiLU. Document resets follow "FLA Mamba and Mamba2" (packing paragraph):
+// a tap whose token lies in another document than the output token reads 0.
+//
+// HBM-bound: each thread owns 8 consecutive tokens of one (b, d) row, read
+// and written as one 16-byte vector (bf16) or two (fp32); the 3-token halo
+// on each side comes from L1 (its neighbours read those lines).
+#include "common.cuh"
+#include "internal.h"
+
+namespace ssm {
+
+namespace {
+
+template <typename T, bool VEC, bool SEQ>
+__global__ void __launch_bounds__(kConvThreads)
+conv1d_fwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
+                  const float* __restrict__ bias, const int32_t* __restrict__ seq,
+                  T* __restrict__ u, int D, int L, int silu) {
+  const int d = blockIdx.y, b = blockIdx.z;
+  const int t0 = (blockIdx.x * kConvThreads + threadIdx.x) * 8;
+  if (t0 >= L) return;
+  const size_t row = ((size_t)b * D + d) * L;
+  const T* xr = x + row;
+  float wk[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) wk[k] = __ldg(w + d * 4 + k);
+  const float bs = bias ? __ldg(bias + d) : 0.0f;
+
+  float xv[11];  // x[t0-3 .. t0+7]
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    const int s = t0 - 3 + i;
+    xv[i] = s >= 0 ? Io<T>::ld(xr + s) : 0.0f;
+  }
+  load_row8<T, VEC>(xr, t0, L, xv + 3);
+
+  int sg[11];
+  if (SEQ) {
+    const int32_t* sr = seq + (size_t)b * L;
+#pragma unroll
+    for (int i = 0; i < 11; ++i) {
+      const int s = t0 - 3 + i;
+      sg[i] = (s >= 0 && s < L) ? __ldg(sr + s) : 0;
+    }
+  }
+
+  float out[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float acc = bs;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      // tap k of output t0+i reads x_{t0+i-3+k} = xv[i+k]; xv is 0 before t=0
+      const bool ok = !SEQ || sg[i + k] == sg[i + 3];
+      acc = fmaf(wk[k], ok ? xv[i + k] : 0.0f, acc);
+    }
+    out[i] = silu ? acc * sigmoidf_(acc) : acc;
+  }
+  store_row8<T, VEC>(u + row, t0, L, out);
+}
+
+// dx_s = sum_k w_k dc_{s+3-k} [same document], dc_t = du_t * silu'(c_t).
+// Each thread recomputes c_t for its 8 tokens plus the 3 after them, writes
+// dx for its 8 tokens, and adds its tokens' share of dw and dbias into a
+// per-CTA partial (reduced over (b, tile) by conv1d_wreduce_kernel).
+template <typename T, bool VEC, bool SEQ>
+__global__ void __launch_bounds__(kConvThreads)
+conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
+                  const float* __restrict__ bias, const int32_t* __restrict__ seq,
+                  const T* __restrict__ du, T* __restrict__ dx,
+                  float* __restrict__ partial, int D, int L, int silu) {
+  const int d = blockIdx.y, b = blockIdx.z;
+  const int t0 = (blockIdx.x * kConvThreads + threadIdx.x) * 8;
+  const bool live = t0 < L;
+  const size_t row = ((size_t)b * D + d) * L;
+  const T* xr = x + row;
+  const T* dur = du + row;
+  float wk[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) wk[k] = __ldg(w + d * 4 + k);
+  const float bs = bias ? __ldg(bias + d) : 0.0f;
+
+  float xv[14];   // x[t0-3 .. t0+10]
+  float duv[11];  // du[t0 .. t0+10]
+  int sg[14];     // seg[t0-3 .. t0+10]
+#pragma unroll
+  for (int i = 0; i < 14; ++i) { xv[i] = 0.0f; sg[i] = 0; }
+#pragma unroll
+  for (int i = 0; i < 11; ++i) duv[i] = 0.0f;
+  if (live) {
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+      const int s = t0 - 3 + i;
+      if (s >= 0) xv[i] = Io<T>::ld(xr + s);
+    }
+    load_row8<T, VEC>(xr, t0, L, xv + 3);
+    load_row8<T, VEC>(dur, t0, L, duv);
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+      const int s = t0 + 8 + i;
+      if (s < L) {
+        xv[11 + i] = Io<T>::ld(xr + s);
+        duv[8 + i] = Io<T>::ld(dur + s);
+      }
+    }
+    if (SEQ) {
+      const int32_t* sr = seq + (size_t)b * L;
+#pragma unroll
+      for (int i = 0; i < 14; ++i) {
+        const int s = t0 - 3 + i;
+        sg[i] = (s >= 0 && s < L) ? __ldg(sr + s) : 0;
+      }
+    }
+  }
+
+  // dc for tokens t0 .. t0+10 (token t0+j: x window xv[j..j+3], segment sg[j+3])
+  float dc[11];
+#pragma unroll
+  for (int j = 0; j < 11; ++j) {
+    float c = bs;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const bool ok = !SEQ || sg[j + k] == sg[j + 3];
+      c = fmaf(wk[k], ok ? xv[j + k] : 0.0f, c);
+    }
+    float g = duv[j];
+    if (silu) {
+      const float sgm = sigmoidf_(c);
+      g *= sgm * (1.0f + c * (1.0f - sgm));
+    }
+    dc[j] = (t0 + j < L) ? g : 0.0f;
+  }
+
+  if (live) {
+    float o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float acc = 0.0f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int j = i + 3 - k;  // output token t0+j uses x_{t0+i} through tap k
+        const bool ok = !SEQ || sg[j + 3] == sg[i + 3];
+        acc = fmaf(wk[k], ok ? dc[j] : 0.0f, acc);
+      }
+      o[i] = acc;
+    }
+    store_row8<T, VEC>(dx + row, t0, L, o);
+  }
+
+  float pw[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const bool ok = !SEQ || sg[i + k] == sg[i + 3];
+      pw[k] = fmaf(dc[i], ok ? xv[i + k] : 0.0f, pw[k]);
+    }
+    pw[4] += dc[i];
+  }
+#pragma unroll
+  for (int k = 0; k < 5; ++k)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) pw[k] += __shfl_xor_sync(kFull, pw[k], off);
+  __shared__ float red[kConvThreads / 32][5];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0)
+#pragma unroll
+    for (int k = 0; k < 5; ++k) red[warp][k] = pw[k];
+  __syncthreads();
+  if (threadIdx.x < 5) {
+    float s = 0.0f;
+#pragma unroll
+    for (int wi = 0; wi < kConvThreads / 32; ++wi) s += red[wi][threadIdx.x];
+    partial[(((size_t)b * gridDim.x + blockIdx.x) * D + d) * 5 + threadIdx.x] = s;
+  }
+}
+
+// dw[d][k] = sum over (b, tile) of partial[b][tile][d][k], fixed order.
+__global__ void conv1d_wreduce_kernel(const float* __restrict__ partial, float* __restrict__ dw,
+                                      float* __restrict__ dbias, int B, int tiles, int D) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= D * 5) return;
+  const int d = i / 5, k = i % 5;
+  float s = 0.0f;
+  for (int b = 0; b < B; ++b)
+    for (int t = 0; t < tiles; ++t) s += partial[(((size_t)b * tiles + t) * D + d) * 5 + k];
+  if (k < 4) dw[d * 4 + k] = s;
+  else if (dbias) dbias[d] = s;
+}
+
+template <typename T, bool VEC, bool SEQ>
+void conv_fwd_t(const ConvArgs& a, cudaStream_t s) {
+  dim3 grid(conv_tiles(a.L), a.D, a.B);
+  conv1d_fwd_kernel<T, VEC, SEQ><<<grid, kConvThreads, 0, s>>>(
+      static_cast<const T*>(a.x), a.w, a.bias, a.seq, static_cast<T*>(a.out), a.D, a.L, a.silu);
+}
+
+template <typename T, bool VEC, bool SEQ>
+void conv_bwd_t(const ConvArgs& a, cudaStream_t s) {
+  dim3 grid(conv_tiles(a.L), a.D, a.B);
+  conv1d_bwd_kernel<T, VEC, SEQ><<<grid, kConvThreads, 0, s>>>(
+      static_cast<const T*>(a.x), a.w, a.bias, a.seq, static_cast<const T*>(a.du),
+      static_cast<T*>(a.out), a.partial, a.D, a.L, a.silu);
+  const int n = a.D * 5;
+  conv1d_wreduce_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.partial, a.dw, a.dbias, a.B,
+                                                        conv_tiles(a.L), a.D);
+}
+
+}  // namespace
+
+cudaError_t launch_conv1d_fwd(const ConvArgs& a, cudaStream_t s) {
+  const bool sq = a.seq != nullptr;
+  if (a.bf16) {
+    if (a.vec) { sq ? conv_fwd_t<__nv_bfloat16, true, true>(a, s) : conv_fwd_t<__nv_bfloat16, true, false>(a, s); }
+    else { sq ? conv_fwd_t<__nv_bfloat16, false, true>(a, s) : conv_fwd_t<__nv_bfloat16, false, false>(a, s); }
+  } else {
+    if (a.vec) { sq ? conv_fwd_t<float, true, true>(a, s) : conv_fwd_t<float, true, false>(a, s); }
+    else { sq ? conv_fwd_t<float, false, true>(a, s) : conv_fwd_t<float, false, false>(a, s); }
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_conv1d_bwd(const ConvArgs& a, cudaStream_t s) {
+  const bool sq = a.seq != nullptr;
+  if (a.bf16) {
+    if (a.vec) { sq ? conv_bwd_t<__nv_bfloat16, true, true>(a, s) : conv_bwd_t<__nv_bfloat16, true, false>(a, s); }
+    else { sq ? conv_bwd_t<__nv_bfloat16, false, true>(a, s) : conv_bwd_t<__nv_bfloat16, false, false>(a, s); }
+  } else {
+    if (a.vec) { sq ? conv_bwd_t<float, true, true>(a, s) : conv_bwd_t<float, true, false>(a, s); }
+    else { sq ? conv_bwd_t<float, false, true>(a, s) : conv_bwd_t<float, false, false>(a, s); }
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace ssm

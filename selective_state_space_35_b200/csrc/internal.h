@@ -1,0 +1,78 @@
+// Host-side internal interface between the C ABI (abi.cu) and the kernel
+// launchers. Not installed; the public interface is include/ssmscan.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace ssm {
+
+constexpr int kS = 8;                 // tokens per lane in the scan kernels
+constexpr int kChunk = 32 * kS;       // tokens per warp-chunk
+constexpr int kNMax = 16;             // largest supported state size
+constexpr int kConvThreads = 128;     // threads per conv CTA (8 tokens each)
+constexpr int kConvTile = kConvThreads * 8;
+
+struct ConvArgs {
+  const void* x;
+  const float* w;
+  const float* bias;
+  const int32_t* seq;
+  const void* du;     // bwd only
+  void* out;          // u (fwd) or dx (bwd)
+  float* dw;          // bwd only
+  float* dbias;       // bwd only, nullable
+  float* partial;     // bwd only: [B][tiles][D][5]
+  int B, D, L, silu;
+  bool bf16, vec;
+};
+
+cudaError_t launch_conv1d_fwd(const ConvArgs& a, cudaStream_t s);
+cudaError_t launch_conv1d_bwd(const ConvArgs& a, cudaStream_t s);
+inline int conv_tiles(int L) { return (L + kConvTile - 1) / kConvTile; }
+
+struct ScanArgs {
+  // inputs
+  const void* u;
+  const void* delta;
+  const void* z;
+  const float* A;
+  const float* Dskip;
+  const float* delta_bias;
+  const void* Bm;
+  const void* Cm;
+  const int32_t* seq;
+  int softplus;
+  // forward outputs
+  void* out;
+  float* final_state;
+  // backward inputs / outputs
+  const void* dout;
+  void* du;
+  void* ddelta;
+  void* dz;
+  float* dA;
+  float* dB;
+  float* dC;
+  float* dD;
+  float* ddelta_bias;
+  // workspace pieces
+  float* ckpt;        // [B*D][nchunks][N] state entering each chunk
+  float* split_P;     // [B*D][P][N] per-split decay product (pass 1)
+  float* split_H;     // [B*D][P][N] per-split end value from zero (pass 1)
+  float* split_in;    // [B*D][P][N] carry into each split
+  float* part_dA;     // [B*D][N]
+  float* part_dD;     // [B*D]
+  float* part_ddb;    // [B*D]
+  int B, D, L, N;
+  int nchunks, nsplits, chunks_per_split;
+  bool bf16, vec;
+};
+
+cudaError_t launch_scan_fwd(const ScanArgs& a, cudaStream_t s);
+cudaError_t launch_scan_bwd(const ScanArgs& a, cudaStream_t s);
+cudaError_t launch_cu_seqlens_to_seq(const int32_t* cu, int n_docs, int L, int32_t* seq,
+                                     cudaStream_t s);
+
+}  // namespace ssm

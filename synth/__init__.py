@@ -33,9 +33,13 @@ SEED_BASE = 20261202
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round float32 values to bfloat16 (RNE); return the raw uint16 bits."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    bias = 0x7FFF + ((u >> 16) & 1)
-    return ((u + bias) >> 16).astype(np.uint16)
+    u = x.view(np.uint32)
+    bias = (u >> 16) & np.uint32(1)
+    bias += np.uint32(0x7FFF)
+    # finite inputs cannot wrap: u + 0x8000 overflows only for NaN bit patterns
+    bias += u
+    bias >>= np.uint32(16)
+    return bias.astype(np.uint16)
 
 
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
@@ -136,14 +140,16 @@ class LayerInputs:
     extra: dict = field(default_factory=dict)
 
 
-def _act(rng: np.random.Generator, shape, dtype: str, scale: float = 1.0) -> Tensor:
+def _act(rng: np.random.Generator, shape, dtype: str, scale: float = 1.0,
+         want_f64: bool = True) -> Tensor:
     v = rng.standard_normal(shape, dtype=np.float32)
     if scale != 1.0:
         v *= np.float32(scale)
     if dtype == "bf16":
         bits = f32_to_bf16_bits(v)
-        return Tensor(f64=bf16_bits_to_f32(bits).astype(np.float64), bits=bits)
-    return Tensor(f64=v.astype(np.float64), f32=v)
+        f64 = bf16_bits_to_f32(bits).astype(np.float64) if want_f64 else None
+        return Tensor(f64=f64, bits=bits)
+    return Tensor(f64=v.astype(np.float64) if want_f64 else None, f32=v)
 
 
 def make_inputs(shape: Shape, seed: int, *, want_f64: bool = True,
@@ -167,21 +173,18 @@ def make_inputs(shape: Shape, seed: int, *, want_f64: bool = True,
              else np.ones(D, dtype=np.float32))
     dt0 = rng.uniform(1e-3, 1e-1, size=D)
     delta_bias = np.log(np.expm1(dt0)).astype(np.float32)  # inverse softplus
-    x = _act(rng, (B, D, L), shape.dtype)
-    z = _act(rng, (B, D, L), shape.dtype)
-    delta = _act(rng, (B, D, L), shape.dtype, 0.5)
-    Bm = _act(rng, (B, N, L), shape.dtype)
-    Cm = _act(rng, (B, N, L), shape.dtype)
-    dout = _act(rng, (B, D, L), shape.dtype)
+    x = _act(rng, (B, D, L), shape.dtype, want_f64=want_f64)
+    z = _act(rng, (B, D, L), shape.dtype, want_f64=want_f64)
+    delta = _act(rng, (B, D, L), shape.dtype, 0.5, want_f64=want_f64)
+    Bm = _act(rng, (B, N, L), shape.dtype, want_f64=want_f64)
+    Cm = _act(rng, (B, N, L), shape.dtype, want_f64=want_f64)
+    dout = _act(rng, (B, D, L), shape.dtype, want_f64=want_f64)
     seq = None
     if shape.packed:
         seq = np.stack([packed_seq_idx(rng, L) for _ in range(B)])
     elif shape.boundary_at is not None:
         seq = np.zeros((B, L), dtype=np.int32)
         seq[:, shape.boundary_at:] = 1
-    if not want_f64:
-        for t in (x, z, delta, Bm, Cm, dout):
-            t.f64 = None
     return LayerInputs(shape, x, z, delta, Bm, Cm, dout, A, Dskip, delta_bias,
                        conv_w, conv_b, seq)
 

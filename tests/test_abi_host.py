@@ -1,0 +1,153 @@
+"""Host-side checks of the C ABI: the library loads, exports every function
+include/ssmscan.h declares, and rejects bad arguments before any launch.
+No GPU is needed: every call here returns before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssmscan.h")
+
+
+@pytest.fixture(scope="module")
+def ssm():
+    from selective_state_space_35_b200 import build
+    build.build()
+    import selective_state_space_35_b200 as m
+    m.load()
+    return m
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ssm_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_expected_entry_points():
+    names = _declared()
+    for n in ("ssm_conv1d_fwd", "ssm_conv1d_bwd", "ssm_conv1d_bwd_workspace_size",
+              "ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_scan_bwd", "ssm_last_error",
+              "ssm_abi_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(ssm):
+    from selective_state_space_35_b200 import _lib
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (ssm_\w+)", out))
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+    lib = ctypes.CDLL(_lib.LIB_PATH)
+    for n in _declared():
+        assert hasattr(lib, n), n
+
+
+def test_abi_version(ssm):
+    src = open(HEADER).read()
+    v = int(re.search(r"#define SSM_ABI_VERSION (\d+)", src).group(1))
+    assert ssm.ssm_abi_version() == v
+
+
+def _params(ssm, **kw):
+    p = ssm.ssm_scan_params()
+    p.struct_size = ctypes.sizeof(ssm.ssm_scan_params)
+    p.B, p.D, p.L, p.N = 2, 8, 1000, 16
+    p.dtype = 1
+    p.delta_softplus = 1
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+def test_workspace_size_layout(ssm):
+    p = _params(ssm, n_splits=1)
+    n1 = ssm.ssm_scan_workspace_size(p)
+    nchunks = (1000 + 255) // 256
+    ckpt = 2 * 8 * nchunks * 16 * 4
+    assert n1 >= ckpt
+    p2 = _params(ssm, n_splits=3)
+    assert ssm.ssm_scan_workspace_size(p2) > n1
+    assert ssm.ssm_conv1d_bwd_workspace_size(2, 8, 1000, 4) >= 2 * 8 * 5 * 4
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("struct_size", 3, 1), ("B", 0, 1), ("N", 17, 2), ("N", 0, 1), ("dtype", 7, 1),
+    ("n_splits", -1, 1),
+])
+def test_scan_param_validation(ssm, field, value, status):
+    from selective_state_space_35_b200 import _lib
+    p = _params(ssm, **{field: value})
+    n = ctypes.c_size_t(0)
+    st = _lib.load().ssm_scan_workspace_size(ctypes.byref(p), ctypes.byref(n))
+    assert st == status
+    assert ssm.ssm_last_error()
+
+
+def test_scan_fwd_rejects_null_and_small_workspace(ssm):
+    from selective_state_space_35_b200 import _lib
+    p = _params(ssm)
+    assert ssm.ssm_scan_fwd(p, None) == _lib.SSM_ERR_INVALID_ARG  # null inputs
+    fake = 1 << 20  # never dereferenced: validation fails first
+    p = _params(ssm, u=fake, delta=fake, A=fake, Bm=fake, Cm=fake, out=fake, workspace=fake,
+                workspace_bytes=16)
+    assert ssm.ssm_scan_fwd(p, None) == _lib.SSM_ERR_INVALID_ARG
+    assert "workspace" in ssm.ssm_last_error()
+    p = _params(ssm, u=fake, delta=fake, A=fake, Bm=fake, Cm=fake, out=fake, workspace=fake + 8,
+                workspace_bytes=1 << 30)
+    assert ssm.ssm_scan_fwd(p, None) == _lib.SSM_ERR_INVALID_ARG
+    assert "aligned" in ssm.ssm_last_error()
+
+
+def test_cu_seqlens_rules(ssm):
+    from selective_state_space_35_b200 import _lib
+    fake = 1 << 20
+    p = _params(ssm, seq_idx=fake, cu_seqlens=fake, n_docs=2)
+    n = ctypes.c_size_t(0)
+    assert _lib.load().ssm_scan_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 1
+    p = _params(ssm, cu_seqlens=fake, n_docs=2)  # B=2
+    assert _lib.load().ssm_scan_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 1
+    p = _params(ssm, B=1, cu_seqlens=fake, n_docs=0)
+    assert _lib.load().ssm_scan_workspace_size(ctypes.byref(p), ctypes.byref(n)) == 1
+
+
+def test_conv_validation(ssm):
+    fake = ctypes.c_void_p(1 << 20)
+    assert ssm.ssm_conv1d_fwd(None, fake, None, None, fake, 1, 1, 8, 4, 1, 1, None) == 1
+    assert ssm.ssm_conv1d_fwd(fake, fake, None, None, fake, 1, 1, 8, 4, 1, 1, None) == 1  # u aliases x
+    other = ctypes.c_void_p((1 << 20) + 4096)
+    assert ssm.ssm_conv1d_fwd(fake, fake, None, None, other, 1, 1, 8, 3, 1, 1, None) == 2  # W=3
+    assert ssm.ssm_conv1d_fwd(fake, fake, None, None, other, 1, 0, 8, 4, 1, 1, None) == 1
+    assert ssm.ssm_conv1d_bwd(fake, fake, None, None, fake, other, fake, None, 1, 1, 8, 4, 1, 1,
+                              None, 0, None) == 1  # workspace missing
+
+
+def test_fault_injection_is_host_only():
+    code = r"""
+import ctypes, os, sys
+sys.path.insert(0, %r)
+os.environ["SSM_INJECT_FAIL"] = "ssm_scan_fwd,ssm_conv1d_fwd"
+import selective_state_space_35_b200 as ssm
+p = ssm.ssm_scan_params()
+p.struct_size = ctypes.sizeof(p)
+assert ssm.ssm_scan_fwd(p, None) == 5, ssm.ssm_last_error()
+assert "injected" in ssm.ssm_last_error()
+assert ssm.ssm_conv1d_fwd(None, None, None, None, None, 1, 1, 1, 4, 1, 1, None) == 5
+# not named: normal validation
+assert ssm.ssm_scan_bwd(p, None, None) == 1
+""" % ROOT
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
+def test_binding_rejects_cpu_tensors(ssm):
+    torch = pytest.importorskip("torch")
+    x = torch.zeros(1, 2, 8, dtype=torch.bfloat16)
+    w = torch.zeros(2, 4)
+    with pytest.raises(ValueError):
+        ssm.conv1d_fwd(x, w)

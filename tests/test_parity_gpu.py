@@ -1,0 +1,359 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Same seeded inputs on both sides; the oracle never sees a GPU value. fp32:
+rel-L2 <= 1e-5 everywhere. bf16 inputs with fp32 state: out rel-L2 <= 2e-3
+and max-abs <= 2e-2 against the oracle rounded to bf16, gradients rel-L2 <=
+5e-3. Segment handling is checked exactly where it is exact (packed ==
+separate in the oracle) and by parity everywhere else.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from pipeline import (TOL_BF16_OUT, TOL_BF16_OUT_MAX, TOL_F32, TOL_GRAD, device_inputs, gpu_layer,
+                      host64, max_abs, rel_l2)
+
+pytestmark = pytest.mark.gpu
+
+GRAD_KEYS = ("du", "ddelta", "dz", "dA", "dB", "dC", "dD", "ddelta_bias", "dx", "dconv_w", "dconv_b")
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _compare_all(res, want, *, fp32, use_z=True, keys_out=("u", "out", "final_state")):
+    errs = {}
+    for k in keys_out:
+        if res.get(k) is None:
+            continue
+        w = want["u_stored"] if k == "u" else want[k]
+        if k in ("u", "out") and not fp32:
+            w = oracle.round_bf16(w)
+        errs[k] = rel_l2(host64(res[k]), w)
+        tol = TOL_F32 if fp32 else TOL_BF16_OUT
+        assert errs[k] <= tol, (k, errs[k])
+        if not fp32 and k == "out":
+            assert max_abs(host64(res[k]), w) <= TOL_BF16_OUT_MAX
+    for k in GRAD_KEYS:
+        if k == "dz" and not use_z:
+            continue
+        w = want[k]
+        if k in ("du", "ddelta", "dz", "dx") and not fp32:
+            w = oracle.round_bf16(w)
+        errs[k] = rel_l2(host64(res[k]), w)
+        tol = TOL_F32 if fp32 else TOL_GRAD
+        assert errs[k] <= tol, (k, errs[k])
+    return errs
+
+
+def _oracle_layer(inp, *, bf16_points, use_z=True, use_seq=True, softplus=True, nthreads=8):
+    seq = inp.seq_idx if use_seq else None
+    z = inp.z.f64 if use_z else None
+    c, u = oracle.conv1d_fwd(inp.x.f64, inp.conv_w, inp.conv_b, seq)
+    u_s = oracle.round_bf16(u) if bf16_points else u
+    kw = dict(z=z, Dskip=inp.Dskip, delta_bias=inp.delta_bias, softplus=softplus, seq_idx=seq,
+              nthreads=nthreads)
+    f = oracle.scan_fwd(u_s, inp.delta.f64, inp.A, inp.Bm.f64, inp.Cm.f64, **kw)
+    g = oracle.scan_bwd(u_s, inp.delta.f64, inp.A, inp.Bm.f64, inp.Cm.f64, inp.dout.f64, **kw)
+    du_s = oracle.round_bf16(g["du"]) if bf16_points else g["du"]
+    dx, dw, dcb = oracle.conv1d_bwd(inp.x.f64, inp.conv_w, inp.conv_b, seq, du_s)
+    r = {"u_stored": u_s, "dx": dx, "dconv_w": dw, "dconv_b": dcb}
+    r.update(f)
+    r.update(g)
+    return r
+
+
+def _small(B, D, N, L, seed, *, dtype="f32", nbound=0, packed=False, boundary_at=None):
+    sh = synth.Shape("test", B, D, N, L, dtype, packed=packed, boundary_at=boundary_at)
+    inp = synth.make_inputs(sh, seed, conv_bias_scale=0.3, dskip_random=True)
+    if nbound:
+        inp.seq_idx = synth.random_segments(np.random.Generator(np.random.PCG64(seed)), B, L, nbound)
+    return inp
+
+
+def test_config1_tiny_fp32_layer():
+    inp = synth.make_inputs(synth.CONFIGS[1], synth.seed_for(1))
+    res = gpu_layer(device_inputs(inp))
+    want = _oracle_layer(inp, bf16_points=False)
+    _compare_all(res, want, fp32=True)
+
+
+SMALL_CASES = [
+    # B, D, N, L, nbound
+    (1, 1, 1, 1, 0),
+    (1, 3, 4, 7, 0),
+    (2, 5, 16, 64, 3),
+    (1, 4, 8, 255, 5),
+    (1, 4, 16, 256, 4),
+    (2, 3, 16, 257, 6),
+    (1, 6, 5, 600, 9),
+    (2, 9, 16, 1031, 12),
+    (1, 4, 16, 2048, 0),
+]
+
+
+@pytest.mark.parametrize("B,D,N,L,nb", SMALL_CASES)
+def test_small_fp32_shapes(B, D, N, L, nb):
+    inp = _small(B, D, N, L, 1000 + L + D, nbound=nb)
+    res = gpu_layer(device_inputs(inp))
+    want = _oracle_layer(inp, bf16_points=False)
+    _compare_all(res, want, fp32=True)
+
+
+@pytest.mark.parametrize("B,D,N,L,nb", [(1, 5, 16, 520, 7), (2, 4, 16, 1024, 5), (1, 3, 4, 13, 2)])
+def test_small_bf16_shapes(B, D, N, L, nb):
+    inp = _small(B, D, N, L, 2000 + L, dtype="bf16", nbound=nb)
+    res = gpu_layer(device_inputs(inp))
+    want = _oracle_layer(inp, bf16_points=True)
+    _compare_all(res, want, fp32=False)
+
+
+def test_one_token_documents_and_edge_boundaries():
+    B, D, N, L = 1, 4, 16, 300
+    inp = _small(B, D, N, L, 77)
+    seq = np.zeros((B, L), dtype=np.int32)
+    doc = 0
+    for t in range(L):  # 1-token documents at the start, chunk edge, and end
+        if t in (1, 2, 3, 4, 255, 256, 257, 298, 299) or t % 37 == 0:
+            doc += 1
+        seq[0, t] = doc
+    inp.seq_idx = seq
+    res = gpu_layer(device_inputs(inp))
+    want = _oracle_layer(inp, bf16_points=False)
+    _compare_all(res, want, fp32=True)
+
+
+@pytest.mark.parametrize("use_z,softplus,noD", [(False, True, False), (True, False, False),
+                                                 (False, False, True)])
+def test_optional_inputs(use_z, softplus, noD):
+    inp = _small(2, 5, 8, 333, 555, nbound=3)
+    if not softplus:
+        inp.delta.f32 = np.abs(inp.delta.f32) * np.float32(0.2)
+        inp.delta.f64 = inp.delta.f32.astype(np.float64)
+    if noD:
+        inp.Dskip = np.zeros_like(inp.Dskip)
+    res = gpu_layer(device_inputs(inp), use_z=use_z, softplus=softplus)
+    want = _oracle_layer(inp, bf16_points=False, use_z=use_z, softplus=softplus)
+    _compare_all(res, want, fp32=True, use_z=use_z)
+
+
+@pytest.mark.parametrize("P", [2, 3, 5])
+def test_forced_splits_fp32(P):
+    inp = _small(2, 5, 16, 1500, 31 + P, nbound=4)
+    res = gpu_layer(device_inputs(inp), n_splits=P)
+    want = _oracle_layer(inp, bf16_points=False)
+    _compare_all(res, want, fp32=True)
+
+
+def test_config2_bf16_full():
+    inp = synth.make_inputs(synth.CONFIGS[2], synth.seed_for(2))
+    res = gpu_layer(device_inputs(inp))
+    want = _oracle_layer(inp, bf16_points=True)
+    _compare_all(res, want, fp32=False)
+
+
+def test_config2_splits_match_unsplit():
+    torch = _torch()
+    inp = synth.make_inputs(synth.CONFIGS[2], synth.seed_for(2, 1))
+    dv = device_inputs(inp)
+    r1 = gpu_layer(dv, n_splits=1)
+    r4 = gpu_layer(dv, n_splits=4)
+    for k in ("out", "final_state", "du", "ddelta", "dz", "dA", "dB", "dC", "dD", "dx"):
+        assert rel_l2(host64(r4[k]), host64(r1[k])) <= 1e-3, k
+    torch.cuda.synchronize()
+
+
+def test_cu_seqlens_equals_seq_idx():
+    torch = _torch()
+    import selective_state_space_35_b200 as ssm
+    B, D, N, L = 1, 6, 16, 777
+    inp = _small(B, D, N, L, 91)
+    cuts = [0, 1, 100, 256, 257, 600, 776, L]
+    seq = np.zeros((1, L), dtype=np.int32)
+    for i in range(len(cuts) - 1):
+        seq[0, cuts[i]:cuts[i + 1]] = i
+    inp.seq_idx = seq
+    dv = device_inputs(inp)
+    cu = torch.tensor(cuts, dtype=torch.int32, device="cuda")
+    u = ssm.conv1d_fwd(dv["x"], dv["conv_w"], dv["conv_b"], dv["seq_idx"])
+    kw = dict(z=dv["z"], Dskip=dv["Dskip"], delta_bias=dv["delta_bias"])
+    o1, f1, w1 = ssm.scan_fwd(u, dv["delta"], dv["A"], dv["Bm"], dv["Cm"], seq_idx=dv["seq_idx"],
+                              return_final_state=True, **kw)
+    o2, f2, w2 = ssm.scan_fwd(u, dv["delta"], dv["A"], dv["Bm"], dv["Cm"], cu_seqlens=cu,
+                              return_final_state=True, **kw)
+    assert torch.equal(o1, o2) and torch.equal(f1, f2)
+    g1 = ssm.scan_bwd(u, dv["delta"], dv["A"], dv["Bm"], dv["Cm"], dv["dout"], w1,
+                      seq_idx=dv["seq_idx"], **kw)
+    g2 = ssm.scan_bwd(u, dv["delta"], dv["A"], dv["Bm"], dv["Cm"], dv["dout"], w2, cu_seqlens=cu,
+                      **kw)
+    for k in ("du", "ddelta", "dz", "dA", "dD", "ddelta_bias"):
+        assert torch.equal(g1[k], g2[k]), k
+    for k in ("dB", "dC"):
+        assert rel_l2(host64(g2[k]), host64(g1[k])) <= 1e-6, k
+
+
+def test_run_twice_bitwise():
+    torch = _torch()
+    inp = _small(2, 9, 16, 1200, 5, dtype="bf16", nbound=3)
+    dv = device_inputs(inp)
+    r1 = gpu_layer(dv)
+    r2 = gpu_layer(dv)
+    for k in ("u", "out", "final_state", "du", "ddelta", "dz", "dA", "dD", "ddelta_bias", "dx",
+              "dconv_w", "dconv_b"):
+        assert torch.equal(r1[k], r2[k]), k
+
+
+def test_packed_equals_separate_on_gpu():
+    torch = _torch()
+    B, D, N, L = 1, 4, 16, 700
+    inp = _small(B, D, N, L, 606)
+    cuts = [0, 3, 260, 261, 512, L]
+    seq = np.zeros((1, L), dtype=np.int32)
+    for i in range(len(cuts) - 1):
+        seq[0, cuts[i]:cuts[i + 1]] = i
+    inp.seq_idx = seq
+    full = gpu_layer(device_inputs(inp))
+    for s, e in zip(cuts[:-1], cuts[1:]):
+        sub = _small(B, D, N, e - s, 606)
+        for name in ("x", "z", "delta", "dout"):
+            t = getattr(inp, name)
+            getattr(sub, name).f32 = np.ascontiguousarray(t.f32[:, :, s:e])
+        for name in ("Bm", "Cm"):
+            getattr(sub, name).f32 = np.ascontiguousarray(getattr(inp, name).f32[:, :, s:e])
+        for name in ("A", "Dskip", "delta_bias", "conv_w", "conv_b"):
+            setattr(sub, name, getattr(inp, name))
+        sub.seq_idx = None
+        part = gpu_layer(device_inputs(sub))
+        for k in ("u", "out", "du", "ddelta", "dz", "dx"):
+            a = host64(full[k])[:, :, s:e]
+            assert rel_l2(a, host64(part[k])) <= 1e-6, k
+        for k in ("dB", "dC"):
+            assert rel_l2(host64(full[k])[:, :, s:e], host64(part[k])) <= 1e-6, k
+    torch.cuda.synchronize()
+
+
+def test_output_red_zones_untouched():
+    torch = _torch()
+    import selective_state_space_35_b200 as ssm
+    B, D, N, L = 1, 3, 16, 300
+    inp = _small(B, D, N, L, 4242, dtype="bf16", nbound=2)
+    dv = device_inputs(inp)
+    pad = 64
+    n = B * D * L
+
+    def guarded():
+        buf = torch.full((n + 2 * pad,), float("nan"), dtype=torch.bfloat16, device="cuda")
+        return buf, buf[pad:pad + n].view(B, D, L)
+
+    bu, u = guarded()
+    ssm.conv1d_fwd(dv["x"], dv["conv_w"], dv["conv_b"], dv["seq_idx"], out=u)
+    bo, o = guarded()
+    _, _, ws = ssm.scan_fwd(u, dv["delta"], dv["A"], dv["Bm"], dv["Cm"], z=dv["z"],
+                            Dskip=dv["Dskip"], delta_bias=dv["delta_bias"], seq_idx=dv["seq_idx"],
+                            out=o)
+    bufs = {k: guarded() for k in ("du", "ddelta", "dz")}
+    ssm.scan_bwd(u, dv["delta"], dv["A"], dv["Bm"], dv["Cm"], dv["dout"], ws, z=dv["z"],
+                 Dskip=dv["Dskip"], delta_bias=dv["delta_bias"], seq_idx=dv["seq_idx"],
+                 grads={k: v[1] for k, v in bufs.items()})
+    bx, dx = guarded()
+    ssm.conv1d_bwd(dv["x"], dv["conv_w"], dv["conv_b"], dv["seq_idx"], bufs["du"][1], dx=dx)
+    torch.cuda.synchronize()
+    for buf in [bu, bo, bx] + [v[0] for v in bufs.values()]:
+        assert torch.isnan(buf[:pad]).all() and torch.isnan(buf[-pad:]).all()
+        assert not torch.isnan(buf[pad:-pad]).any()
+
+
+# ---------------------------------------------------------------------------
+# Full-size workloads: the GPU runs the whole layer in the benchmark's launch
+# configuration; the oracle computes sampled rows exactly (rows are
+# independent), dC on a prefix (it depends only on earlier tokens) and dB on
+# a suffix (it depends only on later tokens).
+# ---------------------------------------------------------------------------
+def _row_inputs(inp, b, d, t0=0, t1=None):
+    t1 = inp.shape.L if t1 is None else t1
+    sl = np.s_[b:b + 1, d:d + 1, t0:t1]
+    seq = None if inp.seq_idx is None else np.ascontiguousarray(inp.seq_idx[b:b + 1, t0:t1])
+    return sl, seq
+
+
+@pytest.mark.parametrize("cfg", [3, 4, 5])
+def test_full_size_sampled(cfg):
+    torch = _torch()
+    sh = synth.CONFIGS[cfg]
+    inp = synth.make_inputs(sh, synth.seed_for(cfg))
+    res = gpu_layer(device_inputs(inp))
+    torch.cuda.synchronize()
+    rng = np.random.Generator(np.random.PCG64(cfg))
+    ds = sorted(set(int(v) for v in rng.integers(0, sh.D, size=2)) | {sh.D - 1})
+    L = sh.L
+
+    def h(k, sl):  # copy only the sampled slice to the host
+        return host64(res[k][sl])
+
+    for d in ds:
+        dA = np.zeros(sh.N)
+        dD = ddb = 0.0
+        dw = np.zeros(4)
+        db = 0.0
+        for b in range(sh.B):
+            sl, seq = _row_inputs(inp, b, d)
+            x = inp.x.f64[sl]
+            w = inp.conv_w[d:d + 1]
+            cb = inp.conv_b[d:d + 1]
+            _, u = oracle.conv1d_fwd(x, w, cb, seq)
+            u_s = oracle.round_bf16(u)
+            assert rel_l2(h("u", sl), u_s) <= TOL_BF16_OUT
+            kw = dict(z=inp.z.f64[sl], Dskip=inp.Dskip[d:d + 1], delta_bias=inp.delta_bias[d:d + 1],
+                      seq_idx=seq)
+            Bm = inp.Bm.f64[b:b + 1]
+            Cm = inp.Cm.f64[b:b + 1]
+            f = oracle.scan_fwd(u_s, inp.delta.f64[sl], inp.A[d:d + 1], Bm, Cm, **kw)
+            o = h("out", sl)
+            assert rel_l2(o, oracle.round_bf16(f["out"])) <= TOL_BF16_OUT
+            assert max_abs(o, oracle.round_bf16(f["out"])) <= TOL_BF16_OUT_MAX
+            assert rel_l2(h("final_state", np.s_[b, d]), f["final_state"][0, 0]) <= TOL_BF16_OUT
+            g = oracle.scan_bwd(u_s, inp.delta.f64[sl], inp.A[d:d + 1], Bm, Cm, inp.dout.f64[sl], **kw)
+            for k in ("du", "ddelta", "dz"):
+                assert rel_l2(h(k, sl), oracle.round_bf16(g[k])) <= TOL_GRAD, (k, b, d)
+            dA += g["dA"][0]
+            dD += g["dD"][0]
+            ddb += g["ddelta_bias"][0]
+            dx, dwi, dbi = oracle.conv1d_bwd(x, w, cb, seq, oracle.round_bf16(g["du"]))
+            # dx depends on du, which the GPU rounds to bf16 on its own path
+            assert rel_l2(h("dx", sl), oracle.round_bf16(dx)) <= TOL_GRAD
+            dw += dwi[0]
+            db += dbi[0]
+        assert rel_l2(host64(res["dA"])[d], dA) <= TOL_GRAD
+        assert rel_l2(host64(res["dD"])[d], dD) <= TOL_GRAD
+        assert rel_l2(host64(res["ddelta_bias"])[d], ddb) <= TOL_GRAD
+        assert rel_l2(host64(res["dconv_w"])[d], dw) <= TOL_GRAD
+        assert rel_l2(host64(res["dconv_b"])[d], db) <= TOL_GRAD
+
+    # dC on a prefix of T tokens (all channels, batch row 0)
+    T = 384
+    sl = np.s_[0:1, :, 0:T]
+    seq = None if inp.seq_idx is None else np.ascontiguousarray(inp.seq_idx[0:1, :T])
+    _, u = oracle.conv1d_fwd(inp.x.f64[sl], inp.conv_w, inp.conv_b, seq)
+    u_s = oracle.round_bf16(u)
+    kw = dict(z=inp.z.f64[sl], Dskip=inp.Dskip, delta_bias=inp.delta_bias, seq_idx=seq, nthreads=8)
+    g = oracle.scan_bwd(u_s, inp.delta.f64[sl], inp.A, inp.Bm.f64[0:1, :, :T], inp.Cm.f64[0:1, :, :T],
+                        inp.dout.f64[sl], **kw)
+    assert rel_l2(h("dC", np.s_[0:1, :, :T]), g["dC"]) <= TOL_GRAD
+
+    # dB on a suffix of T tokens (conv needs 3 tokens of history)
+    b = sh.B - 1
+    s0 = L - T
+    slx = np.s_[b:b + 1, :, s0 - 3:L]
+    seqx = None if inp.seq_idx is None else np.ascontiguousarray(inp.seq_idx[b:b + 1, s0 - 3:L])
+    _, u = oracle.conv1d_fwd(inp.x.f64[slx], inp.conv_w, inp.conv_b, seqx)
+    u_s = oracle.round_bf16(u[:, :, 3:])
+    sl = np.s_[b:b + 1, :, s0:L]
+    seq = None if inp.seq_idx is None else np.ascontiguousarray(inp.seq_idx[b:b + 1, s0:L])
+    kw = dict(z=inp.z.f64[sl], Dskip=inp.Dskip, delta_bias=inp.delta_bias, seq_idx=seq, nthreads=8)
+    g = oracle.scan_bwd(u_s, inp.delta.f64[sl], inp.A, inp.Bm.f64[b:b + 1, :, s0:], inp.Cm.f64[b:b + 1, :, s0:],
+                        inp.dout.f64[sl], **kw)
+    assert rel_l2(h("dB", np.s_[b:b + 1, :, s0:]), g["dB"]) <= TOL_GRAD
+    assert rel_l2(h("du", sl), oracle.round_bf16(g["du"])) <= TOL_GRAD

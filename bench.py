@@ -282,6 +282,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", type=int, default=3)
     ap.add_argument("--n-splits", type=int, default=0)
+    ap.add_argument("--layers", type=int, default=0, help="limit the layer count (profiling)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -309,7 +310,8 @@ def main():
                                 device_id=device)
 
     sh = synth.CONFIGS[cfg]
-    inps = [synth.make_inputs(sh, synth.seed_for(cfg, l), want_f64=False) for l in range(sh.layers)]
+    nlayers = args.layers if args.layers > 0 else sh.layers
+    inps = [synth.make_inputs(sh, synth.seed_for(cfg, l), want_f64=False) for l in range(nlayers)]
     layers = [Layer(inp, device, args.n_splits) for inp in inps]
     stream = torch.cuda.current_stream(device)
 

@@ -130,9 +130,10 @@ def test_one_token_documents_and_edge_boundaries():
                                                  (False, False, True)])
 def test_optional_inputs(use_z, softplus, noD):
     inp = _small(2, 5, 8, 333, 555, nbound=3)
-    if not softplus:
+    if not softplus:  # the step is used as given: keep it positive
         inp.delta.f32 = np.abs(inp.delta.f32) * np.float32(0.2)
         inp.delta.f64 = inp.delta.f32.astype(np.float64)
+        inp.delta_bias = np.zeros_like(inp.delta_bias)
     if noD:
         inp.Dskip = np.zeros_like(inp.Dskip)
     res = gpu_layer(device_inputs(inp), use_z=use_z, softplus=softplus)

@@ -167,6 +167,20 @@ typedef struct {
 ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
                           ssm_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * ssm_probe_ex2_rate — diagnostic: measures this device's sustained rate of
+ * the ex2.approx.f32 instruction (base-2 exponential on the special-function
+ * unit), the instruction the scan issues once per (token, state). Launches a
+ * fixed microkernel (8 CTAs of 256 threads per SM, ~20 ms) on `stream`, times
+ * it with CUDA events and SYNCHRONISES the stream before returning.
+ *   sink            device scratch of >= 2048 * SM-count floats (never read back)
+ *   ex2_per_second  host output: ex2 results per second, whole device
+ * Not part of the layer's math (no counterpart on the pages): it supplies the
+ * measured SFU peak for the roofline the benchmark reports.
+ * ------------------------------------------------------------------------ */
+ssm_status_t ssm_probe_ex2_rate(float* sink, size_t sink_floats, double* ex2_per_second,
+                                ssm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

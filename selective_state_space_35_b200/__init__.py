@@ -13,13 +13,13 @@ import ctypes
 
 from . import _lib
 from ._lib import (SsmError, ssm_abi_version, ssm_conv1d_bwd, ssm_conv1d_bwd_workspace_size,
-                   ssm_conv1d_fwd, ssm_last_error, ssm_scan_bwd, ssm_scan_fwd,
-                   ssm_scan_grads, ssm_scan_params, ssm_scan_workspace_size)
+                   ssm_conv1d_fwd, ssm_last_error, ssm_probe_ex2_rate, ssm_scan_bwd,
+                   ssm_scan_fwd, ssm_scan_grads, ssm_scan_params, ssm_scan_workspace_size)
 
 __all__ = [
     "SsmError", "ssm_abi_version", "ssm_last_error", "ssm_conv1d_fwd", "ssm_conv1d_bwd",
     "ssm_conv1d_bwd_workspace_size", "ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_scan_bwd",
-    "ssm_scan_params", "ssm_scan_grads", "conv1d_fwd", "conv1d_bwd", "scan_params",
+    "ssm_scan_params", "ssm_scan_grads", "ssm_probe_ex2_rate", "probe_ex2_rate", "conv1d_fwd", "conv1d_bwd", "scan_params",
     "scan_workspace_size", "scan_fwd", "scan_bwd", "load",
 ]
 
@@ -64,6 +64,15 @@ def _stream(stream, device):
     torch = _torch()
     s = stream if stream is not None else torch.cuda.current_stream(device)
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def probe_ex2_rate(device=None) -> float:
+    """Measured ex2.approx.f32 results per second of the current device."""
+    torch = _torch()
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    sink = torch.empty(sms * 2048, dtype=torch.float32, device=dev)
+    return ssm_probe_ex2_rate(_ptr(sink), sink.numel(), _stream(None, dev))
 
 
 def conv1d_fwd(x, w, bias=None, seq_idx=None, *, silu=True, out=None, stream=None):

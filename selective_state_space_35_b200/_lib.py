@@ -64,11 +64,12 @@ EXPORTS = ("ssm_last_error", "ssm_abi_version", "ssm_conv1d_fwd", "ssm_conv1d_bw
 
 
 def load(path: str | None = None):
-    """Load libssmscan.so (built in-tree by build.py); raises if it is missing."""
+    """Load libssmscan.so (built in-tree by build.py; env SSM_LIBRARY may name
+    another build of it); raises if it is missing."""
     global _lib
     if _lib is not None and path is None:
         return _lib
-    p = path or LIB_PATH
+    p = path or os.environ.get("SSM_LIBRARY") or LIB_PATH
     if not os.path.exists(p):
         raise ImportError(f"{p} is missing: build it with `python -m selective_state_space_35_b200.build`"
                           " (the package has no CPU fallback)")
@@ -90,6 +91,8 @@ def load(path: str | None = None):
     L.ssm_scan_fwd.argtypes = [ctypes.POINTER(ssm_scan_params), _vp]
     L.ssm_scan_bwd.restype = _i
     L.ssm_scan_bwd.argtypes = [ctypes.POINTER(ssm_scan_params), ctypes.POINTER(ssm_scan_grads), _vp]
+    L.ssm_probe_ex2_rate.restype = _i
+    L.ssm_probe_ex2_rate.argtypes = [_vp, _sz, ctypes.POINTER(ctypes.c_double), _vp]
     if path is None:
         _lib = L
     return L
@@ -127,6 +130,12 @@ def ssm_scan_workspace_size(params: ssm_scan_params) -> int:
     n = _sz(0)
     check(load().ssm_scan_workspace_size(ctypes.byref(params), ctypes.byref(n)))
     return n.value
+
+
+def ssm_probe_ex2_rate(sink, sink_floats: int, stream) -> float:
+    r = ctypes.c_double(0.0)
+    check(load().ssm_probe_ex2_rate(sink, sink_floats, ctypes.byref(r), stream))
+    return r.value
 
 
 def _ref(x):

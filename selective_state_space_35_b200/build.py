@@ -42,17 +42,21 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, out: str | None = None,
+          defines: tuple = ()) -> str:
+    """Compile csrc/*.cu into `out` (default: the in-tree libssmscan.so)."""
+    lib = out or LIB
+    objdir = OBJDIR if out is None else out + ".objs"
+    if out is None and not force and not defines and up_to_date():
         return LIB
-    os.makedirs(OBJDIR, exist_ok=True)
+    os.makedirs(objdir, exist_ok=True)
     cc = nvcc()
     srcs = _sources()
-    objs = [os.path.join(OBJDIR, os.path.basename(s)[:-3] + ".o") for s in srcs]
+    objs = [os.path.join(objdir, os.path.basename(s)[:-3] + ".o") for s in srcs]
 
     def comp(pair):
         s, o = pair
-        cmd = [cc, *ARCH, *FLAGS, "-c", s, "-o", o]
+        cmd = [cc, *ARCH, *FLAGS, *[f"-D{d}" for d in defines], "-c", s, "-o", o]
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -64,13 +68,20 @@ def build(force: bool = False, verbose: bool = False) -> str:
         logs = list(ex.map(comp, zip(srcs, objs)))
     if verbose:
         print("\n".join(logs))
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     # cudart linked statically: the library does not depend on which CUDA
     # runtime (if any) the host process loaded.
     subprocess.run([cc, *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs], check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    import argparse
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("-v", action="store_true")
+    ap.add_argument("--out", default=None, help="write the library here instead of in-tree")
+    ap.add_argument("-D", action="append", default=[], help="preprocessor define (repeatable)")
+    a = ap.parse_args()
+    print(build(force=a.force, verbose=a.v, out=a.out, defines=tuple(a.D)))

@@ -110,8 +110,9 @@ ScanPlan plan_scan(const ssm_scan_params* p) {
   s.off_seq = off;
   off += p->cu_seqlens ? up((size_t)p->B * p->L * sizeof(int32_t)) : 0;
   s.off_ckpt = off;
-  off += up(rows * s.nchunks * p->N * sizeof(float));
-  const size_t per_split = up(rows * s.nsplits * p->N * sizeof(float));
+  const size_t npad = (size_t)((p->N + 1) & ~1);
+  off += up(rows * s.nchunks * npad * sizeof(float));
+  const size_t per_split = up(rows * s.nsplits * npad * sizeof(float));
   s.off_sP = off;
   off += s.nsplits > 1 ? per_split : 0;
   s.off_sH = off;
@@ -154,6 +155,7 @@ ssm_status_t build_args(const ssm_scan_params* p, const ScanPlan& pl, ssm::ScanA
   a->D = p->D;
   a->L = p->L;
   a->N = p->N;
+  a->Npad = (p->N + 1) & ~1;
   a->nchunks = pl.nchunks;
   a->nsplits = pl.nsplits;
   a->chunks_per_split = pl.chunks_per_split;
@@ -320,7 +322,9 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
   a.dC = g->dC;
   a.dD = g->dD;
   a.ddelta_bias = g->ddelta_bias;
-  a.vec = vec_ok(p->L, {p->u, p->delta, p->z, p->Bm, p->Cm, g->dout, g->du, g->ddelta, a.dz, a.seq});
+  // dB and dC take 16-byte vector atomics on the vector path
+  a.vec = vec_ok(p->L, {p->u, p->delta, p->z, p->Bm, p->Cm, g->dout, g->du, g->ddelta, a.dz, a.seq,
+                        g->dB, g->dC});
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (p->cu_seqlens) {
     cudaError_t e = ssm::launch_cu_seqlens_to_seq(p->cu_seqlens, p->n_docs, p->L,
@@ -332,6 +336,14 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
   if (e == cudaSuccess) e = cudaMemsetAsync(g->dC, 0, bc, s);
   if (e != cudaSuccess) return cuda_status(e, "ssm_scan_bwd memset");
   return cuda_status(ssm::launch_scan_bwd(a, s), "ssm_scan_bwd launch");
+}
+
+ssm_status_t ssm_probe_ex2_rate(float* sink, size_t sink_floats, double* ex2_per_second,
+                               ssm_stream_t stream) {
+  if (!sink || !ex2_per_second) return fail(SSM_ERR_INVALID_ARG, "sink and ex2_per_second must be non-NULL");
+  return cuda_status(ssm::probe_ex2_rate(sink, sink_floats, ex2_per_second,
+                                         reinterpret_cast<cudaStream_t>(stream)),
+                     "ssm_probe_ex2_rate");
 }
 
 }  // extern "C"

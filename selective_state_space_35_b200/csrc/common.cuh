@@ -19,6 +19,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
 
 __device__ __forceinline__ float sigmoidf_(float v) { return 1.0f / (1.0f + expf(-v)); }
 
+// sigmoid on the SFU: e^-v via ex2, reciprocal via rcp (relative error a few
+// ulp; 1 for v -> +inf, 0 for v -> -inf).
+__device__ __forceinline__ float sigmoid_fast(float v) {
+  return __fdividef(1.0f, 1.0f + __expf(-v));
+}
+
 // softplus(v) = log(1 + e^v); for v > 20 it equals v to within 2.1e-9.
 __device__ __forceinline__ float softplusf_(float v) {
   return v > 20.0f ? v : log1pf(expf(v));

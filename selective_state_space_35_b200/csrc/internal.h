@@ -58,20 +58,22 @@ struct ScanArgs {
   float* dD;
   float* ddelta_bias;
   // workspace pieces
-  float* ckpt;        // [B*D][nchunks][N] state entering each chunk
-  float* split_P;     // [B*D][P][N] per-split decay product (pass 1)
-  float* split_H;     // [B*D][P][N] per-split end value from zero (pass 1)
-  float* split_in;    // [B*D][P][N] carry into each split
+  float* ckpt;        // [B*D][nchunks][Npad] state entering each chunk
+  float* split_P;     // [B*D][P][Npad] per-split decay product (pass 1)
+  float* split_H;     // [B*D][P][Npad] per-split end value from zero (pass 1)
+  float* split_in;    // [B*D][P][Npad] carry into each split
   float* part_dA;     // [B*D][N]
   float* part_dD;     // [B*D]
   float* part_ddb;    // [B*D]
   int B, D, L, N;
+  int Npad;           // N rounded up to even: state pairs; stride of ckpt / split arrays
   int nchunks, nsplits, chunks_per_split;
   bool bf16, vec;
 };
 
 cudaError_t launch_scan_fwd(const ScanArgs& a, cudaStream_t s);
 cudaError_t launch_scan_bwd(const ScanArgs& a, cudaStream_t s);
+cudaError_t probe_ex2_rate(float* sink, size_t sink_floats, double* rate, cudaStream_t s);
 cudaError_t launch_cu_seqlens_to_seq(const int32_t* cu, int n_docs, int L, int32_t* seq,
                                      cudaStream_t s);
 

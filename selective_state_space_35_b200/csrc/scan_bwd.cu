@@ -12,23 +12,68 @@
 //   ddt_t  = u_t sum_n g_t B_nt + sum_n A_n q_t    -> d(raw delta) = ddt * sigmoid(v)
 //   dA_n  += dt_t q_t,  dB_nt += g_t dt_t u_t,  dC_nt += dy_t h_t
 //   dz_t   = dout_t y_t silu'(z_t),  dD += dy_t u_t
-// with dy_t = dout_t silu(z_t). dB and dC sum over every channel of a batch
-// row: the CTA's warps add into shared memory, then one fp32 atomic per
-// element and CTA goes to HBM. dA, dD and the delta-bias gradient are per-row
-// partials reduced over batch (and splits) in a fixed order by a small kernel.
+// with dy_t = dout_t silu(z_t).
+//
+// One state at a time, with the element-wise work packed two tokens per
+// fp32x2 instruction; the recurrences themselves are scalar chains. A lane's
+// product of a over its 8 tokens is one ex2 of the summed step. dB and dC sum
+// over every channel of a batch row: each warp writes its per-token values
+// into its own shared-memory slice (conflict-free 16-byte stores), the CTA
+// adds the slices and sends one float4 atomic per 4 tokens to HBM. dA, dD and
+// the delta-bias gradient are per-row partials reduced over batch (and
+// splits) in a fixed order by a small kernel.
 #include "scan_common.cuh"
+
+// Resident CTAs per SM the backward is compiled for (register budget).
+#ifndef SSM_BWD_MIN_BLOCKS
+#define SSM_BWD_MIN_BLOCKS 3
+#endif
 
 namespace ssm {
 
 namespace {
 
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
+
+// float4-piece layout of a [kNMax][kChunk] fp32 tile: lane j's tokens
+// [8j, 8j+4) at float4 index j, [8j+4, 8j+8) at 32 + j (per state row of 64).
+template <typename T, bool VEC>
+__device__ __forceinline__ void stage_rows(const T* __restrict__ M, float* s, int b, int N, int L,
+                                           int t0) {
+  for (int idx = threadIdx.x; idx < N * 32; idx += blockDim.x) {
+    const int n = idx >> 5, j = idx & 31;
+    float v[8];
+    load_row8<T, VEC>(M + ((size_t)b * N + n) * L, t0 + 8 * j, L, v);
+    float4* dst = reinterpret_cast<float4*>(s + n * kChunk);
+    dst[j] = make_float4(v[0], v[1], v[2], v[3]);
+    dst[32 + j] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+}
+
+__device__ __forceinline__ void lds_tokpairs(const float* row, int lane, float2 v[4]) {
+  const float4 q0 = reinterpret_cast<const float4*>(row)[lane];
+  const float4 q1 = reinterpret_cast<const float4*>(row)[32 + lane];
+  v[0] = make_float2(q0.x, q0.y);
+  v[1] = make_float2(q0.z, q0.w);
+  v[2] = make_float2(q1.x, q1.y);
+  v[3] = make_float2(q1.z, q1.w);
+}
+
+template <int G>
+struct BwdSmem {
+  float B[kNMax * kChunk];
+  float C[kNMax * kChunk];
+  __nv_bfloat16 raw[2][kNMax][kChunk];  // next chunk's raw B / C (async path)
+  float4 slice[2][G][2][64];            // [state parity][warp][dB | dC][piece]
+  float dA[G][kNMax][32];
+};
+
 template <typename T, int G, bool VEC>
-__global__ void __launch_bounds__(G * 32)
+__global__ void __launch_bounds__(G * 32, SSM_BWD_MIN_BLOCKS)
 scan_bwd_kernel(const ScanArgs p) {
-  __shared__ __align__(16) float sB[kNMax * kChunk];
-  __shared__ __align__(16) float sC[kNMax * kChunk];
-  __shared__ __align__(16) float sRed[2][2][kChunk];  // [n parity][dB | dC][chunk pos]
-  __shared__ float sdA[G][kNMax][32];
+  constexpr bool ASYNC = VEC && sizeof(T) == 2;  // B / C tiles by cp.async one chunk ahead
+  extern __shared__ float4 smem_dyn[];
+  BwdSmem<G>& sm = *reinterpret_cast<BwdSmem<G>*>(smem_dyn);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
@@ -55,93 +100,145 @@ scan_bwd_kernel(const ScanArgs p) {
   // lane n holds c_n = a g of the first token after the current chunk
   float gcarry = 0.0f;
   if (split + 1 < p.nsplits && active && lane < N)
-    gcarry = p.split_in[(rowid * p.nsplits + split) * N + lane];
+    gcarry = p.split_in[(rowid * p.nsplits + split) * p.Npad + lane];
 
-  for (int i = threadIdx.x; i < 4 * kChunk; i += blockDim.x) (&sRed[0][0][0])[i] = 0.0f;
+  {
+    float4* s = &sm.slice[0][0][0][0];
+    for (int i = threadIdx.x; i < 2 * G * 2 * 64; i += blockDim.x) s[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int n = 0; n < kNMax; ++n) sdA[warp][n][lane] = 0.0f;
+    for (int n = 0; n < kNMax; ++n) sm.dA[warp][n][lane] = 0.0f;
+  }
   float dDp = 0.0f, ddbp = 0.0f;
+
+  if (ASYNC)
+    issue_bc_raw(reinterpret_cast<const __nv_bfloat16*>(Bm), reinterpret_cast<const __nv_bfloat16*>(Cm),
+                 &sm.raw[0][0][0], 2, b, N, L, (c_end - 1) * kChunk);
+  Tok8<T, VEC> pf_dl, pf_u, pf_z, pf_go;
+  if (active) {
+    const int tl = (c_end - 1) * kChunk + lane * 8;
+    pf_dl.load(dl_row, tl, L);
+    pf_u.load(u_row, tl, L);
+    pf_go.load(go_row, tl, L);
+    if (z_row) pf_z.load(z_row, tl, L);
+  }
 
   for (int c = c_end - 1; c >= c_begin; --c) {
     const int t0 = c * kChunk;
-    __syncthreads();
-    stage_bc<T, VEC>(Bm, Cm, sB, sC, b, N, L, t0);
+    if (ASYNC) {
+      cp_async_wait_all();
+      __syncthreads();  // the previous chunk's readers of B / C are done
+      convert_bc_rows(&sm.raw[0][0][0], sm.B, sm.C, 2, N);
+      if (c - 1 >= c_begin)  // each thread refills only the pieces it just converted
+        issue_bc_raw(reinterpret_cast<const __nv_bfloat16*>(Bm),
+                     reinterpret_cast<const __nv_bfloat16*>(Cm), &sm.raw[0][0][0], 2, b, N, L,
+                     t0 - kChunk);
+    } else {
+      __syncthreads();
+      stage_rows<T, VEC>(Bm, sm.B, b, N, L, t0);
+      stage_rows<T, VEC>(Cm, sm.C, b, N, L, t0);
+    }
     __syncthreads();
 
     const int tl = t0 + lane * 8;
-    float dl[8], uu[8], xu[8], dy[8];
+    float2 dlp[4], xup[4], dyp[4];
+    float Sdl = 0.0f;
     unsigned rmask = 0u;
     float hck = 0.0f;
     if (active) {
-      float zz[8], go[8];
-      load_row8<T, VEC>(dl_row, tl, L, dl);
-      load_row8<T, VEC>(u_row, tl, L, uu);
-      load_row8<T, VEC>(go_row, tl, L, go);
-      if (z_row) load_row8<T, VEC>(z_row, tl, L, zz);
+      float dl[8], uu[8], go[8], zz[8];
+      pf_dl.get(dl);
+      pf_u.get(uu);
+      pf_go.get(go);
+      if (z_row) pf_z.get(zz);
+      if (c - 1 >= c_begin) {  // previous chunk's inputs, consumed next iteration
+        pf_dl.load(dl_row, tl - kChunk, L);
+        pf_u.load(u_row, tl - kChunk, L);
+        pf_go.load(go_row, tl - kChunk, L);
+        if (z_row) pf_z.load(z_row, tl - kChunk, L);
+      }
+      float dt[8], dy[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float v = dl[i] + bias;
-        const float s = p.softplus ? softplusf_(v) : v;
-        dl[i] = (tl + i < L) ? s : 0.0f;
-        xu[i] = dl[i] * uu[i];
-        dy[i] = z_row ? go[i] * (zz[i] * sigmoidf_(zz[i])) : go[i];
+        const float s = p.softplus ? (v > 20.0f ? v : log1pf(__expf(v))) : v;
+        dt[i] = (tl + i < L) ? s : 0.0f;
+        Sdl += dt[i];
+        dy[i] = z_row ? go[i] * (zz[i] * sigmoid_fast(zz[i])) : go[i];
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        dlp[k] = f2(dt[2 * k], dt[2 * k + 1]);
+        xup[k] = f2(dt[2 * k] * uu[2 * k], dt[2 * k + 1] * uu[2 * k + 1]);
+        dyp[k] = f2(dy[2 * k], dy[2 * k + 1]);
       }
       rmask = reset_mask(p.seq, b, L, tl);
-      if (lane < N) hck = p.ckpt[(rowid * p.nchunks + c) * N + lane];
+      if (lane < N) hck = p.ckpt[(rowid * p.nchunks + c) * p.Npad + lane];
     }
     const bool any_reset = __any_sync(kFull, rmask != 0u);
 
-    float y[8], sgB[8], dd[8];
+    float2 y2[4], sgB2[4], dd2[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) { y[i] = 0.0f; sgB[i] = 0.0f; dd[i] = 0.0f; }
+    for (int k = 0; k < 4; ++k) {
+      y2[k] = f2(0.f, 0.f);
+      sgB2[k] = f2(0.f, 0.f);
+      dd2[k] = f2(0.f, 0.f);
+    }
 
     for (int n = 0; n < N; ++n) {
-      float* red = &sRed[n & 1][0][0];
+      float4* mysl = &sm.slice[n & 1][warp][0][0];
       if (active) {
         const float An2 = __shfl_sync(kFull, A2_lane, n);
         const float Anat = __shfl_sync(kFull, A_lane, n);
-        float bv[8], cv[8];
-        lds8(sB + n * kChunk, lane, bv);
-        lds8(sC + n * kChunk, lane, cv);
+        float2 bp[4], cp[4];
+        lds_tokpairs(sm.B + n * kChunk, lane, bp);
+        lds_tokpairs(sm.C + n * kChunk, lane, cp);
         float a[8], bx[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          a[i] = ex2_approx(dl[i] * An2);
-          bx[i] = xu[i] * bv[i];
+        for (int k = 0; k < 4; ++k) {
+          const float2 e = fmul2(dlp[k], f2(An2, An2));
+          a[2 * k] = ex2_approx(e.x);
+          a[2 * k + 1] = ex2_approx(e.y);
+          const float2 q = fmul2(xup[k], bp[k]);
+          bx[2 * k] = q.x;
+          bx[2 * k + 1] = q.y;
         }
+        float Ploc = ex2_approx(An2 * Sdl);
         if (any_reset) {
 #pragma unroll
           for (int i = 0; i < 8; ++i)
             if ((rmask >> i) & 1u) a[i] = 0.0f;
+          if (rmask) Ploc = 0.0f;
         }
         // forward recompute of this lane's 8 states
-        float P = 1.0f, H = 0.0f;
+        float H = bx[0];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          H = fmaf(a[i], H, bx[i]);
-          P *= a[i];
-        }
-        const float Ploc = P;
+        for (int i = 1; i < 8; ++i) H = fmaf(a[i], H, bx[i]);
+        float P = Ploc;
         warp_scan_fwd(P, H, lane);
         const float hin = __shfl_sync(kFull, hck, n);
         const float end = fmaf(P, hin, H);
         float start = __shfl_up_sync(kFull, end, 1);
         if (lane == 0) start = hin;
         float hs[8];
-        float h = start;
+        {
+          float h = start;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          h = fmaf(a[i], h, bx[i]);
-          hs[i] = h;
-          y[i] = fmaf(cv[i], h, y[i]);
+          for (int i = 0; i < 8; ++i) {
+            h = fmaf(a[i], h, bx[i]);
+            hs[i] = h;
+          }
+        }
+        float2 hp[4], gy[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          hp[k] = f2(hs[2 * k], hs[2 * k + 1]);
+          y2[k] = ffma2(cp[k], hp[k], y2[k]);
+          gy[k] = fmul2(dyp[k], cp[k]);
         }
         // adjoint: lane map c_in -> c_out = a_first * g_first
-        float gy[8];
+        float Gl = gy[3].y;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) gy[i] = dy[i] * cv[i];
-        float Gl = gy[7];
-#pragma unroll
-        for (int i = 6; i >= 0; --i) Gl = fmaf(a[i + 1], Gl, gy[i]);
+        for (int i = 6; i >= 0; --i) Gl = fmaf(a[i + 1], Gl, (i & 1) ? gy[i >> 1].y : gy[i >> 1].x);
         float Gc = a[0] * Gl;
         float Pr = Ploc;
         warp_scan_bwd(Pr, Gc, lane);
@@ -152,54 +249,86 @@ scan_bwd_kernel(const ScanArgs p) {
         const float ncar = __shfl_sync(kFull, cout, 0);
         if (lane == n) gcarry = ncar;
 
-        float g = gy[7] + cin;
-        float dAl = 0.0f;
+        // reverse replay, two tokens at a time: g for tokens 2k+1 and 2k,
+        // then every per-token product for that pair
+        float2 dAp = f2(0.f, 0.f), dBp[4], dCp[4];
+        float g = gy[3].y + cin;
 #pragma unroll
-        for (int i = 7; i >= 0; --i) {
-          if (i < 7) g = fmaf(a[i + 1], g, gy[i]);
-          const float hp = i ? hs[i - 1] : start;
-          const float q = g * a[i] * hp;
-          dAl = fmaf(dl[i], q, dAl);
-          dd[i] = fmaf(Anat, q, dd[i]);
-          sgB[i] = fmaf(g, bv[i], sgB[i]);
-          atomicAdd(red + chunk_pos(lane, i), g * xu[i]);
-          atomicAdd(red + kChunk + chunk_pos(lane, i), dy[i] * hs[i]);
+        for (int k = 3; k >= 0; --k) {
+          const float g_hi = g;  // token 2k+1
+          const float g_lo = fmaf(a[2 * k + 1], g_hi, gy[k].x);  // token 2k
+          if (k > 0) g = fmaf(a[2 * k], g_lo, gy[k - 1].y);   // token 2k-1
+          const float2 gp = f2(g_lo, g_hi);
+          // a_t h_{t-1} = h_t - B_t dt_t u_t (the forward step without its input)
+          const float2 ahp = fsub2(hp[k], f2(bx[2 * k], bx[2 * k + 1]));
+          const float2 q = fmul2(gp, ahp);
+          dAp = ffma2(dlp[k], q, dAp);
+          dd2[k] = ffma2(f2(Anat, Anat), q, dd2[k]);
+          sgB2[k] = ffma2(gp, bp[k], sgB2[k]);
+          dBp[k] = fmul2(gp, xup[k]);
+          dCp[k] = fmul2(dyp[k], hp[k]);
         }
-        sdA[warp][n][lane] += dAl;
+        mysl[lane] = make_float4(dBp[0].x, dBp[0].y, dBp[1].x, dBp[1].y);
+        mysl[32 + lane] = make_float4(dBp[2].x, dBp[2].y, dBp[3].x, dBp[3].y);
+        mysl[64 + lane] = make_float4(dCp[0].x, dCp[0].y, dCp[1].x, dCp[1].y);
+        mysl[96 + lane] = make_float4(dCp[2].x, dCp[2].y, dCp[3].x, dCp[3].y);
+        sm.dA[warp][n][lane] += dAp.x + dAp.y;
       }
       __syncthreads();
-      // flush this state's channel sums: dB, dC [b][n][t0 + tau]
-      for (int k = threadIdx.x; k < 2 * kChunk; k += blockDim.x) {
-        const int m = k >= kChunk;
-        const int tau = k - m * kChunk;
-        const int pos = chunk_pos(tau >> 3, tau & 7);
-        const float v = red[m * kChunk + pos];
-        red[m * kChunk + pos] = 0.0f;
+      // sum the warps' slices of this state and add them to dB, dC [b][n][t0 + tau]
+      for (int it = threadIdx.x; it < 128; it += blockDim.x) {
+        const int m = it >> 6, q = it & 63;
+        float4 s = sm.slice[n & 1][0][m][q];
+#pragma unroll
+        for (int w = 1; w < G; ++w) {
+          const float4 v = sm.slice[n & 1][w][m][q];
+          s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+        }
+        const int tau = (q & 31) * 8 + (q >> 5) * 4;
         const int t = t0 + tau;
-        if (t < L) atomicAdd((m ? p.dC : p.dB) + ((size_t)b * N + n) * L + t, v);
+        float* dst = (m ? p.dC : p.dB) + ((size_t)b * N + n) * L + t;
+        if (VEC) {
+          if (t < L) atomicAdd(reinterpret_cast<float4*>(dst), s);
+        } else {
+          if (t < L) atomicAdd(dst, s.x);
+          if (t + 1 < L) atomicAdd(dst + 1, s.y);
+          if (t + 2 < L) atomicAdd(dst + 2, s.z);
+          if (t + 3 < L) atomicAdd(dst + 3, s.w);
+        }
       }
     }
 
     if (active) {
-      float sgv[8], zz[8], go[8];
-      load_row8<T, VEC>(dl_row, tl, L, sgv);
+      // this chunk's u, raw delta, dout, z again (L2-resident since the prefetch)
+      float uu[8], dl[8], go[8], zz[8];
+      load_row8<T, VEC>(u_row, tl, L, uu);
+      load_row8<T, VEC>(dl_row, tl, L, dl);
       load_row8<T, VEC>(go_row, tl, L, go);
       if (z_row) load_row8<T, VEC>(z_row, tl, L, zz);
       float o_du[8], o_dd[8], o_dz[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
+        const int k = i >> 1;
+        const float sg = (i & 1) ? sgB2[k].y : sgB2[k].x;
+        const float dsum = (i & 1) ? dd2[k].y : dd2[k].x;
+        const float yv = (i & 1) ? y2[k].y : y2[k].x;
+        const float dt = (i & 1) ? dlp[k].y : dlp[k].x;
+        const float dyi = (i & 1) ? dyp[k].y : dyp[k].x;
         const bool in = tl + i < L;
-        const float yfull = fmaf(Dv, uu[i], y[i]);
-        o_du[i] = fmaf(dy[i], Dv, dl[i] * sgB[i]);
-        const float ddt = fmaf(uu[i], sgB[i], dd[i]);
-        const float dv = p.softplus ? ddt * sigmoidf_(sgv[i] + bias) : ddt;
+        o_du[i] = fmaf(dyi, Dv, dt * sg);
+        const float ddt = fmaf(uu[i], sg, dsum);
+        // softplus'(v) = e^v / (1 + e^v)
+        const float v = dl[i] + bias;
+        const float ev = __expf(v);
+        const float dv = p.softplus ? ddt * (v > 20.0f ? 1.0f : __fdividef(ev, 1.0f + ev)) : ddt;
         o_dd[i] = dv;
         if (z_row) {
-          const float sz = sigmoidf_(zz[i]);
+          const float yfull = fmaf(Dv, uu[i], yv);
+          const float sz = sigmoid_fast(zz[i]);
           o_dz[i] = go[i] * yfull * (sz * (1.0f + zz[i] * (1.0f - sz)));
         }
         if (in) {
-          dDp = fmaf(dy[i], uu[i], dDp);
+          dDp = fmaf(dyi, uu[i], dDp);
           ddbp += dv;
         }
       }
@@ -219,7 +348,7 @@ scan_bwd_kernel(const ScanArgs p) {
   const size_t ps = rowid * p.nsplits + split;
   if (lane < N) {
     float s = 0.0f;
-    for (int j = 0; j < 32; ++j) s += sdA[warp][lane][j];
+    for (int j = 0; j < 32; ++j) s += sm.dA[warp][lane][j];
     p.part_dA[ps * N + lane] = s;
   }
   if (lane == 0) {
@@ -254,8 +383,7 @@ scan_bwd_summary_kernel(const ScanArgs p) {
   for (int c = c_end - 1; c >= c_begin; --c) {
     const int t0 = c * kChunk;
     __syncthreads();
-    stage_bc<T, VEC>(static_cast<const T*>(p.Bm), static_cast<const T*>(p.Cm), nullptr, sC, b,
-                     N, L, t0);
+    stage_rows<T, VEC>(static_cast<const T*>(p.Cm), sC, b, N, L, t0);
     __syncthreads();
     if (!active) continue;
     const int tl = t0 + lane * 8;
@@ -274,8 +402,14 @@ scan_bwd_summary_kernel(const ScanArgs p) {
     const bool any_reset = __any_sync(kFull, rmask != 0u);
     for (int n = 0; n < N; ++n) {
       const float An2 = __shfl_sync(kFull, A2_lane, n);
+      float2 cp[4];
+      lds_tokpairs(sC + n * kChunk, lane, cp);
       float cv[8], a[8];
-      lds8(sC + n * kChunk, lane, cv);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        cv[2 * k] = cp[k].x;
+        cv[2 * k + 1] = cp[k].y;
+      }
 #pragma unroll
       for (int i = 0; i < 8; ++i) a[i] = ex2_approx(dl[i] * An2);
       if (any_reset) {
@@ -302,20 +436,20 @@ scan_bwd_summary_kernel(const ScanArgs p) {
     }
   }
   if (!active || lane >= N) return;
-  p.split_P[(rowid * p.nsplits + split) * N + lane] = Ptot;
-  p.split_H[(rowid * p.nsplits + split) * N + lane] = gcarry;
+  p.split_P[(rowid * p.nsplits + split) * p.Npad + lane] = Ptot;
+  p.split_H[(rowid * p.nsplits + split) * p.Npad + lane] = gcarry;
 }
 
 // Adjoint carry into split s from the right: c[P-1] = 0,
 // c[s-1] = P[s] c[s] + G[s].
 __global__ void bwd_split_carry_kernel(const float* __restrict__ P, const float* __restrict__ Gs,
-                                       float* __restrict__ cin, int rows, int nsplits, int N) {
+                                       float* __restrict__ cin, int rows, int nsplits, int Np) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= rows * N) return;
-  const int r = i / N, n = i % N;
+  if (i >= rows * Np) return;
+  const int r = i / Np, n = i % Np;
   float c = 0.0f;
   for (int s = nsplits - 1; s >= 0; --s) {
-    const size_t k = ((size_t)r * nsplits + s) * N + n;
+    const size_t k = ((size_t)r * nsplits + s) * Np + n;
     cin[k] = c;
     if (s > 0) c = fmaf(P[k], c, Gs[k]);
   }
@@ -353,12 +487,20 @@ cudaError_t bwd_t(const ScanArgs& a, cudaStream_t s) {
   if (a.nsplits > 1) {
     dim3 g1((a.D + G - 1) / G, a.B, a.nsplits - 1);
     scan_bwd_summary_kernel<T, G, VEC><<<g1, block, 0, s>>>(a);
-    const int n = a.B * a.D * a.N;
+    const int n = a.B * a.D * a.Npad;
     bwd_split_carry_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.split_P, a.split_H, a.split_in,
-                                                          a.B * a.D, a.nsplits, a.N);
+                                                          a.B * a.D, a.nsplits, a.Npad);
+  }
+  const size_t smem = sizeof(BwdSmem<G>);
+  static bool smem_set = false;  // once per instantiation and process (a benign race)
+  if (!smem_set) {
+    cudaError_t e = cudaFuncSetAttribute(scan_bwd_kernel<T, G, VEC>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    smem_set = true;
   }
   dim3 g2((a.D + G - 1) / G, a.B, a.nsplits);
-  scan_bwd_kernel<T, G, VEC><<<g2, block, 0, s>>>(a);
+  scan_bwd_kernel<T, G, VEC><<<g2, block, smem, s>>>(a);
   const int m = a.D * a.N > a.D ? a.D * a.N : a.D;
   bwd_param_reduce_kernel<<<(m + 255) / 256, 256, 0, s>>>(a.part_dA, a.part_dD, a.part_ddb, a.dA,
                                                          a.dD, a.ddelta_bias, a.B, a.D, a.N,

@@ -43,11 +43,205 @@ __device__ __forceinline__ void stage_bc(const T* __restrict__ Bm, const T* __re
   }
 }
 
+// Paired layout: states (2m, 2m+1) of token tau share one float2; lane j's 8
+// tokens sit in four 16-byte pieces at float4 index k*32 + j (tokens 2k, 2k+1),
+// so a warp reads 512 contiguous bytes per piece.
+template <typename T, bool VEC>
+__device__ __forceinline__ void stage_pairs(const T* __restrict__ M, float2* s, int b, int N, int L,
+                                            int t0) {
+  const int NP = (N + 1) >> 1;
+  for (int idx = threadIdx.x; idx < NP * 32; idx += blockDim.x) {
+    const int m = idx >> 5, j = idx & 31;
+    const int n0 = 2 * m, n1 = 2 * m + 1;
+    float v0[8], v1[8];
+    load_row8<T, VEC>(M + ((size_t)b * N + n0) * L, t0 + 8 * j, L, v0);
+    if (n1 < N) {
+      load_row8<T, VEC>(M + ((size_t)b * N + n1) * L, t0 + 8 * j, L, v1);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v1[i] = 0.0f;
+    }
+    float4* dst = reinterpret_cast<float4*>(s + m * kChunk);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      dst[k * 32 + j] = make_float4(v0[2 * k], v1[2 * k], v0[2 * k + 1], v1[2 * k + 1]);
+  }
+}
+
+// Lane `lane`'s 8 tokens of one state pair from a paired tile.
+__device__ __forceinline__ void lds_pair8(const float2* tile, int lane, float2 v[8]) {
+  const float4* t4 = reinterpret_cast<const float4*>(tile);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float4 q = t4[k * 32 + lane];
+    v[2 * k] = make_float2(q.x, q.y);
+    v[2 * k + 1] = make_float2(q.z, q.w);
+  }
+}
+
+// 8 consecutive activations of one lane, held raw in registers between the
+// load (issued one chunk ahead) and their use.
+template <typename T, bool VEC>
+struct Tok8 {
+  float v[8];
+  __device__ __forceinline__ void load(const T* row, int t, int L) { load_row8<T, VEC>(row, t, L, v); }
+  __device__ __forceinline__ void get(float o[8]) const {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i] = v[i];
+  }
+};
+
+template <>
+struct Tok8<__nv_bfloat16, true> {
+  uint4 r;
+  __device__ __forceinline__ void load(const __nv_bfloat16* row, int t, int L) {
+    r = (t < L) ? __ldg(reinterpret_cast<const uint4*>(row + t)) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  __device__ __forceinline__ void get(float o[8]) const {
+    o[0] = bf16lo(r.x); o[1] = bf16hi(r.x); o[2] = bf16lo(r.y); o[3] = bf16hi(r.y);
+    o[4] = bf16lo(r.z); o[5] = bf16hi(r.z); o[6] = bf16lo(r.w); o[7] = bf16hi(r.w);
+  }
+};
+
+__device__ __forceinline__ float2 f2(float x, float y) { return make_float2(x, y); }
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 ex2x2(float2 e) { return make_float2(ex2_approx(e.x), ex2_approx(e.y)); }
+__device__ __forceinline__ float2 shfl_up2(float2 v, int off) {
+  return make_float2(__shfl_up_sync(kFull, v.x, off), __shfl_up_sync(kFull, v.y, off));
+}
+__device__ __forceinline__ float2 shfl_down2(float2 v, int off) {
+  return make_float2(__shfl_down_sync(kFull, v.x, off), __shfl_down_sync(kFull, v.y, off));
+}
+__device__ __forceinline__ float2 shfl2(float2 v, int src) {
+  return make_float2(__shfl_sync(kFull, v.x, src), __shfl_sync(kFull, v.y, src));
+}
+
+// Pair versions of the two warp scans (two independent states at once).
+__device__ __forceinline__ void warp_scan_fwd2(float2& P, float2& H, int lane) {
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float2 Pp = shfl_up2(P, off);
+    const float2 Hp = shfl_up2(H, off);
+    if (lane >= off) {
+      H = ffma2(P, Hp, H);
+      P = fmul2(P, Pp);
+    }
+  }
+}
+
+__device__ __forceinline__ void warp_scan_bwd2(float2& P, float2& G, int lane) {
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float2 Pn = shfl_down2(P, off);
+    const float2 Gn = shfl_down2(G, off);
+    if (lane + off < 32) {
+      G = ffma2(P, Gn, G);
+      P = fmul2(P, Pn);
+    }
+  }
+}
+
 __device__ __forceinline__ void lds8(const float* base, int lane, float v[8]) {
   const float4 a = reinterpret_cast<const float4*>(base)[lane];
   const float4 b = reinterpret_cast<const float4*>(base + 128)[lane];
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// ---------------------------------------------------------------------------
+// Asynchronous staging of the raw bf16 B / C chunk tiles (vector path): the
+// copies for chunk c+1 are issued with cp.async while chunk c is computed, so
+// their latency is hidden; each thread later converts exactly the pieces it
+// copied. raw layout: [mat][n][kChunk] bf16 (mat 0 = B, 1 = C).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src, bool valid) {
+  const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+  const int n = valid ? 16 : 0;  // 0 source bytes: the 16 bytes are zero-filled
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(gmem_src), "r"(n)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
+
+// Issue this thread's copies of chunk tokens [t0, t0+kChunk) of rows n of B
+// (and C): item (mat, n, j) = 16 bytes = tokens [8j, 8j+8) of row n.
+__device__ __forceinline__ void issue_bc_raw(const __nv_bfloat16* __restrict__ Bm,
+                                             const __nv_bfloat16* __restrict__ Cm,
+                                             __nv_bfloat16* raw, int mats, int b, int N, int L,
+                                             int t0) {
+  const int per = N * 32;
+  for (int idx = threadIdx.x; idx < mats * per; idx += blockDim.x) {
+    const int mat = idx >= per;
+    const int rem = idx - mat * per;
+    const int n = rem >> 5, j = rem & 31;
+    const __nv_bfloat16* rowp = (mat ? Cm : Bm) + ((size_t)b * N + n) * L;
+    const int t = t0 + 8 * j;
+    const bool ok = t < L;
+    cp_async16(raw + ((size_t)mat * kNMax + n) * kChunk + 8 * j, ok ? rowp + t : rowp, ok);
+  }
+  cp_async_commit();
+}
+
+// Convert this thread's pieces (same idx mapping as issue_bc_raw) into the
+// fp32 row tile layout: row n, float4 index j = tokens [8j, 8j+4), 32 + j =
+// [8j+4, 8j+8).
+__device__ __forceinline__ void convert_bc_rows(const __nv_bfloat16* raw, float* sB, float* sC,
+                                                int mats, int N) {
+  const int per = N * 32;
+  for (int idx = threadIdx.x; idx < mats * per; idx += blockDim.x) {
+    const int mat = idx >= per;
+    const int rem = idx - mat * per;
+    const int n = rem >> 5, j = rem & 31;
+    const uint4 r = *reinterpret_cast<const uint4*>(raw + ((size_t)mat * kNMax + n) * kChunk + 8 * j);
+    float4* dst = reinterpret_cast<float4*>((mat ? sC : sB) + n * kChunk);
+    dst[j] = make_float4(bf16lo(r.x), bf16hi(r.x), bf16lo(r.y), bf16hi(r.y));
+    dst[32 + j] = make_float4(bf16lo(r.z), bf16hi(r.z), bf16lo(r.w), bf16hi(r.w));
+  }
+}
+
+// Same, into the state-pair layout of stage_pairs; items are (mat, m, j) and
+// cover rows 2m and 2m+1, so a thread converts what it copied only when the
+// copy used the pair mapping below.
+__device__ __forceinline__ void issue_bc_raw_pairs(const __nv_bfloat16* __restrict__ Bm,
+                                                   const __nv_bfloat16* __restrict__ Cm,
+                                                   __nv_bfloat16* raw, int mats, int b, int N,
+                                                   int L, int t0) {
+  const int NP = (N + 1) >> 1;
+  const int per = NP * 32;
+  for (int idx = threadIdx.x; idx < mats * per; idx += blockDim.x) {
+    const int mat = idx >= per;
+    const int rem = idx - mat * per;
+    const int m = rem >> 5, j = rem & 31;
+    const int t = t0 + 8 * j;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int n = 2 * m + h;
+      const bool rowok = n < N;
+      const __nv_bfloat16* rowp = (mat ? Cm : Bm) + ((size_t)b * N + (rowok ? n : 0)) * L;
+      const bool ok = rowok && t < L;
+      cp_async16(raw + ((size_t)mat * kNMax + n) * kChunk + 8 * j, ok ? rowp + t : rowp, ok);
+    }
+  }
+  cp_async_commit();
+}
+
+__device__ __forceinline__ void convert_bc_pairs(const __nv_bfloat16* raw, float2* sB, float2* sC,
+                                                 int mats, int N) {
+  const int NP = (N + 1) >> 1;
+  const int per = NP * 32;
+  for (int idx = threadIdx.x; idx < mats * per; idx += blockDim.x) {
+    const int mat = idx >= per;
+    const int rem = idx - mat * per;
+    const int m = rem >> 5, j = rem & 31;
+    const uint4 r0 = *reinterpret_cast<const uint4*>(raw + ((size_t)mat * kNMax + 2 * m) * kChunk + 8 * j);
+    const uint4 r1 = *reinterpret_cast<const uint4*>(raw + ((size_t)mat * kNMax + 2 * m + 1) * kChunk + 8 * j);
+    float4* dst = reinterpret_cast<float4*>((mat ? sC : sB) + m * kChunk);
+    dst[j] = make_float4(bf16lo(r0.x), bf16lo(r1.x), bf16hi(r0.x), bf16hi(r1.x));
+    dst[32 + j] = make_float4(bf16lo(r0.y), bf16lo(r1.y), bf16hi(r0.y), bf16hi(r1.y));
+    dst[64 + j] = make_float4(bf16lo(r0.z), bf16lo(r1.z), bf16hi(r0.z), bf16hi(r1.z));
+    dst[96 + j] = make_float4(bf16lo(r0.w), bf16lo(r1.w), bf16hi(r0.w), bf16hi(r1.w));
+  }
 }
 
 // Bit i set <=> token tl+i (< L, > 0) starts a new document.

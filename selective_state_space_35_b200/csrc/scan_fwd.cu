@@ -7,9 +7,15 @@
 //   h_t = a_t h_{t-1} + dt_t B_nt u_t;  y_t = sum_n C_nt h_t + D_d u_t
 //   out_t = y_t silu(z_t)
 // with a_t := 0 at the first token of a document ("FLA Mamba and Mamba2",
-// packing paragraph). The state never leaves registers; the only state
-// written to HBM is one checkpoint per 256-token chunk (read by the
-// backward's recompute) and the optional final state.
+// packing paragraph). The state never leaves the SM; the only state written
+// to HBM is one checkpoint per 256-token chunk (read by the backward's
+// recompute) and the optional final state.
+//
+// States are processed two at a time with packed fp32x2 arithmetic: one
+// instruction advances states 2m and 2m+1 together, halving the issue slots
+// per (token, state) so that the ex2 unit, not instruction issue, bounds the
+// kernel. The per-lane inputs of the next chunk are loaded into registers one
+// chunk ahead.
 //
 // Long rows can be split over P CTAs ("n_splits"): pass 1 runs the splits
 // 0..P-2 from a zero state and keeps (prod a, h_end) per split, a tiny kernel
@@ -21,18 +27,33 @@ namespace ssm {
 
 namespace {
 
+constexpr int kNP = kNMax / 2;  // state pairs
+
+template <int G>
+struct FwdSmem {
+  float2 B[kNP * kChunk];                 // B tile, state-pair layout
+  float2 C[kNP * kChunk];                 // C tile, state-pair layout
+  __nv_bfloat16 raw[2][kNMax][kChunk];    // next chunk's raw B / C (async path)
+  float2 A[G][kNP];                       // A' = A log2(e), per state pair
+  float2 H[G][kNP];                       // running state entering the current chunk
+  float2 P[G][kNP];                       // SUMMARY: running product of a over the split
+};
+
 template <typename T, int G, bool VEC, bool SUMMARY>
-__global__ void __launch_bounds__(G * 32)
+__global__ void __launch_bounds__(G * 32, 4)
 scan_fwd_kernel(const ScanArgs p) {
-  __shared__ __align__(16) float sB[kNMax * kChunk];
-  __shared__ __align__(16) float sC[kNMax * kChunk];
+  // bf16 on the vector path: B / C tiles arrive by cp.async one chunk ahead
+  constexpr bool ASYNC = VEC && sizeof(T) == 2;
+  extern __shared__ float4 smem_dyn[];
+  FwdSmem<G>& sm = *reinterpret_cast<FwdSmem<G>*>(smem_dyn);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
   const int d = blockIdx.x * G + warp;
   const bool active = d < p.D;
   const int split = blockIdx.z;
-  const int N = p.N, L = p.L;
+  const int N = p.N, L = p.L, NP = p.Npad >> 1;
+  const int mats = SUMMARY ? 1 : 2;
   const int c_begin = split * p.chunks_per_split;
   const int c_end = min(c_begin + p.chunks_per_split, p.nchunks);
   const size_t rowid = (size_t)b * p.D + (active ? d : 0);
@@ -44,121 +65,149 @@ scan_fwd_kernel(const ScanArgs p) {
   const T* dl_row = static_cast<const T*>(p.delta) + row;
   const T* z_row = p.z ? static_cast<const T*>(p.z) + row : nullptr;
 
-  // lane n holds A'_n = A_dn log2(e), and the running state h_n
-  const float A2_lane = (active && lane < N) ? __ldg(p.A + (size_t)d * N + lane) * kLog2e : 0.0f;
+  if (ASYNC)
+    issue_bc_raw_pairs(reinterpret_cast<const __nv_bfloat16*>(Bm),
+                       reinterpret_cast<const __nv_bfloat16*>(Cm), &sm.raw[0][0][0], mats, b, N, L,
+                       c_begin * kChunk);
+  if (lane < kNP) {
+    float a0 = 0.0f, a1 = 0.0f;
+    if (active && 2 * lane < N) a0 = __ldg(p.A + (size_t)d * N + 2 * lane) * kLog2e;
+    if (active && 2 * lane + 1 < N) a1 = __ldg(p.A + (size_t)d * N + 2 * lane + 1) * kLog2e;
+    sm.A[warp][lane] = f2(a0, a1);
+    float2 h0 = f2(0.0f, 0.0f);
+    if (!SUMMARY && split > 0 && active && lane < NP)
+      h0 = reinterpret_cast<const float2*>(p.split_in)[(rowid * p.nsplits + split) * NP + lane];
+    sm.H[warp][lane] = h0;
+    sm.P[warp][lane] = f2(1.0f, 1.0f);
+  }
   const float Dv = (active && p.Dskip) ? __ldg(p.Dskip + d) : 0.0f;
   const float bias = (active && p.delta_bias) ? __ldg(p.delta_bias + d) : 0.0f;
-  float carry = 0.0f;
-  if (!SUMMARY && split > 0 && active && lane < N)
-    carry = p.split_in[(rowid * p.nsplits + split) * N + lane];
-  float Pacc = 1.0f;  // SUMMARY: lane n holds prod a over the split
+
+  Tok8<T, VEC> pf_dl, pf_u, pf_z;
+  if (active) {
+    const int tl = c_begin * kChunk + lane * 8;
+    pf_dl.load(dl_row, tl, L);
+    pf_u.load(u_row, tl, L);
+    if (!SUMMARY && z_row) pf_z.load(z_row, tl, L);
+  }
 
   for (int c = c_begin; c < c_end; ++c) {
     const int t0 = c * kChunk;
-    __syncthreads();
-    stage_bc<T, VEC>(Bm, Cm, sB, SUMMARY ? nullptr : sC, b, N, L, t0);
+    if (ASYNC) {
+      cp_async_wait_all();
+      __syncthreads();  // the previous chunk's readers of B / C are done
+      convert_bc_pairs(&sm.raw[0][0][0], sm.B, sm.C, mats, N);
+      if (c + 1 < c_end)  // each thread refills only the pieces it just converted
+        issue_bc_raw_pairs(reinterpret_cast<const __nv_bfloat16*>(Bm),
+                           reinterpret_cast<const __nv_bfloat16*>(Cm), &sm.raw[0][0][0], mats, b,
+                           N, L, t0 + kChunk);
+    } else {
+      __syncthreads();
+      stage_pairs<T, VEC>(Bm, sm.B, b, N, L, t0);
+      if (!SUMMARY) stage_pairs<T, VEC>(Cm, sm.C, b, N, L, t0);
+    }
     __syncthreads();
     if (!active) continue;
 
-    if (!SUMMARY && p.ckpt && lane < N) p.ckpt[(rowid * p.nchunks + c) * N + lane] = carry;
-
     const int tl = t0 + lane * 8;
-    float dl[8], uu[8], xu[8];
-    load_row8<T, VEC>(dl_row, tl, L, dl);
-    load_row8<T, VEC>(u_row, tl, L, uu);
+    float dl[8], uu[8], zz[8];
+    pf_dl.get(dl);
+    pf_u.get(uu);
+    if (!SUMMARY && z_row) pf_z.get(zz);
+    if (c + 1 < c_end) {  // next chunk's inputs, consumed one iteration later
+      pf_dl.load(dl_row, tl + kChunk, L);
+      pf_u.load(u_row, tl + kChunk, L);
+      if (!SUMMARY && z_row) pf_z.load(z_row, tl + kChunk, L);
+    }
+    float2 dd[8], xx[8], y2[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float v = dl[i] + bias;
-      const float s = p.softplus ? softplusf_(v) : v;
-      dl[i] = (tl + i < L) ? s : 0.0f;  // dt = 0 past the end: a = 1, no input
-      xu[i] = dl[i] * uu[i];
+      const float s = p.softplus ? (v > 20.0f ? v : log1pf(__expf(v))) : v;
+      const float dt = (tl + i < L) ? s : 0.0f;  // dt = 0 past the end: a = 1, no input
+      dd[i] = f2(dt, dt);
+      xx[i] = f2(dt * uu[i], dt * uu[i]);
+      y2[i] = f2(Dv * uu[i], 0.0f);  // y starts from the D u feed-through
     }
     const unsigned rmask = reset_mask(p.seq, b, L, tl);
     const bool any_reset = __any_sync(kFull, rmask != 0u);
 
-    float y[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) y[i] = 0.0f;
+    if (!SUMMARY && lane < NP)
+      reinterpret_cast<float2*>(p.ckpt)[(rowid * p.nchunks + c) * NP + lane] = sm.H[warp][lane];
 
-    for (int n = 0; n < N; ++n) {
-      const float An = __shfl_sync(kFull, A2_lane, n);
-      float bv[8];
-      lds8(sB + n * kChunk, lane, bv);
-      float a[8], bx[8];
-      float P = 1.0f, H = 0.0f;
+    for (int m = 0; m < NP; ++m) {
+      const float2 A2 = sm.A[warp][m];
+      float2 bv[8], a[8], bx[8];
+      lds_pair8(sm.B + m * kChunk, lane, bv);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        a[i] = ex2_approx(dl[i] * An);
-        bx[i] = xu[i] * bv[i];
+        a[i] = ex2x2(fmul2(dd[i], A2));
+        bx[i] = fmul2(xx[i], bv[i]);
       }
       if (any_reset) {
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          if ((rmask >> i) & 1u) a[i] = 0.0f;
+          if ((rmask >> i) & 1u) a[i] = f2(0.0f, 0.0f);
       }
+      float2 P = a[0], H = bx[0];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        H = fmaf(a[i], H, bx[i]);
-        P *= a[i];
+      for (int i = 1; i < 8; ++i) {
+        H = ffma2(a[i], H, bx[i]);
+        P = fmul2(P, a[i]);
       }
-      warp_scan_fwd(P, H, lane);
-      const float cin = __shfl_sync(kFull, carry, n);
-      const float end = fmaf(P, cin, H);
-      float start = __shfl_up_sync(kFull, end, 1);
+      warp_scan_fwd2(P, H, lane);
+      const float2 cin = sm.H[warp][m];
+      const float2 end = ffma2(P, cin, H);
+      float2 start = shfl_up2(end, 1);
       if (lane == 0) start = cin;
-      const float nc = __shfl_sync(kFull, end, 31);
-      if (lane == n) carry = nc;
-      if (SUMMARY) {
-        const float Pt = __shfl_sync(kFull, P, 31);
-        if (lane == n) Pacc *= Pt;
-        continue;
+      if (lane == 31) {
+        sm.H[warp][m] = end;
+        if (SUMMARY) sm.P[warp][m] = fmul2(sm.P[warp][m], P);
       }
-      float cv[8];
-      lds8(sC + n * kChunk, lane, cv);
-      float h = start;
+      if (!SUMMARY) {
+        float2 cv[8];
+        lds_pair8(sm.C + m * kChunk, lane, cv);
+        float2 h = start;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        h = fmaf(a[i], h, bx[i]);
-        y[i] = fmaf(cv[i], h, y[i]);
+        for (int i = 0; i < 8; ++i) {
+          h = ffma2(a[i], h, bx[i]);
+          y2[i] = ffma2(cv[i], h, y2[i]);
+        }
       }
     }
 
     if (!SUMMARY) {
       float o[8];
-      if (z_row) {
-        float zz[8];
-        load_row8<T, VEC>(z_row, tl, L, zz);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float yy = fmaf(Dv, uu[i], y[i]);
-          o[i] = yy * (zz[i] * sigmoidf_(zz[i]));
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = fmaf(Dv, uu[i], y[i]);
+      for (int i = 0; i < 8; ++i) {
+        const float yy = y2[i].x + y2[i].y;
+        o[i] = z_row ? yy * (zz[i] * sigmoid_fast(zz[i])) : yy;
       }
       store_row8<T, VEC>(static_cast<T*>(p.out) + row, tl, L, o);
     }
   }
 
-  if (!active || lane >= N) return;
+  __syncwarp();
+  if (!active || lane >= NP) return;
+  const float2 h = sm.H[warp][lane];
   if (SUMMARY) {
-    p.split_P[(rowid * p.nsplits + split) * N + lane] = Pacc;
-    p.split_H[(rowid * p.nsplits + split) * N + lane] = carry;
+    reinterpret_cast<float2*>(p.split_P)[(rowid * p.nsplits + split) * NP + lane] = sm.P[warp][lane];
+    reinterpret_cast<float2*>(p.split_H)[(rowid * p.nsplits + split) * NP + lane] = h;
   } else if (p.final_state && split == p.nsplits - 1) {
-    p.final_state[rowid * N + lane] = carry;
+    p.final_state[rowid * N + 2 * lane] = h.x;
+    if (2 * lane + 1 < N) p.final_state[rowid * N + 2 * lane + 1] = h.y;
   }
 }
 
 // Carry into split s: h_in[0] = 0, h_in[s+1] = P[s] h_in[s] + H[s].
 __global__ void fwd_split_carry_kernel(const float* __restrict__ P, const float* __restrict__ H,
-                                       float* __restrict__ hin, int rows, int nsplits, int N) {
+                                       float* __restrict__ hin, int rows, int nsplits, int Np) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= rows * N) return;
-  const int r = i / N, n = i % N;
+  if (i >= rows * Np) return;
+  const int r = i / Np, n = i % Np;
   float h = 0.0f;
   for (int s = 0; s < nsplits; ++s) {
-    const size_t k = ((size_t)r * nsplits + s) * N + n;
+    const size_t k = ((size_t)r * nsplits + s) * Np + n;
     hin[k] = h;
     if (s + 1 < nsplits) h = fmaf(P[k], h, H[k]);
   }
@@ -177,18 +226,33 @@ __global__ void cu_seqlens_to_seq_kernel(const int32_t* __restrict__ cu, int n_d
   seq[t] = lo;
 }
 
+template <typename T, int G, bool VEC, bool SUMMARY>
+cudaError_t fwd_smem_attr() {
+  static bool done = false;  // once per instantiation and process (a benign race)
+  if (done) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(scan_fwd_kernel<T, G, VEC, SUMMARY>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sizeof(FwdSmem<G>));
+  if (e == cudaSuccess) done = true;
+  return e;
+}
+
 template <typename T, int G, bool VEC>
 cudaError_t fwd_t(const ScanArgs& a, cudaStream_t s) {
   dim3 block(G * 32);
+  const size_t smem = sizeof(FwdSmem<G>);
+  cudaError_t e = fwd_smem_attr<T, G, VEC, false>();
+  if (e == cudaSuccess && a.nsplits > 1) e = fwd_smem_attr<T, G, VEC, true>();
+  if (e != cudaSuccess) return e;
   if (a.nsplits > 1) {
     dim3 g1((a.D + G - 1) / G, a.B, a.nsplits - 1);
-    scan_fwd_kernel<T, G, VEC, true><<<g1, block, 0, s>>>(a);
-    const int n = a.B * a.D * a.N;
+    scan_fwd_kernel<T, G, VEC, true><<<g1, block, smem, s>>>(a);
+    const int n = a.B * a.D * a.Npad;
     fwd_split_carry_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.split_P, a.split_H, a.split_in,
-                                                          a.B * a.D, a.nsplits, a.N);
+                                                          a.B * a.D, a.nsplits, a.Npad);
   }
   dim3 g2((a.D + G - 1) / G, a.B, a.nsplits);
-  scan_fwd_kernel<T, G, VEC, false><<<g2, block, 0, s>>>(a);
+  scan_fwd_kernel<T, G, VEC, false><<<g2, block, smem, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -358,3 +358,22 @@ def test_full_size_sampled(cfg):
                         inp.dout.f64[sl], **kw)
     assert rel_l2(h("dB", np.s_[b:b + 1, :, s0:]), g["dB"]) <= TOL_GRAD
     assert rel_l2(h("du", sl), oracle.round_bf16(g["du"])) <= TOL_GRAD
+
+
+def test_unaligned_gradient_buffers_take_scalar_path():
+    torch = _torch()
+    import selective_state_space_35_b200 as ssm
+    B, D, N, L = 1, 5, 16, 512
+    inp = _small(B, D, N, L, 808, dtype="bf16", nbound=2)
+    dv = device_inputs(inp)
+    u = ssm.conv1d_fwd(dv["x"], dv["conv_w"], dv["conv_b"], dv["seq_idx"])
+    kw = dict(z=dv["z"], Dskip=dv["Dskip"], delta_bias=dv["delta_bias"], seq_idx=dv["seq_idx"])
+    _, _, ws = ssm.scan_fwd(u, dv["delta"], dv["A"], dv["Bm"], dv["Cm"], **kw)
+    ref = ssm.scan_bwd(u, dv["delta"], dv["A"], dv["Bm"], dv["Cm"], dv["dout"], ws, **kw)
+    n = B * N * L
+    bufB = torch.empty(n + 1, dtype=torch.float32, device="cuda")
+    bufC = torch.empty(n + 1, dtype=torch.float32, device="cuda")
+    g = ssm.scan_bwd(u, dv["delta"], dv["A"], dv["Bm"], dv["Cm"], dv["dout"], ws,
+                     grads={"dB": bufB[1:].view(B, N, L), "dC": bufC[1:].view(B, N, L)}, **kw)
+    for k in ("dB", "dC", "du", "ddelta", "dz"):
+        assert rel_l2(host64(g[k]), host64(ref[k])) <= 1e-6, k

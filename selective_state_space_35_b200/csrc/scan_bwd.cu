@@ -33,7 +33,6 @@ namespace ssm {
 
 namespace {
 
-__device__ __forceinline__ float2 fsub2(float2 a, float2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
 
 // float4-piece layout of a [kNMax][kChunk] fp32 tile: lane j's tokens
 // [8j, 8j+4) at float4 index j, [8j+4, 8j+8) at 32 + j (per state row of 64).
@@ -68,7 +67,130 @@ struct BwdSmem {
   float dA[G][kNMax][32];
 };
 
-template <typename T, int G, bool VEC>
+// One state n of one chunk for one lane: rebuild the lane's 8 states from the
+// chunk checkpoint (warp scan), run the adjoint backwards (reverse warp scan,
+// carry-in from the next chunk in lane n's gcarry), accumulate the per-token
+// sums over states, and write this row's dB / dC contributions into the
+// warp's slice.
+__device__ __forceinline__ void bwd_state(int n, int lane, const float* __restrict__ sB,
+                                          const float* __restrict__ sC, float4* mysl,
+                                          float* sdA_n, float A_lane, float A2_lane, float hck,
+                                          float& gcarry, const float2 dlp[4], const float2 xup[4],
+                                          const float2 dyp[4], float Sdl, unsigned rmask,
+                                          bool any_reset, float2 y2[4], float2 sgB2[4],
+                                          float2 dd2[4]) {
+  const float An2 = __shfl_sync(kFull, A2_lane, n);
+  const float Anat = __shfl_sync(kFull, A_lane, n);
+  float2 bp[4], cp[4];
+  lds_tokpairs(sB + n * kChunk, lane, bp);
+  lds_tokpairs(sC + n * kChunk, lane, cp);
+  float a[8], bx[8];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 e = fmul2(dlp[k], f2(An2, An2));
+    a[2 * k] = ex2_approx(e.x);
+    a[2 * k + 1] = ex2_approx(e.y);
+    const float2 q = fmul2(xup[k], bp[k]);
+    bx[2 * k] = q.x;
+    bx[2 * k + 1] = q.y;
+  }
+  float Ploc = ex2_approx(An2 * Sdl);
+  if (any_reset) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if ((rmask >> i) & 1u) a[i] = 0.0f;
+    if (rmask) Ploc = 0.0f;
+  }
+  // forward recompute of this lane's 8 states
+  float H = bx[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) H = fmaf(a[i], H, bx[i]);
+  float P = Ploc;
+  warp_scan_fwd(P, H, lane);
+  const float hin = __shfl_sync(kFull, hck, n);
+  const float end = fmaf(P, hin, H);
+  float start = __shfl_up_sync(kFull, end, 1);
+  if (lane == 0) start = hin;
+  float2 hp[4], gy[4];
+  {
+    float h = start;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      hp[k].x = h = fmaf(a[2 * k], h, bx[2 * k]);
+      hp[k].y = h = fmaf(a[2 * k + 1], h, bx[2 * k + 1]);
+      y2[k] = ffma2(cp[k], hp[k], y2[k]);
+      gy[k] = fmul2(dyp[k], cp[k]);
+    }
+  }
+  // adjoint: lane map c_in -> c_out = a_first * g_first
+  float Gl = gy[3].y;
+#pragma unroll
+  for (int i = 6; i >= 0; --i) Gl = fmaf(a[i + 1], Gl, (i & 1) ? gy[i >> 1].y : gy[i >> 1].x);
+  float Gc = a[0] * Gl;
+  float Pr = Ploc;
+  warp_scan_bwd(Pr, Gc, lane);
+  const float cc = __shfl_sync(kFull, gcarry, n);
+  const float cout = fmaf(Pr, cc, Gc);
+  float cin = __shfl_down_sync(kFull, cout, 1);
+  if (lane == 31) cin = cc;
+  const float ncar = __shfl_sync(kFull, cout, 0);
+  if (lane == n) gcarry = ncar;
+
+  // reverse replay, two tokens at a time: g for tokens 2k+1 and 2k, then
+  // every per-token product for that pair
+  const float2 minus1 = f2(-1.0f, -1.0f);
+  float2 dAp = f2(0.f, 0.f), dBp[4], dCp[4];
+  float g = gy[3].y + cin;
+#pragma unroll
+  for (int k = 3; k >= 0; --k) {
+    float2 gp;
+    gp.y = g;                                   // token 2k+1
+    gp.x = fmaf(a[2 * k + 1], g, gy[k].x);      // token 2k
+    if (k > 0) g = fmaf(a[2 * k], gp.x, gy[k - 1].y);  // token 2k-1
+    // a_t h_{t-1} = h_t - B_t dt_t u_t (the forward step without its input)
+    const float2 ahp = ffma2(f2(bx[2 * k], bx[2 * k + 1]), minus1, hp[k]);
+    const float2 q = fmul2(gp, ahp);
+    dAp = ffma2(dlp[k], q, dAp);
+    dd2[k] = ffma2(f2(Anat, Anat), q, dd2[k]);
+    sgB2[k] = ffma2(gp, bp[k], sgB2[k]);
+    dBp[k] = fmul2(gp, xup[k]);
+    dCp[k] = fmul2(dyp[k], hp[k]);
+  }
+  mysl[lane] = make_float4(dBp[0].x, dBp[0].y, dBp[1].x, dBp[1].y);
+  mysl[32 + lane] = make_float4(dBp[2].x, dBp[2].y, dBp[3].x, dBp[3].y);
+  mysl[64 + lane] = make_float4(dCp[0].x, dCp[0].y, dCp[1].x, dCp[1].y);
+  mysl[96 + lane] = make_float4(dCp[2].x, dCp[2].y, dCp[3].x, dCp[3].y);
+  sdA_n[lane] += dAp.x + dAp.y;
+}
+
+// Sum the G warps' slices of state n (parity n & 1) and add them to dB / dC
+// (one float4 = 4 tokens per thread; `dst` points at this thread's 4 tokens
+// of state 0 in dB or dC, `L` apart per state).
+template <int G, bool VEC>
+__device__ __forceinline__ void bwd_reduce(int n, const float4 (*slice)[G][2][64], int m, int q,
+                                           float* dst, int L, bool valid4, int tleft) {
+  const float4* sl = &slice[n & 1][0][m][q];
+  float4 s = sl[0];
+#pragma unroll
+  for (int w = 1; w < G; ++w) {
+    const float4 v = sl[w * 128];
+    const float2 lo = __fadd2_rn(f2(s.x, s.y), f2(v.x, v.y));
+    const float2 hi = __fadd2_rn(f2(s.z, s.w), f2(v.z, v.w));
+    s = make_float4(lo.x, lo.y, hi.x, hi.y);
+  }
+  float* d = dst + (size_t)n * L;
+  if (VEC) {
+    if (valid4) atomicAdd(reinterpret_cast<float4*>(d), s);
+  } else {
+    if (tleft > 0) atomicAdd(d, s.x);
+    if (tleft > 1) atomicAdd(d + 1, s.y);
+    if (tleft > 2) atomicAdd(d + 2, s.z);
+    if (tleft > 3) atomicAdd(d + 3, s.w);
+  }
+}
+
+// NT: state count fixed at compile time (16), or 0 for any N <= 16.
+template <typename T, int G, bool VEC, int NT>
 __global__ void __launch_bounds__(G * 32, SSM_BWD_MIN_BLOCKS)
 scan_bwd_kernel(const ScanArgs p) {
   constexpr bool ASYNC = VEC && sizeof(T) == 2;  // B / C tiles by cp.async one chunk ahead
@@ -80,7 +202,7 @@ scan_bwd_kernel(const ScanArgs p) {
   const int d = blockIdx.x * G + warp;
   const bool active = d < p.D;
   const int split = blockIdx.z;
-  const int N = p.N, L = p.L;
+  const int N = NT ? NT : p.N, L = p.L;
   const int c_begin = split * p.chunks_per_split;
   const int c_end = min(c_begin + p.chunks_per_split, p.nchunks);
   const size_t rowid = (size_t)b * p.D + (active ? d : 0);
@@ -184,117 +306,29 @@ scan_bwd_kernel(const ScanArgs p) {
       dd2[k] = f2(0.f, 0.f);
     }
 
-    for (int n = 0; n < N; ++n) {
-      float4* mysl = &sm.slice[n & 1][warp][0][0];
-      if (active) {
-        const float An2 = __shfl_sync(kFull, A2_lane, n);
-        const float Anat = __shfl_sync(kFull, A_lane, n);
-        float2 bp[4], cp[4];
-        lds_tokpairs(sm.B + n * kChunk, lane, bp);
-        lds_tokpairs(sm.C + n * kChunk, lane, cp);
-        float a[8], bx[8];
+    // this thread's share of the per-state dB / dC reduction: item (m, q)
+    const int rm = threadIdx.x >> 6, rq = threadIdx.x & 63;  // blockDim = 128 = 2 x 64 items
+    const int rt = t0 + (rq & 31) * 8 + (rq >> 5) * 4;
+    float* rdst = (rm ? p.dC : p.dB) + (size_t)b * N * L + rt;
+    const bool rvalid = rt < L;
+    const int rleft = L - rt;
+    if (NT) {  // compile-time state count: fully unrolled, immediate offsets
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float2 e = fmul2(dlp[k], f2(An2, An2));
-          a[2 * k] = ex2_approx(e.x);
-          a[2 * k + 1] = ex2_approx(e.y);
-          const float2 q = fmul2(xup[k], bp[k]);
-          bx[2 * k] = q.x;
-          bx[2 * k + 1] = q.y;
-        }
-        float Ploc = ex2_approx(An2 * Sdl);
-        if (any_reset) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            if ((rmask >> i) & 1u) a[i] = 0.0f;
-          if (rmask) Ploc = 0.0f;
-        }
-        // forward recompute of this lane's 8 states
-        float H = bx[0];
-#pragma unroll
-        for (int i = 1; i < 8; ++i) H = fmaf(a[i], H, bx[i]);
-        float P = Ploc;
-        warp_scan_fwd(P, H, lane);
-        const float hin = __shfl_sync(kFull, hck, n);
-        const float end = fmaf(P, hin, H);
-        float start = __shfl_up_sync(kFull, end, 1);
-        if (lane == 0) start = hin;
-        float hs[8];
-        {
-          float h = start;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            h = fmaf(a[i], h, bx[i]);
-            hs[i] = h;
-          }
-        }
-        float2 hp[4], gy[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          hp[k] = f2(hs[2 * k], hs[2 * k + 1]);
-          y2[k] = ffma2(cp[k], hp[k], y2[k]);
-          gy[k] = fmul2(dyp[k], cp[k]);
-        }
-        // adjoint: lane map c_in -> c_out = a_first * g_first
-        float Gl = gy[3].y;
-#pragma unroll
-        for (int i = 6; i >= 0; --i) Gl = fmaf(a[i + 1], Gl, (i & 1) ? gy[i >> 1].y : gy[i >> 1].x);
-        float Gc = a[0] * Gl;
-        float Pr = Ploc;
-        warp_scan_bwd(Pr, Gc, lane);
-        const float cc = __shfl_sync(kFull, gcarry, n);
-        const float cout = fmaf(Pr, cc, Gc);
-        float cin = __shfl_down_sync(kFull, cout, 1);
-        if (lane == 31) cin = cc;
-        const float ncar = __shfl_sync(kFull, cout, 0);
-        if (lane == n) gcarry = ncar;
-
-        // reverse replay, two tokens at a time: g for tokens 2k+1 and 2k,
-        // then every per-token product for that pair
-        float2 dAp = f2(0.f, 0.f), dBp[4], dCp[4];
-        float g = gy[3].y + cin;
-#pragma unroll
-        for (int k = 3; k >= 0; --k) {
-          const float g_hi = g;  // token 2k+1
-          const float g_lo = fmaf(a[2 * k + 1], g_hi, gy[k].x);  // token 2k
-          if (k > 0) g = fmaf(a[2 * k], g_lo, gy[k - 1].y);   // token 2k-1
-          const float2 gp = f2(g_lo, g_hi);
-          // a_t h_{t-1} = h_t - B_t dt_t u_t (the forward step without its input)
-          const float2 ahp = fsub2(hp[k], f2(bx[2 * k], bx[2 * k + 1]));
-          const float2 q = fmul2(gp, ahp);
-          dAp = ffma2(dlp[k], q, dAp);
-          dd2[k] = ffma2(f2(Anat, Anat), q, dd2[k]);
-          sgB2[k] = ffma2(gp, bp[k], sgB2[k]);
-          dBp[k] = fmul2(gp, xup[k]);
-          dCp[k] = fmul2(dyp[k], hp[k]);
-        }
-        mysl[lane] = make_float4(dBp[0].x, dBp[0].y, dBp[1].x, dBp[1].y);
-        mysl[32 + lane] = make_float4(dBp[2].x, dBp[2].y, dBp[3].x, dBp[3].y);
-        mysl[64 + lane] = make_float4(dCp[0].x, dCp[0].y, dCp[1].x, dCp[1].y);
-        mysl[96 + lane] = make_float4(dCp[2].x, dCp[2].y, dCp[3].x, dCp[3].y);
-        sm.dA[warp][n][lane] += dAp.x + dAp.y;
+      for (int n = 0; n < NT; ++n) {
+        if (active)
+          bwd_state(n, lane, sm.B, sm.C, &sm.slice[n & 1][warp][0][0], &sm.dA[warp][n][0], A_lane,
+                    A2_lane, hck, gcarry, dlp, xup, dyp, Sdl, rmask, any_reset, y2, sgB2, dd2);
+        __syncthreads();
+        bwd_reduce<G, VEC>(n, sm.slice, rm, rq, rdst, L, rvalid, rleft);
       }
-      __syncthreads();
-      // sum the warps' slices of this state and add them to dB, dC [b][n][t0 + tau]
-      for (int it = threadIdx.x; it < 128; it += blockDim.x) {
-        const int m = it >> 6, q = it & 63;
-        float4 s = sm.slice[n & 1][0][m][q];
-#pragma unroll
-        for (int w = 1; w < G; ++w) {
-          const float4 v = sm.slice[n & 1][w][m][q];
-          s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
-        }
-        const int tau = (q & 31) * 8 + (q >> 5) * 4;
-        const int t = t0 + tau;
-        float* dst = (m ? p.dC : p.dB) + ((size_t)b * N + n) * L + t;
-        if (VEC) {
-          if (t < L) atomicAdd(reinterpret_cast<float4*>(dst), s);
-        } else {
-          if (t < L) atomicAdd(dst, s.x);
-          if (t + 1 < L) atomicAdd(dst + 1, s.y);
-          if (t + 2 < L) atomicAdd(dst + 2, s.z);
-          if (t + 3 < L) atomicAdd(dst + 3, s.w);
-        }
+    } else {
+#pragma unroll 1
+      for (int n = 0; n < N; ++n) {
+        if (active)
+          bwd_state(n, lane, sm.B, sm.C, &sm.slice[n & 1][warp][0][0], &sm.dA[warp][n][0], A_lane,
+                    A2_lane, hck, gcarry, dlp, xup, dyp, Sdl, rmask, any_reset, y2, sgB2, dd2);
+        __syncthreads();
+        bwd_reduce<G, VEC>(n, sm.slice, rm, rq, rdst, L, rvalid, rleft);
       }
     }
 
@@ -481,7 +515,7 @@ __global__ void bwd_param_reduce_kernel(const float* __restrict__ pA, const floa
   }
 }
 
-template <typename T, int G, bool VEC>
+template <typename T, int G, bool VEC, int NT>
 cudaError_t bwd_t(const ScanArgs& a, cudaStream_t s) {
   dim3 block(G * 32);
   if (a.nsplits > 1) {
@@ -494,13 +528,13 @@ cudaError_t bwd_t(const ScanArgs& a, cudaStream_t s) {
   const size_t smem = sizeof(BwdSmem<G>);
   static bool smem_set = false;  // once per instantiation and process (a benign race)
   if (!smem_set) {
-    cudaError_t e = cudaFuncSetAttribute(scan_bwd_kernel<T, G, VEC>,
+    cudaError_t e = cudaFuncSetAttribute(scan_bwd_kernel<T, G, VEC, NT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     smem_set = true;
   }
   dim3 g2((a.D + G - 1) / G, a.B, a.nsplits);
-  scan_bwd_kernel<T, G, VEC><<<g2, block, smem, s>>>(a);
+  scan_bwd_kernel<T, G, VEC, NT><<<g2, block, smem, s>>>(a);
   const int m = a.D * a.N > a.D ? a.D * a.N : a.D;
   bwd_param_reduce_kernel<<<(m + 255) / 256, 256, 0, s>>>(a.part_dA, a.part_dD, a.part_ddb, a.dA,
                                                          a.dD, a.ddelta_bias, a.B, a.D, a.N,
@@ -510,9 +544,17 @@ cudaError_t bwd_t(const ScanArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+template <int NT>
+cudaError_t bwd_dispatch(const ScanArgs& a, cudaStream_t s) {
+  if (a.bf16)
+    return a.vec ? bwd_t<__nv_bfloat16, 4, true, NT>(a, s) : bwd_t<__nv_bfloat16, 4, false, NT>(a, s);
+  return a.vec ? bwd_t<float, 4, true, NT>(a, s) : bwd_t<float, 4, false, NT>(a, s);
+}
+
 cudaError_t launch_scan_bwd(const ScanArgs& a, cudaStream_t s) {
-  if (a.bf16) return a.vec ? bwd_t<__nv_bfloat16, 4, true>(a, s) : bwd_t<__nv_bfloat16, 4, false>(a, s);
-  return a.vec ? bwd_t<float, 4, true>(a, s) : bwd_t<float, 4, false>(a, s);
+  // the runtime state loop: fully unrolling 16 states overflows the
+  // instruction cache and spills more (measured slower)
+  return bwd_dispatch<0>(a, s);
 }
 
 }  // namespace ssm

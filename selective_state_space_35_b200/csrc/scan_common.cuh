@@ -263,16 +263,17 @@ __device__ __forceinline__ unsigned reset_mask(const int32_t* __restrict__ seq, 
 }
 
 // Inclusive warp scan of affine maps h -> P h + H, earlier lanes applied
-// first: lane j ends with the composition of lanes 0..j.
+// first: lane j ends with the composition of lanes 0..j. The combine is a
+// predicated FMA / MUL pair (lanes below the offset keep their value).
 __device__ __forceinline__ void warp_scan_fwd(float& P, float& H, int lane) {
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const float Pp = __shfl_up_sync(kFull, P, off);
     const float Hp = __shfl_up_sync(kFull, H, off);
-    if (lane >= off) {
-      H = fmaf(P, Hp, H);
-      P *= Pp;
-    }
+    asm("{\n\t.reg .pred q;\n\tsetp.ge.s32 q, %2, %3;\n\t"
+        "@q fma.rn.f32 %1, %0, %5, %1;\n\t@q mul.rn.f32 %0, %0, %4;\n\t}"
+        : "+f"(P), "+f"(H)
+        : "r"(lane), "r"(off), "f"(Pp), "f"(Hp));
   }
 }
 
@@ -283,10 +284,10 @@ __device__ __forceinline__ void warp_scan_bwd(float& P, float& G, int lane) {
   for (int off = 1; off < 32; off <<= 1) {
     const float Pn = __shfl_down_sync(kFull, P, off);
     const float Gn = __shfl_down_sync(kFull, G, off);
-    if (lane + off < 32) {
-      G = fmaf(P, Gn, G);
-      P *= Pn;
-    }
+    asm("{\n\t.reg .pred q;\n\tsetp.lt.s32 q, %2, %3;\n\t"
+        "@q fma.rn.f32 %1, %0, %5, %1;\n\t@q mul.rn.f32 %0, %0, %4;\n\t}"
+        : "+f"(P), "+f"(G)
+        : "r"(lane), "r"(32 - off), "f"(Pn), "f"(Gn));
   }
 }
 

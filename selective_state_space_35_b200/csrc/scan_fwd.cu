@@ -39,8 +39,68 @@ struct FwdSmem {
   float2 P[G][kNP];                       // SUMMARY: running product of a over the split
 };
 
-template <typename T, int G, bool VEC, bool SUMMARY>
-__global__ void __launch_bounds__(G * 32, 4)
+// One state pair (2m, 2m+1) of one chunk for one lane, in two halves so that
+// the discretisation of pair m+1 (ex2-heavy) can overlap the shuffle-latency-
+// bound warp scan of pair m.
+// fwd_pair_pre: a = 2^(dt A'), bx = dt u B for the lane's 8 tokens.
+__device__ __forceinline__ void fwd_pair_pre(int m, int lane, const float2* __restrict__ sBt,
+                                             const float2 A2, const float2 dd[8],
+                                             const float2 xx[8], unsigned rmask, bool any_reset,
+                                             float2 a[8], float2 bx[8]) {
+  float2 bv[8];
+  lds_pair8(sBt + m * kChunk, lane, bv);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    a[i] = ex2x2(fmul2(dd[i], A2));
+    bx[i] = fmul2(xx[i], bv[i]);
+  }
+  if (any_reset) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if ((rmask >> i) & 1u) a[i] = f2(0.0f, 0.0f);
+  }
+}
+
+// fwd_pair_post: compose the lane's 8 steps, join the lanes with the warp scan
+// (carry-in from the previous chunk in H[m]), and replay to accumulate y.
+template <bool SUMMARY>
+__device__ __forceinline__ void fwd_pair_post(int m, int lane, const float2* __restrict__ sCt,
+                                              float2* sH, float2* sP, const float2 a[8],
+                                              const float2 bx[8], float2 y2[8]) {
+  float2 P = a[0], H = bx[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    H = ffma2(a[i], H, bx[i]);
+    P = fmul2(P, a[i]);
+  }
+  warp_scan_fwd2(P, H, lane);
+  const float2 cin = sH[m];
+  const float2 end = ffma2(P, cin, H);
+  float2 start = shfl_up2(end, 1);
+  if (lane == 0) start = cin;
+  if (lane == 31) {
+    sH[m] = end;
+    if (SUMMARY) sP[m] = fmul2(sP[m], P);
+  }
+  if (!SUMMARY) {
+    float2 cv[8];
+    lds_pair8(sCt + m * kChunk, lane, cv);
+    float2 h = start;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      h = ffma2(a[i], h, bx[i]);
+      y2[i] = ffma2(cv[i], h, y2[i]);
+    }
+  }
+}
+
+// NT: state count fixed at compile time (16), or 0 for any N <= 16.
+#ifndef SSM_FWD_MIN_BLOCKS
+#define SSM_FWD_MIN_BLOCKS 3
+#endif
+
+template <typename T, int G, bool VEC, bool SUMMARY, int NT>
+__global__ void __launch_bounds__(G * 32, SSM_FWD_MIN_BLOCKS)
 scan_fwd_kernel(const ScanArgs p) {
   // bf16 on the vector path: B / C tiles arrive by cp.async one chunk ahead
   constexpr bool ASYNC = VEC && sizeof(T) == 2;
@@ -52,7 +112,7 @@ scan_fwd_kernel(const ScanArgs p) {
   const int d = blockIdx.x * G + warp;
   const bool active = d < p.D;
   const int split = blockIdx.z;
-  const int N = p.N, L = p.L, NP = p.Npad >> 1;
+  const int N = NT ? NT : p.N, L = p.L, NP = NT ? (NT + 1) / 2 : p.Npad >> 1;
   const int mats = SUMMARY ? 1 : 2;
   const int c_begin = split * p.chunks_per_split;
   const int c_end = min(c_begin + p.chunks_per_split, p.nchunks);
@@ -135,44 +195,31 @@ scan_fwd_kernel(const ScanArgs p) {
     if (!SUMMARY && lane < NP)
       reinterpret_cast<float2*>(p.ckpt)[(rowid * p.nchunks + c) * NP + lane] = sm.H[warp][lane];
 
-    for (int m = 0; m < NP; ++m) {
-      const float2 A2 = sm.A[warp][m];
-      float2 bv[8], a[8], bx[8];
-      lds_pair8(sm.B + m * kChunk, lane, bv);
+    if (NT) {
+      // compile-time state count: fully unrolled and software-pipelined (the
+      // ex2 work of pair m+1 is issued before the scan of pair m)
+      float2 a0[8], b0[8];
+      fwd_pair_pre(0, lane, sm.B, sm.A[warp][0], dd, xx, rmask, any_reset, a0, b0);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        a[i] = ex2x2(fmul2(dd[i], A2));
-        bx[i] = fmul2(xx[i], bv[i]);
-      }
-      if (any_reset) {
+      for (int m = 0; m < (NT + 1) / 2; ++m) {
+        float2 a1[8], b1[8];
+        if (m + 1 < (NT + 1) / 2)
+          fwd_pair_pre(m + 1, lane, sm.B, sm.A[warp][m + 1], dd, xx, rmask, any_reset, a1, b1);
+        fwd_pair_post<SUMMARY>(m, lane, sm.C, sm.H[warp], sm.P[warp], a0, b0, y2);
+        if (m + 1 < (NT + 1) / 2) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if ((rmask >> i) & 1u) a[i] = f2(0.0f, 0.0f);
-      }
-      float2 P = a[0], H = bx[0];
-#pragma unroll
-      for (int i = 1; i < 8; ++i) {
-        H = ffma2(a[i], H, bx[i]);
-        P = fmul2(P, a[i]);
-      }
-      warp_scan_fwd2(P, H, lane);
-      const float2 cin = sm.H[warp][m];
-      const float2 end = ffma2(P, cin, H);
-      float2 start = shfl_up2(end, 1);
-      if (lane == 0) start = cin;
-      if (lane == 31) {
-        sm.H[warp][m] = end;
-        if (SUMMARY) sm.P[warp][m] = fmul2(sm.P[warp][m], P);
-      }
-      if (!SUMMARY) {
-        float2 cv[8];
-        lds_pair8(sm.C + m * kChunk, lane, cv);
-        float2 h = start;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          h = ffma2(a[i], h, bx[i]);
-          y2[i] = ffma2(cv[i], h, y2[i]);
+          for (int i = 0; i < 8; ++i) {
+            a0[i] = a1[i];
+            b0[i] = b1[i];
+          }
         }
+      }
+    } else {
+#pragma unroll 1
+      for (int m = 0; m < NP; ++m) {
+        float2 a0[8], b0[8];
+        fwd_pair_pre(m, lane, sm.B, sm.A[warp][m], dd, xx, rmask, any_reset, a0, b0);
+        fwd_pair_post<SUMMARY>(m, lane, sm.C, sm.H[warp], sm.P[warp], a0, b0, y2);
       }
     }
 
@@ -226,41 +273,47 @@ __global__ void cu_seqlens_to_seq_kernel(const int32_t* __restrict__ cu, int n_d
   seq[t] = lo;
 }
 
-template <typename T, int G, bool VEC, bool SUMMARY>
+template <typename T, int G, bool VEC, bool SUMMARY, int NT>
 cudaError_t fwd_smem_attr() {
   static bool done = false;  // once per instantiation and process (a benign race)
   if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(scan_fwd_kernel<T, G, VEC, SUMMARY>,
+  cudaError_t e = cudaFuncSetAttribute(scan_fwd_kernel<T, G, VEC, SUMMARY, NT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sizeof(FwdSmem<G>));
   if (e == cudaSuccess) done = true;
   return e;
 }
 
-template <typename T, int G, bool VEC>
+template <typename T, int G, bool VEC, int NT>
 cudaError_t fwd_t(const ScanArgs& a, cudaStream_t s) {
   dim3 block(G * 32);
   const size_t smem = sizeof(FwdSmem<G>);
-  cudaError_t e = fwd_smem_attr<T, G, VEC, false>();
-  if (e == cudaSuccess && a.nsplits > 1) e = fwd_smem_attr<T, G, VEC, true>();
+  cudaError_t e = fwd_smem_attr<T, G, VEC, false, NT>();
+  if (e == cudaSuccess && a.nsplits > 1) e = fwd_smem_attr<T, G, VEC, true, NT>();
   if (e != cudaSuccess) return e;
   if (a.nsplits > 1) {
     dim3 g1((a.D + G - 1) / G, a.B, a.nsplits - 1);
-    scan_fwd_kernel<T, G, VEC, true><<<g1, block, smem, s>>>(a);
+    scan_fwd_kernel<T, G, VEC, true, NT><<<g1, block, smem, s>>>(a);
     const int n = a.B * a.D * a.Npad;
     fwd_split_carry_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.split_P, a.split_H, a.split_in,
                                                           a.B * a.D, a.nsplits, a.Npad);
   }
   dim3 g2((a.D + G - 1) / G, a.B, a.nsplits);
-  scan_fwd_kernel<T, G, VEC, false><<<g2, block, smem, s>>>(a);
+  scan_fwd_kernel<T, G, VEC, false, NT><<<g2, block, smem, s>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+template <int NT>
+cudaError_t fwd_dispatch(const ScanArgs& a, cudaStream_t s) {
+  if (a.bf16)
+    return a.vec ? fwd_t<__nv_bfloat16, 4, true, NT>(a, s) : fwd_t<__nv_bfloat16, 4, false, NT>(a, s);
+  return a.vec ? fwd_t<float, 4, true, NT>(a, s) : fwd_t<float, 4, false, NT>(a, s);
+}
+
 cudaError_t launch_scan_fwd(const ScanArgs& a, cudaStream_t s) {
-  if (a.bf16) return a.vec ? fwd_t<__nv_bfloat16, 4, true>(a, s) : fwd_t<__nv_bfloat16, 4, false>(a, s);
-  return a.vec ? fwd_t<float, 4, true>(a, s) : fwd_t<float, 4, false>(a, s);
+  return a.N == 16 ? fwd_dispatch<16>(a, s) : fwd_dispatch<0>(a, s);
 }
 
 cudaError_t launch_cu_seqlens_to_seq(const int32_t* cu, int n_docs, int L, int32_t* seq,

@@ -389,7 +389,7 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": dict(workload_config(sh, cfg), parallelism=f"replicas x{world}"),
         "roofline": roof,
-        "scan": {"tokens_per_s": world * nlay * B * L / (scan_ms * 1e-3),
+        "scan": {"tokens_per_s": world * B * L / (scan_ms * 1e-3),  # scan fwd+bwd per layer
                  "ms_per_layer": {n: avg[n] for n in names},
                  "hbm_gbs": hbm, "hbm_frac_of_measured": {n: hbm[n] / pk["hbm_gbs"] for n in names},
                  "roofline_ms_per_layer": {"sfu_2BDLN": t_sfu, "hbm_alg_bytes": t_hbm},

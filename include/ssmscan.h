@@ -56,7 +56,7 @@ typedef enum {
     SSM_ERR_INVALID_ARG = 1, /* null pointer, bad size, bad alignment, bad struct_size */
     SSM_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. N > 16, W != 4) */
     SSM_ERR_CUDA = 3,        /* a CUDA launch or runtime call failed */
-    SSM_ERR_TIMEOUT = 4,     /* reserved: a bounded device-side wait gave up */
+    SSM_ERR_TIMEOUT = 4,     /* a bounded device-side wait gave up (see ssm_scan_status) */
     SSM_ERR_INJECTED = 5     /* host-side fault injection (env SSM_INJECT_FAIL) */
 } ssm_status_t;
 
@@ -166,6 +166,16 @@ typedef struct {
  * state is not differentiated (it has no incoming gradient). */
 ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
                           ssm_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * ssm_scan_status — device-side status of the last ssm_scan_fwd / ssm_scan_bwd
+ * that used p->workspace: 0 when every bounded wait inside the kernels (the
+ * completion waits of the TMA tile copies) completed, SSM_ERR_TIMEOUT when one
+ * gave up (the kernel then stopped early and its outputs are invalid). The
+ * forward resets the word; the backward only sets it. Copies 4 bytes from the
+ * workspace to *device_status and SYNCHRONISES `stream`.
+ * ------------------------------------------------------------------------ */
+ssm_status_t ssm_scan_status(const ssm_scan_params* p, int* device_status, ssm_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * ssm_probe_ex2_rate — diagnostic: measures this device's sustained rate of

@@ -13,13 +13,14 @@ import ctypes
 
 from . import _lib
 from ._lib import (SsmError, ssm_abi_version, ssm_conv1d_bwd, ssm_conv1d_bwd_workspace_size,
-                   ssm_conv1d_fwd, ssm_last_error, ssm_probe_ex2_rate, ssm_scan_bwd,
+                   ssm_conv1d_fwd, ssm_last_error, ssm_probe_ex2_rate, ssm_scan_bwd, ssm_scan_status,
                    ssm_scan_fwd, ssm_scan_grads, ssm_scan_params, ssm_scan_workspace_size)
 
 __all__ = [
     "SsmError", "ssm_abi_version", "ssm_last_error", "ssm_conv1d_fwd", "ssm_conv1d_bwd",
     "ssm_conv1d_bwd_workspace_size", "ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_scan_bwd",
-    "ssm_scan_params", "ssm_scan_grads", "ssm_probe_ex2_rate", "probe_ex2_rate", "conv1d_fwd", "conv1d_bwd", "scan_params",
+    "ssm_scan_params", "ssm_scan_grads", "ssm_probe_ex2_rate", "probe_ex2_rate", "ssm_scan_status",
+    "scan_status", "conv1d_fwd", "conv1d_bwd", "scan_params",
     "scan_workspace_size", "scan_fwd", "scan_bwd", "load",
 ]
 
@@ -156,6 +157,18 @@ def scan_params(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, sof
 
 def scan_workspace_size(p: ssm_scan_params) -> int:
     return ssm_scan_workspace_size(p)
+
+
+def scan_status(u, A, workspace, stream=None) -> int:
+    """Device status word of `workspace` (0 = ok, 4 = a bounded wait timed out);
+    synchronises the stream."""
+    B, D, L = u.shape
+    p = ssm_scan_params()
+    p.struct_size = ctypes.sizeof(ssm_scan_params)
+    p.B, p.D, p.L, p.N = B, D, L, A.shape[1]
+    p.dtype = _dtype_code(u)
+    p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    return ssm_scan_status(p, _stream(stream, u.device))
 
 
 def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softplus=True,

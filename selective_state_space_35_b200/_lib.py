@@ -91,6 +91,8 @@ def load(path: str | None = None):
     L.ssm_scan_fwd.argtypes = [ctypes.POINTER(ssm_scan_params), _vp]
     L.ssm_scan_bwd.restype = _i
     L.ssm_scan_bwd.argtypes = [ctypes.POINTER(ssm_scan_params), ctypes.POINTER(ssm_scan_grads), _vp]
+    L.ssm_scan_status.restype = _i
+    L.ssm_scan_status.argtypes = [ctypes.POINTER(ssm_scan_params), ctypes.POINTER(_i), _vp]
     L.ssm_probe_ex2_rate.restype = _i
     L.ssm_probe_ex2_rate.argtypes = [_vp, _sz, ctypes.POINTER(ctypes.c_double), _vp]
     if path is None:
@@ -130,6 +132,12 @@ def ssm_scan_workspace_size(params: ssm_scan_params) -> int:
     n = _sz(0)
     check(load().ssm_scan_workspace_size(ctypes.byref(params), ctypes.byref(n)))
     return n.value
+
+
+def ssm_scan_status(params: ssm_scan_params, stream) -> int:
+    v = _i(0)
+    check(load().ssm_scan_status(ctypes.byref(params), ctypes.byref(v), stream))
+    return v.value
 
 
 def ssm_probe_ex2_rate(sink, sink_floats: int, stream) -> float:

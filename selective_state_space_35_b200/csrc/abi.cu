@@ -106,7 +106,7 @@ ScanPlan plan_scan(const ssm_scan_params* p) {
   s.chunks_per_split = (s.nchunks + P - 1) / P;
   s.nsplits = (s.nchunks + s.chunks_per_split - 1) / s.chunks_per_split;
   const size_t rows = (size_t)p->B * p->D;
-  size_t off = 0;
+  size_t off = up(sizeof(int));  // status word first
   s.off_seq = off;
   off += p->cu_seqlens ? up((size_t)p->B * p->L * sizeof(int32_t)) : 0;
   s.off_ckpt = off;
@@ -144,6 +144,7 @@ ssm_status_t build_args(const ssm_scan_params* p, const ScanPlan& pl, ssm::ScanA
   a->softplus = p->delta_softplus ? 1 : 0;
   a->out = p->out;
   a->final_state = p->final_state;
+  a->status = reinterpret_cast<int*>(ws);
   a->ckpt = reinterpret_cast<float*>(ws + pl.off_ckpt);
   a->split_P = pl.nsplits > 1 ? reinterpret_cast<float*>(ws + pl.off_sP) : nullptr;
   a->split_H = pl.nsplits > 1 ? reinterpret_cast<float*>(ws + pl.off_sH) : nullptr;
@@ -281,6 +282,8 @@ ssm_status_t ssm_scan_fwd(const ssm_scan_params* p, ssm_stream_t stream) {
   build_args(p, pl, &a);
   a.vec = vec_ok(p->L, {p->u, p->delta, p->z, p->Bm, p->Cm, p->out, a.seq});
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e0 = cudaMemsetAsync(a.status, 0, sizeof(int), s);  // fresh status for this fwd/bwd
+  if (e0 != cudaSuccess) return cuda_status(e0, "ssm_scan_fwd status reset");
   if (p->cu_seqlens) {
     cudaError_t e = ssm::launch_cu_seqlens_to_seq(p->cu_seqlens, p->n_docs, p->L,
                                                   const_cast<int32_t*>(a.seq), s);
@@ -336,6 +339,17 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
   if (e == cudaSuccess) e = cudaMemsetAsync(g->dC, 0, bc, s);
   if (e != cudaSuccess) return cuda_status(e, "ssm_scan_bwd memset");
   return cuda_status(ssm::launch_scan_bwd(a, s), "ssm_scan_bwd launch");
+}
+
+ssm_status_t ssm_scan_status(const ssm_scan_params* p, int* device_status, ssm_stream_t stream) {
+  if (!device_status) return fail(SSM_ERR_INVALID_ARG, "device_status is NULL");
+  ssm_status_t st = check_params(p);
+  if (st != SSM_OK) return st;
+  if (!p->workspace) return fail(SSM_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(device_status, p->workspace, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  return cuda_status(e, "ssm_scan_status");
 }
 
 ssm_status_t ssm_probe_ex2_rate(float* sink, size_t sink_floats, double* ex2_per_second,

@@ -19,6 +19,26 @@ __device__ __forceinline__ float ex2_approx(float x) {
 
 __device__ __forceinline__ float sigmoidf_(float v) { return 1.0f / (1.0f + expf(-v)); }
 
+// softplus(v) = log(1 + x), x = e^v, without branches: both candidates are
+// computed and one is selected (no divergence inside a warp).
+//  * x < 1/32: x - x^2/2 + x^3/3 - x^4/4 + x^5/5 (truncation < x^6/6, i.e. a
+//    relative error below 5e-9);
+//  * otherwise log2(1 + x) on the SFU times ln 2 (log(1+x) > 0.03 there, so
+//    the SFU's absolute error of a few 1e-7 and the rounding of 1 + x stay
+//    below 1e-5 relative);
+//  * v > 20: v (the difference is below 2.1e-9).
+__device__ __forceinline__ float softplus_sfu(float v) {
+  const float x = __expf(v);
+  float q = fmaf(x, 0.2f, -0.25f);
+  q = fmaf(x, q, 0.33333334f);
+  q = fmaf(x, q, -0.5f);
+  q = fmaf(x, q, 1.0f);
+  const float series = x * q;
+  const float lg = __log2f(1.0f + x) * 0.69314718f;
+  const float r = x < 0.03125f ? series : lg;
+  return v > 20.0f ? v : r;
+}
+
 // sigmoid on the SFU: e^-v via ex2, reciprocal via rcp (relative error a few
 // ulp; 1 for v -> +inf, 0 for v -> -inf).
 __device__ __forceinline__ float sigmoid_fast(float v) {

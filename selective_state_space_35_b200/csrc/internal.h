@@ -58,6 +58,7 @@ struct ScanArgs {
   float* dD;
   float* ddelta_bias;
   // workspace pieces
+  int* status;        // sticky device status word (0 = ok, 4 = a bounded wait timed out)
   float* ckpt;        // [B*D][nchunks][Npad] state entering each chunk
   float* split_P;     // [B*D][P][Npad] per-split decay product (pass 1)
   float* split_H;     // [B*D][P][Npad] per-split end value from zero (pass 1)

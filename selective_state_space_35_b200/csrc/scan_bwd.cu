@@ -62,7 +62,7 @@ template <int G>
 struct BwdSmem {
   float B[kNMax * kChunk];
   float C[kNMax * kChunk];
-  __nv_bfloat16 raw[2][kNMax][kChunk];  // next chunk's raw B / C (async path)
+  __nv_bfloat16 raw[2][kNMax][kChunk];  // raw B / C of the next chunk, by cp.async
   float4 slice[2][G][2][64];            // [state parity][warp][dB | dC][piece]
   float dA[G][kNMax][32];
 };
@@ -193,7 +193,10 @@ __device__ __forceinline__ void bwd_reduce(int n, const float4 (*slice)[G][2][64
 template <typename T, int G, bool VEC, int NT>
 __global__ void __launch_bounds__(G * 32, SSM_BWD_MIN_BLOCKS)
 scan_bwd_kernel(const ScanArgs p) {
-  constexpr bool ASYNC = VEC && sizeof(T) == 2;  // B / C tiles by cp.async one chunk ahead
+  // bf16 on the vector path: B / C tiles arrive by cp.async one chunk ahead
+  // (per-thread 16-byte copies; on this kernel, with a CTA barrier per state,
+  // they measured faster than warp-issued TMA bulk copies)
+  constexpr bool ASYNC = VEC && sizeof(T) == 2;
   extern __shared__ float4 smem_dyn[];
   BwdSmem<G>& sm = *reinterpret_cast<BwdSmem<G>*>(smem_dyn);
 
@@ -249,17 +252,18 @@ scan_bwd_kernel(const ScanArgs p) {
     if (ASYNC) {
       cp_async_wait_all();
       __syncthreads();  // the previous chunk's readers of B / C are done
-      convert_bc_rows(&sm.raw[0][0][0], sm.B, sm.C, 2, N);
+      convert_bc_rows(&sm.raw[0][0][0], sm.B, sm.C, 2, N, L - t0);
       if (c - 1 >= c_begin)  // each thread refills only the pieces it just converted
         issue_bc_raw(reinterpret_cast<const __nv_bfloat16*>(Bm),
                      reinterpret_cast<const __nv_bfloat16*>(Cm), &sm.raw[0][0][0], 2, b, N, L,
                      t0 - kChunk);
+      __syncthreads();
     } else {
       __syncthreads();
       stage_rows<T, VEC>(Bm, sm.B, b, N, L, t0);
       stage_rows<T, VEC>(Cm, sm.C, b, N, L, t0);
+      __syncthreads();
     }
-    __syncthreads();
 
     const int tl = t0 + lane * 8;
     float2 dlp[4], xup[4], dyp[4];
@@ -282,7 +286,7 @@ scan_bwd_kernel(const ScanArgs p) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float v = dl[i] + bias;
-        const float s = p.softplus ? (v > 20.0f ? v : log1pf(__expf(v))) : v;
+        const float s = p.softplus ? softplus_sfu(v) : v;
         dt[i] = (tl + i < L) ? s : 0.0f;
         Sdl += dt[i];
         dy[i] = z_row ? go[i] * (zz[i] * sigmoid_fast(zz[i])) : go[i];

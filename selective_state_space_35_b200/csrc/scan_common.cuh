@@ -150,6 +150,80 @@ __device__ __forceinline__ void lds8(const float* base, int lane, float v[8]) {
 }
 
 // ---------------------------------------------------------------------------
+// TMA bulk copies (cp.async.bulk, no multicast) completing on an mbarrier.
+// Every wait is bounded: after kMaxWaitIters polls the kernel records
+// SSM_ERR_TIMEOUT in the status word and stops, instead of hanging.
+// ---------------------------------------------------------------------------
+constexpr int kMaxWaitIters = 1 << 22;
+constexpr int kStatusTimeout = 4;  // == SSM_ERR_TIMEOUT
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+// 1-D bulk copy global -> shared; src, dst 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void tma_load_1d(void* dst, const void* src, unsigned bytes,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Returns false (and records a timeout in *status) if the phase never completes.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity, int* status) {
+  for (int i = 0; i < kMaxWaitIters; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  if (status) atomicExch(status, kStatusTimeout);
+  return false;
+}
+
+// Issue, from warp 0, the bulk copies of rows [0, N) of B (and C) for chunk
+// tokens [t0, t0 + kChunk) into raw[mat][n][.] bf16: lane 0 arms the
+// mbarrier with the total byte count, then lane i copies row i (mats * N <=
+// 32 rows). Rows past L are shorter; the converter masks them.
+__device__ __forceinline__ void tma_issue_bc(const __nv_bfloat16* __restrict__ Bm,
+                                             const __nv_bfloat16* __restrict__ Cm,
+                                             __nv_bfloat16* raw, int mats, int b, int N, int L,
+                                             int t0, uint64_t* bar) {
+  const int lane = threadIdx.x & 31;
+  const int ntok = min(kChunk, L - t0);
+  const unsigned bytes = static_cast<unsigned>(ntok) * 2u;  // multiple of 16: L % 8 == 0
+  // The raw buffer was last read (generic loads) before the CTA barrier that
+  // precedes this call, so the async-proxy writes below cannot overtake them.
+  if (lane == 0) mbar_expect_tx(bar, bytes * static_cast<unsigned>(mats * N));
+  __syncwarp();
+  if (lane < mats * N) {
+    const int mat = lane >= N, n = lane - mat * N;
+    tma_load_1d(raw + ((size_t)mat * kNMax + n) * kChunk,
+                (mat ? Cm : Bm) + ((size_t)b * N + n) * L + t0, bytes, bar);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Asynchronous staging of the raw bf16 B / C chunk tiles (vector path): the
 // copies for chunk c+1 are issued with cp.async while chunk c is computed, so
 // their latency is hidden; each thread later converts exactly the pieces it
@@ -187,13 +261,14 @@ __device__ __forceinline__ void issue_bc_raw(const __nv_bfloat16* __restrict__ B
 // fp32 row tile layout: row n, float4 index j = tokens [8j, 8j+4), 32 + j =
 // [8j+4, 8j+8).
 __device__ __forceinline__ void convert_bc_rows(const __nv_bfloat16* raw, float* sB, float* sC,
-                                                int mats, int N) {
+                                                int mats, int N, int tleft = kChunk) {
   const int per = N * 32;
   for (int idx = threadIdx.x; idx < mats * per; idx += blockDim.x) {
     const int mat = idx >= per;
     const int rem = idx - mat * per;
     const int n = rem >> 5, j = rem & 31;
-    const uint4 r = *reinterpret_cast<const uint4*>(raw + ((size_t)mat * kNMax + n) * kChunk + 8 * j);
+    uint4 r = *reinterpret_cast<const uint4*>(raw + ((size_t)mat * kNMax + n) * kChunk + 8 * j);
+    if (8 * j >= tleft) r = make_uint4(0u, 0u, 0u, 0u);  // past the end of the row
     float4* dst = reinterpret_cast<float4*>((mat ? sC : sB) + n * kChunk);
     dst[j] = make_float4(bf16lo(r.x), bf16hi(r.x), bf16lo(r.y), bf16hi(r.y));
     dst[32 + j] = make_float4(bf16lo(r.z), bf16hi(r.z), bf16lo(r.w), bf16hi(r.w));
@@ -227,15 +302,17 @@ __device__ __forceinline__ void issue_bc_raw_pairs(const __nv_bfloat16* __restri
 }
 
 __device__ __forceinline__ void convert_bc_pairs(const __nv_bfloat16* raw, float2* sB, float2* sC,
-                                                 int mats, int N) {
+                                                 int mats, int N, int tleft = kChunk) {
   const int NP = (N + 1) >> 1;
   const int per = NP * 32;
   for (int idx = threadIdx.x; idx < mats * per; idx += blockDim.x) {
     const int mat = idx >= per;
     const int rem = idx - mat * per;
     const int m = rem >> 5, j = rem & 31;
-    const uint4 r0 = *reinterpret_cast<const uint4*>(raw + ((size_t)mat * kNMax + 2 * m) * kChunk + 8 * j);
-    const uint4 r1 = *reinterpret_cast<const uint4*>(raw + ((size_t)mat * kNMax + 2 * m + 1) * kChunk + 8 * j);
+    uint4 r0 = *reinterpret_cast<const uint4*>(raw + ((size_t)mat * kNMax + 2 * m) * kChunk + 8 * j);
+    uint4 r1 = *reinterpret_cast<const uint4*>(raw + ((size_t)mat * kNMax + 2 * m + 1) * kChunk + 8 * j);
+    if (8 * j >= tleft) r0 = r1 = make_uint4(0u, 0u, 0u, 0u);  // past the end of the row
+    if (2 * m + 1 >= N) r1 = make_uint4(0u, 0u, 0u, 0u);        // padding state of an odd N
     float4* dst = reinterpret_cast<float4*>((mat ? sC : sB) + m * kChunk);
     dst[j] = make_float4(bf16lo(r0.x), bf16lo(r1.x), bf16hi(r0.x), bf16hi(r1.x));
     dst[32 + j] = make_float4(bf16lo(r0.y), bf16lo(r1.y), bf16hi(r0.y), bf16hi(r1.y));

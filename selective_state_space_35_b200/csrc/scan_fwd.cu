@@ -33,7 +33,8 @@ template <int G>
 struct FwdSmem {
   float2 B[kNP * kChunk];                 // B tile, state-pair layout
   float2 C[kNP * kChunk];                 // C tile, state-pair layout
-  __nv_bfloat16 raw[2][kNMax][kChunk];    // next chunk's raw B / C (async path)
+  __nv_bfloat16 raw[2][kNMax][kChunk];    // raw B / C of the next chunk, by TMA
+  uint64_t bar;                           // TMA completion (one phase per chunk)
   float2 A[G][kNP];                       // A' = A log2(e), per state pair
   float2 H[G][kNP];                       // running state entering the current chunk
   float2 P[G][kNP];                       // SUMMARY: running product of a over the split
@@ -102,7 +103,7 @@ __device__ __forceinline__ void fwd_pair_post(int m, int lane, const float2* __r
 template <typename T, int G, bool VEC, bool SUMMARY, int NT>
 __global__ void __launch_bounds__(G * 32, SSM_FWD_MIN_BLOCKS)
 scan_fwd_kernel(const ScanArgs p) {
-  // bf16 on the vector path: B / C tiles arrive by cp.async one chunk ahead
+  // bf16 on the vector path: B / C tiles arrive by TMA one chunk ahead
   constexpr bool ASYNC = VEC && sizeof(T) == 2;
   extern __shared__ float4 smem_dyn[];
   FwdSmem<G>& sm = *reinterpret_cast<FwdSmem<G>*>(smem_dyn);
@@ -125,10 +126,14 @@ scan_fwd_kernel(const ScanArgs p) {
   const T* dl_row = static_cast<const T*>(p.delta) + row;
   const T* z_row = p.z ? static_cast<const T*>(p.z) + row : nullptr;
 
-  if (ASYNC)
-    issue_bc_raw_pairs(reinterpret_cast<const __nv_bfloat16*>(Bm),
-                       reinterpret_cast<const __nv_bfloat16*>(Cm), &sm.raw[0][0][0], mats, b, N, L,
-                       c_begin * kChunk);
+  if (ASYNC && threadIdx.x == 0) {
+    mbar_init(&sm.bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (ASYNC && threadIdx.x < 32)
+    tma_issue_bc(reinterpret_cast<const __nv_bfloat16*>(Bm), reinterpret_cast<const __nv_bfloat16*>(Cm),
+                 &sm.raw[0][0][0], mats, b, N, L, c_begin * kChunk, &sm.bar);
   if (lane < kNP) {
     float a0 = 0.0f, a1 = 0.0f;
     if (active && 2 * lane < N) a0 = __ldg(p.A + (size_t)d * N + 2 * lane) * kLog2e;
@@ -154,19 +159,22 @@ scan_fwd_kernel(const ScanArgs p) {
   for (int c = c_begin; c < c_end; ++c) {
     const int t0 = c * kChunk;
     if (ASYNC) {
-      cp_async_wait_all();
-      __syncthreads();  // the previous chunk's readers of B / C are done
-      convert_bc_pairs(&sm.raw[0][0][0], sm.B, sm.C, mats, N);
-      if (c + 1 < c_end)  // each thread refills only the pieces it just converted
-        issue_bc_raw_pairs(reinterpret_cast<const __nv_bfloat16*>(Bm),
-                           reinterpret_cast<const __nv_bfloat16*>(Cm), &sm.raw[0][0][0], mats, b,
-                           N, L, t0 + kChunk);
+      // chunk c is the (c - c_begin)-th phase of the barrier
+      const bool ok = mbar_wait_bounded(&sm.bar, (c - c_begin) & 1, p.status);
+      // also: every thread is done with chunk c - 1's tiles; all leave together on a timeout
+      if (!__syncthreads_and(ok)) break;
+      convert_bc_pairs(&sm.raw[0][0][0], sm.B, sm.C, mats, N, L - t0);
+      __syncthreads();  // tiles complete; raw free again
+      if (threadIdx.x < 32 && c + 1 < c_end)  // next chunk, hidden behind this chunk's work
+        tma_issue_bc(reinterpret_cast<const __nv_bfloat16*>(Bm),
+                     reinterpret_cast<const __nv_bfloat16*>(Cm), &sm.raw[0][0][0], mats, b, N, L,
+                     t0 + kChunk, &sm.bar);
     } else {
       __syncthreads();
       stage_pairs<T, VEC>(Bm, sm.B, b, N, L, t0);
       if (!SUMMARY) stage_pairs<T, VEC>(Cm, sm.C, b, N, L, t0);
+      __syncthreads();
     }
-    __syncthreads();
     if (!active) continue;
 
     const int tl = t0 + lane * 8;
@@ -183,7 +191,7 @@ scan_fwd_kernel(const ScanArgs p) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float v = dl[i] + bias;
-      const float s = p.softplus ? (v > 20.0f ? v : log1pf(__expf(v))) : v;
+      const float s = p.softplus ? softplus_sfu(v) : v;
       const float dt = (tl + i < L) ? s : 0.0f;  // dt = 0 past the end: a = 1, no input
       dd[i] = f2(dt, dt);
       xx[i] = f2(dt * uu[i], dt * uu[i]);

@@ -377,3 +377,15 @@ def test_unaligned_gradient_buffers_take_scalar_path():
                      grads={"dB": bufB[1:].view(B, N, L), "dC": bufC[1:].view(B, N, L)}, **kw)
     for k in ("dB", "dC", "du", "ddelta", "dz"):
         assert rel_l2(host64(g[k]), host64(ref[k])) <= 1e-6, k
+
+
+def test_device_status_word_clear_after_tma_staged_runs():
+    import selective_state_space_35_b200 as ssm
+    inp = _small(2, 9, 16, 2048, 909, dtype="bf16", nbound=3)  # bf16, L % 8 == 0: TMA-staged tiles
+    dv = device_inputs(inp)
+    u = ssm.conv1d_fwd(dv["x"], dv["conv_w"], dv["conv_b"], dv["seq_idx"])
+    kw = dict(z=dv["z"], Dskip=dv["Dskip"], delta_bias=dv["delta_bias"], seq_idx=dv["seq_idx"])
+    for P in (1, 3):
+        _, _, ws = ssm.scan_fwd(u, dv["delta"], dv["A"], dv["Bm"], dv["Cm"], n_splits=P, **kw)
+        ssm.scan_bwd(u, dv["delta"], dv["A"], dv["Bm"], dv["Cm"], dv["dout"], ws, n_splits=P, **kw)
+        assert ssm.scan_status(u, dv["A"], ws) == 0

@@ -104,6 +104,32 @@ ssm_status_t ssm_conv1d_bwd(const void* x, const float* w, const float* bias,
                             size_t workspace_bytes, ssm_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * ssm_conv1d_bwd_noalloc — ssm_conv1d_bwd for callers that cannot allocate
+ * device memory: hosts that hand a library only its input and output
+ * buffers (plugin interfaces of serving runtimes and frameworks that own all
+ * device memory) and loops that must not call cudaMalloc / cudaFree, which
+ * can synchronise the whole device. There is no counterpart on the pages;
+ * this is a deployment variant of the call above.
+ *   Arguments and results are those of ssm_conv1d_bwd without the workspace.
+ *   Scratch: the per-tile dw / dbias partial sums go to a fixed device array
+ *   of 2^20 floats (4 MiB) that every device using the library keeps until
+ *   the process exits; sizes with B * ceil(L / 1024) * D * 5 > 2^20 are
+ *   rejected with SSM_ERR_UNSUPPORTED and a message naming the limit.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *   first call before any stream capture on the device.
+ *   The array is shared by every call and keeps the last call's contents;
+ *   each call overwrites every partial it reads, so nothing needs clearing,
+ *   but two calls that overlap on the GPU (other streams, other threads) race
+ *   on it: serialise them.
+ *   Allocates nothing and calls no allocating routine.
+ * ------------------------------------------------------------------------ */
+ssm_status_t ssm_conv1d_bwd_noalloc(const void* x, const float* w, const float* bias,
+                                    const int32_t* seq_idx, const void* du, void* dx,
+                                    float* dw, float* dbias, int B, int D, int L, int W,
+                                    ssm_dtype_t dtype, int silu, ssm_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Selective scan. For each row (b, d) and state n < N, with
  *   dt_t = softplus(delta[b][d][t] + delta_bias[d])   (or without softplus)
  *   a_t  = exp(dt_t * A[d][n])      (0 at the first token of a document)

@@ -12,13 +12,14 @@ from __future__ import annotations
 import ctypes
 
 from . import _lib
-from ._lib import (SsmError, ssm_abi_version, ssm_conv1d_bwd, ssm_conv1d_bwd_workspace_size,
+from ._lib import (SsmError, ssm_abi_version, ssm_conv1d_bwd, ssm_conv1d_bwd_noalloc,
+                   ssm_conv1d_bwd_workspace_size,
                    ssm_conv1d_fwd, ssm_last_error, ssm_probe_ex2_rate, ssm_scan_bwd, ssm_scan_status,
                    ssm_scan_fwd, ssm_scan_grads, ssm_scan_params, ssm_scan_workspace_size)
 
 __all__ = [
     "SsmError", "ssm_abi_version", "ssm_last_error", "ssm_conv1d_fwd", "ssm_conv1d_bwd",
-    "ssm_conv1d_bwd_workspace_size", "ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_scan_bwd",
+    "ssm_conv1d_bwd_workspace_size", "ssm_conv1d_bwd_noalloc", "ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_scan_bwd",
     "ssm_scan_params", "ssm_scan_grads", "ssm_probe_ex2_rate", "probe_ex2_rate", "ssm_scan_status",
     "scan_status", "conv1d_fwd", "conv1d_bwd", "scan_params",
     "scan_workspace_size", "scan_fwd", "scan_bwd", "load",

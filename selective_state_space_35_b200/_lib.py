@@ -85,6 +85,9 @@ def load(path: str | None = None):
     L.ssm_conv1d_bwd.restype = _i
     L.ssm_conv1d_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                  _vp, _sz, _vp]
+    L.ssm_conv1d_bwd_noalloc.restype = _i
+    L.ssm_conv1d_bwd_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
+                                         _i, _i, _vp]
     L.ssm_scan_workspace_size.restype = _i
     L.ssm_scan_workspace_size.argtypes = [ctypes.POINTER(ssm_scan_params), ctypes.POINTER(_sz)]
     L.ssm_scan_fwd.restype = _i
@@ -126,6 +129,10 @@ def ssm_conv1d_bwd_workspace_size(B, D, L, W) -> int:
 
 def ssm_conv1d_bwd(*args) -> int:
     return load().ssm_conv1d_bwd(*args)
+
+
+def ssm_conv1d_bwd_noalloc(*args) -> int:
+    return load().ssm_conv1d_bwd_noalloc(*args)
 
 
 def ssm_scan_workspace_size(params: ssm_scan_params) -> int:

@@ -263,6 +263,45 @@ ssm_status_t ssm_conv1d_bwd(const void* x, const float* w, const float* bias,
                      "ssm_conv1d_bwd launch");
 }
 
+ssm_status_t ssm_conv1d_bwd_noalloc(const void* x, const float* w, const float* bias,
+                                    const int32_t* seq_idx, const void* du, void* dx, float* dw,
+                                    float* dbias, int B, int D, int L, int W, ssm_dtype_t dtype,
+                                    int silu, ssm_stream_t stream) {
+  if (injected("ssm_conv1d_bwd_noalloc"))
+    return fail(SSM_ERR_INJECTED, "ssm_conv1d_bwd_noalloc: injected failure");
+  if (!x || !w || !du || !dx || !dw)
+    return fail(SSM_ERR_INVALID_ARG, "x, w, du, dx and dw must be non-NULL");
+  size_t need = 0;
+  ssm_status_t st = ssm_conv1d_bwd_workspace_size(B, D, L, W, &need);
+  if (st != SSM_OK) return st;
+  const size_t floats = (size_t)B * ssm::conv_tiles(L) * D * 5;
+  if (floats > ssm::kConvBwdScratchFloats)
+    return fail(SSM_ERR_UNSUPPORTED,
+                "ssm_conv1d_bwd_noalloc: B * ceil(L / %d) * D * 5 = %zu partial sums exceed the fixed "
+                "scratch of %zu floats; use ssm_conv1d_bwd with a workspace",
+                ssm::kConvTile, floats, ssm::kConvBwdScratchFloats);
+  if (B > 65535 || D > 65535) return fail(SSM_ERR_UNSUPPORTED, "B and D must be <= 65535");
+  if (dtype != SSM_DTYPE_F32 && dtype != SSM_DTYPE_BF16)
+    return fail(SSM_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (dx == x || dx == du) return fail(SSM_ERR_INVALID_ARG, "dx may not alias x or du");
+  const size_t es = elem_size(dtype);
+  if (!aligned(x, es) || !aligned(du, es) || !aligned(dx, es) || !aligned(w, 4) ||
+      !aligned(dw, 4) || (bias && !aligned(bias, 4)) || (dbias && !aligned(dbias, 4)) ||
+      (seq_idx && !aligned(seq_idx, 4)))
+    return fail(SSM_ERR_INVALID_ARG, "misaligned pointer");
+  float* scratch = nullptr;
+  cudaError_t e = ssm::conv_bwd_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_status(e, "ssm_conv1d_bwd_noalloc scratch address");
+  ssm::ConvArgs a{};
+  a.x = x; a.w = w; a.bias = bias; a.seq = seq_idx; a.du = du; a.out = dx;
+  a.dw = dw; a.dbias = dbias; a.partial = scratch;
+  a.B = B; a.D = D; a.L = L; a.silu = silu ? 1 : 0;
+  a.bf16 = dtype == SSM_DTYPE_BF16;
+  a.vec = vec_ok(L, {x, du, dx, seq_idx});
+  return cuda_status(ssm::launch_conv1d_bwd(a, reinterpret_cast<cudaStream_t>(stream)),
+                     "ssm_conv1d_bwd_noalloc launch");
+}
+
 ssm_status_t ssm_scan_workspace_size(const ssm_scan_params* p, size_t* bytes) {
   if (!bytes) return fail(SSM_ERR_INVALID_ARG, "bytes is NULL");
   ssm_status_t st = check_params(p);

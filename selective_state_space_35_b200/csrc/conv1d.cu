@@ -238,3 +238,41 @@ cudaError_t launch_conv1d_bwd(const ConvArgs& a, cudaStream_t s) {
 }
 
 }  // namespace ssm
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the conv1d backward (ssm_conv1d_bwd_noalloc).
+// Its scratch (the per-tile dw / dbias partial sums) lives in a fixed
+// file-scope device array instead of a caller workspace.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace ssm {
+
+namespace {
+// 4 MiB on every device that loads the library, held until the process exits.
+__device__ __align__(256) float g_conv_bwd_scratch[kConvBwdScratchFloats];
+
+std::mutex g_scratch_mu;
+float* g_scratch_ptr[kMaxScratchDevices] = {};  // device address per device ordinal
+}  // namespace
+
+// Device address of g_conv_bwd_scratch on the current device. The host-side
+// name of the array is only a stand-in; the address is looked up once per
+// device (with that device current) and cached.
+cudaError_t conv_bwd_scratch(float** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxScratchDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_conv_bwd_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_ptr[dev] = static_cast<float*>(p);
+  }
+  *ptr = g_scratch_ptr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace ssm

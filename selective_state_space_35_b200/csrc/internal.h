@@ -29,6 +29,10 @@ struct ConvArgs {
 };
 
 cudaError_t launch_conv1d_fwd(const ConvArgs& a, cudaStream_t s);
+// Fixed device scratch of the allocation-free conv1d backward.
+constexpr size_t kConvBwdScratchFloats = size_t(1) << 20;  // 4 MiB per device
+constexpr int kMaxScratchDevices = 64;
+cudaError_t conv_bwd_scratch(float** ptr);
 cudaError_t launch_conv1d_bwd(const ConvArgs& a, cudaStream_t s);
 inline int conv_tiles(int L) { return (L + kConvTile - 1) / kConvTile; }
 

@@ -64,7 +64,7 @@ int sm_count() {
 
 struct ScanPlan {
   int nchunks, nsplits, chunks_per_split;
-  size_t off_seq, off_ckpt, off_sP, off_sH, off_sIn, off_pA, off_pD, off_pB, total;
+  size_t off_seq, off_ckpt, off_y, off_sP, off_sH, off_sIn, off_pA, off_pD, off_pB, total;
 };
 
 ssm_status_t check_params(const ssm_scan_params* p) {
@@ -111,7 +111,10 @@ ScanPlan plan_scan(const ssm_scan_params* p) {
   off += p->cu_seqlens ? up((size_t)p->B * p->L * sizeof(int32_t)) : 0;
   s.off_ckpt = off;
   const size_t npad = (size_t)((p->N + 1) & ~1);
-  off += up(rows * s.nchunks * npad * sizeof(float));
+  // one state checkpoint per 32-token block, kNMax wide
+  off += up(rows * s.nchunks * 8 * ssm::kNMax * sizeof(float));
+  s.off_y = off;
+  off += p->z ? up(rows * (size_t)p->L * elem_size(p->dtype)) : 0;
   const size_t per_split = up(rows * s.nsplits * npad * sizeof(float));
   s.off_sP = off;
   off += s.nsplits > 1 ? per_split : 0;
@@ -146,6 +149,7 @@ ssm_status_t build_args(const ssm_scan_params* p, const ScanPlan& pl, ssm::ScanA
   a->final_state = p->final_state;
   a->status = reinterpret_cast<int*>(ws);
   a->ckpt = reinterpret_cast<float*>(ws + pl.off_ckpt);
+  a->ysave = p->z ? static_cast<void*>(ws + pl.off_y) : nullptr;
   a->split_P = pl.nsplits > 1 ? reinterpret_cast<float*>(ws + pl.off_sP) : nullptr;
   a->split_H = pl.nsplits > 1 ? reinterpret_cast<float*>(ws + pl.off_sH) : nullptr;
   a->split_in = pl.nsplits > 1 ? reinterpret_cast<float*>(ws + pl.off_sIn) : nullptr;

@@ -58,338 +58,409 @@ __device__ __forceinline__ void lds_tokpairs(const float* row, int lane, float2 
   v[3] = make_float2(q1.z, q1.w);
 }
 
-template <int G>
+// ---------------------------------------------------------------------------
+// Main backward kernel: one thread per (row, state). A warp holds two rows x
+// 16 states, a CTA eight rows of one batch entry, which share the B / C
+// tiles. Time runs backwards in 32-token blocks, each started from the
+// forward's checkpoint; every global input of a block is copied into shared
+// memory by cp.async while the block before it is being processed.
+// ---------------------------------------------------------------------------
+constexpr int kBlk = 32;                   // tokens per block (= checkpoint interval)
+constexpr int kWarps = 4;
+constexpr int kRows = 2 * kWarps;          // rows per CTA
+constexpr int kLd = kBlk + 4;              // fp32 row stride: the 16 state rows on distinct banks
+constexpr int kRowArrays = 5;              // delta, u, dout, z, y (y: forward output before the gate)
+
+template <typename T>
 struct BwdSmem {
-  float B[kNMax * kChunk];
-  float C[kNMax * kChunk];
-  __nv_bfloat16 raw[2][kNMax][kChunk];  // raw B / C of the next chunk, by cp.async
-  float4 slice[2][G][2][64];            // [state parity][warp][dB | dC][piece]
-  float dA[G][kNMax][32];
+  T rawT[2][kNMax][kBlk];                  // B / C of the next block (each thread its own pieces)
+  T rawR[kRowArrays][kRows][kBlk];         // per-row inputs of the next block
+  float B[kNMax][kLd];
+  float C[kNMax][kLd];
+  float dt[kRows][kBlk];                   // step size (0 past the end)
+  float xu[kRows][kBlk];                   // dt u
+  float dy[kRows][kBlk];                   // dL/dy = dout silu(z)
+  float X[kWarps][2][2][kNMax][kLd];       // [warp][array][row half][state][token]
 };
 
-// One state n of one chunk for one lane: rebuild the lane's 8 states from the
-// chunk checkpoint (warp scan), run the adjoint backwards (reverse warp scan,
-// carry-in from the next chunk in lane n's gcarry), accumulate the per-token
-// sums over states, and write this row's dB / dC contributions into the
-// warp's slice.
-__device__ __forceinline__ void bwd_state(int n, int lane, const float* __restrict__ sB,
-                                          const float* __restrict__ sC, float4* mysl,
-                                          float* sdA_n, float A_lane, float A2_lane, float hck,
-                                          float& gcarry, const float2 dlp[4], const float2 xup[4],
-                                          const float2 dyp[4], float Sdl, unsigned rmask,
-                                          bool any_reset, float2 y2[4], float2 sgB2[4],
-                                          float2 dd2[4]) {
-  const float An2 = __shfl_sync(kFull, A2_lane, n);
-  const float Anat = __shfl_sync(kFull, A_lane, n);
-  float2 bp[4], cp[4];
-  lds_tokpairs(sB + n * kChunk, lane, bp);
-  lds_tokpairs(sC + n * kChunk, lane, cp);
-  float a[8], bx[8];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const float2 e = fmul2(dlp[k], f2(An2, An2));
-    a[2 * k] = ex2_approx(e.x);
-    a[2 * k + 1] = ex2_approx(e.y);
-    const float2 q = fmul2(xup[k], bp[k]);
-    bx[2 * k] = q.x;
-    bx[2 * k + 1] = q.y;
+template <int BYTES>
+__device__ __forceinline__ void cp_async_n(void* smem_dst, const void* gmem_src, bool valid) {
+  const unsigned d = smem_u32(smem_dst);
+  const int n = valid ? BYTES : 0;  // 0 source bytes: zero fill
+  asm volatile("cp.async.ca.shared.global [%0], [%1], %2, %3;\n" ::"r"(d), "l"(gmem_src),
+               "n"(BYTES), "r"(n)
+               : "memory");
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f(T v);
+template <>
+__device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T>
+__device__ __forceinline__ T from_f(float v);
+template <>
+__device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+// Two consecutive tokens t, t + 1 of a row (VEC: both in range or both not).
+template <typename T, bool VEC>
+__device__ __forceinline__ void store2(T* row, int t, int L, float v0, float v1) {
+  if (VEC) {
+    if (t < L) {
+      if (sizeof(T) == 2)
+        *reinterpret_cast<uint32_t*>(row + t) = Io<__nv_bfloat16>::pack2(v0, v1);
+      else
+        *reinterpret_cast<float2*>(row + t) = make_float2(v0, v1);
+    }
+  } else {
+    if (t < L) row[t] = from_f<T>(v0);
+    if (t + 1 < L) row[t + 1] = from_f<T>(v1);
   }
-  float Ploc = ex2_approx(An2 * Sdl);
-  if (any_reset) {
+}
+
+struct RowPtrs {
+  const void* p[kRowArrays];
+};
+
+// Copies of the thread's own pieces of block [tb, tb + 32): one (or two, fp32)
+// 16-byte piece of the B / C tiles and tokens tb + 2j, tb + 2j + 1 of each row
+// array of row r. VEC: cp.async (completes later); otherwise plain loads.
+template <typename T, bool VEC>
+__device__ __forceinline__ void issue_block(BwdSmem<T>& sm, const T* __restrict__ Bm,
+                                            const T* __restrict__ Cm, const RowPtrs& rp,
+                                            int n_arrays, int b, int N, int L, int tb, int r,
+                                            int j, bool active) {
+  constexpr int kPiece = 16 / (int)sizeof(T);  // tokens per 16-byte piece
+  constexpr int kPPR = kBlk / kPiece;
+  constexpr int kPieces = 2 * kNMax * kPPR;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if ((rmask >> i) & 1u) a[i] = 0.0f;
-    if (rmask) Ploc = 0.0f;
-  }
-  // forward recompute of this lane's 8 states
-  float H = bx[0];
+  for (int pc = threadIdx.x; pc < kPieces; pc += kWarps * 32) {
+    const int mat = pc / (kNMax * kPPR), rem = pc % (kNMax * kPPR);
+    const int n = rem / kPPR, jj = rem % kPPR;
+    const int t = tb + jj * kPiece;
+    const T* src = (mat ? Cm : Bm) + ((size_t)b * N + (n < N ? n : 0)) * L;
+    T* dst = &sm.rawT[mat][n][jj * kPiece];
+    if (VEC) {
+      const bool ok = n < N && t < L;
+      cp_async_n<16>(dst, src + (ok ? t : 0), ok);
+    } else {
 #pragma unroll
-  for (int i = 1; i < 8; ++i) H = fmaf(a[i], H, bx[i]);
-  float P = Ploc;
-  warp_scan_fwd(P, H, lane);
-  const float hin = __shfl_sync(kFull, hck, n);
-  const float end = fmaf(P, hin, H);
-  float start = __shfl_up_sync(kFull, end, 1);
-  if (lane == 0) start = hin;
-  float2 hp[4], gy[4];
-  {
-    float h = start;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      hp[k].x = h = fmaf(a[2 * k], h, bx[2 * k]);
-      hp[k].y = h = fmaf(a[2 * k + 1], h, bx[2 * k + 1]);
-      y2[k] = ffma2(cp[k], hp[k], y2[k]);
-      gy[k] = fmul2(dyp[k], cp[k]);
+      for (int e = 0; e < kPiece; ++e)
+        dst[e] = (n < N && t + e < L) ? src[t + e] : from_f<T>(0.0f);
     }
   }
-  // adjoint: lane map c_in -> c_out = a_first * g_first
-  float Gl = gy[3].y;
-#pragma unroll
-  for (int i = 6; i >= 0; --i) Gl = fmaf(a[i + 1], Gl, (i & 1) ? gy[i >> 1].y : gy[i >> 1].x);
-  float Gc = a[0] * Gl;
-  float Pr = Ploc;
-  warp_scan_bwd(Pr, Gc, lane);
-  const float cc = __shfl_sync(kFull, gcarry, n);
-  const float cout = fmaf(Pr, cc, Gc);
-  float cin = __shfl_down_sync(kFull, cout, 1);
-  if (lane == 31) cin = cc;
-  const float ncar = __shfl_sync(kFull, cout, 0);
-  if (lane == n) gcarry = ncar;
-
-  // reverse replay, two tokens at a time: g for tokens 2k+1 and 2k, then
-  // every per-token product for that pair
-  const float2 minus1 = f2(-1.0f, -1.0f);
-  float2 dAp = f2(0.f, 0.f), dBp[4], dCp[4];
-  float g = gy[3].y + cin;
-#pragma unroll
-  for (int k = 3; k >= 0; --k) {
-    float2 gp;
-    gp.y = g;                                   // token 2k+1
-    gp.x = fmaf(a[2 * k + 1], g, gy[k].x);      // token 2k
-    if (k > 0) g = fmaf(a[2 * k], gp.x, gy[k - 1].y);  // token 2k-1
-    // a_t h_{t-1} = h_t - B_t dt_t u_t (the forward step without its input)
-    const float2 ahp = ffma2(f2(bx[2 * k], bx[2 * k + 1]), minus1, hp[k]);
-    const float2 q = fmul2(gp, ahp);
-    dAp = ffma2(dlp[k], q, dAp);
-    dd2[k] = ffma2(f2(Anat, Anat), q, dd2[k]);
-    sgB2[k] = ffma2(gp, bp[k], sgB2[k]);
-    dBp[k] = fmul2(gp, xup[k]);
-    dCp[k] = fmul2(dyp[k], hp[k]);
+  const int t = tb + 2 * j;
+  for (int a = 0; a < n_arrays; ++a) {
+    const T* src = static_cast<const T*>(rp.p[a]);
+    T* dst = &sm.rawR[a][r][2 * j];
+    if (VEC) {
+      const bool ok = active && t < L;
+      cp_async_n<2 * sizeof(T)>(dst, src + (ok ? t : 0), ok);
+    } else {
+      dst[0] = (active && t < L) ? src[t] : from_f<T>(0.0f);
+      dst[1] = (active && t + 1 < L) ? src[t + 1] : from_f<T>(0.0f);
+    }
   }
-  mysl[lane] = make_float4(dBp[0].x, dBp[0].y, dBp[1].x, dBp[1].y);
-  mysl[32 + lane] = make_float4(dBp[2].x, dBp[2].y, dBp[3].x, dBp[3].y);
-  mysl[64 + lane] = make_float4(dCp[0].x, dCp[0].y, dCp[1].x, dCp[1].y);
-  mysl[96 + lane] = make_float4(dCp[2].x, dCp[2].y, dCp[3].x, dCp[3].y);
-  sdA_n[lane] += dAp.x + dAp.y;
+  if (VEC) cp_async_commit();
 }
 
-// Sum the G warps' slices of state n (parity n & 1) and add them to dB / dC
-// (one float4 = 4 tokens per thread; `dst` points at this thread's 4 tokens
-// of state 0 in dB or dC, `L` apart per state).
-template <int G, bool VEC>
-__device__ __forceinline__ void bwd_reduce(int n, const float4 (*slice)[G][2][64], int m, int q,
-                                           float* dst, int L, bool valid4, int tleft) {
-  const float4* sl = &slice[n & 1][0][m][q];
-  float4 s = sl[0];
-#pragma unroll
-  for (int w = 1; w < G; ++w) {
-    const float4 v = sl[w * 128];
-    const float2 lo = __fadd2_rn(f2(s.x, s.y), f2(v.x, v.y));
-    const float2 hi = __fadd2_rn(f2(s.z, s.w), f2(v.z, v.w));
-    s = make_float4(lo.x, lo.y, hi.x, hi.y);
-  }
-  float* d = dst + (size_t)n * L;
-  if (VEC) {
-    if (valid4) atomicAdd(reinterpret_cast<float4*>(d), s);
-  } else {
-    if (tleft > 0) atomicAdd(d, s.x);
-    if (tleft > 1) atomicAdd(d + 1, s.y);
-    if (tleft > 2) atomicAdd(d + 2, s.z);
-    if (tleft > 3) atomicAdd(d + 3, s.w);
-  }
-}
-
-// NT: state count fixed at compile time (16), or 0 for any N <= 16.
-template <typename T, int G, bool VEC, int NT>
-__global__ void __launch_bounds__(G * 32, SSM_BWD_MIN_BLOCKS)
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(kWarps * 32, SSM_BWD_MIN_BLOCKS)
 scan_bwd_kernel(const ScanArgs p) {
-  // bf16 on the vector path: B / C tiles arrive by cp.async one chunk ahead
-  // (per-thread 16-byte copies; on this kernel, with a CTA barrier per state,
-  // they measured faster than warp-issued TMA bulk copies)
-  constexpr bool ASYNC = VEC && sizeof(T) == 2;
   extern __shared__ float4 smem_dyn[];
-  BwdSmem<G>& sm = *reinterpret_cast<BwdSmem<G>*>(smem_dyn);
+  BwdSmem<T>& sm = *reinterpret_cast<BwdSmem<T>*>(smem_dyn);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hf = lane >> 4;   // which of the warp's two rows
+  const int n = lane & 15;    // state; in the per-token phases, tokens 2n and 2n + 1
+  const int r = 2 * warp + hf;
   const int b = blockIdx.y;
-  const int d = blockIdx.x * G + warp;
+  const int d = blockIdx.x * kRows + r;
   const bool active = d < p.D;
   const int split = blockIdx.z;
-  const int N = NT ? NT : p.N, L = p.L;
-  const int c_begin = split * p.chunks_per_split;
-  const int c_end = min(c_begin + p.chunks_per_split, p.nchunks);
+  const int N = p.N, L = p.L;
+  const bool nval = active && n < N;
+  const int t_begin = split * p.chunks_per_split * kChunk;
+  const int t_end = min((split + 1) * p.chunks_per_split * kChunk, L);
   const size_t rowid = (size_t)b * p.D + (active ? d : 0);
   const size_t row = rowid * L;
+  const size_t nblk = (size_t)p.nchunks * (kChunk / kBlk);
+  const bool has_z = p.z != nullptr;
 
   const T* Bm = static_cast<const T*>(p.Bm);
   const T* Cm = static_cast<const T*>(p.Cm);
-  const T* u_row = static_cast<const T*>(p.u) + row;
-  const T* dl_row = static_cast<const T*>(p.delta) + row;
-  const T* z_row = p.z ? static_cast<const T*>(p.z) + row : nullptr;
-  const T* go_row = static_cast<const T*>(p.dout) + row;
+  RowPtrs rp;
+  rp.p[0] = static_cast<const T*>(p.delta) + row;
+  rp.p[1] = static_cast<const T*>(p.u) + row;
+  rp.p[2] = static_cast<const T*>(p.dout) + row;
+  rp.p[3] = has_z ? static_cast<const T*>(p.z) + row : nullptr;
+  rp.p[4] = has_z ? static_cast<const T*>(p.ysave) + row : nullptr;
+  const int n_arrays = has_z ? 5 : 3;
+  const int32_t* seqb = p.seq ? p.seq + (size_t)b * L : nullptr;
 
-  const float A_lane = (active && lane < N) ? __ldg(p.A + (size_t)d * N + lane) : 0.0f;
-  const float A2_lane = A_lane * kLog2e;
+  const float An = nval ? __ldg(p.A + (size_t)d * N + n) : 0.0f;
+  const float2 A2 = f2(An * kLog2e, An * kLog2e);
+  const float2 Ap = f2(An, An);
   const float Dv = (active && p.Dskip) ? __ldg(p.Dskip + d) : 0.0f;
   const float bias = (active && p.delta_bias) ? __ldg(p.delta_bias + d) : 0.0f;
-  // lane n holds c_n = a g of the first token after the current chunk
-  float gcarry = 0.0f;
-  if (split + 1 < p.nsplits && active && lane < N)
-    gcarry = p.split_in[(rowid * p.nsplits + split) * p.Npad + lane];
-
-  {
-    float4* s = &sm.slice[0][0][0][0];
-    for (int i = threadIdx.x; i < 2 * G * 2 * 64; i += blockDim.x) s[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int n = 0; n < kNMax; ++n) sm.dA[warp][n][lane] = 0.0f;
-  }
+  // a_{t+1} g_{t+1} for the first token after the current block
+  float Gn = 0.0f;
+  if (split + 1 < p.nsplits && nval) Gn = p.split_in[(rowid * p.nsplits + split) * p.Npad + n];
+  float2 dA2 = f2(0.0f, 0.0f);
   float dDp = 0.0f, ddbp = 0.0f;
 
-  if (ASYNC)
-    issue_bc_raw(reinterpret_cast<const __nv_bfloat16*>(Bm), reinterpret_cast<const __nv_bfloat16*>(Cm),
-                 &sm.raw[0][0][0], 2, b, N, L, (c_end - 1) * kChunk);
-  Tok8<T, VEC> pf_dl, pf_u, pf_z, pf_go;
-  if (active) {
-    const int tl = (c_end - 1) * kChunk + lane * 8;
-    pf_dl.load(dl_row, tl, L);
-    pf_u.load(u_row, tl, L);
-    pf_go.load(go_row, tl, L);
-    if (z_row) pf_z.load(z_row, tl, L);
-  }
+  // per-block values carried from the staging of a block to its processing
+  float ck_issued = 0.0f, ck_ready = 0.0f;   // checkpoint h entering the block (state n)
+  int sq_cur = 0, sq_prev = 0;               // seq_idx of token tb + lane and the one before
+  unsigned rm_ready = 0u;                    // document starts inside the block
+  float e_u[2], e_dt[2], e_dy[2], e_dsp[2];  // per-token values of tokens 2n, 2n + 1
 
-  for (int c = c_end - 1; c >= c_begin; --c) {
-    const int t0 = c * kChunk;
-    if (ASYNC) {
-      cp_async_wait_all();
-      __syncthreads();  // the previous chunk's readers of B / C are done
-      convert_bc_rows(&sm.raw[0][0][0], sm.B, sm.C, 2, N, L - t0);
-      if (c - 1 >= c_begin)  // each thread refills only the pieces it just converted
-        issue_bc_raw(reinterpret_cast<const __nv_bfloat16*>(Bm),
-                     reinterpret_cast<const __nv_bfloat16*>(Cm), &sm.raw[0][0][0], 2, b, N, L,
-                     t0 - kChunk);
-      __syncthreads();
-    } else {
-      __syncthreads();
-      stage_rows<T, VEC>(Bm, sm.B, b, N, L, t0);
-      stage_rows<T, VEC>(Cm, sm.C, b, N, L, t0);
-      __syncthreads();
+  auto prefetch = [&](int kb) {
+    const int tb = t_begin + kb * kBlk;
+    issue_block<T, VEC>(sm, Bm, Cm, rp, n_arrays, b, N, L, tb, r, n, active);
+    if (nval) ck_issued = __ldg(p.ckpt + (rowid * nblk + tb / kBlk) * kNMax + n);
+    if (seqb) {
+      const int t = tb + lane;
+      sq_cur = t < L ? __ldg(seqb + t) : 0;
+      sq_prev = (t > 0 && t < L) ? __ldg(seqb + t - 1) : sq_cur;
     }
-
-    const int tl = t0 + lane * 8;
-    float2 dlp[4], xup[4], dyp[4];
-    float Sdl = 0.0f;
-    unsigned rmask = 0u;
-    float hck = 0.0f;
-    if (active) {
-      float dl[8], uu[8], go[8], zz[8];
-      pf_dl.get(dl);
-      pf_u.get(uu);
-      pf_go.get(go);
-      if (z_row) pf_z.get(zz);
-      if (c - 1 >= c_begin) {  // previous chunk's inputs, consumed next iteration
-        pf_dl.load(dl_row, tl - kChunk, L);
-        pf_u.load(u_row, tl - kChunk, L);
-        pf_go.load(go_row, tl - kChunk, L);
-        if (z_row) pf_z.load(z_row, tl - kChunk, L);
-      }
-      float dt[8], dy[8];
+  };
+  // the thread's own raw pieces of block kb -> fp32 tiles and per-token arrays
+  auto convert = [&](int kb) {
+    const int tb = t_begin + kb * kBlk;
+    if (VEC) cp_async_wait_all();
+    constexpr int kPiece = 16 / (int)sizeof(T);
+    constexpr int kPPR = kBlk / kPiece;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float v = dl[i] + bias;
-        const float s = p.softplus ? softplus_sfu(v) : v;
-        dt[i] = (tl + i < L) ? s : 0.0f;
-        Sdl += dt[i];
-        dy[i] = z_row ? go[i] * (zz[i] * sigmoid_fast(zz[i])) : go[i];
-      }
+    for (int pc = threadIdx.x; pc < 2 * kNMax * kPPR; pc += kWarps * 32) {
+      const int mat = pc / (kNMax * kPPR), rem = pc % (kNMax * kPPR);
+      const int nn = rem / kPPR, jj = rem % kPPR;
+      float* dst = mat ? &sm.C[nn][jj * kPiece] : &sm.B[nn][jj * kPiece];
+      const T* src = &sm.rawT[mat][nn][jj * kPiece];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        dlp[k] = f2(dt[2 * k], dt[2 * k + 1]);
-        xup[k] = f2(dt[2 * k] * uu[2 * k], dt[2 * k + 1] * uu[2 * k + 1]);
-        dyp[k] = f2(dy[2 * k], dy[2 * k + 1]);
-      }
-      rmask = reset_mask(p.seq, b, L, tl);
-      if (lane < N) hck = p.ckpt[(rowid * p.nchunks + c) * p.Npad + lane];
+      for (int e = 0; e < kPiece; e += 4)
+        *reinterpret_cast<float4*>(dst + e) =
+            make_float4(to_f(src[e]), to_f(src[e + 1]), to_f(src[e + 2]), to_f(src[e + 3]));
     }
-    const bool any_reset = __any_sync(kFull, rmask != 0u);
-
-    float2 y2[4], sgB2[4], dd2[4];
+    const int t = tb + 2 * n;
+    float dt[2], xu[2], dy[2], dz[2];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      y2[k] = f2(0.f, 0.f);
-      sgB2[k] = f2(0.f, 0.f);
-      dd2[k] = f2(0.f, 0.f);
-    }
-
-    // this thread's share of the per-state dB / dC reduction: item (m, q)
-    const int rm = threadIdx.x >> 6, rq = threadIdx.x & 63;  // blockDim = 128 = 2 x 64 items
-    const int rt = t0 + (rq & 31) * 8 + (rq >> 5) * 4;
-    float* rdst = (rm ? p.dC : p.dB) + (size_t)b * N * L + rt;
-    const bool rvalid = rt < L;
-    const int rleft = L - rt;
-    if (NT) {  // compile-time state count: fully unrolled, immediate offsets
-#pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        if (active)
-          bwd_state(n, lane, sm.B, sm.C, &sm.slice[n & 1][warp][0][0], &sm.dA[warp][n][0], A_lane,
-                    A2_lane, hck, gcarry, dlp, xup, dyp, Sdl, rmask, any_reset, y2, sgB2, dd2);
-        __syncthreads();
-        bwd_reduce<G, VEC>(n, sm.slice, rm, rq, rdst, L, rvalid, rleft);
+    for (int e = 0; e < 2; ++e) {
+      const bool in = active && t + e < L;
+      const float dl = to_f(sm.rawR[0][r][2 * n + e]);
+      const float uu = to_f(sm.rawR[1][r][2 * n + e]);
+      const float go = to_f(sm.rawR[2][r][2 * n + e]);
+      const float v = dl + bias;
+      const float s = p.softplus ? softplus_sfu(v) : v;
+      dt[e] = in ? s : 0.0f;
+      xu[e] = dt[e] * uu;
+      float gate = 1.0f;
+      dz[e] = 0.0f;
+      if (has_z) {
+        const float zz = to_f(sm.rawR[3][r][2 * n + e]);
+        const float yv = to_f(sm.rawR[4][r][2 * n + e]);
+        const float sz = sigmoid_fast(zz);
+        gate = zz * sz;
+        dz[e] = go * yv * (sz * (1.0f + zz * (1.0f - sz)));
       }
-    } else {
+      dy[e] = in ? go * gate : 0.0f;
+      if (in) dDp = fmaf(dy[e], uu, dDp);
+      e_u[e] = uu;
+      e_dt[e] = dt[e];
+      e_dy[e] = dy[e];
+      // d softplus(v) / dv = sigmoid(v)
+      e_dsp[e] = p.softplus ? (v > 20.0f ? 1.0f : sigmoid_fast(v)) : 1.0f;
+    }
+    *reinterpret_cast<float2*>(&sm.dt[r][2 * n]) = f2(dt[0], dt[1]);
+    *reinterpret_cast<float2*>(&sm.xu[r][2 * n]) = f2(xu[0], xu[1]);
+    *reinterpret_cast<float2*>(&sm.dy[r][2 * n]) = f2(dy[0], dy[1]);
+    if (has_z && active) store2<T, VEC>(static_cast<T*>(p.dz) + row, t, L, dz[0], dz[1]);
+    ck_ready = ck_issued;
+    rm_ready = seqb ? __ballot_sync(kFull, tb + lane < L && tb + lane > 0 && sq_cur != sq_prev) : 0u;
+  };
+
+  const int nb = (t_end - t_begin + kBlk - 1) / kBlk;
+  prefetch(nb - 1);
+  convert(nb - 1);
+  if (nb >= 2) prefetch(nb - 2);
+
+  float* Xg = &sm.X[warp][0][hf][n][0];
+  float* Xa = &sm.X[warp][1][hf][n][0];
+  const float4* dt4 = reinterpret_cast<const float4*>(&sm.dt[r][0]);
+  const float4* xu4 = reinterpret_cast<const float4*>(&sm.xu[r][0]);
+  const float4* dy4 = reinterpret_cast<const float4*>(&sm.dy[r][0]);
+  const float4* B4 = reinterpret_cast<const float4*>(&sm.B[n][0]);
+  const float4* C4 = reinterpret_cast<const float4*>(&sm.C[n][0]);
+
 #pragma unroll 1
-      for (int n = 0; n < N; ++n) {
-        if (active)
-          bwd_state(n, lane, sm.B, sm.C, &sm.slice[n & 1][warp][0][0], &sm.dA[warp][n][0], A_lane,
-                    A2_lane, hck, gcarry, dlp, xup, dyp, Sdl, rmask, any_reset, y2, sgB2, dd2);
-        __syncthreads();
-        bwd_reduce<G, VEC>(n, sm.slice, rm, rq, rdst, L, rvalid, rleft);
+  for (int kb = nb - 1; kb >= 0; --kb) {
+    const int tb = t_begin + kb * kBlk;
+    __syncthreads();  // block kb's tiles and per-token arrays are complete; X is free
+    const float hck = ck_ready;
+    const unsigned rm = rm_ready;
+
+    // forward recompute of h over the block from its checkpoint
+    float4 H4[kBlk / 4];
+    {
+      float hh = hck;
+#pragma unroll
+      for (int q = 0; q < kBlk / 4; ++q) {
+        const float4 dq = dt4[q], xq = xu4[q], bq = B4[q];
+        const float2 e0 = fmul2(f2(dq.x, dq.y), A2), e1 = fmul2(f2(dq.z, dq.w), A2);
+        float a0 = ex2_approx(e0.x), a1 = ex2_approx(e0.y);
+        float a2 = ex2_approx(e1.x), a3 = ex2_approx(e1.y);
+        if (rm) {
+          const unsigned m4 = rm >> (4 * q);
+          if (m4 & 1u) a0 = 0.0f;
+          if (m4 & 2u) a1 = 0.0f;
+          if (m4 & 4u) a2 = 0.0f;
+          if (m4 & 8u) a3 = 0.0f;
+        }
+        const float2 b0 = fmul2(f2(xq.x, xq.y), f2(bq.x, bq.y));
+        const float2 b1 = fmul2(f2(xq.z, xq.w), f2(bq.z, bq.w));
+        H4[q].x = hh = fmaf(a0, hh, b0.x);
+        H4[q].y = hh = fmaf(a1, hh, b0.y);
+        H4[q].z = hh = fmaf(a2, hh, b1.x);
+        H4[q].w = hh = fmaf(a3, hh, b1.y);
       }
     }
 
-    if (active) {
-      // this chunk's u, raw delta, dout, z again (L2-resident since the prefetch)
-      float uu[8], dl[8], go[8], zz[8];
-      load_row8<T, VEC>(u_row, tl, L, uu);
-      load_row8<T, VEC>(dl_row, tl, L, dl);
-      load_row8<T, VEC>(go_row, tl, L, go);
-      if (z_row) load_row8<T, VEC>(z_row, tl, L, zz);
-      float o_du[8], o_dd[8], o_dz[8];
+    // adjoint backwards over the block, g_t = dy_t C_t + a_{t+1} g_{t+1}
+    // (a recomputed), with q_t = g_t a_t h_{t-1} and this state's terms of
+    // the per-token sums
+    float4 G4[kBlk / 4];
+    {
+      float gnext = Gn, anext = 1.0f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int k = i >> 1;
-        const float sg = (i & 1) ? sgB2[k].y : sgB2[k].x;
-        const float dsum = (i & 1) ? dd2[k].y : dd2[k].x;
-        const float yv = (i & 1) ? y2[k].y : y2[k].x;
-        const float dt = (i & 1) ? dlp[k].y : dlp[k].x;
-        const float dyi = (i & 1) ? dyp[k].y : dyp[k].x;
-        const bool in = tl + i < L;
-        o_du[i] = fmaf(dyi, Dv, dt * sg);
-        const float ddt = fmaf(uu[i], sg, dsum);
-        // softplus'(v) = e^v / (1 + e^v)
-        const float v = dl[i] + bias;
-        const float ev = __expf(v);
-        const float dv = p.softplus ? ddt * (v > 20.0f ? 1.0f : __fdividef(ev, 1.0f + ev)) : ddt;
-        o_dd[i] = dv;
-        if (z_row) {
-          const float yfull = fmaf(Dv, uu[i], yv);
-          const float sz = sigmoid_fast(zz[i]);
-          o_dz[i] = go[i] * yfull * (sz * (1.0f + zz[i] * (1.0f - sz)));
+      for (int q = kBlk / 4 - 1; q >= 0; --q) {
+        const float4 yq = dy4[q], cq = C4[q], dq = dt4[q], bq = B4[q];
+        const float2 gy0 = fmul2(f2(yq.x, yq.y), f2(cq.x, cq.y));
+        const float2 gy1 = fmul2(f2(yq.z, yq.w), f2(cq.z, cq.w));
+        const float2 e0 = fmul2(f2(dq.x, dq.y), A2), e1 = fmul2(f2(dq.z, dq.w), A2);
+        float a0 = ex2_approx(e0.x), a1 = ex2_approx(e0.y);
+        float a2 = ex2_approx(e1.x), a3 = ex2_approx(e1.y);
+        if (rm) {
+          const unsigned m4 = rm >> (4 * q);
+          if (m4 & 1u) a0 = 0.0f;
+          if (m4 & 2u) a1 = 0.0f;
+          if (m4 & 4u) a2 = 0.0f;
+          if (m4 & 8u) a3 = 0.0f;
         }
-        if (in) {
-          dDp = fmaf(dyi, uu[i], dDp);
-          ddbp += dv;
+        const float g3 = fmaf(anext, gnext, gy1.y);
+        const float g2 = fmaf(a3, g3, gy1.x);
+        const float g1 = fmaf(a2, g2, gy0.y);
+        const float g0 = fmaf(a1, g1, gy0.x);
+        anext = a0;
+        gnext = g0;
+        G4[q] = make_float4(g0, g1, g2, g3);
+        const float hp = q ? H4[q - 1].w : hck;
+        const float2 q0 = fmul2(f2(g0, g1), f2(a0 * hp, a1 * H4[q].x));
+        const float2 q1 = fmul2(f2(g2, g3), f2(a2 * H4[q].y, a3 * H4[q].z));
+        dA2 = ffma2(f2(dq.x, dq.y), q0, dA2);
+        dA2 = ffma2(f2(dq.z, dq.w), q1, dA2);
+        const float2 gb0 = fmul2(f2(g0, g1), f2(bq.x, bq.y));
+        const float2 gb1 = fmul2(f2(g2, g3), f2(bq.z, bq.w));
+        const float2 aq0 = fmul2(Ap, q0), aq1 = fmul2(Ap, q1);
+        reinterpret_cast<float4*>(Xg)[q] = make_float4(gb0.x, gb0.y, gb1.x, gb1.y);
+        reinterpret_cast<float4*>(Xa)[q] = make_float4(aq0.x, aq0.y, aq1.x, aq1.y);
+      }
+      Gn = anext * gnext;
+    }
+    __syncwarp();
+    // sums over the states for tokens 2n, 2n + 1 of row r
+    float2 sg, sq;
+    {
+      float2 s1a = f2(0.0f, 0.0f), s1b = s1a, s2a = s1a, s2b = s1a;
+#pragma unroll
+      for (int m = 0; m < kNMax; m += 2) {
+        s1a = __fadd2_rn(s1a, *reinterpret_cast<const float2*>(&sm.X[warp][0][hf][m][2 * n]));
+        s1b = __fadd2_rn(s1b, *reinterpret_cast<const float2*>(&sm.X[warp][0][hf][m + 1][2 * n]));
+        s2a = __fadd2_rn(s2a, *reinterpret_cast<const float2*>(&sm.X[warp][1][hf][m][2 * n]));
+        s2b = __fadd2_rn(s2b, *reinterpret_cast<const float2*>(&sm.X[warp][1][hf][m + 1][2 * n]));
+      }
+      sg = __fadd2_rn(s1a, s1b);
+      sq = __fadd2_rn(s2a, s2b);
+    }
+    __syncwarp();
+    // this row's dB_t = g_t dt_t u_t and dC_t = dy_t h_t
+#pragma unroll
+    for (int q = 0; q < kBlk / 4; ++q) {
+      const float4 xq = xu4[q], yq = dy4[q];
+      const float2 db0 = fmul2(f2(G4[q].x, G4[q].y), f2(xq.x, xq.y));
+      const float2 db1 = fmul2(f2(G4[q].z, G4[q].w), f2(xq.z, xq.w));
+      const float2 dc0 = fmul2(f2(yq.x, yq.y), f2(H4[q].x, H4[q].y));
+      const float2 dc1 = fmul2(f2(yq.z, yq.w), f2(H4[q].z, H4[q].w));
+      reinterpret_cast<float4*>(Xg)[q] = make_float4(db0.x, db0.y, db1.x, db1.y);
+      reinterpret_cast<float4*>(Xa)[q] = make_float4(dc0.x, dc0.y, dc1.x, dc1.y);
+    }
+    __syncthreads();  // every row's dB / dC terms are in X; tiles and per-token arrays are free
+    // CTA sum over its 8 rows; one float4 atomic per 4 tokens of dB / dC
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int item = threadIdx.x + it * (kWarps * 32);
+      const int arr = item >> 7, m = (item >> 3) & 15, q = item & 7;
+      float4 v[2 * kWarps];
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        v[2 * w] = *reinterpret_cast<const float4*>(&sm.X[w][arr][0][m][4 * q]);
+        v[2 * w + 1] = *reinterpret_cast<const float4*>(&sm.X[w][arr][1][m][4 * q]);
+      }
+#pragma unroll
+      for (int s = 1; s < 2 * kWarps; s <<= 1)
+#pragma unroll
+        for (int i = 0; i + s < 2 * kWarps; i += 2 * s) {
+          const float2 lo = __fadd2_rn(f2(v[i].x, v[i].y), f2(v[i + s].x, v[i + s].y));
+          const float2 hi = __fadd2_rn(f2(v[i].z, v[i].w), f2(v[i + s].z, v[i + s].w));
+          v[i] = make_float4(lo.x, lo.y, hi.x, hi.y);
+        }
+      const int t = tb + 4 * q;
+      if (m < N && t < L) {
+        float* dst = (arr ? p.dC : p.dB) + ((size_t)b * N + m) * L + t;
+        if (VEC) {
+          atomicAdd(reinterpret_cast<float4*>(dst), v[0]);
+        } else {
+          const int left = L - t;
+          atomicAdd(dst, v[0].x);
+          if (left > 1) atomicAdd(dst + 1, v[0].y);
+          if (left > 2) atomicAdd(dst + 2, v[0].z);
+          if (left > 3) atomicAdd(dst + 3, v[0].w);
         }
       }
-      store_row8<T, VEC>(static_cast<T*>(p.du) + row, tl, L, o_du);
-      store_row8<T, VEC>(static_cast<T*>(p.ddelta) + row, tl, L, o_dd);
-      if (z_row) store_row8<T, VEC>(static_cast<T*>(p.dz) + row, tl, L, o_dz);
+    }
+    // per-token outputs of tokens 2n, 2n + 1 of row r
+    {
+      const int t = tb + 2 * n;
+      float du[2], dd[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float s1 = e ? sg.y : sg.x, s2 = e ? sq.y : sq.x;
+        du[e] = fmaf(e_dy[e], Dv, e_dt[e] * s1);
+        dd[e] = fmaf(e_u[e], s1, s2) * e_dsp[e];
+        if (active && t + e < L) ddbp += dd[e];
+      }
+      if (active) {
+        store2<T, VEC>(static_cast<T*>(p.du) + row, t, L, du[0], du[1]);
+        store2<T, VEC>(static_cast<T*>(p.ddelta) + row, t, L, dd[0], dd[1]);
+      }
+    }
+    if (kb >= 1) {
+      convert(kb - 1);
+      if (kb >= 2) prefetch(kb - 2);
     }
   }
 
-  if (!active) return;
+  // per-(row, split) partials of dA, dD and the delta-bias gradient
+  const size_t ps = rowid * p.nsplits + split;
+  if (nval) p.part_dA[ps * N + n] = dA2.x + dA2.y;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
+  for (int off = 8; off > 0; off >>= 1) {
     dDp += __shfl_xor_sync(kFull, dDp, off);
     ddbp += __shfl_xor_sync(kFull, ddbp, off);
   }
-  __syncwarp();
-  const size_t ps = rowid * p.nsplits + split;
-  if (lane < N) {
-    float s = 0.0f;
-    for (int j = 0; j < 32; ++j) s += sm.dA[warp][lane][j];
-    p.part_dA[ps * N + lane] = s;
-  }
-  if (lane == 0) {
+  if (active && n == 0) {
     p.part_dD[ps] = dDp;
     p.part_ddb[ps] = ddbp;
   }
@@ -519,26 +590,27 @@ __global__ void bwd_param_reduce_kernel(const float* __restrict__ pA, const floa
   }
 }
 
-template <typename T, int G, bool VEC, int NT>
+template <typename T, bool VEC>
 cudaError_t bwd_t(const ScanArgs& a, cudaStream_t s) {
-  dim3 block(G * 32);
   if (a.nsplits > 1) {
+    // adjoint carry into each split from the right (lanes-over-time summary)
+    constexpr int G = 4;
     dim3 g1((a.D + G - 1) / G, a.B, a.nsplits - 1);
-    scan_bwd_summary_kernel<T, G, VEC><<<g1, block, 0, s>>>(a);
+    scan_bwd_summary_kernel<T, G, VEC><<<g1, G * 32, 0, s>>>(a);
     const int n = a.B * a.D * a.Npad;
     bwd_split_carry_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.split_P, a.split_H, a.split_in,
                                                           a.B * a.D, a.nsplits, a.Npad);
   }
-  const size_t smem = sizeof(BwdSmem<G>);
+  const size_t smem = sizeof(BwdSmem<T>);
   static bool smem_set = false;  // once per instantiation and process (a benign race)
   if (!smem_set) {
-    cudaError_t e = cudaFuncSetAttribute(scan_bwd_kernel<T, G, VEC, NT>,
+    cudaError_t e = cudaFuncSetAttribute(scan_bwd_kernel<T, VEC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     smem_set = true;
   }
-  dim3 g2((a.D + G - 1) / G, a.B, a.nsplits);
-  scan_bwd_kernel<T, G, VEC, NT><<<g2, block, smem, s>>>(a);
+  dim3 g2((a.D + kRows - 1) / kRows, a.B, a.nsplits);
+  scan_bwd_kernel<T, VEC><<<g2, kWarps * 32, smem, s>>>(a);
   const int m = a.D * a.N > a.D ? a.D * a.N : a.D;
   bwd_param_reduce_kernel<<<(m + 255) / 256, 256, 0, s>>>(a.part_dA, a.part_dD, a.part_ddb, a.dA,
                                                          a.dD, a.ddelta_bias, a.B, a.D, a.N,
@@ -548,17 +620,9 @@ cudaError_t bwd_t(const ScanArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-template <int NT>
-cudaError_t bwd_dispatch(const ScanArgs& a, cudaStream_t s) {
-  if (a.bf16)
-    return a.vec ? bwd_t<__nv_bfloat16, 4, true, NT>(a, s) : bwd_t<__nv_bfloat16, 4, false, NT>(a, s);
-  return a.vec ? bwd_t<float, 4, true, NT>(a, s) : bwd_t<float, 4, false, NT>(a, s);
-}
-
 cudaError_t launch_scan_bwd(const ScanArgs& a, cudaStream_t s) {
-  // the runtime state loop: fully unrolling 16 states overflows the
-  // instruction cache and spills more (measured slower)
-  return bwd_dispatch<0>(a, s);
+  if (a.bf16) return a.vec ? bwd_t<__nv_bfloat16, true>(a, s) : bwd_t<__nv_bfloat16, false>(a, s);
+  return a.vec ? bwd_t<float, true>(a, s) : bwd_t<float, false>(a, s);
 }
 
 }  // namespace ssm

@@ -67,7 +67,8 @@ __device__ __forceinline__ void fwd_pair_pre(int m, int lane, const float2* __re
 template <bool SUMMARY>
 __device__ __forceinline__ void fwd_pair_post(int m, int lane, const float2* __restrict__ sCt,
                                               float2* sH, float2* sP, const float2 a[8],
-                                              const float2 bx[8], float2 y2[8]) {
+                                              const float2 bx[8], float2 y2[8],
+                                              float2* __restrict__ ck32) {
   float2 P = a[0], H = bx[0];
 #pragma unroll
   for (int i = 1; i < 8; ++i) {
@@ -84,6 +85,8 @@ __device__ __forceinline__ void fwd_pair_post(int m, int lane, const float2* __r
     if (SUMMARY) sP[m] = fmul2(sP[m], P);
   }
   if (!SUMMARY) {
+    // every fourth lane starts a 32-token block: keep its entering state
+    if ((lane & 3) == 0) ck32[(lane >> 2) * (kNMax / 2) + m] = start;
     float2 cv[8];
     lds_pair8(sCt + m * kChunk, lane, cv);
     float2 h = start;
@@ -200,8 +203,8 @@ scan_fwd_kernel(const ScanArgs p) {
     const unsigned rmask = reset_mask(p.seq, b, L, tl);
     const bool any_reset = __any_sync(kFull, rmask != 0u);
 
-    if (!SUMMARY && lane < NP)
-      reinterpret_cast<float2*>(p.ckpt)[(rowid * p.nchunks + c) * NP + lane] = sm.H[warp][lane];
+    // 32-token checkpoints of this chunk: [row][c * 8 + k][kNMax] fp32 pairs
+    float2* ck32 = reinterpret_cast<float2*>(p.ckpt) + (rowid * p.nchunks + c) * 8 * (kNMax / 2);
 
     if (NT) {
       // compile-time state count: fully unrolled and software-pipelined (the
@@ -213,7 +216,7 @@ scan_fwd_kernel(const ScanArgs p) {
         float2 a1[8], b1[8];
         if (m + 1 < (NT + 1) / 2)
           fwd_pair_pre(m + 1, lane, sm.B, sm.A[warp][m + 1], dd, xx, rmask, any_reset, a1, b1);
-        fwd_pair_post<SUMMARY>(m, lane, sm.C, sm.H[warp], sm.P[warp], a0, b0, y2);
+        fwd_pair_post<SUMMARY>(m, lane, sm.C, sm.H[warp], sm.P[warp], a0, b0, y2, ck32);
         if (m + 1 < (NT + 1) / 2) {
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -227,18 +230,20 @@ scan_fwd_kernel(const ScanArgs p) {
       for (int m = 0; m < NP; ++m) {
         float2 a0[8], b0[8];
         fwd_pair_pre(m, lane, sm.B, sm.A[warp][m], dd, xx, rmask, any_reset, a0, b0);
-        fwd_pair_post<SUMMARY>(m, lane, sm.C, sm.H[warp], sm.P[warp], a0, b0, y2);
+        fwd_pair_post<SUMMARY>(m, lane, sm.C, sm.H[warp], sm.P[warp], a0, b0, y2, ck32);
       }
     }
 
     if (!SUMMARY) {
-      float o[8];
+      float o[8], yv[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float yy = y2[i].x + y2[i].y;
-        o[i] = z_row ? yy * (zz[i] * sigmoid_fast(zz[i])) : yy;
+        yv[i] = y2[i].x + y2[i].y;
+        o[i] = z_row ? yv[i] * (zz[i] * sigmoid_fast(zz[i])) : yv[i];
       }
       store_row8<T, VEC>(static_cast<T*>(p.out) + row, tl, L, o);
+      // y before the gate, for the backward's dz
+      if (z_row) store_row8<T, VEC>(static_cast<T*>(p.ysave) + row, tl, L, yv);
     }
   }
 

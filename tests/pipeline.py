@@ -61,6 +61,8 @@ def gpu_layer(dv, *, n_splits=0, use_z=True, use_seq=True, softplus=True, final_
     out, fs, ws = ssm.scan_fwd(u, dv["delta"], dv["A"], dv["Bm"], dv["Cm"], z=z,
                                Dskip=dv["Dskip"], delta_bias=dv["delta_bias"], softplus=softplus,
                                seq_idx=seq, n_splits=n_splits, return_final_state=final_state)
+    # the forward's bounded tile waits record a timeout in the status word
+    assert ssm.scan_status(u, dv["A"], ws) == 0
     g = ssm.scan_bwd(u, dv["delta"], dv["A"], dv["Bm"], dv["Cm"], dv["dout"], ws, z=z,
                      Dskip=dv["Dskip"], delta_bias=dv["delta_bias"], softplus=softplus,
                      seq_idx=seq, n_splits=n_splits)

@@ -31,13 +31,14 @@ def lib():
         L.oracle_round_bf16.argtypes = [dp, dp, sz]
         L.oracle_conv1d_fwd.argtypes = [dp, dp, dp, ip, dp, dp, i, i, i, i, i]
         L.oracle_conv1d_bwd.argtypes = [dp, dp, dp, ip, dp, dp, dp, dp, i, i, i, i, i]
-        L.oracle_scan_fwd.argtypes = [dp] * 8 + [i, ip, dp, dp, dp, i, i, i, i]
-        L.oracle_scan_bwd.argtypes = [dp] * 8 + [i, ip] + [dp] * 9 + [i, i, i, i]
-        L.oracle_scan_fwd_mt.argtypes = [dp] * 8 + [i, ip, dp, dp, dp, i, i, i, i, i]
-        L.oracle_scan_bwd_mt.argtypes = [dp] * 8 + [i, ip] + [dp] * 9 + [i, i, i, i, i]
+        L.oracle_scan_fwd.argtypes = [dp] * 8 + [i, ip, dp, dp, dp, dp, i, i, i, i]
+        L.oracle_scan_bwd.argtypes = [dp] * 8 + [i, ip] + [dp] * 11 + [i, i, i, i]
+        L.oracle_scan_fwd_mt.argtypes = [dp] * 8 + [i, ip, dp, dp, dp, dp, i, i, i, i, i]
+        L.oracle_scan_bwd_mt.argtypes = [dp] * 8 + [i, ip] + [dp] * 11 + [i, i, i, i, i]
+        L.oracle_decode_step.argtypes = [dp] * 11 + [i] + [dp] * 3 + [i, i, i, i]
         for f in ("oracle_round_bf16", "oracle_conv1d_fwd", "oracle_conv1d_bwd",
                   "oracle_scan_fwd", "oracle_scan_bwd", "oracle_scan_fwd_mt",
-                  "oracle_scan_bwd_mt"):
+                  "oracle_scan_bwd_mt", "oracle_decode_step"):
             getattr(L, f).restype = None
         _lib = L
     return _lib
@@ -104,22 +105,23 @@ def conv1d_bwd(x, w, bias, seq_idx, du, silu=True):
 
 
 def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None,
-             softplus=True, seq_idx=None, nthreads=1):
+             softplus=True, seq_idx=None, h0=None, nthreads=1):
     """Selective scan forward. Returns dict(out, y, final_state).
 
     u, delta, z: [B, D, L]; A: [D, N]; Bm, Cm: [B, N, L]; Dskip,
-    delta_bias: [D] or None; seq_idx: [B, L] or None.
+    delta_bias: [D] or None; seq_idx: [B, L] or None; h0: [B, D, N] state
+    before token 0, or None for zero.
     """
     u, delta, z, A = _f64(u), _f64(delta), _f64(z), _f64(A)
     Dskip, delta_bias, Bm, Cm = _f64(Dskip), _f64(delta_bias), _f64(Bm), _f64(Cm)
-    seq = _i32(seq_idx)
+    seq, h0 = _i32(seq_idx), _f64(h0)
     B, D, L = u.shape
     N = A.shape[1]
     out = np.empty_like(u)
     y = np.empty_like(u)
     fs = np.empty((B, D, N))
     args = [_d(u), _d(delta), _d(z), _d(A), _d(Dskip), _d(delta_bias), _d(Bm),
-            _d(Cm), int(softplus), _i(seq), _d(out), _d(y), _d(fs), B, D, L, N]
+            _d(Cm), int(softplus), _i(seq), _d(h0), _d(out), _d(y), _d(fs), B, D, L, N]
     if nthreads > 1:
         lib().oracle_scan_fwd_mt(*args, int(nthreads))
     else:
@@ -128,12 +130,13 @@ def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None,
 
 
 def scan_bwd(u, delta, A, Bm, Cm, dout, *, z=None, Dskip=None, delta_bias=None,
-             softplus=True, seq_idx=None, nthreads=1):
+             softplus=True, seq_idx=None, h0=None, nthreads=1):
     """Selective scan backward. Returns dict of gradients (fp64):
-    du, ddelta (w.r.t. the raw delta), dz, dA, dB, dC, dD, ddelta_bias."""
+    du, ddelta (w.r.t. the raw delta), dz, dA, dB, dC, dD, ddelta_bias and
+    dh0 (w.r.t. the state before token 0)."""
     u, delta, z, A = _f64(u), _f64(delta), _f64(z), _f64(A)
     Dskip, delta_bias, Bm, Cm = _f64(Dskip), _f64(delta_bias), _f64(Bm), _f64(Cm)
-    seq, dout = _i32(seq_idx), _f64(dout)
+    seq, dout, h0 = _i32(seq_idx), _f64(dout), _f64(h0)
     B, D, L = u.shape
     N = A.shape[1]
     du = np.empty_like(u)
@@ -144,15 +147,39 @@ def scan_bwd(u, delta, A, Bm, Cm, dout, *, z=None, Dskip=None, delta_bias=None,
     dC = np.empty((B, N, L))
     dD = np.empty(D)
     ddb = np.empty(D)
+    dh0 = np.empty((B, D, N))
     args = [_d(u), _d(delta), _d(z), _d(A), _d(Dskip), _d(delta_bias), _d(Bm),
-            _d(Cm), int(softplus), _i(seq), _d(dout), _d(du), _d(ddelta), _d(dz),
-            _d(dA), _d(dB), _d(dC), _d(dD), _d(ddb), B, D, L, N]
+            _d(Cm), int(softplus), _i(seq), _d(h0), _d(dout), _d(du), _d(ddelta), _d(dz),
+            _d(dA), _d(dB), _d(dC), _d(dD), _d(ddb), _d(dh0), B, D, L, N]
     if nthreads > 1:
         lib().oracle_scan_bwd_mt(*args, int(nthreads))
     else:
         lib().oracle_scan_bwd(*args)
     return {"du": du, "ddelta": ddelta, "dz": dz, "dA": dA, "dB": dB, "dC": dC,
-            "dD": dD, "ddelta_bias": ddb}
+            "dD": dD, "ddelta_bias": ddb, "dh0": dh0}
+
+
+def decode_step(x, conv_state, w, conv_bias, delta, Bt, Ct, A, h, *, z=None,
+                Dskip=None, delta_bias=None, softplus=True):
+    """One token of the recurrent form for every (b, d).
+
+    x, delta, z: [B, D]; conv_state: [B, D, W-1] (previous inputs, oldest
+    first); w: [D, W]; conv_bias, Dskip, delta_bias: [D] or None; Bt, Ct:
+    [B, N]; A: [D, N]; h: [B, D, N] state after the previous token.
+    Returns (out [B, D], u [B, D], new conv_state, new h); inputs unchanged.
+    """
+    x, w, cb, delta, z = _f64(x), _f64(w), _f64(conv_bias), _f64(delta), _f64(z)
+    Bt, Ct, A, Dskip, delta_bias = _f64(Bt), _f64(Ct), _f64(A), _f64(Dskip), _f64(delta_bias)
+    cs = np.array(conv_state, dtype=np.float64, order="C", copy=True)
+    hh = np.array(h, dtype=np.float64, order="C", copy=True)
+    B, D = x.shape
+    N, W = A.shape[1], w.shape[1]
+    out = np.empty((B, D))
+    u = np.empty((B, D))
+    lib().oracle_decode_step(_d(x), _d(cs), _d(w), _d(cb), _d(delta), _d(z), _d(Bt),
+                             _d(Ct), _d(A), _d(Dskip), _d(delta_bias), int(softplus),
+                             _d(hh), _d(out), _d(u), B, D, N, W)
+    return out, u, cs, hh
 
 
 def layer_fwd_bwd(inp, *, bf16_points: bool, softplus=True, nthreads=1):
@@ -183,4 +210,4 @@ def layer_fwd_bwd(inp, *, bf16_points: bool, softplus=True, nthreads=1):
 
 
 __all__ = ["round_bf16", "conv1d_fwd", "conv1d_bwd", "scan_fwd", "scan_bwd",
-           "layer_fwd_bwd", "lib"]
+           "decode_step", "layer_fwd_bwd", "lib"]

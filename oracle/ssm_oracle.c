@@ -151,7 +151,13 @@ typedef struct {
     const double *u, *delta, *z, *A, *Dskip, *delta_bias, *Bm, *Cm;
     const int32_t* seq;
     int B, D, L, N, softplus_on;
+    const double* h0;   /* [B][D][N] state before token 0, NULL = zero */
 } scan_in_t;
+
+/* State before token 0 of row (b, d), state n. */
+static double h0_at(const scan_in_t* p, int b, int d, int n) {
+    return p->h0 ? p->h0[((size_t)b * p->D + d) * p->N + n] : 0.0;
+}
 
 /* delta_t for row (b, d), token t (softplus of raw + bias, or raw + bias). */
 static double delta_at(const scan_in_t* p, int d, size_t row, int t) {
@@ -166,6 +172,7 @@ static void scan_fwd_row(const scan_in_t* p, int b, int d, double* out,
     const int L = p->L, N = p->N;
     size_t row = ((size_t)b * p->D + d) * L;
     double* h = (double*)calloc((size_t)N, sizeof(double));
+    for (int n = 0; n < N; ++n) h[n] = h0_at(p, b, d, n);
     for (int t = 0; t < L; ++t) {
         double dt = delta_at(p, d, row, t);
         double ut = p->u[row + t];
@@ -196,9 +203,9 @@ static void scan_fwd_row(const scan_in_t* p, int b, int d, double* out,
 void oracle_scan_fwd(const double* u, const double* delta, const double* z,
                      const double* A, const double* Dskip, const double* delta_bias,
                      const double* Bm, const double* Cm, int softplus_on,
-                     const int32_t* seq, double* out, double* y_out,
+                     const int32_t* seq, const double* h0, double* out, double* y_out,
                      double* final_state, int B, int D, int L, int N) {
-    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on};
+    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0};
     for (int b = 0; b < B; ++b)
         for (int d = 0; d < D; ++d) scan_fwd_row(&p, b, d, out, y_out, final_state);
 }
@@ -208,6 +215,7 @@ typedef struct {
     const double* dout;
     double *du, *ddelta, *dz;          /* per row, overwritten */
     double *dA, *dB, *dC, *dD, *ddb;   /* accumulated */
+    double* dh0;                       /* [B][D][N] per row, overwritten; may be NULL */
 } scan_grad_t;
 
 /* One row. Re-runs the forward keeping every h_t and A_bar_t, then walks t
@@ -236,7 +244,7 @@ static void scan_bwd_row(const scan_in_t* p, const scan_grad_t* g, int b, int d)
             double abar = exp(dt * p->A[(size_t)d * N + n]);
             double bt = p->Bm[((size_t)b * N + n) * L + t];
             double ct = p->Cm[((size_t)b * N + n) * L + t];
-            double hprev = (t == 0 || reset) ? 0.0 : hs[(size_t)(t - 1) * N + n];
+            double hprev = reset ? 0.0 : (t == 0 ? h0_at(p, b, d, n) : hs[(size_t)(t - 1) * N + n]);
             double h = abar * hprev + dt * bt * ut;
             hs[(size_t)t * N + n] = h;
             ab[(size_t)t * N + n] = abar;
@@ -265,7 +273,7 @@ static void scan_bwd_row(const scan_in_t* p, const scan_grad_t* g, int b, int d)
             size_t bn = ((size_t)b * N + n) * L + t;
             double An = p->A[(size_t)d * N + n];
             double gt = dy * p->Cm[bn] + carry[n];
-            double hprev = (t == 0) ? 0.0 : hs[(size_t)(t - 1) * N + n];
+            double hprev = (t == 0) ? h0_at(p, b, d, n) : hs[(size_t)(t - 1) * N + n];
             double q = gt * rs[t] * ab[(size_t)t * N + n] * hprev; /* g * dh/d(A_bar) * A_bar */
             g->dC[bn] += dy * hs[(size_t)t * N + n];
             g->dB[bn] += gt * dt * ut;
@@ -284,23 +292,27 @@ static void scan_bwd_row(const scan_in_t* p, const scan_grad_t* g, int b, int d)
         g->ddelta[row + t] = dv;
         if (g->ddb) g->ddb[d] += dv;
     }
+    /* h_{-1} enters token 0 only through A_bar_0 h_{-1}: its gradient is the
+     * carry left after token 0 */
+    if (g->dh0)
+        for (int n = 0; n < N; ++n) g->dh0[((size_t)b * p->D + d) * N + n] = carry[n];
     free(hs); free(ab); free(dts); free(ys); free(rs); free(carry);
 }
 
 void oracle_scan_bwd(const double* u, const double* delta, const double* z,
                      const double* A, const double* Dskip, const double* delta_bias,
                      const double* Bm, const double* Cm, int softplus_on,
-                     const int32_t* seq, const double* dout, double* du,
+                     const int32_t* seq, const double* h0, const double* dout, double* du,
                      double* ddelta, double* dz, double* dA, double* dB,
-                     double* dC, double* dD, double* ddelta_bias,
+                     double* dC, double* dD, double* ddelta_bias, double* dh0,
                      int B, int D, int L, int N) {
-    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on};
+    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0};
     memset(dA, 0, sizeof(double) * (size_t)D * N);
     memset(dB, 0, sizeof(double) * (size_t)B * N * L);
     memset(dC, 0, sizeof(double) * (size_t)B * N * L);
     if (dD) memset(dD, 0, sizeof(double) * (size_t)D);
     if (ddelta_bias) memset(ddelta_bias, 0, sizeof(double) * (size_t)D);
-    scan_grad_t g = {dout, du, ddelta, dz, dA, dB, dC, dD, ddelta_bias};
+    scan_grad_t g = {dout, du, ddelta, dz, dA, dB, dC, dD, ddelta_bias, dh0};
     for (int b = 0; b < B; ++b)
         for (int d = 0; d < D; ++d) scan_bwd_row(&p, &g, b, d);
 }
@@ -328,9 +340,9 @@ static void* run_job(void* arg) {
 void oracle_scan_fwd_mt(const double* u, const double* delta, const double* z,
                         const double* A, const double* Dskip, const double* delta_bias,
                         const double* Bm, const double* Cm, int softplus_on,
-                        const int32_t* seq, double* out, double* y_out,
+                        const int32_t* seq, const double* h0, double* out, double* y_out,
                         double* final_state, int B, int D, int L, int N, int nthreads) {
-    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on};
+    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0};
     int rows = B * D;
     if (nthreads < 1) nthreads = 1;
     if (nthreads > rows) nthreads = rows;
@@ -350,11 +362,11 @@ void oracle_scan_fwd_mt(const double* u, const double* delta, const double* z,
 void oracle_scan_bwd_mt(const double* u, const double* delta, const double* z,
                         const double* A, const double* Dskip, const double* delta_bias,
                         const double* Bm, const double* Cm, int softplus_on,
-                        const int32_t* seq, const double* dout, double* du,
+                        const int32_t* seq, const double* h0, const double* dout, double* du,
                         double* ddelta, double* dz, double* dA, double* dB,
-                        double* dC, double* dD, double* ddelta_bias,
+                        double* dC, double* dD, double* ddelta_bias, double* dh0,
                         int B, int D, int L, int N, int nthreads) {
-    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on};
+    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0};
     int rows = B * D;
     if (nthreads < 1) nthreads = 1;
     if (nthreads > rows) nthreads = rows;
@@ -366,6 +378,7 @@ void oracle_scan_bwd_mt(const double* u, const double* delta, const double* z,
         jobs[i].bwd = 1;
         jobs[i].g.dout = dout;
         jobs[i].g.du = du; jobs[i].g.ddelta = ddelta; jobs[i].g.dz = dz;
+        jobs[i].g.dh0 = dh0;
         jobs[i].g.dA = (double*)calloc(nA, sizeof(double));
         jobs[i].g.dB = (double*)calloc(nBC, sizeof(double));
         jobs[i].g.dC = (double*)calloc(nBC, sizeof(double));
@@ -392,4 +405,41 @@ void oracle_scan_bwd_mt(const double* u, const double* delta, const double* z,
         free(jobs[i].g.dD); free(jobs[i].g.ddb);
     }
     free(th); free(jobs);
+}
+
+/* ------------------------------------------------------- recurrent step */
+/* One token for every (b, d): the recurrent (decode) form of the layer.
+ * conv_state[b][d][0..W-2] holds the W-1 previous inputs x_{t-W+1} .. x_{t-1}
+ * (oldest first); the causal conv reads them and x_t, then the window shifts
+ * by one. The state h[b][d][n] (h_{t-1} on entry) becomes h_t. Follows the
+ * same definitions as the sequence form: conv taps w[d][k] on x_{t-W+1+k},
+ * u = SiLU(c), delta = softplus(raw + bias), h_t = exp(delta A) h_{t-1} +
+ * delta B_t u, y = C_t . h_t + D u, out = y SiLU(z). u_out may be NULL. */
+void oracle_decode_step(const double* x, double* conv_state, const double* w,
+                        const double* conv_bias, const double* delta, const double* z,
+                        const double* Bt, const double* Ct, const double* A,
+                        const double* Dskip, const double* delta_bias, int softplus_on,
+                        double* h, double* out, double* u_out, int B, int D, int N, int W) {
+    for (int b = 0; b < B; ++b)
+        for (int d = 0; d < D; ++d) {
+            size_t bd = (size_t)b * D + d;
+            double* cs = conv_state + bd * (size_t)(W - 1);
+            double c = conv_bias ? conv_bias[d] : 0.0;
+            for (int k = 0; k < W - 1; ++k) c += w[(size_t)d * W + k] * cs[k];
+            c += w[(size_t)d * W + W - 1] * x[bd];
+            for (int k = 0; k + 1 < W - 1; ++k) cs[k] = cs[k + 1];
+            if (W > 1) cs[W - 2] = x[bd];
+            double u = c * sigm(c);
+            if (u_out) u_out[bd] = u;
+            double v = delta[bd] + (delta_bias ? delta_bias[d] : 0.0);
+            double dt = softplus_on ? softplus(v) : v;
+            double y = 0.0;
+            for (int n = 0; n < N; ++n) {
+                double* hn = h + bd * (size_t)N + n;
+                *hn = exp(dt * A[(size_t)d * N + n]) * *hn + dt * Bt[(size_t)b * N + n] * u;
+                y += Ct[(size_t)b * N + n] * *hn;
+            }
+            if (Dskip) y += Dskip[d] * u;
+            out[bd] = z ? y * z[bd] * sigm(z[bd]) : y;
+        }
 }

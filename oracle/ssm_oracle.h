@@ -5,7 +5,8 @@
  *
  * Layouts (all contiguous): activations [B][D][L]; B/C [B][N][L];
  * A [D][N]; conv weight [D][W]; per-channel vectors [D]; seq_idx [B][L]
- * (NULL = one segment per row); final state [B][D][N].
+ * (NULL = one segment per row); initial / final state [B][D][N] (h0 NULL =
+ * zero state).
  */
 #ifndef SSM_ORACLE_H
 #define SSM_ORACLE_H
@@ -24,26 +25,33 @@ void oracle_conv1d_bwd(const double* x, const double* w, const double* bias,
 void oracle_scan_fwd(const double* u, const double* delta, const double* z,
                      const double* A, const double* Dskip, const double* delta_bias,
                      const double* Bm, const double* Cm, int softplus_on,
-                     const int32_t* seq, double* out, double* y_out,
+                     const int32_t* seq, const double* h0, double* out, double* y_out,
                      double* final_state, int B, int D, int L, int N);
 void oracle_scan_bwd(const double* u, const double* delta, const double* z,
                      const double* A, const double* Dskip, const double* delta_bias,
                      const double* Bm, const double* Cm, int softplus_on,
-                     const int32_t* seq, const double* dout, double* du,
+                     const int32_t* seq, const double* h0, const double* dout, double* du,
                      double* ddelta, double* dz, double* dA, double* dB,
-                     double* dC, double* dD, double* ddelta_bias,
+                     double* dC, double* dD, double* ddelta_bias, double* dh0,
                      int B, int D, int L, int N);
 
 void oracle_scan_fwd_mt(const double* u, const double* delta, const double* z,
                         const double* A, const double* Dskip, const double* delta_bias,
                         const double* Bm, const double* Cm, int softplus_on,
-                        const int32_t* seq, double* out, double* y_out,
+                        const int32_t* seq, const double* h0, double* out, double* y_out,
                         double* final_state, int B, int D, int L, int N, int nthreads);
 void oracle_scan_bwd_mt(const double* u, const double* delta, const double* z,
                         const double* A, const double* Dskip, const double* delta_bias,
                         const double* Bm, const double* Cm, int softplus_on,
-                        const int32_t* seq, const double* dout, double* du,
+                        const int32_t* seq, const double* h0, const double* dout, double* du,
                         double* ddelta, double* dz, double* dA, double* dB,
-                        double* dC, double* dD, double* ddelta_bias,
+                        double* dC, double* dD, double* ddelta_bias, double* dh0,
                         int B, int D, int L, int N, int nthreads);
+/* Recurrent form, one token (x, delta, z [B][D]; Bt, Ct [B][N];
+ * conv_state [B][D][W-1] and h [B][D][N] updated in place). */
+void oracle_decode_step(const double* x, double* conv_state, const double* w,
+                        const double* conv_bias, const double* delta, const double* z,
+                        const double* Bt, const double* Ct, const double* A,
+                        const double* Dskip, const double* delta_bias, int softplus_on,
+                        double* h, double* out, double* u_out, int B, int D, int N, int W);
 #endif

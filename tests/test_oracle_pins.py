@@ -423,3 +423,107 @@ def test_softplus_reading_is_exact_log1p_exp():
     y = oracle.scan_fwd(u, v, A, Bm, Cm, softplus=True)["y"][0, 0]
     want = np.cumsum([math.log1p(math.exp(t)) for t in v.ravel()])
     np.testing.assert_allclose(y, want, rtol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# initial state and the recurrent (decode) form
+# --------------------------------------------------------------------------
+def test_scan_h0_continues_a_prefix():
+    """A suffix started from the prefix's final state reproduces the full run
+    (the recurrence carries nothing else across the cut)."""
+    rng = _rng(61)
+    p = _problem(rng, B=2, D=3, N=4, L=40)
+    full = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], z=p["z"],
+                           Dskip=p["Dskip"], delta_bias=p["delta_bias"])
+    for s in (1, 17, 39):
+        pre = oracle.scan_fwd(p["u"][..., :s], p["delta"][..., :s], p["A"], p["Bm"][..., :s],
+                              p["Cm"][..., :s], z=p["z"][..., :s], Dskip=p["Dskip"],
+                              delta_bias=p["delta_bias"])
+        suf = oracle.scan_fwd(p["u"][..., s:], p["delta"][..., s:], p["A"], p["Bm"][..., s:],
+                              p["Cm"][..., s:], z=p["z"][..., s:], Dskip=p["Dskip"],
+                              delta_bias=p["delta_bias"], h0=pre["final_state"])
+        np.testing.assert_allclose(suf["out"], full["out"][..., s:], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(suf["final_state"], full["final_state"], rtol=1e-12,
+                                   atol=1e-12)
+
+
+def test_scan_h0_reset_at_document_start():
+    """With seq_idx, h0 feeds the first document only."""
+    rng = _rng(62)
+    seq = np.array([[0] * 12 + [1] * 20], dtype=np.int32)
+    p = _problem(rng, B=1, D=2, N=3, L=32, seq=seq)
+    h0 = rng.standard_normal((1, 2, 3))
+    a = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], seq_idx=seq, h0=h0)
+    b = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], seq_idx=seq)
+    assert np.abs(a["out"][..., :12] - b["out"][..., :12]).max() > 1e-6
+    np.testing.assert_array_equal(a["out"][..., 12:], b["out"][..., 12:])
+
+
+@pytest.mark.parametrize("softplus", [True, False])
+def test_scan_bwd_h0_finite_differences(softplus):
+    """dh0, and the h0 term inside dA and d(delta), against finite differences."""
+    rng = _rng(63)
+    p = _problem(rng, B=2, D=3, N=4, L=24)
+    if not softplus:
+        p["delta"] = np.abs(p["delta"]) * 0.2
+        p["delta_bias"] = np.zeros_like(p["delta_bias"])
+    h0 = rng.standard_normal((2, 3, 4))
+    dout = rng.standard_normal(p["u"].shape)
+
+    def loss():
+        r = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], z=p["z"],
+                            Dskip=p["Dskip"], delta_bias=p["delta_bias"], softplus=softplus,
+                            h0=h0)
+        return float(np.sum(r["out"] * dout))
+
+    g = oracle.scan_bwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], dout, z=p["z"],
+                        Dskip=p["Dskip"], delta_bias=p["delta_bias"], softplus=softplus, h0=h0)
+    _close(_fd(loss, h0), g["dh0"])
+    _close(_fd(loss, p["A"]), g["dA"])
+    _close(_fd(loss, p["delta"]), g["ddelta"])
+
+
+def test_decode_steps_equal_the_sequence_form():
+    """Stepping the recurrent form over a sequence from a zero conv window and
+    a zero state gives the sequence form's u, out and final state."""
+    rng = _rng(64)
+    B, D, N, L, W = 2, 3, 4, 30, 4
+    p = _problem(rng, B=B, D=D, N=N, L=L)
+    x = rng.standard_normal((B, D, L))
+    w = rng.uniform(-0.5, 0.5, size=(D, W))
+    cb = rng.uniform(-0.2, 0.2, size=D)
+    _, u = oracle.conv1d_fwd(x, w, cb, None)
+    full = oracle.scan_fwd(u, p["delta"], p["A"], p["Bm"], p["Cm"], z=p["z"],
+                           Dskip=p["Dskip"], delta_bias=p["delta_bias"])
+    cs = np.zeros((B, D, W - 1))
+    h = np.zeros((B, D, N))
+    for t in range(L):
+        out, ut, cs, h = oracle.decode_step(x[..., t], cs, w, cb, p["delta"][..., t],
+                                            p["Bm"][..., t], p["Cm"][..., t], p["A"], h,
+                                            z=p["z"][..., t], Dskip=p["Dskip"],
+                                            delta_bias=p["delta_bias"])
+        np.testing.assert_allclose(ut, u[..., t], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(out, full["out"][..., t], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(h, full["final_state"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(cs, x[..., L - W + 1:])
+
+
+def test_decode_continues_a_prefill():
+    """Prefill with the sequence form, then decode: conv window = the last
+    W-1 inputs, state = the prefill's final state."""
+    rng = _rng(65)
+    B, D, N, L, W, s = 1, 2, 3, 20, 4, 13
+    p = _problem(rng, B=B, D=D, N=N, L=L)
+    x = rng.standard_normal((B, D, L))
+    w = rng.uniform(-0.5, 0.5, size=(D, W))
+    _, u = oracle.conv1d_fwd(x, w, None, None)
+    full = oracle.scan_fwd(u, p["delta"], p["A"], p["Bm"], p["Cm"], Dskip=p["Dskip"],
+                           delta_bias=p["delta_bias"])
+    pre = oracle.scan_fwd(u[..., :s], p["delta"][..., :s], p["A"], p["Bm"][..., :s],
+                          p["Cm"][..., :s], Dskip=p["Dskip"], delta_bias=p["delta_bias"])
+    cs, h = x[..., s - W + 1:s].copy(), pre["final_state"]
+    for t in range(s, L):
+        out, _, cs, h = oracle.decode_step(x[..., t], cs, w, None, p["delta"][..., t],
+                                           p["Bm"][..., t], p["Cm"][..., t], p["A"], h,
+                                           Dskip=p["Dskip"], delta_bias=p["delta_bias"])
+        np.testing.assert_allclose(out, full["out"][..., t], rtol=1e-12, atol=1e-12)

@@ -66,7 +66,7 @@ typedef enum { SSM_DTYPE_F32 = 0, SSM_DTYPE_BF16 = 1 } ssm_dtype_t;
 const char* ssm_last_error(void);
 
 /* ABI version of this header (bumped on any incompatible change). */
-#define SSM_ABI_VERSION 1
+#define SSM_ABI_VERSION 2
 int ssm_abi_version(void);
 
 /* ---------------------------------------------------------------------------
@@ -133,7 +133,8 @@ ssm_status_t ssm_conv1d_bwd_noalloc(const void* x, const float* w, const float* 
  * Selective scan. For each row (b, d) and state n < N, with
  *   dt_t = softplus(delta[b][d][t] + delta_bias[d])   (or without softplus)
  *   a_t  = exp(dt_t * A[d][n])      (0 at the first token of a document)
- *   h_t  = a_t * h_{t-1} + dt_t * Bm[b][n][t] * u[b][d][t],   h_{-1} = 0
+ *   h_t  = a_t * h_{t-1} + dt_t * Bm[b][n][t] * u[b][d][t],
+ *   h_{-1} = initial_state[b][d][n]  (0 when initial_state is NULL)
  *   y_t  = sum_n Cm[b][n][t] * h_t + Dskip[d] * u[b][d][t]
  *   out  = y_t * silu(z[b][d][t])   (or y_t when z is NULL)
  * final_state[b][d][n] = h_{L-1}.
@@ -161,11 +162,14 @@ typedef struct {
     float* final_state;        /* [B][D][N] nullable */
     void* workspace;           /* device scratch, >= ssm_scan_workspace_size bytes, 256-B aligned */
     size_t workspace_bytes;
+    const float* initial_state;/* [B][D][N] nullable: the state before token 0 (h_{-1}); with
+                                  seq_idx it feeds the first document of each row only */
 } ssm_scan_params;
 
-/* Workspace bytes for these params: per-chunk state checkpoints (read by the
- * backward), split carries, segment ids built from cu_seqlens, and partial
- * sums of the backward's parameter reductions. */
+/* Workspace bytes for these params: the state entering every 32-token block
+ * and, with a gate, y before the gate (both written by the forward, read by
+ * the backward), split carries, segment ids built from cu_seqlens, and
+ * partial sums of the backward's parameter reductions. */
 ssm_status_t ssm_scan_workspace_size(const ssm_scan_params* p, size_t* bytes);
 
 /* Forward. Also writes the checkpoints the backward reads into p->workspace:
@@ -185,6 +189,8 @@ typedef struct {
     float* ddelta_bias;        /* [D] nullable output */
     int deterministic;         /* reserved; dA, dD, ddelta_bias are always reduced in a fixed
                                   order, dB and dC are summed over channels with fp32 atomics */
+    float* dinitial_state;     /* [B][D][N] nullable output: dL/dh_{-1} (the gradient with
+                                  respect to initial_state, or to the zero state when NULL) */
 } ssm_scan_grads;
 
 /* Backward. Recomputes states from the checkpoints in p->workspace, so the
@@ -216,6 +222,47 @@ ssm_status_t ssm_scan_status(const ssm_scan_params* p, int* device_status, ssm_s
  * ------------------------------------------------------------------------ */
 ssm_status_t ssm_probe_ex2_rate(float* sink, size_t sink_floats, double* ex2_per_second,
                                 ssm_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Recurrent form, one token per row: the layer's inference mode
+ * ("hung-phan ml-skills mamba", "Dual Computation Modes": recurrent mode,
+ * token by token with O(1) memory per step; "Inference (Generation)": no KV
+ * cache, a (B, D, N) state is carried forward). The same conv, step and
+ * state update as the sequence form, for every (b, d):
+ *   c = conv_bias[d] + sum_{k < W-1} conv_w[d][k] conv_state[b][d][k]
+ *                    + conv_w[d][W-1] x[b][d]
+ *   conv_state[b][d] <- (conv_state[b][d][1 .. W-2], x[b][d])
+ *   u = silu(c);  dt = softplus(delta[b][d] + delta_bias[d])  (or without softplus)
+ *   state[b][d][n] <- exp(dt A[d][n]) state[b][d][n] + dt Bm[b][n] u
+ *   out[b][d] = (sum_n Cm[b][n] state[b][d][n] + Dskip[d] u) silu(z[b][d])
+ * so stepping it over a sequence from a zero conv window and a zero state
+ * reproduces ssm_conv1d_fwd + ssm_scan_fwd, and after a prefill (conv window
+ * = the last W-1 inputs, state = the prefill's final_state) it continues it.
+ * Sizes: B, D >= 1, 1 <= N <= 16, W == 4 (else SSM_ERR_UNSUPPORTED).
+ * conv_state and state are updated in place; no other input is written.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    size_t struct_size;        /* = sizeof(ssm_decode_params) */
+    int B, D, N, W;
+    ssm_dtype_t dtype;         /* dtype of x, conv_state, delta, z, Bm, Cm, out, u_out */
+    const void* x;             /* [B][D] conv input of this token */
+    void* conv_state;          /* [B][D][W-1] in/out: the previous W-1 inputs, oldest first */
+    const float* conv_w;       /* [D][W] */
+    const float* conv_bias;    /* [D] nullable (0) */
+    const void* delta;         /* [B][D] raw step, before bias and softplus */
+    const void* z;             /* [B][D] gate input, nullable (no gate) */
+    const void* Bm;            /* [B][N] */
+    const void* Cm;            /* [B][N] */
+    const float* A;            /* [D][N] */
+    const float* Dskip;        /* [D] nullable (0) */
+    const float* delta_bias;   /* [D] nullable (0) */
+    int delta_softplus;        /* as in ssm_scan_params */
+    float* state;              /* [B][D][N] fp32 in/out: h_{t-1} on entry, h_t on return */
+    void* out;                 /* [B][D] output */
+    void* u_out;               /* [B][D] nullable output: the conv+SiLU value u */
+} ssm_decode_params;
+
+ssm_status_t ssm_decode_step(const ssm_decode_params* p, ssm_stream_t stream);
 
 #ifdef __cplusplus
 }

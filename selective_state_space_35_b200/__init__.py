@@ -14,7 +14,8 @@ import ctypes
 from . import _lib
 from ._lib import (SsmError, ssm_abi_version, ssm_conv1d_bwd, ssm_conv1d_bwd_noalloc,
                    ssm_conv1d_bwd_workspace_size,
-                   ssm_conv1d_fwd, ssm_last_error, ssm_probe_ex2_rate, ssm_scan_bwd, ssm_scan_status,
+                   ssm_conv1d_fwd, ssm_decode_params, ssm_decode_step, ssm_last_error,
+                   ssm_probe_ex2_rate, ssm_scan_bwd, ssm_scan_status,
                    ssm_scan_fwd, ssm_scan_grads, ssm_scan_params, ssm_scan_workspace_size)
 
 __all__ = [
@@ -23,6 +24,7 @@ __all__ = [
     "ssm_scan_params", "ssm_scan_grads", "ssm_probe_ex2_rate", "probe_ex2_rate", "ssm_scan_status",
     "scan_status", "conv1d_fwd", "conv1d_bwd", "scan_params",
     "scan_workspace_size", "scan_fwd", "scan_bwd", "load",
+    "ssm_decode_params", "ssm_decode_step", "decode_step",
 ]
 
 load = _lib.load
@@ -118,7 +120,7 @@ def conv1d_bwd(x, w, bias, seq_idx, du, *, silu=True, dx=None, dw=None, dbias=No
 
 def scan_params(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softplus=True,
                 seq_idx=None, cu_seqlens=None, n_splits=0, out=None, final_state=None,
-                workspace=None) -> ssm_scan_params:
+                workspace=None, initial_state=None) -> ssm_scan_params:
     """Fill an ssm_scan_params from tensors (validating shapes and dtypes)."""
     torch = _torch()
     B, D, L = u.shape
@@ -135,6 +137,7 @@ def scan_params(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, sof
     _need(cu_seqlens, "cu_seqlens", torch.int32)
     _need(out, "out", u.dtype, (B, D, L))
     _need(final_state, "final_state", torch.float32, (B, D, N))
+    _need(initial_state, "initial_state", torch.float32, (B, D, N))
     p = ssm_scan_params()
     p.struct_size = ctypes.sizeof(ssm_scan_params)
     p.B, p.D, p.L, p.N = B, D, L, N
@@ -153,6 +156,7 @@ def scan_params(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, sof
     p.final_state = final_state.data_ptr() if final_state is not None else None
     p.workspace = workspace.data_ptr() if workspace is not None else None
     p.workspace_bytes = workspace.numel() if workspace is not None else 0
+    p.initial_state = initial_state.data_ptr() if initial_state is not None else None
     return p
 
 
@@ -174,11 +178,12 @@ def scan_status(u, A, workspace, stream=None) -> int:
 
 def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softplus=True,
              seq_idx=None, cu_seqlens=None, n_splits=0, return_final_state=False, out=None,
-             workspace=None, stream=None):
+             workspace=None, initial_state=None, stream=None):
     """Selective scan forward.
 
     Returns (out, final_state or None, workspace). Keep `workspace` (it holds
-    the per-chunk state checkpoints) and pass it to scan_bwd unchanged.
+    the state checkpoints and the pre-gate output) and pass it to scan_bwd
+    unchanged. `initial_state` [B, D, N] fp32 is the state before token 0.
     """
     torch = _torch()
     B, D, L = u.shape
@@ -187,7 +192,7 @@ def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softpl
     fs = torch.empty((B, D, N), dtype=torch.float32, device=u.device) if return_final_state else None
     p = scan_params(u, delta, A, Bm, Cm, z=z, Dskip=Dskip, delta_bias=delta_bias, softplus=softplus,
                     seq_idx=seq_idx, cu_seqlens=cu_seqlens, n_splits=n_splits, out=out,
-                    final_state=fs)
+                    final_state=fs, initial_state=initial_state)
     need = ssm_scan_workspace_size(p)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=u.device)
@@ -197,11 +202,14 @@ def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softpl
 
 
 def scan_bwd(u, delta, A, Bm, Cm, dout, workspace, *, z=None, Dskip=None, delta_bias=None,
-             softplus=True, seq_idx=None, cu_seqlens=None, n_splits=0, grads=None, stream=None):
-    """Selective scan backward; `workspace` must come from the matching scan_fwd.
+             softplus=True, seq_idx=None, cu_seqlens=None, n_splits=0, grads=None,
+             initial_state=None, stream=None):
+    """Selective scan backward; `workspace` must come from the matching scan_fwd
+    (called with the same `initial_state`).
 
     Returns a dict: du, ddelta (w.r.t. the raw delta), dz (or None), dA, dB,
-    dC, dD, ddelta_bias. Preallocated outputs may be passed in `grads`.
+    dC, dD, ddelta_bias, dinitial_state (w.r.t. the state before token 0).
+    Preallocated outputs may be passed in `grads`.
     """
     torch = _torch()
     B, D, L = u.shape
@@ -217,9 +225,10 @@ def scan_bwd(u, delta, A, Bm, Cm, dout, workspace, *, z=None, Dskip=None, delta_
     g.setdefault("dC", torch.empty((B, N, L), dtype=torch.float32, device=dev))
     g.setdefault("dD", torch.empty((D,), dtype=torch.float32, device=dev))
     g.setdefault("ddelta_bias", torch.empty((D,), dtype=torch.float32, device=dev))
+    g.setdefault("dinitial_state", torch.empty((B, D, N), dtype=torch.float32, device=dev))
     p = scan_params(u, delta, A, Bm, Cm, z=z, Dskip=Dskip, delta_bias=delta_bias, softplus=softplus,
                     seq_idx=seq_idx, cu_seqlens=cu_seqlens, n_splits=n_splits, out=None,
-                    workspace=workspace)
+                    workspace=workspace, initial_state=initial_state)
     p.out = dout.data_ptr()  # not written by the backward; any valid activation pointer
     gr = ssm_scan_grads()
     gr.struct_size = ctypes.sizeof(ssm_scan_grads)
@@ -229,5 +238,52 @@ def scan_bwd(u, delta, A, Bm, Cm, dout, workspace, *, z=None, Dskip=None, delta_
     gr.dA, gr.dB, gr.dC = g["dA"].data_ptr(), g["dB"].data_ptr(), g["dC"].data_ptr()
     gr.dD = g["dD"].data_ptr() if g["dD"] is not None else None
     gr.ddelta_bias = g["ddelta_bias"].data_ptr() if g["ddelta_bias"] is not None else None
+    gr.dinitial_state = (g["dinitial_state"].data_ptr() if g["dinitial_state"] is not None
+                         else None)
     _lib.check(ssm_scan_bwd(p, gr, _stream(stream, u.device)))
     return g
+
+
+def decode_step(x, conv_state, conv_w, delta, A, Bm, Cm, state, *, conv_bias=None, z=None,
+                Dskip=None, delta_bias=None, softplus=True, out=None, u_out=None, stream=None):
+    """One token of the recurrent form for every (b, d).
+
+    x, delta, z: [B, D] activations; conv_state: [B, D, 3] activation dtype,
+    the previous three conv inputs (updated in place); conv_w [D, 4],
+    conv_bias [D]; Bm, Cm: [B, N]; A: [D, N]; state: [B, D, N] fp32 (updated
+    in place). Returns out [B, D] (and writes u_out [B, D] if given).
+    """
+    torch = _torch()
+    B, D = x.shape
+    N = A.shape[1]
+    _need(x, "x", shape=(B, D))
+    _need(conv_state, "conv_state", x.dtype, (B, D, 3))
+    _need(conv_w, "conv_w", torch.float32, (D, 4))
+    _need(conv_bias, "conv_bias", torch.float32, (D,))
+    _need(delta, "delta", x.dtype, (B, D))
+    _need(z, "z", x.dtype, (B, D))
+    _need(Bm, "Bm", x.dtype, (B, N))
+    _need(Cm, "Cm", x.dtype, (B, N))
+    _need(A, "A", torch.float32, (D, N))
+    _need(Dskip, "Dskip", torch.float32, (D,))
+    _need(delta_bias, "delta_bias", torch.float32, (D,))
+    _need(state, "state", torch.float32, (B, D, N))
+    out = torch.empty_like(x) if out is None else out
+    _need(out, "out", x.dtype, (B, D))
+    _need(u_out, "u_out", x.dtype, (B, D))
+    p = ssm_decode_params()
+    p.struct_size = ctypes.sizeof(ssm_decode_params)
+    p.B, p.D, p.N, p.W = B, D, N, 4
+    p.dtype = _dtype_code(x)
+    p.x, p.conv_state, p.conv_w = x.data_ptr(), conv_state.data_ptr(), conv_w.data_ptr()
+    p.conv_bias = conv_bias.data_ptr() if conv_bias is not None else None
+    p.delta = delta.data_ptr()
+    p.z = z.data_ptr() if z is not None else None
+    p.Bm, p.Cm, p.A = Bm.data_ptr(), Cm.data_ptr(), A.data_ptr()
+    p.Dskip = Dskip.data_ptr() if Dskip is not None else None
+    p.delta_bias = delta_bias.data_ptr() if delta_bias is not None else None
+    p.delta_softplus = int(softplus)
+    p.state, p.out = state.data_ptr(), out.data_ptr()
+    p.u_out = u_out.data_ptr() if u_out is not None else None
+    _lib.check(ssm_decode_step(p, _stream(stream, x.device)))
+    return out

@@ -45,6 +45,7 @@ class ssm_scan_params(ctypes.Structure):
         ("n_splits", _i),
         ("out", _vp), ("final_state", _vp),
         ("workspace", _vp), ("workspace_bytes", _sz),
+        ("initial_state", _vp),
     ]
 
 
@@ -54,13 +55,28 @@ class ssm_scan_grads(ctypes.Structure):
         ("dout", _vp), ("du", _vp), ("ddelta", _vp), ("dz", _vp),
         ("dA", _vp), ("dB", _vp), ("dC", _vp), ("dD", _vp), ("ddelta_bias", _vp),
         ("deterministic", _i),
+        ("dinitial_state", _vp),
+    ]
+
+
+class ssm_decode_params(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", _sz),
+        ("B", _i), ("D", _i), ("N", _i), ("W", _i),
+        ("dtype", _i),
+        ("x", _vp), ("conv_state", _vp), ("conv_w", _vp), ("conv_bias", _vp),
+        ("delta", _vp), ("z", _vp), ("Bm", _vp), ("Cm", _vp),
+        ("A", _vp), ("Dskip", _vp), ("delta_bias", _vp),
+        ("delta_softplus", _i),
+        ("state", _vp), ("out", _vp), ("u_out", _vp),
     ]
 
 
 _lib = None
 
 EXPORTS = ("ssm_last_error", "ssm_abi_version", "ssm_conv1d_fwd", "ssm_conv1d_bwd_workspace_size",
-           "ssm_conv1d_bwd", "ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_scan_bwd")
+           "ssm_conv1d_bwd", "ssm_conv1d_bwd_noalloc", "ssm_scan_workspace_size", "ssm_scan_fwd",
+           "ssm_scan_bwd", "ssm_scan_status", "ssm_probe_ex2_rate", "ssm_decode_step")
 
 
 def load(path: str | None = None):
@@ -98,6 +114,8 @@ def load(path: str | None = None):
     L.ssm_scan_status.argtypes = [ctypes.POINTER(ssm_scan_params), ctypes.POINTER(_i), _vp]
     L.ssm_probe_ex2_rate.restype = _i
     L.ssm_probe_ex2_rate.argtypes = [_vp, _sz, ctypes.POINTER(ctypes.c_double), _vp]
+    L.ssm_decode_step.restype = _i
+    L.ssm_decode_step.argtypes = [ctypes.POINTER(ssm_decode_params), _vp]
     if path is None:
         _lib = L
     return L
@@ -163,3 +181,7 @@ def ssm_scan_fwd(params: ssm_scan_params, stream) -> int:
 
 def ssm_scan_bwd(params: ssm_scan_params, grads: ssm_scan_grads, stream) -> int:
     return load().ssm_scan_bwd(_ref(params), _ref(grads), stream)
+
+
+def ssm_decode_step(params: ssm_decode_params, stream) -> int:
+    return load().ssm_decode_step(_ref(params), stream)

@@ -144,6 +144,7 @@ ssm_status_t build_args(const ssm_scan_params* p, const ScanPlan& pl, ssm::ScanA
   a->Bm = p->Bm;
   a->Cm = p->Cm;
   a->seq = p->cu_seqlens ? reinterpret_cast<int32_t*>(ws + pl.off_seq) : p->seq_idx;
+  a->h0 = p->initial_state;
   a->softplus = p->delta_softplus ? 1 : 0;
   a->out = p->out;
   a->final_state = p->final_state;
@@ -181,7 +182,8 @@ ssm_status_t check_scan_buffers(const ssm_scan_params* p, const ScanPlan& pl) {
   const void* acts[] = {p->u, p->delta, p->z, p->Bm, p->Cm, p->out};
   for (const void* q : acts)
     if (q && !aligned(q, es)) return fail(SSM_ERR_INVALID_ARG, "activation pointer misaligned");
-  const void* f32s[] = {p->A, p->Dskip, p->delta_bias, p->final_state, p->seq_idx, p->cu_seqlens};
+  const void* f32s[] = {p->A, p->Dskip, p->delta_bias, p->final_state, p->seq_idx, p->cu_seqlens,
+                        p->initial_state};
   for (const void* q : f32s)
     if (q && !aligned(q, 4)) return fail(SSM_ERR_INVALID_ARG, "fp32/int32 pointer misaligned");
   return ok();
@@ -354,7 +356,7 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
   const void* acts[] = {g->dout, g->du, g->ddelta, g->dz};
   for (const void* q : acts)
     if (q && !aligned(q, es)) return fail(SSM_ERR_INVALID_ARG, "gradient pointer misaligned");
-  const void* f32s[] = {g->dA, g->dB, g->dC, g->dD, g->ddelta_bias};
+  const void* f32s[] = {g->dA, g->dB, g->dC, g->dD, g->ddelta_bias, g->dinitial_state};
   for (const void* q : f32s)
     if (q && !aligned(q, 4)) return fail(SSM_ERR_INVALID_ARG, "fp32 gradient pointer misaligned");
   ssm::ScanArgs a;
@@ -368,6 +370,7 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
   a.dC = g->dC;
   a.dD = g->dD;
   a.ddelta_bias = g->ddelta_bias;
+  a.dh0 = g->dinitial_state;
   // dB and dC take 16-byte vector atomics on the vector path
   a.vec = vec_ok(p->L, {p->u, p->delta, p->z, p->Bm, p->Cm, g->dout, g->du, g->ddelta, a.dz, a.seq,
                         g->dB, g->dC});
@@ -393,6 +396,43 @@ ssm_status_t ssm_scan_status(const ssm_scan_params* p, int* device_status, ssm_s
   cudaError_t e = cudaMemcpyAsync(device_status, p->workspace, sizeof(int), cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   return cuda_status(e, "ssm_scan_status");
+}
+
+ssm_status_t ssm_decode_step(const ssm_decode_params* p, ssm_stream_t stream) {
+  if (injected("ssm_decode_step")) return fail(SSM_ERR_INJECTED, "ssm_decode_step: injected failure");
+  if (!p) return fail(SSM_ERR_INVALID_ARG, "params is NULL");
+  if (p->struct_size != sizeof(ssm_decode_params))
+    return fail(SSM_ERR_INVALID_ARG, "params.struct_size %zu != %zu", p->struct_size,
+                sizeof(ssm_decode_params));
+  if (p->B < 1 || p->D < 1 || p->N < 1)
+    return fail(SSM_ERR_INVALID_ARG, "sizes must be >= 1 (B=%d D=%d N=%d)", p->B, p->D, p->N);
+  if (p->N > ssm::kNMax) return fail(SSM_ERR_UNSUPPORTED, "N=%d > %d", p->N, ssm::kNMax);
+  if (p->W != 4) return fail(SSM_ERR_UNSUPPORTED, "conv width W=%d (only 4)", p->W);
+  if ((long)p->B * p->D > (1L << 30))
+    return fail(SSM_ERR_UNSUPPORTED, "B * D = %ld rows exceed 2^30", (long)p->B * p->D);
+  if (p->dtype != SSM_DTYPE_F32 && p->dtype != SSM_DTYPE_BF16)
+    return fail(SSM_ERR_INVALID_ARG, "unknown dtype %d", (int)p->dtype);
+  if (!p->x || !p->conv_state || !p->conv_w || !p->delta || !p->Bm || !p->Cm || !p->A ||
+      !p->state || !p->out)
+    return fail(SSM_ERR_INVALID_ARG,
+                "x, conv_state, conv_w, delta, Bm, Cm, A, state and out must be non-NULL");
+  const size_t es = elem_size(p->dtype);
+  const void* acts[] = {p->x, p->conv_state, p->delta, p->z, p->Bm, p->Cm, p->out, p->u_out};
+  for (const void* q : acts)
+    if (q && !aligned(q, es)) return fail(SSM_ERR_INVALID_ARG, "activation pointer misaligned");
+  const void* f32s[] = {p->conv_w, p->conv_bias, p->A, p->Dskip, p->delta_bias, p->state};
+  for (const void* q : f32s)
+    if (q && !aligned(q, 4)) return fail(SSM_ERR_INVALID_ARG, "fp32 pointer misaligned");
+  if (p->out == p->x || p->out == p->delta || (p->z && p->out == p->z))
+    return fail(SSM_ERR_INVALID_ARG, "out may not alias an input");
+  ssm::DecodeArgs a{};
+  a.x = p->x; a.conv_state = p->conv_state; a.conv_w = p->conv_w; a.conv_bias = p->conv_bias;
+  a.delta = p->delta; a.z = p->z; a.Bm = p->Bm; a.Cm = p->Cm; a.A = p->A; a.Dskip = p->Dskip;
+  a.delta_bias = p->delta_bias; a.state = p->state; a.out = p->out; a.u_out = p->u_out;
+  a.B = p->B; a.D = p->D; a.N = p->N; a.softplus = p->delta_softplus ? 1 : 0;
+  a.bf16 = p->dtype == SSM_DTYPE_BF16;
+  return cuda_status(ssm::launch_decode_step(a, reinterpret_cast<cudaStream_t>(stream)),
+                     "ssm_decode_step launch");
 }
 
 ssm_status_t ssm_probe_ex2_rate(float* sink, size_t sink_floats, double* ex2_per_second,

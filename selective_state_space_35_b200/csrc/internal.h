@@ -47,6 +47,7 @@ struct ScanArgs {
   const void* Bm;
   const void* Cm;
   const int32_t* seq;
+  const float* h0;    // [B*D][N] state before token 0, nullable
   int softplus;
   // forward outputs
   void* out;
@@ -61,6 +62,7 @@ struct ScanArgs {
   float* dC;
   float* dD;
   float* ddelta_bias;
+  float* dh0;         // [B*D][N] nullable
   // workspace pieces
   int* status;        // sticky device status word (0 = ok, 4 = a bounded wait timed out)
   float* ckpt;        // [B*D][nchunks * 8][kNMax] state entering each 32-token block
@@ -78,6 +80,27 @@ struct ScanArgs {
 };
 
 cudaError_t launch_scan_fwd(const ScanArgs& a, cudaStream_t s);
+
+struct DecodeArgs {
+  const void* x;
+  void* conv_state;
+  const float* conv_w;
+  const float* conv_bias;
+  const void* delta;
+  const void* z;
+  const void* Bm;
+  const void* Cm;
+  const float* A;
+  const float* Dskip;
+  const float* delta_bias;
+  float* state;
+  void* out;
+  void* u_out;
+  int B, D, N, softplus;
+  bool bf16;
+};
+
+cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_scan_bwd(const ScanArgs& a, cudaStream_t s);
 cudaError_t probe_ex2_rate(float* sink, size_t sink_floats, double* rate, cudaStream_t s);
 cudaError_t launch_cu_seqlens_to_seq(const int32_t* cu, int n_docs, int L, int32_t* seq,

@@ -66,7 +66,10 @@ __device__ __forceinline__ void lds_tokpairs(const float* row, int lane, float2 
 // memory by cp.async while the block before it is being processed.
 // ---------------------------------------------------------------------------
 constexpr int kBlk = 32;                   // tokens per block (= checkpoint interval)
-constexpr int kWarps = 4;
+#ifndef SSM_BWD_WARPS
+#define SSM_BWD_WARPS 4
+#endif
+constexpr int kWarps = SSM_BWD_WARPS;
 constexpr int kRows = 2 * kWarps;          // rows per CTA
 constexpr int kLd = kBlk + 4;              // fp32 row stride: the 16 state rows on distinct banks
 constexpr int kRowArrays = 5;              // delta, u, dout, z, y (y: forward output before the gate)
@@ -397,9 +400,9 @@ scan_bwd_kernel(const ScanArgs p) {
       reinterpret_cast<float4*>(Xa)[q] = make_float4(dc0.x, dc0.y, dc1.x, dc1.y);
     }
     __syncthreads();  // every row's dB / dC terms are in X; tiles and per-token arrays are free
-    // CTA sum over its 8 rows; one float4 atomic per 4 tokens of dB / dC
+    // CTA sum over its rows; one float4 atomic per 4 tokens of dB / dC
 #pragma unroll
-    for (int it = 0; it < 2; ++it) {
+    for (int it = 0; it < 256 / (kWarps * 32); ++it) {
       const int item = threadIdx.x + it * (kWarps * 32);
       const int arr = item >> 7, m = (item >> 3) & 15, q = item & 7;
       float4 v[2 * kWarps];
@@ -455,6 +458,9 @@ scan_bwd_kernel(const ScanArgs p) {
   // per-(row, split) partials of dA, dD and the delta-bias gradient
   const size_t ps = rowid * p.nsplits + split;
   if (nval) p.part_dA[ps * N + n] = dA2.x + dA2.y;
+  // the state before token 0 enters only through a_0 h_{-1}: its gradient is
+  // the carry a_0 g_0 left after the first block
+  if (split == 0 && nval && p.dh0) p.dh0[rowid * N + n] = Gn;
 #pragma unroll
   for (int off = 8; off > 0; off >>= 1) {
     dDp += __shfl_xor_sync(kFull, dDp, off);

@@ -145,6 +145,10 @@ scan_fwd_kernel(const ScanArgs p) {
     float2 h0 = f2(0.0f, 0.0f);
     if (!SUMMARY && split > 0 && active && lane < NP)
       h0 = reinterpret_cast<const float2*>(p.split_in)[(rowid * p.nsplits + split) * NP + lane];
+    if (!SUMMARY && split == 0 && active && p.h0) {  // the state before token 0
+      if (2 * lane < N) h0.x = __ldg(p.h0 + rowid * N + 2 * lane);
+      if (2 * lane + 1 < N) h0.y = __ldg(p.h0 + rowid * N + 2 * lane + 1);
+    }
     sm.H[warp][lane] = h0;
     sm.P[warp][lane] = f2(1.0f, 1.0f);
   }
@@ -259,13 +263,14 @@ scan_fwd_kernel(const ScanArgs p) {
   }
 }
 
-// Carry into split s: h_in[0] = 0, h_in[s+1] = P[s] h_in[s] + H[s].
+// Carry into split s: h_in[0] = h0 (0 when absent), h_in[s+1] = P[s] h_in[s] + H[s].
 __global__ void fwd_split_carry_kernel(const float* __restrict__ P, const float* __restrict__ H,
-                                       float* __restrict__ hin, int rows, int nsplits, int Np) {
+                                       const float* __restrict__ h0, float* __restrict__ hin,
+                                       int rows, int nsplits, int Np, int N) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= rows * Np) return;
   const int r = i / Np, n = i % Np;
-  float h = 0.0f;
+  float h = (h0 && n < N) ? h0[(size_t)r * N + n] : 0.0f;
   for (int s = 0; s < nsplits; ++s) {
     const size_t k = ((size_t)r * nsplits + s) * Np + n;
     hin[k] = h;
@@ -308,8 +313,8 @@ cudaError_t fwd_t(const ScanArgs& a, cudaStream_t s) {
     dim3 g1((a.D + G - 1) / G, a.B, a.nsplits - 1);
     scan_fwd_kernel<T, G, VEC, true, NT><<<g1, block, smem, s>>>(a);
     const int n = a.B * a.D * a.Npad;
-    fwd_split_carry_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.split_P, a.split_H, a.split_in,
-                                                          a.B * a.D, a.nsplits, a.Npad);
+    fwd_split_carry_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.split_P, a.split_H, a.h0, a.split_in,
+                                                          a.B * a.D, a.nsplits, a.Npad, a.N);
   }
   dim3 g2((a.D + G - 1) / G, a.B, a.nsplits);
   scan_fwd_kernel<T, G, VEC, false, NT><<<g2, block, smem, s>>>(a);

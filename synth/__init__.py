@@ -214,3 +214,50 @@ def random_segments(rng: np.random.Generator, B: int, L: int, n_bound: int,
             prev = c
         seq[b, prev:] = cur
     return seq
+
+
+def initial_state(B: int, D: int, N: int, seed: int, scale: float = 0.5) -> np.ndarray:
+    """A state before token 0, float32 [B, D, N] ~ scale * N(0, 1)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return (scale * rng.standard_normal((B, D, N), dtype=np.float32)).astype(np.float32)
+
+
+@dataclass
+class DecodeInputs:
+    """Inputs of `steps` consecutive tokens of the recurrent form.
+
+    Per-token activations are [steps, B, D] (x, delta, z) and [steps, B, N]
+    (Bm, Cm); the starting conv window is [B, D, 3] (activation dtype) and the
+    starting state [B, D, N] float32."""
+    x: Tensor
+    delta: Tensor
+    z: Tensor
+    Bm: Tensor
+    Cm: Tensor
+    conv_state: Tensor
+    h0: np.ndarray
+    A: np.ndarray
+    Dskip: np.ndarray
+    delta_bias: np.ndarray
+    conv_w: np.ndarray
+    conv_b: np.ndarray
+
+
+def decode_inputs(B: int, D: int, N: int, steps: int, dtype: str, seed: int) -> DecodeInputs:
+    """Seeded inputs for a run of decode steps, with the value distributions
+    of `make_inputs` (A = -(n+1), softplus-inverse delta bias) plus a nonzero
+    conv bias, random D, a random starting conv window and starting state."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    conv_w = rng.uniform(-0.5, 0.5, size=(D, 4)).astype(np.float32)
+    conv_b = rng.uniform(-0.2, 0.2, size=D).astype(np.float32)
+    A = -np.tile(np.arange(1, N + 1, dtype=np.float32), (D, 1))
+    Dskip = rng.uniform(0.5, 1.5, size=D).astype(np.float32)
+    delta_bias = np.log(np.expm1(rng.uniform(1e-3, 1e-1, size=D))).astype(np.float32)
+    x = _act(rng, (steps, B, D), dtype)
+    z = _act(rng, (steps, B, D), dtype)
+    delta = _act(rng, (steps, B, D), dtype, 0.5)
+    Bm = _act(rng, (steps, B, N), dtype)
+    Cm = _act(rng, (steps, B, N), dtype)
+    conv_state = _act(rng, (B, D, 3), dtype)
+    h0 = (0.5 * rng.standard_normal((B, D, N), dtype=np.float32)).astype(np.float32)
+    return DecodeInputs(x, delta, z, Bm, Cm, conv_state, h0, A, Dskip, delta_bias, conv_w, conv_b)

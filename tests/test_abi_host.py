@@ -32,7 +32,7 @@ def test_header_declares_expected_entry_points():
     names = _declared()
     for n in ("ssm_conv1d_fwd", "ssm_conv1d_bwd", "ssm_conv1d_bwd_workspace_size",
               "ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_scan_bwd", "ssm_last_error",
-              "ssm_abi_version"):
+              "ssm_abi_version", "ssm_decode_step", "ssm_scan_status"):
         assert n in names
 
 
@@ -69,8 +69,10 @@ def test_workspace_size_layout(ssm):
     p = _params(ssm, n_splits=1)
     n1 = ssm.ssm_scan_workspace_size(p)
     nchunks = (1000 + 255) // 256
-    ckpt = 2 * 8 * nchunks * 16 * 4
+    ckpt = 2 * 8 * nchunks * 8 * 16 * 4  # the state entering every 32-token block
     assert n1 >= ckpt
+    # with a gate, y before the gate is kept for the backward (bf16 here)
+    assert ssm.ssm_scan_workspace_size(_params(ssm, n_splits=1, z=1 << 20)) >= n1 + 2 * 8 * 1000 * 2
     p2 = _params(ssm, n_splits=3)
     assert ssm.ssm_scan_workspace_size(p2) > n1
     assert ssm.ssm_conv1d_bwd_workspace_size(2, 8, 1000, 4) >= 2 * 8 * 5 * 4
@@ -151,3 +153,42 @@ def test_binding_rejects_cpu_tensors(ssm):
     w = torch.zeros(2, 4)
     with pytest.raises(ValueError):
         ssm.conv1d_fwd(x, w)
+
+
+def _decode_params(ssm, **kw):
+    fake = 1 << 20
+    p = ssm.ssm_decode_params()
+    p.struct_size = ctypes.sizeof(ssm.ssm_decode_params)
+    p.B, p.D, p.N, p.W = 2, 8, 16, 4
+    p.dtype = 1
+    p.delta_softplus = 1
+    p.x, p.conv_state, p.conv_w, p.delta = fake, fake + 4096, fake + 8192, fake + 12288
+    p.Bm, p.Cm, p.A, p.state = fake + 16384, fake + 20480, fake + 24576, fake + 28672
+    p.out = fake + 32768
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("struct_size", 3, 1), ("B", 0, 1), ("D", 0, 1), ("N", 0, 1), ("N", 17, 2), ("W", 3, 2),
+    ("dtype", 7, 1), ("x", None, 1), ("state", None, 1), ("out", None, 1),
+    ("out", 1 << 20, 1),            # aliases x
+    ("state", (1 << 20) + 2, 1),    # fp32 state misaligned
+    ("x", (1 << 20) + 1, 1),        # bf16 activation misaligned
+])
+def test_decode_param_validation(ssm, field, value, status):
+    """Every check fails before a launch (the fake pointers are never touched)."""
+    p = _decode_params(ssm, **{field: value})
+    assert ssm.ssm_decode_step(p, None) == status
+    assert ssm.ssm_last_error()
+
+
+def test_decode_null_params(ssm):
+    assert ssm.ssm_decode_step(None, None) == 1
+
+
+def test_grads_struct_has_initial_state_gradient(ssm):
+    names = [f[0] for f in ssm.ssm_scan_grads._fields_]
+    assert names[-1] == "dinitial_state"
+    assert [f[0] for f in ssm.ssm_scan_params._fields_][-1] == "initial_state"

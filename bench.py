@@ -287,6 +287,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-decode", action="store_true", help="skip the recurrent-step measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -402,6 +403,9 @@ def main():
     if not args.no_e2e:
         line["e2e"] = e2e(layers, device, args, world)
 
+    if not args.no_decode:
+        line["decode"] = decode_bench(device, sh, pk)
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = cpu_count()
         v, rows, secs = oracle_sample(inps[0], args.cpu_seconds, threads)
@@ -416,7 +420,70 @@ def main():
     return 0
 
 
-def e2e(layers, device, args, world):
+def decode_bench(device, sh, pk, rows_b=2048, steps=200, graph_steps=50):
+    """The recurrent one-token step at the bench layer's width: `rows_b`
+    sequences x D channels x N states (bf16 activations, fp32 state). The
+    state (rows_b*D*N*4 bytes, 201 MB at 2048 x 1536 x 16) exceeds the 126 MB
+    L2, so every step reads and writes it in HBM. Timed two ways with CUDA
+    events: back-to-back launches, and a CUDA graph of `graph_steps` steps
+    (kernel time without launch gaps)."""
+    import torch
+    import selective_state_space_35_b200 as ssm
+    D, N = sh.D, sh.N
+    di = synth.decode_inputs(rows_b, D, N, 1, "bf16", synth.seed_for(9))
+
+    def bf(t):
+        return torch.from_numpy(t.bits.view(np.int16).copy()).view(torch.bfloat16).to(device)
+
+    def f32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+
+    x, dl, z, Bm, Cm = bf(di.x)[0], bf(di.delta)[0], bf(di.z)[0], bf(di.Bm)[0], bf(di.Cm)[0]
+    cs, st = bf(di.conv_state), f32(di.h0)
+    A, w, cb, Dk, db = (f32(di.A), f32(di.conv_w), f32(di.conv_b), f32(di.Dskip),
+                        f32(di.delta_bias))
+    out = torch.empty_like(x)
+
+    def step():
+        ssm.decode_step(x, cs, w, dl, A, Bm, Cm, st, conv_bias=cb, z=z, Dskip=Dk,
+                        delta_bias=db, out=out)
+
+    for _ in range(20):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    us_launch = e0.elapsed_time(e1) / steps * 1e3
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(graph_steps):
+            step()
+    g.replay()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(4):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    us_graph = e0.elapsed_time(e1) / (4 * graph_steps) * 1e3
+    del g
+    e_sz, rows = 2, rows_b * D
+    # state read + write; x, delta, z, out and the 3-token window read + write
+    # per row; B and C per sequence; A, conv weight and bias, D, delta bias
+    nbytes = (rows * N * 4 * 2 + rows * e_sz * 10 + rows_b * N * e_sz * 2 + D * N * 4
+              + D * 4 * 4 + 3 * D * 4)
+    gbs = nbytes / (us_graph * 1e-6) / 1e9
+    return {"workload": f"recurrent step, {rows_b} sequences x D{D} x N{N}, bf16 activations, "
+                        f"fp32 state ({rows * N * 4 / 1e6:.0f} MB > L2)",
+            "us_per_step": us_launch, "us_per_step_graph": us_graph,
+            "tokens_per_s": rows_b / (us_graph * 1e-6), "bytes_per_step": nbytes,
+            "hbm_gbs": gbs, "hbm_frac_of_measured": gbs / pk["hbm_gbs"],
+            "launches": steps + 20 + 5 * graph_steps}
+
     import torch
     import torch.distributed as dist
     bf = torch.bfloat16

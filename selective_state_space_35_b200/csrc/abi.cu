@@ -431,6 +431,8 @@ ssm_status_t ssm_decode_step(const ssm_decode_params* p, ssm_stream_t stream) {
   a.delta_bias = p->delta_bias; a.state = p->state; a.out = p->out; a.u_out = p->u_out;
   a.B = p->B; a.D = p->D; a.N = p->N; a.softplus = p->delta_softplus ? 1 : 0;
   a.bf16 = p->dtype == SSM_DTYPE_BF16;
+  a.vec = p->N == 16 && aligned(p->state, 16) && aligned(p->A, 16) && aligned(p->Bm, 4 * es) &&
+          aligned(p->Cm, 4 * es);
   return cuda_status(ssm::launch_decode_step(a, reinterpret_cast<cudaStream_t>(stream)),
                      "ssm_decode_step launch");
 }

@@ -8,9 +8,11 @@
 //   h_n <- exp(dt A_n) h_n + dt B_n u,  y = sum_n C_n h_n + D u,  out = y silu(z)
 //
 // HBM-bound: per (b, d) the state is read and written once (8 N bytes) plus a
-// few activation values. 16 threads per (b, d), one per state: the state
-// row is one coalesced 64-byte access, the per-(b, d) scalar work is done by
-// all 16 threads on broadcast loads, and y is a 16-lane shuffle sum.
+// few activation values. 4 threads per (b, d), 4 states each: the state row
+// is one coalesced 16-byte access per thread, the per-(b, d) scalar work
+// (conv, SiLU, softplus) is shared by only 4 threads, and y is a 4-lane
+// shuffle sum. exp, softplus and sigmoid use the same SFU forms as the
+// sequence kernels.
 #include "common.cuh"
 #include "internal.h"
 
@@ -19,58 +21,102 @@ namespace ssm {
 namespace {
 
 constexpr int kDecThreads = 256;
-constexpr int kGroup = 16;  // threads per (b, d)
+constexpr int kPerRow = 4;   // threads per (b, d)
+constexpr int kPerThr = 4;   // states per thread
 
 template <typename T>
 __device__ __forceinline__ float ldf(const T* p, size_t i) {
   return Io<T>::ld(p + i);
 }
 
-template <typename T>
+// Four consecutive values of Bm / Cm (VEC: one 8- or 16-byte load).
+template <typename T, bool VEC>
+__device__ __forceinline__ float4 ld4(const T* p, int n0, int N) {
+  if (VEC) {
+    if (sizeof(T) == 2) {
+      const uint2 r = __ldg(reinterpret_cast<const uint2*>(p + n0));
+      return make_float4(bf16lo(r.x), bf16hi(r.x), bf16lo(r.y), bf16hi(r.y));
+    }
+    return __ldg(reinterpret_cast<const float4*>(p + n0));
+  }
+  float v[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = (n0 + i < N) ? ldf(p, n0 + i) : 0.0f;
+  return make_float4(v[0], v[1], v[2], v[3]);
+}
+
+// VEC: N == 16 and the state, A, Bm, Cm pointers allow 16-byte (8-byte for
+// bf16 Bm / Cm) vector accesses.
+template <typename T, bool VEC>
 __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(const DecodeArgs a) {
-  const size_t g = (size_t)blockIdx.x * (kDecThreads / kGroup) + threadIdx.x / kGroup;
-  const int n = threadIdx.x % kGroup;
+  const size_t g = (size_t)blockIdx.x * (kDecThreads / kPerRow) + threadIdx.x / kPerRow;
+  const int q = threadIdx.x % kPerRow;
   const size_t rows = (size_t)a.B * a.D;
-  if (g >= rows) return;  // whole 16-lane groups leave together
+  if (g >= rows) return;  // whole 4-lane groups leave together
   const int d = (int)(g % a.D);
   const int b = (int)(g / a.D);
-  const unsigned gmask = 0xffffu << (threadIdx.x & 16);  // this group's half of the warp
+  const int N = a.N;
+  const unsigned qmask = 0xfu << (threadIdx.x & 28);  // this group's 4 lanes
 
   const T* x = static_cast<const T*>(a.x);
   T* win = static_cast<T*>(a.conv_state) + g * 3;
   const float* w = a.conv_w + (size_t)d * 4;
-  const float x0 = ldf(win, 0), x1 = ldf(win, 1), x2 = ldf(win, 2), xt = ldf(x, g);
   float c = a.conv_bias ? __ldg(a.conv_bias + d) : 0.0f;
-  c = fmaf(__ldg(w + 0), x0, c);
-  c = fmaf(__ldg(w + 1), x1, c);
-  c = fmaf(__ldg(w + 2), x2, c);
-  c = fmaf(__ldg(w + 3), xt, c);
-  const float u = c * sigmoidf_(c);
+  c = fmaf(__ldg(w + 0), ldf(win, 0), c);
+  c = fmaf(__ldg(w + 1), ldf(win, 1), c);
+  c = fmaf(__ldg(w + 2), ldf(win, 2), c);
+  c = fmaf(__ldg(w + 3), ldf(x, g), c);
+  const float u = c * sigmoid_fast(c);
   const float v = ldf(static_cast<const T*>(a.delta), g) + (a.delta_bias ? __ldg(a.delta_bias + d) : 0.0f);
-  const float dt = a.softplus ? softplusf_(v) : v;
+  const float dt = a.softplus ? softplus_sfu(v) : v;
+  const float dtl = dt * kLog2e, dtu = dt * u;
 
+  const int n0 = kPerThr * q;
   float hy = 0.0f;
-  if (n < a.N) {
-    float* hp = a.state + g * a.N + n;
-    const float An = __ldg(a.A + (size_t)d * a.N + n);
-    const float Bn = ldf(static_cast<const T*>(a.Bm), (size_t)b * a.N + n);
-    const float Cn = ldf(static_cast<const T*>(a.Cm), (size_t)b * a.N + n);
-    const float h = fmaf(expf(dt * An), *hp, dt * Bn * u);
-    *hp = h;
-    hy = Cn * h;
-  }
+  if (n0 < N) {
+    float* hp = a.state + g * N + n0;
+    const float* Ap = a.A + (size_t)d * N + n0;
+    const float4 Bv = ld4<T, VEC>(static_cast<const T*>(a.Bm) + (size_t)b * N, n0, N);
+    const float4 Cv = ld4<T, VEC>(static_cast<const T*>(a.Cm) + (size_t)b * N, n0, N);
+    float h[4], Av[4];
+    if (VEC) {
+      const float4 h4 = *reinterpret_cast<const float4*>(hp);
+      const float4 A4 = __ldg(reinterpret_cast<const float4*>(Ap));
+      h[0] = h4.x; h[1] = h4.y; h[2] = h4.z; h[3] = h4.w;
+      Av[0] = A4.x; Av[1] = A4.y; Av[2] = A4.z; Av[3] = A4.w;
+    } else {
 #pragma unroll
-  for (int off = kGroup / 2; off > 0; off >>= 1) hy += __shfl_xor_sync(gmask, hy, off);
+      for (int i = 0; i < 4; ++i) {
+        h[i] = (n0 + i < N) ? hp[i] : 0.0f;
+        Av[i] = (n0 + i < N) ? __ldg(Ap + i) : 0.0f;
+      }
+    }
+    const float bv[4] = {Bv.x, Bv.y, Bv.z, Bv.w}, cv[4] = {Cv.x, Cv.y, Cv.z, Cv.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      h[i] = fmaf(ex2_approx(dtl * Av[i]), h[i], dtu * bv[i]);
+      hy = fmaf(cv[i], h[i], hy);
+    }
+    if (VEC) {
+      *reinterpret_cast<float4*>(hp) = make_float4(h[0], h[1], h[2], h[3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (n0 + i < N) hp[i] = h[i];
+    }
+  }
+  hy += __shfl_xor_sync(qmask, hy, 1);
+  hy += __shfl_xor_sync(qmask, hy, 2);
 
-  if (n == 0) {
-    float y = hy + (a.Dskip ? __ldg(a.Dskip + d) : 0.0f) * u;
+  if (q == 0) {
+    float y = fmaf(a.Dskip ? __ldg(a.Dskip + d) : 0.0f, u, hy);
     if (a.z) {
       const float zz = ldf(static_cast<const T*>(a.z), g);
-      y *= zz * sigmoidf_(zz);
+      y *= zz * sigmoid_fast(zz);
     }
     Io<T>::st(static_cast<T*>(a.out) + g, y);
     if (a.u_out) Io<T>::st(static_cast<T*>(a.u_out) + g, u);
-    // the window moves by one token (the inputs are stored values: no rounding)
+    // the window moves by one token (stored input values: no rounding)
     win[0] = win[1];
     win[1] = win[2];
     win[2] = x[g];
@@ -81,12 +127,15 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(const DecodeAr
 
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s) {
   const size_t rows = (size_t)a.B * a.D;
-  const size_t per_cta = kDecThreads / kGroup;
+  const size_t per_cta = kDecThreads / kPerRow;
   const unsigned grid = (unsigned)((rows + per_cta - 1) / per_cta);
-  if (a.bf16)
-    decode_step_kernel<__nv_bfloat16><<<grid, kDecThreads, 0, s>>>(a);
-  else
-    decode_step_kernel<float><<<grid, kDecThreads, 0, s>>>(a);
+  if (a.bf16) {
+    if (a.vec) decode_step_kernel<__nv_bfloat16, true><<<grid, kDecThreads, 0, s>>>(a);
+    else decode_step_kernel<__nv_bfloat16, false><<<grid, kDecThreads, 0, s>>>(a);
+  } else {
+    if (a.vec) decode_step_kernel<float, true><<<grid, kDecThreads, 0, s>>>(a);
+    else decode_step_kernel<float, false><<<grid, kDecThreads, 0, s>>>(a);
+  }
   return cudaGetLastError();
 }
 

@@ -98,6 +98,7 @@ struct DecodeArgs {
   void* u_out;
   int B, D, N, softplus;
   bool bf16;
+  bool vec;  // N == 16 with 16-byte aligned state / A and vector-aligned Bm / Cm
 };
 
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s);

@@ -176,6 +176,23 @@ ssm_status_t ssm_scan_workspace_size(const ssm_scan_params* p, size_t* bytes);
  * keep the workspace unchanged between ssm_scan_fwd and ssm_scan_bwd. */
 ssm_status_t ssm_scan_fwd(const ssm_scan_params* p, ssm_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * ssm_conv1d_scan_fwd — ssm_conv1d_fwd (W = 4, SiLU on) and ssm_scan_fwd in
+ * one kernel: the pages' kernel fusion ("hung-phan ml-skills mamba",
+ * "Hardware-Aware Parallel Scan") applied to the conv and SiLU of "Mamba:
+ * Selective State Spaces (S6)". Reads x [B][D][L] (dtype p->dtype),
+ * conv_w [D][4] and conv_bias [D] (nullable); the conv taps follow p's
+ * document ids (a tap in another document reads 0). Computes u =
+ * silu(conv(x)) inside the scan, WRITES it to p->u (writable device memory,
+ * not aliasing x: ssm_scan_bwd reads it, and it is the conv output a caller
+ * differentiates with ssm_conv1d_bwd), and writes everything ssm_scan_fwd
+ * writes. u, out, final_state and the workspace are bitwise equal to those of
+ * ssm_conv1d_fwd followed by ssm_scan_fwd. Errors as ssm_scan_fwd, plus
+ * SSM_ERR_INVALID_ARG for a NULL x / conv_w, x == p->u, or misalignment.
+ * ------------------------------------------------------------------------ */
+ssm_status_t ssm_conv1d_scan_fwd(const ssm_scan_params* p, const void* x, const float* conv_w,
+                                 const float* conv_bias, ssm_stream_t stream);
+
 typedef struct {
     size_t struct_size;        /* = sizeof(ssm_scan_grads) */
     const void* dout;          /* [B][D][L] dtype, dL/dout */

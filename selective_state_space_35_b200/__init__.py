@@ -14,7 +14,8 @@ import ctypes
 from . import _lib
 from ._lib import (SsmError, ssm_abi_version, ssm_conv1d_bwd, ssm_conv1d_bwd_noalloc,
                    ssm_conv1d_bwd_workspace_size,
-                   ssm_conv1d_fwd, ssm_decode_params, ssm_decode_step, ssm_last_error,
+                   ssm_conv1d_fwd, ssm_conv1d_scan_fwd, ssm_decode_params, ssm_decode_step,
+                   ssm_last_error,
                    ssm_probe_ex2_rate, ssm_scan_bwd, ssm_scan_status,
                    ssm_scan_fwd, ssm_scan_grads, ssm_scan_params, ssm_scan_workspace_size)
 
@@ -24,7 +25,8 @@ __all__ = [
     "ssm_scan_params", "ssm_scan_grads", "ssm_probe_ex2_rate", "probe_ex2_rate", "ssm_scan_status",
     "scan_status", "conv1d_fwd", "conv1d_bwd", "scan_params",
     "scan_workspace_size", "scan_fwd", "scan_bwd", "load",
-    "ssm_decode_params", "ssm_decode_step", "decode_step",
+    "ssm_decode_params", "ssm_decode_step", "decode_step", "ssm_conv1d_scan_fwd",
+    "conv1d_scan_fwd",
 ]
 
 load = _lib.load
@@ -199,6 +201,40 @@ def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softpl
     p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
     _lib.check(ssm_scan_fwd(p, _stream(stream, u.device)))
     return out, fs, workspace
+
+
+def conv1d_scan_fwd(x, conv_w, conv_bias, delta, A, Bm, Cm, *, z=None, Dskip=None,
+                    delta_bias=None, softplus=True, seq_idx=None, cu_seqlens=None, n_splits=0,
+                    return_final_state=False, u=None, out=None, workspace=None,
+                    initial_state=None, stream=None):
+    """Fused depthwise conv (W = 4) + SiLU + selective scan forward.
+
+    x [B, D, L] is the conv input; conv_w [D, 4], conv_bias [D] or None.
+    Returns (out, u, final_state or None, workspace): u = silu(conv(x)) is
+    written by the kernel (pass it, with `workspace`, to scan_bwd; it is the
+    conv output for conv1d_bwd). Bitwise equal to conv1d_fwd + scan_fwd.
+    """
+    torch = _torch()
+    B, D, L = x.shape
+    N = A.shape[1]
+    _need(x, "x", shape=(B, D, L))
+    _need(conv_w, "conv_w", torch.float32, (D, 4))
+    _need(conv_bias, "conv_bias", torch.float32, (D,))
+    u = torch.empty_like(x) if u is None else u
+    _need(u, "u", x.dtype, (B, D, L))
+    out = torch.empty_like(x) if out is None else out
+    fs = torch.empty((B, D, N), dtype=torch.float32, device=x.device) if return_final_state else None
+    p = scan_params(u, delta, A, Bm, Cm, z=z, Dskip=Dskip, delta_bias=delta_bias, softplus=softplus,
+                    seq_idx=seq_idx, cu_seqlens=cu_seqlens, n_splits=n_splits, out=out,
+                    final_state=fs, initial_state=initial_state)
+    need = ssm_scan_workspace_size(p)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    _lib.check(ssm_conv1d_scan_fwd(p, x.data_ptr(), conv_w.data_ptr(),
+                                   conv_bias.data_ptr() if conv_bias is not None else None,
+                                   _stream(stream, x.device)))
+    return out, u, fs, workspace
 
 
 def scan_bwd(u, delta, A, Bm, Cm, dout, workspace, *, z=None, Dskip=None, delta_bias=None,

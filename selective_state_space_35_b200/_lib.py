@@ -76,7 +76,8 @@ _lib = None
 
 EXPORTS = ("ssm_last_error", "ssm_abi_version", "ssm_conv1d_fwd", "ssm_conv1d_bwd_workspace_size",
            "ssm_conv1d_bwd", "ssm_conv1d_bwd_noalloc", "ssm_scan_workspace_size", "ssm_scan_fwd",
-           "ssm_scan_bwd", "ssm_scan_status", "ssm_probe_ex2_rate", "ssm_decode_step")
+           "ssm_scan_bwd", "ssm_scan_status", "ssm_probe_ex2_rate", "ssm_decode_step",
+           "ssm_conv1d_scan_fwd")
 
 
 def load(path: str | None = None):
@@ -114,6 +115,8 @@ def load(path: str | None = None):
     L.ssm_scan_status.argtypes = [ctypes.POINTER(ssm_scan_params), ctypes.POINTER(_i), _vp]
     L.ssm_probe_ex2_rate.restype = _i
     L.ssm_probe_ex2_rate.argtypes = [_vp, _sz, ctypes.POINTER(ctypes.c_double), _vp]
+    L.ssm_conv1d_scan_fwd.restype = _i
+    L.ssm_conv1d_scan_fwd.argtypes = [ctypes.POINTER(ssm_scan_params), _vp, _vp, _vp, _vp]
     L.ssm_decode_step.restype = _i
     L.ssm_decode_step.argtypes = [ctypes.POINTER(ssm_decode_params), _vp]
     if path is None:
@@ -181,6 +184,10 @@ def ssm_scan_fwd(params: ssm_scan_params, stream) -> int:
 
 def ssm_scan_bwd(params: ssm_scan_params, grads: ssm_scan_grads, stream) -> int:
     return load().ssm_scan_bwd(_ref(params), _ref(grads), stream)
+
+
+def ssm_conv1d_scan_fwd(params: ssm_scan_params, x, conv_w, conv_bias, stream) -> int:
+    return load().ssm_conv1d_scan_fwd(_ref(params), x, conv_w, conv_bias, stream)
 
 
 def ssm_decode_step(params: ssm_decode_params, stream) -> int:

@@ -196,6 +196,37 @@ bool vec_ok(int L, std::initializer_list<const void*> ptrs) {
   return true;
 }
 
+// ssm_scan_fwd, or with x set the fused conv + scan forward that writes u.
+ssm_status_t scan_fwd_impl(const ssm_scan_params* p, const void* x, const float* conv_w,
+                           const float* conv_bias, ssm_stream_t stream) {
+  ssm_status_t st = check_params(p);
+  if (st != SSM_OK) return st;
+  const ScanPlan pl = plan_scan(p);
+  st = check_scan_buffers(p, pl);
+  if (st != SSM_OK) return st;
+  if (x) {
+    if (x == p->u) return fail(SSM_ERR_INVALID_ARG, "u (written) may not alias x");
+    if (!aligned(x, elem_size(p->dtype)) || !aligned(conv_w, 4) ||
+        (conv_bias && !aligned(conv_bias, 4)))
+      return fail(SSM_ERR_INVALID_ARG, "x, conv_w or conv_bias misaligned");
+  }
+  ssm::ScanArgs a;
+  build_args(p, pl, &a);
+  a.xconv = x;
+  a.conv_w = conv_w;
+  a.conv_b = conv_bias;
+  a.vec = vec_ok(p->L, {p->u, p->delta, p->z, p->Bm, p->Cm, p->out, a.seq, x});
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e0 = cudaMemsetAsync(a.status, 0, sizeof(int), s);  // fresh status for this fwd/bwd
+  if (e0 != cudaSuccess) return cuda_status(e0, "scan forward status reset");
+  if (p->cu_seqlens) {
+    cudaError_t e = ssm::launch_cu_seqlens_to_seq(p->cu_seqlens, p->n_docs, p->L,
+                                                  const_cast<int32_t*>(a.seq), s);
+    if (e != cudaSuccess) return cuda_status(e, "cu_seqlens conversion");
+  }
+  return cuda_status(ssm::launch_scan_fwd(a, s), x ? "ssm_conv1d_scan_fwd launch" : "ssm_scan_fwd launch");
+}
+
 }  // namespace
 
 extern "C" {
@@ -318,23 +349,15 @@ ssm_status_t ssm_scan_workspace_size(const ssm_scan_params* p, size_t* bytes) {
 
 ssm_status_t ssm_scan_fwd(const ssm_scan_params* p, ssm_stream_t stream) {
   if (injected("ssm_scan_fwd")) return fail(SSM_ERR_INJECTED, "ssm_scan_fwd: injected failure");
-  ssm_status_t st = check_params(p);
-  if (st != SSM_OK) return st;
-  const ScanPlan pl = plan_scan(p);
-  st = check_scan_buffers(p, pl);
-  if (st != SSM_OK) return st;
-  ssm::ScanArgs a;
-  build_args(p, pl, &a);
-  a.vec = vec_ok(p->L, {p->u, p->delta, p->z, p->Bm, p->Cm, p->out, a.seq});
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e0 = cudaMemsetAsync(a.status, 0, sizeof(int), s);  // fresh status for this fwd/bwd
-  if (e0 != cudaSuccess) return cuda_status(e0, "ssm_scan_fwd status reset");
-  if (p->cu_seqlens) {
-    cudaError_t e = ssm::launch_cu_seqlens_to_seq(p->cu_seqlens, p->n_docs, p->L,
-                                                  const_cast<int32_t*>(a.seq), s);
-    if (e != cudaSuccess) return cuda_status(e, "cu_seqlens conversion");
-  }
-  return cuda_status(ssm::launch_scan_fwd(a, s), "ssm_scan_fwd launch");
+  return scan_fwd_impl(p, nullptr, nullptr, nullptr, stream);
+}
+
+ssm_status_t ssm_conv1d_scan_fwd(const ssm_scan_params* p, const void* x, const float* conv_w,
+                                 const float* conv_bias, ssm_stream_t stream) {
+  if (injected("ssm_conv1d_scan_fwd"))
+    return fail(SSM_ERR_INJECTED, "ssm_conv1d_scan_fwd: injected failure");
+  if (!x || !conv_w) return fail(SSM_ERR_INVALID_ARG, "x and conv_w must be non-NULL");
+  return scan_fwd_impl(p, x, conv_w, conv_bias, stream);
 }
 
 ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,

@@ -59,7 +59,9 @@ conv1d_fwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
       const bool ok = !SEQ || sg[i + k] == sg[i + 3];
       acc = fmaf(wk[k], ok ? xv[i + k] : 0.0f, acc);
     }
-    out[i] = silu ? acc * sigmoidf_(acc) : acc;
+    // SiLU with the SFU sigmoid (the fused conv + scan forward computes the
+    // same expression, so both store identical u)
+    out[i] = silu ? acc * sigmoid_fast(acc) : acc;
   }
   store_row8<T, VEC>(u + row, t0, L, out);
 }

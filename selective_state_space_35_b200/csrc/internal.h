@@ -48,6 +48,11 @@ struct ScanArgs {
   const void* Cm;
   const int32_t* seq;
   const float* h0;    // [B*D][N] state before token 0, nullable
+  // fused conv (forward only): when xconv is set the forward reads x, computes
+  // u = silu(conv(x)) itself and writes it to u (which is then an output)
+  const void* xconv;
+  const float* conv_w;
+  const float* conv_b;
   int softplus;
   // forward outputs
   void* out;

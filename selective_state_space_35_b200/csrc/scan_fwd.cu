@@ -98,12 +98,58 @@ __device__ __forceinline__ void fwd_pair_post(int m, int lane, const float2* __r
   }
 }
 
+// Fused conv: v[8] holds x of the lane's tokens tl .. tl+7 and becomes
+// u = silu(bias + sum_k w_k x_{t-3+k}) (taps in another document read 0),
+// rounded to the storage type T exactly as the separate conv kernel stores
+// it (same operations in the same order, SFU sigmoid), so the fused and
+// separate paths agree bitwise.
+// The 3-token halo comes from the previous lane; lane 0 takes the previous
+// chunk's last three tokens from (c5, c6, c7), which are then advanced.
+template <typename T>
+__device__ __forceinline__ void conv_silu8(float v[8], float& c5, float& c6, float& c7, int lane,
+                                           const float wk[4], float bs,
+                                           const int32_t* __restrict__ seqb, int tl, int L) {
+  float xv[11];
+  xv[0] = __shfl_up_sync(kFull, v[5], 1);
+  xv[1] = __shfl_up_sync(kFull, v[6], 1);
+  xv[2] = __shfl_up_sync(kFull, v[7], 1);
+  if (lane == 0) {
+    xv[0] = c5;
+    xv[1] = c6;
+    xv[2] = c7;
+  }
+  c5 = __shfl_sync(kFull, v[5], 31);
+  c6 = __shfl_sync(kFull, v[6], 31);
+  c7 = __shfl_sync(kFull, v[7], 31);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) xv[3 + i] = v[i];
+  int sg[11];
+  if (seqb) {
+#pragma unroll
+    for (int i = 0; i < 11; ++i) {
+      const int s = tl - 3 + i;
+      sg[i] = (s >= 0 && s < L) ? __ldg(seqb + s) : 0;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float acc = bs;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const bool ok = !seqb || sg[i + k] == sg[i + 3];
+      acc = fmaf(wk[k], ok ? xv[i + k] : 0.0f, acc);
+    }
+    const float uo = acc * sigmoid_fast(acc);
+    v[i] = sizeof(T) == 2 ? __bfloat162float(__float2bfloat16_rn(uo)) : uo;
+  }
+}
+
 // NT: state count fixed at compile time (16), or 0 for any N <= 16.
 #ifndef SSM_FWD_MIN_BLOCKS
 #define SSM_FWD_MIN_BLOCKS 3
 #endif
 
-template <typename T, int G, bool VEC, bool SUMMARY, int NT>
+template <typename T, int G, bool VEC, bool SUMMARY, int NT, bool CONV>
 __global__ void __launch_bounds__(G * 32, SSM_FWD_MIN_BLOCKS)
 scan_fwd_kernel(const ScanArgs p) {
   // bf16 on the vector path: B / C tiles arrive by TMA one chunk ahead
@@ -125,7 +171,8 @@ scan_fwd_kernel(const ScanArgs p) {
 
   const T* Bm = static_cast<const T*>(p.Bm);
   const T* Cm = static_cast<const T*>(p.Cm);
-  const T* u_row = static_cast<const T*>(p.u) + row;
+  // with the fused conv the per-token stream read here is x, and u is written
+  const T* u_row = static_cast<const T*>(CONV ? p.xconv : p.u) + row;
   const T* dl_row = static_cast<const T*>(p.delta) + row;
   const T* z_row = p.z ? static_cast<const T*>(p.z) + row : nullptr;
 
@@ -154,6 +201,19 @@ scan_fwd_kernel(const ScanArgs p) {
   }
   const float Dv = (active && p.Dskip) ? __ldg(p.Dskip + d) : 0.0f;
   const float bias = (active && p.delta_bias) ? __ldg(p.delta_bias + d) : 0.0f;
+  float wk[4] = {0.0f, 0.0f, 0.0f, 0.0f}, cbias = 0.0f, c5 = 0.0f, c6 = 0.0f, c7 = 0.0f;
+  const int32_t* seqb = p.seq ? p.seq + (size_t)b * L : nullptr;
+  if (CONV && active) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) wk[k] = __ldg(p.conv_w + (size_t)d * 4 + k);
+    cbias = p.conv_b ? __ldg(p.conv_b + d) : 0.0f;
+    const int t0 = c_begin * kChunk;  // 0 or >= 256: the halo before it is in range
+    if (t0 > 0) {
+      c5 = Io<T>::ld(u_row + t0 - 3);
+      c6 = Io<T>::ld(u_row + t0 - 2);
+      c7 = Io<T>::ld(u_row + t0 - 1);
+    }
+  }
 
   Tok8<T, VEC> pf_dl, pf_u, pf_z;
   if (active) {
@@ -193,6 +253,10 @@ scan_fwd_kernel(const ScanArgs p) {
       pf_dl.load(dl_row, tl + kChunk, L);
       pf_u.load(u_row, tl + kChunk, L);
       if (!SUMMARY && z_row) pf_z.load(z_row, tl + kChunk, L);
+    }
+    if (CONV) {
+      conv_silu8<T>(uu, c5, c6, c7, lane, wk, cbias, seqb, tl, L);
+      if (!SUMMARY) store_row8<T, VEC>(static_cast<T*>(const_cast<void*>(p.u)) + row, tl, L, uu);
     }
     float2 dd[8], xx[8], y2[8];
 #pragma unroll
@@ -291,47 +355,49 @@ __global__ void cu_seqlens_to_seq_kernel(const int32_t* __restrict__ cu, int n_d
   seq[t] = lo;
 }
 
-template <typename T, int G, bool VEC, bool SUMMARY, int NT>
+template <typename T, int G, bool VEC, bool SUMMARY, int NT, bool CONV>
 cudaError_t fwd_smem_attr() {
   static bool done = false;  // once per instantiation and process (a benign race)
   if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(scan_fwd_kernel<T, G, VEC, SUMMARY, NT>,
+  cudaError_t e = cudaFuncSetAttribute(scan_fwd_kernel<T, G, VEC, SUMMARY, NT, CONV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sizeof(FwdSmem<G>));
   if (e == cudaSuccess) done = true;
   return e;
 }
 
-template <typename T, int G, bool VEC, int NT>
+template <typename T, int G, bool VEC, int NT, bool CONV>
 cudaError_t fwd_t(const ScanArgs& a, cudaStream_t s) {
   dim3 block(G * 32);
   const size_t smem = sizeof(FwdSmem<G>);
-  cudaError_t e = fwd_smem_attr<T, G, VEC, false, NT>();
-  if (e == cudaSuccess && a.nsplits > 1) e = fwd_smem_attr<T, G, VEC, true, NT>();
+  cudaError_t e = fwd_smem_attr<T, G, VEC, false, NT, CONV>();
+  if (e == cudaSuccess && a.nsplits > 1) e = fwd_smem_attr<T, G, VEC, true, NT, CONV>();
   if (e != cudaSuccess) return e;
   if (a.nsplits > 1) {
     dim3 g1((a.D + G - 1) / G, a.B, a.nsplits - 1);
-    scan_fwd_kernel<T, G, VEC, true, NT><<<g1, block, smem, s>>>(a);
+    scan_fwd_kernel<T, G, VEC, true, NT, CONV><<<g1, block, smem, s>>>(a);
     const int n = a.B * a.D * a.Npad;
     fwd_split_carry_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.split_P, a.split_H, a.h0, a.split_in,
                                                           a.B * a.D, a.nsplits, a.Npad, a.N);
   }
   dim3 g2((a.D + G - 1) / G, a.B, a.nsplits);
-  scan_fwd_kernel<T, G, VEC, false, NT><<<g2, block, smem, s>>>(a);
+  scan_fwd_kernel<T, G, VEC, false, NT, CONV><<<g2, block, smem, s>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-template <int NT>
+template <int NT, bool CONV>
 cudaError_t fwd_dispatch(const ScanArgs& a, cudaStream_t s) {
   if (a.bf16)
-    return a.vec ? fwd_t<__nv_bfloat16, 4, true, NT>(a, s) : fwd_t<__nv_bfloat16, 4, false, NT>(a, s);
-  return a.vec ? fwd_t<float, 4, true, NT>(a, s) : fwd_t<float, 4, false, NT>(a, s);
+    return a.vec ? fwd_t<__nv_bfloat16, 4, true, NT, CONV>(a, s)
+                 : fwd_t<__nv_bfloat16, 4, false, NT, CONV>(a, s);
+  return a.vec ? fwd_t<float, 4, true, NT, CONV>(a, s) : fwd_t<float, 4, false, NT, CONV>(a, s);
 }
 
 cudaError_t launch_scan_fwd(const ScanArgs& a, cudaStream_t s) {
-  return a.N == 16 ? fwd_dispatch<16>(a, s) : fwd_dispatch<0>(a, s);
+  if (a.xconv) return a.N == 16 ? fwd_dispatch<16, true>(a, s) : fwd_dispatch<0, true>(a, s);
+  return a.N == 16 ? fwd_dispatch<16, false>(a, s) : fwd_dispatch<0, false>(a, s);
 }
 
 cudaError_t launch_cu_seqlens_to_seq(const int32_t* cu, int n_docs, int L, int32_t* seq,

@@ -192,3 +192,16 @@ def test_grads_struct_has_initial_state_gradient(ssm):
     names = [f[0] for f in ssm.ssm_scan_grads._fields_]
     assert names[-1] == "dinitial_state"
     assert [f[0] for f in ssm.ssm_scan_params._fields_][-1] == "initial_state"
+
+
+def test_fused_forward_validation(ssm):
+    from selective_state_space_35_b200 import _lib
+    fake = 1 << 20
+    p = _params(ssm, u=fake, delta=fake + 4096, A=fake + 8192, Bm=fake + 12288, Cm=fake + 16384,
+                out=fake + 20480, workspace=fake + 65536, workspace_bytes=1 << 30)
+    L = _lib.load()
+    assert L.ssm_conv1d_scan_fwd(ctypes.byref(p), None, fake, None, None) == 1     # no x
+    assert L.ssm_conv1d_scan_fwd(ctypes.byref(p), fake + 40960, None, None, None) == 1  # no w
+    assert L.ssm_conv1d_scan_fwd(ctypes.byref(p), fake, fake + 40960, None, None) == 1  # x == u
+    assert "alias" in ssm.ssm_last_error()
+    assert L.ssm_conv1d_scan_fwd(ctypes.byref(p), fake + 40961, fake + 44000, None, None) == 1

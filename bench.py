@@ -41,9 +41,10 @@ UNIT = "layer-tokens/s"
 SFU_EX2_PER_CLK_PER_SM = 16  # MUFU ex2 throughput per SM per clock
 
 
-# DRAM bytes per launch of the current scan kernels at this workload, from
-# one ncu capture (profiles/scan_kernels_32K_1layer.md); a kernel changed
-# since its capture has no entry.
+# DRAM bytes per launch of the current scan kernels at the 32K bench workload
+# (one layer B2 D1536 N16 L32768 bf16), from
+# one ncu capture (summarised under profiles/); a kernel changed since its
+# capture has no entry.
 NCU_TRAFFIC = {"scan_bwd": 1231155e3 + 595630e3, "scan_fwd": 611286e3 + 561725e3}
 
 
@@ -381,7 +382,7 @@ def main():
     if dom.startswith("scan"):
         achieved = exps / (avg[dom] * 1e-3) / 1e12
         roof = {"bound": "alu", "achieved": achieved, "peak": ex2_peak, "unit": "Tex2/s",
-                "frac": achieved / ex2_peak, "traffic": NCU_TRAFFIC.get(dom),
+                "frac": achieved / ex2_peak, "traffic": NCU_TRAFFIC.get(dom) if cfg == 3 else None,
                 "traffic_unit": "bytes per launch (ncu dram__bytes_read.sum + "
                                 "dram__bytes_write.sum)",
                 "kernel": f"ssm_{dom}",

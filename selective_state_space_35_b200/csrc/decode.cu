@@ -8,10 +8,10 @@
 //   h_n <- exp(dt A_n) h_n + dt B_n u,  y = sum_n C_n h_n + D u,  out = y silu(z)
 //
 // HBM-bound: per (b, d) the state is read and written once (8 N bytes) plus a
-// few activation values. 4 threads per (b, d), 4 states each: the state row
-// is one coalesced 16-byte access per thread, the per-(b, d) scalar work
-// (conv, SiLU, softplus) is shared by only 4 threads, and y is a 4-lane
-// shuffle sum. exp, softplus and sigmoid use the same SFU forms as the
+// few activation values. kPerRow threads per (b, d), kNMax / kPerRow states
+// each in 16-byte pieces: the state row is read with coalesced 16-byte
+// accesses, the per-(b, d) scalar work (conv, SiLU, softplus) is repeated by
+// only kPerRow threads, and y is a kPerRow-lane shuffle sum. exp, softplus and sigmoid use the same SFU forms as the
 // sequence kernels.
 #include "common.cuh"
 #include "internal.h"
@@ -20,9 +20,12 @@ namespace ssm {
 
 namespace {
 
+#ifndef SSM_DECODE_THREADS_PER_ROW
+#define SSM_DECODE_THREADS_PER_ROW 2
+#endif
 constexpr int kDecThreads = 256;
-constexpr int kPerRow = 4;   // threads per (b, d)
-constexpr int kPerThr = 4;   // states per thread
+constexpr int kPerRow = SSM_DECODE_THREADS_PER_ROW;  // threads per (b, d): 1, 2 or 4
+constexpr int kPerThr = kNMax / kPerRow;             // states per thread
 
 template <typename T>
 __device__ __forceinline__ float ldf(const T* p, size_t i) {
@@ -56,7 +59,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(const DecodeAr
   const int d = (int)(g % a.D);
   const int b = (int)(g / a.D);
   const int N = a.N;
-  const unsigned qmask = 0xfu << (threadIdx.x & 28);  // this group's 4 lanes
+  // this row's kPerRow lanes
+  const unsigned qmask = ((1u << kPerRow) - 1u) << (threadIdx.x & (32 - kPerRow));
 
   const T* x = static_cast<const T*>(a.x);
   T* win = static_cast<T*>(a.conv_state) + g * 3;
@@ -71,42 +75,45 @@ __global__ void __launch_bounds__(kDecThreads) decode_step_kernel(const DecodeAr
   const float dt = a.softplus ? softplus_sfu(v) : v;
   const float dtl = dt * kLog2e, dtu = dt * u;
 
-  const int n0 = kPerThr * q;
   float hy = 0.0f;
-  if (n0 < N) {
-    float* hp = a.state + g * N + n0;
-    const float* Ap = a.A + (size_t)d * N + n0;
-    const float4 Bv = ld4<T, VEC>(static_cast<const T*>(a.Bm) + (size_t)b * N, n0, N);
-    const float4 Cv = ld4<T, VEC>(static_cast<const T*>(a.Cm) + (size_t)b * N, n0, N);
-    float h[4], Av[4];
-    if (VEC) {
-      const float4 h4 = *reinterpret_cast<const float4*>(hp);
-      const float4 A4 = __ldg(reinterpret_cast<const float4*>(Ap));
-      h[0] = h4.x; h[1] = h4.y; h[2] = h4.z; h[3] = h4.w;
-      Av[0] = A4.x; Av[1] = A4.y; Av[2] = A4.z; Av[3] = A4.w;
-    } else {
+#pragma unroll
+  for (int j = 0; j < kPerThr / 4; ++j) {  // groups of 4 states
+    const int n0 = kPerThr * q + 4 * j;
+    if (n0 < N) {
+      float* hp = a.state + g * N + n0;
+      const float* Ap = a.A + (size_t)d * N + n0;
+      const float4 Bv = ld4<T, VEC>(static_cast<const T*>(a.Bm) + (size_t)b * N, n0, N);
+      const float4 Cv = ld4<T, VEC>(static_cast<const T*>(a.Cm) + (size_t)b * N, n0, N);
+      float h[4], Av[4];
+      if (VEC) {
+        const float4 h4 = *reinterpret_cast<const float4*>(hp);
+        const float4 A4 = __ldg(reinterpret_cast<const float4*>(Ap));
+        h[0] = h4.x; h[1] = h4.y; h[2] = h4.z; h[3] = h4.w;
+        Av[0] = A4.x; Av[1] = A4.y; Av[2] = A4.z; Av[3] = A4.w;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          h[i] = (n0 + i < N) ? hp[i] : 0.0f;
+          Av[i] = (n0 + i < N) ? __ldg(Ap + i) : 0.0f;
+        }
+      }
+      const float bv[4] = {Bv.x, Bv.y, Bv.z, Bv.w}, cv[4] = {Cv.x, Cv.y, Cv.z, Cv.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        h[i] = (n0 + i < N) ? hp[i] : 0.0f;
-        Av[i] = (n0 + i < N) ? __ldg(Ap + i) : 0.0f;
+        h[i] = fmaf(ex2_approx(dtl * Av[i]), h[i], dtu * bv[i]);
+        hy = fmaf(cv[i], h[i], hy);
+      }
+      if (VEC) {
+        *reinterpret_cast<float4*>(hp) = make_float4(h[0], h[1], h[2], h[3]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (n0 + i < N) hp[i] = h[i];
       }
     }
-    const float bv[4] = {Bv.x, Bv.y, Bv.z, Bv.w}, cv[4] = {Cv.x, Cv.y, Cv.z, Cv.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      h[i] = fmaf(ex2_approx(dtl * Av[i]), h[i], dtu * bv[i]);
-      hy = fmaf(cv[i], h[i], hy);
-    }
-    if (VEC) {
-      *reinterpret_cast<float4*>(hp) = make_float4(h[0], h[1], h[2], h[3]);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        if (n0 + i < N) hp[i] = h[i];
-    }
   }
-  hy += __shfl_xor_sync(qmask, hy, 1);
-  hy += __shfl_xor_sync(qmask, hy, 2);
+#pragma unroll
+  for (int off = 1; off < kPerRow; off <<= 1) hy += __shfl_xor_sync(qmask, hy, off);
 
   if (q == 0) {
     float y = fmaf(a.Dskip ? __ldg(a.Dskip + d) : 0.0f, u, hy);

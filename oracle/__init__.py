@@ -31,10 +31,10 @@ def lib():
         L.oracle_round_bf16.argtypes = [dp, dp, sz]
         L.oracle_conv1d_fwd.argtypes = [dp, dp, dp, ip, dp, dp, i, i, i, i, i]
         L.oracle_conv1d_bwd.argtypes = [dp, dp, dp, ip, dp, dp, dp, dp, i, i, i, i, i]
-        L.oracle_scan_fwd.argtypes = [dp] * 8 + [i, ip, dp, dp, dp, dp, i, i, i, i]
-        L.oracle_scan_bwd.argtypes = [dp] * 8 + [i, ip] + [dp] * 11 + [i, i, i, i]
-        L.oracle_scan_fwd_mt.argtypes = [dp] * 8 + [i, ip, dp, dp, dp, dp, i, i, i, i, i]
-        L.oracle_scan_bwd_mt.argtypes = [dp] * 8 + [i, ip] + [dp] * 11 + [i, i, i, i, i]
+        L.oracle_scan_fwd.argtypes = [dp] * 8 + [i, i, ip, dp, dp, dp, dp, i, i, i, i]
+        L.oracle_scan_bwd.argtypes = [dp] * 8 + [i, i, ip] + [dp] * 11 + [i, i, i, i]
+        L.oracle_scan_fwd_mt.argtypes = [dp] * 8 + [i, i, ip, dp, dp, dp, dp, i, i, i, i, i]
+        L.oracle_scan_bwd_mt.argtypes = [dp] * 8 + [i, i, ip] + [dp] * 11 + [i, i, i, i, i]
         L.oracle_decode_step.argtypes = [dp] * 11 + [i] + [dp] * 3 + [i, i, i, i]
         for f in ("oracle_round_bf16", "oracle_conv1d_fwd", "oracle_conv1d_bwd",
                   "oracle_scan_fwd", "oracle_scan_bwd", "oracle_scan_fwd_mt",
@@ -105,12 +105,13 @@ def conv1d_bwd(x, w, bias, seq_idx, du, silu=True):
 
 
 def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None,
-             softplus=True, seq_idx=None, h0=None, nthreads=1):
+             softplus=True, seq_idx=None, h0=None, zoh=False, nthreads=1):
     """Selective scan forward. Returns dict(out, y, final_state).
 
     u, delta, z: [B, D, L]; A: [D, N]; Bm, Cm: [B, N, L]; Dskip,
     delta_bias: [D] or None; seq_idx: [B, L] or None; h0: [B, D, N] state
-    before token 0, or None for zero.
+    before token 0, or None for zero. zoh: zero-order-hold B_bar
+    ((exp(dt A) - 1) / A B) instead of dt B.
     """
     u, delta, z, A = _f64(u), _f64(delta), _f64(z), _f64(A)
     Dskip, delta_bias, Bm, Cm = _f64(Dskip), _f64(delta_bias), _f64(Bm), _f64(Cm)
@@ -121,7 +122,7 @@ def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None,
     y = np.empty_like(u)
     fs = np.empty((B, D, N))
     args = [_d(u), _d(delta), _d(z), _d(A), _d(Dskip), _d(delta_bias), _d(Bm),
-            _d(Cm), int(softplus), _i(seq), _d(h0), _d(out), _d(y), _d(fs), B, D, L, N]
+            _d(Cm), int(softplus), int(zoh), _i(seq), _d(h0), _d(out), _d(y), _d(fs), B, D, L, N]
     if nthreads > 1:
         lib().oracle_scan_fwd_mt(*args, int(nthreads))
     else:
@@ -130,7 +131,7 @@ def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None,
 
 
 def scan_bwd(u, delta, A, Bm, Cm, dout, *, z=None, Dskip=None, delta_bias=None,
-             softplus=True, seq_idx=None, h0=None, nthreads=1):
+             softplus=True, seq_idx=None, h0=None, zoh=False, nthreads=1):
     """Selective scan backward. Returns dict of gradients (fp64):
     du, ddelta (w.r.t. the raw delta), dz, dA, dB, dC, dD, ddelta_bias and
     dh0 (w.r.t. the state before token 0)."""
@@ -149,7 +150,7 @@ def scan_bwd(u, delta, A, Bm, Cm, dout, *, z=None, Dskip=None, delta_bias=None,
     ddb = np.empty(D)
     dh0 = np.empty((B, D, N))
     args = [_d(u), _d(delta), _d(z), _d(A), _d(Dskip), _d(delta_bias), _d(Bm),
-            _d(Cm), int(softplus), _i(seq), _d(h0), _d(dout), _d(du), _d(ddelta), _d(dz),
+            _d(Cm), int(softplus), int(zoh), _i(seq), _d(h0), _d(dout), _d(du), _d(ddelta), _d(dz),
             _d(dA), _d(dB), _d(dC), _d(dD), _d(ddb), _d(dh0), B, D, L, N]
     if nthreads > 1:
         lib().oracle_scan_bwd_mt(*args, int(nthreads))

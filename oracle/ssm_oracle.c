@@ -152,7 +152,26 @@ typedef struct {
     const int32_t* seq;
     int B, D, L, N, softplus_on;
     const double* h0;   /* [B][D][N] state before token 0, NULL = zero */
+    int zoh;            /* 0: B_bar = dt B; 1: zero-order hold B_bar = (exp(dt A) - 1) / A B */
 } scan_in_t;
+
+/* The factor multiplying B_t u_t in the state update: dt (the S6 block of
+ * "Architecture Diagram") or, with zero-order hold ("Discretization"),
+ * A^{-1} (exp(dt A) - 1), whose A -> 0 limit is dt. */
+static double bbar_factor(const scan_in_t* p, double dt, double A) {
+    if (!p->zoh) return dt;
+    return A == 0.0 ? dt : expm1(dt * A) / A;
+}
+
+/* d(bbar_factor)/dA for zero-order hold: (dt e^{dt A} A - (e^{dt A} - 1)) / A^2,
+ * by its Taylor series dt^2 (1/2 + x/3 + x^2/8 + x^3/30 + x^4/144) near
+ * x = dt A = 0 (where the closed form cancels). */
+static double bbar_factor_dA(double dt, double A) {
+    double x = dt * A;
+    if (fabs(x) < 1e-3)
+        return dt * dt * (0.5 + x * (1.0 / 3.0 + x * (1.0 / 8.0 + x * (1.0 / 30.0 + x / 144.0))));
+    return (dt * exp(x) * A - expm1(x)) / (A * A);
+}
 
 /* State before token 0 of row (b, d), state n. */
 static double h0_at(const scan_in_t* p, int b, int d, int n) {
@@ -183,7 +202,7 @@ static void scan_fwd_row(const scan_in_t* p, int b, int d, double* out,
             double bt = p->Bm[((size_t)b * N + n) * L + t];
             double ct = p->Cm[((size_t)b * N + n) * L + t];
             double hprev = reset ? 0.0 : h[n];
-            h[n] = abar * hprev + dt * bt * ut;
+            h[n] = abar * hprev + bbar_factor(p, dt, p->A[(size_t)d * N + n]) * bt * ut;
             y += ct * h[n];
         }
         if (p->Dskip) y += p->Dskip[d] * ut;
@@ -202,10 +221,10 @@ static void scan_fwd_row(const scan_in_t* p, int b, int d, double* out,
 
 void oracle_scan_fwd(const double* u, const double* delta, const double* z,
                      const double* A, const double* Dskip, const double* delta_bias,
-                     const double* Bm, const double* Cm, int softplus_on,
+                     const double* Bm, const double* Cm, int softplus_on, int zoh,
                      const int32_t* seq, const double* h0, double* out, double* y_out,
                      double* final_state, int B, int D, int L, int N) {
-    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0};
+    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0, zoh};
     for (int b = 0; b < B; ++b)
         for (int d = 0; d < D; ++d) scan_fwd_row(&p, b, d, out, y_out, final_state);
 }
@@ -245,7 +264,7 @@ static void scan_bwd_row(const scan_in_t* p, const scan_grad_t* g, int b, int d)
             double bt = p->Bm[((size_t)b * N + n) * L + t];
             double ct = p->Cm[((size_t)b * N + n) * L + t];
             double hprev = reset ? 0.0 : (t == 0 ? h0_at(p, b, d, n) : hs[(size_t)(t - 1) * N + n]);
-            double h = abar * hprev + dt * bt * ut;
+            double h = abar * hprev + bbar_factor(p, dt, p->A[(size_t)d * N + n]) * bt * ut;
             hs[(size_t)t * N + n] = h;
             ab[(size_t)t * N + n] = abar;
             y += ct * h;
@@ -276,14 +295,24 @@ static void scan_bwd_row(const scan_in_t* p, const scan_grad_t* g, int b, int d)
             double hprev = (t == 0) ? h0_at(p, b, d, n) : hs[(size_t)(t - 1) * N + n];
             double q = gt * rs[t] * ab[(size_t)t * N + n] * hprev; /* g * dh/d(A_bar) * A_bar */
             g->dC[bn] += dy * hs[(size_t)t * N + n];
-            g->dB[bn] += gt * dt * ut;
-            g->dA[(size_t)d * N + n] += q * dt;
-            sgB += gt * p->Bm[bn];
-            sAq += An * q;
+            if (p->zoh) {
+                /* h_t = A_bar h_{t-1} + phi B u with phi = (e^{dt A} - 1) / A:
+                 * dphi/d(dt) = A_bar, dphi/dA from bbar_factor_dA */
+                double phi = bbar_factor(p, dt, An);
+                g->dB[bn] += gt * phi * ut;
+                g->dA[(size_t)d * N + n] += q * dt + gt * p->Bm[bn] * ut * bbar_factor_dA(dt, An);
+                sgB += gt * phi * p->Bm[bn];                       /* -> du */
+                sAq += An * q + gt * p->Bm[bn] * ut * ab[(size_t)t * N + n];  /* -> d(dt) */
+            } else {
+                g->dB[bn] += gt * dt * ut;
+                g->dA[(size_t)d * N + n] += q * dt;
+                sgB += gt * p->Bm[bn];
+                sAq += An * q;
+            }
             carry[n] = rs[t] * ab[(size_t)t * N + n] * gt;
         }
-        g->du[row + t] = dy * Dd + dt * sgB;
-        double ddt = ut * sgB + sAq;
+        g->du[row + t] = dy * Dd + (p->zoh ? sgB : dt * sgB);
+        double ddt = p->zoh ? sAq : ut * sgB + sAq;
         double dv = ddt;
         if (p->softplus_on) {
             double v = p->delta[row + t] + (p->delta_bias ? p->delta_bias[d] : 0.0);
@@ -301,12 +330,12 @@ static void scan_bwd_row(const scan_in_t* p, const scan_grad_t* g, int b, int d)
 
 void oracle_scan_bwd(const double* u, const double* delta, const double* z,
                      const double* A, const double* Dskip, const double* delta_bias,
-                     const double* Bm, const double* Cm, int softplus_on,
+                     const double* Bm, const double* Cm, int softplus_on, int zoh,
                      const int32_t* seq, const double* h0, const double* dout, double* du,
                      double* ddelta, double* dz, double* dA, double* dB,
                      double* dC, double* dD, double* ddelta_bias, double* dh0,
                      int B, int D, int L, int N) {
-    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0};
+    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0, zoh};
     memset(dA, 0, sizeof(double) * (size_t)D * N);
     memset(dB, 0, sizeof(double) * (size_t)B * N * L);
     memset(dC, 0, sizeof(double) * (size_t)B * N * L);
@@ -339,10 +368,10 @@ static void* run_job(void* arg) {
 
 void oracle_scan_fwd_mt(const double* u, const double* delta, const double* z,
                         const double* A, const double* Dskip, const double* delta_bias,
-                        const double* Bm, const double* Cm, int softplus_on,
+                        const double* Bm, const double* Cm, int softplus_on, int zoh,
                         const int32_t* seq, const double* h0, double* out, double* y_out,
                         double* final_state, int B, int D, int L, int N, int nthreads) {
-    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0};
+    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0, zoh};
     int rows = B * D;
     if (nthreads < 1) nthreads = 1;
     if (nthreads > rows) nthreads = rows;
@@ -361,12 +390,12 @@ void oracle_scan_fwd_mt(const double* u, const double* delta, const double* z,
 
 void oracle_scan_bwd_mt(const double* u, const double* delta, const double* z,
                         const double* A, const double* Dskip, const double* delta_bias,
-                        const double* Bm, const double* Cm, int softplus_on,
+                        const double* Bm, const double* Cm, int softplus_on, int zoh,
                         const int32_t* seq, const double* h0, const double* dout, double* du,
                         double* ddelta, double* dz, double* dA, double* dB,
                         double* dC, double* dD, double* ddelta_bias, double* dh0,
                         int B, int D, int L, int N, int nthreads) {
-    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0};
+    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0, zoh};
     int rows = B * D;
     if (nthreads < 1) nthreads = 1;
     if (nthreads > rows) nthreads = rows;

@@ -6,7 +6,8 @@
  * Layouts (all contiguous): activations [B][D][L]; B/C [B][N][L];
  * A [D][N]; conv weight [D][W]; per-channel vectors [D]; seq_idx [B][L]
  * (NULL = one segment per row); initial / final state [B][D][N] (h0 NULL =
- * zero state).
+ * zero state). zoh = 0: B_bar = dt B; zoh = 1: zero-order hold,
+ * B_bar = (exp(dt A) - 1) / A B.
  */
 #ifndef SSM_ORACLE_H
 #define SSM_ORACLE_H
@@ -24,12 +25,12 @@ void oracle_conv1d_bwd(const double* x, const double* w, const double* bias,
 
 void oracle_scan_fwd(const double* u, const double* delta, const double* z,
                      const double* A, const double* Dskip, const double* delta_bias,
-                     const double* Bm, const double* Cm, int softplus_on,
+                     const double* Bm, const double* Cm, int softplus_on, int zoh,
                      const int32_t* seq, const double* h0, double* out, double* y_out,
                      double* final_state, int B, int D, int L, int N);
 void oracle_scan_bwd(const double* u, const double* delta, const double* z,
                      const double* A, const double* Dskip, const double* delta_bias,
-                     const double* Bm, const double* Cm, int softplus_on,
+                     const double* Bm, const double* Cm, int softplus_on, int zoh,
                      const int32_t* seq, const double* h0, const double* dout, double* du,
                      double* ddelta, double* dz, double* dA, double* dB,
                      double* dC, double* dD, double* ddelta_bias, double* dh0,
@@ -37,12 +38,12 @@ void oracle_scan_bwd(const double* u, const double* delta, const double* z,
 
 void oracle_scan_fwd_mt(const double* u, const double* delta, const double* z,
                         const double* A, const double* Dskip, const double* delta_bias,
-                        const double* Bm, const double* Cm, int softplus_on,
+                        const double* Bm, const double* Cm, int softplus_on, int zoh,
                         const int32_t* seq, const double* h0, double* out, double* y_out,
                         double* final_state, int B, int D, int L, int N, int nthreads);
 void oracle_scan_bwd_mt(const double* u, const double* delta, const double* z,
                         const double* A, const double* Dskip, const double* delta_bias,
-                        const double* Bm, const double* Cm, int softplus_on,
+                        const double* Bm, const double* Cm, int softplus_on, int zoh,
                         const int32_t* seq, const double* h0, const double* dout, double* du,
                         double* ddelta, double* dz, double* dA, double* dB,
                         double* dC, double* dD, double* ddelta_bias, double* dh0,

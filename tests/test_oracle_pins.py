@@ -527,3 +527,94 @@ def test_decode_continues_a_prefill():
                                            p["Bm"][..., t], p["Cm"][..., t], p["A"], h,
                                            Dskip=p["Dskip"], delta_bias=p["delta_bias"])
         np.testing.assert_allclose(out, full["out"][..., t], rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# zero-order-hold discretisation ("Discretization": B_bar = A^-1 (exp(dA) - I) B)
+# --------------------------------------------------------------------------
+def test_zoh_equals_ode_integration():
+    """ZOH is the exact solution of dh/dtau = A h + B u over a step of length
+    dt with u and B held constant: integrate that ODE with fine RK4 steps
+    from the previous state (zero at a document start) and compare."""
+    rng = _rng(71)
+    seq = np.array([[0, 0, 0, 1, 1, 1, 1]], dtype=np.int32)
+    p = _problem(rng, B=1, D=2, N=3, L=7, seq=seq)
+    r = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], z=p["z"], Dskip=p["Dskip"],
+                        delta_bias=p["delta_bias"], seq_idx=seq, zoh=True)
+    v = p["delta"] + p["delta_bias"][None, :, None]
+    dt = np.log1p(np.exp(v))
+    out = np.zeros_like(p["u"])
+    for d in range(2):
+        h = np.zeros(3)
+        for t in range(7):
+            if t > 0 and seq[0, t] != seq[0, t - 1]:
+                h = np.zeros(3)
+            A, Bv, u = p["A"][d], p["Bm"][0, :, t], p["u"][0, d, t]
+            steps = 2000
+            k = dt[0, d, t] / steps
+            f = lambda hh: A * hh + Bv * u  # noqa: E731
+            for _ in range(steps):
+                k1 = f(h)
+                k2 = f(h + 0.5 * k * k1)
+                k3 = f(h + 0.5 * k * k2)
+                k4 = f(h + k * k3)
+                h = h + k / 6.0 * (k1 + 2 * k2 + 2 * k3 + k4)
+            y = float(p["Cm"][0, :, t] @ h) + p["Dskip"][d] * u
+            out[0, d, t] = y * p["z"][0, d, t] * _sig(p["z"][0, d, t])
+    np.testing.assert_allclose(r["out"], out, rtol=1e-10, atol=1e-12)
+
+
+def test_zoh_lti_is_causal_convolution():
+    """Constant dt, B, C: y = u * K + D u with K_k = sum_n C_n A_bar^k phi_n B_n,
+    phi_n = (exp(dt A_n) - 1) / A_n."""
+    rng = _rng(72)
+    L, N = 50, 4
+    A = -rng.uniform(0.2, 2.0, size=(1, N))
+    Bc, Cc = rng.standard_normal(N), rng.standard_normal(N)
+    u = rng.standard_normal((1, 1, L))
+    dt = 0.3
+    r = oracle.scan_fwd(u, np.full((1, 1, L), dt), A, np.tile(Bc[None, :, None], (1, 1, L)),
+                        np.tile(Cc[None, :, None], (1, 1, L)), Dskip=np.array([0.7]),
+                        softplus=False, zoh=True)
+    a = np.exp(dt * A[0])
+    phi = np.expm1(dt * A[0]) / A[0]
+    K = np.array([np.sum(Cc * a ** k * phi * Bc) for k in range(L)])
+    want = np.convolve(u[0, 0], K)[:L] + 0.7 * u[0, 0]
+    np.testing.assert_allclose(r["out"][0, 0], want, rtol=1e-12, atol=1e-12)
+
+
+def test_zoh_small_A_limit_is_dt_B():
+    """As A -> 0 the ZOH factor (exp(dt A) - 1) / A tends to dt."""
+    rng = _rng(73)
+    p = _problem(rng, B=1, D=2, N=3, L=20)
+    A = np.full((2, 3), -1e-9)
+    a = oracle.scan_fwd(p["u"], p["delta"], A, p["Bm"], p["Cm"], delta_bias=p["delta_bias"], zoh=True)
+    b = oracle.scan_fwd(p["u"], p["delta"], A, p["Bm"], p["Cm"], delta_bias=p["delta_bias"])
+    np.testing.assert_allclose(a["out"], b["out"], rtol=1e-7, atol=1e-12)
+
+
+@pytest.mark.parametrize("softplus", [True, False])
+def test_zoh_bwd_finite_differences(softplus):
+    """Every gradient of the ZOH scan (incl. dA through B_bar and dh0)."""
+    rng = _rng(74)
+    p = _problem(rng, B=2, D=3, N=4, L=20, seq=np.array([[0] * 8 + [1] * 12, [0] * 20],
+                                                        dtype=np.int32))
+    if not softplus:
+        p["delta"] = np.abs(p["delta"]) * 0.2
+        p["delta_bias"] = np.zeros_like(p["delta_bias"])
+    p["A"][0, 0] = -1e-5  # exercises the series branch of dB_bar/dA
+    h0 = rng.standard_normal((2, 3, 4))
+    dout = rng.standard_normal(p["u"].shape)
+    kw = dict(z=p["z"], Dskip=p["Dskip"], delta_bias=p["delta_bias"], softplus=softplus,
+              seq_idx=p["seq_idx"], h0=h0, zoh=True)
+
+    def loss():
+        r = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], **kw)
+        return float(np.sum(r["out"] * dout))
+
+    g = oracle.scan_bwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], dout, **kw)
+    for name, gname in [("u", "du"), ("delta", "ddelta"), ("z", "dz"), ("A", "dA"),
+                        ("Bm", "dB"), ("Cm", "dC"), ("Dskip", "dD"),
+                        ("delta_bias", "ddelta_bias")]:
+        _close(_fd(loss, p[name]), g[gname])
+    _close(_fd(loss, h0), g["dh0"])

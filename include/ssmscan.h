@@ -66,7 +66,7 @@ typedef enum { SSM_DTYPE_F32 = 0, SSM_DTYPE_BF16 = 1 } ssm_dtype_t;
 const char* ssm_last_error(void);
 
 /* ABI version of this header (bumped on any incompatible change). */
-#define SSM_ABI_VERSION 2
+#define SSM_ABI_VERSION 3
 int ssm_abi_version(void);
 
 /* ---------------------------------------------------------------------------
@@ -133,7 +133,7 @@ ssm_status_t ssm_conv1d_bwd_noalloc(const void* x, const float* w, const float* 
  * Selective scan. For each row (b, d) and state n < N, with
  *   dt_t = softplus(delta[b][d][t] + delta_bias[d])   (or without softplus)
  *   a_t  = exp(dt_t * A[d][n])      (0 at the first token of a document)
- *   h_t  = a_t * h_{t-1} + dt_t * Bm[b][n][t] * u[b][d][t],
+ *   h_t  = a_t * h_{t-1} + dt_t * Bm[b][n][t] * u[b][d][t]   (see discretization),
  *   h_{-1} = initial_state[b][d][n]  (0 when initial_state is NULL)
  *   y_t  = sum_n Cm[b][n][t] * h_t + Dskip[d] * u[b][d][t]
  *   out  = y_t * silu(z[b][d][t])   (or y_t when z is NULL)
@@ -164,6 +164,10 @@ typedef struct {
     size_t workspace_bytes;
     const float* initial_state;/* [B][D][N] nullable: the state before token 0 (h_{-1}); with
                                   seq_idx it feeds the first document of each row only */
+    int discretization;        /* 0: B_bar = dt B (the S6 block, "Architecture Diagram");
+                                  1: zero-order hold ("Discretization"), for diagonal A
+                                  B_bar = (exp(dt A) - 1) / A B (-> dt B as A -> 0).
+                                  ssm_conv1d_scan_fwd supports 0 only */
 } ssm_scan_params;
 
 /* Workspace bytes for these params: the state entering every 32-token block

@@ -122,7 +122,7 @@ def conv1d_bwd(x, w, bias, seq_idx, du, *, silu=True, dx=None, dw=None, dbias=No
 
 def scan_params(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softplus=True,
                 seq_idx=None, cu_seqlens=None, n_splits=0, out=None, final_state=None,
-                workspace=None, initial_state=None) -> ssm_scan_params:
+                workspace=None, initial_state=None, zoh=False) -> ssm_scan_params:
     """Fill an ssm_scan_params from tensors (validating shapes and dtypes)."""
     torch = _torch()
     B, D, L = u.shape
@@ -159,6 +159,7 @@ def scan_params(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, sof
     p.workspace = workspace.data_ptr() if workspace is not None else None
     p.workspace_bytes = workspace.numel() if workspace is not None else 0
     p.initial_state = initial_state.data_ptr() if initial_state is not None else None
+    p.discretization = 1 if zoh else 0
     return p
 
 
@@ -180,12 +181,13 @@ def scan_status(u, A, workspace, stream=None) -> int:
 
 def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softplus=True,
              seq_idx=None, cu_seqlens=None, n_splits=0, return_final_state=False, out=None,
-             workspace=None, initial_state=None, stream=None):
+             workspace=None, initial_state=None, zoh=False, stream=None):
     """Selective scan forward.
 
     Returns (out, final_state or None, workspace). Keep `workspace` (it holds
     the state checkpoints and the pre-gate output) and pass it to scan_bwd
-    unchanged. `initial_state` [B, D, N] fp32 is the state before token 0.
+    unchanged. `initial_state` [B, D, N] fp32 is the state before token 0;
+    `zoh` selects the zero-order-hold B_bar = (exp(dt A) - 1) / A B.
     """
     torch = _torch()
     B, D, L = u.shape
@@ -194,7 +196,7 @@ def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softpl
     fs = torch.empty((B, D, N), dtype=torch.float32, device=u.device) if return_final_state else None
     p = scan_params(u, delta, A, Bm, Cm, z=z, Dskip=Dskip, delta_bias=delta_bias, softplus=softplus,
                     seq_idx=seq_idx, cu_seqlens=cu_seqlens, n_splits=n_splits, out=out,
-                    final_state=fs, initial_state=initial_state)
+                    final_state=fs, initial_state=initial_state, zoh=zoh)
     need = ssm_scan_workspace_size(p)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=u.device)
@@ -239,7 +241,7 @@ def conv1d_scan_fwd(x, conv_w, conv_bias, delta, A, Bm, Cm, *, z=None, Dskip=Non
 
 def scan_bwd(u, delta, A, Bm, Cm, dout, workspace, *, z=None, Dskip=None, delta_bias=None,
              softplus=True, seq_idx=None, cu_seqlens=None, n_splits=0, grads=None,
-             initial_state=None, stream=None):
+             initial_state=None, zoh=False, stream=None):
     """Selective scan backward; `workspace` must come from the matching scan_fwd
     (called with the same `initial_state`).
 
@@ -264,7 +266,7 @@ def scan_bwd(u, delta, A, Bm, Cm, dout, workspace, *, z=None, Dskip=None, delta_
     g.setdefault("dinitial_state", torch.empty((B, D, N), dtype=torch.float32, device=dev))
     p = scan_params(u, delta, A, Bm, Cm, z=z, Dskip=Dskip, delta_bias=delta_bias, softplus=softplus,
                     seq_idx=seq_idx, cu_seqlens=cu_seqlens, n_splits=n_splits, out=None,
-                    workspace=workspace, initial_state=initial_state)
+                    workspace=workspace, initial_state=initial_state, zoh=zoh)
     p.out = dout.data_ptr()  # not written by the backward; any valid activation pointer
     gr = ssm_scan_grads()
     gr.struct_size = ctypes.sizeof(ssm_scan_grads)

@@ -46,6 +46,7 @@ class ssm_scan_params(ctypes.Structure):
         ("out", _vp), ("final_state", _vp),
         ("workspace", _vp), ("workspace_bytes", _sz),
         ("initial_state", _vp),
+        ("discretization", _i),
     ]
 
 

@@ -80,6 +80,9 @@ ssm_status_t check_params(const ssm_scan_params* p) {
   if (p->dtype != SSM_DTYPE_F32 && p->dtype != SSM_DTYPE_BF16)
     return fail(SSM_ERR_INVALID_ARG, "unknown dtype %d", (int)p->dtype);
   if (p->n_splits < 0) return fail(SSM_ERR_INVALID_ARG, "n_splits=%d < 0", p->n_splits);
+  if (p->discretization != 0 && p->discretization != 1)
+    return fail(SSM_ERR_INVALID_ARG, "discretization=%d (0: dt B, 1: zero-order hold)",
+                p->discretization);
   if (p->seq_idx && p->cu_seqlens)
     return fail(SSM_ERR_INVALID_ARG, "seq_idx and cu_seqlens are mutually exclusive");
   if (p->cu_seqlens && p->B != 1)
@@ -145,6 +148,7 @@ ssm_status_t build_args(const ssm_scan_params* p, const ScanPlan& pl, ssm::ScanA
   a->Cm = p->Cm;
   a->seq = p->cu_seqlens ? reinterpret_cast<int32_t*>(ws + pl.off_seq) : p->seq_idx;
   a->h0 = p->initial_state;
+  a->zoh = p->discretization == 1 ? 1 : 0;
   a->softplus = p->delta_softplus ? 1 : 0;
   a->out = p->out;
   a->final_state = p->final_state;
@@ -205,6 +209,8 @@ ssm_status_t scan_fwd_impl(const ssm_scan_params* p, const void* x, const float*
   st = check_scan_buffers(p, pl);
   if (st != SSM_OK) return st;
   if (x) {
+    if (p->discretization != 0)
+      return fail(SSM_ERR_UNSUPPORTED, "ssm_conv1d_scan_fwd: only discretization 0 (dt B)");
     if (x == p->u) return fail(SSM_ERR_INVALID_ARG, "u (written) may not alias x");
     if (!aligned(x, elem_size(p->dtype)) || !aligned(conv_w, 4) ||
         (conv_bias && !aligned(conv_bias, 4)))

@@ -45,6 +45,37 @@ __device__ __forceinline__ float sigmoid_fast(float v) {
   return __fdividef(1.0f, 1.0f + __expf(-v));
 }
 
+// Zero-order hold ("Discretization": B_bar = A^{-1} (exp(dt A) - I) B) for
+// a diagonal A: B_bar = dt E1(x) B with x = dt A <= 0 and
+//   E1(x) = (e^x - 1) / x = sum_k x^k / (k+1)!,
+// and d B_bar / dA = dt^2 E2(x) B with
+//   E2(x) = (x e^x - e^x + 1) / x^2 = sum_k (k+1) x^k / (k+2)!.
+// Both take the series through x^6 for |x| < 1/2 (truncation below 3e-7
+// relative) and the closed form from a = e^x otherwise, where a - 1 and
+// x a - (a - 1) are far enough from 0 that rounding stays near 1e-6.
+// Branch-free: both candidates are computed and one selected.
+__device__ __forceinline__ float zoh_e1(float x, float a) {
+  float s = fmaf(x, 1.0f / 5040.0f, 1.0f / 720.0f);
+  s = fmaf(x, s, 1.0f / 120.0f);
+  s = fmaf(x, s, 1.0f / 24.0f);
+  s = fmaf(x, s, 1.0f / 6.0f);
+  s = fmaf(x, s, 0.5f);
+  s = fmaf(x, s, 1.0f);
+  const float closed = __fdividef(a - 1.0f, x);
+  return fabsf(x) < 0.5f ? s : closed;
+}
+__device__ __forceinline__ float zoh_e2(float x, float a) {
+  float s = fmaf(x, 1.0f / 5760.0f, 1.0f / 840.0f);
+  s = fmaf(x, s, 1.0f / 144.0f);
+  s = fmaf(x, s, 1.0f / 30.0f);
+  s = fmaf(x, s, 1.0f / 8.0f);
+  s = fmaf(x, s, 1.0f / 3.0f);
+  s = fmaf(x, s, 0.5f);
+  const float closed = __fdividef(fmaf(x, a, 1.0f - a), x * x);
+  return fabsf(x) < 0.5f ? s : closed;
+}
+constexpr float kLn2 = 0.6931471805599453f;
+
 // softplus(v) = log(1 + e^v); for v > 20 it equals v to within 2.1e-9.
 __device__ __forceinline__ float softplusf_(float v) {
   return v > 20.0f ? v : log1pf(expf(v));

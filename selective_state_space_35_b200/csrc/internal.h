@@ -53,6 +53,7 @@ struct ScanArgs {
   const void* xconv;
   const float* conv_w;
   const float* conv_b;
+  int zoh;            // 1: zero-order-hold B_bar = (exp(dt A) - 1) / A B instead of dt B
   int softplus;
   // forward outputs
   void* out;

@@ -83,6 +83,7 @@ struct BwdSmem {
   float dt[kRows][kBlk];                   // step size (0 past the end)
   float xu[kRows][kBlk];                   // dt u
   float dy[kRows][kBlk];                   // dL/dy = dout silu(z)
+  float uu[kRows][kBlk];                   // u (zero-order hold only)
   float X[kWarps][2][2][kNMax][kLd];       // [warp][array][row half][state][token]
 };
 
@@ -170,7 +171,10 @@ __device__ __forceinline__ void issue_block(BwdSmem<T>& sm, const T* __restrict_
   if (VEC) cp_async_commit();
 }
 
-template <typename T, bool VEC>
+// ZOH: zero-order-hold B_bar = dt E1(dt A) B. Then d(B_bar x)/d(dt) =
+// a B u and d(B_bar x)/dA = dt^2 E2(dt A) B u join the terms through a, du
+// takes dt E1 B, and dB takes dt E1 u.
+template <typename T, bool VEC, bool ZOH>
 __global__ void __launch_bounds__(kWarps * 32, SSM_BWD_MIN_BLOCKS)
 scan_bwd_kernel(const ScanArgs p) {
   extern __shared__ float4 smem_dyn[];
@@ -280,6 +284,7 @@ scan_bwd_kernel(const ScanArgs p) {
     *reinterpret_cast<float2*>(&sm.dt[r][2 * n]) = f2(dt[0], dt[1]);
     *reinterpret_cast<float2*>(&sm.xu[r][2 * n]) = f2(xu[0], xu[1]);
     *reinterpret_cast<float2*>(&sm.dy[r][2 * n]) = f2(dy[0], dy[1]);
+    if (ZOH) *reinterpret_cast<float2*>(&sm.uu[r][2 * n]) = f2(e_u[0], e_u[1]);
     if (has_z && active) store2<T, VEC>(static_cast<T*>(p.dz) + row, t, L, dz[0], dz[1]);
     ck_ready = ck_issued;
     rm_ready = seqb ? __ballot_sync(kFull, tb + lane < L && tb + lane > 0 && sq_cur != sq_prev) : 0u;
@@ -295,6 +300,7 @@ scan_bwd_kernel(const ScanArgs p) {
   const float4* dt4 = reinterpret_cast<const float4*>(&sm.dt[r][0]);
   const float4* xu4 = reinterpret_cast<const float4*>(&sm.xu[r][0]);
   const float4* dy4 = reinterpret_cast<const float4*>(&sm.dy[r][0]);
+  const float4* uu4 = reinterpret_cast<const float4*>(&sm.uu[r][0]);
   const float4* B4 = reinterpret_cast<const float4*>(&sm.B[n][0]);
   const float4* C4 = reinterpret_cast<const float4*>(&sm.C[n][0]);
 
@@ -322,8 +328,12 @@ scan_bwd_kernel(const ScanArgs p) {
           if (m4 & 4u) a2 = 0.0f;
           if (m4 & 8u) a3 = 0.0f;
         }
-        const float2 b0 = fmul2(f2(xq.x, xq.y), f2(bq.x, bq.y));
-        const float2 b1 = fmul2(f2(xq.z, xq.w), f2(bq.z, bq.w));
+        float2 b0 = fmul2(f2(xq.x, xq.y), f2(bq.x, bq.y));
+        float2 b1 = fmul2(f2(xq.z, xq.w), f2(bq.z, bq.w));
+        if (ZOH) {  // the unmasked a: B_bar does not reset at a document start
+          b0 = fmul2(b0, f2(zoh_e1(e0.x * kLn2, ex2_approx(e0.x)), zoh_e1(e0.y * kLn2, ex2_approx(e0.y))));
+          b1 = fmul2(b1, f2(zoh_e1(e1.x * kLn2, ex2_approx(e1.x)), zoh_e1(e1.y * kLn2, ex2_approx(e1.y))));
+        }
         H4[q].x = hh = fmaf(a0, hh, b0.x);
         H4[q].y = hh = fmaf(a1, hh, b0.y);
         H4[q].z = hh = fmaf(a2, hh, b1.x);
@@ -345,6 +355,7 @@ scan_bwd_kernel(const ScanArgs p) {
         const float2 e0 = fmul2(f2(dq.x, dq.y), A2), e1 = fmul2(f2(dq.z, dq.w), A2);
         float a0 = ex2_approx(e0.x), a1 = ex2_approx(e0.y);
         float a2 = ex2_approx(e1.x), a3 = ex2_approx(e1.y);
+        const float4 au = make_float4(a0, a1, a2, a3);  // before document resets (ZOH terms)
         if (rm) {
           const unsigned m4 = rm >> (4 * q);
           if (m4 & 1u) a0 = 0.0f;
@@ -358,15 +369,35 @@ scan_bwd_kernel(const ScanArgs p) {
         const float g0 = fmaf(a1, g1, gy0.x);
         anext = a0;
         gnext = g0;
-        G4[q] = make_float4(g0, g1, g2, g3);
         const float hp = q ? H4[q - 1].w : hck;
         const float2 q0 = fmul2(f2(g0, g1), f2(a0 * hp, a1 * H4[q].x));
         const float2 q1 = fmul2(f2(g2, g3), f2(a2 * H4[q].y, a3 * H4[q].z));
         dA2 = ffma2(f2(dq.x, dq.y), q0, dA2);
         dA2 = ffma2(f2(dq.z, dq.w), q1, dA2);
-        const float2 gb0 = fmul2(f2(g0, g1), f2(bq.x, bq.y));
-        const float2 gb1 = fmul2(f2(g2, g3), f2(bq.z, bq.w));
-        const float2 aq0 = fmul2(Ap, q0), aq1 = fmul2(Ap, q1);
+        float2 gb0, gb1, aq0 = fmul2(Ap, q0), aq1 = fmul2(Ap, q1);
+        if (ZOH) {
+          const float4 uq = uu4[q];
+          const float x0 = e0.x * kLn2, x1 = e0.y * kLn2, x2 = e1.x * kLn2, x3 = e1.y * kLn2;
+          // g E1 carries B_bar's factor into du (via g E1 B) and dB (via g E1 dt u)
+          const float2 ge0 = fmul2(f2(g0, g1), f2(zoh_e1(x0, au.x), zoh_e1(x1, au.y)));
+          const float2 ge1 = fmul2(f2(g2, g3), f2(zoh_e1(x2, au.z), zoh_e1(x3, au.w)));
+          G4[q] = make_float4(ge0.x, ge0.y, ge1.x, ge1.y);
+          gb0 = fmul2(ge0, f2(bq.x, bq.y));
+          gb1 = fmul2(ge1, f2(bq.z, bq.w));
+          // g B u: d(dt) takes it times a, dA times dt^2 E2(dt A)
+          const float2 gbu0 = fmul2(fmul2(f2(g0, g1), f2(bq.x, bq.y)), f2(uq.x, uq.y));
+          const float2 gbu1 = fmul2(fmul2(f2(g2, g3), f2(bq.z, bq.w)), f2(uq.z, uq.w));
+          aq0 = ffma2(gbu0, f2(au.x, au.y), aq0);
+          aq1 = ffma2(gbu1, f2(au.z, au.w), aq1);
+          const float2 d2a = fmul2(f2(dq.x, dq.y), f2(dq.x, dq.y));
+          const float2 d2b = fmul2(f2(dq.z, dq.w), f2(dq.z, dq.w));
+          dA2 = ffma2(fmul2(gbu0, d2a), f2(zoh_e2(x0, au.x), zoh_e2(x1, au.y)), dA2);
+          dA2 = ffma2(fmul2(gbu1, d2b), f2(zoh_e2(x2, au.z), zoh_e2(x3, au.w)), dA2);
+        } else {
+          G4[q] = make_float4(g0, g1, g2, g3);
+          gb0 = fmul2(f2(g0, g1), f2(bq.x, bq.y));
+          gb1 = fmul2(f2(g2, g3), f2(bq.z, bq.w));
+        }
         reinterpret_cast<float4*>(Xg)[q] = make_float4(gb0.x, gb0.y, gb1.x, gb1.y);
         reinterpret_cast<float4*>(Xa)[q] = make_float4(aq0.x, aq0.y, aq1.x, aq1.y);
       }
@@ -441,7 +472,8 @@ scan_bwd_kernel(const ScanArgs p) {
       for (int e = 0; e < 2; ++e) {
         const float s1 = e ? sg.y : sg.x, s2 = e ? sq.y : sq.x;
         du[e] = fmaf(e_dy[e], Dv, e_dt[e] * s1);
-        dd[e] = fmaf(e_u[e], s1, s2) * e_dsp[e];
+        // zero-order hold: s2 already holds the whole d(dt)
+        dd[e] = (ZOH ? s2 : fmaf(e_u[e], s1, s2)) * e_dsp[e];
         if (active && t + e < L) ddbp += dd[e];
       }
       if (active) {
@@ -596,7 +628,7 @@ __global__ void bwd_param_reduce_kernel(const float* __restrict__ pA, const floa
   }
 }
 
-template <typename T, bool VEC>
+template <typename T, bool VEC, bool ZOH>
 cudaError_t bwd_t(const ScanArgs& a, cudaStream_t s) {
   if (a.nsplits > 1) {
     // adjoint carry into each split from the right (lanes-over-time summary)
@@ -610,13 +642,13 @@ cudaError_t bwd_t(const ScanArgs& a, cudaStream_t s) {
   const size_t smem = sizeof(BwdSmem<T>);
   static bool smem_set = false;  // once per instantiation and process (a benign race)
   if (!smem_set) {
-    cudaError_t e = cudaFuncSetAttribute(scan_bwd_kernel<T, VEC>,
+    cudaError_t e = cudaFuncSetAttribute(scan_bwd_kernel<T, VEC, ZOH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     smem_set = true;
   }
   dim3 g2((a.D + kRows - 1) / kRows, a.B, a.nsplits);
-  scan_bwd_kernel<T, VEC><<<g2, kWarps * 32, smem, s>>>(a);
+  scan_bwd_kernel<T, VEC, ZOH><<<g2, kWarps * 32, smem, s>>>(a);
   const int m = a.D * a.N > a.D ? a.D * a.N : a.D;
   bwd_param_reduce_kernel<<<(m + 255) / 256, 256, 0, s>>>(a.part_dA, a.part_dD, a.part_ddb, a.dA,
                                                          a.dD, a.ddelta_bias, a.B, a.D, a.N,
@@ -626,9 +658,15 @@ cudaError_t bwd_t(const ScanArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+template <bool ZOH>
+cudaError_t bwd_dispatch(const ScanArgs& a, cudaStream_t s) {
+  if (a.bf16)
+    return a.vec ? bwd_t<__nv_bfloat16, true, ZOH>(a, s) : bwd_t<__nv_bfloat16, false, ZOH>(a, s);
+  return a.vec ? bwd_t<float, true, ZOH>(a, s) : bwd_t<float, false, ZOH>(a, s);
+}
+
 cudaError_t launch_scan_bwd(const ScanArgs& a, cudaStream_t s) {
-  if (a.bf16) return a.vec ? bwd_t<__nv_bfloat16, true>(a, s) : bwd_t<__nv_bfloat16, false>(a, s);
-  return a.vec ? bwd_t<float, true>(a, s) : bwd_t<float, false>(a, s);
+  return a.zoh ? bwd_dispatch<true>(a, s) : bwd_dispatch<false>(a, s);
 }
 
 }  // namespace ssm

@@ -43,7 +43,9 @@ struct FwdSmem {
 // One state pair (2m, 2m+1) of one chunk for one lane, in two halves so that
 // the discretisation of pair m+1 (ex2-heavy) can overlap the shuffle-latency-
 // bound warp scan of pair m.
-// fwd_pair_pre: a = 2^(dt A'), bx = dt u B for the lane's 8 tokens.
+// fwd_pair_pre: a = 2^(dt A'), bx = dt u B (ZOH: dt E1(dt A) u B) for the
+// lane's 8 tokens.
+template <bool ZOH = false>
 __device__ __forceinline__ void fwd_pair_pre(int m, int lane, const float2* __restrict__ sBt,
                                              const float2 A2, const float2 dd[8],
                                              const float2 xx[8], unsigned rmask, bool any_reset,
@@ -52,8 +54,11 @@ __device__ __forceinline__ void fwd_pair_pre(int m, int lane, const float2* __re
   lds_pair8(sBt + m * kChunk, lane, bv);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    a[i] = ex2x2(fmul2(dd[i], A2));
+    const float2 e = fmul2(dd[i], A2);
+    a[i] = ex2x2(e);
     bx[i] = fmul2(xx[i], bv[i]);
+    if (ZOH)
+      bx[i] = fmul2(bx[i], f2(zoh_e1(e.x * kLn2, a[i].x), zoh_e1(e.y * kLn2, a[i].y)));
   }
   if (any_reset) {
 #pragma unroll
@@ -149,7 +154,7 @@ __device__ __forceinline__ void conv_silu8(float v[8], float& c5, float& c6, flo
 #define SSM_FWD_MIN_BLOCKS 3
 #endif
 
-template <typename T, int G, bool VEC, bool SUMMARY, int NT, bool CONV>
+template <typename T, int G, bool VEC, bool SUMMARY, int NT, bool CONV, bool ZOH>
 __global__ void __launch_bounds__(G * 32, SSM_FWD_MIN_BLOCKS)
 scan_fwd_kernel(const ScanArgs p) {
   // bf16 on the vector path: B / C tiles arrive by TMA one chunk ahead
@@ -278,12 +283,12 @@ scan_fwd_kernel(const ScanArgs p) {
       // compile-time state count: fully unrolled and software-pipelined (the
       // ex2 work of pair m+1 is issued before the scan of pair m)
       float2 a0[8], b0[8];
-      fwd_pair_pre(0, lane, sm.B, sm.A[warp][0], dd, xx, rmask, any_reset, a0, b0);
+      fwd_pair_pre<ZOH>(0, lane, sm.B, sm.A[warp][0], dd, xx, rmask, any_reset, a0, b0);
 #pragma unroll
       for (int m = 0; m < (NT + 1) / 2; ++m) {
         float2 a1[8], b1[8];
         if (m + 1 < (NT + 1) / 2)
-          fwd_pair_pre(m + 1, lane, sm.B, sm.A[warp][m + 1], dd, xx, rmask, any_reset, a1, b1);
+          fwd_pair_pre<ZOH>(m + 1, lane, sm.B, sm.A[warp][m + 1], dd, xx, rmask, any_reset, a1, b1);
         fwd_pair_post<SUMMARY>(m, lane, sm.C, sm.H[warp], sm.P[warp], a0, b0, y2, ck32);
         if (m + 1 < (NT + 1) / 2) {
 #pragma unroll
@@ -297,7 +302,7 @@ scan_fwd_kernel(const ScanArgs p) {
 #pragma unroll 1
       for (int m = 0; m < NP; ++m) {
         float2 a0[8], b0[8];
-        fwd_pair_pre(m, lane, sm.B, sm.A[warp][m], dd, xx, rmask, any_reset, a0, b0);
+        fwd_pair_pre<ZOH>(m, lane, sm.B, sm.A[warp][m], dd, xx, rmask, any_reset, a0, b0);
         fwd_pair_post<SUMMARY>(m, lane, sm.C, sm.H[warp], sm.P[warp], a0, b0, y2, ck32);
       }
     }
@@ -355,49 +360,52 @@ __global__ void cu_seqlens_to_seq_kernel(const int32_t* __restrict__ cu, int n_d
   seq[t] = lo;
 }
 
-template <typename T, int G, bool VEC, bool SUMMARY, int NT, bool CONV>
+template <typename T, int G, bool VEC, bool SUMMARY, int NT, bool CONV, bool ZOH>
 cudaError_t fwd_smem_attr() {
   static bool done = false;  // once per instantiation and process (a benign race)
   if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(scan_fwd_kernel<T, G, VEC, SUMMARY, NT, CONV>,
+  cudaError_t e = cudaFuncSetAttribute(scan_fwd_kernel<T, G, VEC, SUMMARY, NT, CONV, ZOH>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sizeof(FwdSmem<G>));
   if (e == cudaSuccess) done = true;
   return e;
 }
 
-template <typename T, int G, bool VEC, int NT, bool CONV>
+template <typename T, int G, bool VEC, int NT, bool CONV, bool ZOH>
 cudaError_t fwd_t(const ScanArgs& a, cudaStream_t s) {
   dim3 block(G * 32);
   const size_t smem = sizeof(FwdSmem<G>);
-  cudaError_t e = fwd_smem_attr<T, G, VEC, false, NT, CONV>();
-  if (e == cudaSuccess && a.nsplits > 1) e = fwd_smem_attr<T, G, VEC, true, NT, CONV>();
+  cudaError_t e = fwd_smem_attr<T, G, VEC, false, NT, CONV, ZOH>();
+  if (e == cudaSuccess && a.nsplits > 1) e = fwd_smem_attr<T, G, VEC, true, NT, CONV, ZOH>();
   if (e != cudaSuccess) return e;
   if (a.nsplits > 1) {
     dim3 g1((a.D + G - 1) / G, a.B, a.nsplits - 1);
-    scan_fwd_kernel<T, G, VEC, true, NT, CONV><<<g1, block, smem, s>>>(a);
+    scan_fwd_kernel<T, G, VEC, true, NT, CONV, ZOH><<<g1, block, smem, s>>>(a);
     const int n = a.B * a.D * a.Npad;
     fwd_split_carry_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.split_P, a.split_H, a.h0, a.split_in,
                                                           a.B * a.D, a.nsplits, a.Npad, a.N);
   }
   dim3 g2((a.D + G - 1) / G, a.B, a.nsplits);
-  scan_fwd_kernel<T, G, VEC, false, NT, CONV><<<g2, block, smem, s>>>(a);
+  scan_fwd_kernel<T, G, VEC, false, NT, CONV, ZOH><<<g2, block, smem, s>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-template <int NT, bool CONV>
+template <int NT, bool CONV, bool ZOH>
 cudaError_t fwd_dispatch(const ScanArgs& a, cudaStream_t s) {
   if (a.bf16)
-    return a.vec ? fwd_t<__nv_bfloat16, 4, true, NT, CONV>(a, s)
-                 : fwd_t<__nv_bfloat16, 4, false, NT, CONV>(a, s);
-  return a.vec ? fwd_t<float, 4, true, NT, CONV>(a, s) : fwd_t<float, 4, false, NT, CONV>(a, s);
+    return a.vec ? fwd_t<__nv_bfloat16, 4, true, NT, CONV, ZOH>(a, s)
+                 : fwd_t<__nv_bfloat16, 4, false, NT, CONV, ZOH>(a, s);
+  return a.vec ? fwd_t<float, 4, true, NT, CONV, ZOH>(a, s)
+               : fwd_t<float, 4, false, NT, CONV, ZOH>(a, s);
 }
 
 cudaError_t launch_scan_fwd(const ScanArgs& a, cudaStream_t s) {
-  if (a.xconv) return a.N == 16 ? fwd_dispatch<16, true>(a, s) : fwd_dispatch<0, true>(a, s);
-  return a.N == 16 ? fwd_dispatch<16, false>(a, s) : fwd_dispatch<0, false>(a, s);
+  // zero-order hold: runtime state loop, separate conv only
+  if (a.zoh) return fwd_dispatch<0, false, true>(a, s);
+  if (a.xconv) return a.N == 16 ? fwd_dispatch<16, true, false>(a, s) : fwd_dispatch<0, true, false>(a, s);
+  return a.N == 16 ? fwd_dispatch<16, false, false>(a, s) : fwd_dispatch<0, false, false>(a, s);
 }
 
 cudaError_t launch_cu_seqlens_to_seq(const int32_t* cu, int n_docs, int L, int32_t* seq,

@@ -80,7 +80,7 @@ def test_workspace_size_layout(ssm):
 
 @pytest.mark.parametrize("field,value,status", [
     ("struct_size", 3, 1), ("B", 0, 1), ("N", 17, 2), ("N", 0, 1), ("dtype", 7, 1),
-    ("n_splits", -1, 1),
+    ("n_splits", -1, 1), ("discretization", 2, 1),
 ])
 def test_scan_param_validation(ssm, field, value, status):
     from selective_state_space_35_b200 import _lib
@@ -191,7 +191,7 @@ def test_decode_null_params(ssm):
 def test_grads_struct_has_initial_state_gradient(ssm):
     names = [f[0] for f in ssm.ssm_scan_grads._fields_]
     assert names[-1] == "dinitial_state"
-    assert [f[0] for f in ssm.ssm_scan_params._fields_][-1] == "initial_state"
+    assert [f[0] for f in ssm.ssm_scan_params._fields_][-2:] == ["initial_state", "discretization"]
 
 
 def test_fused_forward_validation(ssm):
@@ -205,3 +205,12 @@ def test_fused_forward_validation(ssm):
     assert L.ssm_conv1d_scan_fwd(ctypes.byref(p), fake, fake + 40960, None, None) == 1  # x == u
     assert "alias" in ssm.ssm_last_error()
     assert L.ssm_conv1d_scan_fwd(ctypes.byref(p), fake + 40961, fake + 44000, None, None) == 1
+
+
+def test_fused_forward_rejects_zero_order_hold(ssm):
+    from selective_state_space_35_b200 import _lib
+    fake = 1 << 20
+    p = _params(ssm, u=fake, delta=fake + 4096, A=fake + 8192, Bm=fake + 12288, Cm=fake + 16384,
+                out=fake + 20480, workspace=fake + 65536, workspace_bytes=1 << 30, discretization=1)
+    assert _lib.load().ssm_conv1d_scan_fwd(ctypes.byref(p), fake + 40960, fake + 44000, None,
+                                           None) == 2

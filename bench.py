@@ -45,7 +45,7 @@ SFU_EX2_PER_CLK_PER_SM = 16  # MUFU ex2 throughput per SM per clock (see DESIGN.
 # (one layer B2 D1536 N16 L32768 bf16), from
 # one ncu capture (summarised under profiles/); a kernel changed since its
 # capture has no entry.
-NCU_TRAFFIC = {"scan_bwd": 1231155e3 + 595630e3, "scan_fwd": 611286e3 + 561725e3}
+NCU_TRAFFIC = {}
 
 
 def _peaks():

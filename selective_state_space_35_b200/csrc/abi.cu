@@ -114,8 +114,8 @@ ScanPlan plan_scan(const ssm_scan_params* p) {
   off += p->cu_seqlens ? up((size_t)p->B * p->L * sizeof(int32_t)) : 0;
   s.off_ckpt = off;
   const size_t npad = (size_t)((p->N + 1) & ~1);
-  // one state checkpoint per 32-token block, kNMax wide
-  off += up(rows * s.nchunks * 8 * ssm::kNMax * sizeof(float));
+  // one state checkpoint per 16-token block, kNMax wide
+  off += up(rows * s.nchunks * (ssm::kChunk / 16) * ssm::kNMax * sizeof(float));
   s.off_y = off;
   off += p->z ? up(rows * (size_t)p->L * elem_size(p->dtype)) : 0;
   const size_t per_split = up(rows * s.nsplits * npad * sizeof(float));

@@ -71,7 +71,7 @@ struct ScanArgs {
   float* dh0;         // [B*D][N] nullable
   // workspace pieces
   int* status;        // sticky device status word (0 = ok, 4 = a bounded wait timed out)
-  float* ckpt;        // [B*D][nchunks * 8][kNMax] state entering each 32-token block
+  float* ckpt;        // [B*D][nchunks * 16][kNMax] state entering each 16-token block
   void* ysave;        // [B*D][L] activation dtype: y before the gate (written by fwd when z)
   float* split_P;     // [B*D][P][Npad] per-split decay product (pass 1)
   float* split_H;     // [B*D][P][Npad] per-split end value from zero (pass 1)

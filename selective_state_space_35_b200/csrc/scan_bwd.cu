@@ -1,12 +1,11 @@
 // Selective scan, backward.
 //
 // Recompute-in-backward ("hung-phan ml-skills mamba", "Hardware-Aware
-// Parallel Scan", memory note): the forward keeps only the state entering
-// every 256-token chunk; the backward walks each row's chunks in reverse,
-// rebuilds the chunk's states h_t from that checkpoint (same warp scan as the
-// forward), and runs the adjoint recurrence backwards:
+// Parallel Scan", memory note): the forward keeps the state entering every
+// 16-token block (and, with a gate, y before the gate); the backward walks
+// each row's 32-token blocks in reverse, rebuilds the block's states h_t from
+// the checkpoint at its start and runs the adjoint recurrence backwards:
 //   g_t = dy_t C_t + a_{t+1} g_{t+1}           (g = dLoss/dh, per state n)
-// a reverse warp scan of the maps c -> (prod a) c + G combines the lanes.
 // From g and the rebuilt states (q_t = g_t a_t h_{t-1}):
 //   du_t   = dy_t D + dt_t sum_n g_t B_nt
 //   ddt_t  = u_t sum_n g_t B_nt + sum_n A_n q_t    -> d(raw delta) = ddt * sigmoid(v)
@@ -14,14 +13,13 @@
 //   dz_t   = dout_t y_t silu'(z_t),  dD += dy_t u_t
 // with dy_t = dout_t silu(z_t).
 //
-// One state at a time, with the element-wise work packed two tokens per
-// fp32x2 instruction; the recurrences themselves are scalar chains. A lane's
-// product of a over its 8 tokens is one ex2 of the summed step. dB and dC sum
-// over every channel of a batch row: each warp writes its per-token values
-// into its own shared-memory slice (conflict-free 16-byte stores), the CTA
-// adds the slices and sends one float4 atomic per 4 tokens to HBM. dA, dD and
-// the delta-bias gradient are per-row partials reduced over batch (and
-// splits) in a fixed order by a small kernel.
+// One thread per (row, state): both recurrences are serial per-thread
+// chains, so there is no scan. The per-token sums over states go through a
+// per-warp shared-memory transposition; dB / dC (sums over every channel of a
+// batch row) are added over the CTA's rows in shared memory and sent to HBM
+// with one float4 atomic per 4 tokens. dA, dD and the delta-bias gradient are
+// per-row partials reduced over batch (and splits) in a fixed order by a
+// small kernel.
 #include "scan_common.cuh"
 
 // Resident CTAs per SM the backward is compiled for (register budget).
@@ -194,7 +192,10 @@ scan_bwd_kernel(const ScanArgs p) {
   const int t_end = min((split + 1) * p.chunks_per_split * kChunk, L);
   const size_t rowid = (size_t)b * p.D + (active ? d : 0);
   const size_t row = rowid * L;
-  const size_t nblk = (size_t)p.nchunks * (kChunk / kBlk);
+  // the forward keeps the state entering every 16-token block; this kernel
+  // starts from every other one
+  constexpr int kCk = 16;
+  const size_t nblk = (size_t)p.nchunks * (kChunk / kCk);
   const bool has_z = p.z != nullptr;
 
   const T* Bm = static_cast<const T*>(p.Bm);
@@ -228,7 +229,7 @@ scan_bwd_kernel(const ScanArgs p) {
   auto prefetch = [&](int kb) {
     const int tb = t_begin + kb * kBlk;
     issue_block<T, VEC>(sm, Bm, Cm, rp, n_arrays, b, N, L, tb, r, n, active);
-    if (nval) ck_issued = __ldg(p.ckpt + (rowid * nblk + tb / kBlk) * kNMax + n);
+    if (nval) ck_issued = __ldg(p.ckpt + (rowid * nblk + tb / kCk) * kNMax + n);
     if (seqb) {
       const int t = tb + lane;
       sq_cur = t < L ? __ldg(seqb + t) : 0;

@@ -73,7 +73,7 @@ template <bool SUMMARY>
 __device__ __forceinline__ void fwd_pair_post(int m, int lane, const float2* __restrict__ sCt,
                                               float2* sH, float2* sP, const float2 a[8],
                                               const float2 bx[8], float2 y2[8],
-                                              float2* __restrict__ ck32) {
+                                              float2* __restrict__ ck16) {
   float2 P = a[0], H = bx[0];
 #pragma unroll
   for (int i = 1; i < 8; ++i) {
@@ -90,8 +90,8 @@ __device__ __forceinline__ void fwd_pair_post(int m, int lane, const float2* __r
     if (SUMMARY) sP[m] = fmul2(sP[m], P);
   }
   if (!SUMMARY) {
-    // every fourth lane starts a 32-token block: keep its entering state
-    if ((lane & 3) == 0) ck32[(lane >> 2) * (kNMax / 2) + m] = start;
+    // every other lane starts a 16-token block: keep its entering state
+    if ((lane & 1) == 0) ck16[(lane >> 1) * (kNMax / 2) + m] = start;
     float2 cv[8];
     lds_pair8(sCt + m * kChunk, lane, cv);
     float2 h = start;
@@ -276,8 +276,8 @@ scan_fwd_kernel(const ScanArgs p) {
     const unsigned rmask = reset_mask(p.seq, b, L, tl);
     const bool any_reset = __any_sync(kFull, rmask != 0u);
 
-    // 32-token checkpoints of this chunk: [row][c * 8 + k][kNMax] fp32 pairs
-    float2* ck32 = reinterpret_cast<float2*>(p.ckpt) + (rowid * p.nchunks + c) * 8 * (kNMax / 2);
+    // 16-token checkpoints of this chunk: [row][c * 16 + k][kNMax] fp32 pairs
+    float2* ck16 = reinterpret_cast<float2*>(p.ckpt) + (rowid * p.nchunks + c) * 16 * (kNMax / 2);
 
     if (NT) {
       // compile-time state count: fully unrolled and software-pipelined (the
@@ -289,7 +289,7 @@ scan_fwd_kernel(const ScanArgs p) {
         float2 a1[8], b1[8];
         if (m + 1 < (NT + 1) / 2)
           fwd_pair_pre<ZOH>(m + 1, lane, sm.B, sm.A[warp][m + 1], dd, xx, rmask, any_reset, a1, b1);
-        fwd_pair_post<SUMMARY>(m, lane, sm.C, sm.H[warp], sm.P[warp], a0, b0, y2, ck32);
+        fwd_pair_post<SUMMARY>(m, lane, sm.C, sm.H[warp], sm.P[warp], a0, b0, y2, ck16);
         if (m + 1 < (NT + 1) / 2) {
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
@@ -303,7 +303,7 @@ scan_fwd_kernel(const ScanArgs p) {
       for (int m = 0; m < NP; ++m) {
         float2 a0[8], b0[8];
         fwd_pair_pre<ZOH>(m, lane, sm.B, sm.A[warp][m], dd, xx, rmask, any_reset, a0, b0);
-        fwd_pair_post<SUMMARY>(m, lane, sm.C, sm.H[warp], sm.P[warp], a0, b0, y2, ck32);
+        fwd_pair_post<SUMMARY>(m, lane, sm.C, sm.H[warp], sm.P[warp], a0, b0, y2, ck16);
       }
     }
 

@@ -69,7 +69,7 @@ def test_workspace_size_layout(ssm):
     p = _params(ssm, n_splits=1)
     n1 = ssm.ssm_scan_workspace_size(p)
     nchunks = (1000 + 255) // 256
-    ckpt = 2 * 8 * nchunks * 8 * 16 * 4  # the state entering every 32-token block
+    ckpt = 2 * 8 * nchunks * 16 * 16 * 4  # the state entering every 16-token block
     assert n1 >= ckpt
     # with a gate, y before the gate is kept for the backward (bf16 here)
     assert ssm.ssm_scan_workspace_size(_params(ssm, n_splits=1, z=1 << 20)) >= n1 + 2 * 8 * 1000 * 2

@@ -45,7 +45,7 @@ SFU_EX2_PER_CLK_PER_SM = 16  # MUFU ex2 throughput per SM per clock (see DESIGN.
 # (one layer B2 D1536 N16 L32768 bf16), from
 # one ncu capture (summarised under profiles/); a kernel changed since its
 # capture has no entry.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {"scan_bwd": 1433020e3 + 597357e3, "scan_fwd": 612253e3 + 757312e3}
 
 
 def _peaks():
@@ -494,6 +494,14 @@ def decode_bench(device, sh, pk, rows_b=2048, steps=200, graph_steps=50):
             "hbm_gbs": gbs, "hbm_frac_of_measured": gbs / pk["hbm_gbs"],
             "launches": steps + 20 + 5 * graph_steps}
 
+
+def e2e(layers, device, args, world):
+    """Whole step through the public API from pinned host memory: every step
+    copies each layer's inputs in and its results out. Copies run on their
+    own streams so that layer i's compute overlaps layer i+1's inputs and
+    layer i-1's results (events keep each layer's buffers until their copies
+    are done); the step is timed with CUDA events on the compute stream, after
+    it has waited for the last copy out."""
     import torch
     import torch.distributed as dist
     bf = torch.bfloat16
@@ -504,24 +512,41 @@ def decode_bench(device, sh, pk, rows_b=2048, steps=200, graph_steps=50):
             t = torch.from_numpy(ly.host[k].bits.view(np.int16)).view(bf)
             d[k] = t.pin_memory()
         pinned_in.append(d)
-    ly0 = layers[0]
-    outs = {"out": ly0.out, "dx": ly0.dx, "ddelta": ly0.g["ddelta"], "dz": ly0.g["dz"],
-            "dB": ly0.g["dB"], "dC": ly0.g["dC"], "dA": ly0.g["dA"], "dD": ly0.g["dD"],
-            "ddelta_bias": ly0.g["ddelta_bias"], "dconv_w": ly0.dw, "dconv_b": ly0.dcb}
-    pinned_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outs.items()}
+
+    def outputs(ly):
+        return {"out": ly.out, "dx": ly.dx, "ddelta": ly.g["ddelta"], "dz": ly.g["dz"],
+                "dB": ly.g["dB"], "dC": ly.g["dC"], "dA": ly.g["dA"], "dD": ly.g["dD"],
+                "ddelta_bias": ly.g["ddelta_bias"], "dconv_w": ly.dw, "dconv_b": ly.dcb}
+
+    pinned_out = [{k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+                   for k, v in outputs(ly).items()} for ly in layers]
     h2d = sum(t.numel() * t.element_size() for d in pinned_in for t in d.values())
-    d2h = len(layers) * sum(t.numel() * t.element_size() for t in pinned_out.values())
+    d2h = sum(t.numel() * t.element_size() for d in pinned_out for t in d.values())
+
+    comp = torch.cuda.current_stream(device)
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    in_free = [torch.cuda.Event() for _ in layers]    # compute of the layer is done
+    out_free = [torch.cuda.Event() for _ in layers]   # the layer's results are copied out
+    for e in in_free + out_free:
+        e.record(comp)
 
     def step():
-        for ly, hin in zip(layers, pinned_in):
-            for k, t in hin.items():
-                getattr(ly, k).copy_(t, non_blocking=True)
+        for i, (ly, hin) in enumerate(zip(layers, pinned_in)):
+            s_in.wait_event(in_free[i])  # the previous step has finished reading the inputs
+            with torch.cuda.stream(s_in):
+                for k, t in hin.items():
+                    getattr(ly, k).copy_(t, non_blocking=True)
+            ready = torch.cuda.Event()
+            ready.record(s_in)
+            comp.wait_event(ready)
+            comp.wait_event(out_free[i])  # the previous step's results are out
             ly.step()
-            o = {"out": ly.out, "dx": ly.dx, "ddelta": ly.g["ddelta"], "dz": ly.g["dz"],
-                 "dB": ly.g["dB"], "dC": ly.g["dC"], "dA": ly.g["dA"], "dD": ly.g["dD"],
-                 "ddelta_bias": ly.g["ddelta_bias"], "dconv_w": ly.dw, "dconv_b": ly.dcb}
-            for k, t in o.items():
-                pinned_out[k].copy_(t, non_blocking=True)
+            in_free[i].record(comp)
+            s_out.wait_event(in_free[i])
+            with torch.cuda.stream(s_out):
+                for k, t in outputs(ly).items():
+                    pinned_out[i][k].copy_(t, non_blocking=True)
+            out_free[i].record(s_out)
 
     step()
     torch.cuda.synchronize()
@@ -530,10 +555,12 @@ def decode_bench(device, sh, pk, rows_b=2048, steps=200, graph_steps=50):
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    a.record()
+    a.record(comp)
+    s_in.wait_event(a)
     for _ in range(n):
         step()
-    b.record()
+    comp.wait_event(out_free[-1])
+    b.record(comp)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b)
     if world > 1:
@@ -543,7 +570,9 @@ def decode_bench(device, sh, pk, rows_b=2048, steps=200, graph_steps=50):
     sh = layers[0].shape
     tokens = world * len(layers) * sh.B * sh.L
     return {"value": tokens / (ms / n * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": ms / n}
+            "d2h_bytes_per_step": d2h, "steps": n, "ms_per_step": ms / n,
+            "copies": "inputs in and results out every step, overlapped with compute on two "
+                      "copy streams"}
 
 
 if __name__ == "__main__":

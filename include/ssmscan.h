@@ -166,8 +166,7 @@ typedef struct {
                                   seq_idx it feeds the first document of each row only */
     int discretization;        /* 0: B_bar = dt B (the S6 block, "Architecture Diagram");
                                   1: zero-order hold ("Discretization"), for diagonal A
-                                  B_bar = (exp(dt A) - 1) / A B (-> dt B as A -> 0).
-                                  ssm_conv1d_scan_fwd supports 0 only */
+                                  B_bar = (exp(dt A) - 1) / A B (-> dt B as A -> 0) */
 } ssm_scan_params;
 
 /* Workspace bytes for these params: the state entering every 32-token block

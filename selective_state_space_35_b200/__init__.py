@@ -208,7 +208,7 @@ def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softpl
 def conv1d_scan_fwd(x, conv_w, conv_bias, delta, A, Bm, Cm, *, z=None, Dskip=None,
                     delta_bias=None, softplus=True, seq_idx=None, cu_seqlens=None, n_splits=0,
                     return_final_state=False, u=None, out=None, workspace=None,
-                    initial_state=None, stream=None):
+                    initial_state=None, zoh=False, stream=None):
     """Fused depthwise conv (W = 4) + SiLU + selective scan forward.
 
     x [B, D, L] is the conv input; conv_w [D, 4], conv_bias [D] or None.
@@ -228,7 +228,7 @@ def conv1d_scan_fwd(x, conv_w, conv_bias, delta, A, Bm, Cm, *, z=None, Dskip=Non
     fs = torch.empty((B, D, N), dtype=torch.float32, device=x.device) if return_final_state else None
     p = scan_params(u, delta, A, Bm, Cm, z=z, Dskip=Dskip, delta_bias=delta_bias, softplus=softplus,
                     seq_idx=seq_idx, cu_seqlens=cu_seqlens, n_splits=n_splits, out=out,
-                    final_state=fs, initial_state=initial_state)
+                    final_state=fs, initial_state=initial_state, zoh=zoh)
     need = ssm_scan_workspace_size(p)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)

@@ -209,8 +209,6 @@ ssm_status_t scan_fwd_impl(const ssm_scan_params* p, const void* x, const float*
   st = check_scan_buffers(p, pl);
   if (st != SSM_OK) return st;
   if (x) {
-    if (p->discretization != 0)
-      return fail(SSM_ERR_UNSUPPORTED, "ssm_conv1d_scan_fwd: only discretization 0 (dt B)");
     if (x == p->u) return fail(SSM_ERR_INVALID_ARG, "u (written) may not alias x");
     if (!aligned(x, elem_size(p->dtype)) || !aligned(conv_w, 4) ||
         (conv_bias && !aligned(conv_bias, 4)))

@@ -132,7 +132,7 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
     }
     float g = duv[j];
     if (silu) {
-      const float sgm = sigmoidf_(c);
+      const float sgm = sigmoid_fast(c);  // SFU sigmoid, as in the forward
       g *= sgm * (1.0f + c * (1.0f - sgm));
     }
     dc[j] = (t0 + j < L) ? g : 0.0f;

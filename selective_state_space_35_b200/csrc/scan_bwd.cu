@@ -542,9 +542,9 @@ scan_bwd_summary_kernel(const ScanArgs p) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float v = dl[i] + bias;
-      const float s = p.softplus ? softplusf_(v) : v;
+      const float s = p.softplus ? softplus_sfu(v) : v;  // as the main kernel computes dt
       dl[i] = (tl + i < L) ? s : 0.0f;
-      if (z_row) dy[i] *= zz[i] * sigmoidf_(zz[i]);
+      if (z_row) dy[i] *= zz[i] * sigmoid_fast(zz[i]);
     }
     const unsigned rmask = reset_mask(p.seq, b, L, tl);
     const bool any_reset = __any_sync(kFull, rmask != 0u);

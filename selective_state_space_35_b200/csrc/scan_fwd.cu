@@ -402,8 +402,8 @@ cudaError_t fwd_dispatch(const ScanArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_scan_fwd(const ScanArgs& a, cudaStream_t s) {
-  // zero-order hold: runtime state loop, separate conv only
-  if (a.zoh) return fwd_dispatch<0, false, true>(a, s);
+  // zero-order hold: runtime state loop
+  if (a.zoh) return a.xconv ? fwd_dispatch<0, true, true>(a, s) : fwd_dispatch<0, false, true>(a, s);
   if (a.xconv) return a.N == 16 ? fwd_dispatch<16, true, false>(a, s) : fwd_dispatch<0, true, false>(a, s);
   return a.N == 16 ? fwd_dispatch<16, false, false>(a, s) : fwd_dispatch<0, false, false>(a, s);
 }

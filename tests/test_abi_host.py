@@ -205,12 +205,3 @@ def test_fused_forward_validation(ssm):
     assert L.ssm_conv1d_scan_fwd(ctypes.byref(p), fake, fake + 40960, None, None) == 1  # x == u
     assert "alias" in ssm.ssm_last_error()
     assert L.ssm_conv1d_scan_fwd(ctypes.byref(p), fake + 40961, fake + 44000, None, None) == 1
-
-
-def test_fused_forward_rejects_zero_order_hold(ssm):
-    from selective_state_space_35_b200 import _lib
-    fake = 1 << 20
-    p = _params(ssm, u=fake, delta=fake + 4096, A=fake + 8192, Bm=fake + 12288, Cm=fake + 16384,
-                out=fake + 20480, workspace=fake + 65536, workspace_bytes=1 << 30, discretization=1)
-    assert _lib.load().ssm_conv1d_scan_fwd(ctypes.byref(p), fake + 40960, fake + 44000, None,
-                                           None) == 2

@@ -14,14 +14,15 @@ from pipeline import (TOL_BF16_OUT, TOL_F32, TOL_GRAD, device_inputs, f32_dev, h
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("dtype,L,N,packed,n_splits", [
-    ("bf16", 2048, 16, False, 1),
-    ("bf16", 2048, 16, True, 3),
-    ("bf16", 1001, 16, True, 1),     # ragged: scalar path
-    ("f32", 777, 5, False, 2),
-    ("f32", 512, 16, True, 1),
+@pytest.mark.parametrize("dtype,L,N,packed,n_splits,zoh", [
+    ("bf16", 2048, 16, False, 1, False),
+    ("bf16", 2048, 16, True, 3, False),
+    ("bf16", 1001, 16, True, 1, False),     # ragged: scalar path
+    ("f32", 777, 5, False, 2, False),
+    ("f32", 512, 16, True, 1, False),
+    ("bf16", 1024, 16, True, 2, True),      # zero-order hold
 ])
-def test_fused_equals_separate_bitwise(dtype, L, N, packed, n_splits):
+def test_fused_equals_separate_bitwise(dtype, L, N, packed, n_splits, zoh):
     import torch
     import selective_state_space_35_b200 as ssm
     B, D = 2, 24
@@ -32,7 +33,7 @@ def test_fused_equals_separate_bitwise(dtype, L, N, packed, n_splits):
         inp.seq_idx = synth.random_segments(np.random.Generator(np.random.PCG64(seed)), B, L, 9)
     dv = device_inputs(inp)
     kw = dict(z=dv["z"], Dskip=dv["Dskip"], delta_bias=dv["delta_bias"], seq_idx=dv["seq_idx"],
-              n_splits=n_splits)
+              n_splits=n_splits, zoh=zoh)
     # zero-filled workspaces: the regions the forward does not write compare equal too
     size = ssm.scan_workspace_size(ssm.scan_params(dv["x"], dv["delta"], dv["A"], dv["Bm"],
                                                    dv["Cm"], z=dv["z"], seq_idx=dv["seq_idx"],

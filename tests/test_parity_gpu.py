@@ -90,6 +90,8 @@ SMALL_CASES = [
     (1, 4, 16, 256, 4),
     (2, 3, 16, 257, 6),
     (1, 6, 5, 600, 9),
+    (2, 13, 16, 33, 2),     # backward: a second CTA with 5 of its 8 rows; one token past a block
+    (1, 9, 3, 95, 3),       # L just short of three 32-token blocks
     (2, 9, 16, 1031, 12),
     (1, 4, 16, 2048, 0),
 ]

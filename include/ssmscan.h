@@ -2,7 +2,9 @@
  * libssmscan — C ABI for the Mamba-1 selective-SSM layer core on NVIDIA B200
  * (sm_100a): depthwise causal conv1d + SiLU, and the selective scan with
  * softplus step, D skip and SiLU(z) gate, forward and backward, with state
- * and conv resets at packed-document boundaries.
+ * and conv resets at packed-document boundaries; an initial state and its
+ * gradient, a zero-order-hold discretisation, a fused conv + scan forward,
+ * and the one-token recurrent step for inference.
  *
  * Where each operation is defined (page title, section):
  *   conv1d   "hung-phan ml-skills mamba", "Mamba: Selective State Spaces
@@ -17,6 +19,10 @@
  *            recurrent state start independently for every document.
  *   recompute in backward: "hung-phan ml-skills mamba", "Hardware-Aware
  *            Parallel Scan", memory-optimisation note.
+ *   zero-order hold: same page, "Discretization" (B_bar = A^{-1}(exp(dt A) - I) B).
+ *   fused conv + scan: same page, "Hardware-Aware Parallel Scan" (kernel fusion).
+ *   recurrent step: same page, "Dual Computation Modes" (recurrent mode) and
+ *            "Inference (Generation)" (a (B, D, N) state carried forward).
  *
  * Conventions for every call:
  *   - All array pointers are caller-owned DEVICE memory, C-contiguous, in the

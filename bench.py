@@ -38,7 +38,7 @@ import synth  # noqa: E402
 
 METRIC = "scan fwd+bwd tokens/s (B2×1536ch×32K, N=16); achieved HBM GB/s % of roofline"
 UNIT = "layer-tokens/s"
-SFU_EX2_PER_CLK_PER_SM = 16  # MUFU ex2 throughput per SM per clock
+SFU_EX2_PER_CLK_PER_SM = 16  # MUFU ex2 results per SM per clock (ssm_probe_ex2_rate measures it)
 
 
 # DRAM bytes per launch of the current scan kernels at the 32K bench workload
@@ -275,7 +275,7 @@ def run_reference(args, cfg, rank):
 
 def workload_config(sh, cfg):
     return {"workload": f"{sh.name} bf16, conv1d+SiLU -> selective scan fwd+bwd -> conv1d bwd",
-            "config_index": cfg, "layers": sh.layers, "B": sh.B, "D": sh.D, "N": sh.N, "L": sh.L,
+            "layers": sh.layers, "B": sh.B, "D": sh.D, "N": sh.N, "L": sh.L,
             "conv_width": 4, "storage": sh.dtype, "state": "f32", "packed": sh.packed,
             "l2": "inputs larger than L2 (each layer's inputs > 126 MB, layers rotated); no flush"}
 

@@ -19,7 +19,7 @@
  *   resets "FLA Mamba and Mamba2" (Axolotl), packing paragraph: convolution
  *          and recurrent state start independently for every document.
  *
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent:
  *   - A is passed directly (negative for the S4D-real init), not A_log.exp().
  *   - conv taps are cross-correlation: w[d][W-1] multiplies x_t and w[d][0]
  *     multiplies x_{t-W+1} (PyTorch Conv1d with left padding W-1).

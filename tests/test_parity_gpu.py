@@ -74,7 +74,7 @@ def _small(B, D, N, L, seed, *, dtype="f32", nbound=0, packed=False, boundary_at
     return inp
 
 
-def test_config1_tiny_fp32_layer():
+def test_tiny_fp32_layer_with_boundary():
     inp = synth.make_inputs(synth.CONFIGS[1], synth.seed_for(1))
     res = gpu_layer(device_inputs(inp))
     want = _oracle_layer(inp, bf16_points=False)
@@ -151,14 +151,14 @@ def test_forced_splits_fp32(P):
     _compare_all(res, want, fp32=True)
 
 
-def test_config2_bf16_full():
+def test_mamba130m_layer_bf16_full():
     inp = synth.make_inputs(synth.CONFIGS[2], synth.seed_for(2))
     res = gpu_layer(device_inputs(inp))
     want = _oracle_layer(inp, bf16_points=True)
     _compare_all(res, want, fp32=False)
 
 
-def test_config2_splits_match_unsplit():
+def test_mamba130m_layer_splits_match_unsplit():
     torch = _torch()
     inp = synth.make_inputs(synth.CONFIGS[2], synth.seed_for(2, 1))
     dv = device_inputs(inp)

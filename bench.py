@@ -394,6 +394,11 @@ def main():
                 "frac": achieved / pk["hbm_gbs"], "traffic": None, "kernel": f"ssm_{dom}"}
     t_sfu = 2 * exps / (ex2_peak * 1e12) * 1e3
     t_hbm = (bytes_tok["scan_fwd"] + bytes_tok["scan_bwd"]) * B * L / (pk["hbm_gbs"] * 1e9) * 1e3
+    # secondary bound: the fp32 arithmetic the recurrences need per (token,
+    # state), ~4 ops forward and ~13 backward besides the exp, on 128 fp32
+    # lanes per SM at the max SM clock (an FMA counted as one op)
+    fp32_lane_ops = 148 * 128 * pk["sm_max_mhz"] * 1e6
+    t_fp32 = {"scan_fwd": exps * 4 / fp32_lane_ops * 1e3, "scan_bwd": exps * 13 / fp32_lane_ops * 1e3}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -403,7 +408,9 @@ def main():
         "scan": {"tokens_per_s": world * B * L / (scan_ms * 1e-3),  # scan fwd+bwd per layer
                  "ms_per_layer": {n: avg[n] for n in names},
                  "hbm_gbs": hbm, "hbm_frac_of_measured": {n: hbm[n] / pk["hbm_gbs"] for n in names},
-                 "roofline_ms_per_layer": {"sfu_2BDLN": t_sfu, "hbm_alg_bytes": t_hbm},
+                 "hbm_frac_of_nominal_8tbs": {n: hbm[n] / 8000.0 for n in names},
+                 "roofline_ms_per_layer": {"sfu_2BDLN": t_sfu, "hbm_alg_bytes": t_hbm,
+                                           "fp32_pipe": t_fp32},
                  "frac_of_roofline": max(t_sfu, t_hbm) / scan_ms},
         "gpu_launches": args.steps * sum(ly.launches() for ly in layers),
         "clocks": ck,

@@ -36,9 +36,12 @@ def lib():
         L.oracle_scan_fwd_mt.argtypes = [dp] * 8 + [i, i, ip, dp, dp, dp, dp, i, i, i, i, i]
         L.oracle_scan_bwd_mt.argtypes = [dp] * 8 + [i, i, ip] + [dp] * 11 + [i, i, i, i, i]
         L.oracle_decode_step.argtypes = [dp] * 11 + [i] + [dp] * 3 + [i, i, i, i]
+        L.oracle_cscan_fwd.argtypes = [dp] * 8 + [i, ip, dp, dp, dp, dp, i, i, i, i]
+        L.oracle_cscan_bwd.argtypes = [dp] * 8 + [i, ip] + [dp] * 11 + [i, i, i, i]
         for f in ("oracle_round_bf16", "oracle_conv1d_fwd", "oracle_conv1d_bwd",
                   "oracle_scan_fwd", "oracle_scan_bwd", "oracle_scan_fwd_mt",
-                  "oracle_scan_bwd_mt", "oracle_decode_step"):
+                  "oracle_scan_bwd_mt", "oracle_decode_step", "oracle_cscan_fwd",
+                  "oracle_cscan_bwd"):
             getattr(L, f).restype = None
         _lib = L
     return _lib
@@ -181,6 +184,72 @@ def decode_step(x, conv_state, w, conv_bias, delta, Bt, Ct, A, h, *, z=None,
                              _d(Ct), _d(A), _d(Dskip), _d(delta_bias), int(softplus),
                              _d(hh), _d(out), _d(u), B, D, N, W)
     return out, u, cs, hh
+
+
+def cscan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None,
+              softplus=True, seq_idx=None, h0=None):
+    """Selective scan with complex diagonal A. Returns dict(out, y, final_state).
+
+    u, delta, z: [B, D, L]; A: [D, N] complex; Bm, Cm: [B, N, L] complex;
+    h0: [B, D, N] complex or None. y = 2 Re(sum_n C h) + D u; final_state is
+    complex [B, D, N].
+    """
+    u, delta, z = _f64(u), _f64(delta), _f64(z)
+    Dskip, delta_bias, seq = _f64(Dskip), _f64(delta_bias), _i32(seq_idx)
+    B, D, L = u.shape
+    N = A.shape[1]
+    Ar = _cplx_pairs(A)
+    Bp, Cp = _cplx_planes(Bm), _cplx_planes(Cm)
+    h0p = None if h0 is None else _cplx_pairs(h0)
+    out = np.empty_like(u)
+    y = np.empty_like(u)
+    fs = np.empty((B, D, N, 2))
+    lib().oracle_cscan_fwd(_d(u), _d(delta), _d(z), _d(Ar), _d(Dskip), _d(delta_bias), _d(Bp),
+                           _d(Cp), int(softplus), _i(seq), _d(h0p), _d(out), _d(y), _d(fs),
+                           B, D, L, N)
+    return {"out": out, "y": y, "final_state": fs[..., 0] + 1j * fs[..., 1]}
+
+
+def cscan_bwd(u, delta, A, Bm, Cm, dout, *, z=None, Dskip=None, delta_bias=None,
+              softplus=True, seq_idx=None, h0=None):
+    """Backward of cscan_fwd. Real inputs get real gradients; for a complex
+    input w the gradient is returned as dL/dRe(w) + i dL/dIm(w) (dA, dB, dC,
+    dh0)."""
+    u, delta, z, dout = _f64(u), _f64(delta), _f64(z), _f64(dout)
+    Dskip, delta_bias, seq = _f64(Dskip), _f64(delta_bias), _i32(seq_idx)
+    B, D, L = u.shape
+    N = A.shape[1]
+    Ar = _cplx_pairs(A)
+    Bp, Cp = _cplx_planes(Bm), _cplx_planes(Cm)
+    h0p = None if h0 is None else _cplx_pairs(h0)
+    du = np.empty_like(u)
+    ddelta = np.empty_like(u)
+    dz = np.zeros_like(u)
+    dA = np.empty((D, N, 2))
+    dB = np.empty((B, N, 2, L))
+    dC = np.empty((B, N, 2, L))
+    dD = np.empty(D)
+    ddb = np.empty(D)
+    dh0 = np.empty((B, D, N, 2))
+    lib().oracle_cscan_bwd(_d(u), _d(delta), _d(z), _d(Ar), _d(Dskip), _d(delta_bias), _d(Bp),
+                           _d(Cp), int(softplus), _i(seq), _d(h0p), _d(dout), _d(du),
+                           _d(ddelta), _d(dz), _d(dA), _d(dB), _d(dC), _d(dD), _d(ddb), _d(dh0),
+                           B, D, L, N)
+    return {"du": du, "ddelta": ddelta, "dz": dz, "dA": dA[..., 0] + 1j * dA[..., 1],
+            "dB": dB[:, :, 0] + 1j * dB[:, :, 1], "dC": dC[:, :, 0] + 1j * dC[:, :, 1],
+            "dD": dD, "ddelta_bias": ddb, "dh0": dh0[..., 0] + 1j * dh0[..., 1]}
+
+
+def _cplx_pairs(a):
+    """Complex array [..] -> float64 [.., 2] (re, im interleaved)."""
+    a = np.asarray(a, dtype=np.complex128)
+    return np.ascontiguousarray(np.stack([a.real, a.imag], axis=-1))
+
+
+def _cplx_planes(a):
+    """Complex [B, N, L] -> float64 [B, N, 2, L] (real plane, imaginary plane)."""
+    a = np.asarray(a, dtype=np.complex128)
+    return np.ascontiguousarray(np.stack([a.real, a.imag], axis=2))
 
 
 def layer_fwd_bwd(inp, *, bf16_points: bool, softplus=True, nthreads=1):

@@ -32,6 +32,7 @@
  * drivers only hand rows to pthreads and add per-thread partial sums in a
  * fixed order. Nothing is blocked, fused or reordered inside a row.
  */
+#include <complex.h>
 #include <math.h>
 #include <pthread.h>
 #include <stdint.h>
@@ -471,4 +472,161 @@ void oracle_decode_step(const double* x, double* conv_state, const double* w,
             if (Dskip) y += Dskip[d] * u;
             out[bd] = z ? y * z[bd] * sigm(z[bd]) : y;
         }
+}
+
+/* ------------------------------------------------- complex diagonal A */
+/* Diagonal A with complex entries ("hung-phan ml-skills mamba", section
+ * "S4: Structured State Spaces for Sequences", the S4D simplification; the
+ * same page's Mamba-3 list names a complex-valued state update), made
+ * selective like the real scan:
+ *   a_t = exp(dt_t A_n),  h_t = a_t h_{t-1} + dt_t u_t B_t   (complex h, B)
+ *   y_t = 2 Re(sum_n C_t h_t) + D u_t,  out = y silu(z)
+ * The pages do not say how a complex state yields a real output; this takes
+ * S4D's convention that each state stands for itself and its conjugate,
+ * hence 2 Re. Layouts: A [D][N][2] (re, im); Bm, Cm [B][N][2][L] (real
+ * plane then imaginary plane per state); h0 / final state [B][D][N][2].
+ * Document resets as in the real scan. */
+typedef double complex cplx;
+
+static cplx cld(const double* p) { return p[0] + I * p[1]; }
+
+/* One row. out_row / y_row point at the row's L outputs (y_row nullable);
+ * with hs / as (L x N each) the states and decays are kept for the
+ * backward. */
+static void cscan_fwd_row(const scan_in_t* p, int b, int d, double* out_row, double* y_row,
+                          double* final_state, cplx* hs, cplx* as) {
+    const int L = p->L, N = p->N;
+    size_t row = ((size_t)b * p->D + d) * L;
+    size_t bd = (size_t)b * p->D + d;
+    cplx* h = (cplx*)calloc((size_t)N, sizeof(cplx));
+    for (int n = 0; n < N; ++n)
+        if (p->h0) h[n] = cld(p->h0 + (bd * N + n) * 2);
+    for (int t = 0; t < L; ++t) {
+        double dt = delta_at(p, d, row, t);
+        double ut = p->u[row + t];
+        int reset = (t > 0) && seg_of(p->seq, L, b, t) != seg_of(p->seq, L, b, t - 1);
+        double y = 0.0;
+        for (int n = 0; n < N; ++n) {
+            cplx An = cld(p->A + ((size_t)d * N + n) * 2);
+            size_t bn = (((size_t)b * N + n) * 2) * L + t;   /* real plane; imag at + L */
+            cplx Bt = p->Bm[bn] + I * p->Bm[bn + L];
+            cplx Ct = p->Cm[bn] + I * p->Cm[bn + L];
+            cplx a = cexp(dt * An);
+            cplx hp = reset ? 0.0 : h[n];
+            h[n] = a * hp + dt * ut * Bt;
+            if (hs) {
+                hs[(size_t)t * N + n] = h[n];
+                as[(size_t)t * N + n] = a;
+            }
+            y += 2.0 * creal(Ct * h[n]);
+        }
+        if (p->Dskip) y += p->Dskip[d] * ut;
+        if (y_row) y_row[t] = y;
+        out_row[t] = p->z ? y * p->z[row + t] * sigm(p->z[row + t]) : y;
+    }
+    if (final_state)
+        for (int n = 0; n < N; ++n) {
+            double* f = final_state + (bd * N + n) * 2;
+            f[0] = creal(h[n]);
+            f[1] = cimag(h[n]);
+        }
+    free(h);
+}
+
+void oracle_cscan_fwd(const double* u, const double* delta, const double* z, const double* A,
+                      const double* Dskip, const double* delta_bias, const double* Bm,
+                      const double* Cm, int softplus_on, const int32_t* seq, const double* h0,
+                      double* out, double* y_out, double* final_state, int B, int D, int L, int N) {
+    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0, 0};
+    for (int b = 0; b < B; ++b)
+        for (int d = 0; d < D; ++d) {
+            size_t row = ((size_t)b * D + d) * L;
+            cscan_fwd_row(&p, b, d, out + row, y_out ? y_out + row : NULL, final_state, NULL, NULL);
+        }
+}
+
+/* Reverse mode, with g_t = dL/dRe(h_t) + i dL/dIm(h_t):
+ *   g_t = 2 dy_t conj(C_t) + conj(a_{t+1}) g_{t+1}   (no carry into a document's end)
+ * For a real parameter theta entering through a complex w(theta) the
+ * gradient is Re(conj(dL/dw) dw/dtheta): dL/da_t = g_t conj(h_{t-1}) (0 at a
+ * document start), da/d(dt) = A a, da/dRe A = dt a, da/dIm A = i dt a;
+ * dL/d(dt u) = Re(conj(g) B); dL/dB = dt u g; dL/dC = 2 dy conj(h). */
+void oracle_cscan_bwd(const double* u, const double* delta, const double* z, const double* A,
+                      const double* Dskip, const double* delta_bias, const double* Bm,
+                      const double* Cm, int softplus_on, const int32_t* seq, const double* h0,
+                      const double* dout, double* du, double* ddelta, double* dz, double* dA,
+                      double* dB, double* dC, double* dD, double* ddelta_bias, double* dh0,
+                      int B, int D, int L, int N) {
+    scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0, 0};
+    memset(dA, 0, sizeof(double) * (size_t)D * N * 2);
+    memset(dB, 0, sizeof(double) * (size_t)B * N * 2 * L);
+    memset(dC, 0, sizeof(double) * (size_t)B * N * 2 * L);
+    if (dD) memset(dD, 0, sizeof(double) * (size_t)D);
+    if (ddelta_bias) memset(ddelta_bias, 0, sizeof(double) * (size_t)D);
+    cplx* hs = (cplx*)malloc(sizeof(cplx) * (size_t)L * N);
+    cplx* as = (cplx*)malloc(sizeof(cplx) * (size_t)L * N);
+    double* ys = (double*)malloc(sizeof(double) * (size_t)L);
+    double* os = (double*)malloc(sizeof(double) * (size_t)L);
+    cplx* carry = (cplx*)malloc(sizeof(cplx) * (size_t)N);
+    for (int b = 0; b < B; ++b)
+        for (int d = 0; d < D; ++d) {
+            size_t row = ((size_t)b * D + d) * L;
+            size_t bd = (size_t)b * D + d;
+            cscan_fwd_row(&p, b, d, os, ys, NULL, hs, as);  /* h_t, a_t, y_t of this row */
+            double Dd = Dskip ? Dskip[d] : 0.0;
+            for (int n = 0; n < N; ++n) carry[n] = 0.0;
+            for (int t = L - 1; t >= 0; --t) {
+                double ut = u[row + t];
+                double dt = delta_at(&p, d, row, t);
+                double go = dout[row + t];
+                int reset = (t > 0) && seg_of(seq, L, b, t) != seg_of(seq, L, b, t - 1);
+                double dy;
+                if (z) {
+                    double zt = z[row + t], sg = sigm(zt);
+                    dy = go * zt * sg;
+                    dz[row + t] = go * ys[t] * sg * (1.0 + zt * (1.0 - sg));
+                } else {
+                    dy = go;
+                    if (dz) dz[row + t] = 0.0;
+                }
+                if (dD) dD[d] += dy * ut;
+                double sgB = 0.0, sA = 0.0;
+                for (int n = 0; n < N; ++n) {
+                    cplx An = cld(A + ((size_t)d * N + n) * 2);
+                    size_t bn = (((size_t)b * N + n) * 2) * L + t;
+                    cplx Bt = Bm[bn] + I * Bm[bn + L];
+                    cplx Ct = Cm[bn] + I * Cm[bn + L];
+                    cplx h = hs[(size_t)t * N + n], a = as[(size_t)t * N + n];
+                    cplx g = 2.0 * dy * conj(Ct) + carry[n];
+                    cplx hprev = t == 0 ? (h0 ? cld(h0 + (bd * N + n) * 2) : 0.0)
+                                        : hs[(size_t)(t - 1) * N + n];
+                    cplx Ga = reset ? 0.0 : g * conj(hprev);
+                    double* dAn = dA + ((size_t)d * N + n) * 2;
+                    dAn[0] += creal(conj(Ga) * dt * a);
+                    dAn[1] += creal(conj(Ga) * I * dt * a);
+                    sA += creal(conj(Ga) * An * a);
+                    sgB += creal(conj(g) * Bt);
+                    dB[bn] += creal(g) * dt * ut;
+                    dB[bn + L] += cimag(g) * dt * ut;
+                    dC[bn] += 2.0 * dy * creal(h);
+                    dC[bn + L] += -2.0 * dy * cimag(h);
+                    carry[n] = reset ? 0.0 : conj(a) * g;
+                    if (t == 0 && dh0) {
+                        double* o = dh0 + (bd * N + n) * 2;
+                        o[0] = creal(carry[n]);
+                        o[1] = cimag(carry[n]);
+                    }
+                }
+                du[row + t] = dy * Dd + dt * sgB;
+                double ddt = ut * sgB + sA;
+                double dv = ddt;
+                if (softplus_on) {
+                    double v = delta[row + t] + (delta_bias ? delta_bias[d] : 0.0);
+                    dv = ddt * sigm(v);
+                }
+                ddelta[row + t] = dv;
+                if (ddelta_bias) ddelta_bias[d] += dv;
+            }
+        }
+    free(hs); free(as); free(ys); free(os); free(carry);
 }

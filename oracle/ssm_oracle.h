@@ -55,4 +55,17 @@ void oracle_decode_step(const double* x, double* conv_state, const double* w,
                         const double* Bt, const double* Ct, const double* A,
                         const double* Dskip, const double* delta_bias, int softplus_on,
                         double* h, double* out, double* u_out, int B, int D, int N, int W);
+/* Complex diagonal A (S4D), selective: A [D][N][2], Bm / Cm [B][N][2][L]
+ * (real, imaginary planes), h0 / final state / dh0 [B][D][N][2], dA
+ * [D][N][2], dB / dC [B][N][2][L]; y = 2 Re(sum_n C h) + D u. */
+void oracle_cscan_fwd(const double* u, const double* delta, const double* z, const double* A,
+                      const double* Dskip, const double* delta_bias, const double* Bm,
+                      const double* Cm, int softplus_on, const int32_t* seq, const double* h0,
+                      double* out, double* y_out, double* final_state, int B, int D, int L, int N);
+void oracle_cscan_bwd(const double* u, const double* delta, const double* z, const double* A,
+                      const double* Dskip, const double* delta_bias, const double* Bm,
+                      const double* Cm, int softplus_on, const int32_t* seq, const double* h0,
+                      const double* dout, double* du, double* ddelta, double* dz, double* dA,
+                      double* dB, double* dC, double* dD, double* ddelta_bias, double* dh0,
+                      int B, int D, int L, int N);
 #endif

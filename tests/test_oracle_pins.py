@@ -618,3 +618,129 @@ def test_zoh_bwd_finite_differences(softplus):
                         ("delta_bias", "ddelta_bias")]:
         _close(_fd(loss, p[name]), g[gname])
     _close(_fd(loss, h0), g["dh0"])
+
+
+# --------------------------------------------------------------------------
+# complex diagonal A (S4D form): h_t = exp(dt A) h_{t-1} + dt u B_t,
+# y = 2 Re(sum_n C_t h_t) + D u
+# --------------------------------------------------------------------------
+def _cproblem(rng, B=2, D=3, N=4, L=20, seq=None):
+    p = _problem(rng, B=B, D=D, N=N, L=L, seq=seq)
+    p["A"] = p["A"] + 1j * np.pi * rng.integers(0, 4, size=(D, N))  # S4D-Lin style phases
+    p["Bm"] = p["Bm"] + 1j * rng.standard_normal((B, N, L))
+    p["Cm"] = p["Cm"] + 1j * rng.standard_normal((B, N, L))
+    return p
+
+
+def test_cscan_real_case_equals_real_scan():
+    """Imaginary parts zero: the complex scan is the real scan with C doubled,
+    forward and every gradient (dC picks up the same factor 2)."""
+    rng = _rng(81)
+    seq = np.array([[0] * 9 + [1] * 11, [0] * 20], dtype=np.int32)
+    p = _problem(rng, B=2, D=3, N=4, L=20, seq=seq)
+    h0 = rng.standard_normal((2, 3, 4))
+    dout = rng.standard_normal(p["u"].shape)
+    kw = dict(z=p["z"], Dskip=p["Dskip"], delta_bias=p["delta_bias"], seq_idx=seq, h0=h0)
+    c = oracle.cscan_fwd(p["u"], p["delta"], p["A"] + 0j, p["Bm"] + 0j, p["Cm"] + 0j, **kw)
+    r = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], 2 * p["Cm"], **kw)
+    np.testing.assert_allclose(c["out"], r["out"], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(c["final_state"].real, r["final_state"], rtol=1e-13, atol=1e-13)
+    assert np.all(c["final_state"].imag == 0)
+    gc = oracle.cscan_bwd(p["u"], p["delta"], p["A"] + 0j, p["Bm"] + 0j, p["Cm"] + 0j, dout, **kw)
+    gr = oracle.scan_bwd(p["u"], p["delta"], p["A"], p["Bm"], 2 * p["Cm"], dout, **kw)
+    for k in ("du", "ddelta", "dz", "dD", "ddelta_bias"):
+        np.testing.assert_allclose(gc[k], gr[k], rtol=1e-12, atol=1e-12)
+    for k in ("dA", "dB", "dh0"):
+        np.testing.assert_allclose(gc[k].real, gr[k], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(gc["dC"].real, 2 * gr["dC"], rtol=1e-12, atol=1e-12)
+
+
+def test_cscan_unrolled_sum_brute_force():
+    """y_t = 2 Re sum_n C_t,n [ sum_{s<=t, same document} prod_{s<r<=t} a_r dt_s u_s B_s
+    + prod_{r<=t} a_r h0 (if t is in the first document) ] + D u_t, by numpy
+    complex products, no recurrence."""
+    rng = _rng(82)
+    B, D, N, L = 2, 2, 3, 17
+    seq = np.array([[0] * 6 + [1] * 11, [0] * 17], dtype=np.int32)
+    p = _cproblem(rng, B=B, D=D, N=N, L=L, seq=seq)
+    p["A"] += 1j * rng.standard_normal((D, N))
+    h0 = rng.standard_normal((B, D, N)) + 1j * rng.standard_normal((B, D, N))
+    c = oracle.cscan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], z=None,
+                         Dskip=p["Dskip"], delta_bias=p["delta_bias"], seq_idx=seq, h0=h0)
+    dt = np.log1p(np.exp(p["delta"] + p["delta_bias"][None, :, None]))
+    want = np.empty((B, D, L))
+    for b in range(B):
+        for d in range(D):
+            for t in range(L):
+                acc = 0j
+                for n in range(N):
+                    hn = 0j
+                    for s in range(t + 1):
+                        if seq[b, s] != seq[b, t]:
+                            continue
+                        decay = np.prod(np.exp(dt[b, d, s + 1:t + 1] * p["A"][d, n]))
+                        hn += decay * dt[b, d, s] * p["u"][b, d, s] * p["Bm"][b, n, s]
+                    if seq[b, t] == seq[b, 0]:
+                        hn += np.prod(np.exp(dt[b, d, :t + 1] * p["A"][d, n])) * h0[b, d, n]
+                    acc += p["Cm"][b, n, t] * hn
+                want[b, d, t] = 2 * acc.real + p["Dskip"][d] * p["u"][b, d, t]
+    np.testing.assert_allclose(c["y"], want, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(c["out"], want, rtol=1e-12, atol=1e-12)
+
+
+def test_cscan_pure_rotation_keeps_modulus():
+    """Re A = 0, no input after t=0: |h_t| = |h_0| and arg h_t advances by
+    Im(A) * sum dt (a lossless oscillator)."""
+    rng = _rng(83)
+    B, D, N, L = 1, 1, 2, 12
+    u = np.zeros((B, D, L))
+    u[0, 0, 0] = 1.0
+    delta = 0.3 * rng.standard_normal((B, D, L))
+    A = np.array([[1.7j, -0.4j]])
+    Bm = np.ones((B, N, L)) + 0j
+    Cm = np.zeros((B, N, L)) + 0j
+    c = oracle.cscan_fwd(u, delta, A, Bm, Cm, delta_bias=np.zeros(1))
+    dt = np.log1p(np.exp(delta[0, 0]))
+    h_end = c["final_state"][0, 0]
+    np.testing.assert_allclose(np.abs(h_end), dt[0], rtol=1e-13)
+    phase = A[0].imag * dt[1:].sum()
+    np.testing.assert_allclose(h_end, dt[0] * np.exp(1j * phase), rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("softplus", [True, False])
+def test_cscan_bwd_finite_differences(softplus):
+    """Every gradient of the complex scan, each complex input through its real
+    and imaginary parts, with a document reset and an initial state."""
+    rng = _rng(84)
+    seq = np.array([[0] * 8 + [1] * 12, [0] * 20], dtype=np.int32)
+    p = _cproblem(rng, seq=seq)
+    p["A"] = p["A"] + 1j * rng.standard_normal(p["A"].shape)
+    if not softplus:
+        p["delta"] = np.abs(p["delta"]) * 0.2
+        p["delta_bias"] = np.zeros_like(p["delta_bias"])
+    h0 = rng.standard_normal((2, 3, 4)) + 1j * rng.standard_normal((2, 3, 4))
+    dout = rng.standard_normal(p["u"].shape)
+    parts = {"u": p["u"], "delta": p["delta"], "z": p["z"], "Dskip": p["Dskip"],
+             "delta_bias": p["delta_bias"]}
+    for k, v in (("A", p["A"]), ("Bm", p["Bm"]), ("Cm", p["Cm"]), ("h0", h0)):
+        parts[k + ".re"] = np.ascontiguousarray(v.real)
+        parts[k + ".im"] = np.ascontiguousarray(v.imag)
+
+    def cx(k):
+        return parts[k + ".re"] + 1j * parts[k + ".im"]
+
+    def loss():
+        r = oracle.cscan_fwd(parts["u"], parts["delta"], cx("A"), cx("Bm"), cx("Cm"),
+                             z=parts["z"], Dskip=parts["Dskip"], delta_bias=parts["delta_bias"],
+                             softplus=softplus, seq_idx=seq, h0=cx("h0"))
+        return float(np.sum(r["out"] * dout))
+
+    g = oracle.cscan_bwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], dout, z=p["z"],
+                         Dskip=p["Dskip"], delta_bias=p["delta_bias"], softplus=softplus,
+                         seq_idx=seq, h0=h0)
+    for name, gname in [("u", "du"), ("delta", "ddelta"), ("z", "dz"), ("Dskip", "dD"),
+                        ("delta_bias", "ddelta_bias")]:
+        _close(_fd(loss, parts[name]), g[gname])
+    for name, gname in [("A", "dA"), ("Bm", "dB"), ("Cm", "dC"), ("h0", "dh0")]:
+        _close(_fd(loss, parts[name + ".re"]), g[gname].real)
+        _close(_fd(loss, parts[name + ".im"]), g[gname].imag)

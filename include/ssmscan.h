@@ -3,8 +3,8 @@
  * (sm_100a): depthwise causal conv1d + SiLU, and the selective scan with
  * softplus step, D skip and SiLU(z) gate, forward and backward, with state
  * and conv resets at packed-document boundaries; an initial state and its
- * gradient, a zero-order-hold discretisation, a fused conv + scan forward,
- * and the one-token recurrent step for inference.
+ * gradient, a zero-order-hold discretisation, a complex diagonal A, a fused
+ * conv + scan forward, and the one-token recurrent step for inference.
  *
  * Where each operation is defined (page title, section):
  *   conv1d   "hung-phan ml-skills mamba", "Mamba: Selective State Spaces
@@ -20,6 +20,8 @@
  *   recompute in backward: "hung-phan ml-skills mamba", "Hardware-Aware
  *            Parallel Scan", memory-optimisation note.
  *   zero-order hold: same page, "Discretization" (B_bar = A^{-1}(exp(dt A) - I) B).
+ *   complex A: same page, "S4: Structured State Spaces for Sequences" (S4D:
+ *            a diagonal A with complex entries).
  *   fused conv + scan: same page, "Hardware-Aware Parallel Scan" (kernel fusion).
  *   recurrent step: same page, "Dual Computation Modes" (recurrent mode) and
  *            "Inference (Generation)" (a (B, D, N) state carried forward).
@@ -72,7 +74,7 @@ typedef enum { SSM_DTYPE_F32 = 0, SSM_DTYPE_BF16 = 1 } ssm_dtype_t;
 const char* ssm_last_error(void);
 
 /* ABI version of this header (bumped on any incompatible change). */
-#define SSM_ABI_VERSION 3
+#define SSM_ABI_VERSION 4
 int ssm_abi_version(void);
 
 /* ---------------------------------------------------------------------------
@@ -173,9 +175,21 @@ typedef struct {
     int discretization;        /* 0: B_bar = dt B (the S6 block, "Architecture Diagram");
                                   1: zero-order hold ("Discretization"), for diagonal A
                                   B_bar = (exp(dt A) - 1) / A B (-> dt B as A -> 0) */
+    int state_complex;         /* 0: real A as above. 1: complex diagonal A, the S4D form
+                                  ("S4: Structured State Spaces for Sequences"), made selective:
+                                  A [D][N][2] (re, im), Bm / Cm [B][N][2][L] (per state a real
+                                  then an imaginary row), initial_state / final_state
+                                  [B][D][N][2]; a_t = exp(dt_t A) complex, h complex and
+                                  y_t = 2 Re(sum_n C h_t) + Dskip u_t (each state stands for
+                                  itself and its conjugate). Needs discretization 0 and
+                                  n_splits 0 or 1 (else SSM_ERR_UNSUPPORTED), A, initial_state
+                                  and final_state 8-byte aligned; not available in
+                                  ssm_conv1d_scan_fwd. Gradients take the same layouts
+                                  (dA [D][N][2], dB / dC [B][N][2][L], dinitial_state
+                                  [B][D][N][2]), each pair holding dL/dRe and dL/dIm. */
 } ssm_scan_params;
 
-/* Workspace bytes for these params: the state entering every 32-token block
+/* Workspace bytes for these params: the state entering every 16-token block
  * and, with a gate, y before the gate (both written by the forward, read by
  * the backward), split carries, segment ids built from cu_seqlens, and
  * partial sums of the backward's parameter reductions. */

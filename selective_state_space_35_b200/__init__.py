@@ -123,23 +123,29 @@ def conv1d_bwd(x, w, bias, seq_idx, du, *, silu=True, dx=None, dw=None, dbias=No
 def scan_params(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softplus=True,
                 seq_idx=None, cu_seqlens=None, n_splits=0, out=None, final_state=None,
                 workspace=None, initial_state=None, zoh=False) -> ssm_scan_params:
-    """Fill an ssm_scan_params from tensors (validating shapes and dtypes)."""
+    """Fill an ssm_scan_params from tensors (validating shapes and dtypes).
+
+    A of shape [D, N, 2] selects the complex diagonal A ((re, im) pairs); Bm
+    and Cm are then [B, N, 2, L] and the states [B, D, N, 2].
+    """
     torch = _torch()
     B, D, L = u.shape
     N = A.shape[1]
+    cplx = A.dim() == 3
+    c2 = (2,) if cplx else ()
     _need(u, "u", shape=(B, D, L))
     _need(delta, "delta", u.dtype, (B, D, L))
     _need(z, "z", u.dtype, (B, D, L))
-    _need(A, "A", torch.float32, (D, N))
+    _need(A, "A", torch.float32, (D, N) + c2)
     _need(Dskip, "Dskip", torch.float32, (D,))
     _need(delta_bias, "delta_bias", torch.float32, (D,))
-    _need(Bm, "Bm", u.dtype, (B, N, L))
-    _need(Cm, "Cm", u.dtype, (B, N, L))
+    _need(Bm, "Bm", u.dtype, (B, N) + c2 + (L,))
+    _need(Cm, "Cm", u.dtype, (B, N) + c2 + (L,))
     _need(seq_idx, "seq_idx", torch.int32, (B, L))
     _need(cu_seqlens, "cu_seqlens", torch.int32)
     _need(out, "out", u.dtype, (B, D, L))
-    _need(final_state, "final_state", torch.float32, (B, D, N))
-    _need(initial_state, "initial_state", torch.float32, (B, D, N))
+    _need(final_state, "final_state", torch.float32, (B, D, N) + c2)
+    _need(initial_state, "initial_state", torch.float32, (B, D, N) + c2)
     p = ssm_scan_params()
     p.struct_size = ctypes.sizeof(ssm_scan_params)
     p.B, p.D, p.L, p.N = B, D, L, N
@@ -160,6 +166,7 @@ def scan_params(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, sof
     p.workspace_bytes = workspace.numel() if workspace is not None else 0
     p.initial_state = initial_state.data_ptr() if initial_state is not None else None
     p.discretization = 1 if zoh else 0
+    p.state_complex = int(cplx)
     return p
 
 
@@ -187,13 +194,16 @@ def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softpl
     Returns (out, final_state or None, workspace). Keep `workspace` (it holds
     the state checkpoints and the pre-gate output) and pass it to scan_bwd
     unchanged. `initial_state` [B, D, N] fp32 is the state before token 0;
-    `zoh` selects the zero-order-hold B_bar = (exp(dt A) - 1) / A B.
+    `zoh` selects the zero-order-hold B_bar = (exp(dt A) - 1) / A B. A of
+    shape [D, N, 2] selects the complex diagonal A (see scan_params).
     """
     torch = _torch()
     B, D, L = u.shape
     N = A.shape[1]
+    c2 = (2,) if A.dim() == 3 else ()
     out = torch.empty_like(u) if out is None else out
-    fs = torch.empty((B, D, N), dtype=torch.float32, device=u.device) if return_final_state else None
+    fs = (torch.empty((B, D, N) + c2, dtype=torch.float32, device=u.device)
+          if return_final_state else None)
     p = scan_params(u, delta, A, Bm, Cm, z=z, Dskip=Dskip, delta_bias=delta_bias, softplus=softplus,
                     seq_idx=seq_idx, cu_seqlens=cu_seqlens, n_splits=n_splits, out=out,
                     final_state=fs, initial_state=initial_state, zoh=zoh)
@@ -252,18 +262,19 @@ def scan_bwd(u, delta, A, Bm, Cm, dout, workspace, *, z=None, Dskip=None, delta_
     torch = _torch()
     B, D, L = u.shape
     N = A.shape[1]
+    c2 = (2,) if A.dim() == 3 else ()
     _need(dout, "dout", u.dtype, (B, D, L))
     g = dict(grads or {})
     dev = u.device
     g.setdefault("du", torch.empty_like(u))
     g.setdefault("ddelta", torch.empty_like(u))
     g.setdefault("dz", torch.empty_like(u) if z is not None else None)
-    g.setdefault("dA", torch.empty((D, N), dtype=torch.float32, device=dev))
-    g.setdefault("dB", torch.empty((B, N, L), dtype=torch.float32, device=dev))
-    g.setdefault("dC", torch.empty((B, N, L), dtype=torch.float32, device=dev))
+    g.setdefault("dA", torch.empty((D, N) + c2, dtype=torch.float32, device=dev))
+    g.setdefault("dB", torch.empty((B, N) + c2 + (L,), dtype=torch.float32, device=dev))
+    g.setdefault("dC", torch.empty((B, N) + c2 + (L,), dtype=torch.float32, device=dev))
     g.setdefault("dD", torch.empty((D,), dtype=torch.float32, device=dev))
     g.setdefault("ddelta_bias", torch.empty((D,), dtype=torch.float32, device=dev))
-    g.setdefault("dinitial_state", torch.empty((B, D, N), dtype=torch.float32, device=dev))
+    g.setdefault("dinitial_state", torch.empty((B, D, N) + c2, dtype=torch.float32, device=dev))
     p = scan_params(u, delta, A, Bm, Cm, z=z, Dskip=Dskip, delta_bias=delta_bias, softplus=softplus,
                     seq_idx=seq_idx, cu_seqlens=cu_seqlens, n_splits=n_splits, out=None,
                     workspace=workspace, initial_state=initial_state, zoh=zoh)

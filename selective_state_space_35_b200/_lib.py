@@ -47,6 +47,7 @@ class ssm_scan_params(ctypes.Structure):
         ("workspace", _vp), ("workspace_bytes", _sz),
         ("initial_state", _vp),
         ("discretization", _i),
+        ("state_complex", _i),
     ]
 
 

@@ -83,6 +83,14 @@ ssm_status_t check_params(const ssm_scan_params* p) {
   if (p->discretization != 0 && p->discretization != 1)
     return fail(SSM_ERR_INVALID_ARG, "discretization=%d (0: dt B, 1: zero-order hold)",
                 p->discretization);
+  if (p->state_complex != 0 && p->state_complex != 1)
+    return fail(SSM_ERR_INVALID_ARG, "state_complex=%d (0: real A, 1: complex A)",
+                p->state_complex);
+  if (p->state_complex && p->discretization != 0)
+    return fail(SSM_ERR_UNSUPPORTED, "complex A supports discretization 0 (dt B) only");
+  if (p->state_complex && p->n_splits > 1)
+    return fail(SSM_ERR_UNSUPPORTED, "complex A runs each row on one CTA (n_splits=%d)",
+                p->n_splits);
   if (p->seq_idx && p->cu_seqlens)
     return fail(SSM_ERR_INVALID_ARG, "seq_idx and cu_seqlens are mutually exclusive");
   if (p->cu_seqlens && p->B != 1)
@@ -95,7 +103,7 @@ ssm_status_t check_params(const ssm_scan_params* p) {
 ScanPlan plan_scan(const ssm_scan_params* p) {
   ScanPlan s{};
   s.nchunks = (p->L + ssm::kChunk - 1) / ssm::kChunk;
-  int P = p->n_splits;
+  int P = p->state_complex ? 1 : p->n_splits;
   if (P == 0) {
     // enough warps to keep every SM busy without splitting? (a split costs a
     // second pass over all but the last range)
@@ -114,8 +122,9 @@ ScanPlan plan_scan(const ssm_scan_params* p) {
   off += p->cu_seqlens ? up((size_t)p->B * p->L * sizeof(int32_t)) : 0;
   s.off_ckpt = off;
   const size_t npad = (size_t)((p->N + 1) & ~1);
-  // one state checkpoint per 16-token block, kNMax wide
-  off += up(rows * s.nchunks * (ssm::kChunk / 16) * ssm::kNMax * sizeof(float));
+  // one state checkpoint per 16-token block, kNMax wide (complex: (re, im) pairs)
+  const size_t cw = p->state_complex ? 2 : 1;
+  off += up(rows * s.nchunks * (ssm::kChunk / 16) * ssm::kNMax * cw * sizeof(float));
   s.off_y = off;
   off += p->z ? up(rows * (size_t)p->L * elem_size(p->dtype)) : 0;
   const size_t per_split = up(rows * s.nsplits * npad * sizeof(float));
@@ -126,7 +135,7 @@ ScanPlan plan_scan(const ssm_scan_params* p) {
   s.off_sIn = off;
   off += s.nsplits > 1 ? per_split : 0;
   s.off_pA = off;
-  off += per_split;
+  off += per_split * cw;
   s.off_pD = off;
   off += up(rows * s.nsplits * sizeof(float));
   s.off_pB = off;
@@ -190,6 +199,9 @@ ssm_status_t check_scan_buffers(const ssm_scan_params* p, const ScanPlan& pl) {
                         p->initial_state};
   for (const void* q : f32s)
     if (q && !aligned(q, 4)) return fail(SSM_ERR_INVALID_ARG, "fp32/int32 pointer misaligned");
+  if (p->state_complex && (!aligned(p->A, 8) || !aligned(p->initial_state, 8) ||
+                           !aligned(p->final_state, 8)))
+    return fail(SSM_ERR_INVALID_ARG, "complex A: A and the states must be 8-byte aligned");
   return ok();
 }
 
@@ -208,6 +220,8 @@ ssm_status_t scan_fwd_impl(const ssm_scan_params* p, const void* x, const float*
   const ScanPlan pl = plan_scan(p);
   st = check_scan_buffers(p, pl);
   if (st != SSM_OK) return st;
+  if (x && p->state_complex)
+    return fail(SSM_ERR_UNSUPPORTED, "ssm_conv1d_scan_fwd: complex A is not fused with the conv");
   if (x) {
     if (x == p->u) return fail(SSM_ERR_INVALID_ARG, "u (written) may not alias x");
     if (!aligned(x, elem_size(p->dtype)) || !aligned(conv_w, 4) ||
@@ -228,6 +242,7 @@ ssm_status_t scan_fwd_impl(const ssm_scan_params* p, const void* x, const float*
                                                   const_cast<int32_t*>(a.seq), s);
     if (e != cudaSuccess) return cuda_status(e, "cu_seqlens conversion");
   }
+  if (p->state_complex) return cuda_status(ssm::launch_cscan_fwd(a, s), "ssm_scan_fwd launch");
   return cuda_status(ssm::launch_scan_fwd(a, s), x ? "ssm_conv1d_scan_fwd launch" : "ssm_scan_fwd launch");
 }
 
@@ -386,6 +401,8 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
   const void* f32s[] = {g->dA, g->dB, g->dC, g->dD, g->ddelta_bias, g->dinitial_state};
   for (const void* q : f32s)
     if (q && !aligned(q, 4)) return fail(SSM_ERR_INVALID_ARG, "fp32 gradient pointer misaligned");
+  if (p->state_complex && (!aligned(g->dA, 8) || !aligned(g->dinitial_state, 8)))
+    return fail(SSM_ERR_INVALID_ARG, "complex A: dA and dinitial_state must be 8-byte aligned");
   ssm::ScanArgs a;
   build_args(p, pl, &a);
   a.dout = g->dout;
@@ -407,10 +424,11 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
                                                   const_cast<int32_t*>(a.seq), s);
     if (e != cudaSuccess) return cuda_status(e, "cu_seqlens conversion");
   }
-  const size_t bc = (size_t)p->B * p->N * p->L * sizeof(float);
+  const size_t bc = (size_t)p->B * p->N * p->L * sizeof(float) * (p->state_complex ? 2 : 1);
   cudaError_t e = cudaMemsetAsync(g->dB, 0, bc, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(g->dC, 0, bc, s);
   if (e != cudaSuccess) return cuda_status(e, "ssm_scan_bwd memset");
+  if (p->state_complex) return cuda_status(ssm::launch_cscan_bwd(a, s), "ssm_scan_bwd launch");
   return cuda_status(ssm::launch_scan_bwd(a, s), "ssm_scan_bwd launch");
 }
 

@@ -86,6 +86,10 @@ struct ScanArgs {
 };
 
 cudaError_t launch_scan_fwd(const ScanArgs& a, cudaStream_t s);
+// Complex diagonal A (A [D][N][2], Bm / Cm [B][N][2][L], states as (re, im)
+// pairs, checkpoints [B*D][nchunks * 16][kNMax][2], part_dA [B*D][N][2]).
+cudaError_t launch_cscan_fwd(const ScanArgs& a, cudaStream_t s);
+cudaError_t launch_cscan_bwd(const ScanArgs& a, cudaStream_t s);
 
 struct DecodeArgs {
   const void* x;

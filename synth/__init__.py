@@ -261,3 +261,47 @@ def decode_inputs(B: int, D: int, N: int, steps: int, dtype: str, seed: int) -> 
     conv_state = _act(rng, (B, D, 3), dtype)
     h0 = (0.5 * rng.standard_normal((B, D, N), dtype=np.float32)).astype(np.float32)
     return DecodeInputs(x, delta, z, Bm, Cm, conv_state, h0, A, Dskip, delta_bias, conv_w, conv_b)
+
+
+@dataclass
+class ComplexInputs:
+    """Inputs of the scan with a complex diagonal A.
+
+    u, delta, z, dout: [B, D, L]; Bm, Cm: [B, N, 2, L] (per state a real then
+    an imaginary row); A: float32 [D, N, 2] (re, im); h0: float32
+    [B, D, N, 2] or None."""
+    u: Tensor
+    delta: Tensor
+    z: Tensor
+    dout: Tensor
+    Bm: Tensor
+    Cm: Tensor
+    A: np.ndarray
+    Dskip: np.ndarray
+    delta_bias: np.ndarray
+    seq_idx: np.ndarray | None
+    h0: np.ndarray | None
+
+
+
+def complex_inputs(B: int, D: int, N: int, L: int, dtype: str, seed: int, *,
+                   seq_idx: np.ndarray | None = None, with_h0: bool = False) -> ComplexInputs:
+    """Seeded inputs for the complex-A scan. A follows S4D-Lin:
+    A[d, n] = -1/2 + i pi n; the delta bias, D, u, z, delta and dout follow
+    `make_inputs` (u ~ N(0, 1) stands for the conv output); the real and
+    imaginary parts of B and C are each ~ N(0, 1)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    A = np.zeros((D, N, 2), dtype=np.float32)
+    A[:, :, 0] = -0.5
+    A[:, :, 1] = (np.pi * np.arange(N)).astype(np.float32)[None, :]
+    Dskip = rng.uniform(0.5, 1.5, size=D).astype(np.float32)
+    delta_bias = np.log(np.expm1(rng.uniform(1e-3, 1e-1, size=D))).astype(np.float32)
+    u = _act(rng, (B, D, L), dtype)
+    z = _act(rng, (B, D, L), dtype)
+    delta = _act(rng, (B, D, L), dtype, 0.5)
+    Bm = _act(rng, (B, N, 2, L), dtype)
+    Cm = _act(rng, (B, N, 2, L), dtype)
+    dout = _act(rng, (B, D, L), dtype)
+    h0 = (0.5 * rng.standard_normal((B, D, N, 2), dtype=np.float32)).astype(np.float32) \
+        if with_h0 else None
+    return ComplexInputs(u, delta, z, dout, Bm, Cm, A, Dskip, delta_bias, seq_idx, h0)

@@ -80,7 +80,7 @@ def test_workspace_size_layout(ssm):
 
 @pytest.mark.parametrize("field,value,status", [
     ("struct_size", 3, 1), ("B", 0, 1), ("N", 17, 2), ("N", 0, 1), ("dtype", 7, 1),
-    ("n_splits", -1, 1), ("discretization", 2, 1),
+    ("n_splits", -1, 1), ("discretization", 2, 1), ("state_complex", 2, 1),
 ])
 def test_scan_param_validation(ssm, field, value, status):
     from selective_state_space_35_b200 import _lib
@@ -191,7 +191,8 @@ def test_decode_null_params(ssm):
 def test_grads_struct_has_initial_state_gradient(ssm):
     names = [f[0] for f in ssm.ssm_scan_grads._fields_]
     assert names[-1] == "dinitial_state"
-    assert [f[0] for f in ssm.ssm_scan_params._fields_][-2:] == ["initial_state", "discretization"]
+    assert [f[0] for f in ssm.ssm_scan_params._fields_][-3:] == ["initial_state", "discretization",
+                                                                 "state_complex"]
 
 
 def test_fused_forward_validation(ssm):
@@ -205,3 +206,27 @@ def test_fused_forward_validation(ssm):
     assert L.ssm_conv1d_scan_fwd(ctypes.byref(p), fake, fake + 40960, None, None) == 1  # x == u
     assert "alias" in ssm.ssm_last_error()
     assert L.ssm_conv1d_scan_fwd(ctypes.byref(p), fake + 40961, fake + 44000, None, None) == 1
+
+
+def test_complex_a_rules(ssm):
+    """Complex A: dt B discretisation and one CTA per row only, doubled
+    checkpoints, 8-byte aligned A / states, not fused with the conv."""
+    from selective_state_space_35_b200 import _lib
+    L = _lib.load()
+    n = ctypes.c_size_t(0)
+    for kw, status in [(dict(discretization=1), 2), (dict(n_splits=2), 2),
+                       (dict(n_splits=1), 0), (dict(n_splits=0), 0)]:
+        p = _params(ssm, state_complex=1, **kw)
+        assert L.ssm_scan_workspace_size(ctypes.byref(p), ctypes.byref(n)) == status, kw
+    real = ssm.ssm_scan_workspace_size(_params(ssm, n_splits=1))
+    cplx = ssm.ssm_scan_workspace_size(_params(ssm, state_complex=1))
+    nchunks = (1000 + 255) // 256
+    assert cplx >= real + 2 * 8 * nchunks * 16 * 16 * 4  # (re, im) checkpoints
+    fake = 1 << 20
+    good = dict(u=fake, delta=fake + 4096, A=fake + 8192, Bm=fake + 12288, Cm=fake + 16384,
+                out=fake + 20480, workspace=fake + 65536, workspace_bytes=1 << 30, state_complex=1)
+    p = _params(ssm, **dict(good, A=fake + 8196))   # 4-byte but not 8-byte aligned
+    assert L.ssm_scan_fwd(ctypes.byref(p), None) == 1
+    assert "8-byte" in ssm.ssm_last_error()
+    p = _params(ssm, **good)
+    assert L.ssm_conv1d_scan_fwd(ctypes.byref(p), fake + (1 << 24), fake, None, None) == 2

@@ -32,12 +32,12 @@ def lib():
         L.oracle_conv1d_fwd.argtypes = [dp, dp, dp, ip, dp, dp, i, i, i, i, i]
         L.oracle_conv1d_bwd.argtypes = [dp, dp, dp, ip, dp, dp, dp, dp, i, i, i, i, i]
         L.oracle_scan_fwd.argtypes = [dp] * 8 + [i, i, ip, dp, dp, dp, dp, i, i, i, i]
-        L.oracle_scan_bwd.argtypes = [dp] * 8 + [i, i, ip] + [dp] * 11 + [i, i, i, i]
+        L.oracle_scan_bwd.argtypes = [dp] * 8 + [i, i, ip] + [dp] * 12 + [i, i, i, i]
         L.oracle_scan_fwd_mt.argtypes = [dp] * 8 + [i, i, ip, dp, dp, dp, dp, i, i, i, i, i]
-        L.oracle_scan_bwd_mt.argtypes = [dp] * 8 + [i, i, ip] + [dp] * 11 + [i, i, i, i, i]
+        L.oracle_scan_bwd_mt.argtypes = [dp] * 8 + [i, i, ip] + [dp] * 12 + [i, i, i, i, i]
         L.oracle_decode_step.argtypes = [dp] * 11 + [i] + [dp] * 3 + [i, i, i, i]
         L.oracle_cscan_fwd.argtypes = [dp] * 8 + [i, ip, dp, dp, dp, dp, i, i, i, i]
-        L.oracle_cscan_bwd.argtypes = [dp] * 8 + [i, ip] + [dp] * 11 + [i, i, i, i]
+        L.oracle_cscan_bwd.argtypes = [dp] * 8 + [i, ip] + [dp] * 12 + [i, i, i, i]
         for f in ("oracle_round_bf16", "oracle_conv1d_fwd", "oracle_conv1d_bwd",
                   "oracle_scan_fwd", "oracle_scan_bwd", "oracle_scan_fwd_mt",
                   "oracle_scan_bwd_mt", "oracle_decode_step", "oracle_cscan_fwd",
@@ -134,13 +134,14 @@ def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None,
 
 
 def scan_bwd(u, delta, A, Bm, Cm, dout, *, z=None, Dskip=None, delta_bias=None,
-             softplus=True, seq_idx=None, h0=None, zoh=False, nthreads=1):
+             softplus=True, seq_idx=None, h0=None, zoh=False, dhL=None, nthreads=1):
     """Selective scan backward. Returns dict of gradients (fp64):
     du, ddelta (w.r.t. the raw delta), dz, dA, dB, dC, dD, ddelta_bias and
-    dh0 (w.r.t. the state before token 0)."""
+    dh0 (w.r.t. the state before token 0). dhL [B, D, N]: a gradient reaching
+    the final state from outside (None: 0)."""
     u, delta, z, A = _f64(u), _f64(delta), _f64(z), _f64(A)
     Dskip, delta_bias, Bm, Cm = _f64(Dskip), _f64(delta_bias), _f64(Bm), _f64(Cm)
-    seq, dout, h0 = _i32(seq_idx), _f64(dout), _f64(h0)
+    seq, dout, h0, dhL = _i32(seq_idx), _f64(dout), _f64(h0), _f64(dhL)
     B, D, L = u.shape
     N = A.shape[1]
     du = np.empty_like(u)
@@ -154,7 +155,7 @@ def scan_bwd(u, delta, A, Bm, Cm, dout, *, z=None, Dskip=None, delta_bias=None,
     dh0 = np.empty((B, D, N))
     args = [_d(u), _d(delta), _d(z), _d(A), _d(Dskip), _d(delta_bias), _d(Bm),
             _d(Cm), int(softplus), int(zoh), _i(seq), _d(h0), _d(dout), _d(du), _d(ddelta), _d(dz),
-            _d(dA), _d(dB), _d(dC), _d(dD), _d(ddb), _d(dh0), B, D, L, N]
+            _d(dA), _d(dB), _d(dC), _d(dD), _d(ddb), _d(dh0), _d(dhL), B, D, L, N]
     if nthreads > 1:
         lib().oracle_scan_bwd_mt(*args, int(nthreads))
     else:
@@ -211,10 +212,11 @@ def cscan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None,
 
 
 def cscan_bwd(u, delta, A, Bm, Cm, dout, *, z=None, Dskip=None, delta_bias=None,
-              softplus=True, seq_idx=None, h0=None):
+              softplus=True, seq_idx=None, h0=None, dhL=None):
     """Backward of cscan_fwd. Real inputs get real gradients; for a complex
     input w the gradient is returned as dL/dRe(w) + i dL/dIm(w) (dA, dB, dC,
-    dh0)."""
+    dh0). dhL [B, D, N] complex: dL/dRe h_{L-1} + i dL/dIm h_{L-1} from
+    outside (None: 0)."""
     u, delta, z, dout = _f64(u), _f64(delta), _f64(z), _f64(dout)
     Dskip, delta_bias, seq = _f64(Dskip), _f64(delta_bias), _i32(seq_idx)
     B, D, L = u.shape
@@ -222,6 +224,7 @@ def cscan_bwd(u, delta, A, Bm, Cm, dout, *, z=None, Dskip=None, delta_bias=None,
     Ar = _cplx_pairs(A)
     Bp, Cp = _cplx_planes(Bm), _cplx_planes(Cm)
     h0p = None if h0 is None else _cplx_pairs(h0)
+    dhLp = None if dhL is None else _cplx_pairs(dhL)
     du = np.empty_like(u)
     ddelta = np.empty_like(u)
     dz = np.zeros_like(u)
@@ -234,7 +237,7 @@ def cscan_bwd(u, delta, A, Bm, Cm, dout, *, z=None, Dskip=None, delta_bias=None,
     lib().oracle_cscan_bwd(_d(u), _d(delta), _d(z), _d(Ar), _d(Dskip), _d(delta_bias), _d(Bp),
                            _d(Cp), int(softplus), _i(seq), _d(h0p), _d(dout), _d(du),
                            _d(ddelta), _d(dz), _d(dA), _d(dB), _d(dC), _d(dD), _d(ddb), _d(dh0),
-                           B, D, L, N)
+                           _d(dhLp), B, D, L, N)
     return {"du": du, "ddelta": ddelta, "dz": dz, "dA": dA[..., 0] + 1j * dA[..., 1],
             "dB": dB[:, :, 0] + 1j * dB[:, :, 1], "dC": dC[:, :, 0] + 1j * dC[:, :, 1],
             "dD": dD, "ddelta_bias": ddb, "dh0": dh0[..., 0] + 1j * dh0[..., 1]}

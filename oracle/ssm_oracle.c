@@ -236,6 +236,7 @@ typedef struct {
     double *du, *ddelta, *dz;          /* per row, overwritten */
     double *dA, *dB, *dC, *dD, *ddb;   /* accumulated */
     double* dh0;                       /* [B][D][N] per row, overwritten; may be NULL */
+    const double* dhL;                 /* [B][D][N] dL/dh_{L-1} from outside; may be NULL */
 } scan_grad_t;
 
 /* One row. Re-runs the forward keeping every h_t and A_bar_t, then walks t
@@ -252,6 +253,9 @@ static void scan_bwd_row(const scan_in_t* p, const scan_grad_t* g, int b, int d)
     int* rs = (int*)malloc(sizeof(int) * (size_t)L);
     double* carry = (double*)calloc((size_t)N, sizeof(double));
     double Dd = p->Dskip ? p->Dskip[d] : 0.0;
+    /* a gradient reaching h_{L-1} from outside enters g_{L-1} like the carry */
+    if (g->dhL)
+        for (int n = 0; n < N; ++n) carry[n] = g->dhL[((size_t)b * p->D + d) * N + n];
 
     for (int t = 0; t < L; ++t) {
         double dt = delta_at(p, d, row, t);
@@ -335,14 +339,14 @@ void oracle_scan_bwd(const double* u, const double* delta, const double* z,
                      const int32_t* seq, const double* h0, const double* dout, double* du,
                      double* ddelta, double* dz, double* dA, double* dB,
                      double* dC, double* dD, double* ddelta_bias, double* dh0,
-                     int B, int D, int L, int N) {
+                     const double* dhL, int B, int D, int L, int N) {
     scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0, zoh};
     memset(dA, 0, sizeof(double) * (size_t)D * N);
     memset(dB, 0, sizeof(double) * (size_t)B * N * L);
     memset(dC, 0, sizeof(double) * (size_t)B * N * L);
     if (dD) memset(dD, 0, sizeof(double) * (size_t)D);
     if (ddelta_bias) memset(ddelta_bias, 0, sizeof(double) * (size_t)D);
-    scan_grad_t g = {dout, du, ddelta, dz, dA, dB, dC, dD, ddelta_bias, dh0};
+    scan_grad_t g = {dout, du, ddelta, dz, dA, dB, dC, dD, ddelta_bias, dh0, dhL};
     for (int b = 0; b < B; ++b)
         for (int d = 0; d < D; ++d) scan_bwd_row(&p, &g, b, d);
 }
@@ -395,7 +399,7 @@ void oracle_scan_bwd_mt(const double* u, const double* delta, const double* z,
                         const int32_t* seq, const double* h0, const double* dout, double* du,
                         double* ddelta, double* dz, double* dA, double* dB,
                         double* dC, double* dD, double* ddelta_bias, double* dh0,
-                        int B, int D, int L, int N, int nthreads) {
+                        const double* dhL, int B, int D, int L, int N, int nthreads) {
     scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0, zoh};
     int rows = B * D;
     if (nthreads < 1) nthreads = 1;
@@ -409,6 +413,7 @@ void oracle_scan_bwd_mt(const double* u, const double* delta, const double* z,
         jobs[i].g.dout = dout;
         jobs[i].g.du = du; jobs[i].g.ddelta = ddelta; jobs[i].g.dz = dz;
         jobs[i].g.dh0 = dh0;
+        jobs[i].g.dhL = dhL;
         jobs[i].g.dA = (double*)calloc(nA, sizeof(double));
         jobs[i].g.dB = (double*)calloc(nBC, sizeof(double));
         jobs[i].g.dC = (double*)calloc(nBC, sizeof(double));
@@ -556,7 +561,7 @@ void oracle_cscan_bwd(const double* u, const double* delta, const double* z, con
                       const double* Cm, int softplus_on, const int32_t* seq, const double* h0,
                       const double* dout, double* du, double* ddelta, double* dz, double* dA,
                       double* dB, double* dC, double* dD, double* ddelta_bias, double* dh0,
-                      int B, int D, int L, int N) {
+                      const double* dhL, int B, int D, int L, int N) {
     scan_in_t p = {u, delta, z, A, Dskip, delta_bias, Bm, Cm, seq, B, D, L, N, softplus_on, h0, 0};
     memset(dA, 0, sizeof(double) * (size_t)D * N * 2);
     memset(dB, 0, sizeof(double) * (size_t)B * N * 2 * L);
@@ -574,7 +579,8 @@ void oracle_cscan_bwd(const double* u, const double* delta, const double* z, con
             size_t bd = (size_t)b * D + d;
             cscan_fwd_row(&p, b, d, os, ys, NULL, hs, as);  /* h_t, a_t, y_t of this row */
             double Dd = Dskip ? Dskip[d] : 0.0;
-            for (int n = 0; n < N; ++n) carry[n] = 0.0;
+            for (int n = 0; n < N; ++n)  /* dL/dh_{L-1} from outside, or 0 */
+                carry[n] = dhL ? cld(dhL + (bd * N + n) * 2) : 0.0;
             for (int t = L - 1; t >= 0; --t) {
                 double ut = u[row + t];
                 double dt = delta_at(&p, d, row, t);

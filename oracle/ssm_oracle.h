@@ -34,7 +34,7 @@ void oracle_scan_bwd(const double* u, const double* delta, const double* z,
                      const int32_t* seq, const double* h0, const double* dout, double* du,
                      double* ddelta, double* dz, double* dA, double* dB,
                      double* dC, double* dD, double* ddelta_bias, double* dh0,
-                     int B, int D, int L, int N);
+                     const double* dhL, int B, int D, int L, int N);
 
 void oracle_scan_fwd_mt(const double* u, const double* delta, const double* z,
                         const double* A, const double* Dskip, const double* delta_bias,
@@ -47,7 +47,7 @@ void oracle_scan_bwd_mt(const double* u, const double* delta, const double* z,
                         const int32_t* seq, const double* h0, const double* dout, double* du,
                         double* ddelta, double* dz, double* dA, double* dB,
                         double* dC, double* dD, double* ddelta_bias, double* dh0,
-                        int B, int D, int L, int N, int nthreads);
+                        const double* dhL, int B, int D, int L, int N, int nthreads);
 /* Recurrent form, one token (x, delta, z [B][D]; Bt, Ct [B][N];
  * conv_state [B][D][W-1] and h [B][D][N] updated in place). */
 void oracle_decode_step(const double* x, double* conv_state, const double* w,
@@ -67,5 +67,5 @@ void oracle_cscan_bwd(const double* u, const double* delta, const double* z, con
                       const double* Cm, int softplus_on, const int32_t* seq, const double* h0,
                       const double* dout, double* du, double* ddelta, double* dz, double* dA,
                       double* dB, double* dC, double* dD, double* ddelta_bias, double* dh0,
-                      int B, int D, int L, int N);
+                      const double* dhL, int B, int D, int L, int N);
 #endif

@@ -744,3 +744,65 @@ def test_cscan_bwd_finite_differences(softplus):
     for name, gname in [("A", "dA"), ("Bm", "dB"), ("Cm", "dC"), ("h0", "dh0")]:
         _close(_fd(loss, parts[name + ".re"]), g[gname].real)
         _close(_fd(loss, parts[name + ".im"]), g[gname].imag)
+
+
+# --------------------------------------------------------------------------
+# a gradient reaching the final state from outside (dhL)
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("zoh", [False, True])
+def test_scan_bwd_final_state_gradient_fd(zoh):
+    """loss = <out, dout> + <final state, dhL>: every gradient against finite
+    differences, with a reset (which must stop dhL) and an initial state."""
+    rng = _rng(91)
+    seq = np.array([[0] * 6 + [1] * 14, [0] * 20], dtype=np.int32)
+    p = _problem(rng, B=2, D=3, N=4, L=20, seq=seq)
+    h0 = rng.standard_normal((2, 3, 4))
+    dout = rng.standard_normal(p["u"].shape)
+    dhL = rng.standard_normal((2, 3, 4))
+    kw = dict(z=p["z"], Dskip=p["Dskip"], delta_bias=p["delta_bias"], seq_idx=seq, zoh=zoh)
+
+    def loss():
+        r = oracle.scan_fwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], h0=h0, **kw)
+        return float(np.sum(r["out"] * dout) + np.sum(r["final_state"] * dhL))
+
+    g = oracle.scan_bwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], dout, h0=h0, dhL=dhL, **kw)
+    for name, gname in [("u", "du"), ("delta", "ddelta"), ("z", "dz"), ("A", "dA"),
+                        ("Bm", "dB"), ("Cm", "dC"), ("Dskip", "dD"),
+                        ("delta_bias", "ddelta_bias")]:
+        _close(_fd(loss, p[name]), g[gname])
+    _close(_fd(loss, h0), g["dh0"])
+    # the reset at t=6 of row 0 stops dhL from reaching h0 there
+    g0 = oracle.scan_bwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], dout, h0=h0, **kw)
+    np.testing.assert_allclose(g["dh0"][0], g0["dh0"][0], rtol=1e-13, atol=1e-13)
+    assert np.abs(g["dh0"][1] - g0["dh0"][1]).max() > 1e-6
+
+
+def test_cscan_bwd_final_state_gradient_fd():
+    rng = _rng(92)
+    seq = np.array([[0] * 11 + [1] * 9, [0] * 20], dtype=np.int32)
+    p = _cproblem(rng, seq=seq)
+    p["A"] = p["A"] + 1j * rng.standard_normal(p["A"].shape)
+    h0 = rng.standard_normal((2, 3, 4)) + 1j * rng.standard_normal((2, 3, 4))
+    dhL = rng.standard_normal((2, 3, 4)) + 1j * rng.standard_normal((2, 3, 4))
+    dout = rng.standard_normal(p["u"].shape)
+    parts = {"u": p["u"], "delta": p["delta"]}
+    for k, v in (("A", p["A"]), ("Bm", p["Bm"]), ("Cm", p["Cm"]), ("h0", h0)):
+        parts[k + ".re"] = np.ascontiguousarray(v.real)
+        parts[k + ".im"] = np.ascontiguousarray(v.imag)
+    kw = dict(z=p["z"], Dskip=p["Dskip"], delta_bias=p["delta_bias"], seq_idx=seq)
+
+    def cx(k):
+        return parts[k + ".re"] + 1j * parts[k + ".im"]
+
+    def loss():
+        r = oracle.cscan_fwd(parts["u"], parts["delta"], cx("A"), cx("Bm"), cx("Cm"), h0=cx("h0"),
+                             **kw)
+        fs = r["final_state"]
+        return float(np.sum(r["out"] * dout) + np.sum(fs.real * dhL.real + fs.imag * dhL.imag))
+
+    g = oracle.cscan_bwd(p["u"], p["delta"], p["A"], p["Bm"], p["Cm"], dout, h0=h0, dhL=dhL, **kw)
+    _close(_fd(loss, parts["u"]), g["du"])
+    _close(_fd(loss, parts["delta"]), g["ddelta"])
+    for name, gname in [("A", "dA"), ("Bm", "dB"), ("Cm", "dC"), ("h0", "dh0")]:
+        _close(_fd(loss, parts[name + ".re"]), g[gname].real)
+        _close(_fd(loss, parts[name + ".im"]), g[gname].imag)

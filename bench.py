@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -295,6 +296,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-decode", action="store_true", help="skip the recurrent-step measurement")
+    ap.add_argument("--no-complex", action="store_true", help="skip the complex-A scan measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -422,6 +424,8 @@ def main():
 
     if not args.no_decode:
         line["decode"] = decode_bench(device, sh, pk)
+    if not args.no_complex:
+        line["complex_a"] = complex_bench(device, layers[0], pk)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = cpu_count()
@@ -435,6 +439,43 @@ def main():
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def complex_bench(device, ly, pk, reps=5):
+    """The scan with a complex diagonal A (S4D-Lin: A = -1/2 + i pi n) on the
+    bench layer's shape and activations: B and C take (re, im) planes from the
+    layer's own B and C. Forward and backward timed separately with CUDA
+    events over `reps` launches each (inputs > L2)."""
+    import torch
+    import selective_state_space_35_b200 as ssm
+    B, D, N, L = ly.shape.B, ly.shape.D, ly.shape.N, ly.shape.L
+    Bc = torch.stack([ly.Bm, ly.Cm], dim=2).contiguous()
+    Cc = torch.stack([ly.Cm, ly.Bm], dim=2).contiguous()
+    A = torch.zeros((D, N, 2), dtype=torch.float32, device=device)
+    A[..., 0] = -0.5
+    A[..., 1] = torch.arange(N, dtype=torch.float32, device=device) * math.pi
+    kw = dict(z=ly.z, Dskip=ly.Dskip, delta_bias=ly.dbias, seq_idx=ly.seq)
+    out, _, ws = ssm.scan_fwd(ly.x, ly.delta, A, Bc, Cc, **kw)
+    g = ssm.scan_bwd(ly.x, ly.delta, A, Bc, Cc, ly.dout, ws, **kw)
+    torch.cuda.synchronize()
+
+    # fwd and bwd alternate (so a profiler's launch filter sees one of each
+    # per round); each is timed with its own events
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps + 1)]
+    for e in ev:
+        e[0].record()
+        ssm.scan_fwd(ly.x, ly.delta, A, Bc, Cc, out=out, workspace=ws, **kw)
+        e[1].record()
+        ssm.scan_bwd(ly.x, ly.delta, A, Bc, Cc, ly.dout, ws, grads=g, **kw)
+        e[2].record()
+    torch.cuda.synchronize()
+    fwd = sum(e[0].elapsed_time(e[1]) for e in ev[1:]) / reps   # round 0 is a warm-up
+    bwd = sum(e[1].elapsed_time(e[2]) for e in ev[1:]) / reps
+    del ws, g, out
+    return {"workload": f"complex diagonal A (S4D-Lin), B{B} x D{D} x N{N} x L{L}, bf16 "
+                        "activations, fp32 complex state, fwd + bwd",
+            "fwd_ms": fwd, "bwd_ms": bwd, "tokens_per_s": B * L / ((fwd + bwd) * 1e-3),
+            "launches": 3 * (reps + 2)}
 
 
 def decode_bench(device, sh, pk, rows_b=2048, steps=200, graph_steps=50):

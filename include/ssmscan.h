@@ -22,6 +22,11 @@
  *   zero-order hold: same page, "Discretization" (B_bar = A^{-1}(exp(dt A) - I) B).
  *   complex A: same page, "S4: Structured State Spaces for Sequences" (S4D:
  *            a diagonal A with complex entries).
+ *   pieces of a longer sequence (summaries, carries, conv halos, the final-
+ *            state gradient): the same page's associative operator ("Hardware-
+ *            Aware Parallel Scan") applied between pieces cut along L; the
+ *            Axolotl page ("FLA Mamba and Mamba2") on context parallelism
+ *            exchanging conv halos and recurrent states between shards.
  *   fused conv + scan: same page, "Hardware-Aware Parallel Scan" (kernel fusion).
  *   recurrent step: same page, "Dual Computation Modes" (recurrent mode) and
  *            "Inference (Generation)" (a (B, D, N) state carried forward).
@@ -74,7 +79,7 @@ typedef enum { SSM_DTYPE_F32 = 0, SSM_DTYPE_BF16 = 1 } ssm_dtype_t;
 const char* ssm_last_error(void);
 
 /* ABI version of this header (bumped on any incompatible change). */
-#define SSM_ABI_VERSION 4
+#define SSM_ABI_VERSION 5
 int ssm_abi_version(void);
 
 /* ---------------------------------------------------------------------------
@@ -231,13 +236,90 @@ typedef struct {
                                   order, dB and dC are summed over channels with fp32 atomics */
     float* dinitial_state;     /* [B][D][N] nullable output: dL/dh_{-1} (the gradient with
                                   respect to initial_state, or to the zero state when NULL) */
+    const float* dfinal_state; /* [B][D][N] nullable input: dL/dh_{L-1}, a gradient reaching the
+                                  final state from outside (a later piece of the sequence, a
+                                  loss on the state); NULL = 0. Complex A: (re, im) pairs */
 } ssm_scan_grads;
 
 /* Backward. Recomputes states from the checkpoints in p->workspace, so the
- * same params (inputs and workspace) as the forward must be passed. The final
- * state is not differentiated (it has no incoming gradient). */
+ * same params (inputs and workspace) as the forward must be passed. A
+ * gradient of the final state enters through g->dfinal_state. */
 ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
                           ssm_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Pieces of a longer sequence. A sequence cut along L into R consecutive
+ * pieces (for instance one per rank) is scanned piece by piece: the state
+ * entering piece r is the fold of the earlier pieces' summaries, and the
+ * gradient reaching piece r's final state is the fold of the later pieces'
+ * backward summaries. Every piece is then an ordinary ssm_scan_fwd /
+ * ssm_scan_bwd call with initial_state / dfinal_state set. Real A only
+ * (state_complex != 0: SSM_ERR_UNSUPPORTED).
+ *
+ * ssm_scan_fwd_summary — for every (b, d, n) of this piece:
+ *   decay[b][d][n]     = prod_t a_t over the piece (0 when a document starts
+ *                        inside it, or at token 0 relative to seq_prev)
+ *   state_end[b][d][n] = the final state from a zero initial state
+ * so that final state = decay * (state entering) + state_end. Reads u,
+ * delta, A, Bm (and delta_bias, seq_idx / cu_seqlens, discretization) of p;
+ * ignores initial_state, z, Cm and out. seq_prev [B] nullable: the document
+ * id of the token before token 0 (from the previous piece). Uses
+ * p->workspace as scratch (size from ssm_scan_workspace_size): call it
+ * before the piece's ssm_scan_fwd, not between that and its ssm_scan_bwd.
+ * ------------------------------------------------------------------------ */
+ssm_status_t ssm_scan_fwd_summary(const ssm_scan_params* p, const int32_t* seq_prev,
+                                  float* decay, float* state_end, ssm_stream_t stream);
+
+/* ssm_scan_bwd_summary — for every (b, d, n) of this piece, from dout alone:
+ *   decay[b][d][n]     as above
+ *   adj_start[b][d][n] = dL/dh_{-1} of the piece with no gradient reaching its
+ *                        final state (0 when token 0 starts a document)
+ * so that the gradient leaving the piece through its start is
+ * decay * (gradient of its final state) + adj_start. Reads delta, A, Cm,
+ * z, delta_bias, seq_idx / cu_seqlens of p and dout [B][D][L]; the
+ * workspace is scratch as for ssm_scan_fwd_summary (call it before the
+ * piece's ssm_scan_fwd, or after its ssm_scan_bwd). */
+ssm_status_t ssm_scan_bwd_summary(const ssm_scan_params* p, const void* dout,
+                                  const int32_t* seq_prev, float* decay, float* adj_start,
+                                  ssm_stream_t stream);
+
+/* ssm_state_carry — fold R pieces' summaries, each [B][D][N] fp32, stacked
+ * as decay [R][B][D][N] and value [R][B][D][N]:
+ *   reverse = 0: out = state entering piece r: h = init (NULL = 0), then
+ *                h = decay[j] h + value[j] for j = 0 .. r-1; h = 0 when piece
+ *                r's token 0 starts a document (seq_prev [B] and seq_idx
+ *                [B][L] of piece r given and different).
+ *   reverse = 1: out = gradient reaching piece r's final state: c = init
+ *                (NULL = 0), then c = decay[j] c + value[j] for j = R-1 .. r+1.
+ * 0 <= r < R. out [B][D][N] may not alias the inputs. */
+ssm_status_t ssm_state_carry(const float* decay, const float* value, int R, int r, int reverse,
+                             const float* init, const int32_t* seq_prev, const int32_t* seq_idx,
+                             int L, float* out, int B, int D, int N, ssm_stream_t stream);
+
+/* ssm_conv1d_fwd_ctx — ssm_conv1d_fwd for a piece of a longer sequence:
+ * the taps before token 0 read x_prev [B][D][W-1] (the W-1 inputs before
+ * the piece, oldest first; NULL = 0) under document ids seq_prev [B][W-1]
+ * (required when seq_idx and x_prev are both given). */
+ssm_status_t ssm_conv1d_fwd_ctx(const void* x, const float* w, const float* bias,
+                                const int32_t* seq_idx, const void* x_prev,
+                                const int32_t* seq_prev, void* u, int B, int D, int L, int W,
+                                ssm_dtype_t dtype, int silu, ssm_stream_t stream);
+
+/* ssm_conv1d_bwd_ctx — ssm_conv1d_bwd for a piece of a longer sequence:
+ * x_prev / seq_prev as in ssm_conv1d_fwd_ctx (the recomputed pre-activation
+ * and dw use them); x_next, du_next [B][D][W-1] and seq_next [B][W-1] are
+ * the next piece's first inputs, their upstream gradients and ids, which
+ * reach this piece's last W-1 dx through the taps (NULL = none; x_next and
+ * du_next come together; seq_next is required when seq_idx and x_next are
+ * both given). dw and dbias sum this piece's own tokens only, so a caller
+ * adds the pieces' dw and dbias. */
+ssm_status_t ssm_conv1d_bwd_ctx(const void* x, const float* w, const float* bias,
+                                const int32_t* seq_idx, const void* x_prev,
+                                const int32_t* seq_prev, const void* x_next,
+                                const void* du_next, const int32_t* seq_next, const void* du,
+                                void* dx, float* dw, float* dbias, int B, int D, int L, int W,
+                                ssm_dtype_t dtype, int silu, void* workspace,
+                                size_t workspace_bytes, ssm_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * ssm_scan_status — device-side status of the last ssm_scan_fwd / ssm_scan_bwd

@@ -17,7 +17,9 @@ from ._lib import (SsmError, ssm_abi_version, ssm_conv1d_bwd, ssm_conv1d_bwd_noa
                    ssm_conv1d_fwd, ssm_conv1d_scan_fwd, ssm_decode_params, ssm_decode_step,
                    ssm_last_error,
                    ssm_probe_ex2_rate, ssm_scan_bwd, ssm_scan_status,
-                   ssm_scan_fwd, ssm_scan_grads, ssm_scan_params, ssm_scan_workspace_size)
+                   ssm_scan_fwd, ssm_scan_grads, ssm_scan_params, ssm_scan_workspace_size,
+                   ssm_scan_fwd_summary, ssm_scan_bwd_summary, ssm_state_carry,
+                   ssm_conv1d_fwd_ctx, ssm_conv1d_bwd_ctx)
 
 __all__ = [
     "SsmError", "ssm_abi_version", "ssm_last_error", "ssm_conv1d_fwd", "ssm_conv1d_bwd",
@@ -26,7 +28,9 @@ __all__ = [
     "scan_status", "conv1d_fwd", "conv1d_bwd", "scan_params",
     "scan_workspace_size", "scan_fwd", "scan_bwd", "load",
     "ssm_decode_params", "ssm_decode_step", "decode_step", "ssm_conv1d_scan_fwd",
-    "conv1d_scan_fwd",
+    "conv1d_scan_fwd", "ssm_scan_fwd_summary", "ssm_scan_bwd_summary", "ssm_state_carry",
+    "ssm_conv1d_fwd_ctx", "ssm_conv1d_bwd_ctx", "scan_fwd_summary", "scan_bwd_summary",
+    "state_carry",
 ]
 
 load = _lib.load
@@ -81,25 +85,42 @@ def probe_ex2_rate(device=None) -> float:
     return ssm_probe_ex2_rate(_ptr(sink), sink.numel(), _stream(None, dev))
 
 
-def conv1d_fwd(x, w, bias=None, seq_idx=None, *, silu=True, out=None, stream=None):
-    """u = silu(causal depthwise conv1d(x)) (width 4, segment-masked taps)."""
+def conv1d_fwd(x, w, bias=None, seq_idx=None, *, silu=True, out=None, x_prev=None,
+               seq_prev=None, stream=None):
+    """u = silu(causal depthwise conv1d(x)) (width 4, segment-masked taps).
+
+    For a piece of a longer sequence, x_prev [B, D, 3] (x dtype) holds the 3
+    inputs before token 0 and seq_prev [B, 3] their document ids."""
     torch = _torch()
     B, D, L = x.shape
     _need(x, "x", shape=(B, D, L))
     _need(w, "w", torch.float32, (D, 4))
     _need(bias, "bias", torch.float32, (D,))
     _need(seq_idx, "seq_idx", torch.int32, (B, L))
+    _need(x_prev, "x_prev", x.dtype, (B, D, 3))
+    _need(seq_prev, "seq_prev", torch.int32, (B, 3))
     if out is None:
         out = torch.empty_like(x)
     _need(out, "out", x.dtype, (B, D, L))
-    _lib.check(ssm_conv1d_fwd(_ptr(x), _ptr(w), _ptr(bias), _ptr(seq_idx), _ptr(out), B, D, L, 4,
-                              _dtype_code(x), int(silu), _stream(stream, x.device)))
+    if x_prev is None and seq_prev is None:
+        _lib.check(ssm_conv1d_fwd(_ptr(x), _ptr(w), _ptr(bias), _ptr(seq_idx), _ptr(out), B, D, L,
+                                  4, _dtype_code(x), int(silu), _stream(stream, x.device)))
+    else:
+        _lib.check(ssm_conv1d_fwd_ctx(_ptr(x), _ptr(w), _ptr(bias), _ptr(seq_idx), _ptr(x_prev),
+                                      _ptr(seq_prev), _ptr(out), B, D, L, 4, _dtype_code(x),
+                                      int(silu), _stream(stream, x.device)))
     return out
 
 
 def conv1d_bwd(x, w, bias, seq_idx, du, *, silu=True, dx=None, dw=None, dbias=None,
-               workspace=None, stream=None):
-    """Gradients of conv1d_fwd: returns (dx, dw, dbias)."""
+               workspace=None, x_prev=None, seq_prev=None, x_next=None, du_next=None,
+               seq_next=None, stream=None):
+    """Gradients of conv1d_fwd: returns (dx, dw, dbias).
+
+    For a piece of a longer sequence: x_prev / seq_prev as in conv1d_fwd, and
+    x_next, du_next [B, D, 3], seq_next [B, 3] the next piece's first inputs,
+    upstream gradients and ids (they reach this piece's last 3 dx); dw and
+    dbias then cover this piece's own tokens."""
     torch = _torch()
     B, D, L = x.shape
     _need(x, "x", shape=(B, D, L))
@@ -107,6 +128,10 @@ def conv1d_bwd(x, w, bias, seq_idx, du, *, silu=True, dx=None, dw=None, dbias=No
     _need(w, "w", torch.float32, (D, 4))
     _need(bias, "bias", torch.float32, (D,))
     _need(seq_idx, "seq_idx", torch.int32, (B, L))
+    for t, nm in ((x_prev, "x_prev"), (x_next, "x_next"), (du_next, "du_next")):
+        _need(t, nm, x.dtype, (B, D, 3))
+    for t, nm in ((seq_prev, "seq_prev"), (seq_next, "seq_next")):
+        _need(t, nm, torch.int32, (B, 3))
     dx = torch.empty_like(x) if dx is None else dx
     dw = torch.empty((D, 4), dtype=torch.float32, device=x.device) if dw is None else dw
     if dbias is None:
@@ -114,9 +139,16 @@ def conv1d_bwd(x, w, bias, seq_idx, du, *, silu=True, dx=None, dw=None, dbias=No
     ws_bytes = ssm_conv1d_bwd_workspace_size(B, D, L, 4)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=x.device)
-    _lib.check(ssm_conv1d_bwd(_ptr(x), _ptr(w), _ptr(bias), _ptr(seq_idx), _ptr(du), _ptr(dx),
-                              _ptr(dw), _ptr(dbias), B, D, L, 4, _dtype_code(x), int(silu),
-                              _ptr(workspace), workspace.numel(), _stream(stream, x.device)))
+    if all(t is None for t in (x_prev, seq_prev, x_next, du_next, seq_next)):
+        _lib.check(ssm_conv1d_bwd(_ptr(x), _ptr(w), _ptr(bias), _ptr(seq_idx), _ptr(du), _ptr(dx),
+                                  _ptr(dw), _ptr(dbias), B, D, L, 4, _dtype_code(x), int(silu),
+                                  _ptr(workspace), workspace.numel(), _stream(stream, x.device)))
+    else:
+        _lib.check(ssm_conv1d_bwd_ctx(_ptr(x), _ptr(w), _ptr(bias), _ptr(seq_idx), _ptr(x_prev),
+                                      _ptr(seq_prev), _ptr(x_next), _ptr(du_next), _ptr(seq_next),
+                                      _ptr(du), _ptr(dx), _ptr(dw), _ptr(dbias), B, D, L, 4,
+                                      _dtype_code(x), int(silu), _ptr(workspace),
+                                      workspace.numel(), _stream(stream, x.device)))
     return dx, dw, dbias
 
 
@@ -251,13 +283,14 @@ def conv1d_scan_fwd(x, conv_w, conv_bias, delta, A, Bm, Cm, *, z=None, Dskip=Non
 
 def scan_bwd(u, delta, A, Bm, Cm, dout, workspace, *, z=None, Dskip=None, delta_bias=None,
              softplus=True, seq_idx=None, cu_seqlens=None, n_splits=0, grads=None,
-             initial_state=None, zoh=False, stream=None):
+             initial_state=None, dfinal_state=None, zoh=False, stream=None):
     """Selective scan backward; `workspace` must come from the matching scan_fwd
     (called with the same `initial_state`).
 
     Returns a dict: du, ddelta (w.r.t. the raw delta), dz (or None), dA, dB,
     dC, dD, ddelta_bias, dinitial_state (w.r.t. the state before token 0).
-    Preallocated outputs may be passed in `grads`.
+    `dfinal_state` (shaped like the final state) is a gradient reaching the
+    final state from outside. Preallocated outputs may be passed in `grads`.
     """
     torch = _torch()
     B, D, L = u.shape
@@ -289,6 +322,8 @@ def scan_bwd(u, delta, A, Bm, Cm, dout, workspace, *, z=None, Dskip=None, delta_
     gr.ddelta_bias = g["ddelta_bias"].data_ptr() if g["ddelta_bias"] is not None else None
     gr.dinitial_state = (g["dinitial_state"].data_ptr() if g["dinitial_state"] is not None
                          else None)
+    _need(dfinal_state, "dfinal_state", torch.float32, (B, D, N) + c2)
+    gr.dfinal_state = dfinal_state.data_ptr() if dfinal_state is not None else None
     _lib.check(ssm_scan_bwd(p, gr, _stream(stream, u.device)))
     return g
 
@@ -335,4 +370,71 @@ def decode_step(x, conv_state, conv_w, delta, A, Bm, Cm, state, *, conv_bias=Non
     p.state, p.out = state.data_ptr(), out.data_ptr()
     p.u_out = u_out.data_ptr() if u_out is not None else None
     _lib.check(ssm_decode_step(p, _stream(stream, x.device)))
+    return out
+
+
+def scan_fwd_summary(u, delta, A, Bm, *, delta_bias=None, softplus=True, seq_idx=None,
+                     seq_prev=None, zoh=False, workspace=None, stream=None):
+    """Summary of this piece of a longer sequence: (decay, state_end), each
+    [B, D, N] fp32, with final state = decay * (state entering) + state_end.
+    seq_prev [B] int32: document id of the token before token 0."""
+    torch = _torch()
+    B, D, L = u.shape
+    N = A.shape[1]
+    _need(seq_prev, "seq_prev", torch.int32, (B,))
+    p = scan_params(u, delta, A, Bm, Bm, delta_bias=delta_bias, softplus=softplus,
+                    seq_idx=seq_idx, zoh=zoh)
+    need = ssm_scan_workspace_size(p)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=u.device)
+    p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    decay = torch.empty((B, D, N), dtype=torch.float32, device=u.device)
+    end = torch.empty_like(decay)
+    _lib.check(ssm_scan_fwd_summary(p, _ptr(seq_prev), decay.data_ptr(), end.data_ptr(),
+                                    _stream(stream, u.device)))
+    return decay, end
+
+
+def scan_bwd_summary(delta, A, Cm, dout, *, z=None, delta_bias=None, softplus=True,
+                     seq_idx=None, seq_prev=None, workspace=None, stream=None):
+    """Backward summary of this piece from dout alone: (decay, adj_start),
+    each [B, D, N] fp32; the gradient leaving the piece through its start is
+    decay * (gradient of its final state) + adj_start."""
+    torch = _torch()
+    B, D, L = delta.shape
+    N = A.shape[1]
+    _need(dout, "dout", delta.dtype, (B, D, L))
+    _need(seq_prev, "seq_prev", torch.int32, (B,))
+    p = scan_params(delta, delta, A, Cm, Cm, z=z, delta_bias=delta_bias, softplus=softplus,
+                    seq_idx=seq_idx)
+    need = ssm_scan_workspace_size(p)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=delta.device)
+    p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    decay = torch.empty((B, D, N), dtype=torch.float32, device=delta.device)
+    adj = torch.empty_like(decay)
+    _lib.check(ssm_scan_bwd_summary(p, dout.data_ptr(), _ptr(seq_prev), decay.data_ptr(),
+                                    adj.data_ptr(), _stream(stream, delta.device)))
+    return decay, adj
+
+
+def state_carry(decay, value, r, *, reverse=False, init=None, seq_prev=None, seq_idx=None,
+                out=None, stream=None):
+    """Fold stacked piece summaries decay, value [R, B, D, N] fp32: the state
+    entering piece r (reverse=False; zero when piece r's token 0 starts a
+    document per seq_prev [B] / seq_idx [B, L]) or the gradient reaching
+    piece r's final state (reverse=True)."""
+    torch = _torch()
+    R, B, D, N = decay.shape
+    _need(decay, "decay", torch.float32)
+    _need(value, "value", torch.float32, (R, B, D, N))
+    _need(init, "init", torch.float32, (B, D, N))
+    _need(seq_prev, "seq_prev", torch.int32, (B,))
+    _need(seq_idx, "seq_idx", torch.int32)
+    L = seq_idx.shape[1] if seq_idx is not None else 0
+    out = torch.empty((B, D, N), dtype=torch.float32, device=decay.device) if out is None else out
+    _need(out, "out", torch.float32, (B, D, N))
+    _lib.check(ssm_state_carry(decay.data_ptr(), value.data_ptr(), R, int(r), int(reverse),
+                               _ptr(init), _ptr(seq_prev), _ptr(seq_idx), L, out.data_ptr(), B, D,
+                               N, _stream(stream, decay.device)))
     return out

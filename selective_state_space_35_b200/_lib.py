@@ -58,6 +58,7 @@ class ssm_scan_grads(ctypes.Structure):
         ("dA", _vp), ("dB", _vp), ("dC", _vp), ("dD", _vp), ("ddelta_bias", _vp),
         ("deterministic", _i),
         ("dinitial_state", _vp),
+        ("dfinal_state", _vp),
     ]
 
 
@@ -79,7 +80,8 @@ _lib = None
 EXPORTS = ("ssm_last_error", "ssm_abi_version", "ssm_conv1d_fwd", "ssm_conv1d_bwd_workspace_size",
            "ssm_conv1d_bwd", "ssm_conv1d_bwd_noalloc", "ssm_scan_workspace_size", "ssm_scan_fwd",
            "ssm_scan_bwd", "ssm_scan_status", "ssm_probe_ex2_rate", "ssm_decode_step",
-           "ssm_conv1d_scan_fwd")
+           "ssm_conv1d_scan_fwd", "ssm_scan_fwd_summary", "ssm_scan_bwd_summary",
+           "ssm_state_carry", "ssm_conv1d_fwd_ctx", "ssm_conv1d_bwd_ctx")
 
 
 def load(path: str | None = None):
@@ -121,6 +123,17 @@ def load(path: str | None = None):
     L.ssm_conv1d_scan_fwd.argtypes = [ctypes.POINTER(ssm_scan_params), _vp, _vp, _vp, _vp]
     L.ssm_decode_step.restype = _i
     L.ssm_decode_step.argtypes = [ctypes.POINTER(ssm_decode_params), _vp]
+    L.ssm_scan_fwd_summary.restype = _i
+    L.ssm_scan_fwd_summary.argtypes = [ctypes.POINTER(ssm_scan_params), _vp, _vp, _vp, _vp]
+    L.ssm_scan_bwd_summary.restype = _i
+    L.ssm_scan_bwd_summary.argtypes = [ctypes.POINTER(ssm_scan_params), _vp, _vp, _vp, _vp, _vp]
+    L.ssm_state_carry.restype = _i
+    L.ssm_state_carry.argtypes = [_vp, _vp, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _i, _i, _i, _vp]
+    L.ssm_conv1d_fwd_ctx.restype = _i
+    L.ssm_conv1d_fwd_ctx.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]
+    L.ssm_conv1d_bwd_ctx.restype = _i
+    L.ssm_conv1d_bwd_ctx.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                     _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
     if path is None:
         _lib = L
     return L
@@ -194,3 +207,23 @@ def ssm_conv1d_scan_fwd(params: ssm_scan_params, x, conv_w, conv_bias, stream) -
 
 def ssm_decode_step(params: ssm_decode_params, stream) -> int:
     return load().ssm_decode_step(_ref(params), stream)
+
+
+def ssm_scan_fwd_summary(params: ssm_scan_params, seq_prev, decay, state_end, stream) -> int:
+    return load().ssm_scan_fwd_summary(_ref(params), seq_prev, decay, state_end, stream)
+
+
+def ssm_scan_bwd_summary(params: ssm_scan_params, dout, seq_prev, decay, adj_start, stream) -> int:
+    return load().ssm_scan_bwd_summary(_ref(params), dout, seq_prev, decay, adj_start, stream)
+
+
+def ssm_state_carry(*args) -> int:
+    return load().ssm_state_carry(*args)
+
+
+def ssm_conv1d_fwd_ctx(*args) -> int:
+    return load().ssm_conv1d_fwd_ctx(*args)
+
+
+def ssm_conv1d_bwd_ctx(*args) -> int:
+    return load().ssm_conv1d_bwd_ctx(*args)

@@ -64,7 +64,8 @@ int sm_count() {
 
 struct ScanPlan {
   int nchunks, nsplits, chunks_per_split;
-  size_t off_seq, off_ckpt, off_y, off_sP, off_sH, off_sIn, off_pA, off_pD, off_pB, total;
+  size_t off_seq, off_ckpt, off_y, off_sP, off_sH, off_sIn, off_pA, off_pD, off_pB, off_sum,
+      total;
 };
 
 ssm_status_t check_params(const ssm_scan_params* p) {
@@ -140,6 +141,9 @@ ScanPlan plan_scan(const ssm_scan_params* p) {
   off += up(rows * s.nsplits * sizeof(float));
   s.off_pB = off;
   off += up(rows * s.nsplits * sizeof(float));
+  // whole-row summaries (ssm_scan_fwd_summary / ssm_scan_bwd_summary): two [rows][npad]
+  s.off_sum = off;
+  off += 2 * up(rows * npad * sizeof(float));
   s.total = off;
   return s;
 }
@@ -175,6 +179,7 @@ ssm_status_t build_args(const ssm_scan_params* p, const ScanPlan& pl, ssm::ScanA
   a->L = p->L;
   a->N = p->N;
   a->Npad = (p->N + 1) & ~1;
+  a->split_base = 1;
   a->nchunks = pl.nchunks;
   a->nsplits = pl.nsplits;
   a->chunks_per_split = pl.chunks_per_split;
@@ -258,7 +263,19 @@ ssm_status_t ssm_conv1d_fwd(const void* x, const float* w, const float* bias,
                             const int32_t* seq_idx, void* u, int B, int D, int L, int W,
                             ssm_dtype_t dtype, int silu, ssm_stream_t stream) {
   if (injected("ssm_conv1d_fwd")) return fail(SSM_ERR_INJECTED, "ssm_conv1d_fwd: injected failure");
+  return ssm_conv1d_fwd_ctx(x, w, bias, seq_idx, nullptr, nullptr, u, B, D, L, W, dtype, silu,
+                            stream);
+}
+
+ssm_status_t ssm_conv1d_fwd_ctx(const void* x, const float* w, const float* bias,
+                                const int32_t* seq_idx, const void* x_prev,
+                                const int32_t* seq_prev, void* u, int B, int D, int L, int W,
+                                ssm_dtype_t dtype, int silu, ssm_stream_t stream) {
+  if (injected("ssm_conv1d_fwd_ctx"))
+    return fail(SSM_ERR_INJECTED, "ssm_conv1d_fwd_ctx: injected failure");
   if (!x || !w || !u) return fail(SSM_ERR_INVALID_ARG, "x, w and u must be non-NULL");
+  if (seq_idx && x_prev && !seq_prev)
+    return fail(SSM_ERR_INVALID_ARG, "seq_prev is required with seq_idx and x_prev");
   if (B < 1 || D < 1 || L < 1) return fail(SSM_ERR_INVALID_ARG, "sizes must be >= 1");
   if (W != 4) return fail(SSM_ERR_UNSUPPORTED, "conv width W=%d (only 4)", W);
   if (B > 65535 || D > 65535) return fail(SSM_ERR_UNSUPPORTED, "B and D must be <= 65535");
@@ -267,15 +284,17 @@ ssm_status_t ssm_conv1d_fwd(const void* x, const float* w, const float* bias,
   if (x == u) return fail(SSM_ERR_INVALID_ARG, "u may not alias x");
   const size_t es = elem_size(dtype);
   if (!aligned(x, es) || !aligned(u, es) || !aligned(w, 4) || (bias && !aligned(bias, 4)) ||
-      (seq_idx && !aligned(seq_idx, 4)))
+      (seq_idx && !aligned(seq_idx, 4)) || (x_prev && !aligned(x_prev, es)) ||
+      (seq_prev && !aligned(seq_prev, 4)))
     return fail(SSM_ERR_INVALID_ARG, "misaligned pointer");
   ssm::ConvArgs a{};
   a.x = x; a.w = w; a.bias = bias; a.seq = seq_idx; a.out = u;
+  a.x_prev = x_prev; a.seq_prev = seq_idx ? seq_prev : nullptr;
   a.B = B; a.D = D; a.L = L; a.silu = silu ? 1 : 0;
   a.bf16 = dtype == SSM_DTYPE_BF16;
   a.vec = vec_ok(L, {x, u, seq_idx});
   return cuda_status(ssm::launch_conv1d_fwd(a, reinterpret_cast<cudaStream_t>(stream)),
-                     "ssm_conv1d_fwd launch");
+                     x_prev ? "ssm_conv1d_fwd_ctx launch" : "ssm_conv1d_fwd launch");
 }
 
 ssm_status_t ssm_conv1d_bwd_workspace_size(int B, int D, int L, int W, size_t* bytes) {
@@ -292,6 +311,26 @@ ssm_status_t ssm_conv1d_bwd(const void* x, const float* w, const float* bias,
                             int silu, void* workspace, size_t workspace_bytes,
                             ssm_stream_t stream) {
   if (injected("ssm_conv1d_bwd")) return fail(SSM_ERR_INJECTED, "ssm_conv1d_bwd: injected failure");
+  return ssm_conv1d_bwd_ctx(x, w, bias, seq_idx, nullptr, nullptr, nullptr, nullptr, nullptr, du,
+                            dx, dw, dbias, B, D, L, W, dtype, silu, workspace, workspace_bytes,
+                            stream);
+}
+
+ssm_status_t ssm_conv1d_bwd_ctx(const void* x, const float* w, const float* bias,
+                                const int32_t* seq_idx, const void* x_prev,
+                                const int32_t* seq_prev, const void* x_next,
+                                const void* du_next, const int32_t* seq_next, const void* du,
+                                void* dx, float* dw, float* dbias, int B, int D, int L, int W,
+                                ssm_dtype_t dtype, int silu, void* workspace,
+                                size_t workspace_bytes, ssm_stream_t stream) {
+  if (injected("ssm_conv1d_bwd_ctx"))
+    return fail(SSM_ERR_INJECTED, "ssm_conv1d_bwd_ctx: injected failure");
+  if (seq_idx && x_prev && !seq_prev)
+    return fail(SSM_ERR_INVALID_ARG, "seq_prev is required with seq_idx and x_prev");
+  if ((x_next == nullptr) != (du_next == nullptr))
+    return fail(SSM_ERR_INVALID_ARG, "x_next and du_next come together");
+  if (seq_idx && x_next && !seq_next)
+    return fail(SSM_ERR_INVALID_ARG, "seq_next is required with seq_idx and x_next");
   if (!x || !w || !du || !dx || !dw)
     return fail(SSM_ERR_INVALID_ARG, "x, w, du, dx and dw must be non-NULL");
   size_t need = 0;
@@ -307,16 +346,20 @@ ssm_status_t ssm_conv1d_bwd(const void* x, const float* w, const float* bias,
   const size_t es = elem_size(dtype);
   if (!aligned(x, es) || !aligned(du, es) || !aligned(dx, es) || !aligned(w, 4) ||
       !aligned(dw, 4) || (bias && !aligned(bias, 4)) || (dbias && !aligned(dbias, 4)) ||
-      (seq_idx && !aligned(seq_idx, 4)))
+      (seq_idx && !aligned(seq_idx, 4)) || (x_prev && !aligned(x_prev, es)) ||
+      (x_next && !aligned(x_next, es)) || (du_next && !aligned(du_next, es)) ||
+      (seq_prev && !aligned(seq_prev, 4)) || (seq_next && !aligned(seq_next, 4)))
     return fail(SSM_ERR_INVALID_ARG, "misaligned pointer");
   ssm::ConvArgs a{};
   a.x = x; a.w = w; a.bias = bias; a.seq = seq_idx; a.du = du; a.out = dx;
   a.dw = dw; a.dbias = dbias; a.partial = static_cast<float*>(workspace);
+  a.x_prev = x_prev; a.seq_prev = seq_idx ? seq_prev : nullptr;
+  a.x_next = x_next; a.du_next = du_next; a.seq_next = seq_idx ? seq_next : nullptr;
   a.B = B; a.D = D; a.L = L; a.silu = silu ? 1 : 0;
   a.bf16 = dtype == SSM_DTYPE_BF16;
   a.vec = vec_ok(L, {x, du, dx, seq_idx});
   return cuda_status(ssm::launch_conv1d_bwd(a, reinterpret_cast<cudaStream_t>(stream)),
-                     "ssm_conv1d_bwd launch");
+                     (x_prev || x_next) ? "ssm_conv1d_bwd_ctx launch" : "ssm_conv1d_bwd launch");
 }
 
 ssm_status_t ssm_conv1d_bwd_noalloc(const void* x, const float* w, const float* bias,
@@ -401,7 +444,10 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
   const void* f32s[] = {g->dA, g->dB, g->dC, g->dD, g->ddelta_bias, g->dinitial_state};
   for (const void* q : f32s)
     if (q && !aligned(q, 4)) return fail(SSM_ERR_INVALID_ARG, "fp32 gradient pointer misaligned");
-  if (p->state_complex && (!aligned(g->dA, 8) || !aligned(g->dinitial_state, 8)))
+  if (g->dfinal_state && !aligned(g->dfinal_state, 4))
+    return fail(SSM_ERR_INVALID_ARG, "dfinal_state misaligned");
+  if (p->state_complex && (!aligned(g->dA, 8) || !aligned(g->dinitial_state, 8) ||
+                           !aligned(g->dfinal_state, 8)))
     return fail(SSM_ERR_INVALID_ARG, "complex A: dA and dinitial_state must be 8-byte aligned");
   ssm::ScanArgs a;
   build_args(p, pl, &a);
@@ -415,6 +461,7 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
   a.dD = g->dD;
   a.ddelta_bias = g->ddelta_bias;
   a.dh0 = g->dinitial_state;
+  a.dhL = g->dfinal_state;
   // dB and dC take 16-byte vector atomics on the vector path
   a.vec = vec_ok(p->L, {p->u, p->delta, p->z, p->Bm, p->Cm, g->dout, g->du, g->ddelta, a.dz, a.seq,
                         g->dB, g->dC});
@@ -430,6 +477,116 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
   if (e != cudaSuccess) return cuda_status(e, "ssm_scan_bwd memset");
   if (p->state_complex) return cuda_status(ssm::launch_cscan_bwd(a, s), "ssm_scan_bwd launch");
   return cuda_status(ssm::launch_scan_bwd(a, s), "ssm_scan_bwd launch");
+}
+
+// Shared part of the two whole-row summaries: validation, args with one
+// split over the whole row, scratch in the workspace, cu_seqlens ids.
+static ssm_status_t summary_setup(const ssm_scan_params* p, const int32_t* seq_prev,
+                                  const float* decay, const float* value, ssm::ScanArgs* a,
+                                  cudaStream_t s) {
+  ssm_status_t st = check_params(p);
+  if (st != SSM_OK) return st;
+  if (p->state_complex) return fail(SSM_ERR_UNSUPPORTED, "summaries are for a real A");
+  if (!decay || !value) return fail(SSM_ERR_INVALID_ARG, "summary outputs must be non-NULL");
+  if (!p->delta || !p->A) return fail(SSM_ERR_INVALID_ARG, "delta and A must be non-NULL");
+  if (!p->workspace) return fail(SSM_ERR_INVALID_ARG, "workspace is NULL");
+  if (!aligned(p->workspace, kAlign))
+    return fail(SSM_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  const ScanPlan pl = plan_scan(p);
+  if (p->workspace_bytes < pl.total)
+    return fail(SSM_ERR_INVALID_ARG, "workspace_bytes %zu < required %zu", p->workspace_bytes,
+                pl.total);
+  const size_t es = elem_size(p->dtype);
+  const void* acts[] = {p->u, p->delta, p->z, p->Bm, p->Cm};
+  for (const void* q : acts)
+    if (q && !aligned(q, es)) return fail(SSM_ERR_INVALID_ARG, "activation pointer misaligned");
+  const void* f32s[] = {p->A, p->delta_bias, p->seq_idx, p->cu_seqlens, seq_prev, decay, value};
+  for (const void* q : f32s)
+    if (q && !aligned(q, 4)) return fail(SSM_ERR_INVALID_ARG, "fp32/int32 pointer misaligned");
+  build_args(p, pl, a);
+  a->nsplits = 1;
+  a->chunks_per_split = a->nchunks;
+  a->split_base = 0;
+  char* ws = static_cast<char*>(p->workspace);
+  const size_t rows = (size_t)p->B * p->D;
+  a->split_P = reinterpret_cast<float*>(ws + pl.off_sum);
+  a->split_H = reinterpret_cast<float*>(ws + pl.off_sum + up(rows * a->Npad * sizeof(float)));
+  return ok();
+}
+
+// First launches of a summary (after every argument check): a fresh status
+// word and the document ids from cu_seqlens.
+static ssm_status_t summary_prep(const ssm_scan_params* p, const ssm::ScanArgs& a, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(a.status, 0, sizeof(int), s);
+  if (e != cudaSuccess) return cuda_status(e, "summary status reset");
+  if (p->cu_seqlens) {
+    e = ssm::launch_cu_seqlens_to_seq(p->cu_seqlens, p->n_docs, p->L, const_cast<int32_t*>(a.seq), s);
+    if (e != cudaSuccess) return cuda_status(e, "cu_seqlens conversion");
+  }
+  return ok();
+}
+
+ssm_status_t ssm_scan_fwd_summary(const ssm_scan_params* p, const int32_t* seq_prev,
+                                  float* decay, float* state_end, ssm_stream_t stream) {
+  if (injected("ssm_scan_fwd_summary"))
+    return fail(SSM_ERR_INJECTED, "ssm_scan_fwd_summary: injected failure");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ssm::ScanArgs a;
+  ssm_status_t st = summary_setup(p, seq_prev, decay, state_end, &a, s);
+  if (st != SSM_OK) return st;
+  if (!p->u || !p->Bm) return fail(SSM_ERR_INVALID_ARG, "u and Bm must be non-NULL");
+  a.h0 = nullptr;
+  a.vec = vec_ok(p->L, {p->u, p->delta, p->Bm, a.seq});
+  st = summary_prep(p, a, s);
+  if (st != SSM_OK) return st;
+  cudaError_t e = ssm::launch_scan_fwd_summary(a, s);
+  if (e == cudaSuccess)
+    e = ssm::launch_summary_out(a.split_P, a.split_H, a.seq, seq_prev, p->L, decay, state_end,
+                                p->B, p->D, p->N, a.Npad, false, s);
+  return cuda_status(e, "ssm_scan_fwd_summary launch");
+}
+
+ssm_status_t ssm_scan_bwd_summary(const ssm_scan_params* p, const void* dout,
+                                  const int32_t* seq_prev, float* decay, float* adj_start,
+                                  ssm_stream_t stream) {
+  if (injected("ssm_scan_bwd_summary"))
+    return fail(SSM_ERR_INJECTED, "ssm_scan_bwd_summary: injected failure");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  ssm::ScanArgs a;
+  ssm_status_t st = summary_setup(p, seq_prev, decay, adj_start, &a, s);
+  if (st != SSM_OK) return st;
+  if (!p->Cm || !dout) return fail(SSM_ERR_INVALID_ARG, "Cm and dout must be non-NULL");
+  if (!aligned(dout, elem_size(p->dtype))) return fail(SSM_ERR_INVALID_ARG, "dout misaligned");
+  a.dout = dout;
+  a.vec = vec_ok(p->L, {p->delta, p->z, p->Cm, dout, a.seq});
+  st = summary_prep(p, a, s);
+  if (st != SSM_OK) return st;
+  cudaError_t e = ssm::launch_scan_bwd_summary(a, s);
+  if (e == cudaSuccess)
+    e = ssm::launch_summary_out(a.split_P, a.split_H, a.seq, seq_prev, p->L, decay, adj_start,
+                                p->B, p->D, p->N, a.Npad, true, s);
+  return cuda_status(e, "ssm_scan_bwd_summary launch");
+}
+
+ssm_status_t ssm_state_carry(const float* decay, const float* value, int R, int r, int reverse,
+                             const float* init, const int32_t* seq_prev, const int32_t* seq_idx,
+                             int L, float* out, int B, int D, int N, ssm_stream_t stream) {
+  if (injected("ssm_state_carry")) return fail(SSM_ERR_INJECTED, "ssm_state_carry: injected failure");
+  if (!decay || !value || !out) return fail(SSM_ERR_INVALID_ARG, "decay, value and out must be non-NULL");
+  if (B < 1 || D < 1 || N < 1 || R < 1 || r < 0 || r >= R)
+    return fail(SSM_ERR_INVALID_ARG, "bad sizes (B=%d D=%d N=%d R=%d r=%d)", B, D, N, R, r);
+  if (reverse != 0 && reverse != 1) return fail(SSM_ERR_INVALID_ARG, "reverse=%d", reverse);
+  if (!reverse && seq_prev && seq_idx && L < 1) return fail(SSM_ERR_INVALID_ARG, "L=%d", L);
+  if (out == decay || out == value || (init && out == init))
+    return fail(SSM_ERR_INVALID_ARG, "out may not alias the inputs");
+  const void* ps[] = {decay, value, init, seq_prev, seq_idx, out};
+  for (const void* q : ps)
+    if (q && !aligned(q, 4)) return fail(SSM_ERR_INVALID_ARG, "misaligned pointer");
+  return cuda_status(ssm::launch_state_carry(decay, value, R, r, reverse != 0, init,
+                                             reverse ? nullptr : seq_prev,
+                                             reverse ? nullptr : seq_idx, L, out, B, D, N,
+                                             reinterpret_cast<cudaStream_t>(stream)),
+                     "ssm_state_carry launch");
 }
 
 ssm_status_t ssm_scan_status(const ssm_scan_params* p, int* device_status, ssm_stream_t stream) {

@@ -20,6 +20,7 @@ template <typename T, bool VEC, bool SEQ>
 __global__ void __launch_bounds__(kConvThreads)
 conv1d_fwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
                   const float* __restrict__ bias, const int32_t* __restrict__ seq,
+                  const T* __restrict__ x_prev, const int32_t* __restrict__ seq_prev,
                   T* __restrict__ u, int D, int L, int silu) {
   const int d = blockIdx.y, b = blockIdx.z;
   const int t0 = (blockIdx.x * kConvThreads + threadIdx.x) * 8;
@@ -31,11 +32,14 @@ conv1d_fwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
   for (int k = 0; k < 4; ++k) wk[k] = __ldg(w + d * 4 + k);
   const float bs = bias ? __ldg(bias + d) : 0.0f;
 
-  float xv[11];  // x[t0-3 .. t0+7]
+  // x[t0-3 .. t0+7]; before token 0 the halo x_prev (the 3 preceding inputs)
+  // or 0
+  const T* xp = x_prev ? x_prev + ((size_t)b * D + d) * 3 : nullptr;
+  float xv[11];
 #pragma unroll
   for (int i = 0; i < 3; ++i) {
     const int s = t0 - 3 + i;
-    xv[i] = s >= 0 ? Io<T>::ld(xr + s) : 0.0f;
+    xv[i] = s >= 0 ? Io<T>::ld(xr + s) : (xp ? Io<T>::ld(xp + 3 + s) : 0.0f);
   }
   load_row8<T, VEC>(xr, t0, L, xv + 3);
 
@@ -45,7 +49,8 @@ conv1d_fwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
 #pragma unroll
     for (int i = 0; i < 11; ++i) {
       const int s = t0 - 3 + i;
-      sg[i] = (s >= 0 && s < L) ? __ldg(sr + s) : 0;
+      sg[i] = (s >= 0 && s < L) ? __ldg(sr + s)
+                                : ((s < 0 && seq_prev) ? __ldg(seq_prev + (size_t)b * 3 + 3 + s) : 0);
     }
   }
 
@@ -75,7 +80,10 @@ __global__ void __launch_bounds__(kConvThreads)
 conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
                   const float* __restrict__ bias, const int32_t* __restrict__ seq,
                   const T* __restrict__ du, T* __restrict__ dx,
-                  float* __restrict__ partial, int D, int L, int silu) {
+                  float* __restrict__ partial, const T* __restrict__ x_prev,
+                  const int32_t* __restrict__ seq_prev, const T* __restrict__ x_next,
+                  const T* __restrict__ du_next, const int32_t* __restrict__ seq_next, int D,
+                  int L, int silu) {
   const int d = blockIdx.y, b = blockIdx.z;
   const int t0 = (blockIdx.x * kConvThreads + threadIdx.x) * 8;
   const bool live = t0 < L;
@@ -94,11 +102,15 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
   for (int i = 0; i < 14; ++i) { xv[i] = 0.0f; sg[i] = 0; }
 #pragma unroll
   for (int i = 0; i < 11; ++i) duv[i] = 0.0f;
+  // halos of a row cut out of a longer sequence: the 3 inputs before token 0,
+  // and the 3 inputs and upstream gradients after token L-1
+  const size_t hrow = ((size_t)b * D + d) * 3;
   if (live) {
 #pragma unroll
     for (int i = 0; i < 3; ++i) {
       const int s = t0 - 3 + i;
       if (s >= 0) xv[i] = Io<T>::ld(xr + s);
+      else if (x_prev) xv[i] = Io<T>::ld(x_prev + hrow + 3 + s);
     }
     load_row8<T, VEC>(xr, t0, L, xv + 3);
     load_row8<T, VEC>(dur, t0, L, duv);
@@ -110,12 +122,27 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
         duv[8 + i] = Io<T>::ld(dur + s);
       }
     }
+    if (x_next && t0 + 11 > L) {
+      // tokens L .. L+2 of the window come from the next piece
+#pragma unroll
+      for (int i = 3; i < 14; ++i) {
+        const int s = t0 - 3 + i;
+        if (s >= L && s < L + 3) {
+          xv[i] = Io<T>::ld(x_next + hrow + (s - L));
+          duv[i - 3] = Io<T>::ld(du_next + hrow + (s - L));
+        }
+      }
+    }
     if (SEQ) {
       const int32_t* sr = seq + (size_t)b * L;
 #pragma unroll
       for (int i = 0; i < 14; ++i) {
         const int s = t0 - 3 + i;
-        sg[i] = (s >= 0 && s < L) ? __ldg(sr + s) : 0;
+        int v = 0;
+        if (s >= 0 && s < L) v = __ldg(sr + s);
+        else if (s < 0 && seq_prev) v = __ldg(seq_prev + (size_t)b * 3 + 3 + s);
+        else if (s >= L && s < L + 3 && seq_next) v = __ldg(seq_next + (size_t)b * 3 + (s - L));
+        sg[i] = v;
       }
     }
   }
@@ -135,7 +162,8 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
       const float sgm = sigmoid_fast(c);  // SFU sigmoid, as in the forward
       g *= sgm * (1.0f + c * (1.0f - sgm));
     }
-    dc[j] = (t0 + j < L) ? g : 0.0f;
+    // tokens past the row exist only as the next piece's halo
+    dc[j] = (t0 + j < L || (x_next && t0 + j < L + 3)) ? g : 0.0f;
   }
 
   if (live) {
@@ -157,12 +185,13 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
   float pw[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
+    const float dci = (t0 + i < L) ? dc[i] : 0.0f;  // this row's own tokens only
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const bool ok = !SEQ || sg[i + k] == sg[i + 3];
-      pw[k] = fmaf(dc[i], ok ? xv[i + k] : 0.0f, pw[k]);
+      pw[k] = fmaf(dci, ok ? xv[i + k] : 0.0f, pw[k]);
     }
-    pw[4] += dc[i];
+    pw[4] += dci;
   }
 #pragma unroll
   for (int k = 0; k < 5; ++k)
@@ -199,7 +228,8 @@ template <typename T, bool VEC, bool SEQ>
 void conv_fwd_t(const ConvArgs& a, cudaStream_t s) {
   dim3 grid(conv_tiles(a.L), a.D, a.B);
   conv1d_fwd_kernel<T, VEC, SEQ><<<grid, kConvThreads, 0, s>>>(
-      static_cast<const T*>(a.x), a.w, a.bias, a.seq, static_cast<T*>(a.out), a.D, a.L, a.silu);
+      static_cast<const T*>(a.x), a.w, a.bias, a.seq, static_cast<const T*>(a.x_prev), a.seq_prev,
+      static_cast<T*>(a.out), a.D, a.L, a.silu);
 }
 
 template <typename T, bool VEC, bool SEQ>
@@ -207,7 +237,9 @@ void conv_bwd_t(const ConvArgs& a, cudaStream_t s) {
   dim3 grid(conv_tiles(a.L), a.D, a.B);
   conv1d_bwd_kernel<T, VEC, SEQ><<<grid, kConvThreads, 0, s>>>(
       static_cast<const T*>(a.x), a.w, a.bias, a.seq, static_cast<const T*>(a.du),
-      static_cast<T*>(a.out), a.partial, a.D, a.L, a.silu);
+      static_cast<T*>(a.out), a.partial, static_cast<const T*>(a.x_prev), a.seq_prev,
+      static_cast<const T*>(a.x_next), static_cast<const T*>(a.du_next), a.seq_next, a.D, a.L,
+      a.silu);
   const int n = a.D * 5;
   conv1d_wreduce_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.partial, a.dw, a.dbias, a.B,
                                                         conv_tiles(a.L), a.D);

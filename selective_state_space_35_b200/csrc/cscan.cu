@@ -166,6 +166,29 @@ __device__ __forceinline__ unsigned block_resets(int sq, int sqp, int tok, int L
   return __ballot_sync(kFull, start) & 0xffffu;
 }
 
+// a_t = e^{dt Re A} e^{i dt Im A} for the block's 16 tokens (A's real part
+// pre-scaled by log2 e), 0 at a document start (rm: warp-uniform bit mask).
+__device__ __forceinline__ void decays(const float4* dt4, float Ar2, float Ai, unsigned rm,
+                                       float ar[kCB], float ai[kCB]) {
+#pragma unroll
+  for (int q = 0; q < kCB / 4; ++q) {
+    const float4 dq = dt4[q];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float dt = comp(dq, j);
+      const float mag = ex2_approx(dt * Ar2);
+      const float2 cs = cis(dt * Ai);
+      ar[4 * q + j] = mag * cs.x;
+      ai[4 * q + j] = mag * cs.y;
+    }
+  }
+  if (rm) {
+#pragma unroll
+    for (int t = 0; t < kCB; ++t)
+      if ((rm >> t) & 1u) ar[t] = ai[t] = 0.0f;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Forward.
 // ---------------------------------------------------------------------------
@@ -259,18 +282,16 @@ cscan_fwd_kernel(const ScanArgs p) {
     const int tb = kb * kCB;
     __syncthreads();  // block kb's tiles are complete
     if (nval) ck[(size_t)kb * kNMax] = make_float2(hr, hi);
-    const unsigned rmk = rm;
+    // the block's decays first (independent of h), then the serial chain
+    float ar_[kCB], ai_[kCB];
+    decays(dt4, Ar2, Ai, rm, ar_, ai_);
 #pragma unroll
     for (int q = 0; q < kCB / 4; ++q) {
-      const float4 dq = dt4[q], xq = xu4[q], br = Br4[q], bi = Bi4[q], cr = Cr4[q], ci = Ci4[q];
+      const float4 xq = xu4[q], br = Br4[q], bi = Bi4[q], cr = Cr4[q], ci = Ci4[q];
       float part[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const float dt = comp(dq, j), xu = comp(xq, j);
-        const float mag = ex2_approx(dt * Ar2);
-        const float2 cs = cis(dt * Ai);
-        float ar = mag * cs.x, ai = mag * cs.y;
-        if ((rmk >> (4 * q + j)) & 1u) ar = ai = 0.0f;
+        const float ar = ar_[4 * q + j], ai = ai_[4 * q + j], xu = comp(xq, j);
         const float nr = fmaf(ar, hr, fmaf(-ai, hi, xu * comp(br, j)));
         const float ni = fmaf(ar, hi, fmaf(ai, hr, xu * comp(bi, j)));
         hr = nr;
@@ -423,7 +444,14 @@ cscan_bwd_kernel(const ScanArgs p) {
   const float4* Cr4 = reinterpret_cast<const float4*>(&sm.BC[2][n][0]);
   const float4* Ci4 = reinterpret_cast<const float4*>(&sm.BC[3][n][0]);
 
-  float gr = 0.0f, gi = 0.0f;      // conj(a_{t+1}) g_{t+1} for the token after the block
+  // conj(a_{t+1}) g_{t+1} for the token after the block; after the last token
+  // the gradient of the final state
+  float gr = 0.0f, gi = 0.0f;
+  if (nval && p.dhL) {
+    const float2 v = reinterpret_cast<const float2*>(p.dhL)[rowid * N + n];
+    gr = v.x;
+    gi = v.y;
+  }
   float dAr = 0.0f, dAi = 0.0f;
 
 #pragma unroll 1
@@ -431,25 +459,19 @@ cscan_bwd_kernel(const ScanArgs p) {
     const int tb = kb * kCB;
     __syncthreads();  // block kb's tiles are complete; X is free
     const float2 hck = ck_ready;
-    const unsigned rmk = rm;
 
     // forward recompute of a_t and h_t over the block
     float Hr[kCB], Hi[kCB], Ar_[kCB], Ai_[kCB];
+    decays(dt4, Ar2, Ai, rm, Ar_, Ai_);
     {
       float hr = hck.x, hi = hck.y;
 #pragma unroll
       for (int q = 0; q < kCB / 4; ++q) {
-        const float4 dq = dt4[q], xq = xu4[q], br = Br4[q], bi = Bi4[q];
+        const float4 xq = xu4[q], br = Br4[q], bi = Bi4[q];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int t = 4 * q + j;
-          const float dt = comp(dq, j), xu = comp(xq, j);
-          const float mag = ex2_approx(dt * Ar2);
-          const float2 cs = cis(dt * Ai);
-          float ar = mag * cs.x, ai = mag * cs.y;
-          if ((rmk >> t) & 1u) ar = ai = 0.0f;
-          Ar_[t] = ar;
-          Ai_[t] = ai;
+          const float ar = Ar_[t], ai = Ai_[t], xu = comp(xq, j);
           const float nr = fmaf(ar, hr, fmaf(-ai, hi, xu * comp(br, j)));
           const float ni = fmaf(ar, hi, fmaf(ai, hr, xu * comp(bi, j)));
           Hr[t] = hr = nr;

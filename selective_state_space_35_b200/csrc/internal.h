@@ -24,6 +24,14 @@ struct ConvArgs {
   float* dw;          // bwd only
   float* dbias;       // bwd only, nullable
   float* partial;     // bwd only: [B][tiles][D][5]
+  // halos of a row cut out of a longer sequence (all nullable): the 3 inputs
+  // (and document ids) before token 0, and for the backward the 3 inputs,
+  // upstream gradients and ids after token L-1
+  const void* x_prev;       // [B][D][3]
+  const int32_t* seq_prev;  // [B][3]
+  const void* x_next;       // [B][D][3]
+  const void* du_next;      // [B][D][3]
+  const int32_t* seq_next;  // [B][3]
   int B, D, L, silu;
   bool bf16, vec;
 };
@@ -69,6 +77,8 @@ struct ScanArgs {
   float* dD;
   float* ddelta_bias;
   float* dh0;         // [B*D][N] nullable
+  const float* dhL;   // [B*D][N] nullable: dL/d(final state), the adjoint entering from the right
+  int split_base;     // first split the backward summary kernel handles (1; 0 for a whole-row summary)
   // workspace pieces
   int* status;        // sticky device status word (0 = ok, 4 = a bounded wait timed out)
   float* ckpt;        // [B*D][nchunks * 16][kNMax] state entering each 16-token block
@@ -86,6 +96,19 @@ struct ScanArgs {
 };
 
 cudaError_t launch_scan_fwd(const ScanArgs& a, cudaStream_t s);
+// Whole-row summaries (nsplits must be 1): the forward writes (prod a, h_end
+// from 0) and the backward (prod a, a_0 g_0 from a zero incoming adjoint)
+// into split_P / split_H with row stride Npad.
+cudaError_t launch_scan_fwd_summary(const ScanArgs& a, cudaStream_t s);
+cudaError_t launch_scan_bwd_summary(const ScanArgs& a, cudaStream_t s);
+// Repack [rows][Npad] summaries to [rows][N], zeroing the decay (and, with
+// zero_value, the value) of rows whose token 0 starts a new document.
+cudaError_t launch_summary_out(const float* sP, const float* sV, const int32_t* seq,
+                               const int32_t* seq_prev, int L, float* decay, float* value,
+                               int B, int D, int N, int Npad, bool zero_value, cudaStream_t s);
+cudaError_t launch_state_carry(const float* decay, const float* value, int R, int r, bool reverse,
+                               const float* init, const int32_t* seq_prev, const int32_t* seq,
+                               int L, float* out, int B, int D, int N, cudaStream_t s);
 // Complex diagonal A (A [D][N][2], Bm / Cm [B][N][2][L], states as (re, im)
 // pairs, checkpoints [B*D][nchunks * 16][kNMax][2], part_dA [B*D][N][2]).
 cudaError_t launch_cscan_fwd(const ScanArgs& a, cudaStream_t s);

@@ -217,6 +217,7 @@ scan_bwd_kernel(const ScanArgs p) {
   // a_{t+1} g_{t+1} for the first token after the current block
   float Gn = 0.0f;
   if (split + 1 < p.nsplits && nval) Gn = p.split_in[(rowid * p.nsplits + split) * p.Npad + n];
+  else if (nval && p.dhL) Gn = __ldg(p.dhL + rowid * N + n);  // the adjoint entering from the right
   float2 dA2 = f2(0.0f, 0.0f);
   float dDp = 0.0f, ddbp = 0.0f;
 
@@ -515,7 +516,7 @@ scan_bwd_summary_kernel(const ScanArgs p) {
   const int b = blockIdx.y;
   const int d = blockIdx.x * G + warp;
   const bool active = d < p.D;
-  const int split = blockIdx.z + 1;
+  const int split = blockIdx.z + p.split_base;
   const int N = p.N, L = p.L;
   const int c_begin = split * p.chunks_per_split;
   const int c_end = min(c_begin + p.chunks_per_split, p.nchunks);
@@ -588,14 +589,15 @@ scan_bwd_summary_kernel(const ScanArgs p) {
   p.split_H[(rowid * p.nsplits + split) * p.Npad + lane] = gcarry;
 }
 
-// Adjoint carry into split s from the right: c[P-1] = 0,
-// c[s-1] = P[s] c[s] + G[s].
+// Adjoint carry into split s from the right: c[P-1] = dL/d(final state)
+// (0 when absent), c[s-1] = P[s] c[s] + G[s].
 __global__ void bwd_split_carry_kernel(const float* __restrict__ P, const float* __restrict__ Gs,
-                                       float* __restrict__ cin, int rows, int nsplits, int Np) {
+                                       const float* __restrict__ dhL, float* __restrict__ cin,
+                                       int rows, int nsplits, int Np, int N) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= rows * Np) return;
   const int r = i / Np, n = i % Np;
-  float c = 0.0f;
+  float c = (dhL && n < N) ? dhL[(size_t)r * N + n] : 0.0f;
   for (int s = nsplits - 1; s >= 0; --s) {
     const size_t k = ((size_t)r * nsplits + s) * Np + n;
     cin[k] = c;
@@ -637,8 +639,9 @@ cudaError_t bwd_t(const ScanArgs& a, cudaStream_t s) {
     dim3 g1((a.D + G - 1) / G, a.B, a.nsplits - 1);
     scan_bwd_summary_kernel<T, G, VEC><<<g1, G * 32, 0, s>>>(a);
     const int n = a.B * a.D * a.Npad;
-    bwd_split_carry_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.split_P, a.split_H, a.split_in,
-                                                          a.B * a.D, a.nsplits, a.Npad);
+    bwd_split_carry_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.split_P, a.split_H, a.dhL,
+                                                          a.split_in, a.B * a.D, a.nsplits,
+                                                          a.Npad, a.N);
   }
   const size_t smem = sizeof(BwdSmem<T>);
   static bool smem_set = false;  // once per instantiation and process (a benign race)
@@ -668,6 +671,20 @@ cudaError_t bwd_dispatch(const ScanArgs& a, cudaStream_t s) {
 
 cudaError_t launch_scan_bwd(const ScanArgs& a, cudaStream_t s) {
   return a.zoh ? bwd_dispatch<true>(a, s) : bwd_dispatch<false>(a, s);
+}
+
+cudaError_t launch_scan_bwd_summary(const ScanArgs& a, cudaStream_t s) {
+  // the whole row as one split: split index 0 covers every chunk
+  constexpr int G = 4;
+  dim3 g((a.D + G - 1) / G, a.B, 1);
+  if (a.bf16) {
+    if (a.vec) scan_bwd_summary_kernel<__nv_bfloat16, G, true><<<g, G * 32, 0, s>>>(a);
+    else scan_bwd_summary_kernel<__nv_bfloat16, G, false><<<g, G * 32, 0, s>>>(a);
+  } else {
+    if (a.vec) scan_bwd_summary_kernel<float, G, true><<<g, G * 32, 0, s>>>(a);
+    else scan_bwd_summary_kernel<float, G, false><<<g, G * 32, 0, s>>>(a);
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace ssm

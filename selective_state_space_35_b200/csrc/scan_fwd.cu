@@ -408,6 +408,31 @@ cudaError_t launch_scan_fwd(const ScanArgs& a, cudaStream_t s) {
   return a.N == 16 ? fwd_dispatch<16, false, false>(a, s) : fwd_dispatch<0, false, false>(a, s);
 }
 
+namespace {
+template <typename T, int G, bool VEC, int NT, bool ZOH>
+cudaError_t fwd_summary_t(const ScanArgs& a, cudaStream_t s) {
+  cudaError_t e = fwd_smem_attr<T, G, VEC, true, NT, false, ZOH>();
+  if (e != cudaSuccess) return e;
+  dim3 g((a.D + G - 1) / G, a.B, 1);  // one split: the whole row
+  scan_fwd_kernel<T, G, VEC, true, NT, false, ZOH><<<g, G * 32, sizeof(FwdSmem<G>), s>>>(a);
+  return cudaGetLastError();
+}
+
+template <int NT, bool ZOH>
+cudaError_t fwd_summary_dispatch(const ScanArgs& a, cudaStream_t s) {
+  if (a.bf16)
+    return a.vec ? fwd_summary_t<__nv_bfloat16, 4, true, NT, ZOH>(a, s)
+                 : fwd_summary_t<__nv_bfloat16, 4, false, NT, ZOH>(a, s);
+  return a.vec ? fwd_summary_t<float, 4, true, NT, ZOH>(a, s)
+               : fwd_summary_t<float, 4, false, NT, ZOH>(a, s);
+}
+}  // namespace
+
+cudaError_t launch_scan_fwd_summary(const ScanArgs& a, cudaStream_t s) {
+  if (a.zoh) return fwd_summary_dispatch<0, true>(a, s);
+  return a.N == 16 ? fwd_summary_dispatch<16, false>(a, s) : fwd_summary_dispatch<0, false>(a, s);
+}
+
 cudaError_t launch_cu_seqlens_to_seq(const int32_t* cu, int n_docs, int L, int32_t* seq,
                                      cudaStream_t s) {
   cu_seqlens_to_seq_kernel<<<(L + 255) / 256, 256, 0, s>>>(cu, n_docs, L, seq);

@@ -190,7 +190,7 @@ def test_decode_null_params(ssm):
 
 def test_grads_struct_has_initial_state_gradient(ssm):
     names = [f[0] for f in ssm.ssm_scan_grads._fields_]
-    assert names[-1] == "dinitial_state"
+    assert names[-2:] == ["dinitial_state", "dfinal_state"]
     assert [f[0] for f in ssm.ssm_scan_params._fields_][-3:] == ["initial_state", "discretization",
                                                                  "state_complex"]
 
@@ -230,3 +230,35 @@ def test_complex_a_rules(ssm):
     assert "8-byte" in ssm.ssm_last_error()
     p = _params(ssm, **good)
     assert L.ssm_conv1d_scan_fwd(ctypes.byref(p), fake + (1 << 24), fake, None, None) == 2
+
+
+def test_piece_calls_validation(ssm):
+    """Summaries, carry and conv halos reject bad arguments before any launch."""
+    from selective_state_space_35_b200 import _lib
+    L = _lib.load()
+    fake = 1 << 20
+    good = dict(u=fake, delta=fake + 4096, A=fake + 8192, Bm=fake + 12288, Cm=fake + 16384,
+                out=fake + 20480, workspace=fake + 65536, workspace_bytes=1 << 30)
+    dec, val = fake + (1 << 22), fake + (1 << 23)
+    p = _params(ssm, **dict(good, state_complex=1))
+    assert L.ssm_scan_fwd_summary(ctypes.byref(p), None, dec, val, None) == 2
+    p = _params(ssm, **good)
+    assert L.ssm_scan_fwd_summary(ctypes.byref(p), None, None, val, None) == 1
+    assert L.ssm_scan_bwd_summary(ctypes.byref(p), None, None, dec, val, None) == 1   # no dout
+    p = _params(ssm, **dict(good, workspace_bytes=16))
+    assert L.ssm_scan_fwd_summary(ctypes.byref(p), None, dec, val, None) == 1
+    assert "workspace" in ssm.ssm_last_error()
+    # carry: r outside [0, R), bad direction, aliasing
+    assert L.ssm_state_carry(dec, val, 2, 2, 0, None, None, None, 0, fake, 2, 8, 16, None) == 1
+    assert L.ssm_state_carry(dec, val, 2, 1, 3, None, None, None, 0, fake, 2, 8, 16, None) == 1
+    assert L.ssm_state_carry(dec, val, 2, 1, 0, None, None, None, 0, dec, 2, 8, 16, None) == 1
+    # conv halos: ids needed with a segmented row, x_next and du_next together
+    x, w, u = fake, fake + 4096, fake + 8192
+    assert L.ssm_conv1d_fwd_ctx(x, w, None, fake + 12288, fake + 16384, None, u, 2, 8, 64, 4, 1, 1,
+                                None) == 1
+    assert L.ssm_conv1d_bwd_ctx(x, w, None, None, None, None, fake + 16384, None, None, fake, u,
+                                fake + 20480, None, 2, 8, 64, 4, 1, 1, fake + 65536, 1 << 20,
+                                None) == 1
+    assert L.ssm_conv1d_bwd_ctx(x, w, None, fake + 12288, None, None, fake + 16384, fake + 24576,
+                                None, fake, u, fake + 20480, None, 2, 8, 64, 4, 1, 1,
+                                fake + 65536, 1 << 20, None) == 1

@@ -14,10 +14,13 @@
 // with dy_t = dout_t silu(z_t).
 //
 // One thread per (row, state): both recurrences are serial per-thread
-// chains, so there is no scan. The per-token sums over states go through a
-// per-warp shared-memory transposition; dB / dC (sums over every channel of a
-// batch row) are added over the CTA's rows in shared memory and sent to HBM
-// with one float4 atomic per 4 tokens. dA, dD and the delta-bias gradient are
+// chains, so there is no scan. The per-token sums over states (for du and
+// d delta) are a register butterfly of warp shuffles over the 16 lanes of a
+// row, 8 tokens at a time: halving at lane distances 2 and 1, adding at 4
+// and 8, which leaves lane n with tokens 2n and 2n + 1. dB / dC (sums over
+// every channel of a batch row) go from the adjoint into a per-warp shared
+// buffer, are added over the CTA's rows there and sent to HBM with one
+// float4 atomic per 4 tokens. dA, dD and the delta-bias gradient are
 // per-row partials reduced over batch (and splits) in a fixed order by a
 // small kernel.
 #include "scan_common.cuh"
@@ -82,7 +85,7 @@ struct BwdSmem {
   float xu[kRows][kBlk];                   // dt u
   float dy[kRows][kBlk];                   // dL/dy = dout silu(z)
   float uu[kRows][kBlk];                   // u (zero-order hold only)
-  float X[kWarps][2][2][kNMax][kLd];       // [warp][array][row half][state][token]
+  float X[kWarps][2][2][kNMax][kLd];       // [warp][dB, dC][row half][state][token]
 };
 
 template <int BYTES>
@@ -346,9 +349,10 @@ scan_bwd_kernel(const ScanArgs p) {
     // adjoint backwards over the block, g_t = dy_t C_t + a_{t+1} g_{t+1}
     // (a recomputed), with q_t = g_t a_t h_{t-1} and this state's terms of
     // the per-token sums
-    float4 G4[kBlk / 4];
+    float2 sg = f2(0.0f, 0.0f), sq = f2(0.0f, 0.0f);
     {
       float gnext = Gn, anext = 1.0f;
+      float vg[8], va[8];
 #pragma unroll
       for (int q = kBlk / 4 - 1; q >= 0; --q) {
         const float4 yq = dy4[q], cq = C4[q], dq = dt4[q], bq = B4[q];
@@ -377,13 +381,14 @@ scan_bwd_kernel(const ScanArgs p) {
         dA2 = ffma2(f2(dq.x, dq.y), q0, dA2);
         dA2 = ffma2(f2(dq.z, dq.w), q1, dA2);
         float2 gb0, gb1, aq0 = fmul2(Ap, q0), aq1 = fmul2(Ap, q1);
+        float4 gv;
         if (ZOH) {
           const float4 uq = uu4[q];
           const float x0 = e0.x * kLn2, x1 = e0.y * kLn2, x2 = e1.x * kLn2, x3 = e1.y * kLn2;
           // g E1 carries B_bar's factor into du (via g E1 B) and dB (via g E1 dt u)
           const float2 ge0 = fmul2(f2(g0, g1), f2(zoh_e1(x0, au.x), zoh_e1(x1, au.y)));
           const float2 ge1 = fmul2(f2(g2, g3), f2(zoh_e1(x2, au.z), zoh_e1(x3, au.w)));
-          G4[q] = make_float4(ge0.x, ge0.y, ge1.x, ge1.y);
+          gv = make_float4(ge0.x, ge0.y, ge1.x, ge1.y);
           gb0 = fmul2(ge0, f2(bq.x, bq.y));
           gb1 = fmul2(ge1, f2(bq.z, bq.w));
           // g B u: d(dt) takes it times a, dA times dt^2 E2(dt A)
@@ -396,41 +401,58 @@ scan_bwd_kernel(const ScanArgs p) {
           dA2 = ffma2(fmul2(gbu0, d2a), f2(zoh_e2(x0, au.x), zoh_e2(x1, au.y)), dA2);
           dA2 = ffma2(fmul2(gbu1, d2b), f2(zoh_e2(x2, au.z), zoh_e2(x3, au.w)), dA2);
         } else {
-          G4[q] = make_float4(g0, g1, g2, g3);
+          gv = make_float4(g0, g1, g2, g3);
           gb0 = fmul2(f2(g0, g1), f2(bq.x, bq.y));
           gb1 = fmul2(f2(g2, g3), f2(bq.z, bq.w));
         }
-        reinterpret_cast<float4*>(Xg)[q] = make_float4(gb0.x, gb0.y, gb1.x, gb1.y);
-        reinterpret_cast<float4*>(Xa)[q] = make_float4(aq0.x, aq0.y, aq1.x, aq1.y);
+        {
+          // dB_t = g_t dt_t u_t and dC_t = dy_t h_t straight into the row's buffers
+          const float4 xq = xu4[q];
+          const float2 db0 = fmul2(f2(gv.x, gv.y), f2(xq.x, xq.y));
+          const float2 db1 = fmul2(f2(gv.z, gv.w), f2(xq.z, xq.w));
+          const float2 dc0 = fmul2(f2(yq.x, yq.y), f2(H4[q].x, H4[q].y));
+          const float2 dc1 = fmul2(f2(yq.z, yq.w), f2(H4[q].z, H4[q].w));
+          reinterpret_cast<float4*>(Xg)[q] = make_float4(db0.x, db0.y, db1.x, db1.y);
+          reinterpret_cast<float4*>(Xa)[q] = make_float4(dc0.x, dc0.y, dc1.x, dc1.y);
+          // this state's terms of tokens 4q .. 4q+3: slot (q & 1) of the chunk pair
+          const int o = (q & 1) * 4;
+          vg[o] = gb0.x; vg[o + 1] = gb0.y; vg[o + 2] = gb1.x; vg[o + 3] = gb1.y;
+          va[o] = aq0.x; va[o + 1] = aq0.y; va[o + 2] = aq1.x; va[o + 3] = aq1.y;
+          if ((q & 1) == 0) {
+            // sums over the 16 states of tokens 8c .. 8c+7 (c = q / 2): halve at lane
+            // distances 2 and 1, add at 4 and 8; lane n keeps tokens 8c + 2(n&3) + i
+            const bool b1 = (n >> 1) & 1, b0 = n & 1;
+            float g4[4], a4[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float gs = b1 ? vg[i] : vg[i + 4], gk = b1 ? vg[i + 4] : vg[i];
+              const float as = b1 ? va[i] : va[i + 4], ak = b1 ? va[i + 4] : va[i];
+              g4[i] = gk + __shfl_xor_sync(kFull, gs, 2);
+              a4[i] = ak + __shfl_xor_sync(kFull, as, 2);
+            }
+            float g2[2], a2[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const float gs = b0 ? g4[i] : g4[i + 2], gk = b0 ? g4[i + 2] : g4[i];
+              const float as = b0 ? a4[i] : a4[i + 2], ak = b0 ? a4[i + 2] : a4[i];
+              g2[i] = gk + __shfl_xor_sync(kFull, gs, 1);
+              a2[i] = ak + __shfl_xor_sync(kFull, as, 1);
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              g2[i] += __shfl_xor_sync(kFull, g2[i], 4);
+              a2[i] += __shfl_xor_sync(kFull, a2[i], 4);
+              g2[i] += __shfl_xor_sync(kFull, g2[i], 8);
+              a2[i] += __shfl_xor_sync(kFull, a2[i], 8);
+            }
+            if ((q >> 1) == (n >> 2)) {  // lane n takes tokens 2n, 2n + 1
+              sg = f2(g2[0], g2[1]);
+              sq = f2(a2[0], a2[1]);
+            }
+          }
+        }
       }
       Gn = anext * gnext;
-    }
-    __syncwarp();
-    // sums over the states for tokens 2n, 2n + 1 of row r
-    float2 sg, sq;
-    {
-      float2 s1a = f2(0.0f, 0.0f), s1b = s1a, s2a = s1a, s2b = s1a;
-#pragma unroll
-      for (int m = 0; m < kNMax; m += 2) {
-        s1a = __fadd2_rn(s1a, *reinterpret_cast<const float2*>(&sm.X[warp][0][hf][m][2 * n]));
-        s1b = __fadd2_rn(s1b, *reinterpret_cast<const float2*>(&sm.X[warp][0][hf][m + 1][2 * n]));
-        s2a = __fadd2_rn(s2a, *reinterpret_cast<const float2*>(&sm.X[warp][1][hf][m][2 * n]));
-        s2b = __fadd2_rn(s2b, *reinterpret_cast<const float2*>(&sm.X[warp][1][hf][m + 1][2 * n]));
-      }
-      sg = __fadd2_rn(s1a, s1b);
-      sq = __fadd2_rn(s2a, s2b);
-    }
-    __syncwarp();
-    // this row's dB_t = g_t dt_t u_t and dC_t = dy_t h_t
-#pragma unroll
-    for (int q = 0; q < kBlk / 4; ++q) {
-      const float4 xq = xu4[q], yq = dy4[q];
-      const float2 db0 = fmul2(f2(G4[q].x, G4[q].y), f2(xq.x, xq.y));
-      const float2 db1 = fmul2(f2(G4[q].z, G4[q].w), f2(xq.z, xq.w));
-      const float2 dc0 = fmul2(f2(yq.x, yq.y), f2(H4[q].x, H4[q].y));
-      const float2 dc1 = fmul2(f2(yq.z, yq.w), f2(H4[q].z, H4[q].w));
-      reinterpret_cast<float4*>(Xg)[q] = make_float4(db0.x, db0.y, db1.x, db1.y);
-      reinterpret_cast<float4*>(Xa)[q] = make_float4(dc0.x, dc0.y, dc1.x, dc1.y);
     }
     __syncthreads();  // every row's dB / dC terms are in X; tiles and per-token arrays are free
     // CTA sum over its rows; one float4 atomic per 4 tokens of dB / dC

@@ -318,6 +318,7 @@ scan_bwd_kernel(const ScanArgs p) {
 
     // forward recompute of h over the block from its checkpoint
     float4 H4[kBlk / 4];
+    float4 Aq[ZOH ? 1 : kBlk / 4];  // the block's decays, kept for the adjoint (dt B only)
     {
       float hh = hck;
 #pragma unroll
@@ -339,6 +340,7 @@ scan_bwd_kernel(const ScanArgs p) {
           b0 = fmul2(b0, f2(zoh_e1(e0.x * kLn2, ex2_approx(e0.x)), zoh_e1(e0.y * kLn2, ex2_approx(e0.y))));
           b1 = fmul2(b1, f2(zoh_e1(e1.x * kLn2, ex2_approx(e1.x)), zoh_e1(e1.y * kLn2, ex2_approx(e1.y))));
         }
+        if (!ZOH) Aq[q] = make_float4(a0, a1, a2, a3);
         H4[q].x = hh = fmaf(a0, hh, b0.x);
         H4[q].y = hh = fmaf(a1, hh, b0.y);
         H4[q].z = hh = fmaf(a2, hh, b1.x);
@@ -347,8 +349,9 @@ scan_bwd_kernel(const ScanArgs p) {
     }
 
     // adjoint backwards over the block, g_t = dy_t C_t + a_{t+1} g_{t+1}
-    // (a recomputed), with q_t = g_t a_t h_{t-1} and this state's terms of
-    // the per-token sums
+    // (a kept from the recompute; the zero-order hold recomputes it, as its
+    // terms need a before the document mask), with q_t = g_t a_t h_{t-1} and
+    // this state's terms of the per-token sums
     float2 sg = f2(0.0f, 0.0f), sq = f2(0.0f, 0.0f);
     {
       float gnext = Gn, anext = 1.0f;
@@ -359,10 +362,15 @@ scan_bwd_kernel(const ScanArgs p) {
         const float2 gy0 = fmul2(f2(yq.x, yq.y), f2(cq.x, cq.y));
         const float2 gy1 = fmul2(f2(yq.z, yq.w), f2(cq.z, cq.w));
         const float2 e0 = fmul2(f2(dq.x, dq.y), A2), e1 = fmul2(f2(dq.z, dq.w), A2);
-        float a0 = ex2_approx(e0.x), a1 = ex2_approx(e0.y);
-        float a2 = ex2_approx(e1.x), a3 = ex2_approx(e1.y);
+        float a0, a1, a2, a3;
+        if (ZOH) {
+          a0 = ex2_approx(e0.x); a1 = ex2_approx(e0.y);
+          a2 = ex2_approx(e1.x); a3 = ex2_approx(e1.y);
+        } else {
+          a0 = Aq[ZOH ? 0 : q].x; a1 = Aq[ZOH ? 0 : q].y; a2 = Aq[ZOH ? 0 : q].z; a3 = Aq[ZOH ? 0 : q].w;
+        }
         const float4 au = make_float4(a0, a1, a2, a3);  // before document resets (ZOH terms)
-        if (rm) {
+        if (ZOH && rm) {
           const unsigned m4 = rm >> (4 * q);
           if (m4 & 1u) a0 = 0.0f;
           if (m4 & 2u) a1 = 0.0f;

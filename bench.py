@@ -46,7 +46,7 @@ SFU_EX2_PER_CLK_PER_SM = 16  # MUFU ex2 results per SM per clock (ssm_probe_ex2_
 # (one layer B2 D1536 N16 L32768 bf16), from
 # one ncu capture (summarised under profiles/); a kernel changed since its
 # capture has no entry.
-NCU_TRAFFIC = {"scan_fwd": 612253e3 + 757312e3}
+NCU_TRAFFIC = {"scan_bwd": 1432608e3 + 598273e3, "scan_fwd": 612232e3 + 760125e3}
 
 
 def _peaks():

@@ -16,7 +16,9 @@ namespace ssm {
 
 namespace {
 
-template <typename T, bool VEC, bool SEQ>
+// HALO: the row is a piece of a longer sequence (halo pointers may be set);
+// without it the halo code is compiled out of the common path.
+template <typename T, bool VEC, bool SEQ, bool HALO>
 __global__ void __launch_bounds__(kConvThreads)
 conv1d_fwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
                   const float* __restrict__ bias, const int32_t* __restrict__ seq,
@@ -34,7 +36,7 @@ conv1d_fwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
 
   // x[t0-3 .. t0+7]; before token 0 the halo x_prev (the 3 preceding inputs)
   // or 0
-  const T* xp = x_prev ? x_prev + ((size_t)b * D + d) * 3 : nullptr;
+  const T* xp = (HALO && x_prev) ? x_prev + ((size_t)b * D + d) * 3 : nullptr;
   float xv[11];
 #pragma unroll
   for (int i = 0; i < 3; ++i) {
@@ -50,7 +52,7 @@ conv1d_fwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
     for (int i = 0; i < 11; ++i) {
       const int s = t0 - 3 + i;
       sg[i] = (s >= 0 && s < L) ? __ldg(sr + s)
-                                : ((s < 0 && seq_prev) ? __ldg(seq_prev + (size_t)b * 3 + 3 + s) : 0);
+                                : ((HALO && s < 0 && seq_prev) ? __ldg(seq_prev + (size_t)b * 3 + 3 + s) : 0);
     }
   }
 
@@ -75,7 +77,7 @@ conv1d_fwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
 // Each thread recomputes c_t for its 8 tokens plus the 3 after them, writes
 // dx for its 8 tokens, and adds its tokens' share of dw and dbias into a
 // per-CTA partial (reduced over (b, tile) by conv1d_wreduce_kernel).
-template <typename T, bool VEC, bool SEQ>
+template <typename T, bool VEC, bool SEQ, bool HALO>
 __global__ void __launch_bounds__(kConvThreads)
 conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
                   const float* __restrict__ bias, const int32_t* __restrict__ seq,
@@ -110,7 +112,7 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
     for (int i = 0; i < 3; ++i) {
       const int s = t0 - 3 + i;
       if (s >= 0) xv[i] = Io<T>::ld(xr + s);
-      else if (x_prev) xv[i] = Io<T>::ld(x_prev + hrow + 3 + s);
+      else if (HALO && x_prev) xv[i] = Io<T>::ld(x_prev + hrow + 3 + s);
     }
     load_row8<T, VEC>(xr, t0, L, xv + 3);
     load_row8<T, VEC>(dur, t0, L, duv);
@@ -122,7 +124,7 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
         duv[8 + i] = Io<T>::ld(dur + s);
       }
     }
-    if (x_next && t0 + 11 > L) {
+    if (HALO && x_next && t0 + 11 > L) {
       // tokens L .. L+2 of the window come from the next piece
 #pragma unroll
       for (int i = 3; i < 14; ++i) {
@@ -140,8 +142,9 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
         const int s = t0 - 3 + i;
         int v = 0;
         if (s >= 0 && s < L) v = __ldg(sr + s);
-        else if (s < 0 && seq_prev) v = __ldg(seq_prev + (size_t)b * 3 + 3 + s);
-        else if (s >= L && s < L + 3 && seq_next) v = __ldg(seq_next + (size_t)b * 3 + (s - L));
+        else if (HALO && s < 0 && seq_prev) v = __ldg(seq_prev + (size_t)b * 3 + 3 + s);
+        else if (HALO && s >= L && s < L + 3 && seq_next)
+          v = __ldg(seq_next + (size_t)b * 3 + (s - L));
         sg[i] = v;
       }
     }
@@ -163,7 +166,7 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
       g *= sgm * (1.0f + c * (1.0f - sgm));
     }
     // tokens past the row exist only as the next piece's halo
-    dc[j] = (t0 + j < L || (x_next && t0 + j < L + 3)) ? g : 0.0f;
+    dc[j] = (t0 + j < L || (HALO && x_next && t0 + j < L + 3)) ? g : 0.0f;
   }
 
   if (live) {
@@ -185,7 +188,8 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
   float pw[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float dci = (t0 + i < L) ? dc[i] : 0.0f;  // this row's own tokens only
+    // this row's own tokens only (past L, dc is nonzero only with a next-piece halo)
+    const float dci = (HALO && t0 + i >= L) ? 0.0f : dc[i];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const bool ok = !SEQ || sg[i + k] == sg[i + 3];
@@ -224,18 +228,24 @@ __global__ void conv1d_wreduce_kernel(const float* __restrict__ partial, float* 
   else if (dbias) dbias[d] = s;
 }
 
-template <typename T, bool VEC, bool SEQ>
-void conv_fwd_t(const ConvArgs& a, cudaStream_t s) {
+template <typename T, bool VEC, bool SEQ, bool HALO>
+void conv_fwd_h(const ConvArgs& a, cudaStream_t s) {
   dim3 grid(conv_tiles(a.L), a.D, a.B);
-  conv1d_fwd_kernel<T, VEC, SEQ><<<grid, kConvThreads, 0, s>>>(
+  conv1d_fwd_kernel<T, VEC, SEQ, HALO><<<grid, kConvThreads, 0, s>>>(
       static_cast<const T*>(a.x), a.w, a.bias, a.seq, static_cast<const T*>(a.x_prev), a.seq_prev,
       static_cast<T*>(a.out), a.D, a.L, a.silu);
 }
 
 template <typename T, bool VEC, bool SEQ>
-void conv_bwd_t(const ConvArgs& a, cudaStream_t s) {
+void conv_fwd_t(const ConvArgs& a, cudaStream_t s) {
+  if (a.x_prev) conv_fwd_h<T, VEC, SEQ, true>(a, s);
+  else conv_fwd_h<T, VEC, SEQ, false>(a, s);
+}
+
+template <typename T, bool VEC, bool SEQ, bool HALO>
+void conv_bwd_h(const ConvArgs& a, cudaStream_t s) {
   dim3 grid(conv_tiles(a.L), a.D, a.B);
-  conv1d_bwd_kernel<T, VEC, SEQ><<<grid, kConvThreads, 0, s>>>(
+  conv1d_bwd_kernel<T, VEC, SEQ, HALO><<<grid, kConvThreads, 0, s>>>(
       static_cast<const T*>(a.x), a.w, a.bias, a.seq, static_cast<const T*>(a.du),
       static_cast<T*>(a.out), a.partial, static_cast<const T*>(a.x_prev), a.seq_prev,
       static_cast<const T*>(a.x_next), static_cast<const T*>(a.du_next), a.seq_next, a.D, a.L,
@@ -243,6 +253,12 @@ void conv_bwd_t(const ConvArgs& a, cudaStream_t s) {
   const int n = a.D * 5;
   conv1d_wreduce_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.partial, a.dw, a.dbias, a.B,
                                                         conv_tiles(a.L), a.D);
+}
+
+template <typename T, bool VEC, bool SEQ>
+void conv_bwd_t(const ConvArgs& a, cudaStream_t s) {
+  if (a.x_prev || a.x_next) conv_bwd_h<T, VEC, SEQ, true>(a, s);
+  else conv_bwd_h<T, VEC, SEQ, false>(a, s);
 }
 
 }  // namespace

@@ -5,7 +5,10 @@ Each function marshals torch CUDA tensors to the C ABI of libssmscan
 runs in the library's kernels. Tensors must be CUDA and C-contiguous; layouts
 are activations [B, D, L], B/C [B, N, L], A [D, N], per-channel vectors [D],
 conv weight [D, 4], seq_idx int32 [B, L]. Activations are bf16 or fp32;
-parameters and the gradients of parameters, B and C are fp32.
+parameters and the gradients of parameters, B and C are fp32. A complex
+diagonal A is passed as [D, N, 2] (B/C [B, N, 2, L], states [B, D, N, 2]).
+Pieces of a longer sequence (summaries, carries, conv halos) serve the
+context-parallel driver in `cp.py`.
 """
 from __future__ import annotations
 
@@ -382,6 +385,7 @@ def scan_fwd_summary(u, delta, A, Bm, *, delta_bias=None, softplus=True, seq_idx
     B, D, L = u.shape
     N = A.shape[1]
     _need(seq_prev, "seq_prev", torch.int32, (B,))
+    # the forward summary reads no C: Bm fills that slot of the parameter block
     p = scan_params(u, delta, A, Bm, Bm, delta_bias=delta_bias, softplus=softplus,
                     seq_idx=seq_idx, zoh=zoh)
     need = ssm_scan_workspace_size(p)
@@ -405,6 +409,7 @@ def scan_bwd_summary(delta, A, Cm, dout, *, z=None, delta_bias=None, softplus=Tr
     N = A.shape[1]
     _need(dout, "dout", delta.dtype, (B, D, L))
     _need(seq_prev, "seq_prev", torch.int32, (B,))
+    # the backward summary reads no u and no B: delta and Cm fill those slots
     p = scan_params(delta, delta, A, Cm, Cm, z=z, delta_bias=delta_bias, softplus=softplus,
                     seq_idx=seq_idx)
     need = ssm_scan_workspace_size(p)

@@ -97,9 +97,9 @@ class GpuOps:
         return self.conv1d_bwd(x, w, b, seq, du, x_prev=x_prev, seq_prev=seq_prev, x_next=x_next,
                                du_next=du_next, seq_next=seq_next)
 
-    def scan_fwd_summary(self, u, delta, A, Bm, seq, seq_prev, delta_bias, softplus):
+    def scan_fwd_summary(self, u, delta, A, Bm, seq, seq_prev, delta_bias, softplus, zoh):
         return self.fwd_summary(u, delta, A, Bm, delta_bias=delta_bias, softplus=softplus,
-                                seq_idx=seq, seq_prev=seq_prev)
+                                seq_idx=seq, seq_prev=seq_prev, zoh=zoh)
 
     def scan_bwd_summary(self, delta, A, Cm, dout, z, seq, seq_prev, delta_bias, softplus):
         return self.bwd_summary(delta, A, Cm, dout, z=z, delta_bias=delta_bias, softplus=softplus,
@@ -109,31 +109,34 @@ class GpuOps:
         return self.carry(decay, value, r, reverse=reverse, init=init, seq_prev=seq_prev,
                           seq_idx=seq)
 
-    def scan_forward(self, u, delta, A, Bm, Cm, z, Dskip, delta_bias, softplus, seq, h0):
+    def scan_forward(self, u, delta, A, Bm, Cm, z, Dskip, delta_bias, softplus, seq, h0, zoh):
         return self.scan_fwd(u, delta, A, Bm, Cm, z=z, Dskip=Dskip, delta_bias=delta_bias,
                              softplus=softplus, seq_idx=seq, return_final_state=True,
-                             initial_state=h0)
+                             initial_state=h0, zoh=zoh)
 
     def scan_backward(self, u, delta, A, Bm, Cm, dout, ws, z, Dskip, delta_bias, softplus, seq,
-                      h0, dfinal):
+                      h0, dfinal, zoh):
         return self.scan_bwd(u, delta, A, Bm, Cm, dout, ws, z=z, Dskip=Dskip,
                              delta_bias=delta_bias, softplus=softplus, seq_idx=seq,
-                             initial_state=h0, dfinal_state=dfinal)
+                             initial_state=h0, dfinal_state=dfinal, zoh=zoh)
 
 
 class ContextParallelLayer:
     """conv1d + SiLU -> selective scan (softplus step, D skip, SiLU(z) gate),
     forward and backward, over this rank's shard of the sequence.
 
-    Parameters (A [D, N], Dskip, delta_bias [D], conv_w [D, 4], conv_b [D])
-    are replicated; activations are this rank's shard ([B, D, Ls]; B, C
-    [B, N, Ls]; seq_idx [B, Ls] int32 or None), Ls >= 3.
+    Parameters (A [D, N] real, Dskip, delta_bias [D], conv_w [D, 4], conv_b
+    [D]) are replicated; activations are this rank's shard ([B, D, Ls]; B, C
+    [B, N, Ls]; seq_idx [B, Ls] int32 or None), Ls >= 3. `zoh` selects the
+    zero-order-hold discretisation (the summaries are the same: the carry
+    passes through prod a either way).
     """
 
-    def __init__(self, comm, ops=None, softplus=True):
+    def __init__(self, comm, ops=None, softplus=True, zoh=False):
         self.comm = comm
         self.ops = ops if ops is not None else GpuOps()
         self.softplus = softplus
+        self.zoh = zoh
 
     def forward(self, x, delta, z, Bm, Cm, A, Dskip, delta_bias, conv_w, conv_b, seq_idx=None,
                 initial_state=None):
@@ -148,12 +151,12 @@ class ContextParallelLayer:
         seq_prev = seq_prev3[:, -1].contiguous() if seq_prev3 is not None else None
         u = ops.conv_fwd(x, conv_w, conv_b, seq_idx, x_prev, seq_prev3)
         decay, end = ops.scan_fwd_summary(u, delta, A, Bm, seq_idx, seq_prev, delta_bias,
-                                          self.softplus)
+                                          self.softplus, self.zoh)
         summ = c.all_gather(_stack2(decay, end))
         decay_all, end_all = summ[:, 0].contiguous(), summ[:, 1].contiguous()
         h_in = ops.state_carry(decay_all, end_all, c.rank, False, initial_state, seq_prev, seq_idx)
         out, fs, ws = ops.scan_forward(u, delta, A, Bm, Cm, z, Dskip, delta_bias, self.softplus,
-                                       seq_idx, h_in)
+                                       seq_idx, h_in, self.zoh)
         ctx = dict(x=x, delta=delta, z=z, Bm=Bm, Cm=Cm, A=A, Dskip=Dskip, delta_bias=delta_bias,
                    conv_w=conv_w, conv_b=conv_b, seq_idx=seq_idx, u=u, ws=ws, h_in=h_in,
                    x_prev=x_prev, seq_prev3=seq_prev3, seq_prev=seq_prev, decay_all=decay_all)
@@ -172,7 +175,8 @@ class ContextParallelLayer:
         adj_all = c.all_gather(adj)
         dfin = ops.state_carry(k["decay_all"], adj_all, c.rank, True, dfinal_state, None, None)
         g = ops.scan_backward(k["u"], k["delta"], k["A"], k["Bm"], k["Cm"], dout, k["ws"], k["z"],
-                              k["Dskip"], k["delta_bias"], self.softplus, seq, k["h_in"], dfin)
+                              k["Dskip"], k["delta_bias"], self.softplus, seq, k["h_in"], dfin,
+                              self.zoh)
         x_next = c.shift(k["x"][..., :HALO], -1)
         du_next = c.shift(g["du"][..., :HALO], -1)
         seq_next = c.shift(seq[..., :HALO], -1) if seq is not None else None

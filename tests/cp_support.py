@@ -68,10 +68,10 @@ class OracleOps:
             return None
         return _np(seq_prev, np.int64) != _np(seq, np.int64)[:, 0]
 
-    def scan_fwd_summary(self, u, delta, A, Bm, seq, seq_prev, delta_bias, softplus):
+    def scan_fwd_summary(self, u, delta, A, Bm, seq, seq_prev, delta_bias, softplus, zoh=False):
         un, dn, An, Bn = _np(u), _np(delta), _np(A), _np(Bm)
         sq = _np(seq, np.int32)
-        kw = dict(delta_bias=_np(delta_bias), softplus=softplus, seq_idx=sq)
+        kw = dict(delta_bias=_np(delta_bias), softplus=softplus, seq_idx=sq, zoh=zoh)
         f0 = oracle.scan_fwd(un, dn, An, Bn, Bn, **kw)["final_state"]
         f1 = oracle.scan_fwd(un, dn, An, Bn, Bn, h0=np.ones_like(f0), **kw)["final_state"]
         decay = f1 - f0
@@ -107,17 +107,18 @@ class OracleOps:
                 h[cut] = 0.0
         return _t(h)
 
-    def scan_forward(self, u, delta, A, Bm, Cm, z, Dskip, delta_bias, softplus, seq, h0):
+    def scan_forward(self, u, delta, A, Bm, Cm, z, Dskip, delta_bias, softplus, seq, h0,
+                     zoh=False):
         f = oracle.scan_fwd(_np(u), _np(delta), _np(A), _np(Bm), _np(Cm), z=_np(z),
                             Dskip=_np(Dskip), delta_bias=_np(delta_bias), softplus=softplus,
-                            seq_idx=_np(seq, np.int32), h0=_np(h0))
+                            seq_idx=_np(seq, np.int32), h0=_np(h0), zoh=zoh)
         return _t(f["out"]), _t(f["final_state"]), None
 
     def scan_backward(self, u, delta, A, Bm, Cm, dout, ws, z, Dskip, delta_bias, softplus, seq,
-                      h0, dfinal):
+                      h0, dfinal, zoh=False):
         g = oracle.scan_bwd(_np(u), _np(delta), _np(A), _np(Bm), _np(Cm), _np(dout), z=_np(z),
                             Dskip=_np(Dskip), delta_bias=_np(delta_bias), softplus=softplus,
-                            seq_idx=_np(seq, np.int32), h0=_np(h0), dhL=_np(dfinal))
+                            seq_idx=_np(seq, np.int32), h0=_np(h0), dhL=_np(dfinal), zoh=zoh)
         names = {"du": "du", "ddelta": "ddelta", "dz": "dz", "dA": "dA", "dB": "dB", "dC": "dC",
                  "dD": "dD", "ddelta_bias": "ddelta_bias", "dinitial_state": "dh0"}
         return {k: _t(g[v]) for k, v in names.items()}
@@ -207,7 +208,7 @@ def full_problem(B, D, N, L, seed, seq_bounds=None):
     return p
 
 
-def full_reference(p, bf16_points=False):
+def full_reference(p, bf16_points=False, zoh=False):
     """Unsharded oracle: conv -> scan (from h0) -> scan backward (with dhL)
     -> conv backward. With `bf16_points`, u and du are rounded to bf16 where
     bf16 storage rounds them between the stages."""
@@ -215,7 +216,8 @@ def full_reference(p, bf16_points=False):
     _, u = oracle.conv1d_fwd(p["x"], p["conv_w"], p["conv_b"], seq)
     if bf16_points:
         u = oracle.round_bf16(u)
-    kw = dict(z=p["z"], Dskip=p["Dskip"], delta_bias=p["delta_bias"], seq_idx=seq, h0=p["h0"])
+    kw = dict(z=p["z"], Dskip=p["Dskip"], delta_bias=p["delta_bias"], seq_idx=seq, h0=p["h0"],
+              zoh=zoh)
     f = oracle.scan_fwd(u, p["delta"], p["A"], p["Bm"], p["Cm"], **kw)
     g = oracle.scan_bwd(u, p["delta"], p["A"], p["Bm"], p["Cm"], p["dout"], dhL=p["dhL"], **kw)
     du = oracle.round_bf16(g["du"]) if bf16_points else g["du"]

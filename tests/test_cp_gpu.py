@@ -181,12 +181,12 @@ def test_conv_halos_match_oracle(L, vec):
     assert rel_l2(host64(db), wdb.numpy()) <= TOL_F32
 
 
-def _gpu_rank(p, R, r, comm, act_dtype):
+def _gpu_rank(p, R, r, comm, act_dtype, zoh=False):
     import torch
     from selective_state_space_35_b200.cp import ContextParallelLayer
     s, lo, hi = shard(p, R, r)
     d = _devs(s, act_dtype)
-    layer = ContextParallelLayer(comm)
+    layer = ContextParallelLayer(comm, zoh=zoh)
     out, fs, ctx = layer.forward(d["x"], d["delta"], d["z"], d["Bm"], d["Cm"], d["A"], d["Dskip"],
                                  d["delta_bias"], d["conv_w"], d["conv_b"], seq_idx=d["seq_idx"],
                                  initial_state=d["h0"])
@@ -228,3 +228,17 @@ def test_cp_gpu_equal_unsharded(R, L, bounds, dtype):
             assert e <= (TOL_F32 if fp32 else TOL_GRAD), (r, k, e)
     assert rel_l2(results[-1][0]["final_state"], want["final_state"]) <= (TOL_F32 if fp32 else TOL_GRAD)
     assert rel_l2(results[0][0]["dinitial_state"], want["dinitial_state"]) <= (TOL_F32 if fp32 else TOL_GRAD)
+
+
+def test_cp_gpu_zero_order_hold():
+    raw = full_problem(2, 16, 16, 900, seed=990, seq_bounds=(450, 300))
+    p = _f32(raw)
+    import torch
+    results = run_threads(3, lambda r, comm: _gpu_rank(p, 3, r, comm, torch.float32, zoh=True))
+    want = full_reference(p, zoh=True)
+    for r, (res, lo, hi) in enumerate(results):
+        for k in SHARDED + SHARDED_BC:
+            assert rel_l2(res[k], want[k][..., lo:hi]) <= TOL_F32, (r, k)
+        for k in REDUCED:
+            assert rel_l2(res[k], want[k]) <= TOL_F32, (r, k)
+    assert rel_l2(results[0][0]["dinitial_state"], want["dinitial_state"]) <= TOL_F32

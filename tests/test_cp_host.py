@@ -21,12 +21,12 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank_run(p, R, r, comm):
+def _rank_run(p, R, r, comm, zoh=False):
     import torch
     from selective_state_space_35_b200.cp import ContextParallelLayer
     s, lo, hi = shard(p, R, r)
     T = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a))  # noqa: E731
-    layer = ContextParallelLayer(comm, ops=OracleOps())
+    layer = ContextParallelLayer(comm, ops=OracleOps(), zoh=zoh)
     out, fs, ctx = layer.forward(T(s["x"]), T(s["delta"]), T(s["z"]), T(s["Bm"]), T(s["Cm"]),
                                  T(s["A"]), T(s["Dskip"]), T(s["delta_bias"]), T(s["conv_w"]),
                                  T(s["conv_b"]), seq_idx=T(s["seq_idx"]), initial_state=T(s["h0"]))
@@ -37,8 +37,8 @@ def _rank_run(p, R, r, comm):
     return res, lo, hi
 
 
-def _check(p, R, results, tol=1e-10):
-    want = full_reference(p)
+def _check(p, R, results, tol=1e-10, zoh=False):
+    want = full_reference(p, zoh=zoh)
     for r, (res, lo, hi) in enumerate(results):
         for k in SHARDED + SHARDED_BC:
             np.testing.assert_allclose(res[k], want[k][..., lo:hi], rtol=tol, atol=tol,
@@ -64,6 +64,12 @@ def test_cp_threads_equal_unsharded(R, L, bounds):
     p = full_problem(2, 3, 4, L, seed=500 + R + L, seq_bounds=bounds)
     results = run_threads(R, lambda r, comm: _rank_run(p, R, r, comm))
     _check(p, R, results)
+
+
+def test_cp_threads_zero_order_hold():
+    p = full_problem(2, 3, 4, 50, seed=560, seq_bounds=(25, 17))
+    results = run_threads(2, lambda r, comm: _rank_run(p, 2, r, comm, zoh=True))
+    _check(p, 2, results, zoh=True)
 
 
 def _gloo_worker(rank, world, port, L, bounds, q):

@@ -469,7 +469,7 @@ def complex_bench(device, ly, pk, reps=5):
         ssm.scan_bwd(ly.x, ly.delta, A, Bc, Cc, ly.dout, ws, grads=g, **kw)
         e[2].record()
     torch.cuda.synchronize()
-    fwd = sum(e[0].elapsed_time(e[1]) for e in ev[1:]) / reps   # round 0 is a warm-up
+    fwd = sum(e[0].elapsed_time(e[1]) for e in ev[1:]) / reps   # the first pass warms up
     bwd = sum(e[1].elapsed_time(e[2]) for e in ev[1:]) / reps
     del ws, g, out
     return {"workload": f"complex diagonal A (S4D-Lin), B{B} x D{D} x N{N} x L{L}, bf16 "

@@ -199,6 +199,8 @@ def _gpu_rank(p, R, r, comm, act_dtype, zoh=False):
 
 
 @pytest.mark.parametrize("R,L,bounds,dtype", [
+    (1, 300, (100,), "f32"),
+    (3, 9, (3, 5), "f32"),
     (2, 1024, (512, 700), "f32"),
     (3, 771, (257, 516, 100), "f32"),
     (4, 1200, (300, 602, 1000), "f32"),

@@ -56,7 +56,10 @@ def _check(p, R, results, tol=1e-10, zoh=False):
 # boundaries: one at a shard start (L=60, R=3 -> 20, 40), one two tokens
 # after a shard start (inside the conv halo), one mid-shard
 _CASES = [(2, 60, (20, 42, 7)), (3, 60, (20, 42, 7)), (4, 61, (15, 30, 47)), (2, 40, None),
-          (3, 45, ())]
+          (3, 45, ()),
+          (1, 30, (11,)),          # one rank: every exchange is empty
+          (3, 9, (3, 5)),          # shards of 3 tokens, the conv halo's length
+          (4, 13, (3, 4, 9))]      # ragged shards of 3 and 4 tokens
 
 
 @pytest.mark.parametrize("R,L,bounds", _CASES)
@@ -106,3 +109,9 @@ def test_cp_gloo_processes_equal_unsharded(world, L, bounds):
         assert pr.exitcode == 0
     p = full_problem(2, 3, 4, L, seed=700 + world + L, seq_bounds=bounds)
     _check(p, world, [got[r] for r in range(world)])
+
+
+def test_cp_rejects_shards_shorter_than_the_halo():
+    p = full_problem(1, 2, 4, 5, seed=570)
+    with pytest.raises(ValueError, match="halo"):
+        run_threads(2, lambda r, comm: _rank_run(p, 2, r, comm))

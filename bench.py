@@ -297,6 +297,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-decode", action="store_true", help="skip the recurrent-step measurement")
     ap.add_argument("--no-complex", action="store_true", help="skip the complex-A scan measurement")
+    ap.add_argument("--no-cp", action="store_true",
+                    help="skip the per-rank measurement of the context-parallel kernels")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -426,6 +428,8 @@ def main():
         line["decode"] = decode_bench(device, sh, pk)
     if not args.no_complex:
         line["complex_a"] = complex_bench(device, layers[0], pk)
+    if not args.no_cp:
+        line["cp_shard"] = cp_shard_bench(device, layers[0], ranks=8)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = cpu_count()
@@ -476,6 +480,60 @@ def complex_bench(device, ly, pk, reps=5):
                         "activations, fp32 complex state, fwd + bwd",
             "fwd_ms": fwd, "bwd_ms": bwd, "tokens_per_s": B * L / ((fwd + bwd) * 1e-3),
             "launches": 3 * (reps + 2)}
+
+
+def cp_shard_bench(device, ly, ranks=8, reps=5):
+    """One rank's compute when the bench layer's sequence is cut into `ranks`
+    contiguous shards: the forward and backward summaries of its shard, the
+    carry folds over all ranks' summaries, and the shard's scan forward and
+    backward. It is timed on one GPU with CUDA events. The exchanges (a
+    3-token halo each way, 2 x [B, D, N] fp32 summaries per rank and
+    direction) are not part of it."""
+    import torch
+    import selective_state_space_35_b200 as ssm
+    B, D, N, L = ly.shape.B, ly.shape.D, ly.shape.N, ly.shape.L
+    Ls = L // ranks
+    sl = lambda t: t[..., :Ls].contiguous()  # noqa: E731
+    u, dl, z, go, Bm, Cm = (sl(t) for t in (ly.x, ly.delta, ly.z, ly.dout, ly.Bm, ly.Cm))
+    kw = dict(z=z, Dskip=ly.Dskip, delta_bias=ly.dbias)
+    h0 = torch.zeros((B, D, N), dtype=torch.float32, device=device)
+    out, _, ws = ssm.scan_fwd(u, dl, ly.A, Bm, Cm, initial_state=h0, **kw)
+    g = ssm.scan_bwd(u, dl, ly.A, Bm, Cm, go, ws, initial_state=h0, dfinal_state=h0, **kw)
+    sws = torch.empty_like(ws)
+    dec, end = ssm.scan_fwd_summary(u, dl, ly.A, Bm, delta_bias=ly.dbias, workspace=sws)
+    stack = torch.stack([dec] * ranks).contiguous()
+    vals = torch.stack([end] * ranks).contiguous()
+    hin = torch.empty_like(h0)
+
+    steps = {
+        "fwd_summary": lambda: ssm.scan_fwd_summary(u, dl, ly.A, Bm, delta_bias=ly.dbias,
+                                                    workspace=sws),
+        "bwd_summary": lambda: ssm.scan_bwd_summary(dl, ly.A, Cm, go, z=z, delta_bias=ly.dbias,
+                                                    workspace=sws),
+        "carry_fwd": lambda: ssm.state_carry(stack, vals, ranks - 1, out=hin),
+        "carry_bwd": lambda: ssm.state_carry(stack, vals, 0, reverse=True, out=hin),
+        "scan_fwd": lambda: ssm.scan_fwd(u, dl, ly.A, Bm, Cm, out=out, workspace=ws,
+                                         initial_state=hin, **kw),
+        "scan_bwd": lambda: ssm.scan_bwd(u, dl, ly.A, Bm, Cm, go, ws, grads=g,
+                                         initial_state=hin, dfinal_state=hin, **kw),
+    }
+    ms = {}
+    for name, fn in steps.items():
+        fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms[name] = e0.elapsed_time(e1) / reps
+    rank_ms = sum(ms.values())
+    del ws, sws, g, out
+    return {"workload": f"one rank of {ranks}: B{B} x D{D} x N{N} x L{Ls} shard of the L{L} row, "
+                        "bf16 activations, no L2 flush between repeats",
+            "ms": ms, "rank_scan_ms": rank_ms,
+            "overhead_vs_plain_shard": rank_ms / (ms["scan_fwd"] + ms["scan_bwd"]) - 1.0,
+            "launches": 9 * (reps + 1) + 5}
 
 
 def decode_bench(device, sh, pk, rows_b=2048, steps=200, graph_steps=50):

@@ -38,10 +38,12 @@ def lib():
         L.oracle_decode_step.argtypes = [dp] * 11 + [i] + [dp] * 3 + [i, i, i, i]
         L.oracle_cscan_fwd.argtypes = [dp] * 8 + [i, ip, dp, dp, dp, dp, i, i, i, i]
         L.oracle_cscan_bwd.argtypes = [dp] * 8 + [i, ip] + [dp] * 12 + [i, i, i, i]
+        L.oracle_ssd_fwd.argtypes = [dp] * 7 + [i, ip, dp, dp] + [i] * 6
+        L.oracle_ssd_bwd.argtypes = [dp] * 7 + [i, ip] + [dp] * 8 + [i] * 6
         for f in ("oracle_round_bf16", "oracle_conv1d_fwd", "oracle_conv1d_bwd",
                   "oracle_scan_fwd", "oracle_scan_bwd", "oracle_scan_fwd_mt",
                   "oracle_scan_bwd_mt", "oracle_decode_step", "oracle_cscan_fwd",
-                  "oracle_cscan_bwd"):
+                  "oracle_cscan_bwd", "oracle_ssd_fwd", "oracle_ssd_bwd"):
             getattr(L, f).restype = None
         _lib = L
     return _lib
@@ -241,6 +243,42 @@ def cscan_bwd(u, delta, A, Bm, Cm, dout, *, z=None, Dskip=None, delta_bias=None,
     return {"du": du, "ddelta": ddelta, "dz": dz, "dA": dA[..., 0] + 1j * dA[..., 1],
             "dB": dB[:, :, 0] + 1j * dB[:, :, 1], "dC": dC[:, :, 0] + 1j * dC[:, :, 1],
             "dD": dD, "ddelta_bias": ddb, "dh0": dh0[..., 0] + 1j * dh0[..., 1]}
+
+
+def ssd_fwd(x, dt_raw, A, Bm, Cm, *, D=None, dt_bias=None, softplus=True, seq_idx=None):
+    """Mamba-2 SSD forward. x [B, L, H, P]; dt_raw [B, L, H]; A, D, dt_bias
+    [H]; Bm, Cm [B, L, G, N] (head h uses group h // (H // G)); seq_idx
+    [B, L]. Returns dict(y [B, L, H, P], final_state [B, H, P, N])."""
+    x, dt_raw, A, Bm, Cm = _f64(x), _f64(dt_raw), _f64(A), _f64(Bm), _f64(Cm)
+    D, dt_bias, seq = _f64(D), _f64(dt_bias), _i32(seq_idx)
+    B, L, H, P = x.shape
+    G, N = Bm.shape[2], Bm.shape[3]
+    assert H % G == 0
+    y = np.empty_like(x)
+    fs = np.empty((B, H, P, N))
+    lib().oracle_ssd_fwd(_d(x), _d(dt_raw), _d(A), _d(Bm), _d(Cm), _d(D), _d(dt_bias),
+                         int(softplus), _i(seq), _d(y), _d(fs), B, L, H, P, G, N)
+    return {"y": y, "final_state": fs}
+
+
+def ssd_bwd(x, dt_raw, A, Bm, Cm, dy, *, D=None, dt_bias=None, softplus=True, seq_idx=None):
+    """Backward of ssd_fwd: dict(dx, ddt_raw, dA, dB, dC, dD, ddt_bias)."""
+    x, dt_raw, A, Bm, Cm, dy = _f64(x), _f64(dt_raw), _f64(A), _f64(Bm), _f64(Cm), _f64(dy)
+    D, dt_bias, seq = _f64(D), _f64(dt_bias), _i32(seq_idx)
+    B, L, H, P = x.shape
+    G, N = Bm.shape[2], Bm.shape[3]
+    assert H % G == 0
+    dx = np.empty_like(x)
+    ddt = np.empty_like(dt_raw)
+    dA = np.empty(H)
+    dB = np.empty_like(Bm)
+    dC = np.empty_like(Cm)
+    dD = np.empty(H)
+    ddb = np.empty(H)
+    lib().oracle_ssd_bwd(_d(x), _d(dt_raw), _d(A), _d(Bm), _d(Cm), _d(D), _d(dt_bias),
+                         int(softplus), _i(seq), _d(dy), _d(dx), _d(ddt), _d(dA), _d(dB), _d(dC),
+                         _d(dD), _d(ddb), B, L, H, P, G, N)
+    return {"dx": dx, "ddt_raw": ddt, "dA": dA, "dB": dB, "dC": dC, "dD": dD, "ddt_bias": ddb}
 
 
 def _cplx_pairs(a):

@@ -18,6 +18,9 @@
  *          y * silu(z).
  *   resets "FLA Mamba and Mamba2" (Axolotl), packing paragraph: convolution
  *          and recurrent state start independently for every document.
+ *   complex A  "S4: Structured State Spaces for Sequences" (S4D), see below.
+ *   SSD    "Mamba-2: Structured State Space Duality (SSD)": scalar A per
+ *          head, heads, groups of shared B / C (see below).
  *
  * Readings taken where the pages are silent:
  *   - A is passed directly (negative for the S4D-real init), not A_log.exp().
@@ -635,4 +638,129 @@ void oracle_cscan_bwd(const double* u, const double* delta, const double* z, con
             }
         }
     free(hs); free(as); free(ys); free(os); free(carry);
+}
+
+/* ------------------------------------------------------ Mamba-2 SSD form */
+/* "hung-phan ml-skills mamba", section "Mamba-2: Structured State Space
+ * Duality (SSD)": A restricted to a scalar times the identity, per head;
+ * multi-head (d split into H heads of width P); B and C shared by the heads
+ * of a group (G groups, head h in group h / (H / G)). Per (batch, head), with
+ * a_t = exp(dt_t A_h) and a state h of P x N:
+ *   h_t[p][n] = a_t h_{t-1}[p][n] + dt_t x_t[p] B_t[n]
+ *   y_t[p]    = sum_n C_t[n] h_t[p][n] + D_h x_t[p]
+ * dt_t = softplus(dt_raw_t + dt_bias_h) (or without softplus); a document
+ * start (seq_idx change) zeroes a_t as in the Mamba-1 scan. Layouts
+ * (token-major): x, y, dx [B][L][H][P]; dt [B][L][H]; A, D, dt_bias [H];
+ * Bm, Cm [B][L][G][N]; final state [B][H][P][N]. */
+typedef struct {
+    const double *x, *dt_raw, *A, *Bm, *Cm, *Dh, *dt_bias;
+    const int32_t* seq;
+    int B, L, H, P, G, N, softplus_on;
+} ssd_in_t;
+
+static double ssd_dt(const ssd_in_t* p, int b, int t, int h) {
+    double v = p->dt_raw[((size_t)b * p->L + t) * p->H + h] + (p->dt_bias ? p->dt_bias[h] : 0.0);
+    return p->softplus_on ? softplus(v) : v;
+}
+
+/* One (batch, head): runs the recurrence, keeping every state when hs is
+ * non-NULL ([L][P][N]). */
+static void ssd_fwd_head(const ssd_in_t* p, int b, int h, double* y, double* final_state,
+                         double* hs) {
+    const int L = p->L, H = p->H, P = p->P, G = p->G, N = p->N;
+    const int g = h / (H / G);
+    double* st = (double*)calloc((size_t)P * N, sizeof(double));
+    for (int t = 0; t < L; ++t) {
+        const double dt = ssd_dt(p, b, t, h);
+        const int reset = (t > 0) && seg_of(p->seq, L, b, t) != seg_of(p->seq, L, b, t - 1);
+        const double a = reset ? 0.0 : exp(dt * p->A[h]);
+        const double* xt = p->x + (((size_t)b * L + t) * H + h) * P;
+        const double* Bt = p->Bm + (((size_t)b * L + t) * G + g) * N;
+        const double* Ct = p->Cm + (((size_t)b * L + t) * G + g) * N;
+        for (int q = 0; q < P; ++q) {
+            double acc = 0.0;
+            for (int n = 0; n < N; ++n) {
+                double* s = st + (size_t)q * N + n;
+                *s = a * *s + dt * xt[q] * Bt[n];
+                acc += Ct[n] * *s;
+            }
+            if (y) y[(((size_t)b * L + t) * H + h) * P + q] = acc + (p->Dh ? p->Dh[h] * xt[q] : 0.0);
+        }
+        if (hs) memcpy(hs + (size_t)t * P * N, st, sizeof(double) * (size_t)P * N);
+    }
+    if (final_state)
+        memcpy(final_state + ((size_t)b * H + h) * P * N, st, sizeof(double) * (size_t)P * N);
+    free(st);
+}
+
+void oracle_ssd_fwd(const double* x, const double* dt_raw, const double* A, const double* Bm,
+                    const double* Cm, const double* Dh, const double* dt_bias, int softplus_on,
+                    const int32_t* seq, double* y, double* final_state, int B, int L, int H, int P,
+                    int G, int N) {
+    ssd_in_t p = {x, dt_raw, A, Bm, Cm, Dh, dt_bias, seq, B, L, H, P, G, N, softplus_on};
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) ssd_fwd_head(&p, b, h, y, final_state, NULL);
+}
+
+/* Reverse mode, per (batch, head), with the adjoint of the state
+ *   Gs_t[p][n] = dy_t[p] C_t[n] + a_{t+1} Gs_{t+1}[p][n]   (a_{t+1} = 0 at a start)
+ * dx_t[p]   = D_h dy_t[p] + dt_t sum_n Gs_t[p][n] B_t[n]
+ * d dt_t    = sum_{p,n} Gs_t[p][n] (x_t[p] B_t[n] + a_t A_h h_{t-1}[p][n])
+ * dA_h     += sum_t dt_t sum_{p,n} Gs_t[p][n] a_t h_{t-1}[p][n]
+ * dB_t[n]  += dt_t sum_p Gs_t[p][n] x_t[p]      (summed over the group's heads)
+ * dC_t[n]  += sum_p dy_t[p] h_t[p][n]           (same)
+ * dD_h     += sum_t sum_p dy_t[p] x_t[p]; d dt_raw = d dt * sigmoid(v) with softplus. */
+void oracle_ssd_bwd(const double* x, const double* dt_raw, const double* A, const double* Bm,
+                    const double* Cm, const double* Dh, const double* dt_bias, int softplus_on,
+                    const int32_t* seq, const double* dy, double* dx, double* ddt_raw, double* dA,
+                    double* dB, double* dC, double* dD, double* ddt_bias, int B, int L, int H,
+                    int P, int G, int N) {
+    ssd_in_t p = {x, dt_raw, A, Bm, Cm, Dh, dt_bias, seq, B, L, H, P, G, N, softplus_on};
+    memset(dA, 0, sizeof(double) * (size_t)H);
+    memset(dB, 0, sizeof(double) * (size_t)B * L * G * N);
+    memset(dC, 0, sizeof(double) * (size_t)B * L * G * N);
+    if (dD) memset(dD, 0, sizeof(double) * (size_t)H);
+    if (ddt_bias) memset(ddt_bias, 0, sizeof(double) * (size_t)H);
+    double* hs = (double*)malloc(sizeof(double) * (size_t)L * P * N);
+    double* gs = (double*)calloc((size_t)P * N, sizeof(double));   /* a_{t+1} Gs_{t+1} */
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            const int g = h / (H / G);
+            ssd_fwd_head(&p, b, h, NULL, NULL, hs);
+            memset(gs, 0, sizeof(double) * (size_t)P * N);
+            for (int t = L - 1; t >= 0; --t) {
+                const double dt = ssd_dt(&p, b, t, h);
+                const int reset = (t > 0) && seg_of(seq, L, b, t) != seg_of(seq, L, b, t - 1);
+                const double a = reset ? 0.0 : exp(dt * A[h]);
+                const size_t xo = (((size_t)b * L + t) * H + h) * P;
+                const size_t bo = (((size_t)b * L + t) * G + g) * N;
+                double ddt = 0.0, dAh = 0.0;
+                for (int q = 0; q < P; ++q) {
+                    double sgb = 0.0;
+                    const double dyq = dy[xo + q], xq = x[xo + q];
+                    for (int n = 0; n < N; ++n) {
+                        const double G_ = dyq * Cm[bo + n] + gs[(size_t)q * N + n];
+                        const double hprev = t > 0 ? hs[(size_t)(t - 1) * P * N + (size_t)q * N + n] : 0.0;
+                        sgb += G_ * Bm[bo + n];
+                        ddt += G_ * (xq * Bm[bo + n] + a * A[h] * hprev);
+                        dAh += G_ * a * dt * hprev;
+                        dB[bo + n] += G_ * dt * xq;
+                        dC[bo + n] += dyq * hs[(size_t)t * P * N + (size_t)q * N + n];
+                        gs[(size_t)q * N + n] = a * G_;
+                    }
+                    dx[xo + q] = (Dh ? Dh[h] * dyq : 0.0) + dt * sgb;
+                    if (dD) dD[h] += dyq * xq;
+                }
+                dA[h] += dAh;
+                double dv = ddt;
+                if (softplus_on) {
+                    const double v = dt_raw[((size_t)b * L + t) * H + h] + (dt_bias ? dt_bias[h] : 0.0);
+                    dv = ddt * sigm(v);
+                }
+                ddt_raw[((size_t)b * L + t) * H + h] = dv;
+                if (ddt_bias) ddt_bias[h] += dv;
+            }
+        }
+    free(hs);
+    free(gs);
 }

@@ -68,4 +68,17 @@ void oracle_cscan_bwd(const double* u, const double* delta, const double* z, con
                       const double* dout, double* du, double* ddelta, double* dz, double* dA,
                       double* dB, double* dC, double* dD, double* ddelta_bias, double* dh0,
                       const double* dhL, int B, int D, int L, int N);
+/* Mamba-2 SSD (scalar A per head, heads of width P, G groups of shared
+ * B / C): x, y, dx [B][L][H][P]; dt_raw, ddt_raw [B][L][H]; A, Dh, dt_bias,
+ * dA, dD, ddt_bias [H]; Bm, Cm, dB, dC [B][L][G][N]; final state
+ * [B][H][P][N]. */
+void oracle_ssd_fwd(const double* x, const double* dt_raw, const double* A, const double* Bm,
+                    const double* Cm, const double* Dh, const double* dt_bias, int softplus_on,
+                    const int32_t* seq, double* y, double* final_state, int B, int L, int H, int P,
+                    int G, int N);
+void oracle_ssd_bwd(const double* x, const double* dt_raw, const double* A, const double* Bm,
+                    const double* Cm, const double* Dh, const double* dt_bias, int softplus_on,
+                    const int32_t* seq, const double* dy, double* dx, double* ddt_raw, double* dA,
+                    double* dB, double* dC, double* dD, double* ddt_bias, int B, int L, int H,
+                    int P, int G, int N);
 #endif

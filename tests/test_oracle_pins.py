@@ -806,3 +806,101 @@ def test_cscan_bwd_final_state_gradient_fd():
     for name, gname in [("A", "dA"), ("Bm", "dB"), ("Cm", "dC"), ("h0", "dh0")]:
         _close(_fd(loss, parts[name + ".re"]), g[gname].real)
         _close(_fd(loss, parts[name + ".im"]), g[gname].imag)
+
+
+# --------------------------------------------------------------------------
+# Mamba-2 SSD form (scalar A per head, heads, groups of shared B / C)
+# --------------------------------------------------------------------------
+def _ssd_problem(rng, B=2, L=14, H=4, P=3, G=2, N=5):
+    return dict(x=rng.standard_normal((B, L, H, P)), dt_raw=0.5 * rng.standard_normal((B, L, H)),
+                A=-rng.uniform(0.3, 2.0, size=H), Bm=rng.standard_normal((B, L, G, N)),
+                Cm=rng.standard_normal((B, L, G, N)), D=rng.uniform(0.5, 1.5, size=H),
+                dt_bias=rng.uniform(-2.0, -0.5, size=H))
+
+
+def test_ssd_equals_its_attention_form():
+    """The duality the SSD section states: per head, Y = (M o C B^T)(dt x) +
+    D x with M[i][j] = exp(A sum_{j<k<=i} dt_k) for j <= i in the same
+    document, 0 otherwise (numpy matrices, no recurrence)."""
+    rng = _rng(95)
+    p = _ssd_problem(rng)
+    B, L, H, P = p["x"].shape
+    G = p["Bm"].shape[2]
+    seq = np.array([[0] * 6 + [1] * 8, [0] * 14], dtype=np.int32)
+    y = oracle.ssd_fwd(p["x"], p["dt_raw"], p["A"], p["Bm"], p["Cm"], D=p["D"],
+                       dt_bias=p["dt_bias"], seq_idx=seq)["y"]
+    dt = np.log1p(np.exp(p["dt_raw"] + p["dt_bias"][None, None, :]))
+    want = np.empty_like(y)
+    for b in range(B):
+        for h in range(H):
+            g = h // (H // G)
+            cs = np.cumsum(dt[b, :, h] * p["A"][h])
+            M = np.exp(cs[:, None] - cs[None, :])
+            M *= np.tril(np.ones((L, L)))
+            M *= seq[b][:, None] == seq[b][None, :]
+            CB = p["Cm"][b, :, g, :] @ p["Bm"][b, :, g, :].T
+            want[b, :, h, :] = (M * CB) @ (dt[b, :, h, None] * p["x"][b, :, h, :]) \
+                + p["D"][h] * p["x"][b, :, h, :]
+    np.testing.assert_allclose(y, want, rtol=1e-11, atol=1e-11)
+
+
+def test_ssd_one_group_equals_the_mamba1_scan():
+    """With one group, SSD is the Mamba-1 scan over H*P channels whose A is
+    the head's scalar for every state, whose step is the head's and whose B
+    and C are shared by all channels: both oracles (written separately) agree,
+    forward and every gradient."""
+    rng = _rng(96)
+    p = _ssd_problem(rng, G=1)
+    B, L, H, P = p["x"].shape
+    N = p["Bm"].shape[3]
+    seq = np.array([[0] * 5 + [1] * 9, [0] * 3 + [1] * 11], dtype=np.int32)
+    dy = rng.standard_normal(p["x"].shape)
+    kw = dict(D=p["D"], dt_bias=p["dt_bias"], seq_idx=seq)
+    f = oracle.ssd_fwd(p["x"], p["dt_raw"], p["A"], p["Bm"], p["Cm"], **kw)
+    g = oracle.ssd_bwd(p["x"], p["dt_raw"], p["A"], p["Bm"], p["Cm"], dy, **kw)
+    # channel d = h P + q; activations [B, D, L]
+    u = p["x"].reshape(B, L, H * P).transpose(0, 2, 1)
+    delta = np.repeat(p["dt_raw"], P, axis=2).transpose(0, 2, 1)
+    A1 = np.repeat(p["A"], P)[:, None] * np.ones((1, N))
+    Bm1 = p["Bm"][:, :, 0, :].transpose(0, 2, 1)
+    Cm1 = p["Cm"][:, :, 0, :].transpose(0, 2, 1)
+    kw1 = dict(Dskip=np.repeat(p["D"], P), delta_bias=np.repeat(p["dt_bias"], P), seq_idx=seq)
+    r = oracle.scan_fwd(u, delta, A1, Bm1, Cm1, **kw1)
+    gr = oracle.scan_bwd(u, delta, A1, Bm1, Cm1, dy.reshape(B, L, H * P).transpose(0, 2, 1), **kw1)
+    np.testing.assert_allclose(f["y"].reshape(B, L, H * P).transpose(0, 2, 1), r["out"],
+                               rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(f["final_state"].reshape(B, H * P, N), r["final_state"],
+                               rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g["dx"].reshape(B, L, H * P).transpose(0, 2, 1), gr["du"],
+                               rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(g["ddt_raw"], gr["ddelta"].reshape(B, H, P, L).sum(2).transpose(0, 2, 1),
+                               rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(g["dA"], gr["dA"].reshape(H, P, N).sum((1, 2)), rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(g["dB"][:, :, 0, :], gr["dB"].transpose(0, 2, 1), rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(g["dC"][:, :, 0, :], gr["dC"].transpose(0, 2, 1), rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(g["dD"], gr["dD"].reshape(H, P).sum(1), rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(g["ddt_bias"], gr["ddelta_bias"].reshape(H, P).sum(1), rtol=1e-11,
+                               atol=1e-11)
+
+
+@pytest.mark.parametrize("softplus", [True, False])
+def test_ssd_bwd_finite_differences(softplus):
+    """Every SSD gradient against central differences, two groups, a reset."""
+    rng = _rng(97)
+    p = _ssd_problem(rng, L=10)
+    if not softplus:
+        p["dt_raw"] = np.abs(p["dt_raw"]) * 0.3
+        p["dt_bias"] = np.zeros_like(p["dt_bias"])
+    seq = np.array([[0] * 4 + [1] * 6, [0] * 10], dtype=np.int32)
+    dy = rng.standard_normal(p["x"].shape)
+
+    def loss():
+        r = oracle.ssd_fwd(p["x"], p["dt_raw"], p["A"], p["Bm"], p["Cm"], D=p["D"],
+                           dt_bias=p["dt_bias"], softplus=softplus, seq_idx=seq)
+        return float(np.sum(r["y"] * dy))
+
+    g = oracle.ssd_bwd(p["x"], p["dt_raw"], p["A"], p["Bm"], p["Cm"], dy, D=p["D"],
+                       dt_bias=p["dt_bias"], softplus=softplus, seq_idx=seq)
+    for name, gname in [("x", "dx"), ("dt_raw", "ddt_raw"), ("A", "dA"), ("Bm", "dB"),
+                        ("Cm", "dC"), ("D", "dD"), ("dt_bias", "ddt_bias")]:
+        _close(_fd(loss, p[name]), g[gname])

@@ -9,6 +9,7 @@
 
 #include "../../include/ssmscan.h"
 #include "internal.h"
+#include "scan16.cuh"
 
 namespace {
 
@@ -64,8 +65,9 @@ int sm_count() {
 
 struct ScanPlan {
   int nchunks, nsplits, chunks_per_split;
+  bool fast16;  // the N = 16 kernels (scan16_*.cu) and their checkpoint layout
   size_t off_seq, off_ckpt, off_y, off_sP, off_sH, off_sIn, off_pA, off_pD, off_pB, off_sum,
-      total;
+      off_pack, total;
 };
 
 ssm_status_t check_params(const ssm_scan_params* p) {
@@ -117,15 +119,26 @@ ScanPlan plan_scan(const ssm_scan_params* p) {
   if (P < 1) P = 1;
   s.chunks_per_split = (s.nchunks + P - 1) / P;
   s.nsplits = (s.nchunks + s.chunks_per_split - 1) / s.chunks_per_split;
+  // The N = 16 kernels serve the common case: one CTA range per row, dt B
+  // discretisation, real A, L a multiple of 8 and 16-byte aligned inputs.
+  // The forward and the backward read the same inputs, so they agree (out,
+  // written by the forward only, does not take part).
+  s.fast16 = p->N == 16 && !p->state_complex && p->discretization == 0 && s.nsplits == 1 &&
+             p->L % 8 == 0 && aligned(p->u, 16) && aligned(p->delta, 16) && aligned(p->z, 16) &&
+             aligned(p->Bm, 16) && aligned(p->Cm, 16) && aligned(p->seq_idx, 16);
   const size_t rows = (size_t)p->B * p->D;
   size_t off = up(sizeof(int));  // status word first
   s.off_seq = off;
   off += p->cu_seqlens ? up((size_t)p->B * p->L * sizeof(int32_t)) : 0;
   s.off_ckpt = off;
   const size_t npad = (size_t)((p->N + 1) & ~1);
-  // one state checkpoint per 16-token block, kNMax wide (complex: (re, im) pairs)
+  // one state checkpoint per 16-token block, kNMax wide (complex: (re, im) pairs);
+  // N = 16 kernels: one per 8-token segment, per row pair (scan16.cuh)
   const size_t cw = p->state_complex ? 2 : 1;
-  off += up(rows * s.nchunks * (ssm::kChunk / 16) * ssm::kNMax * cw * sizeof(float));
+  if (s.fast16)
+    off += up((size_t)p->B * ((p->D + 1) / 2) * s.nchunks * 16 * 64 * sizeof(float));
+  else
+    off += up(rows * s.nchunks * (ssm::kChunk / 16) * ssm::kNMax * cw * sizeof(float));
   s.off_y = off;
   off += p->z ? up(rows * (size_t)p->L * elem_size(p->dtype)) : 0;
   const size_t per_split = up(rows * s.nsplits * npad * sizeof(float));
@@ -144,6 +157,9 @@ ScanPlan plan_scan(const ssm_scan_params* p) {
   // whole-row summaries (ssm_scan_fwd_summary / ssm_scan_bwd_summary): two [rows][npad]
   s.off_sum = off;
   off += 2 * up(rows * npad * sizeof(float));
+  // N = 16 forward: B / C packed per chunk in its lane layout (32 KB per chunk)
+  s.off_pack = off;
+  off += s.fast16 ? up((size_t)p->B * s.nchunks * 2 * 16 * 256 * sizeof(float)) : 0;
   s.total = off;
   return s;
 }
@@ -180,6 +196,9 @@ ssm_status_t build_args(const ssm_scan_params* p, const ScanPlan& pl, ssm::ScanA
   a->N = p->N;
   a->Npad = (p->N + 1) & ~1;
   a->split_base = 1;
+  a->fast16 = pl.fast16;
+  a->bcpack = pl.fast16 ? reinterpret_cast<float4*>(ws + pl.off_pack) : nullptr;
+  a->Dp = (p->D + 1) / 2;
   a->nchunks = pl.nchunks;
   a->nsplits = pl.nsplits;
   a->chunks_per_split = pl.chunks_per_split;
@@ -248,7 +267,9 @@ ssm_status_t scan_fwd_impl(const ssm_scan_params* p, const void* x, const float*
     if (e != cudaSuccess) return cuda_status(e, "cu_seqlens conversion");
   }
   if (p->state_complex) return cuda_status(ssm::launch_cscan_fwd(a, s), "ssm_scan_fwd launch");
-  return cuda_status(ssm::launch_scan_fwd(a, s), x ? "ssm_conv1d_scan_fwd launch" : "ssm_scan_fwd launch");
+  const char* what = x ? "ssm_conv1d_scan_fwd launch" : "ssm_scan_fwd launch";
+  if (a.fast16) return cuda_status(ssm::launch_scan16_fwd(a, s), what);
+  return cuda_status(ssm::launch_scan_fwd(a, s), what);
 }
 
 }  // namespace
@@ -476,6 +497,7 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
   if (e == cudaSuccess) e = cudaMemsetAsync(g->dC, 0, bc, s);
   if (e != cudaSuccess) return cuda_status(e, "ssm_scan_bwd memset");
   if (p->state_complex) return cuda_status(ssm::launch_cscan_bwd(a, s), "ssm_scan_bwd launch");
+  if (a.fast16) return cuda_status(ssm::launch_scan16_bwd(a, s), "ssm_scan_bwd launch");
   return cuda_status(ssm::launch_scan_bwd(a, s), "ssm_scan_bwd launch");
 }
 

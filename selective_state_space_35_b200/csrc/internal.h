@@ -89,6 +89,11 @@ struct ScanArgs {
   float* part_dA;     // [B*D][N]
   float* part_dD;     // [B*D]
   float* part_ddb;    // [B*D]
+  // N = 16 path (scan16_fwd.cu / scan16_bwd.cu): checkpoints in the row-pair
+  // layout of scan16.cuh, B / C packed per chunk by the forward
+  bool fast16;
+  float4* bcpack;     // [B][nchunks][2][16][64] float4
+  int Dp;             // row pairs per batch entry, ceil(D / 2)
   int B, D, L, N;
   int Npad;           // N rounded up to even: state pairs; stride of ckpt / split arrays
   int nchunks, nsplits, chunks_per_split;

@@ -1,0 +1,117 @@
+// Pieces shared by the N = 16 selective-scan kernels (scan16_fwd.cu,
+// scan16_bwd.cu): the layout constants, the checkpoint indexing the two
+// kernels agree on, and packed (f32x2) element helpers.
+//
+// Work layout of both kernels: time is cut into chunks of 256 tokens and a
+// chunk of one row is spread over 16 (forward) or 32 (backward) lanes of a
+// warp, each lane owning a contiguous run of tokens; the lanes' pieces are
+// joined with the associative operator of "hung-phan ml-skills mamba",
+// "Hardware-Aware Parallel Scan": (a1, b1) + (a2, b2) = (a1 a2, a2 b1 + b2).
+// The forward keeps the state entering every 8-token segment; the backward
+// restarts each lane's 8 tokens from it, so its own scan is the adjoint's.
+#pragma once
+
+#include "scan_common.cuh"
+
+namespace ssm {
+namespace s16 {
+
+constexpr int kN = 16;      // states
+constexpr int kCh = 256;    // tokens per chunk
+constexpr int kSeg = 8;     // tokens per checkpoint segment
+constexpr int kSegs = kCh / kSeg;
+
+// Checkpoints: [B][Dp][nchunks][kN][2][kSegs] fp32 with Dp = ceil(D / 2):
+// rows 2p and 2p + 1 of a batch entry form row pair p, and for every chunk
+// and state the 32 segment-entry states of each row of the pair are
+// contiguous, so one warp-wide 4-byte load per row and state is coalesced in
+// the backward, and a forward lane writes its two segments with one 8-byte
+// store.
+__host__ __device__ __forceinline__ size_t ck_chunk(int b, int rp, int Dp, int nch, int c) {
+  return ((((size_t)b * Dp + rp) * nch + c) * kN) * (2 * kSegs);
+}
+
+// Forward B / C tiles, packed by pack_bc_fwd_kernel into [B][nchunks][mat][kN][64] float4:
+// float4 (k * 16 + jj) of a (mat, state) row holds tokens 16jj+2k, 16jj+8+2k,
+// 16jj+2k+1, 16jj+9+2k, i.e. the (a, b) token pairs of forward lane jj
+// (sub-segment a = tokens 16jj .. 16jj+7, b = 16jj+8 .. 16jj+15).
+constexpr int kFwdTileF4 = 2 * kN * 64;  // float4 per chunk (32 KB)
+
+__device__ __forceinline__ float2 dup(float x) { return make_float2(x, x); }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+// bf16 -> fp32 of the low / high half of a 32-bit word
+__device__ __forceinline__ float lo16(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi16(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Element i (0..7) of 8 bf16 in a uint4
+__device__ __forceinline__ float bf8(const uint4& r, int i) {
+  const uint32_t w = i < 2 ? r.x : i < 4 ? r.y : i < 6 ? r.z : r.w;
+  return (i & 1) ? hi16(w) : lo16(w);
+}
+
+// 8 consecutive elements of a row as raw 16-byte (bf16) or 32-byte (fp32)
+// vectors; `ok` false gives zeros.
+template <typename T>
+struct Raw8;
+template <>
+struct Raw8<__nv_bfloat16> {
+  uint4 r;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p, bool ok) {
+    r = ok ? __ldg(reinterpret_cast<const uint4*>(p)) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  __device__ __forceinline__ float get(int i) const { return bf8(r, i); }
+};
+template <>
+struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p, bool ok) {
+    if (ok) {
+      a = __ldg(reinterpret_cast<const float4*>(p));
+      b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    } else {
+      a = b = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  __device__ __forceinline__ float get(int i) const {
+    const float4& q = i < 4 ? a : b;
+    const int k = i & 3;
+    return k == 0 ? q.x : k == 1 ? q.y : k == 2 ? q.z : q.w;
+  }
+};
+
+// Store 8 consecutive values (one 16-byte vector for bf16, two for fp32).
+template <typename T>
+__device__ __forceinline__ void store8(T* p, const float v[8]);
+template <>
+__device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16* p, const float v[8]) {
+  uint4 r;
+  r.x = Io<__nv_bfloat16>::pack2(v[0], v[1]);
+  r.y = Io<__nv_bfloat16>::pack2(v[2], v[3]);
+  r.z = Io<__nv_bfloat16>::pack2(v[4], v[5]);
+  r.w = Io<__nv_bfloat16>::pack2(v[6], v[7]);
+  *reinterpret_cast<uint4*>(p) = r;
+}
+template <>
+__device__ __forceinline__ void store8<float>(float* p, const float v[8]) {
+  reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+  reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+}
+
+// Round to the storage type and back (the value a later kernel reads).
+template <typename T>
+__device__ __forceinline__ float round_to(float v) {
+  return sizeof(T) == 2 ? __bfloat162float(__float2bfloat16_rn(v)) : v;
+}
+
+// softplus on both halves, the same steps as softplus_sfu (common.cuh).
+__device__ __forceinline__ float2 softplus2(float2 v) {
+  return make_float2(softplus_sfu(v.x), softplus_sfu(v.y));
+}
+
+}  // namespace s16
+
+cudaError_t launch_scan16_fwd(const ScanArgs& a, cudaStream_t s);
+cudaError_t launch_scan16_bwd(const ScanArgs& a, cudaStream_t s);
+
+}  // namespace ssm

@@ -1,0 +1,366 @@
+// Selective scan forward, N = 16 states ("hung-phan ml-skills mamba": the
+// S6 block of "Architecture Diagram", the D term of "Core Concept", the
+// softplus step and SiLU(z) gate of the S6 sketch):
+//   dt_t = softplus(delta_t + bias_d);  a_t = exp(dt_t A_dn) = 2^(dt_t A_dn log2 e)
+//   h_t = a_t h_{t-1} + dt_t B_nt u_t;  y_t = sum_n C_nt h_t + D_d u_t;  out_t = y_t silu(z_t)
+// with a_t := 0 at the first token of a document ("FLA Mamba and Mamba2",
+// packing paragraph).
+//
+// Layout: a warp holds two rows (lanes 0-15 and 16-31) and walks them in
+// 256-token chunks; lane jj of a half owns tokens 16jj .. 16jj+15 of the
+// chunk as two 8-token sub-segments a and b whose matching tokens share one
+// f32x2 register, so every per-token step of the recurrence is one packed
+// instruction for two tokens. States are visited one at a time: the lane
+// composes its two sub-segments (the pages' associative operator), joins the
+// 16 lanes of its row with a 4-step __shfl_up scan, carries the chunk's end
+// state to the next chunk in shared memory and replays its tokens from the
+// exact incoming state, accumulating y. The state entering every 8-token
+// segment is written for the backward (the pages' recompute-in-backward).
+//
+// B and C are packed once per call into the lane layout (pack_bc_fwd_kernel)
+// and each chunk's 32 KB tile arrives by one TMA bulk copy, one chunk ahead,
+// completing on an mbarrier whose wait is bounded.
+#include <atomic>
+
+#include "scan16.cuh"
+
+namespace ssm {
+
+namespace {
+using namespace s16;
+
+constexpr int kFwdWarps = 4;
+constexpr int kFwdRows = 2 * kFwdWarps;
+constexpr unsigned kTileBytes = kFwdTileF4 * 16u;
+
+struct Fwd16Smem {
+  float4 tile[2][kFwdTileF4];  // packed B / C of two chunks
+  uint64_t bar[2];             // TMA completion, one phase per use of a buffer
+  float H[kFwdRows][kN];       // state entering the current chunk
+  float A[kFwdRows][kN];       // A log2(e)
+};
+
+template <typename T>
+__global__ void pack_bc_fwd_kernel(const T* __restrict__ Bm, const T* __restrict__ Cm,
+                                   float4* __restrict__ pk, int L, int nch) {
+  const int b = blockIdx.y;
+  const int q = blockIdx.x * blockDim.x + threadIdx.x;  // float4 index within batch entry b
+  if (q >= nch * kFwdTileF4) return;
+  const int c = q / kFwdTileF4, rem = q % kFwdTileF4;
+  const int mat = rem / (kN * 64), n = (rem / 64) % kN, f = rem % 64;
+  const int k = f >> 4, jj = f & 15;
+  const T* src = (mat ? Cm : Bm) + ((size_t)b * kN + n) * L;
+  const int t0 = c * kCh + 16 * jj + 2 * k;
+  auto g = [&](int t) { return t < L ? Io<T>::ld(src + t) : 0.0f; };
+  pk[(size_t)b * nch * kFwdTileF4 + q] = make_float4(g(t0), g(t0 + 8), g(t0 + 1), g(t0 + 9));
+}
+
+// Loads 8 consecutive elements (zeros when !ok); VEC: one or two vector loads.
+template <typename T, bool VEC>
+__device__ __forceinline__ void load8(const T* p, bool ok, float v[8]) {
+  if (VEC) {
+    Raw8<T> r;
+    r.load(p, ok);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = r.get(i);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = ok ? Io<T>::ld(p + i) : 0.0f;
+  }
+}
+
+// CONV: the per-token stream read is x, and u = silu(conv(x)) is computed
+// here with exactly the separate conv kernel's operations (four fmaf taps in
+// order, document masks, the SFU sigmoid, rounding to T), stored, and scanned.
+// XVEC: x is 16-byte aligned (vector loads).
+template <typename T, bool CONV, bool XVEC>
+__global__ void __launch_bounds__(kFwdWarps * 32, 3) scan16_fwd_kernel(const ScanArgs p) {
+  extern __shared__ float4 smem_dyn[];
+  Fwd16Smem& sm = *reinterpret_cast<Fwd16Smem*>(smem_dyn);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hf = lane >> 4, jj = lane & 15;
+  const int r = 2 * warp + hf;  // row of the CTA
+  const int b = blockIdx.y;
+  const int d = blockIdx.x * kFwdRows + r;
+  const bool active = d < p.D;
+  const int L = p.L, nch = p.nchunks;
+  const size_t rowid = (size_t)b * p.D + (active ? d : 0);
+  const size_t row = rowid * L;
+  const T* u_in = static_cast<const T*>(CONV ? p.xconv : p.u) + row;
+  const T* dl_in = static_cast<const T*>(p.delta) + row;
+  const T* z_in = p.z ? static_cast<const T*>(p.z) + row : nullptr;
+  T* u_out = CONV ? static_cast<T*>(const_cast<void*>(p.u)) + row : nullptr;
+  T* out = static_cast<T*>(p.out) + row;
+  T* ysv = p.z ? static_cast<T*>(p.ysave) + row : nullptr;
+  const int32_t* seqb = p.seq ? p.seq + (size_t)b * L : nullptr;
+  const float4* pk = p.bcpack + (size_t)b * nch * kFwdTileF4;
+  const int rp = d >> 1;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.bar[0], 1);
+    mbar_init(&sm.bar[1], 1);
+    fence_mbar_init();
+  }
+  for (int i = threadIdx.x; i < kFwdRows * kN; i += blockDim.x) {
+    const int rr = i / kN, n = i % kN, dd = blockIdx.x * kFwdRows + rr;
+    const bool act = dd < p.D;
+    sm.A[rr][n] = act ? __ldg(p.A + (size_t)dd * kN + n) * kLog2e : 0.0f;
+    sm.H[rr][n] = (act && p.h0) ? __ldg(p.h0 + ((size_t)b * p.D + dd) * kN + n) : 0.0f;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_expect_tx(&sm.bar[0], kTileBytes);
+    tma_load_1d(&sm.tile[0][0], pk, kTileBytes, &sm.bar[0]);
+  }
+  const float Dv = (active && p.Dskip) ? __ldg(p.Dskip + d) : 0.0f;
+  const float bias = (active && p.delta_bias) ? __ldg(p.delta_bias + d) : 0.0f;
+  float wk[4] = {0.0f, 0.0f, 0.0f, 0.0f}, cbias = 0.0f, c5 = 0.0f, c6 = 0.0f, c7 = 0.0f;
+  if (CONV && active) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) wk[k] = __ldg(p.conv_w + (size_t)d * 4 + k);
+    cbias = p.conv_b ? __ldg(p.conv_b + d) : 0.0f;
+  }
+
+  for (int c = 0; c < nch; ++c) {
+    const int buf = c & 1;
+    const bool ok = mbar_wait_bounded(&sm.bar[buf], (c >> 1) & 1, p.status);
+    // also: every thread is done with chunk c - 1, whose buffer is refilled
+    // next; all threads leave together on a timeout
+    if (!__syncthreads_and(ok)) break;
+    if (threadIdx.x == 0 && c + 1 < nch) {
+      fence_proxy_async_smem();
+      mbar_expect_tx(&sm.bar[buf ^ 1], kTileBytes);
+      tma_load_1d(&sm.tile[buf ^ 1][0], pk + (size_t)(c + 1) * kFwdTileF4, kTileBytes,
+                  &sm.bar[buf ^ 1]);
+    }
+    const int tl = c * kCh + 16 * jj;
+    const bool va = active && tl < L, vb = active && tl + 8 < L;
+    if (c + 1 < nch && (jj & 3) == 0 && active) {  // the next chunk's lines into L2
+      const int tn = tl + kCh;
+      if (tn < L) {
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(dl_in + tn));
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(u_in + tn));
+        if (z_in) asm volatile("prefetch.global.L2 [%0];" ::"l"(z_in + tn));
+      }
+    }
+
+    // per-token values: (sub-segment a, sub-segment b) pairs
+    float ua[8], ub[8], da[8], db[8];
+    load8<T, (!CONV || XVEC)>(u_in + tl, va, ua);
+    load8<T, (!CONV || XVEC)>(u_in + tl + 8, vb, ub);
+    load8<T, true>(dl_in + tl, va, da);
+    load8<T, true>(dl_in + tl + 8, vb, db);
+    // document starts among tokens tl .. tl+15 (bit i), ids tl-3 .. tl+15
+    unsigned rm = 0u;
+    int sg[19];
+    if (seqb) {
+#pragma unroll
+      for (int i = 0; i < 19; ++i) {
+        const int s = tl - 3 + i;
+        sg[i] = (s >= 0 && s < L) ? __ldg(seqb + s) : 0;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        if (tl + i > 0 && tl + i < L && sg[i + 3] != sg[i + 2]) rm |= 1u << i;
+    }
+    if (CONV) {
+      float xv[19];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        xv[3 + i] = ua[i];
+        xv[11 + i] = ub[i];
+      }
+      float h5 = __shfl_up_sync(kFull, xv[16], 1, 16);
+      float h6 = __shfl_up_sync(kFull, xv[17], 1, 16);
+      float h7 = __shfl_up_sync(kFull, xv[18], 1, 16);
+      if (jj == 0) {
+        h5 = c5;
+        h6 = c6;
+        h7 = c7;
+      }
+      c5 = __shfl_sync(kFull, xv[16], 15, 16);
+      c6 = __shfl_sync(kFull, xv[17], 15, 16);
+      c7 = __shfl_sync(kFull, xv[18], 15, 16);
+      xv[0] = h5;
+      xv[1] = h6;
+      xv[2] = h7;
+      float uo[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float acc = cbias;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const bool okk = !seqb || sg[i + k] == sg[i + 3];
+          acc = fmaf(wk[k], okk ? xv[i + k] : 0.0f, acc);
+        }
+        uo[i] = round_to<T>(acc * sigmoid_fast(acc));
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        ua[i] = uo[i];
+        ub[i] = uo[8 + i];
+      }
+      if (va) store8<T>(u_out + tl, ua);
+      if (vb) store8<T>(u_out + tl + 8, ub);
+    }
+    const bool any_reset = __any_sync(kFull, rm != 0u);
+
+    float2 dd[8], xx[8], y2[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float2 v = make_float2(da[i] + bias, db[i] + bias);
+      if (p.softplus) v = softplus2(v);
+      const float2 dt = make_float2(va ? v.x : 0.0f, vb ? v.y : 0.0f);
+      const float2 u2 = make_float2(ua[i], ub[i]);
+      dd[i] = dt;
+      xx[i] = fmul2(dt, u2);
+      y2[i] = fmul2(dup(Dv), u2);
+    }
+
+    const float4* tile = &sm.tile[buf][0];
+    float* ckc = p.ckpt + ck_chunk(b, rp, p.Dp, nch, c) + hf * kSegs + 2 * jj;
+#pragma unroll 1
+    for (int n = 0; n < kN; ++n) {
+      const float2 A2 = dup(sm.A[r][n]);
+      float2 a[8], bx[8];
+      {
+        const float4* Bt = tile + n * 64 + jj;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float4 q = Bt[16 * k];
+          const float2 e0 = fmul2(dd[2 * k], A2), e1 = fmul2(dd[2 * k + 1], A2);
+          a[2 * k] = ex2x2(e0);
+          a[2 * k + 1] = ex2x2(e1);
+          bx[2 * k] = fmul2(xx[2 * k], make_float2(q.x, q.y));
+          bx[2 * k + 1] = fmul2(xx[2 * k + 1], make_float2(q.z, q.w));
+        }
+      }
+      if (any_reset) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if ((rm >> i) & 1u) a[i].x = 0.0f;
+          if ((rm >> (8 + i)) & 1u) a[i].y = 0.0f;
+        }
+      }
+      // compose each sub-segment, then b after a: the lane's map h -> Pl h + Hl
+      float2 P = a[0], H = bx[0];
+#pragma unroll
+      for (int i = 1; i < 8; ++i) {
+        H = ffma2(a[i], H, bx[i]);
+        P = fmul2(P, a[i]);
+      }
+      float Pl = P.x * P.y;
+      float Hl = fmaf(P.y, H.x, H.y);
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1) {
+        const float Pp = __shfl_up_sync(kFull, Pl, off, 16);
+        const float Hp = __shfl_up_sync(kFull, Hl, off, 16);
+        if (jj >= off) {
+          Hl = fmaf(Pl, Hp, Hl);
+          Pl *= Pp;
+        }
+      }
+      const float cin = sm.H[r][n];
+      const float end = fmaf(Pl, cin, Hl);
+      float start = __shfl_up_sync(kFull, end, 1, 16);
+      if (jj == 0) start = cin;
+      if (jj == 15) sm.H[r][n] = end;
+      const float sb = fmaf(P.x, start, H.x);  // state entering sub-segment b
+      if (va) *reinterpret_cast<float2*>(ckc + n * 2 * kSegs) = make_float2(start, sb);
+      float2 h = make_float2(start, sb);
+      const float4* Ct = tile + (kN + n) * 64 + jj;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 q = Ct[16 * k];
+        h = ffma2(a[2 * k], h, bx[2 * k]);
+        y2[2 * k] = ffma2(make_float2(q.x, q.y), h, y2[2 * k]);
+        h = ffma2(a[2 * k + 1], h, bx[2 * k + 1]);
+        y2[2 * k + 1] = ffma2(make_float2(q.z, q.w), h, y2[2 * k + 1]);
+      }
+    }
+
+    if (va || vb) {
+      const bool vo = (reinterpret_cast<uintptr_t>(p.out) & 15) == 0;  // else element stores
+      auto put = [&](T* q, const float v[8]) {
+        if (vo) {
+          store8<T>(q, v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) Io<T>::st(q + i, v[i]);
+        }
+      };
+      float ya[8], yb[8], oa[8], ob[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        ya[i] = y2[i].x;
+        yb[i] = y2[i].y;
+      }
+      if (z_in) {
+        float za[8], zb[8];
+        load8<T, true>(z_in + tl, va, za);
+        load8<T, true>(z_in + tl + 8, vb, zb);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          oa[i] = ya[i] * (za[i] * sigmoid_fast(za[i]));
+          ob[i] = yb[i] * (zb[i] * sigmoid_fast(zb[i]));
+        }
+        if (va) {
+          put(out + tl, oa);
+          store8<T>(ysv + tl, ya);
+        }
+        if (vb) {
+          put(out + tl + 8, ob);
+          store8<T>(ysv + tl + 8, yb);
+        }
+      } else {
+        if (va) put(out + tl, ya);
+        if (vb) put(out + tl + 8, yb);
+      }
+    }
+  }
+
+  __syncwarp();
+  if (active && p.final_state) p.final_state[rowid * kN + jj] = sm.H[r][jj];
+}
+
+// One flag word per device: bit k = 1 once instantiation k has its shared-
+// memory attribute set on that device (the attribute is per device).
+template <typename K>
+cudaError_t smem_attr(K kernel, int bytes, std::atomic<unsigned long long>* done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done->load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done->fetch_or(bit, std::memory_order_release);
+  return e;
+}
+
+template <typename T, bool CONV, bool XVEC>
+cudaError_t fwd16_t(const ScanArgs& a, cudaStream_t s) {
+  static std::atomic<unsigned long long> done{0};
+  const int smem = (int)sizeof(Fwd16Smem);
+  cudaError_t e = smem_attr(scan16_fwd_kernel<T, CONV, XVEC>, smem, &done);
+  if (e != cudaSuccess) return e;
+  const int n4 = a.nchunks * kFwdTileF4;
+  pack_bc_fwd_kernel<T><<<dim3((n4 + 255) / 256, a.B), 256, 0, s>>>(
+      static_cast<const T*>(a.Bm), static_cast<const T*>(a.Cm), a.bcpack, a.L, a.nchunks);
+  dim3 grid((a.D + kFwdRows - 1) / kFwdRows, a.B);
+  scan16_fwd_kernel<T, CONV, XVEC><<<grid, kFwdWarps * 32, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_scan16_fwd(const ScanArgs& a, cudaStream_t s) {
+  const bool xvec = a.xconv && (reinterpret_cast<uintptr_t>(a.xconv) % 16 == 0);
+  if (a.bf16) {
+    if (!a.xconv) return fwd16_t<__nv_bfloat16, false, true>(a, s);
+    return xvec ? fwd16_t<__nv_bfloat16, true, true>(a, s) : fwd16_t<__nv_bfloat16, true, false>(a, s);
+  }
+  if (!a.xconv) return fwd16_t<float, false, true>(a, s);
+  return xvec ? fwd16_t<float, true, true>(a, s) : fwd16_t<float, true, false>(a, s);
+}
+
+}  // namespace ssm

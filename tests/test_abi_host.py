@@ -66,15 +66,21 @@ def _params(ssm, **kw):
 
 
 def test_workspace_size_layout(ssm):
+    nchunks = (1000 + 255) // 256
+    # N = 16, one range per row, L % 8 == 0: the state entering every 8-token
+    # segment (8 bytes per token and row) and B / C packed per chunk (32 KB)
     p = _params(ssm, n_splits=1)
     n1 = ssm.ssm_scan_workspace_size(p)
-    nchunks = (1000 + 255) // 256
-    ckpt = 2 * 8 * nchunks * 16 * 16 * 4  # the state entering every 16-token block
-    assert n1 >= ckpt
+    assert n1 >= 2 * 8 * nchunks * 256 * 8 + 2 * nchunks * 32768
     # with a gate, y before the gate is kept for the backward (bf16 here)
     assert ssm.ssm_scan_workspace_size(_params(ssm, n_splits=1, z=1 << 20)) >= n1 + 2 * 8 * 1000 * 2
-    p2 = _params(ssm, n_splits=3)
-    assert ssm.ssm_scan_workspace_size(p2) > n1
+    # other cases: the state entering every 16-token block, and split carries
+    p8 = _params(ssm, n_splits=1, N=8)
+    n8 = ssm.ssm_scan_workspace_size(p8)
+    assert n8 >= 2 * 8 * nchunks * 16 * 16 * 4
+    assert ssm.ssm_scan_workspace_size(_params(ssm, n_splits=3, N=8)) > n8
+    # a length that is not a multiple of 8 takes the general kernels too
+    assert ssm.ssm_scan_workspace_size(_params(ssm, n_splits=1, L=1001)) < n1 + 2 * 8 * 8
     assert ssm.ssm_conv1d_bwd_workspace_size(2, 8, 1000, 4) >= 2 * 8 * 5 * 4
 
 
@@ -218,8 +224,8 @@ def test_complex_a_rules(ssm):
                        (dict(n_splits=1), 0), (dict(n_splits=0), 0)]:
         p = _params(ssm, state_complex=1, **kw)
         assert L.ssm_scan_workspace_size(ctypes.byref(p), ctypes.byref(n)) == status, kw
-    real = ssm.ssm_scan_workspace_size(_params(ssm, n_splits=1))
-    cplx = ssm.ssm_scan_workspace_size(_params(ssm, state_complex=1))
+    real = ssm.ssm_scan_workspace_size(_params(ssm, n_splits=1, N=8))
+    cplx = ssm.ssm_scan_workspace_size(_params(ssm, state_complex=1, N=8))
     nchunks = (1000 + 255) // 256
     assert cplx >= real + 2 * 8 * nchunks * 16 * 16 * 4  # (re, im) checkpoints
     fake = 1 << 20

@@ -109,6 +109,49 @@ __device__ __forceinline__ float2 softplus2(float2 v) {
   return make_float2(softplus_sfu(v.x), softplus_sfu(v.y));
 }
 
+// Shuffle whose predicate output tells whether the source lane exists
+// (returned as 1 / 0). up: source lane - off within segments of `width`
+// lanes; down: lane + off within the warp.
+template <int WIDTH>
+__device__ __forceinline__ float shfl_up_ok(float v, int off, unsigned& ok) {
+  float r;
+  asm volatile("{\n\t.reg .pred q;\n\tshfl.sync.up.b32 %0|q, %2, %3, %4, -1;\n\tselp.u32 %1, 1, 0, q;\n\t}"
+               : "=f"(r), "=r"(ok)
+               : "f"(v), "r"(off), "r"((32 - WIDTH) << 8));
+  return r;
+}
+__device__ __forceinline__ float shfl_down_ok(float v, int off, unsigned& ok) {
+  float r;
+  asm volatile("{\n\t.reg .pred q;\n\tshfl.sync.down.b32 %0|q, %2, %3, 31, -1;\n\tselp.u32 %1, 1, 0, q;\n\t}"
+               : "=f"(r), "=r"(ok)
+               : "f"(v), "r"(off));
+  return r;
+}
+
+// One step of the forward scan inside groups of 16 lanes: lanes with a
+// source lane off below them compose (P, H) <- (P Pp, P Hp + H).
+__device__ __forceinline__ void fwd_step16(float& P, float& H, int off) {
+  unsigned ok;
+  const float Hp = shfl_up_ok<16>(H, off, ok);
+  const float Pp = __shfl_up_sync(kFull, P, off, 16);
+  if (ok) {
+    H = fmaf(P, Hp, H);
+    P *= Pp;
+  }
+}
+
+// One step of the reverse scan over a warp on (row 0, row 1) pairs: lanes with
+// a source lane off above them compose (P, G) <- (P Pn, P Gn + G).
+__device__ __forceinline__ void bwd_step2(float2& P, float2& G, int off) {
+  unsigned ok;
+  const float2 Gn = make_float2(shfl_down_ok(G.x, off, ok), __shfl_down_sync(kFull, G.y, off));
+  const float2 Pn = shfl_down2(P, off);
+  if (ok) {
+    G = ffma2(P, Gn, G);
+    P = fmul2(P, Pn);
+  }
+}
+
 }  // namespace s16
 
 cudaError_t launch_scan16_fwd(const ScanArgs& a, cudaStream_t s);

@@ -21,6 +21,7 @@
 // and each chunk's 32 KB tile arrives by one TMA bulk copy, one chunk ahead,
 // completing on an mbarrier whose wait is bounded.
 #include <atomic>
+#include <type_traits>
 
 #include "scan16.cuh"
 
@@ -32,12 +33,16 @@ using namespace s16;
 constexpr int kFwdWarps = 4;
 constexpr int kFwdRows = 2 * kFwdWarps;
 constexpr unsigned kTileBytes = kFwdTileF4 * 16u;
+#ifndef SSM_FWD16_STATES
+#define SSM_FWD16_STATES 1
+#endif
+constexpr int kFwdS = SSM_FWD16_STATES;  // states per iteration of the state loop
 
 struct Fwd16Smem {
   float4 tile[2][kFwdTileF4];  // packed B / C of two chunks
   uint64_t bar[2];             // TMA completion, one phase per use of a buffer
   float H[kFwdRows][kN];       // state entering the current chunk
-  float A[kFwdRows][kN];       // A log2(e)
+  float2 A[kFwdRows][kN];      // (A log2(e), A log2(e)): an f32x2 operand as loaded
 };
 
 template <typename T>
@@ -104,7 +109,8 @@ __global__ void __launch_bounds__(kFwdWarps * 32, 3) scan16_fwd_kernel(const Sca
   for (int i = threadIdx.x; i < kFwdRows * kN; i += blockDim.x) {
     const int rr = i / kN, n = i % kN, dd = blockIdx.x * kFwdRows + rr;
     const bool act = dd < p.D;
-    sm.A[rr][n] = act ? __ldg(p.A + (size_t)dd * kN + n) * kLog2e : 0.0f;
+    const float a = act ? __ldg(p.A + (size_t)dd * kN + n) * kLog2e : 0.0f;
+    sm.A[rr][n] = make_float2(a, a);
     sm.H[rr][n] = (act && p.h0) ? __ldg(p.h0 + ((size_t)b * p.D + dd) * kN + n) : 0.0f;
   }
   __syncthreads();
@@ -214,70 +220,83 @@ __global__ void __launch_bounds__(kFwdWarps * 32, 3) scan16_fwd_kernel(const Sca
       const float2 u2 = make_float2(ua[i], ub[i]);
       dd[i] = dt;
       xx[i] = fmul2(dt, u2);
-      y2[i] = fmul2(dup(Dv), u2);
+      y2[i] = make_float2(Dv * u2.x, Dv * u2.y);
     }
 
     const float4* tile = &sm.tile[buf][0];
     float* ckc = p.ckpt + ck_chunk(b, rp, p.Dp, nch, c) + hf * kSegs + 2 * jj;
+    // the state loop, with document starts in this chunk or without
+    auto states = [&](auto RS) {
+    // S states per iteration, their chains interleaved (more independent work
+    // in flight per warp: the scan's shuffles and the replay's FMA chains)
 #pragma unroll 1
-    for (int n = 0; n < kN; ++n) {
-      const float2 A2 = dup(sm.A[r][n]);
-      float2 a[8], bx[8];
-      {
+    for (int n0 = 0; n0 < kN; n0 += kFwdS) {
+      float2 a[kFwdS][8], bx[kFwdS][8], P[kFwdS], H[kFwdS];
+      float Pl[kFwdS], Hl[kFwdS], cin[kFwdS];
+#pragma unroll
+      for (int s = 0; s < kFwdS; ++s) {
+        const int n = n0 + s;
+        cin[s] = sm.H[r][n];
+        const float2 A2 = sm.A[r][n];
         const float4* Bt = tile + n * 64 + jj;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const float4 q = Bt[16 * k];
           const float2 e0 = fmul2(dd[2 * k], A2), e1 = fmul2(dd[2 * k + 1], A2);
-          a[2 * k] = ex2x2(e0);
-          a[2 * k + 1] = ex2x2(e1);
-          bx[2 * k] = fmul2(xx[2 * k], make_float2(q.x, q.y));
-          bx[2 * k + 1] = fmul2(xx[2 * k + 1], make_float2(q.z, q.w));
+          a[s][2 * k] = ex2x2(e0);
+          a[s][2 * k + 1] = ex2x2(e1);
+          bx[s][2 * k] = fmul2(xx[2 * k], make_float2(q.x, q.y));
+          bx[s][2 * k + 1] = fmul2(xx[2 * k + 1], make_float2(q.z, q.w));
         }
-      }
-      if (any_reset) {
+        if constexpr (decltype(RS)::value) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if ((rm >> i) & 1u) a[i].x = 0.0f;
-          if ((rm >> (8 + i)) & 1u) a[i].y = 0.0f;
+          for (int i = 0; i < 8; ++i) {
+            if ((rm >> i) & 1u) a[s][i].x = 0.0f;
+            if ((rm >> (8 + i)) & 1u) a[s][i].y = 0.0f;
+          }
         }
-      }
-      // compose each sub-segment, then b after a: the lane's map h -> Pl h + Hl
-      float2 P = a[0], H = bx[0];
+        // compose each sub-segment, then b after a: the lane's map h -> Pl h + Hl
+        P[s] = a[s][0];
+        H[s] = bx[s][0];
 #pragma unroll
-      for (int i = 1; i < 8; ++i) {
-        H = ffma2(a[i], H, bx[i]);
-        P = fmul2(P, a[i]);
-      }
-      float Pl = P.x * P.y;
-      float Hl = fmaf(P.y, H.x, H.y);
-#pragma unroll
-      for (int off = 1; off < 16; off <<= 1) {
-        const float Pp = __shfl_up_sync(kFull, Pl, off, 16);
-        const float Hp = __shfl_up_sync(kFull, Hl, off, 16);
-        if (jj >= off) {
-          Hl = fmaf(Pl, Hp, Hl);
-          Pl *= Pp;
+        for (int i = 1; i < 8; ++i) {
+          H[s] = ffma2(a[s][i], H[s], bx[s][i]);
+          P[s] = fmul2(P[s], a[s][i]);
         }
+        Pl[s] = P[s].x * P[s].y;
+        Hl[s] = fmaf(P[s].y, H[s].x, H[s].y);
       }
-      const float cin = sm.H[r][n];
-      const float end = fmaf(Pl, cin, Hl);
-      float start = __shfl_up_sync(kFull, end, 1, 16);
-      if (jj == 0) start = cin;
-      if (jj == 15) sm.H[r][n] = end;
-      const float sb = fmaf(P.x, start, H.x);  // state entering sub-segment b
-      if (va) *reinterpret_cast<float2*>(ckc + n * 2 * kSegs) = make_float2(start, sb);
-      float2 h = make_float2(start, sb);
-      const float4* Ct = tile + (kN + n) * 64 + jj;
+#pragma unroll
+      for (int off = 1; off < 16; off <<= 1)
+#pragma unroll
+        for (int s = 0; s < kFwdS; ++s) fwd_step16(Pl[s], Hl[s], off);
+      float2 h[kFwdS];
+#pragma unroll
+      for (int s = 0; s < kFwdS; ++s) {
+        const int n = n0 + s;
+        const float end = fmaf(Pl[s], cin[s], Hl[s]);
+        float start = __shfl_up_sync(kFull, end, 1, 16);
+        if (jj == 0) start = cin[s];
+        if (jj == 15) sm.H[r][n] = end;
+        const float sb = fmaf(P[s].x, start, H[s].x);  // state entering sub-segment b
+        if (va) *reinterpret_cast<float2*>(ckc + n * 2 * kSegs) = make_float2(start, sb);
+        h[s] = make_float2(start, sb);
+      }
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float4 q = Ct[16 * k];
-        h = ffma2(a[2 * k], h, bx[2 * k]);
-        y2[2 * k] = ffma2(make_float2(q.x, q.y), h, y2[2 * k]);
-        h = ffma2(a[2 * k + 1], h, bx[2 * k + 1]);
-        y2[2 * k + 1] = ffma2(make_float2(q.z, q.w), h, y2[2 * k + 1]);
+#pragma unroll
+        for (int s = 0; s < kFwdS; ++s) {
+          const float4 q = tile[(kN + n0 + s) * 64 + jj + 16 * k];
+          h[s] = ffma2(a[s][2 * k], h[s], bx[s][2 * k]);
+          y2[2 * k] = ffma2(make_float2(q.x, q.y), h[s], y2[2 * k]);
+          h[s] = ffma2(a[s][2 * k + 1], h[s], bx[s][2 * k + 1]);
+          y2[2 * k + 1] = ffma2(make_float2(q.z, q.w), h[s], y2[2 * k + 1]);
+        }
       }
     }
+    };
+    if (any_reset) states(std::true_type{});
+    else states(std::false_type{});
 
     if (va || vb) {
       const bool vo = (reinterpret_cast<uintptr_t>(p.out) & 15) == 0;  // else element stores

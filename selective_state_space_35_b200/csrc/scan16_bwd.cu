@@ -25,6 +25,7 @@
 // B and C chunk tiles arrive in shared memory by TMA bulk copies (no
 // multicast), one chunk ahead, completing on an mbarrier with a bounded wait.
 #include <atomic>
+#include <type_traits>
 
 #include "scan16.cuh"
 
@@ -257,6 +258,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2) scan16_bwd_kernel(const Sca
     const T* tileB = &sm.tile[buf][0][0][0];
     const T* tileC = &sm.tile[buf][1][0][0];
     float2 hck = make_float2(ok0 ? __ldg(ckc) : 0.0f, ok1 ? __ldg(ckc + kSegs) : 0.0f);
+    auto states = [&](auto RS) {
 #pragma unroll 1
     for (int n = 0; n < kN; ++n) {
       const float2 hin = hck;
@@ -277,7 +279,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2) scan16_bwd_kernel(const Sca
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           at[i] = ex2x2(fmul2(dd[i], a2));
-          if (any_reset && ((rm >> i) & 1u)) at[i] = make_float2(0.0f, 0.0f);
+          if constexpr (decltype(RS)::value)
+            if ((rm >> i) & 1u) at[i] = make_float2(0.0f, 0.0f);
           const float2 bx = fmul2(xx[i], dup(Bt[i]));
           ah[i] = fmul2(at[i], h);
           h = fadd2(ah[i], bx);
@@ -361,6 +364,9 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2) scan16_bwd_kernel(const Sca
         }
       }
     }
+    };
+    if (any_reset) states(std::true_type{});
+    else states(std::false_type{});
 
     // ---- per-token outputs of the chunk ----
     {

@@ -20,6 +20,7 @@ workload (the reference arm for this project); the oracle is also timed as
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import math
 import os
@@ -46,7 +47,7 @@ SFU_EX2_PER_CLK_PER_SM = 16  # MUFU ex2 results per SM per clock (ssm_probe_ex2_
 # (one layer B2 D1536 N16 L32768 bf16), from
 # one ncu capture (summarised under profiles/); a kernel changed since its
 # capture has no entry.
-NCU_TRAFFIC = {"scan_bwd": 1432608e3 + 598273e3, "scan_fwd": 612232e3 + 760125e3}
+NCU_TRAFFIC = {}
 
 
 def _peaks():
@@ -166,7 +167,7 @@ class Layer:
         self.kw = dict(z=self.z, Dskip=self.Dskip, delta_bias=self.dbias, seq_idx=self.seq,
                        n_splits=n_splits)
 
-    def launches(self) -> int:
+    def launches(self, deterministic=False) -> int:
         """Kernels of this library one step of this layer launches."""
         nch = (self.shape.L + 255) // 256
         P = self.n_splits
@@ -177,7 +178,18 @@ class Layer:
         cps = -(-nch // P)
         P = -(-nch // cps)
         extra = 2 if P > 1 else 0
-        return 1 + (1 + extra) + (2 + extra) + 2
+        # N = 16 on one range per row: B / C packing + scan forward
+        fwd = 2 if (P == 1 and self.shape.N == 16 and self.shape.L % 8 == 0) else 1 + extra
+        return 1 + fwd + (2 + extra + (1 if deterministic else 0)) + 2
+
+    def bytes_held(self) -> dict:
+        """Device bytes of this layer: the scan and conv workspaces, and all
+        buffers (inputs, outputs, gradients, workspaces)."""
+        import torch
+        tens = [v for v in vars(self).values() if isinstance(v, torch.Tensor)]
+        tens += [v for v in self.g.values() if isinstance(v, torch.Tensor)]
+        return {"scan_workspace": self.ws.numel(), "conv_bwd_workspace": self.cws.numel(),
+                "all_buffers": sum(t.numel() * t.element_size() for t in tens)}
 
     def step(self, ev=None):
         ssm = self.ssm
@@ -187,7 +199,8 @@ class Layer:
         if ev is not None:
             ev[1].record()
         ssm.scan_fwd(self.u, self.delta, self.A, self.Bm, self.Cm, out=self.out,
-                     workspace=self.ws, return_final_state=False, **self.kw)
+                     workspace=self.ws,
+                     final_state=self.final_state if self.shape.final_state else None, **self.kw)
         if ev is not None:
             ev[2].record()
         ssm.scan_bwd(self.u, self.delta, self.A, self.Bm, self.Cm, self.dout, self.ws,
@@ -291,7 +304,7 @@ def main():
     ap.add_argument("--config", type=int, default=3)
     ap.add_argument("--n-splits", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0, help="limit the layer count (profiling)")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -299,6 +312,10 @@ def main():
     ap.add_argument("--no-complex", action="store_true", help="skip the complex-A scan measurement")
     ap.add_argument("--no-cp", action="store_true",
                     help="skip the per-rank measurement of the context-parallel kernels")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the scan measurement on the other full-size workloads")
+    ap.add_argument("--no-deterministic", action="store_true",
+                    help="skip the measurement of the deterministic backward")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -418,6 +435,7 @@ def main():
                  "frac_of_roofline": max(t_sfu, t_hbm) / scan_ms},
         "gpu_launches": args.steps * sum(ly.launches() for ly in layers),
         "clocks": ck,
+        "bytes_per_layer": layers[0].bytes_held(),
     }
 
     # e2e: host buffers in, host buffers out, through the same calls
@@ -430,19 +448,112 @@ def main():
         line["complex_a"] = complex_bench(device, layers[0], pk)
     if not args.no_cp:
         line["cp_shard"] = cp_shard_bench(device, layers[0], ranks=8)
+    if not args.no_deterministic:
+        line["deterministic_bwd"] = deterministic_bench(layers[0], avg["scan_bwd"])
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = cpu_count()
         v, rows, secs = oracle_sample(inps[0], args.cpu_seconds, threads)
+        v1, rows1, secs1 = oracle_sample(inps[0], max(2.0, args.cpu_seconds / 3), 1)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": f"{rows} channel rows x {L} tokens of layer 0, conv+scan "
-                                          f"fwd+bwd in fp64, {secs:.1f} s"}
+                                          f"fwd+bwd in fp64, {secs:.1f} s",
+                                "single_thread": {"value": v1, "cores": 1,
+                                                  "sample": f"{rows1} channel rows x {L} tokens, "
+                                                            f"{secs1:.1f} s"}}
+    del inps
+    if not args.no_configs:
+        del layers
+        torch.cuda.empty_cache()
+        line["other_configs"] = {str(c): config_bench(c, device, pk) for c in (2, 4, 5)}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def scan_roofline(sh, fwd_ms, bwd_ms, pk):
+    """Algorithmic HBM bytes and the SFU / HBM bounds of the scan fwd + bwd of
+    one layer of shape `sh` (bf16 activations)."""
+    B, D, N, L = sh.B, sh.D, sh.N, sh.L
+    e_sz = 2
+    by_fwd = (4 * D * e_sz + 2 * N * e_sz) * B * L
+    by_bwd = (7 * D * e_sz + 2 * N * e_sz + 2 * N * 4) * B * L
+    exps = B * D * L * N
+    ex2_peak = SFU_EX2_PER_CLK_PER_SM * 148 * pk["sm_max_mhz"] * 1e6
+    t_sfu = 2 * exps / ex2_peak * 1e3
+    t_hbm = (by_fwd + by_bwd) / (pk["hbm_gbs"] * 1e9) * 1e3
+    return {"hbm_gbs": {"scan_fwd": by_fwd / (fwd_ms * 1e-3) / 1e9,
+                        "scan_bwd": by_bwd / (bwd_ms * 1e-3) / 1e9},
+            "roofline_ms": {"sfu_2BDLN": t_sfu, "hbm_alg_bytes": t_hbm},
+            "frac_of_roofline": max(t_sfu, t_hbm) / (fwd_ms + bwd_ms)}
+
+
+def config_bench(cfg, device, pk, reps=5):
+    """One layer of another full-size workload: the four calls of a step timed
+    with CUDA events per call over `reps` steps after 3 warm-up steps (inputs
+    larger than L2 for every config; the same buffers each step)."""
+    import torch
+    sh = synth.CONFIGS[cfg]
+    inp = synth.make_inputs(sh, synth.seed_for(cfg, 0), want_f64=False)
+    ly = Layer(inp, device, 0)
+    del inp
+    for _ in range(3):
+        ly.step()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(reps)]
+    for e in ev:
+        ly.step(e)
+    torch.cuda.synchronize()
+    names = ["conv1d_fwd", "scan_fwd", "scan_bwd", "conv1d_bwd"]
+    ms = {n: sum(e[k].elapsed_time(e[k + 1]) for e in ev) / reps for k, n in enumerate(names)}
+    scan_ms = ms["scan_fwd"] + ms["scan_bwd"]
+    step_ms = sum(ms.values())
+    r = {"workload": sh.name + (", packed documents" if sh.packed else "")
+                     + (", final state returned" if sh.final_state else ""),
+         "ms_per_layer": ms, "scan_tokens_per_s": sh.B * sh.L / (scan_ms * 1e-3),
+         "step_tokens_per_s": sh.B * sh.L / (step_ms * 1e-3),
+         "bytes_per_layer": ly.bytes_held(), "launches": (reps + 3) * ly.launches()}
+    r.update(scan_roofline(sh, ms["scan_fwd"], ms["scan_bwd"], pk))
+    del ly
+    torch.cuda.empty_cache()
+    return r
+
+
+def deterministic_bench(ly, bwd_ms, reps=5):
+    """The scan backward with deterministic dB / dC (fixed-order sums of the
+    channel groups' partials) on the bench layer, timed with CUDA events over
+    `reps` launches after one warm-up, beside the atomic backward's time."""
+    import torch
+    import selective_state_space_35_b200 as ssm
+    g = {k: torch.empty_like(v) for k, v in ly.g.items()}
+    p = ssm.scan_params(ly.u, ly.delta, ly.A, ly.Bm, ly.Cm, z=ly.z, Dskip=ly.Dskip,
+                        delta_bias=ly.dbias, seq_idx=ly.seq, n_splits=ly.n_splits, out=ly.out,
+                        workspace=ly.ws)
+    gr = ssm.ssm_scan_grads()
+    gr.struct_size = ctypes.sizeof(ssm.ssm_scan_grads)
+    gr.deterministic = 1
+    nbytes = ssm.ssm_scan_bwd_workspace_size(p, gr)
+    bws = torch.empty(nbytes, dtype=torch.uint8, device=ly.u.device)
+
+    def run():
+        ssm.scan_bwd(ly.u, ly.delta, ly.A, ly.Bm, ly.Cm, ly.dout, ly.ws, grads=g,
+                     deterministic=True, bwd_workspace=bws, **ly.kw)
+
+    run()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    same = all(torch.equal(g[k], ly.g[k]) for k in ("du", "ddelta", "dA", "dD"))
+    del bws, g
+    return {"ms_per_layer": ms, "atomic_ms_per_layer": bwd_ms, "cost": ms / bwd_ms - 1.0,
+            "workspace_bytes": nbytes, "other_grads_bitwise_equal_to_atomic": same,
+            "launches": (reps + 1) * 3}
 
 
 def complex_bench(device, ly, pk, reps=5):

@@ -79,7 +79,7 @@ typedef enum { SSM_DTYPE_F32 = 0, SSM_DTYPE_BF16 = 1 } ssm_dtype_t;
 const char* ssm_last_error(void);
 
 /* ABI version of this header (bumped on any incompatible change). */
-#define SSM_ABI_VERSION 5
+#define SSM_ABI_VERSION 6
 int ssm_abi_version(void);
 
 /* ---------------------------------------------------------------------------
@@ -130,7 +130,9 @@ ssm_status_t ssm_conv1d_bwd(const void* x, const float* w, const float* bias,
  *   rejected with SSM_ERR_UNSUPPORTED and a message naming the limit.
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current) and caches it; make that
- *   first call before any stream capture on the device.
+ *   first call before any stream capture on the device. The cached address
+ *   outlives a cudaDeviceReset, so calling again on a device after a reset
+ *   is not supported.
  *   The array is shared by every call and keeps the last call's contents;
  *   each call overwrites every partial it reads, so nothing needs clearing,
  *   but two calls that overlap on the GPU (other streams, other threads) race
@@ -232,14 +234,31 @@ typedef struct {
     float* dC;                 /* [B][N][L] fp32 output */
     float* dD;                 /* [D] nullable output */
     float* ddelta_bias;        /* [D] nullable output */
-    int deterministic;         /* reserved; dA, dD, ddelta_bias are always reduced in a fixed
-                                  order, dB and dC are summed over channels with fp32 atomics */
+    int deterministic;         /* 0: dB and dC are summed over channels with fp32 atomic adds,
+                                  whose order (and so the last bits of the result) varies from
+                                  run to run. 1: every CTA stores the sum over its rows in
+                                  `workspace` below and a second kernel adds the row groups in a
+                                  fixed order, so dB and dC are bitwise reproducible (for the same
+                                  inputs, sizes and device). dA, dD and ddelta_bias are reduced in
+                                  a fixed order either way. */
     float* dinitial_state;     /* [B][D][N] nullable output: dL/dh_{-1} (the gradient with
                                   respect to initial_state, or to the zero state when NULL) */
     const float* dfinal_state; /* [B][D][N] nullable input: dL/dh_{L-1}, a gradient reaching the
                                   final state from outside (a later piece of the sequence, a
                                   loss on the state); NULL = 0. Complex A: (re, im) pairs */
+    void* workspace;           /* device scratch of the backward, caller-owned, 256-byte aligned,
+                                  >= ssm_scan_bwd_workspace_size bytes: the row groups' dB / dC
+                                  sums when deterministic = 1 (NULL and 0 bytes otherwise). Not
+                                  the forward's workspace, which comes in the params. */
+    size_t workspace_bytes;
 } ssm_scan_grads;
+
+/* Bytes of grads->workspace that ssm_scan_bwd needs for these params and
+ * grads: 0 unless grads->deterministic == 1, then (row groups) * 2 * B * N *
+ * L * 4 (twice that for a complex A), with 8 (general kernels) or 12 (N = 16
+ * kernels) rows per group: about 1.1 GB at B = 2, D = 1536, N = 16, L = 32768. */
+ssm_status_t ssm_scan_bwd_workspace_size(const ssm_scan_params* p, const ssm_scan_grads* g,
+                                         size_t* bytes);
 
 /* Backward. Recomputes states from the checkpoints in p->workspace, so the
  * same params (inputs and workspace) as the forward must be passed. A
@@ -328,6 +347,11 @@ ssm_status_t ssm_conv1d_bwd_ctx(const void* x, const float* w, const float* bias
  * gave up (the kernel then stopped early and its outputs are invalid). The
  * forward resets the word; the backward only sets it. Copies 4 bytes from the
  * workspace to *device_status and SYNCHRONISES `stream`.
+ * A timeout means a copy engine or the memory system did not answer within
+ * about 2^22 polls; the kernel waits (again bounded) for its own copies
+ * before it returns, but one that never completed may still be pending. After
+ * SSM_ERR_TIMEOUT treat the stream and the context as unreliable: discard the
+ * outputs and the workspace, and recreate the context before further work.
  * ------------------------------------------------------------------------ */
 ssm_status_t ssm_scan_status(const ssm_scan_params* p, int* device_status, ssm_stream_t stream);
 

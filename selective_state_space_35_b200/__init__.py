@@ -21,13 +21,14 @@ from ._lib import (SsmError, ssm_abi_version, ssm_conv1d_bwd, ssm_conv1d_bwd_noa
                    ssm_last_error,
                    ssm_probe_ex2_rate, ssm_scan_bwd, ssm_scan_status,
                    ssm_scan_fwd, ssm_scan_grads, ssm_scan_params, ssm_scan_workspace_size,
+                   ssm_scan_bwd_workspace_size,
                    ssm_scan_fwd_summary, ssm_scan_bwd_summary, ssm_state_carry,
                    ssm_conv1d_fwd_ctx, ssm_conv1d_bwd_ctx)
 
 __all__ = [
     "SsmError", "ssm_abi_version", "ssm_last_error", "ssm_conv1d_fwd", "ssm_conv1d_bwd",
     "ssm_conv1d_bwd_workspace_size", "ssm_conv1d_bwd_noalloc", "ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_scan_bwd",
-    "ssm_scan_params", "ssm_scan_grads", "ssm_probe_ex2_rate", "probe_ex2_rate", "ssm_scan_status",
+    "ssm_scan_params", "ssm_scan_grads", "ssm_scan_bwd_workspace_size", "ssm_probe_ex2_rate", "probe_ex2_rate", "ssm_scan_status",
     "scan_status", "conv1d_fwd", "conv1d_bwd", "scan_params",
     "scan_workspace_size", "scan_fwd", "scan_bwd", "load",
     "ssm_decode_params", "ssm_decode_step", "decode_step", "ssm_conv1d_scan_fwd",
@@ -223,12 +224,13 @@ def scan_status(u, A, workspace, stream=None) -> int:
 
 def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softplus=True,
              seq_idx=None, cu_seqlens=None, n_splits=0, return_final_state=False, out=None,
-             workspace=None, initial_state=None, zoh=False, stream=None):
+             workspace=None, initial_state=None, zoh=False, final_state=None, stream=None):
     """Selective scan forward.
 
     Returns (out, final_state or None, workspace). Keep `workspace` (it holds
     the state checkpoints and the pre-gate output) and pass it to scan_bwd
-    unchanged. `initial_state` [B, D, N] fp32 is the state before token 0;
+    unchanged. `final_state` is a preallocated output for the final state
+    (implies return_final_state). `initial_state` [B, D, N] fp32 is the state before token 0;
     `zoh` selects the zero-order-hold B_bar = (exp(dt A) - 1) / A B. A of
     shape [D, N, 2] selects the complex diagonal A (see scan_params).
     """
@@ -237,8 +239,12 @@ def scan_fwd(u, delta, A, Bm, Cm, *, z=None, Dskip=None, delta_bias=None, softpl
     N = A.shape[1]
     c2 = (2,) if A.dim() == 3 else ()
     out = torch.empty_like(u) if out is None else out
-    fs = (torch.empty((B, D, N) + c2, dtype=torch.float32, device=u.device)
-          if return_final_state else None)
+    if final_state is not None:
+        _need(final_state, "final_state", torch.float32, (B, D, N) + c2)
+        fs = final_state
+    else:
+        fs = (torch.empty((B, D, N) + c2, dtype=torch.float32, device=u.device)
+              if return_final_state else None)
     p = scan_params(u, delta, A, Bm, Cm, z=z, Dskip=Dskip, delta_bias=delta_bias, softplus=softplus,
                     seq_idx=seq_idx, cu_seqlens=cu_seqlens, n_splits=n_splits, out=out,
                     final_state=fs, initial_state=initial_state, zoh=zoh)
@@ -286,9 +292,15 @@ def conv1d_scan_fwd(x, conv_w, conv_bias, delta, A, Bm, Cm, *, z=None, Dskip=Non
 
 def scan_bwd(u, delta, A, Bm, Cm, dout, workspace, *, z=None, Dskip=None, delta_bias=None,
              softplus=True, seq_idx=None, cu_seqlens=None, n_splits=0, grads=None,
-             initial_state=None, dfinal_state=None, zoh=False, stream=None):
+             initial_state=None, dfinal_state=None, zoh=False, deterministic=False,
+             bwd_workspace=None, stream=None):
     """Selective scan backward; `workspace` must come from the matching scan_fwd
     (called with the same `initial_state`).
+
+    deterministic=True sums dB / dC over channel groups in a fixed order
+    (bitwise reproducible) through a scratch buffer of
+    ssm_scan_bwd_workspace_size bytes: `bwd_workspace` (uint8 on the device)
+    or one allocated here.
 
     Returns a dict: du, ddelta (w.r.t. the raw delta), dz (or None), dA, dB,
     dC, dD, ddelta_bias, dinitial_state (w.r.t. the state before token 0).
@@ -327,6 +339,12 @@ def scan_bwd(u, delta, A, Bm, Cm, dout, workspace, *, z=None, Dskip=None, delta_
                          else None)
     _need(dfinal_state, "dfinal_state", torch.float32, (B, D, N) + c2)
     gr.dfinal_state = dfinal_state.data_ptr() if dfinal_state is not None else None
+    gr.deterministic = 1 if deterministic else 0
+    need = ssm_scan_bwd_workspace_size(p, gr)
+    if need:
+        if bwd_workspace is None:
+            bwd_workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        gr.workspace, gr.workspace_bytes = bwd_workspace.data_ptr(), bwd_workspace.numel()
     _lib.check(ssm_scan_bwd(p, gr, _stream(stream, u.device)))
     return g
 

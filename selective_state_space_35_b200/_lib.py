@@ -59,6 +59,7 @@ class ssm_scan_grads(ctypes.Structure):
         ("deterministic", _i),
         ("dinitial_state", _vp),
         ("dfinal_state", _vp),
+        ("workspace", _vp), ("workspace_bytes", _sz),
     ]
 
 
@@ -79,7 +80,7 @@ _lib = None
 
 EXPORTS = ("ssm_last_error", "ssm_abi_version", "ssm_conv1d_fwd", "ssm_conv1d_bwd_workspace_size",
            "ssm_conv1d_bwd", "ssm_conv1d_bwd_noalloc", "ssm_scan_workspace_size", "ssm_scan_fwd",
-           "ssm_scan_bwd", "ssm_scan_status", "ssm_probe_ex2_rate", "ssm_decode_step",
+           "ssm_scan_bwd", "ssm_scan_bwd_workspace_size", "ssm_scan_status", "ssm_probe_ex2_rate", "ssm_decode_step",
            "ssm_conv1d_scan_fwd", "ssm_scan_fwd_summary", "ssm_scan_bwd_summary",
            "ssm_state_carry", "ssm_conv1d_fwd_ctx", "ssm_conv1d_bwd_ctx")
 
@@ -115,6 +116,9 @@ def load(path: str | None = None):
     L.ssm_scan_fwd.argtypes = [ctypes.POINTER(ssm_scan_params), _vp]
     L.ssm_scan_bwd.restype = _i
     L.ssm_scan_bwd.argtypes = [ctypes.POINTER(ssm_scan_params), ctypes.POINTER(ssm_scan_grads), _vp]
+    L.ssm_scan_bwd_workspace_size.restype = _i
+    L.ssm_scan_bwd_workspace_size.argtypes = [ctypes.POINTER(ssm_scan_params),
+                                              ctypes.POINTER(ssm_scan_grads), ctypes.POINTER(_sz)]
     L.ssm_scan_status.restype = _i
     L.ssm_scan_status.argtypes = [ctypes.POINTER(ssm_scan_params), ctypes.POINTER(_i), _vp]
     L.ssm_probe_ex2_rate.restype = _i
@@ -174,6 +178,13 @@ def ssm_conv1d_bwd_noalloc(*args) -> int:
 def ssm_scan_workspace_size(params: ssm_scan_params) -> int:
     n = _sz(0)
     check(load().ssm_scan_workspace_size(ctypes.byref(params), ctypes.byref(n)))
+    return n.value
+
+
+def ssm_scan_bwd_workspace_size(params: ssm_scan_params, grads: ssm_scan_grads) -> int:
+    n = _sz(0)
+    check(load().ssm_scan_bwd_workspace_size(ctypes.byref(params), ctypes.byref(grads),
+                                             ctypes.byref(n)))
     return n.value
 
 

@@ -443,16 +443,58 @@ ssm_status_t ssm_conv1d_scan_fwd(const ssm_scan_params* p, const void* x, const 
   return scan_fwd_impl(p, x, conv_w, conv_bias, stream);
 }
 
+// Row groups of the backward kernel the plan selects, and the bytes of the
+// deterministic dB / dC partials.
+static size_t dbc_bnl(const ssm_scan_params* p) {
+  return (size_t)p->B * p->N * (p->state_complex ? 2 : 1) * p->L;
+}
+static int dbc_groups(const ssm_scan_params* p, const ScanPlan& pl) {
+  const int rows = pl.fast16 ? ssm::kBwdCtaRows16
+                             : (p->state_complex ? ssm::kCscanCtaRows : ssm::kBwdCtaRows);
+  return (p->D + rows - 1) / rows;
+}
+
+static ssm_status_t check_grads(const ssm_scan_grads* g) {
+  if (!g) return fail(SSM_ERR_INVALID_ARG, "grads is NULL");
+  if (g->struct_size != sizeof(ssm_scan_grads))
+    return fail(SSM_ERR_INVALID_ARG, "grads.struct_size %zu != %zu", g->struct_size,
+                sizeof(ssm_scan_grads));
+  if (g->deterministic != 0 && g->deterministic != 1)
+    return fail(SSM_ERR_INVALID_ARG, "deterministic=%d (0 or 1)", g->deterministic);
+  return ok();
+}
+
+ssm_status_t ssm_scan_bwd_workspace_size(const ssm_scan_params* p, const ssm_scan_grads* g,
+                                         size_t* bytes) {
+  if (!bytes) return fail(SSM_ERR_INVALID_ARG, "bytes is NULL");
+  ssm_status_t st = check_params(p);
+  if (st != SSM_OK) return st;
+  st = check_grads(g);
+  if (st != SSM_OK) return st;
+  *bytes = g->deterministic
+               ? up((size_t)dbc_groups(p, plan_scan(p)) * 2 * dbc_bnl(p) * sizeof(float))
+               : 0;
+  return ok();
+}
+
 ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
                           ssm_stream_t stream) {
   if (injected("ssm_scan_bwd")) return fail(SSM_ERR_INJECTED, "ssm_scan_bwd: injected failure");
   ssm_status_t st = check_params(p);
   if (st != SSM_OK) return st;
-  if (!g) return fail(SSM_ERR_INVALID_ARG, "grads is NULL");
-  if (g->struct_size != sizeof(ssm_scan_grads))
-    return fail(SSM_ERR_INVALID_ARG, "grads.struct_size %zu != %zu", g->struct_size,
-                sizeof(ssm_scan_grads));
+  st = check_grads(g);
+  if (st != SSM_OK) return st;
   const ScanPlan pl = plan_scan(p);
+  size_t det_need = 0;
+  if (g->deterministic) {
+    det_need = up((size_t)dbc_groups(p, pl) * 2 * dbc_bnl(p) * sizeof(float));
+    if (!g->workspace || g->workspace_bytes < det_need)
+      return fail(SSM_ERR_INVALID_ARG,
+                  "deterministic backward: grads.workspace of %zu bytes needed (have %zu)", det_need,
+                  g->workspace ? g->workspace_bytes : (size_t)0);
+    if (!aligned(g->workspace, kAlign))
+      return fail(SSM_ERR_INVALID_ARG, "grads.workspace must be 256-byte aligned");
+  }
   st = check_scan_buffers(p, pl);
   if (st != SSM_OK) return st;
   if (!g->dout || !g->du || !g->ddelta || !g->dA || !g->dB || !g->dC)
@@ -492,13 +534,23 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
                                                   const_cast<int32_t*>(a.seq), s);
     if (e != cudaSuccess) return cuda_status(e, "cu_seqlens conversion");
   }
-  const size_t bc = (size_t)p->B * p->N * p->L * sizeof(float) * (p->state_complex ? 2 : 1);
-  cudaError_t e = cudaMemsetAsync(g->dB, 0, bc, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(g->dC, 0, bc, s);
-  if (e != cudaSuccess) return cuda_status(e, "ssm_scan_bwd memset");
-  if (p->state_complex) return cuda_status(ssm::launch_cscan_bwd(a, s), "ssm_scan_bwd launch");
-  if (a.fast16) return cuda_status(ssm::launch_scan16_bwd(a, s), "ssm_scan_bwd launch");
-  return cuda_status(ssm::launch_scan_bwd(a, s), "ssm_scan_bwd launch");
+  cudaError_t e = cudaSuccess;
+  if (g->deterministic) {
+    // every (group, dB / dC, element) of the partials is stored by the kernel
+    a.dbc_part = static_cast<float*>(g->workspace);
+    a.dbc_bnl = dbc_bnl(p);
+  } else {
+    const size_t bc = dbc_bnl(p) * sizeof(float);
+    e = cudaMemsetAsync(g->dB, 0, bc, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(g->dC, 0, bc, s);
+    if (e != cudaSuccess) return cuda_status(e, "ssm_scan_bwd memset");
+  }
+  if (p->state_complex) e = ssm::launch_cscan_bwd(a, s);
+  else if (a.fast16) e = ssm::launch_scan16_bwd(a, s);
+  else e = ssm::launch_scan_bwd(a, s);
+  if (e == cudaSuccess && g->deterministic)
+    e = ssm::launch_dbc_reduce(a.dbc_part, dbc_groups(p, pl), a.dbc_bnl, g->dB, g->dC, s);
+  return cuda_status(e, "ssm_scan_bwd launch");
 }
 
 // Shared part of the two whole-row summaries: validation, args with one

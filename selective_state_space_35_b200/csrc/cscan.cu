@@ -34,6 +34,7 @@ namespace {
 constexpr int kCB = 16;                    // tokens per block = checkpoint interval
 constexpr int kCWarps = 4;
 constexpr int kCRows = 2 * kCWarps;        // rows per CTA
+static_assert(kCRows == kCscanCtaRows, "row groups of the deterministic dB / dC partials");
 constexpr int kCLd = kCB + 4;              // fp32 state-row stride: 8 lanes on distinct banks
 constexpr int kXHalf = kNMax * kCLd + 16;  // one row half of a transposition array
 constexpr int kCThreads = kCWarps * 32;
@@ -563,7 +564,15 @@ cscan_bwd_kernel(const ScanArgs p) {
           v[i].w += v[i + s].w;
         }
       const int t = tb + 4 * q;
-      if (m < N && t < L) {
+      if (m < N && t < L && p.dbc_part) {  // deterministic: this CTA's sum, added later in order
+        float* dst = p.dbc_part + ((size_t)blockIdx.x * 2 + (arr < 2 ? 1 : 0)) * p.dbc_bnl +
+                     (((size_t)b * N + m) * 2 + (arr & 1)) * L + t;
+        const int left = L - t;
+        dst[0] = v[0].x;
+        if (left > 1) dst[1] = v[0].y;
+        if (left > 2) dst[2] = v[0].z;
+        if (left > 3) dst[3] = v[0].w;
+      } else if (m < N && t < L) {
         float* dst = (arr < 2 ? p.dC : p.dB) + (((size_t)b * N + m) * 2 + (arr & 1)) * L + t;
         if (VEC) {
           atomicAdd(reinterpret_cast<float4*>(dst), v[0]);
@@ -644,13 +653,9 @@ cudaError_t cfwd_t(const ScanArgs& a, cudaStream_t s) {
 template <typename T, bool VEC>
 cudaError_t cbwd_t(const ScanArgs& a, cudaStream_t s) {
   const size_t smem = sizeof(CBwdSmem<T>);
-  static bool smem_set = false;  // once per instantiation and process (a benign race)
-  if (!smem_set) {
-    cudaError_t e = cudaFuncSetAttribute(cscan_bwd_kernel<T, VEC>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    smem_set = true;
-  }
+  static std::atomic<unsigned long long> smem_done{0};
+  cudaError_t e = smem_attr(cscan_bwd_kernel<T, VEC>, (int)smem, &smem_done);
+  if (e != cudaSuccess) return e;
   dim3 g((a.D + kCRows - 1) / kCRows, a.B);
   cscan_bwd_kernel<T, VEC><<<g, kCThreads, smem, s>>>(a);
   const int m = a.D * 2 * a.N;

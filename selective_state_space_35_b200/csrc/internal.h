@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace ssm {
 
 constexpr int kS = 8;                 // tokens per lane in the scan kernels
@@ -35,6 +37,22 @@ struct ConvArgs {
   int B, D, L, silu;
   bool bf16, vec;
 };
+
+// Sets a kernel's dynamic shared-memory limit once per device. The attribute
+// belongs to the (kernel, device) pair, so `done` holds one bit per device
+// (devices 64 and up set it on every call); threads may race to set it, which
+// is harmless since they set the same value.
+template <typename K>
+inline cudaError_t smem_attr(K kernel, int bytes, std::atomic<unsigned long long>* done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done->load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done->fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 cudaError_t launch_conv1d_fwd(const ConvArgs& a, cudaStream_t s);
 // Fixed device scratch of the allocation-free conv1d backward.
@@ -79,6 +97,11 @@ struct ScanArgs {
   float* dh0;         // [B*D][N] nullable
   const float* dhL;   // [B*D][N] nullable: dL/d(final state), the adjoint entering from the right
   int split_base;     // first split the backward summary kernel handles (1; 0 for a whole-row summary)
+  // deterministic dB / dC: each CTA stores its row-group's sums here instead of
+  // adding them atomically, [groups][2 (dB, dC)][dbc_bnl] fp32, and
+  // launch_dbc_reduce sums the groups in order; nullptr: atomic adds
+  float* dbc_part;
+  size_t dbc_bnl;     // B * N * planes * L (planes: 2 for a complex A)
   // workspace pieces
   int* status;        // sticky device status word (0 = ok, 4 = a bounded wait timed out)
   float* ckpt;        // [B*D][nchunks * 16][kNMax] state entering each 16-token block
@@ -141,6 +164,14 @@ struct DecodeArgs {
 
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_scan_bwd(const ScanArgs& a, cudaStream_t s);
+// Rows per CTA of the backward kernels (CTAs along D = row groups of the
+// deterministic dB / dC partials): scan16_bwd.cu, scan_bwd.cu, cscan.cu.
+constexpr int kBwdCtaRows16 = 12;
+constexpr int kBwdCtaRows = 8;
+constexpr int kCscanCtaRows = 8;
+// Fixed-order sum of the row groups' dB / dC partials into dB and dC.
+cudaError_t launch_dbc_reduce(const float* part, int groups, size_t bnl, float* dB, float* dC,
+                              cudaStream_t s);
 cudaError_t probe_ex2_rate(float* sink, size_t sink_floats, double* rate, cudaStream_t s);
 cudaError_t launch_cu_seqlens_to_seq(const int32_t* cu, int n_docs, int L, int32_t* seq,
                                      cudaStream_t s);

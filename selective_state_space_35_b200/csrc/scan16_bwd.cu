@@ -36,6 +36,7 @@ using namespace s16;
 
 constexpr int kBwdWarps = 6;
 constexpr int kBwdRows = 2 * kBwdWarps;
+static_assert(kBwdRows == kBwdCtaRows16, "row groups of the deterministic dB / dC partials");
 
 template <typename T>
 struct Bwd16Smem {
@@ -349,7 +350,13 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2) scan16_bwd_kernel(const Sca
           s = make_float4(lo.x, lo.y, hi.x, hi.y);
         }
         const int t = c * kCh + 8 * (f & 31) + 4 * (f >> 5);
-        if (t < L) {
+        if (t < L && p.dbc_part) {  // deterministic: this CTA's sum, added later in order
+          float* dst = p.dbc_part + ((size_t)blockIdx.x * 2 + mat) * p.dbc_bnl + ((size_t)b * kN + n) * L + t;
+          dst[0] = s.x;
+          dst[1] = s.y;
+          dst[2] = s.z;
+          dst[3] = s.w;
+        } else if (t < L) {
           float* dst = (mat ? p.dC : p.dB) + ((size_t)b * kN + n) * L + t;
           if (VG) {
             asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(s.x),
@@ -432,17 +439,6 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2) scan16_bwd_kernel(const Sca
   }
 }
 
-template <typename K>
-cudaError_t smem_attr(K kernel, int bytes, std::atomic<unsigned long long>* done) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
-  if (bit && (done->load(std::memory_order_acquire) & bit)) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && bit) done->fetch_or(bit, std::memory_order_release);
-  return e;
-}
 
 __global__ void bwd16_param_reduce_kernel(const float* __restrict__ pA, const float* __restrict__ pD,
                                           const float* __restrict__ pB, float* __restrict__ dA,

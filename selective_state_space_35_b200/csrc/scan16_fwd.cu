@@ -342,19 +342,6 @@ __global__ void __launch_bounds__(kFwdWarps * 32, 3) scan16_fwd_kernel(const Sca
   if (active && p.final_state) p.final_state[rowid * kN + jj] = sm.H[r][jj];
 }
 
-// One flag word per device: bit k = 1 once instantiation k has its shared-
-// memory attribute set on that device (the attribute is per device).
-template <typename K>
-cudaError_t smem_attr(K kernel, int bytes, std::atomic<unsigned long long>* done) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
-  if (bit && (done->load(std::memory_order_acquire) & bit)) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && bit) done->fetch_or(bit, std::memory_order_release);
-  return e;
-}
 
 template <typename T, bool CONV, bool XVEC>
 cudaError_t fwd16_t(const ScanArgs& a, cudaStream_t s) {

@@ -72,6 +72,7 @@ constexpr int kBlk = 32;                   // tokens per block (= checkpoint int
 #endif
 constexpr int kWarps = SSM_BWD_WARPS;
 constexpr int kRows = 2 * kWarps;          // rows per CTA
+static_assert(kRows == kBwdCtaRows, "row groups of the deterministic dB / dC partials");
 constexpr int kLd = kBlk + 4;              // fp32 row stride: the 16 state rows on distinct banks
 constexpr int kRowArrays = 5;              // delta, u, dout, z, y (y: forward output before the gate)
 
@@ -483,7 +484,14 @@ scan_bwd_kernel(const ScanArgs p) {
           v[i] = make_float4(lo.x, lo.y, hi.x, hi.y);
         }
       const int t = tb + 4 * q;
-      if (m < N && t < L) {
+      if (m < N && t < L && p.dbc_part) {  // deterministic: this CTA's sum, added later in order
+        float* dst = p.dbc_part + ((size_t)blockIdx.x * 2 + arr) * p.dbc_bnl + ((size_t)b * N + m) * L + t;
+        const int left = L - t;
+        dst[0] = v[0].x;
+        if (left > 1) dst[1] = v[0].y;
+        if (left > 2) dst[2] = v[0].z;
+        if (left > 3) dst[3] = v[0].w;
+      } else if (m < N && t < L) {
         float* dst = (arr ? p.dC : p.dB) + ((size_t)b * N + m) * L + t;
         if (VEC) {
           atomicAdd(reinterpret_cast<float4*>(dst), v[0]);
@@ -663,6 +671,10 @@ __global__ void bwd_param_reduce_kernel(const float* __restrict__ pA, const floa
 
 template <typename T, bool VEC, bool ZOH>
 cudaError_t bwd_t(const ScanArgs& a, cudaStream_t s) {
+  const size_t smem = sizeof(BwdSmem<T>);
+  static std::atomic<unsigned long long> smem_done{0};
+  cudaError_t e = smem_attr(scan_bwd_kernel<T, VEC, ZOH>, (int)smem, &smem_done);
+  if (e != cudaSuccess) return e;
   if (a.nsplits > 1) {
     // adjoint carry into each split from the right (lanes-over-time summary)
     constexpr int G = 4;
@@ -672,14 +684,6 @@ cudaError_t bwd_t(const ScanArgs& a, cudaStream_t s) {
     bwd_split_carry_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.split_P, a.split_H, a.dhL,
                                                           a.split_in, a.B * a.D, a.nsplits,
                                                           a.Npad, a.N);
-  }
-  const size_t smem = sizeof(BwdSmem<T>);
-  static bool smem_set = false;  // once per instantiation and process (a benign race)
-  if (!smem_set) {
-    cudaError_t e = cudaFuncSetAttribute(scan_bwd_kernel<T, VEC, ZOH>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    smem_set = true;
   }
   dim3 g2((a.D + kRows - 1) / kRows, a.B, a.nsplits);
   scan_bwd_kernel<T, VEC, ZOH><<<g2, kWarps * 32, smem, s>>>(a);
@@ -697,6 +701,27 @@ cudaError_t bwd_dispatch(const ScanArgs& a, cudaStream_t s) {
   if (a.bf16)
     return a.vec ? bwd_t<__nv_bfloat16, true, ZOH>(a, s) : bwd_t<__nv_bfloat16, false, ZOH>(a, s);
   return a.vec ? bwd_t<float, true, ZOH>(a, s) : bwd_t<float, false, ZOH>(a, s);
+}
+
+// dB[e] = sum_g part[g][0][e], dC[e] = sum_g part[g][1][e], g in increasing order.
+__global__ void dbc_reduce_kernel(const float* __restrict__ part, int groups, size_t bnl,
+                                  float* __restrict__ dB, float* __restrict__ dC) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= 2 * bnl) return;
+  const int mat = i >= bnl;
+  const size_t e = i - (mat ? bnl : 0);
+  const float* q = part + (size_t)mat * bnl + e;
+  float s = 0.0f;
+#pragma unroll 8
+  for (int g = 0; g < groups; ++g) s += __ldcs(q + (size_t)g * 2 * bnl);
+  (mat ? dC : dB)[e] = s;
+}
+
+cudaError_t launch_dbc_reduce(const float* part, int groups, size_t bnl, float* dB, float* dC,
+                              cudaStream_t s) {
+  const size_t n = 2 * bnl;
+  dbc_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, groups, bnl, dB, dC);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_scan_bwd(const ScanArgs& a, cudaStream_t s) {

@@ -362,13 +362,9 @@ __global__ void cu_seqlens_to_seq_kernel(const int32_t* __restrict__ cu, int n_d
 
 template <typename T, int G, bool VEC, bool SUMMARY, int NT, bool CONV, bool ZOH>
 cudaError_t fwd_smem_attr() {
-  static bool done = false;  // once per instantiation and process (a benign race)
-  if (done) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(scan_fwd_kernel<T, G, VEC, SUMMARY, NT, CONV, ZOH>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)sizeof(FwdSmem<G>));
-  if (e == cudaSuccess) done = true;
-  return e;
+  static std::atomic<unsigned long long> done{0};
+  return smem_attr(scan_fwd_kernel<T, G, VEC, SUMMARY, NT, CONV, ZOH>, (int)sizeof(FwdSmem<G>),
+                   &done);
 }
 
 template <typename T, int G, bool VEC, int NT, bool CONV, bool ZOH>

@@ -196,7 +196,7 @@ def test_decode_null_params(ssm):
 
 def test_grads_struct_has_initial_state_gradient(ssm):
     names = [f[0] for f in ssm.ssm_scan_grads._fields_]
-    assert names[-2:] == ["dinitial_state", "dfinal_state"]
+    assert names[-4:] == ["dinitial_state", "dfinal_state", "workspace", "workspace_bytes"]
     assert [f[0] for f in ssm.ssm_scan_params._fields_][-3:] == ["initial_state", "discretization",
                                                                  "state_complex"]
 
@@ -268,3 +268,44 @@ def test_piece_calls_validation(ssm):
     assert L.ssm_conv1d_bwd_ctx(x, w, None, fake + 12288, None, None, fake + 16384, fake + 24576,
                                 None, fake, u, fake + 20480, None, 2, 8, 64, 4, 1, 1,
                                 fake + 65536, 1 << 20, None) == 1
+
+
+def _grads(ssm, **kw):
+    g = ssm.ssm_scan_grads()
+    g.struct_size = ctypes.sizeof(ssm.ssm_scan_grads)
+    for k, v in kw.items():
+        setattr(g, k, v)
+    return g
+
+
+def test_deterministic_backward_workspace(ssm):
+    """deterministic = 1 needs (channel groups) x (dB, dC) x B x N x L fp32
+    partial sums: groups of 12 rows on the N = 16 kernels, 8 on the others,
+    both planes for a complex A; 0 bytes otherwise; other values rejected."""
+    from selective_state_space_35_b200 import _lib
+    L = _lib.load()
+    up = lambda x: (x + 255) // 256 * 256
+    assert ssm.ssm_scan_bwd_workspace_size(_params(ssm, n_splits=1), _grads(ssm)) == 0
+    for kw, groups, planes in [(dict(n_splits=1, D=30), 3, 1),
+                               (dict(n_splits=1, D=30, N=8), 4, 1),
+                               (dict(n_splits=2, D=30), 4, 1),
+                               (dict(n_splits=1, D=30, L=1001), 4, 1),
+                               (dict(n_splits=1, D=30, N=8, state_complex=1), 4, 2)]:
+        p = _params(ssm, **kw)
+        want = up(groups * 2 * p.B * p.N * planes * p.L * 4)
+        assert ssm.ssm_scan_bwd_workspace_size(p, _grads(ssm, deterministic=1)) == want, kw
+    n = ctypes.c_size_t(0)
+    p = _params(ssm, n_splits=1)
+    g = _grads(ssm, deterministic=2)
+    assert L.ssm_scan_bwd_workspace_size(ctypes.byref(p), ctypes.byref(g), ctypes.byref(n)) == 1
+    fake = 1 << 20
+    p = _params(ssm, u=fake, delta=fake + 4096, A=fake + 8192, Bm=fake + 12288, Cm=fake + 16384,
+                out=fake + 20480, workspace=fake + 65536, workspace_bytes=1 << 30, n_splits=1)
+    g = _grads(ssm, dout=fake, du=fake, ddelta=fake, dA=fake, dB=fake, dC=fake, deterministic=1)
+    assert L.ssm_scan_bwd(ctypes.byref(p), ctypes.byref(g), None) == 1  # no scratch given
+    assert "grads.workspace" in ssm.ssm_last_error()
+    g.workspace, g.workspace_bytes = fake + (1 << 24), 1000
+    assert L.ssm_scan_bwd(ctypes.byref(p), ctypes.byref(g), None) == 1  # too small
+    g.workspace, g.workspace_bytes = fake + (1 << 24) + 16, 1 << 30
+    assert L.ssm_scan_bwd(ctypes.byref(p), ctypes.byref(g), None) == 1  # misaligned
+    assert "aligned" in ssm.ssm_last_error()

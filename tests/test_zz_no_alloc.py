@@ -5,7 +5,9 @@ its input and output buffers, and loops that must not call cudaMalloc /
 cudaFree. For them the library offers a variant of the conv1d backward whose
 scratch lives in a fixed device array. These checks call it through the C
 ABI, twice in a row with different inputs (the array keeps the previous
-call's contents), and compare it with the workspace version. This file is
+call's contents), compare it with the workspace version, and check that a
+call changes neither the memory torch's allocator holds nor the device's
+free memory. This file is
 collected last so that a run stopping at the first failure has already run
 every other test.
 """
@@ -65,3 +67,29 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
                                     4, 4096, 16384, 4, 1, 1, None)
     assert st == 2
     assert "scratch" in ssm.ssm_last_error()
+
+
+def test_noalloc_call_allocates_nothing():
+    """After a first call (which caches the scratch array's address and may load
+    the module), further calls leave both torch's allocated bytes and the
+    driver's free-memory count unchanged."""
+    import torch
+    import selective_state_space_35_b200 as ssm
+    inp = synth.make_inputs(synth.Shape("noalloc", 2, 64, 16, 2048, "bf16"), 71, conv_bias_scale=0.3)
+    dv = device_inputs(inp)
+    _noalloc(ssm, dv["x"], dv["conv_w"], dv["conv_b"], dv["seq_idx"], dv["dout"])
+    B, D, L = dv["x"].shape
+    dx = torch.empty_like(dv["x"])
+    dw = torch.empty((D, 4), dtype=torch.float32, device="cuda")
+    db = torch.empty((D,), dtype=torch.float32, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    alloc0, free0 = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        st = ssm.ssm_conv1d_bwd_noalloc(_p(dv["x"]), _p(dv["conv_w"]), _p(dv["conv_b"]),
+                                        _p(dv["seq_idx"]), _p(dv["dout"]), _p(dx), _p(dw), _p(db),
+                                        B, D, L, 4, 1, 1, stream)
+        assert st == 0, ssm.ssm_last_error()
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert torch.cuda.mem_get_info()[0] == free0

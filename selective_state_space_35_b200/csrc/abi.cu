@@ -443,8 +443,9 @@ ssm_status_t ssm_conv1d_scan_fwd(const ssm_scan_params* p, const void* x, const 
   return scan_fwd_impl(p, x, conv_w, conv_bias, stream);
 }
 
-// Row groups of the backward kernel the plan selects, and the bytes of the
-// deterministic dB / dC partials.
+// Row groups of the backward kernel the plan selects (at most: the N = 16
+// kernels may take larger groups), and the bytes of the deterministic dB / dC
+// partials.
 static size_t dbc_bnl(const ssm_scan_params* p) {
   return (size_t)p->B * p->N * (p->state_complex ? 2 : 1) * p->L;
 }
@@ -548,8 +549,12 @@ ssm_status_t ssm_scan_bwd(const ssm_scan_params* p, const ssm_scan_grads* g,
   if (p->state_complex) e = ssm::launch_cscan_bwd(a, s);
   else if (a.fast16) e = ssm::launch_scan16_bwd(a, s);
   else e = ssm::launch_scan_bwd(a, s);
-  if (e == cudaSuccess && g->deterministic)
-    e = ssm::launch_dbc_reduce(a.dbc_part, dbc_groups(p, pl), a.dbc_bnl, g->dB, g->dC, s);
+  if (e == cudaSuccess && g->deterministic) {
+    // the N = 16 kernels may have used larger row groups than the workspace bound
+    const int groups =
+        a.fast16 ? (p->D + ssm::scan16_bwd_rows(a) - 1) / ssm::scan16_bwd_rows(a) : dbc_groups(p, pl);
+    e = ssm::launch_dbc_reduce(a.dbc_part, groups, a.dbc_bnl, g->dB, g->dC, s);
+  }
   return cuda_status(e, "ssm_scan_bwd launch");
 }
 

@@ -165,7 +165,8 @@ struct DecodeArgs {
 cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_scan_bwd(const ScanArgs& a, cudaStream_t s);
 // Rows per CTA of the backward kernels (CTAs along D = row groups of the
-// deterministic dB / dC partials): scan16_bwd.cu, scan_bwd.cu, cscan.cu.
+// deterministic dB / dC partials): scan16_bwd.cu (its smaller shape; the
+// launch may take 22-row CTAs, i.e. fewer groups), scan_bwd.cu, cscan.cu.
 constexpr int kBwdCtaRows16 = 12;
 constexpr int kBwdCtaRows = 8;
 constexpr int kCscanCtaRows = 8;

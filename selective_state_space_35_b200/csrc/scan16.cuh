@@ -11,6 +11,8 @@
 // restarts each lane's 8 tokens from it, so its own scan is the adjoint's.
 #pragma once
 
+#include <atomic>
+
 #include "scan_common.cuh"
 
 namespace ssm {
@@ -152,9 +154,44 @@ __device__ __forceinline__ void bwd_step2(float2& P, float2& G, int off) {
   }
 }
 
+// SMs of the current device (cached per device; 148 on B200).
+inline int sm_count() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 64) {
+    const int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  if (dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// Both kernels come in two CTA shapes: a small CTA several of which share an
+// SM, and one CTA of 11 warps per SM. A CTA owns a fixed group of rows for the
+// whole sequence, so the grid runs in waves of (SMs x CTAs per SM); the call
+// takes the shape whose waves are fullest (CTAs / capacity of the waves it
+// needs), the small one on a tie. At B = 2, D = 1536 on 148 SMs: 22-row CTAs
+// fill 140 / 148 of one wave, 12-row CTAs 256 / 296.
+inline int pick_shape(int B, int D, int rows_small, int per_sm_small, int rows_big) {
+  const long sms = sm_count();
+  auto fill = [&](int rows, int per_sm) {
+    const long ctas = (long)B * ((D + rows - 1) / rows);
+    const long cap = sms * per_sm;
+    return (double)ctas / (double)(((ctas + cap - 1) / cap) * cap);
+  };
+  return fill(rows_big, 1) > fill(rows_small, per_sm_small) + 1e-9 ? 1 : 0;
+}
+
 }  // namespace s16
 
 cudaError_t launch_scan16_fwd(const ScanArgs& a, cudaStream_t s);
 cudaError_t launch_scan16_bwd(const ScanArgs& a, cudaStream_t s);
+// Rows per CTA the N = 16 backward uses for these arguments (the row groups
+// of its deterministic dB / dC partials).
+int scan16_bwd_rows(const ScanArgs& a);
 
 }  // namespace ssm

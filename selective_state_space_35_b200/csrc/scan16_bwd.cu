@@ -34,25 +34,26 @@ namespace ssm {
 namespace {
 using namespace s16;
 
-constexpr int kBwdWarps = 6;
-constexpr int kBwdRows = 2 * kBwdWarps;
-static_assert(kBwdRows == kBwdCtaRows16, "row groups of the deterministic dB / dC partials");
+// CTA shapes (warps = row pairs): 6 warps, two CTAs per SM, or 11 warps, one
+// per SM (see pick_shape).
+constexpr int kBwdWarpsSmall = 6, kBwdWarpsBig = 11;
+static_assert(2 * kBwdWarpsSmall == kBwdCtaRows16, "smallest row group of the dB / dC partials");
 
-template <typename T>
+template <typename T, int W>
 struct Bwd16Smem {
-  T tile[2][2][kN][kCh];                 // B / C of two chunks, activation dtype
-  float4 red[2][kBwdWarps][2][kCh / 4];  // dB / dC of one state (row-pair sums), two states in flight
-  float4 pv[kBwdWarps][8][32];           // per lane: (sigma'(v) u, sigma'(v)) of both rows, 8 tokens
-  float2 dA[kBwdWarps][kN][32];          // per lane partial dA of both rows
-  float4 A[kBwdWarps][kN];               // (A'_r0, A'_r1, A_r0, A_r1), A' = A log2(e)
-  float2 car[kBwdWarps][kN];             // adjoint carry entering the chunk from the right
+  T tile[2][2][kN][kCh];          // B / C of two chunks, activation dtype
+  float4 red[2][W][2][kCh / 4];   // dB / dC of one state (row-pair sums), two states in flight
+  float4 pv[W][8][32];            // per lane: (sigma'(v) u, sigma'(v)) of both rows, 8 tokens
+  float2 dA[W][kN][32];           // per lane partial dA of both rows
+  float4 A[W][kN];                // (A'_r0, A'_r1, A_r0, A_r1), A' = A log2(e)
+  float2 car[W][kN];              // adjoint carry entering the chunk from the right
   uint64_t bar[2];
 };
 
 // Issue (thread 0) the TMA row copies of chunk c's B / C into tile[buf]:
 // 32 rows of ntok elements. The caller zero-filled the tail of a short chunk.
-template <typename T>
-__device__ __forceinline__ void issue_tile(Bwd16Smem<T>& sm, int buf, const T* __restrict__ Bm,
+template <typename T, int W>
+__device__ __forceinline__ void issue_tile(Bwd16Smem<T, W>& sm, int buf, const T* __restrict__ Bm,
                                            const T* __restrict__ Cm, int b, int L, int c) {
   const int ntok = min(kCh, L - c * kCh);
   const unsigned bytes = static_cast<unsigned>(ntok) * sizeof(T);  // multiple of 16: L % 8 == 0
@@ -107,10 +108,11 @@ __device__ __forceinline__ void st8(T* p, const float v[8]) {
 
 // VG: the gradient buffers (dout, du, ddelta, dz, dB, dC) allow 16-byte
 // vector access.
-template <typename T, bool VG>
-__global__ void __launch_bounds__(kBwdWarps * 32, 2) scan16_bwd_kernel(const ScanArgs p) {
+template <typename T, bool VG, int W>
+__global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_kernel(const ScanArgs p) {
+  constexpr int kBwdWarps = W, kBwdRows = 2 * W;
   extern __shared__ float4 smem_dyn[];
-  Bwd16Smem<T>& sm = *reinterpret_cast<Bwd16Smem<T>*>(smem_dyn);
+  Bwd16Smem<T, W>& sm = *reinterpret_cast<Bwd16Smem<T, W>*>(smem_dyn);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
   const int d0 = blockIdx.x * kBwdRows + 2 * warp;  // rows d0, d0 + 1 (a row pair)
@@ -169,7 +171,12 @@ __global__ void __launch_bounds__(kBwdWarps * 32, 2) scan16_bwd_kernel(const Sca
     const int buf = c & 1;
     // chunk c is the (k_use >> 1)-th use of buffer buf (buffers alternate)
     const bool ok = mbar_wait_bounded(&sm.bar[buf], (k_use >> 1) & 1, p.status);
-    if (!__syncthreads_and(ok)) break;
+    if (!__syncthreads_and(ok)) {
+      // the copy into buf has not arrived: wait for it once more (bounded)
+      // so that it does not land after the CTA has exited, then stop
+      if (threadIdx.x == 0) mbar_wait_bounded(&sm.bar[buf], (k_use >> 1) & 1, nullptr);
+      break;
+    }
     if (threadIdx.x == 0 && c >= 1) issue_tile(sm, buf ^ 1, Bm, Cm, b, L, c - 1);
 
     const int tl = c * kCh + 8 * lane;
@@ -461,25 +468,37 @@ __global__ void bwd16_param_reduce_kernel(const float* __restrict__ pA, const fl
   }
 }
 
-template <typename T, bool VG>
+template <typename T, bool VG, int W>
 cudaError_t bwd16_t(const ScanArgs& a, cudaStream_t s) {
   static std::atomic<unsigned long long> done{0};
-  const int smem = (int)sizeof(Bwd16Smem<T>);
-  cudaError_t e = smem_attr(scan16_bwd_kernel<T, VG>, smem, &done);
+  const int smem = (int)sizeof(Bwd16Smem<T, W>);
+  cudaError_t e = smem_attr(scan16_bwd_kernel<T, VG, W>, smem, &done);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.D + kBwdRows - 1) / kBwdRows, a.B);
-  scan16_bwd_kernel<T, VG><<<grid, kBwdWarps * 32, smem, s>>>(a);
+  dim3 grid((a.D + 2 * W - 1) / (2 * W), a.B);
+  scan16_bwd_kernel<T, VG, W><<<grid, W * 32, smem, s>>>(a);
   const int m = a.D * kN;
   bwd16_param_reduce_kernel<<<(m + 255) / 256, 256, 0, s>>>(a.part_dA, a.part_dD, a.part_ddb, a.dA,
                                                            a.dD, a.ddelta_bias, a.B, a.D);
   return cudaGetLastError();
 }
 
+template <int W>
+cudaError_t bwd16_dispatch(const ScanArgs& a, cudaStream_t s) {
+  if (a.bf16)
+    return a.vec ? bwd16_t<__nv_bfloat16, true, W>(a, s) : bwd16_t<__nv_bfloat16, false, W>(a, s);
+  return a.vec ? bwd16_t<float, true, W>(a, s) : bwd16_t<float, false, W>(a, s);
+}
+
 }  // namespace
 
+int scan16_bwd_rows(const ScanArgs& a) {
+  return s16::pick_shape(a.B, a.D, 2 * kBwdWarpsSmall, 2, 2 * kBwdWarpsBig) ? 2 * kBwdWarpsBig
+                                                                            : 2 * kBwdWarpsSmall;
+}
+
 cudaError_t launch_scan16_bwd(const ScanArgs& a, cudaStream_t s) {
-  if (a.bf16) return a.vec ? bwd16_t<__nv_bfloat16, true>(a, s) : bwd16_t<__nv_bfloat16, false>(a, s);
-  return a.vec ? bwd16_t<float, true>(a, s) : bwd16_t<float, false>(a, s);
+  return scan16_bwd_rows(a) == 2 * kBwdWarpsBig ? bwd16_dispatch<kBwdWarpsBig>(a, s)
+                                                : bwd16_dispatch<kBwdWarpsSmall>(a, s);
 }
 
 }  // namespace ssm

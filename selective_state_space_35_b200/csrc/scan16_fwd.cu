@@ -30,19 +30,21 @@ namespace ssm {
 namespace {
 using namespace s16;
 
-constexpr int kFwdWarps = 4;
-constexpr int kFwdRows = 2 * kFwdWarps;
+// CTA shapes (warps = row pairs): 4 warps, three CTAs per SM, or 11 warps,
+// one per SM (see pick_shape).
+constexpr int kFwdWarpsSmall = 4, kFwdWarpsBig = 11;
 constexpr unsigned kTileBytes = kFwdTileF4 * 16u;
 #ifndef SSM_FWD16_STATES
 #define SSM_FWD16_STATES 1
 #endif
 constexpr int kFwdS = SSM_FWD16_STATES;  // states per iteration of the state loop
 
+template <int W>
 struct Fwd16Smem {
   float4 tile[2][kFwdTileF4];  // packed B / C of two chunks
   uint64_t bar[2];             // TMA completion, one phase per use of a buffer
-  float H[kFwdRows][kN];       // state entering the current chunk
-  float2 A[kFwdRows][kN];      // (A log2(e), A log2(e)): an f32x2 operand as loaded
+  float H[2 * W][kN];          // state entering the current chunk
+  float2 A[2 * W][kN];         // (A log2(e), A log2(e)): an f32x2 operand as loaded
 };
 
 template <typename T>
@@ -78,10 +80,11 @@ __device__ __forceinline__ void load8(const T* p, bool ok, float v[8]) {
 // here with exactly the separate conv kernel's operations (four fmaf taps in
 // order, document masks, the SFU sigmoid, rounding to T), stored, and scanned.
 // XVEC: x is 16-byte aligned (vector loads).
-template <typename T, bool CONV, bool XVEC>
-__global__ void __launch_bounds__(kFwdWarps * 32, 3) scan16_fwd_kernel(const ScanArgs p) {
+template <typename T, bool CONV, bool XVEC, int W>
+__global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const ScanArgs p) {
+  constexpr int kFwdRows = 2 * W;
   extern __shared__ float4 smem_dyn[];
-  Fwd16Smem& sm = *reinterpret_cast<Fwd16Smem*>(smem_dyn);
+  Fwd16Smem<W>& sm = *reinterpret_cast<Fwd16Smem<W>*>(smem_dyn);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hf = lane >> 4, jj = lane & 15;
   const int r = 2 * warp + hf;  // row of the CTA
@@ -132,7 +135,12 @@ __global__ void __launch_bounds__(kFwdWarps * 32, 3) scan16_fwd_kernel(const Sca
     const bool ok = mbar_wait_bounded(&sm.bar[buf], (c >> 1) & 1, p.status);
     // also: every thread is done with chunk c - 1, whose buffer is refilled
     // next; all threads leave together on a timeout
-    if (!__syncthreads_and(ok)) break;
+    if (!__syncthreads_and(ok)) {
+      // the copy into buf has not arrived: wait for it once more (bounded)
+      // so that it does not land after the CTA has exited, then stop
+      if (threadIdx.x == 0) mbar_wait_bounded(&sm.bar[buf], (c >> 1) & 1, nullptr);
+      break;
+    }
     if (threadIdx.x == 0 && c + 1 < nch) {
       fence_proxy_async_smem();
       mbar_expect_tx(&sm.bar[buf ^ 1], kTileBytes);
@@ -343,30 +351,38 @@ __global__ void __launch_bounds__(kFwdWarps * 32, 3) scan16_fwd_kernel(const Sca
 }
 
 
-template <typename T, bool CONV, bool XVEC>
+template <typename T, bool CONV, bool XVEC, int W>
 cudaError_t fwd16_t(const ScanArgs& a, cudaStream_t s) {
   static std::atomic<unsigned long long> done{0};
-  const int smem = (int)sizeof(Fwd16Smem);
-  cudaError_t e = smem_attr(scan16_fwd_kernel<T, CONV, XVEC>, smem, &done);
+  const int smem = (int)sizeof(Fwd16Smem<W>);
+  cudaError_t e = smem_attr(scan16_fwd_kernel<T, CONV, XVEC, W>, smem, &done);
   if (e != cudaSuccess) return e;
   const int n4 = a.nchunks * kFwdTileF4;
   pack_bc_fwd_kernel<T><<<dim3((n4 + 255) / 256, a.B), 256, 0, s>>>(
       static_cast<const T*>(a.Bm), static_cast<const T*>(a.Cm), a.bcpack, a.L, a.nchunks);
-  dim3 grid((a.D + kFwdRows - 1) / kFwdRows, a.B);
-  scan16_fwd_kernel<T, CONV, XVEC><<<grid, kFwdWarps * 32, smem, s>>>(a);
+  dim3 grid((a.D + 2 * W - 1) / (2 * W), a.B);
+  scan16_fwd_kernel<T, CONV, XVEC, W><<<grid, W * 32, smem, s>>>(a);
   return cudaGetLastError();
+}
+
+template <int W>
+cudaError_t fwd16_dispatch(const ScanArgs& a, cudaStream_t s) {
+  const bool xvec = a.xconv && (reinterpret_cast<uintptr_t>(a.xconv) % 16 == 0);
+  if (a.bf16) {
+    if (!a.xconv) return fwd16_t<__nv_bfloat16, false, true, W>(a, s);
+    return xvec ? fwd16_t<__nv_bfloat16, true, true, W>(a, s)
+                : fwd16_t<__nv_bfloat16, true, false, W>(a, s);
+  }
+  if (!a.xconv) return fwd16_t<float, false, true, W>(a, s);
+  return xvec ? fwd16_t<float, true, true, W>(a, s) : fwd16_t<float, true, false, W>(a, s);
 }
 
 }  // namespace
 
 cudaError_t launch_scan16_fwd(const ScanArgs& a, cudaStream_t s) {
-  const bool xvec = a.xconv && (reinterpret_cast<uintptr_t>(a.xconv) % 16 == 0);
-  if (a.bf16) {
-    if (!a.xconv) return fwd16_t<__nv_bfloat16, false, true>(a, s);
-    return xvec ? fwd16_t<__nv_bfloat16, true, true>(a, s) : fwd16_t<__nv_bfloat16, true, false>(a, s);
-  }
-  if (!a.xconv) return fwd16_t<float, false, true>(a, s);
-  return xvec ? fwd16_t<float, true, true>(a, s) : fwd16_t<float, true, false>(a, s);
+  return s16::pick_shape(a.B, a.D, 2 * kFwdWarpsSmall, 3, 2 * kFwdWarpsBig)
+             ? fwd16_dispatch<kFwdWarpsBig>(a, s)
+             : fwd16_dispatch<kFwdWarpsSmall>(a, s);
 }
 
 }  // namespace ssm

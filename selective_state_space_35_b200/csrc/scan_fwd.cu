@@ -233,8 +233,13 @@ scan_fwd_kernel(const ScanArgs p) {
     if (ASYNC) {
       // chunk c is the (c - c_begin)-th phase of the barrier
       const bool ok = mbar_wait_bounded(&sm.bar, (c - c_begin) & 1, p.status);
-      // also: every thread is done with chunk c - 1's tiles; all leave together on a timeout
-      if (!__syncthreads_and(ok)) break;
+      // also: every thread is done with chunk c - 1's tiles; all leave together on a timeout,
+      // after one more bounded wait for the copy that has not arrived (so that it does
+      // not land after the CTA has exited)
+      if (!__syncthreads_and(ok)) {
+        if (threadIdx.x == 0) mbar_wait_bounded(&sm.bar, (c - c_begin) & 1, nullptr);
+        break;
+      }
       convert_bc_pairs(&sm.raw[0][0][0], sm.B, sm.C, mats, N, L - t0);
       __syncthreads();  // tiles complete; raw free again
       if (threadIdx.x < 32 && c + 1 < c_end)  // next chunk, hidden behind this chunk's work

@@ -22,6 +22,24 @@ def max_abs(got, want) -> float:
     return float(np.max(np.abs(np.asarray(got, np.float64) - np.asarray(want, np.float64))))
 
 
+def bf16_out_max_abs_ok(got, want, tol) -> tuple[bool, float]:
+    """The max-abs bound on a bf16 output against the oracle rounded to bf16.
+
+    Both sides round to bf16, so where the exact value sits near a rounding
+    boundary they can land one bf16 step apart; for |y| >= 4 that step
+    (2^-5) already exceeds a bound of 2e-2. So: |got - want| <= tol where
+    |want| < 4, and at most one bf16 step of `want` elsewhere. Returns
+    (ok, worst error in units of the allowed bound)."""
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    err = np.abs(got - want)
+    aw = np.abs(want)
+    step = np.exp2(np.floor(np.log2(np.maximum(aw, 1e-30))) - 7)
+    allowed = np.where(aw < 4.0, tol, np.maximum(tol, step))
+    worst = float(np.max(err / allowed))
+    return worst <= 1.0, worst
+
+
 def to_dev(t: synth.Tensor, device):
     import torch
     if t.bits is not None:

@@ -11,8 +11,8 @@ import pytest
 
 import oracle
 import synth
-from pipeline import (TOL_BF16_OUT, TOL_BF16_OUT_MAX, TOL_F32, TOL_GRAD, device_inputs, gpu_layer,
-                      host64, max_abs, rel_l2)
+from pipeline import (TOL_BF16_OUT, TOL_BF16_OUT_MAX, TOL_F32, TOL_GRAD, bf16_out_max_abs_ok,
+                      device_inputs, gpu_layer, host64, max_abs, rel_l2)
 
 pytestmark = pytest.mark.gpu
 
@@ -271,95 +271,76 @@ def test_output_red_zones_untouched():
 
 # ---------------------------------------------------------------------------
 # Full-size workloads: the GPU runs the whole layer in the benchmark's launch
-# configuration; the oracle computes sampled rows exactly (rows are
-# independent), dC on a prefix (it depends only on earlier tokens) and dB on
-# a suffix (it depends only on later tokens).
+# configuration (at B = 2, D = 1536 one 22-row CTA per SM; at B = 4, D = 5120
+# 12-row CTAs, two per SM); the oracle recomputes every channel of each batch
+# row in fp64 and every output and gradient is compared over the whole row:
+# all CTAs, every channel position within a CTA and a row pair, and dB / dC
+# (sums over all channels) at every token.
 # ---------------------------------------------------------------------------
-def _row_inputs(inp, b, d, t0=0, t1=None):
-    t1 = inp.shape.L if t1 is None else t1
-    sl = np.s_[b:b + 1, d:d + 1, t0:t1]
-    seq = None if inp.seq_idx is None else np.ascontiguousarray(inp.seq_idx[b:b + 1, t0:t1])
-    return sl, seq
+def _nthreads():
+    import os
+    try:
+        return max(1, len(os.sched_getaffinity(0)))
+    except Exception:
+        return os.cpu_count() or 1
 
 
 @pytest.mark.parametrize("cfg", [3, 4, 5])
-def test_full_size_sampled(cfg):
+def test_full_size_all_channels(cfg):
     torch = _torch()
     sh = synth.CONFIGS[cfg]
     inp = synth.make_inputs(sh, synth.seed_for(cfg))
     res = gpu_layer(device_inputs(inp))
     torch.cuda.synchronize()
-    rng = np.random.Generator(np.random.PCG64(cfg))
-    ds = sorted(set(int(v) for v in rng.integers(0, sh.D, size=2)) | {sh.D - 1})
-    L = sh.L
-
-    def h(k, sl):  # copy only the sampled slice to the host
-        return host64(res[k][sl])
-
-    for d in ds:
-        dA = np.zeros(sh.N)
-        dD = ddb = 0.0
-        dw = np.zeros(4)
-        db = 0.0
-        for b in range(sh.B):
-            sl, seq = _row_inputs(inp, b, d)
-            x = inp.x.f64[sl]
-            w = inp.conv_w[d:d + 1]
-            cb = inp.conv_b[d:d + 1]
-            _, u = oracle.conv1d_fwd(x, w, cb, seq)
-            u_s = oracle.round_bf16(u)
-            assert rel_l2(h("u", sl), u_s) <= TOL_BF16_OUT
-            kw = dict(z=inp.z.f64[sl], Dskip=inp.Dskip[d:d + 1], delta_bias=inp.delta_bias[d:d + 1],
-                      seq_idx=seq)
-            Bm = inp.Bm.f64[b:b + 1]
-            Cm = inp.Cm.f64[b:b + 1]
-            f = oracle.scan_fwd(u_s, inp.delta.f64[sl], inp.A[d:d + 1], Bm, Cm, **kw)
-            o = h("out", sl)
-            assert rel_l2(o, oracle.round_bf16(f["out"])) <= TOL_BF16_OUT
-            assert max_abs(o, oracle.round_bf16(f["out"])) <= TOL_BF16_OUT_MAX
-            assert rel_l2(h("final_state", np.s_[b, d]), f["final_state"][0, 0]) <= TOL_BF16_OUT
-            g = oracle.scan_bwd(u_s, inp.delta.f64[sl], inp.A[d:d + 1], Bm, Cm, inp.dout.f64[sl], **kw)
-            for k in ("du", "ddelta", "dz"):
-                assert rel_l2(h(k, sl), oracle.round_bf16(g[k])) <= TOL_GRAD, (k, b, d)
-            dA += g["dA"][0]
-            dD += g["dD"][0]
-            ddb += g["ddelta_bias"][0]
-            dx, dwi, dbi = oracle.conv1d_bwd(x, w, cb, seq, oracle.round_bf16(g["du"]))
-            # dx depends on du, which the GPU rounds to bf16 on its own path
-            assert rel_l2(h("dx", sl), oracle.round_bf16(dx)) <= TOL_GRAD
-            dw += dwi[0]
-            db += dbi[0]
-        assert rel_l2(host64(res["dA"])[d], dA) <= TOL_GRAD
-        assert rel_l2(host64(res["dD"])[d], dD) <= TOL_GRAD
-        assert rel_l2(host64(res["ddelta_bias"])[d], ddb) <= TOL_GRAD
-        assert rel_l2(host64(res["dconv_w"])[d], dw) <= TOL_GRAD
-        assert rel_l2(host64(res["dconv_b"])[d], db) <= TOL_GRAD
-
-    # dC on a prefix of T tokens (all channels, batch row 0)
-    T = 384
-    sl = np.s_[0:1, :, 0:T]
-    seq = None if inp.seq_idx is None else np.ascontiguousarray(inp.seq_idx[0:1, :T])
-    _, u = oracle.conv1d_fwd(inp.x.f64[sl], inp.conv_w, inp.conv_b, seq)
-    u_s = oracle.round_bf16(u)
-    kw = dict(z=inp.z.f64[sl], Dskip=inp.Dskip, delta_bias=inp.delta_bias, seq_idx=seq, nthreads=8)
-    g = oracle.scan_bwd(u_s, inp.delta.f64[sl], inp.A, inp.Bm.f64[0:1, :, :T], inp.Cm.f64[0:1, :, :T],
-                        inp.dout.f64[sl], **kw)
-    assert rel_l2(h("dC", np.s_[0:1, :, :T]), g["dC"]) <= TOL_GRAD
-
-    # dB on a suffix of T tokens (conv needs 3 tokens of history)
-    b = sh.B - 1
-    s0 = L - T
-    slx = np.s_[b:b + 1, :, s0 - 3:L]
-    seqx = None if inp.seq_idx is None else np.ascontiguousarray(inp.seq_idx[b:b + 1, s0 - 3:L])
-    _, u = oracle.conv1d_fwd(inp.x.f64[slx], inp.conv_w, inp.conv_b, seqx)
-    u_s = oracle.round_bf16(u[:, :, 3:])
-    sl = np.s_[b:b + 1, :, s0:L]
-    seq = None if inp.seq_idx is None else np.ascontiguousarray(inp.seq_idx[b:b + 1, s0:L])
-    kw = dict(z=inp.z.f64[sl], Dskip=inp.Dskip, delta_bias=inp.delta_bias, seq_idx=seq, nthreads=8)
-    g = oracle.scan_bwd(u_s, inp.delta.f64[sl], inp.A, inp.Bm.f64[b:b + 1, :, s0:], inp.Cm.f64[b:b + 1, :, s0:],
-                        inp.dout.f64[sl], **kw)
-    assert rel_l2(h("dB", np.s_[b:b + 1, :, s0:]), g["dB"]) <= TOL_GRAD
-    assert rel_l2(h("du", sl), oracle.round_bf16(g["du"])) <= TOL_GRAD
+    nt = _nthreads()
+    acc = {k: 0.0 for k in ("dA", "dD", "ddelta_bias", "dconv_w", "dconv_b")}
+    for b in range(sh.B):
+        sl = np.s_[b:b + 1]
+        seq = None if inp.seq_idx is None else np.ascontiguousarray(inp.seq_idx[sl])
+        x = inp.x.f64[sl]
+        _, u = oracle.conv1d_fwd(x, inp.conv_w, inp.conv_b, seq)
+        u_s = oracle.round_bf16(u)
+        del u
+        kw = dict(z=inp.z.f64[sl], Dskip=inp.Dskip, delta_bias=inp.delta_bias, seq_idx=seq,
+                  nthreads=nt)
+        Bm, Cm = inp.Bm.f64[sl], inp.Cm.f64[sl]
+        f = oracle.scan_fwd(u_s, inp.delta.f64[sl], inp.A, Bm, Cm, **kw)
+        assert rel_l2(host64(res["u"][sl]), u_s) <= TOL_BF16_OUT
+        o, wo = host64(res["out"][sl]), oracle.round_bf16(f["out"])
+        assert rel_l2(o, wo) <= TOL_BF16_OUT, b
+        ok, worst = bf16_out_max_abs_ok(o, wo, TOL_BF16_OUT_MAX)
+        assert ok, (b, worst, max_abs(o, wo))
+        del o, wo
+        assert rel_l2(host64(res["final_state"][sl]), f["final_state"]) <= TOL_BF16_OUT
+        del f
+        g = oracle.scan_bwd(u_s, inp.delta.f64[sl], inp.A, Bm, Cm, inp.dout.f64[sl], **kw)
+        for k in ("du", "ddelta", "dz"):
+            assert rel_l2(host64(res[k][sl]), oracle.round_bf16(g[k])) <= TOL_GRAD, (k, b)
+        for k in ("dB", "dC"):
+            assert rel_l2(host64(res[k][sl]), g[k]) <= TOL_GRAD, (k, b)
+        # a middle window on its own (the sums over all channels)
+        mid = np.s_[b:b + 1, :, sh.L // 2 - 192:sh.L // 2 + 192]
+        for k in ("dB", "dC"):
+            assert rel_l2(host64(res[k][mid]), g[k][(0,) + mid[1:]][None]) <= TOL_GRAD, (k, b)
+        for k in ("dA", "dD", "ddelta_bias"):
+            acc[k] = acc[k] + g[k]
+        dx, dw, db = oracle.conv1d_bwd(x, inp.conv_w, inp.conv_b, seq, oracle.round_bf16(g["du"]))
+        del g
+        # dx depends on du, which the GPU rounds to bf16 on its own path
+        assert rel_l2(host64(res["dx"][sl]), oracle.round_bf16(dx)) <= TOL_GRAD, b
+        acc["dconv_w"] = acc["dconv_w"] + dw
+        acc["dconv_b"] = acc["dconv_b"] + db
+        del dx, u_s
+    for k, w in acc.items():
+        assert rel_l2(host64(res[k]), w) <= TOL_GRAD, k
+        # every channel on its own, against the array's RMS (a channel's sum
+        # over B x L terms of both signs may cancel to far below that scale,
+        # so its own norm is not the yardstick)
+        got = host64(res[k]).reshape(sh.D, -1)
+        want = np.asarray(w).reshape(sh.D, -1)
+        rms = float(np.sqrt(np.mean(want * want)))
+        err = np.sqrt(np.mean((got - want) ** 2, axis=1)) / rms
+        assert float(np.max(err)) <= 2 * TOL_GRAD, (k, int(np.argmax(err)), float(np.max(err)))
 
 
 def test_unaligned_gradient_buffers_take_scalar_path():

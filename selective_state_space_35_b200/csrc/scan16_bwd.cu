@@ -111,6 +111,7 @@ __device__ __forceinline__ void st8(T* p, const float v[8]) {
 template <typename T, bool VG, int W>
 __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_kernel(const ScanArgs p) {
   constexpr int kBwdWarps = W, kBwdRows = 2 * W;
+  static_assert(sizeof(Bwd16Smem<T, W>) <= 227 * 1024, "shared memory per CTA");
   extern __shared__ float4 smem_dyn[];
   Bwd16Smem<T, W>& sm = *reinterpret_cast<Bwd16Smem<T, W>*>(smem_dyn);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -83,6 +83,7 @@ __device__ __forceinline__ void load8(const T* p, bool ok, float v[8]) {
 template <typename T, bool CONV, bool XVEC, int W>
 __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const ScanArgs p) {
   constexpr int kFwdRows = 2 * W;
+  static_assert(sizeof(Fwd16Smem<W>) <= 227 * 1024, "shared memory per CTA");
   extern __shared__ float4 smem_dyn[];
   Fwd16Smem<W>& sm = *reinterpret_cast<Fwd16Smem<W>*>(smem_dyn);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -618,7 +618,8 @@ ssm_status_t ssm_scan_fwd_summary(const ssm_scan_params* p, const int32_t* seq_p
   a.vec = vec_ok(p->L, {p->u, p->delta, p->Bm, a.seq});
   st = summary_prep(p, a, s);
   if (st != SSM_OK) return st;
-  cudaError_t e = ssm::launch_scan_fwd_summary(a, s);
+  // the N = 16 layout where the plan takes it (its packed B / C tiles are in the workspace)
+  cudaError_t e = a.fast16 ? ssm::launch_scan16_fwd_summary(a, s) : ssm::launch_scan_fwd_summary(a, s);
   if (e == cudaSuccess)
     e = ssm::launch_summary_out(a.split_P, a.split_H, a.seq, seq_prev, p->L, decay, state_end,
                                 p->B, p->D, p->N, a.Npad, false, s);
@@ -640,7 +641,8 @@ ssm_status_t ssm_scan_bwd_summary(const ssm_scan_params* p, const void* dout,
   a.vec = vec_ok(p->L, {p->delta, p->z, p->Cm, dout, a.seq});
   st = summary_prep(p, a, s);
   if (st != SSM_OK) return st;
-  cudaError_t e = ssm::launch_scan_bwd_summary(a, s);
+  cudaError_t e = (a.fast16 && aligned(dout, 16)) ? ssm::launch_scan16_bwd_summary(a, s)
+                                                   : ssm::launch_scan_bwd_summary(a, s);
   if (e == cudaSuccess)
     e = ssm::launch_summary_out(a.split_P, a.split_H, a.seq, seq_prev, p->L, decay, adj_start,
                                 p->B, p->D, p->N, a.Npad, true, s);

@@ -190,6 +190,11 @@ inline int pick_shape(int B, int D, int rows_small, int per_sm_small, int rows_b
 
 cudaError_t launch_scan16_fwd(const ScanArgs& a, cudaStream_t s);
 cudaError_t launch_scan16_bwd(const ScanArgs& a, cudaStream_t s);
+// Whole-row summaries of a piece (N = 16 layout): forward (product of the
+// decays, final state from zero) and backward (product of the decays, the
+// adjoint leaving token 0 from the piece's own dout), into split_P / split_H.
+cudaError_t launch_scan16_fwd_summary(const ScanArgs& a, cudaStream_t s);
+cudaError_t launch_scan16_bwd_summary(const ScanArgs& a, cudaStream_t s);
 // Rows per CTA the N = 16 backward uses for these arguments (the row groups
 // of its deterministic dB / dC partials).
 int scan16_bwd_rows(const ScanArgs& a);

@@ -448,6 +448,164 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_kernel(const
 }
 
 
+// ---------------------------------------------------------------------------
+// Whole-row backward summary of a piece (N = 16 layout): per (row, state) the
+// product of the decays and the adjoint leaving token 0 (a_0 g_0) that the
+// piece's own dout produces with no adjoint entering from the right. Only
+// the adjoint map is needed: no recompute of h, no replay, no sums.
+template <typename T, int W>
+struct Bwd16SumSmem {
+  T tileC[2][kN][kCh];  // C of two chunks, activation dtype
+  float4 A[W][kN];      // (A'_r0, A'_r1, -, -), A' = A log2(e)
+  float2 car[W][kN];    // adjoint leaving the chunks done so far
+  float2 dk[W][kN];     // product of their decays
+  uint64_t bar[2];
+};
+
+template <typename T, int W>
+__global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_summary_kernel(const ScanArgs p) {
+  static_assert(sizeof(Bwd16SumSmem<T, W>) <= 227 * 1024, "shared memory per CTA");
+  extern __shared__ float4 smem_dyn[];
+  Bwd16SumSmem<T, W>& sm = *reinterpret_cast<Bwd16SumSmem<T, W>*>(smem_dyn);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  const int d0 = blockIdx.x * (2 * W) + 2 * warp;  // rows d0, d0 + 1
+  const bool act0 = d0 < p.D, act1 = d0 + 1 < p.D;
+  const int L = p.L, nch = p.nchunks;
+  const size_t rid0 = (size_t)b * p.D + (act0 ? d0 : 0);
+  const size_t rid1 = (size_t)b * p.D + (act1 ? d0 + 1 : 0);
+  const size_t row0 = rid0 * L, row1 = rid1 * L;
+  const T* Cm = static_cast<const T*>(p.Cm);
+  const bool has_z = p.z != nullptr;
+  const int32_t* seqb = p.seq ? p.seq + (size_t)b * L : nullptr;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.bar[0], 1);
+    mbar_init(&sm.bar[1], 1);
+    fence_mbar_init();
+  }
+  if (lane < kN) {
+    const int n = lane;
+    const float a0 = act0 ? __ldg(p.A + (size_t)d0 * kN + n) : 0.0f;
+    const float a1 = act1 ? __ldg(p.A + (size_t)(d0 + 1) * kN + n) : 0.0f;
+    sm.A[warp][n] = make_float4(a0 * kLog2e, a1 * kLog2e, 0.0f, 0.0f);
+    sm.car[warp][n] = make_float2(0.0f, 0.0f);
+    sm.dk[warp][n] = make_float2(1.0f, 1.0f);
+  }
+  const int last = nch - 1;
+  const int ntail = L - last * kCh;
+  if (ntail < kCh) {  // a short last chunk: zero the tile tail its copies leave untouched
+    for (int i = threadIdx.x; i < kN * (kCh - ntail); i += blockDim.x) {
+      const int rr = i / (kCh - ntail), t = ntail + i % (kCh - ntail);
+      sm.tileC[last & 1][rr][t] = T(0.0f);
+    }
+  }
+  __syncthreads();
+  auto issue = [&](int buf, int c) {  // thread 0: chunk c's C rows into tileC[buf]
+    const int ntok = min(kCh, L - c * kCh);
+    const unsigned bytes = static_cast<unsigned>(ntok) * sizeof(T);  // multiple of 16: L % 8 == 0
+    fence_proxy_async_smem();
+    mbar_expect_tx(&sm.bar[buf], bytes * kN);
+#pragma unroll 1
+    for (int n = 0; n < kN; ++n)
+      tma_load_1d(&sm.tileC[buf][n][0], Cm + ((size_t)b * kN + n) * L + (size_t)c * kCh, bytes,
+                  &sm.bar[buf]);
+  };
+  if (threadIdx.x == 0) issue(last & 1, last);
+  const float2 bias = make_float2((act0 && p.delta_bias) ? __ldg(p.delta_bias + d0) : 0.0f,
+                                  (act1 && p.delta_bias) ? __ldg(p.delta_bias + d0 + 1) : 0.0f);
+  int k_use = 0;
+#pragma unroll 1
+  for (int c = last; c >= 0; --c, ++k_use) {
+    const int buf = c & 1;
+    const bool ok = mbar_wait_bounded(&sm.bar[buf], (k_use >> 1) & 1, p.status);
+    if (!__syncthreads_and(ok)) {
+      // the copy into buf has not arrived: wait for it once more (bounded), then stop
+      if (threadIdx.x == 0) mbar_wait_bounded(&sm.bar[buf], (k_use >> 1) & 1, nullptr);
+      break;
+    }
+    if (threadIdx.x == 0 && c >= 1) issue(buf ^ 1, c - 1);
+    const int tl = c * kCh + 8 * lane;
+    const bool valid = tl < L;
+    const bool ok0 = valid && act0, ok1 = valid && act1;
+    float2 dd[8], dy[8];
+    {
+      float dl0[8], dl1[8], g0[8], g1[8];
+      ld8<T, true>(static_cast<const T*>(p.delta) + row0 + tl, ok0, dl0);
+      ld8<T, true>(static_cast<const T*>(p.delta) + row1 + tl, ok1, dl1);
+      ld8<T, true>(static_cast<const T*>(p.dout) + row0 + tl, ok0, g0);
+      ld8<T, true>(static_cast<const T*>(p.dout) + row1 + tl, ok1, g1);
+      if (has_z) {
+        float z0[8], z1[8];
+        ld8<T, true>(static_cast<const T*>(p.z) + row0 + tl, ok0, z0);
+        ld8<T, true>(static_cast<const T*>(p.z) + row1 + tl, ok1, z1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          g0[i] *= z0[i] * sigmoid_fast(z0[i]);
+          g1[i] *= z1[i] * sigmoid_fast(z1[i]);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float2 dt = make_float2(dl0[i] + bias.x, dl1[i] + bias.y);
+        if (p.softplus) dt = softplus2(dt);
+        dd[i] = make_float2(ok0 ? dt.x : 0.0f, ok1 ? dt.y : 0.0f);
+        dy[i] = make_float2(g0[i], g1[i]);
+      }
+    }
+    unsigned rm = 0u;
+    if (seqb && valid) {
+      int prev = tl > 0 ? __ldg(seqb + tl - 1) : 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int cur = __ldg(seqb + tl + i);
+        if (tl + i > 0 && cur != prev) rm |= 1u << i;
+        prev = cur;
+      }
+    }
+    const T* tileC = &sm.tileC[buf][0][0];
+#pragma unroll 1
+    for (int n = 0; n < kN; ++n) {
+      const float4 Aq = sm.A[warp][n];
+      const float2 a2 = make_float2(Aq.x, Aq.y);
+      float Ct[8];
+      lds8<T>(tileC + n * kCh, lane, Ct);
+      float2 at[8], gy[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        at[i] = ex2x2(fmul2(dd[i], a2));
+        if ((rm >> i) & 1u) at[i] = make_float2(0.0f, 0.0f);
+        gy[i] = fmul2(dy[i], dup(Ct[i]));
+      }
+      float2 P = fmul2(fmul2(at[0], at[1]), fmul2(at[2], at[3]));
+      P = fmul2(P, fmul2(fmul2(at[4], at[5]), fmul2(at[6], at[7])));
+      float2 G = gy[7];
+#pragma unroll
+      for (int i = 6; i >= 0; --i) G = ffma2(at[i + 1], G, gy[i]);
+      G = fmul2(at[0], G);
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) bwd_step2(P, G, off);
+      if (lane == 0) {  // lane 0 now holds the map of the whole chunk
+        const float2 cin = sm.car[warp][n];
+        sm.car[warp][n] = ffma2(P, cin, G);
+        sm.dk[warp][n] = fmul2(sm.dk[warp][n], P);
+      }
+    }
+  }
+  __syncwarp();
+  if (lane < kN) {
+    const float2 cr = sm.car[warp][lane], dk = sm.dk[warp][lane];
+    if (act0) {
+      p.split_P[rid0 * p.Npad + lane] = dk.x;
+      p.split_H[rid0 * p.Npad + lane] = cr.x;
+    }
+    if (act1) {
+      p.split_P[rid1 * p.Npad + lane] = dk.y;
+      p.split_H[rid1 * p.Npad + lane] = cr.y;
+    }
+  }
+}
+
 __global__ void bwd16_param_reduce_kernel(const float* __restrict__ pA, const float* __restrict__ pD,
                                           const float* __restrict__ pB, float* __restrict__ dA,
                                           float* __restrict__ dD, float* __restrict__ ddb, int B,
@@ -495,6 +653,25 @@ cudaError_t bwd16_dispatch(const ScanArgs& a, cudaStream_t s) {
 int scan16_bwd_rows(const ScanArgs& a) {
   return s16::pick_shape(a.B, a.D, 2 * kBwdWarpsSmall, 2, 2 * kBwdWarpsBig) ? 2 * kBwdWarpsBig
                                                                             : 2 * kBwdWarpsSmall;
+}
+
+template <typename T, int W>
+cudaError_t bwd16_summary_t(const ScanArgs& a, cudaStream_t s) {
+  static std::atomic<unsigned long long> done{0};
+  const int smem = (int)sizeof(Bwd16SumSmem<T, W>);
+  cudaError_t e = smem_attr(scan16_bwd_summary_kernel<T, W>, smem, &done);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.D + 2 * W - 1) / (2 * W), a.B);
+  scan16_bwd_summary_kernel<T, W><<<grid, W * 32, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scan16_bwd_summary(const ScanArgs& a, cudaStream_t s) {
+  const bool big = scan16_bwd_rows(a) == 2 * kBwdWarpsBig;
+  if (a.bf16)
+    return big ? bwd16_summary_t<__nv_bfloat16, kBwdWarpsBig>(a, s)
+               : bwd16_summary_t<__nv_bfloat16, kBwdWarpsSmall>(a, s);
+  return big ? bwd16_summary_t<float, kBwdWarpsBig>(a, s) : bwd16_summary_t<float, kBwdWarpsSmall>(a, s);
 }
 
 cudaError_t launch_scan16_bwd(const ScanArgs& a, cudaStream_t s) {

@@ -44,6 +44,7 @@ struct Fwd16Smem {
   float4 tile[2][kFwdTileF4];  // packed B / C of two chunks
   uint64_t bar[2];             // TMA completion, one phase per use of a buffer
   float H[2 * W][kN];          // state entering the current chunk
+  float Dk[2 * W][kN];         // summary: product of the decays so far
   float2 A[2 * W][kN];         // (A log2(e), A log2(e)): an f32x2 operand as loaded
 };
 
@@ -80,8 +81,12 @@ __device__ __forceinline__ void load8(const T* p, bool ok, float v[8]) {
 // here with exactly the separate conv kernel's operations (four fmaf taps in
 // order, document masks, the SFU sigmoid, rounding to T), stored, and scanned.
 // XVEC: x is 16-byte aligned (vector loads).
-template <typename T, bool CONV, bool XVEC, int W>
+// SUM: the whole-row summary of a piece of a longer sequence instead (the
+// product of the decays and the final state from a zero state, into
+// split_P / split_H): no y, no checkpoints, no replay.
+template <typename T, bool CONV, bool XVEC, int W, bool SUM>
 __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const ScanArgs p) {
+  static_assert(!(SUM && CONV), "the summary reads u");
   constexpr int kFwdRows = 2 * W;
   static_assert(sizeof(Fwd16Smem<W>) <= 227 * 1024, "shared memory per CTA");
   extern __shared__ float4 smem_dyn[];
@@ -97,7 +102,7 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
   const size_t row = rowid * L;
   const T* u_in = static_cast<const T*>(CONV ? p.xconv : p.u) + row;
   const T* dl_in = static_cast<const T*>(p.delta) + row;
-  const T* z_in = p.z ? static_cast<const T*>(p.z) + row : nullptr;
+  const T* z_in = (p.z && !SUM) ? static_cast<const T*>(p.z) + row : nullptr;
   T* u_out = CONV ? static_cast<T*>(const_cast<void*>(p.u)) + row : nullptr;
   T* out = static_cast<T*>(p.out) + row;
   T* ysv = p.z ? static_cast<T*>(p.ysave) + row : nullptr;
@@ -115,7 +120,8 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
     const bool act = dd < p.D;
     const float a = act ? __ldg(p.A + (size_t)dd * kN + n) * kLog2e : 0.0f;
     sm.A[rr][n] = make_float2(a, a);
-    sm.H[rr][n] = (act && p.h0) ? __ldg(p.h0 + ((size_t)b * p.D + dd) * kN + n) : 0.0f;
+    sm.H[rr][n] = (act && p.h0 && !SUM) ? __ldg(p.h0 + ((size_t)b * p.D + dd) * kN + n) : 0.0f;
+    sm.Dk[rr][n] = 1.0f;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -286,20 +292,26 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
         const float end = fmaf(Pl[s], cin[s], Hl[s]);
         float start = __shfl_up_sync(kFull, end, 1, 16);
         if (jj == 0) start = cin[s];
-        if (jj == 15) sm.H[r][n] = end;
+        if (jj == 15) {
+          sm.H[r][n] = end;
+          if constexpr (SUM) sm.Dk[r][n] *= Pl[s];  // the scan left the 16 lanes' product here
+        }
+        if constexpr (SUM) continue;
         const float sb = fmaf(P[s].x, start, H[s].x);  // state entering sub-segment b
         if (va) *reinterpret_cast<float2*>(ckc + n * 2 * kSegs) = make_float2(start, sb);
         h[s] = make_float2(start, sb);
       }
+      if constexpr (!SUM) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < 4; ++k) {
 #pragma unroll
-        for (int s = 0; s < kFwdS; ++s) {
-          const float4 q = tile[(kN + n0 + s) * 64 + jj + 16 * k];
-          h[s] = ffma2(a[s][2 * k], h[s], bx[s][2 * k]);
-          y2[2 * k] = ffma2(make_float2(q.x, q.y), h[s], y2[2 * k]);
-          h[s] = ffma2(a[s][2 * k + 1], h[s], bx[s][2 * k + 1]);
-          y2[2 * k + 1] = ffma2(make_float2(q.z, q.w), h[s], y2[2 * k + 1]);
+          for (int s = 0; s < kFwdS; ++s) {
+            const float4 q = tile[(kN + n0 + s) * 64 + jj + 16 * k];
+            h[s] = ffma2(a[s][2 * k], h[s], bx[s][2 * k]);
+            y2[2 * k] = ffma2(make_float2(q.x, q.y), h[s], y2[2 * k]);
+            h[s] = ffma2(a[s][2 * k + 1], h[s], bx[s][2 * k + 1]);
+            y2[2 * k + 1] = ffma2(make_float2(q.z, q.w), h[s], y2[2 * k + 1]);
+          }
         }
       }
     }
@@ -307,7 +319,7 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
     if (any_reset) states(std::true_type{});
     else states(std::false_type{});
 
-    if (va || vb) {
+    if (!SUM && (va || vb)) {
       const bool vo = (reinterpret_cast<uintptr_t>(p.out) & 15) == 0;  // else element stores
       auto put = [&](T* q, const float v[8]) {
         if (vo) {
@@ -348,21 +360,28 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
   }
 
   __syncwarp();
-  if (active && p.final_state) p.final_state[rowid * kN + jj] = sm.H[r][jj];
+  if constexpr (SUM) {
+    if (active) {
+      p.split_P[rowid * p.Npad + jj] = sm.Dk[r][jj];
+      p.split_H[rowid * p.Npad + jj] = sm.H[r][jj];
+    }
+  } else if (active && p.final_state) {
+    p.final_state[rowid * kN + jj] = sm.H[r][jj];
+  }
 }
 
 
-template <typename T, bool CONV, bool XVEC, int W>
+template <typename T, bool CONV, bool XVEC, int W, bool SUM = false>
 cudaError_t fwd16_t(const ScanArgs& a, cudaStream_t s) {
   static std::atomic<unsigned long long> done{0};
   const int smem = (int)sizeof(Fwd16Smem<W>);
-  cudaError_t e = smem_attr(scan16_fwd_kernel<T, CONV, XVEC, W>, smem, &done);
+  cudaError_t e = smem_attr(scan16_fwd_kernel<T, CONV, XVEC, W, SUM>, smem, &done);
   if (e != cudaSuccess) return e;
   const int n4 = a.nchunks * kFwdTileF4;
   pack_bc_fwd_kernel<T><<<dim3((n4 + 255) / 256, a.B), 256, 0, s>>>(
       static_cast<const T*>(a.Bm), static_cast<const T*>(a.Cm), a.bcpack, a.L, a.nchunks);
   dim3 grid((a.D + 2 * W - 1) / (2 * W), a.B);
-  scan16_fwd_kernel<T, CONV, XVEC, W><<<grid, W * 32, smem, s>>>(a);
+  scan16_fwd_kernel<T, CONV, XVEC, W, SUM><<<grid, W * 32, smem, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -384,6 +403,15 @@ cudaError_t launch_scan16_fwd(const ScanArgs& a, cudaStream_t s) {
   return s16::pick_shape(a.B, a.D, 2 * kFwdWarpsSmall, 3, 2 * kFwdWarpsBig)
              ? fwd16_dispatch<kFwdWarpsBig>(a, s)
              : fwd16_dispatch<kFwdWarpsSmall>(a, s);
+}
+
+cudaError_t launch_scan16_fwd_summary(const ScanArgs& a, cudaStream_t s) {
+  const bool big = s16::pick_shape(a.B, a.D, 2 * kFwdWarpsSmall, 3, 2 * kFwdWarpsBig);
+  if (a.bf16)
+    return big ? fwd16_t<__nv_bfloat16, false, true, kFwdWarpsBig, true>(a, s)
+               : fwd16_t<__nv_bfloat16, false, true, kFwdWarpsSmall, true>(a, s);
+  return big ? fwd16_t<float, false, true, kFwdWarpsBig, true>(a, s)
+             : fwd16_t<float, false, true, kFwdWarpsSmall, true>(a, s);
 }
 
 }  // namespace ssm

@@ -70,7 +70,8 @@ def device_inputs(inp: synth.LayerInputs, device="cuda"):
     return d
 
 
-def gpu_layer(dv, *, n_splits=0, use_z=True, use_seq=True, softplus=True, final_state=True):
+def gpu_layer(dv, *, n_splits=0, use_z=True, use_seq=True, softplus=True, final_state=True,
+              deterministic=False):
     """conv fwd -> scan fwd -> scan bwd -> conv bwd on device tensors `dv`."""
     import selective_state_space_35_b200 as ssm
     seq = dv["seq_idx"] if use_seq else None
@@ -83,7 +84,7 @@ def gpu_layer(dv, *, n_splits=0, use_z=True, use_seq=True, softplus=True, final_
     assert ssm.scan_status(u, dv["A"], ws) == 0
     g = ssm.scan_bwd(u, dv["delta"], dv["A"], dv["Bm"], dv["Cm"], dv["dout"], ws, z=z,
                      Dskip=dv["Dskip"], delta_bias=dv["delta_bias"], softplus=softplus,
-                     seq_idx=seq, n_splits=n_splits)
+                     seq_idx=seq, n_splits=n_splits, deterministic=deterministic)
     dx, dw, dcb = ssm.conv1d_bwd(dv["x"], dv["conv_w"], dv["conv_b"], seq, g["du"])
     res = {"u": u, "out": out, "final_state": fs, "dx": dx, "dconv_w": dw, "dconv_b": dcb}
     res.update(g)

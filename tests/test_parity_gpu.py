@@ -198,14 +198,18 @@ def test_cu_seqlens_equals_seq_idx():
         assert rel_l2(host64(g2[k]), host64(g1[k])) <= 1e-6, k
 
 
-def test_run_twice_bitwise():
+@pytest.mark.parametrize("n_splits", [0, 1])
+def test_run_twice_bitwise(n_splits):
+    """Two runs give the same bits in every output and gradient, dB and dC
+    included with the deterministic backward (n_splits=1: the N = 16
+    kernels; 0: the automatic choice, L split in two at this size)."""
     torch = _torch()
     inp = _small(2, 9, 16, 1200, 5, dtype="bf16", nbound=3)
     dv = device_inputs(inp)
-    r1 = gpu_layer(dv)
-    r2 = gpu_layer(dv)
-    for k in ("u", "out", "final_state", "du", "ddelta", "dz", "dA", "dD", "ddelta_bias", "dx",
-              "dconv_w", "dconv_b"):
+    r1 = gpu_layer(dv, n_splits=n_splits, deterministic=True)
+    r2 = gpu_layer(dv, n_splits=n_splits, deterministic=True)
+    for k in ("u", "out", "final_state", "du", "ddelta", "dz", "dA", "dB", "dC", "dD",
+              "ddelta_bias", "dx", "dconv_w", "dconv_b"):
         assert torch.equal(r1[k], r2[k]), k
 
 

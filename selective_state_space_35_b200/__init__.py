@@ -395,9 +395,10 @@ def decode_step(x, conv_state, conv_w, delta, A, Bm, Cm, state, *, conv_bias=Non
 
 
 def scan_fwd_summary(u, delta, A, Bm, *, delta_bias=None, softplus=True, seq_idx=None,
-                     seq_prev=None, zoh=False, workspace=None, stream=None):
+                     seq_prev=None, zoh=False, workspace=None, n_splits=0, stream=None):
     """Summary of this piece of a longer sequence: (decay, state_end), each
     [B, D, N] fp32, with final state = decay * (state entering) + state_end.
+    n_splits as in scan_fwd (1 selects the N = 16 kernels where they apply).
     seq_prev [B] int32: document id of the token before token 0."""
     torch = _torch()
     B, D, L = u.shape
@@ -405,7 +406,7 @@ def scan_fwd_summary(u, delta, A, Bm, *, delta_bias=None, softplus=True, seq_idx
     _need(seq_prev, "seq_prev", torch.int32, (B,))
     # the forward summary reads no C: Bm fills that slot of the parameter block
     p = scan_params(u, delta, A, Bm, Bm, delta_bias=delta_bias, softplus=softplus,
-                    seq_idx=seq_idx, zoh=zoh)
+                    seq_idx=seq_idx, zoh=zoh, n_splits=n_splits)
     need = ssm_scan_workspace_size(p)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=u.device)
@@ -418,7 +419,7 @@ def scan_fwd_summary(u, delta, A, Bm, *, delta_bias=None, softplus=True, seq_idx
 
 
 def scan_bwd_summary(delta, A, Cm, dout, *, z=None, delta_bias=None, softplus=True,
-                     seq_idx=None, seq_prev=None, workspace=None, stream=None):
+                     seq_idx=None, seq_prev=None, workspace=None, n_splits=0, stream=None):
     """Backward summary of this piece from dout alone: (decay, adj_start),
     each [B, D, N] fp32; the gradient leaving the piece through its start is
     decay * (gradient of its final state) + adj_start."""
@@ -429,7 +430,7 @@ def scan_bwd_summary(delta, A, Cm, dout, *, z=None, delta_bias=None, softplus=Tr
     _need(seq_prev, "seq_prev", torch.int32, (B,))
     # the backward summary reads no u and no B: delta and Cm fill those slots
     p = scan_params(delta, delta, A, Cm, Cm, z=z, delta_bias=delta_bias, softplus=softplus,
-                    seq_idx=seq_idx)
+                    seq_idx=seq_idx, n_splits=n_splits)
     need = ssm_scan_workspace_size(p)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=delta.device)

@@ -458,7 +458,6 @@ struct Bwd16SumSmem {
   T tileC[2][kN][kCh];  // C of two chunks, activation dtype
   float4 A[W][kN];      // (A'_r0, A'_r1, -, -), A' = A log2(e)
   float2 car[W][kN];    // adjoint leaving the chunks done so far
-  float2 dk[W][kN];     // product of their decays
   uint64_t bar[2];
 };
 
@@ -490,7 +489,6 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_summary_kern
     const float a1 = act1 ? __ldg(p.A + (size_t)(d0 + 1) * kN + n) : 0.0f;
     sm.A[warp][n] = make_float4(a0 * kLog2e, a1 * kLog2e, 0.0f, 0.0f);
     sm.car[warp][n] = make_float2(0.0f, 0.0f);
-    sm.dk[warp][n] = make_float2(1.0f, 1.0f);
   }
   const int last = nch - 1;
   const int ntail = L - last * kCh;
@@ -515,6 +513,10 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_summary_kern
   const float2 bias = make_float2((act0 && p.delta_bias) ? __ldg(p.delta_bias + d0) : 0.0f,
                                   (act1 && p.delta_bias) ? __ldg(p.delta_bias + d0 + 1) : 0.0f);
   int k_use = 0;
+  // the lane's sums of dt (both rows) and whether a document starts after
+  // token 0: the decay of the piece is exp(A sum dt), or 0 across a start
+  float2 dt_sum = make_float2(0.0f, 0.0f);
+  bool any_start = false;
 #pragma unroll 1
   for (int c = last; c >= 0; --c, ++k_use) {
     const int buf = c & 1;
@@ -551,6 +553,7 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_summary_kern
         if (p.softplus) dt = softplus2(dt);
         dd[i] = make_float2(ok0 ? dt.x : 0.0f, ok1 ? dt.y : 0.0f);
         dy[i] = make_float2(g0[i], g1[i]);
+        dt_sum = fadd2(dt_sum, dd[i]);
       }
     }
     unsigned rm = 0u;
@@ -563,6 +566,7 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_summary_kern
         prev = cur;
       }
     }
+    any_start = any_start || rm != 0u;
     const T* tileC = &sm.tileC[buf][0][0];
 #pragma unroll 1
     for (int n = 0; n < kN; ++n) {
@@ -588,13 +592,21 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_summary_kern
       if (lane == 0) {  // lane 0 now holds the map of the whole chunk
         const float2 cin = sm.car[warp][n];
         sm.car[warp][n] = ffma2(P, cin, G);
-        sm.dk[warp][n] = fmul2(sm.dk[warp][n], P);
       }
     }
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    dt_sum.x += __shfl_xor_sync(kFull, dt_sum.x, off);
+    dt_sum.y += __shfl_xor_sync(kFull, dt_sum.y, off);
+  }
+  any_start = __any_sync(kFull, any_start);
   __syncwarp();
   if (lane < kN) {
-    const float2 cr = sm.car[warp][lane], dk = sm.dk[warp][lane];
+    const float4 Aq = sm.A[warp][lane];
+    const float2 cr = sm.car[warp][lane];
+    const float2 dk = any_start ? make_float2(0.0f, 0.0f)
+                                : make_float2(ex2_approx(Aq.x * dt_sum.x), ex2_approx(Aq.y * dt_sum.y));
     if (act0) {
       p.split_P[rid0 * p.Npad + lane] = dk.x;
       p.split_H[rid0 * p.Npad + lane] = cr.x;

@@ -44,7 +44,6 @@ struct Fwd16Smem {
   float4 tile[2][kFwdTileF4];  // packed B / C of two chunks
   uint64_t bar[2];             // TMA completion, one phase per use of a buffer
   float H[2 * W][kN];          // state entering the current chunk
-  float Dk[2 * W][kN];         // summary: product of the decays so far
   float2 A[2 * W][kN];         // (A log2(e), A log2(e)): an f32x2 operand as loaded
 };
 
@@ -121,7 +120,6 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
     const float a = act ? __ldg(p.A + (size_t)dd * kN + n) * kLog2e : 0.0f;
     sm.A[rr][n] = make_float2(a, a);
     sm.H[rr][n] = (act && p.h0 && !SUM) ? __ldg(p.h0 + ((size_t)b * p.D + dd) * kN + n) : 0.0f;
-    sm.Dk[rr][n] = 1.0f;
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -131,6 +129,10 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
   const float Dv = (active && p.Dskip) ? __ldg(p.Dskip + d) : 0.0f;
   const float bias = (active && p.delta_bias) ? __ldg(p.delta_bias + d) : 0.0f;
   float wk[4] = {0.0f, 0.0f, 0.0f, 0.0f}, cbias = 0.0f, c5 = 0.0f, c6 = 0.0f, c7 = 0.0f;
+  // summary: the lane's sum of dt and whether a document starts after token 0
+  // (the decay of the piece is exp(A sum dt), or 0 across a start)
+  float dt_sum = 0.0f;
+  bool any_start = false;
   if (CONV && active) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) wk[k] = __ldg(p.conv_w + (size_t)d * 4 + k);
@@ -225,6 +227,7 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
       if (vb) store8<T>(u_out + tl + 8, ub);
     }
     const bool any_reset = __any_sync(kFull, rm != 0u);
+    if constexpr (SUM) any_start = any_start || any_reset;
 
     float2 dd[8], xx[8], y2[8];
 #pragma unroll
@@ -236,6 +239,7 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
       dd[i] = dt;
       xx[i] = fmul2(dt, u2);
       y2[i] = make_float2(Dv * u2.x, Dv * u2.y);
+      if constexpr (SUM) dt_sum += dt.x + dt.y;
     }
 
     const float4* tile = &sm.tile[buf][0];
@@ -292,10 +296,7 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
         const float end = fmaf(Pl[s], cin[s], Hl[s]);
         float start = __shfl_up_sync(kFull, end, 1, 16);
         if (jj == 0) start = cin[s];
-        if (jj == 15) {
-          sm.H[r][n] = end;
-          if constexpr (SUM) sm.Dk[r][n] *= Pl[s];  // the scan left the 16 lanes' product here
-        }
+        if (jj == 15) sm.H[r][n] = end;
         if constexpr (SUM) continue;
         const float sb = fmaf(P[s].x, start, H[s].x);  // state entering sub-segment b
         if (va) *reinterpret_cast<float2*>(ckc + n * 2 * kSegs) = make_float2(start, sb);
@@ -361,8 +362,11 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
 
   __syncwarp();
   if constexpr (SUM) {
+    // the row's sum of dt over its 16 lanes; lane jj writes state jj
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1) dt_sum += __shfl_xor_sync(kFull, dt_sum, off, 16);
     if (active) {
-      p.split_P[rowid * p.Npad + jj] = sm.Dk[r][jj];
+      p.split_P[rowid * p.Npad + jj] = any_start ? 0.0f : ex2_approx(sm.A[r][jj].x * dt_sum);
       p.split_H[rowid * p.Npad + jj] = sm.H[r][jj];
     }
   } else if (active && p.final_state) {

@@ -100,12 +100,15 @@ def test_complex_final_state_gradient_matches_oracle():
     assert rel_l2(host64(g["dinitial_state"]), pairs(w["dh0"])) <= TOL_F32
 
 
-@pytest.mark.parametrize("L,bounds,cut", [(333, (100, 250), False), (333, (100, 250), True),
-                                          (40, (), False), (40, (), True)])
-def test_summaries_and_carry_match_oracle(L, bounds, cut):
+@pytest.mark.parametrize("L,bounds,cut,n_splits", [(333, (100, 250), False, 0), (333, (100, 250), True, 0),
+                                                   (40, (), False, 0), (40, (), True, 0),
+                                                   (40, (), False, 1), (528, (100, 300), True, 1),
+                                                   (528, (), False, 1)])
+def test_summaries_and_carry_match_oracle(L, bounds, cut, n_splits):
     """Summaries against oracle runs; rows with a document start inside have
     decay 0, and a start at token 0 (seq_prev differs) zeroes decay and the
-    backward summary."""
+    backward summary. n_splits=1 with L a multiple of 8 takes the N = 16
+    summary kernels (the automatic choice splits rows this short)."""
     import torch
     import selective_state_space_35_b200 as ssm
     p = _f32(full_problem(2, 12, 16, L, seed=804 + L + int(cut), seq_bounds=bounds))
@@ -114,10 +117,10 @@ def test_summaries_and_carry_match_oracle(L, bounds, cut):
                             dtype=torch.int32, device="cuda")
     dec, end = ssm.scan_fwd_summary(d["x"], d["delta"], d["A"], d["Bm"],
                                     delta_bias=d["delta_bias"], seq_idx=d["seq_idx"],
-                                    seq_prev=seq_prev)
+                                    seq_prev=seq_prev, n_splits=n_splits)
     bdec, adj = ssm.scan_bwd_summary(d["delta"], d["A"], d["Cm"], d["dout"], z=d["z"],
                                      delta_bias=d["delta_bias"], seq_idx=d["seq_idx"],
-                                     seq_prev=seq_prev)
+                                     seq_prev=seq_prev, n_splits=n_splits)
     torch.cuda.synchronize()
     ops = OracleOps()
     T = lambda a: torch.from_numpy(a)  # noqa: E731

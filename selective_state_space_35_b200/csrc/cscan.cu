@@ -52,16 +52,17 @@ __device__ __forceinline__ float2 cis(float theta) {
   const float k = sh - 12582912.0f;
   float r = fmaf(-k, 1.57079637f, theta);                   // float(pi/2)
   r = fmaf(-k, -4.37113883e-8f, r);                         // pi/2 - float(pi/2)
+  // the sine and cosine Horner chains side by side in one f32x2 register
+  // (each half rounds exactly as the scalar chain would)
   const float r2 = r * r;
-  float ps = fmaf(r2, 2.75573192e-6f, -1.98412698e-4f);     // 1/9!, -1/7!
-  ps = fmaf(r2, ps, 8.33333333e-3f);                        // 1/5!
-  ps = fmaf(r2, ps, -1.66666667e-1f);                       // -1/3!
-  const float sn = fmaf(r * r2, ps, r);
-  float pc = fmaf(r2, -2.75573192e-7f, 2.48015873e-5f);     // -1/10!, 1/8!
-  pc = fmaf(r2, pc, -1.38888889e-3f);                       // -1/6!
-  pc = fmaf(r2, pc, 4.16666667e-2f);                        // 1/4!
-  pc = fmaf(r2, pc, -0.5f);                                 // -1/2!
-  const float cs = fmaf(r2, pc, 1.0f);
+  const float2 rr = make_float2(r2, r2);
+  float2 hs = __ffma2_rn(rr, make_float2(2.75573192e-6f, -2.75573192e-7f),
+                         make_float2(-1.98412698e-4f, 2.48015873e-5f));  // (1/9!, -1/10!), (-1/7!, 1/8!)
+  hs = __ffma2_rn(rr, hs, make_float2(8.33333333e-3f, -1.38888889e-3f));   // 1/5!, -1/6!
+  hs = __ffma2_rn(rr, hs, make_float2(-1.66666667e-1f, 4.16666667e-2f));   // -1/3!, 1/4!
+  hs = __ffma2_rn(make_float2(r * r2, r2), hs, make_float2(r, -0.5f));     // sin done; -1/2!
+  const float sn = hs.x;
+  const float cs = fmaf(r2, hs.y, 1.0f);
   const bool odd = q & 1;
   const float c = odd ? sn : cs, s = odd ? cs : sn;
   const unsigned sc = (unsigned)((q + 1) & 2) << 30;        // cos < 0 in quadrants 1, 2

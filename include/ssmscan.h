@@ -410,6 +410,46 @@ typedef struct {
 
 ssm_status_t ssm_decode_step(const ssm_decode_params* p, ssm_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * ssm_ssd_fwd — Mamba-2 SSD forward ("hung-phan ml-skills mamba", section
+ * "Mamba-2: Structured State Space Duality (SSD)": A is a scalar per head).
+ * Per batch b, head h (group g = h / (H / G)) and token t:
+ *   dt_t = softplus(dt_raw[b][t][h] + dt_bias[h])      (or without softplus)
+ *   a_t  = exp(dt_t A[h])                               (0 at a document start)
+ *   S_t[p][n] = a_t S_{t-1}[p][n] + dt_t x[b][t][h][p] B[b][t][g][n],  S_{-1} = 0
+ *   y[b][t][h][p] = sum_n C[b][t][g][n] S_t[p][n] + D[h] x[b][t][h][p]
+ * computed in chunks of 128 tokens as masked matrix products on the tensor
+ * cores (bf16 operands, fp32 accumulation; the state between chunks is kept
+ * in fp32 and enters the next chunk's product rounded to bf16).
+ *   x        [B][L][H][P] bf16         y       [B][L][H][P] bf16 output
+ *   dt_raw   [B][L][H]    bf16         Bm, Cm  [B][L][G][N] bf16
+ *   A        [H] fp32 (negative)       D, dt_bias  [H] fp32, nullable (0)
+ *   seq_idx  [B][L] int32, nullable    final_state [B][H][P][N] fp32, nullable
+ * Supported: dtype bf16, P = 64, N = 128, G >= 1 dividing H, any L >= 1
+ * (else SSM_ERR_UNSUPPORTED); every pointer 16-byte aligned. One CTA per
+ * (b, h); the chunks of a row run in order inside it.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    size_t struct_size;        /* = sizeof(ssm_ssd_params) */
+    int B, L, H, P, G, N;
+    ssm_dtype_t dtype;
+    const void* x;
+    const void* dt_raw;
+    const float* A;
+    const void* Bm;
+    const void* Cm;
+    const float* D;
+    const float* dt_bias;
+    int dt_softplus;
+    const int32_t* seq_idx;
+    void* y;
+    float* final_state;
+    int* status;               /* device int, nullable: SSM_ERR_TIMEOUT if a bounded wait for
+                                  the tensor cores gave up (outputs then invalid) */
+} ssm_ssd_params;
+
+ssm_status_t ssm_ssd_fwd(const ssm_ssd_params* p, ssm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -21,14 +21,15 @@ from ._lib import (SsmError, ssm_abi_version, ssm_conv1d_bwd, ssm_conv1d_bwd_noa
                    ssm_last_error,
                    ssm_probe_ex2_rate, ssm_scan_bwd, ssm_scan_status,
                    ssm_scan_fwd, ssm_scan_grads, ssm_scan_params, ssm_scan_workspace_size,
-                   ssm_scan_bwd_workspace_size,
+                   ssm_scan_bwd_workspace_size, ssm_ssd_params, ssm_ssd_fwd,
                    ssm_scan_fwd_summary, ssm_scan_bwd_summary, ssm_state_carry,
                    ssm_conv1d_fwd_ctx, ssm_conv1d_bwd_ctx)
 
 __all__ = [
     "SsmError", "ssm_abi_version", "ssm_last_error", "ssm_conv1d_fwd", "ssm_conv1d_bwd",
     "ssm_conv1d_bwd_workspace_size", "ssm_conv1d_bwd_noalloc", "ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_scan_bwd",
-    "ssm_scan_params", "ssm_scan_grads", "ssm_scan_bwd_workspace_size", "ssm_probe_ex2_rate", "probe_ex2_rate", "ssm_scan_status",
+    "ssm_scan_params", "ssm_scan_grads", "ssm_scan_bwd_workspace_size", "ssm_ssd_params",
+    "ssm_ssd_fwd", "ssd_fwd", "ssm_probe_ex2_rate", "probe_ex2_rate", "ssm_scan_status",
     "scan_status", "conv1d_fwd", "conv1d_bwd", "scan_params",
     "scan_workspace_size", "scan_fwd", "scan_bwd", "load",
     "ssm_decode_params", "ssm_decode_step", "decode_step", "ssm_conv1d_scan_fwd",
@@ -462,3 +463,42 @@ def state_carry(decay, value, r, *, reverse=False, init=None, seq_prev=None, seq
                                _ptr(init), _ptr(seq_prev), _ptr(seq_idx), L, out.data_ptr(), B, D,
                                N, _stream(stream, decay.device)))
     return out
+
+
+def ssd_fwd(x, dt_raw, A, Bm, Cm, *, D=None, dt_bias=None, softplus=True, seq_idx=None,
+            return_final_state=False, out=None, status=None, stream=None):
+    """Mamba-2 SSD forward on the tensor cores.
+
+    x [B, L, H, 64] bf16; dt_raw [B, L, H] bf16; Bm, Cm [B, L, G, 128] bf16;
+    A, D, dt_bias [H] fp32; seq_idx [B, L] int32. Returns (y [B, L, H, 64]
+    bf16, final_state [B, H, 64, 128] fp32 or None)."""
+    torch = _torch()
+    B, L, H, P = x.shape
+    G, N = Bm.shape[2], Bm.shape[3]
+    _need(x, "x", torch.bfloat16, (B, L, H, P))
+    _need(dt_raw, "dt_raw", torch.bfloat16, (B, L, H))
+    _need(Bm, "Bm", torch.bfloat16, (B, L, G, N))
+    _need(Cm, "Cm", torch.bfloat16, (B, L, G, N))
+    _need(A, "A", torch.float32, (H,))
+    _need(D, "D", torch.float32, (H,))
+    _need(dt_bias, "dt_bias", torch.float32, (H,))
+    _need(seq_idx, "seq_idx", torch.int32, (B, L))
+    y = torch.empty_like(x) if out is None else out
+    _need(y, "out", torch.bfloat16, (B, L, H, P))
+    fs = (torch.empty((B, H, P, N), dtype=torch.float32, device=x.device)
+          if return_final_state else None)
+    p = ssm_ssd_params()
+    p.struct_size = ctypes.sizeof(ssm_ssd_params)
+    p.B, p.L, p.H, p.P, p.G, p.N = B, L, H, P, G, N
+    p.dtype = 1
+    p.x, p.dt_raw, p.A = x.data_ptr(), dt_raw.data_ptr(), A.data_ptr()
+    p.Bm, p.Cm = Bm.data_ptr(), Cm.data_ptr()
+    p.D = D.data_ptr() if D is not None else None
+    p.dt_bias = dt_bias.data_ptr() if dt_bias is not None else None
+    p.dt_softplus = 1 if softplus else 0
+    p.seq_idx = seq_idx.data_ptr() if seq_idx is not None else None
+    p.y = y.data_ptr()
+    p.final_state = fs.data_ptr() if fs is not None else None
+    p.status = status.data_ptr() if status is not None else None
+    _lib.check(ssm_ssd_fwd(p, _stream(stream, x.device)))
+    return y, fs

@@ -63,6 +63,17 @@ class ssm_scan_grads(ctypes.Structure):
     ]
 
 
+class ssm_ssd_params(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", _sz),
+        ("B", _i), ("L", _i), ("H", _i), ("P", _i), ("G", _i), ("N", _i),
+        ("dtype", _i),
+        ("x", _vp), ("dt_raw", _vp), ("A", _vp), ("Bm", _vp), ("Cm", _vp),
+        ("D", _vp), ("dt_bias", _vp), ("dt_softplus", _i), ("seq_idx", _vp),
+        ("y", _vp), ("final_state", _vp), ("status", _vp),
+    ]
+
+
 class ssm_decode_params(ctypes.Structure):
     _fields_ = [
         ("struct_size", _sz),
@@ -82,7 +93,7 @@ EXPORTS = ("ssm_last_error", "ssm_abi_version", "ssm_conv1d_fwd", "ssm_conv1d_bw
            "ssm_conv1d_bwd", "ssm_conv1d_bwd_noalloc", "ssm_scan_workspace_size", "ssm_scan_fwd",
            "ssm_scan_bwd", "ssm_scan_bwd_workspace_size", "ssm_scan_status", "ssm_probe_ex2_rate", "ssm_decode_step",
            "ssm_conv1d_scan_fwd", "ssm_scan_fwd_summary", "ssm_scan_bwd_summary",
-           "ssm_state_carry", "ssm_conv1d_fwd_ctx", "ssm_conv1d_bwd_ctx")
+           "ssm_state_carry", "ssm_conv1d_fwd_ctx", "ssm_conv1d_bwd_ctx", "ssm_ssd_fwd")
 
 
 def load(path: str | None = None):
@@ -127,6 +138,8 @@ def load(path: str | None = None):
     L.ssm_conv1d_scan_fwd.argtypes = [ctypes.POINTER(ssm_scan_params), _vp, _vp, _vp, _vp]
     L.ssm_decode_step.restype = _i
     L.ssm_decode_step.argtypes = [ctypes.POINTER(ssm_decode_params), _vp]
+    L.ssm_ssd_fwd.restype = _i
+    L.ssm_ssd_fwd.argtypes = [ctypes.POINTER(ssm_ssd_params), _vp]
     L.ssm_scan_fwd_summary.restype = _i
     L.ssm_scan_fwd_summary.argtypes = [ctypes.POINTER(ssm_scan_params), _vp, _vp, _vp, _vp]
     L.ssm_scan_bwd_summary.restype = _i
@@ -238,3 +251,7 @@ def ssm_conv1d_fwd_ctx(*args) -> int:
 
 def ssm_conv1d_bwd_ctx(*args) -> int:
     return load().ssm_conv1d_bwd_ctx(*args)
+
+
+def ssm_ssd_fwd(params: ssm_ssd_params, stream) -> int:
+    return load().ssm_ssd_fwd(ctypes.byref(params), stream)

@@ -728,4 +728,49 @@ ssm_status_t ssm_probe_ex2_rate(float* sink, size_t sink_floats, double* ex2_per
                      "ssm_probe_ex2_rate");
 }
 
+
+// ---------------------------------------------------------------------------
+ssm_status_t ssm_ssd_fwd(const ssm_ssd_params* p, ssm_stream_t stream) {
+  if (injected("ssm_ssd_fwd")) return fail(SSM_ERR_INJECTED, "ssm_ssd_fwd: injected failure");
+  if (!p) return fail(SSM_ERR_INVALID_ARG, "params is NULL");
+  if (p->struct_size != sizeof(ssm_ssd_params))
+    return fail(SSM_ERR_INVALID_ARG, "struct_size %zu != %zu", p->struct_size, sizeof(ssm_ssd_params));
+  if (p->B < 1 || p->L < 1 || p->H < 1 || p->G < 1)
+    return fail(SSM_ERR_INVALID_ARG, "B=%d L=%d H=%d G=%d must be >= 1", p->B, p->L, p->H, p->G);
+  if (p->H % p->G != 0) return fail(SSM_ERR_INVALID_ARG, "G=%d does not divide H=%d", p->G, p->H);
+  if (p->dtype != SSM_DTYPE_BF16) return fail(SSM_ERR_UNSUPPORTED, "ssd: bf16 only");
+  if (p->P != 64 || p->N != 128)
+    return fail(SSM_ERR_UNSUPPORTED, "ssd: P=%d N=%d (supported: P=64, N=128)", p->P, p->N);
+  if (!p->x || !p->dt_raw || !p->A || !p->Bm || !p->Cm || !p->y)
+    return fail(SSM_ERR_INVALID_ARG, "x, dt_raw, A, Bm, Cm and y must be non-NULL");
+  const void* v16[] = {p->x, p->Bm, p->Cm, p->y};
+  for (const void* q : v16)
+    if (!aligned(q, 16)) return fail(SSM_ERR_INVALID_ARG, "ssd: x, Bm, Cm, y must be 16-byte aligned");
+  const void* v4[] = {p->A, p->D, p->dt_bias, p->seq_idx, p->final_state, p->status};
+  for (const void* q : v4)
+    if (q && !aligned(q, 4)) return fail(SSM_ERR_INVALID_ARG, "ssd: fp32 / int32 pointer misaligned");
+  if (!aligned(p->dt_raw, 2)) return fail(SSM_ERR_INVALID_ARG, "ssd: dt_raw misaligned");
+  ssm::SsdArgs a;
+  a.x = p->x;
+  a.dt_raw = p->dt_raw;
+  a.A = p->A;
+  a.Bm = p->Bm;
+  a.Cm = p->Cm;
+  a.D = p->D;
+  a.dt_bias = p->dt_bias;
+  a.seq = p->seq_idx;
+  a.y = p->y;
+  a.final_state = p->final_state;
+  a.status = p->status;
+  a.B = p->B;
+  a.L = p->L;
+  a.H = p->H;
+  a.P = p->P;
+  a.G = p->G;
+  a.N = p->N;
+  a.softplus = p->dt_softplus ? 1 : 0;
+  return cuda_status(ssm::launch_ssd_fwd(a, reinterpret_cast<cudaStream_t>(stream)),
+                     "ssm_ssd_fwd launch");
+}
+
 }  // extern "C"

@@ -174,6 +174,26 @@ constexpr int kCscanCtaRows = 8;
 cudaError_t launch_dbc_reduce(const float* part, int groups, size_t bnl, float* dB, float* dC,
                               cudaStream_t s);
 cudaError_t probe_ex2_rate(float* sink, size_t sink_floats, double* rate, cudaStream_t s);
+
+// Mamba-2 SSD forward (ssd_fwd.cu): x [B][L][H][P], dt_raw [B][L][H], B / C
+// [B][L][G][N] bf16; A, D, dt_bias [H] fp32; y [B][L][H][P] bf16; final
+// state [B][H][P][N] fp32. P = 64, N = 128.
+struct SsdArgs {
+  const void* x;
+  const void* dt_raw;
+  const float* A;
+  const void* Bm;
+  const void* Cm;
+  const float* D;
+  const float* dt_bias;
+  const int32_t* seq;
+  void* y;
+  float* final_state;
+  int* status;
+  int B, L, H, P, G, N;
+  int softplus;
+};
+cudaError_t launch_ssd_fwd(const SsdArgs& a, cudaStream_t s);
 cudaError_t launch_cu_seqlens_to_seq(const int32_t* cu, int n_docs, int L, int32_t* seq,
                                      cudaStream_t s);
 

@@ -1,0 +1,358 @@
+// Mamba-2 SSD forward ("hung-phan ml-skills mamba", section "Mamba-2:
+// Structured State Space Duality (SSD)": a scalar decay per head, so the
+// scan over a chunk of tokens is a masked matrix product that runs on the
+// tensor cores). Per (batch b, head h), head dimension P = 64, state N = 128,
+// with dt_t = softplus(dt_raw + bias) and a_t = exp(dt_t A_h) (0 at a
+// document start):
+//   h_t[p][n] = a_t h_{t-1}[p][n] + dt_t x_t[p] B_t[n],   y_t[p] = sum_n C_t[n] h_t[p][n] + D_h x_t[p].
+// Chunks of Q = 128 tokens, with lcs_i = sum_{k<=i} dt_k A_h inside the chunk
+// and ls_i the last document start at or before i (-1: none):
+//   Y_diag = (C B^T o L) (dt x),   L_ij = exp(lcs_i - lcs_j) for ls_i <= j <= i, else 0
+//   Y_off  = diag([ls_i < 0] exp(lcs_i)) C H_prev^T
+//   H_new  = [ls_Q-1 < 0] exp(lcs_Q-1) H_prev + x^T diag(w) B,  w_j = dt_j exp(lcs_Q-1 - lcs_j) [j >= ls_Q-1]
+// The products are bf16 tcgen05.mma with fp32 accumulators in tensor
+// memory (TMEM), issued by one thread, their completion signalled on an
+// mbarrier (bounded waits). Operands are written by the CTA's threads into
+// shared memory in the K-major, no-swizzle core-matrix layout; the state
+// H^T[n][p] stays in fp32 registers (thread n) across the chunks of a
+// sequence and enters the next chunk's product as bf16. The decay-masked
+// C B^T enters as a bf16 pair (rounded value and rounded remainder, two
+// products): its own rounding would otherwise dominate the error of y.
+//
+// One CTA of 128 threads per (b, h); thread i owns token i of the chunk and
+// TMEM lane i. No TMA multicast, no cluster.
+#include <atomic>
+
+#include "scan_common.cuh"
+
+namespace ssm {
+
+namespace {
+
+constexpr int kQ = 128;  // tokens per chunk
+constexpr int kP = 64;   // head dimension
+constexpr int kNs = 128; // state size
+constexpr int kThreads = 128;
+
+// Shared memory: bf16 operands in the K-major, no-swizzle core-matrix layout
+// (8 rows x 16 bytes per core matrix; core matrices 128 B apart along K,
+// 8-row groups 2 KB apart: every operand has K = 128).
+struct SsdSmem {
+  unsigned char C[kQ * kNs * 2];    // C [i][n], then C' = C scaled by [ls_i < 0] exp(lcs_i)
+  unsigned char Bm[kQ * kNs * 2];   // B [j][n]
+  unsigned char M[kQ * kQ * 2];     // (C B^T o L) dt [i][j], rounded to bf16
+  unsigned char Mlo[kQ * kQ * 2];   // its rounding remainder, rounded to bf16 (M = M + Mlo to ~2^-17)
+  unsigned char Bw[kNs * kQ * 2];   // w_j B_j[n] as [n][j]
+  unsigned char Xt[kP * kQ * 2];    // x as [p][j]
+  unsigned char Hb[kP * kNs * 2];   // H_prev [p][n]
+  float lcs[kQ];
+  float dt[kQ];
+  int ls[kQ];
+  float wsum[4];
+  int wmax[4];
+  uint64_t bar;
+  uint32_t tmem;
+};
+
+__device__ __forceinline__ uint32_t tile_off(int r, int k) {
+  return (r >> 3) * 2048 + (k >> 3) * 128 + (r & 7) * 16 + (k & 7) * 2;
+}
+// Shared-memory matrix descriptor (sm100): start >> 4, leading byte offset
+// (between K-adjacent core matrices) 128 B, stride byte offset (between
+// 8-row groups) 2048 B, descriptor version 1, no swizzle.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 16) |
+         ((uint64_t)(2048 >> 4) << 32) | (1ull << 46);
+}
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major, M = 128, N = n.
+__device__ __forceinline__ uint32_t umma_idesc(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+// D (+)= A B^T over K = 128 (eight K = 16 steps), A [128][128], B [n][128].
+__device__ __forceinline__ void umma_k128(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem, int n,
+                                          bool accumulate) {
+  const uint32_t idesc = umma_idesc(n);
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const uint32_t acc = (accumulate || s > 0) ? 1u : 0u;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(umma_desc(a_smem + 256 * s)), "l"(umma_desc(b_smem + 256 * s)), "r"(idesc), "r"(acc), "r"(0u),
+        "r"(0u), "r"(0u), "r"(0u));
+  }
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t addr, float v[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+      "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]),
+        "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+        "=r"(r[30]), "=r"(r[31])
+      : "r"(addr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  SsdSmem& sm = *reinterpret_cast<SsdSmem*>(smem_raw);
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int H = p.H, L = p.L, G = p.G;
+  const int g = h / (H / G);
+  const float Ah = __ldg(p.A + h);
+  const float bias = p.dt_bias ? __ldg(p.dt_bias + h) : 0.0f;
+  const float Dh = p.D ? __ldg(p.D + h) : 0.0f;
+  const __nv_bfloat16* xg = static_cast<const __nv_bfloat16*>(p.x);
+  const __nv_bfloat16* dtg = static_cast<const __nv_bfloat16*>(p.dt_raw);
+  const __nv_bfloat16* Bg = static_cast<const __nv_bfloat16*>(p.Bm);
+  const __nv_bfloat16* Cg = static_cast<const __nv_bfloat16*>(p.Cm);
+  __nv_bfloat16* yg = static_cast<__nv_bfloat16*>(p.y);
+  const int32_t* seqb = p.seq ? p.seq + (size_t)b * L : nullptr;
+
+  if (t == 0) {
+    mbar_init(&sm.bar, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(smem_u32(&sm.tmem))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  // H_prev = 0 before the first chunk
+  for (int i = t; i < kP * kNs * 2 / 16; i += kThreads)
+    reinterpret_cast<uint4*>(sm.Hb)[i] = make_uint4(0u, 0u, 0u, 0u);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem;
+  const uint32_t lane_row = tmem + ((uint32_t)(32 * warp) << 16);  // TMEM lane t
+  // TMEM columns: S [0, 128), Y [128, 192), chunk state S_c^T [192, 256)
+  const uint32_t sC = smem_u32(sm.C), sB = smem_u32(sm.Bm), sM = smem_u32(sm.M);
+  const uint32_t sBw = smem_u32(sm.Bw), sX = smem_u32(sm.Xt), sH = smem_u32(sm.Hb);
+  const uint32_t sMlo = smem_u32(sm.Mlo);
+
+  float Ht[kP];  // H^T[n = t][p], fp32 across the chunks
+#pragma unroll
+  for (int q = 0; q < kP; ++q) Ht[q] = 0.0f;
+  unsigned phase = 0;
+  const int nch = (L + kQ - 1) / kQ;
+  const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+
+#pragma unroll 1
+  for (int c = 0; c < nch; ++c) {
+    const int tok = c * kQ + t;
+    const bool valid = tok < L;
+    // ---- this token: dt, document start, C and B rows, x row ----
+    float dt = 0.0f;
+    bool start = false;
+    if (valid) {
+      const float v = __bfloat162float(dtg[((size_t)b * L + tok) * H + h]) + bias;
+      dt = p.softplus ? (v > 20.0f ? v : log1pf(expf(v))) : v;
+      if (seqb && tok > 0) start = __ldg(seqb + tok) != __ldg(seqb + tok - 1);
+    }
+    const uint4* crow = reinterpret_cast<const uint4*>(Cg + (((size_t)b * L + tok) * G + g) * kNs);
+    const uint4* brow = reinterpret_cast<const uint4*>(Bg + (((size_t)b * L + tok) * G + g) * kNs);
+    uint4 braw[16];
+#pragma unroll
+    for (int k8 = 0; k8 < 16; ++k8) {
+      *reinterpret_cast<uint4*>(sm.C + tile_off(t, 8 * k8)) = valid ? __ldg(crow + k8) : z4;
+      braw[k8] = valid ? __ldg(brow + k8) : z4;
+      *reinterpret_cast<uint4*>(sm.Bm + tile_off(t, 8 * k8)) = braw[k8];
+    }
+    const uint4* xrow = reinterpret_cast<const uint4*>(xg + (((size_t)b * L + tok) * H + h) * kP);
+    uint4 xraw[8];
+#pragma unroll
+    for (int k8 = 0; k8 < 8; ++k8) {
+      xraw[k8] = valid ? __ldg(xrow + k8) : z4;
+      const uint32_t w4[4] = {xraw[k8].x, xraw[k8].y, xraw[k8].z, xraw[k8].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {  // x as [p][j]: element (8 k8 + 2e (+1), t)
+        *reinterpret_cast<uint16_t*>(sm.Xt + tile_off(8 * k8 + 2 * e, t)) = (uint16_t)(w4[e] & 0xffffu);
+        *reinterpret_cast<uint16_t*>(sm.Xt + tile_off(8 * k8 + 2 * e + 1, t)) = (uint16_t)(w4[e] >> 16);
+      }
+    }
+    // ---- chunk scans: lcs = inclusive sum of dt A, ls = last document start ----
+    float la = dt * Ah;
+    int st = start ? t : -1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float lo = __shfl_up_sync(kFull, la, off);
+      const int so = __shfl_up_sync(kFull, st, off);
+      if (lane >= off) {
+        la += lo;
+        st = max(st, so);
+      }
+    }
+    if (lane == 31) {
+      sm.wsum[warp] = la;
+      sm.wmax[warp] = st;
+    }
+    __syncthreads();
+    for (int w = 0; w < warp; ++w) {
+      la += sm.wsum[w];
+      st = max(st, sm.wmax[w]);
+    }
+    sm.lcs[t] = la;
+    sm.dt[t] = dt;
+    sm.ls[t] = st;
+    __syncthreads();
+    const float lcsQ = sm.lcs[kQ - 1];
+    const int lsQ = sm.ls[kQ - 1];
+    // ---- B scaled by w_t = dt_t exp(lcs_Q-1 - lcs_t) [t >= ls_Q-1], as [n][t] ----
+    const float wt = (t >= lsQ) ? dt * __expf(lcsQ - la) : 0.0f;
+#pragma unroll
+    for (int k8 = 0; k8 < 16; ++k8) {
+      const uint32_t w4[4] = {braw[k8].x, braw[k8].y, braw[k8].z, braw[k8].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat16 lo = __float2bfloat16(bf_lo(w4[e]) * wt);
+        const __nv_bfloat16 hi = __float2bfloat16(bf_hi(w4[e]) * wt);
+        *reinterpret_cast<__nv_bfloat16*>(sm.Bw + tile_off(8 * k8 + 2 * e, t)) = lo;
+        *reinterpret_cast<__nv_bfloat16*>(sm.Bw + tile_off(8 * k8 + 2 * e + 1, t)) = hi;
+      }
+    }
+    // ---- S = C B^T on the tensor cores ----
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (t == 0) {
+      umma_k128(tmem, sC, sB, kQ, false);
+      umma_commit(&sm.bar);
+    }
+    bool ok = mbar_wait_bounded(&sm.bar, phase, p.status);
+    phase ^= 1u;
+    if (!__syncthreads_and(ok)) break;
+    tc_fence_after();
+    // ---- row t of M = (C B^T o L) dt, and row t of C' ----
+    {
+      const float lcs_i = la;
+      const int ls_i = st;
+#pragma unroll 1
+      for (int j0 = 0; j0 < kQ; j0 += 32) {
+        float v[32];
+        tmem_ld32(lane_row + j0, v);
+#pragma unroll
+        for (int e = 0; e < 32; e += 8) {
+          float m[8], r[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int j = j0 + e + q;
+            m[q] = (j >= ls_i && j <= t) ? v[e + q] * __expf(lcs_i - sm.lcs[j]) * sm.dt[j] : 0.0f;
+          }
+          const uint4 hi = make_uint4(pack_bf16(m[0], m[1]), pack_bf16(m[2], m[3]), pack_bf16(m[4], m[5]),
+                                      pack_bf16(m[6], m[7]));
+          const uint32_t hw[4] = {hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            r[2 * q] = m[2 * q] - bf_lo(hw[q]);
+            r[2 * q + 1] = m[2 * q + 1] - bf_hi(hw[q]);
+          }
+          *reinterpret_cast<uint4*>(sm.M + tile_off(t, j0 + e)) = hi;
+          *reinterpret_cast<uint4*>(sm.Mlo + tile_off(t, j0 + e)) =
+              make_uint4(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]), pack_bf16(r[4], r[5]),
+                         pack_bf16(r[6], r[7]));
+        }
+      }
+      const float cs = ls_i < 0 ? __expf(lcs_i) : 0.0f;
+#pragma unroll
+      for (int k8 = 0; k8 < 16; ++k8) {
+        uint4* q = reinterpret_cast<uint4*>(sm.C + tile_off(t, 8 * k8));
+        const uint4 cv = *q;
+        *q = make_uint4(pack_bf16(bf_lo(cv.x) * cs, bf_hi(cv.x) * cs), pack_bf16(bf_lo(cv.y) * cs, bf_hi(cv.y) * cs),
+                        pack_bf16(bf_lo(cv.z) * cs, bf_hi(cv.z) * cs), pack_bf16(bf_lo(cv.w) * cs, bf_hi(cv.w) * cs));
+      }
+    }
+    // ---- Y = M x + C' H_prev^T and S_c^T = (diag(w) B)^T x ----
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (t == 0) {
+      umma_k128(tmem + 128, sM, sX, kP, false);
+      umma_k128(tmem + 128, sMlo, sX, kP, true);
+      umma_k128(tmem + 128, sC, sH, kP, true);
+      umma_k128(tmem + 192, sBw, sX, kP, false);
+      umma_commit(&sm.bar);
+    }
+    ok = mbar_wait_bounded(&sm.bar, phase, p.status);
+    phase ^= 1u;
+    if (!__syncthreads_and(ok)) break;
+    tc_fence_after();
+    // ---- y row t; the state row n = t ----
+    {
+      float yv[kP];
+      tmem_ld32(lane_row + 128, yv);
+      tmem_ld32(lane_row + 160, yv + 32);
+      if (valid) {
+        uint4* yrow = reinterpret_cast<uint4*>(yg + (((size_t)b * L + tok) * H + h) * kP);
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8) {
+          const uint32_t w4[4] = {xraw[k8].x, xraw[k8].y, xraw[k8].z, xraw[k8].w};
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int q = 8 * k8 + 2 * e;
+            o[e] = pack_bf16(fmaf(Dh, bf_lo(w4[e]), yv[q]), fmaf(Dh, bf_hi(w4[e]), yv[q + 1]));
+          }
+          yrow[k8] = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+      float sv[kP];
+      tmem_ld32(lane_row + 192, sv);
+      tmem_ld32(lane_row + 224, sv + 32);
+      const float dec = lsQ < 0 ? __expf(lcsQ) : 0.0f;
+#pragma unroll
+      for (int q = 0; q < kP; ++q) {
+        Ht[q] = fmaf(dec, Ht[q], sv[q]);
+        *reinterpret_cast<__nv_bfloat16*>(sm.Hb + tile_off(q, t)) = __float2bfloat16(Ht[q]);
+      }
+    }
+    tc_fence_before();
+  }
+  if (p.final_state) {
+#pragma unroll
+    for (int q = 0; q < kP; ++q) p.final_state[(((size_t)b * H + h) * kP + q) * kNs + t] = Ht[q];
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
+}
+
+}  // namespace
+
+cudaError_t launch_ssd_fwd(const SsdArgs& a, cudaStream_t s) {
+  static std::atomic<unsigned long long> done{0};
+  const int smem = (int)sizeof(SsdSmem);
+  cudaError_t e = smem_attr(ssd_fwd_kernel, smem, &done);
+  if (e != cudaSuccess) return e;
+  ssd_fwd_kernel<<<dim3(a.H, a.B), kThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace ssm

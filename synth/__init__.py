@@ -305,3 +305,34 @@ def complex_inputs(B: int, D: int, N: int, L: int, dtype: str, seed: int, *,
     h0 = (0.5 * rng.standard_normal((B, D, N, 2), dtype=np.float32)).astype(np.float32) \
         if with_h0 else None
     return ComplexInputs(u, delta, z, dout, Bm, Cm, A, Dskip, delta_bias, seq_idx, h0)
+
+
+@dataclass
+class SsdInputs:
+    """Inputs of the Mamba-2 SSD forward: x [B, L, H, P], dt_raw [B, L, H],
+    Bm, Cm [B, L, G, N] (bf16 storage); A, D, dt_bias float32 [H]; seq_idx
+    int32 [B, L] or None."""
+    x: Tensor
+    dt_raw: Tensor
+    Bm: Tensor
+    Cm: Tensor
+    A: np.ndarray
+    D: np.ndarray
+    dt_bias: np.ndarray
+    seq_idx: np.ndarray | None
+
+
+def ssd_inputs(B: int, L: int, H: int, P: int, G: int, N: int, seed: int, *,
+               seq_idx: np.ndarray | None = None) -> SsdInputs:
+    """Seeded SSD inputs, the Mamba-1 recipes with A a scalar per head:
+    A[h] = -U(1, 16), the dt bias the inverse softplus of U(0.001, 0.1),
+    D ~ U(0.5, 1.5), x / B / C ~ N(0, 1), raw dt ~ 0.5 * N(0, 1); bf16 storage."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    A = (-rng.uniform(1.0, 16.0, size=H)).astype(np.float32)
+    D = rng.uniform(0.5, 1.5, size=H).astype(np.float32)
+    dt_bias = np.log(np.expm1(rng.uniform(1e-3, 1e-1, size=H))).astype(np.float32)
+    x = _act(rng, (B, L, H, P), "bf16")
+    dt_raw = _act(rng, (B, L, H), "bf16", 0.5)
+    Bm = _act(rng, (B, L, G, N), "bf16")
+    Cm = _act(rng, (B, L, G, N), "bf16")
+    return SsdInputs(x, dt_raw, Bm, Cm, A, D, dt_bias, seq_idx)

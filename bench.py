@@ -51,14 +51,17 @@ NCU_TRAFFIC = {"scan_bwd": 1832.669e6 + 597.325e6, "scan_fwd": 612.897e6 + 1155.
 
 
 def _peaks():
+    """HBM copy bandwidth and dense bf16 tensor throughput of this machine's B200s
+    (MEASURED_PEAKS.json when present; else the earlier measurement on this
+    pool: 6650 GB/s, 1590 TFLOP/s)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             pk = json.load(f)
         return {"hbm_gbs": float(pk["hbm_gbs"]), "sm_max_mhz": float(pk.get("sm_max_mhz", 1965.0)),
-                "source": "measured"}
+                "bf16_tflops": float(pk.get("bf16_tflops", 1590.0)), "source": "measured"}
     except Exception:
-        return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+        return {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
 # ----------------------------------------------------------------------------
@@ -316,6 +319,7 @@ def main():
                     help="skip the scan measurement on the other full-size workloads")
     ap.add_argument("--no-deterministic", action="store_true",
                     help="skip the measurement of the deterministic backward")
+    ap.add_argument("--no-ssd", action="store_true", help="skip the Mamba-2 SSD forward measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -450,6 +454,9 @@ def main():
         line["cp_shard"] = cp_shard_bench(device, layers[0], ranks=8)
     if not args.no_deterministic:
         line["deterministic_bwd"] = deterministic_bench(layers[0], avg["scan_bwd"])
+    if not args.no_ssd:
+        line["ssd"] = ssd_bench(device, pk)
+    line["peaks"] = {k: pk[k] for k in ("hbm_gbs", "bf16_tflops", "sm_max_mhz", "source")}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = cpu_count()
@@ -519,6 +526,47 @@ def config_bench(cfg, device, pk, reps=5):
     del ly
     torch.cuda.empty_cache()
     return r
+
+
+def ssd_bench(device, pk, B=2, L=8192, H=64, P=64, G=1, N=128, reps=5):
+    """Mamba-2 SSD forward on the tensor cores at a d_inner = 4096 shape (64
+    heads of 64, one B / C group, state 128), B2 L8192 bf16: CUDA events over
+    `reps` calls after two warm-up calls (inputs 0.28 GB, larger than L2)."""
+    import torch
+    import selective_state_space_35_b200 as ssm
+    si = synth.ssd_inputs(B, L, H, P, G, N, synth.seed_for(11))
+
+    def bf(t):
+        return torch.from_numpy(t.bits.view(np.int16).copy()).view(torch.bfloat16).to(device)
+
+    def f32(a):
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(device)
+
+    x, dtr, Bm, Cm = bf(si.x), bf(si.dt_raw), bf(si.Bm), bf(si.Cm)
+    A, D, db = f32(si.A), f32(si.D), f32(si.dt_bias)
+    y = torch.empty_like(x)
+    for _ in range(2):
+        ssm.ssd_fwd(x, dtr, A, Bm, Cm, D=D, dt_bias=db, out=y)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        ssm.ssd_fwd(x, dtr, A, Bm, Cm, D=D, dt_bias=db, out=y)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    Q = 128
+    chunks = B * H * (-(-L // Q))
+    # per chunk: C B^T (2 Q Q N), Y_diag (2 Q P Q), Y_off (2 Q P N), chunk state (2 N P Q)
+    flops = chunks * (2 * Q * Q * N + 2 * Q * P * Q + 2 * Q * P * N + 2 * N * P * Q)
+    issued = flops + chunks * 2 * Q * P * Q  # the remainder product of the decay-masked C B^T
+    nbytes = 2 * B * L * H * P * 2 + 2 * B * L * G * N * 2 + B * L * H * 2
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": f"Mamba-2 SSD forward, B{B} L{L} H{H} P{P} G{G} N{N} bf16, chunks of {Q}, "
+                        "tcgen05 bf16 products with fp32 TMEM accumulators",
+            "ms": ms, "tokens_per_s": B * L / (ms * 1e-3), "tflops": tf,
+            "tflops_issued": issued / (ms * 1e-3) / 1e12,
+            "tensor_frac_of_peak": tf / pk["bf16_tflops"], "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
+            "flops_per_call": flops, "bytes_per_call": nbytes, "launches": reps + 2}
 
 
 def deterministic_bench(ly, bwd_ms, reps=5):

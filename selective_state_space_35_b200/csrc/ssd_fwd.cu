@@ -34,17 +34,19 @@ constexpr int kP = 64;   // head dimension
 constexpr int kNs = 128; // state size
 constexpr int kThreads = 128;
 
-// Shared memory: bf16 operands in the K-major, no-swizzle core-matrix layout
-// (8 rows x 16 bytes per core matrix; core matrices 128 B apart along K,
-// 8-row groups 2 KB apart: every operand has K = 128).
+// Shared memory: bf16 operands in the no-swizzle core-matrix layouts (every
+// operand has K = 128; core matrices 128 B apart along K, 2 KB apart along
+// M / N): K-major where a thread writes a row along K (C, B, the decay-masked
+// product), MN-major where it writes a row along M / N (x, the w-scaled B,
+// the state), so every thread stores 16-byte vectors.
 struct SsdSmem {
   unsigned char C[kQ * kNs * 2];    // C [i][n], then C' = C scaled by [ls_i < 0] exp(lcs_i)
   unsigned char Bm[kQ * kNs * 2];   // B [j][n]
   unsigned char M[kQ * kQ * 2];     // (C B^T o L) dt [i][j], rounded to bf16
   unsigned char Mlo[kQ * kQ * 2];   // its rounding remainder, rounded to bf16 (M = M + Mlo to ~2^-17)
-  unsigned char Bw[kNs * kQ * 2];   // w_j B_j[n] as [n][j]
-  unsigned char Xt[kP * kQ * 2];    // x as [p][j]
-  unsigned char Hb[kP * kNs * 2];   // H_prev [p][n]
+  unsigned char Bw[kNs * kQ * 2];   // w_j B_j[n]: M = n, K = j, MN-major
+  unsigned char Xt[kP * kQ * 2];    // x_j[p]: N = p, K = j, MN-major
+  unsigned char Hb[kP * kNs * 2];   // H_prev[p][n]: N = p, K = n, MN-major
   float lcs[kQ];
   float dt[kQ];
   int ls[kQ];
@@ -54,8 +56,14 @@ struct SsdSmem {
   uint32_t tmem;
 };
 
+// element (r, k) of a K-major operand: a core matrix is 8 rows of 16 bytes along K
 __device__ __forceinline__ uint32_t tile_off(int r, int k) {
   return (r >> 3) * 2048 + (k >> 3) * 128 + (r & 7) * 16 + (k & 7) * 2;
+}
+// element (mn, k) of an MN-major operand: a core matrix is 8 K rows of 16
+// bytes along M / N
+__device__ __forceinline__ uint32_t tile_off_mn(int mn, int k) {
+  return (mn >> 3) * 2048 + (k >> 3) * 128 + (k & 7) * 16 + (mn & 7) * 2;
 }
 // Shared-memory matrix descriptor (sm100): start >> 4, leading byte offset
 // (between K-adjacent core matrices) 128 B, stride byte offset (between
@@ -64,15 +72,17 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t addr) {
   return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)(128 >> 4) << 16) |
          ((uint64_t)(2048 >> 4) << 32) | (1ull << 46);
 }
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
-// K-major, M = 128, N = n.
-__device__ __forceinline__ uint32_t umma_idesc(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, A / B
+// K-major (0) or MN-major (1), M = 128, N = n.
+__device__ __forceinline__ uint32_t umma_idesc(int n, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
-// D (+)= A B^T over K = 128 (eight K = 16 steps), A [128][128], B [n][128].
+// D (+)= A B^T over K = 128 (eight K = 16 steps: two core matrices along K
+// each), A 128 x 128, B n x 128.
 __device__ __forceinline__ void umma_k128(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem, int n,
-                                          bool accumulate) {
-  const uint32_t idesc = umma_idesc(n);
+                                          bool accumulate, int a_mn, int b_mn) {
+  const uint32_t idesc = umma_idesc(n, a_mn, b_mn);
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
     const uint32_t acc = (accumulate || s > 0) ? 1u : 0u;
@@ -187,12 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
 #pragma unroll
     for (int k8 = 0; k8 < 8; ++k8) {
       xraw[k8] = valid ? __ldg(xrow + k8) : z4;
-      const uint32_t w4[4] = {xraw[k8].x, xraw[k8].y, xraw[k8].z, xraw[k8].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {  // x as [p][j]: element (8 k8 + 2e (+1), t)
-        *reinterpret_cast<uint16_t*>(sm.Xt + tile_off(8 * k8 + 2 * e, t)) = (uint16_t)(w4[e] & 0xffffu);
-        *reinterpret_cast<uint16_t*>(sm.Xt + tile_off(8 * k8 + 2 * e + 1, t)) = (uint16_t)(w4[e] >> 16);
-      }
+      *reinterpret_cast<uint4*>(sm.Xt + tile_off_mn(8 * k8, t)) = xraw[k8];  // p = 8 k8 .. 8 k8 + 7
     }
     // ---- chunk scans: lcs = inclusive sum of dt A, ls = last document start ----
     float la = dt * Ah;
@@ -224,15 +229,11 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
     // ---- B scaled by w_t = dt_t exp(lcs_Q-1 - lcs_t) [t >= ls_Q-1], as [n][t] ----
     const float wt = (t >= lsQ) ? dt * __expf(lcsQ - la) : 0.0f;
 #pragma unroll
-    for (int k8 = 0; k8 < 16; ++k8) {
-      const uint32_t w4[4] = {braw[k8].x, braw[k8].y, braw[k8].z, braw[k8].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const __nv_bfloat16 lo = __float2bfloat16(bf_lo(w4[e]) * wt);
-        const __nv_bfloat16 hi = __float2bfloat16(bf_hi(w4[e]) * wt);
-        *reinterpret_cast<__nv_bfloat16*>(sm.Bw + tile_off(8 * k8 + 2 * e, t)) = lo;
-        *reinterpret_cast<__nv_bfloat16*>(sm.Bw + tile_off(8 * k8 + 2 * e + 1, t)) = hi;
-      }
+    for (int k8 = 0; k8 < 16; ++k8) {  // n = 8 k8 .. 8 k8 + 7 of token t
+      const uint4 q = braw[k8];
+      *reinterpret_cast<uint4*>(sm.Bw + tile_off_mn(8 * k8, t)) =
+          make_uint4(pack_bf16(bf_lo(q.x) * wt, bf_hi(q.x) * wt), pack_bf16(bf_lo(q.y) * wt, bf_hi(q.y) * wt),
+                     pack_bf16(bf_lo(q.z) * wt, bf_hi(q.z) * wt), pack_bf16(bf_lo(q.w) * wt, bf_hi(q.w) * wt));
     }
     // ---- S = C B^T on the tensor cores ----
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -240,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
     __syncthreads();
     tc_fence_after();
     if (t == 0) {
-      umma_k128(tmem, sC, sB, kQ, false);
+      umma_k128(tmem, sC, sB, kQ, false, 0, 0);
       umma_commit(&sm.bar);
     }
     bool ok = mbar_wait_bounded(&sm.bar, phase, p.status);
@@ -292,10 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
     __syncthreads();
     tc_fence_after();
     if (t == 0) {
-      umma_k128(tmem + 128, sM, sX, kP, false);
-      umma_k128(tmem + 128, sMlo, sX, kP, true);
-      umma_k128(tmem + 128, sC, sH, kP, true);
-      umma_k128(tmem + 192, sBw, sX, kP, false);
+      umma_k128(tmem + 128, sM, sX, kP, false, 0, 1);
+      umma_k128(tmem + 128, sMlo, sX, kP, true, 0, 1);
+      umma_k128(tmem + 128, sC, sH, kP, true, 0, 1);
+      umma_k128(tmem + 192, sBw, sX, kP, false, 1, 1);
       umma_commit(&sm.bar);
     }
     ok = mbar_wait_bounded(&sm.bar, phase, p.status);
@@ -326,10 +327,12 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
       tmem_ld32(lane_row + 224, sv + 32);
       const float dec = lsQ < 0 ? __expf(lcsQ) : 0.0f;
 #pragma unroll
-      for (int q = 0; q < kP; ++q) {
-        Ht[q] = fmaf(dec, Ht[q], sv[q]);
-        *reinterpret_cast<__nv_bfloat16*>(sm.Hb + tile_off(q, t)) = __float2bfloat16(Ht[q]);
-      }
+      for (int q = 0; q < kP; ++q) Ht[q] = fmaf(dec, Ht[q], sv[q]);
+#pragma unroll
+      for (int k8 = 0; k8 < 8; ++k8)  // p = 8 k8 .. 8 k8 + 7 of state row n = t
+        *reinterpret_cast<uint4*>(sm.Hb + tile_off_mn(8 * k8, t)) =
+            make_uint4(pack_bf16(Ht[8 * k8], Ht[8 * k8 + 1]), pack_bf16(Ht[8 * k8 + 2], Ht[8 * k8 + 3]),
+                       pack_bf16(Ht[8 * k8 + 4], Ht[8 * k8 + 5]), pack_bf16(Ht[8 * k8 + 6], Ht[8 * k8 + 7]));
     }
     tc_fence_before();
   }

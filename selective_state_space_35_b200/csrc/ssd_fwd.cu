@@ -19,8 +19,10 @@
 // C B^T enters as a bf16 pair (rounded value and rounded remainder, two
 // products): its own rounding would otherwise dominate the error of y.
 //
-// One CTA of 128 threads per (b, h); thread i owns token i of the chunk and
-// TMEM lane i. No TMA multicast, no cluster.
+// One CTA of 256 threads per (b, h): threads i and i + 128 own token i of
+// the chunk (and TMEM lane i), each for half of its columns; the next
+// chunk's global inputs are loaded into registers while the current one is
+// computed. No TMA multicast, no cluster.
 #include <atomic>
 
 #include "scan_common.cuh"
@@ -32,7 +34,7 @@ namespace {
 constexpr int kQ = 128;  // tokens per chunk
 constexpr int kP = 64;   // head dimension
 constexpr int kNs = 128; // state size
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;  // two threads per token row
 
 // Shared memory: bf16 operands in the no-swizzle core-matrix layouts (every
 // operand has K = 128; core matrices 128 B apart along K, 2 KB apart along
@@ -125,10 +127,18 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// Global inputs of one chunk for one thread: half hf of token row r.
+struct ChunkIn {
+  uint4 c[8], b[8], x[4];  // C, B: n = 64 hf .. 64 hf + 63; x: p = 32 hf .. 32 hf + 31
+  float dtv;               // raw dt + bias (as read)
+  int seq_cur, seq_prev;
+};
+
 __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   SsdSmem& sm = *reinterpret_cast<SsdSmem*>(smem_raw);
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int r = t & (kQ - 1), hf = t >> 7;  // token row of the chunk, column half
   const int h = blockIdx.x, b = blockIdx.y;
   const int H = p.H, L = p.L, G = p.G;
   const int g = h / (H / G);
@@ -141,6 +151,25 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
   const __nv_bfloat16* Cg = static_cast<const __nv_bfloat16*>(p.Cm);
   __nv_bfloat16* yg = static_cast<__nv_bfloat16*>(p.y);
   const int32_t* seqb = p.seq ? p.seq + (size_t)b * L : nullptr;
+  const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+
+  auto fetch = [&](int c, ChunkIn& in) {
+    const int tok = c * kQ + r;
+    const bool valid = tok < L;
+    const uint4* crow = reinterpret_cast<const uint4*>(Cg + (((size_t)b * L + tok) * G + g) * kNs) + 8 * hf;
+    const uint4* brow = reinterpret_cast<const uint4*>(Bg + (((size_t)b * L + tok) * G + g) * kNs) + 8 * hf;
+    const uint4* xrow = reinterpret_cast<const uint4*>(xg + (((size_t)b * L + tok) * H + h) * kP) + 4 * hf;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      in.c[k] = valid ? __ldg(crow + k) : z4;
+      in.b[k] = valid ? __ldg(brow + k) : z4;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) in.x[k] = valid ? __ldg(xrow + k) : z4;
+    in.dtv = valid ? __bfloat162float(dtg[((size_t)b * L + tok) * H + h]) + bias : 0.0f;
+    in.seq_cur = (seqb && valid) ? __ldg(seqb + tok) : 0;
+    in.seq_prev = (seqb && valid && tok > 0) ? __ldg(seqb + tok - 1) : in.seq_cur;
+  };
 
   if (t == 0) {
     mbar_init(&sm.bar, 1);
@@ -158,80 +187,82 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem;
-  const uint32_t lane_row = tmem + ((uint32_t)(32 * warp) << 16);  // TMEM lane t
+  const uint32_t lane_row = tmem + ((uint32_t)(32 * (warp & 3)) << 16);  // TMEM lane r
   // TMEM columns: S [0, 128), Y [128, 192), chunk state S_c^T [192, 256)
   const uint32_t sC = smem_u32(sm.C), sB = smem_u32(sm.Bm), sM = smem_u32(sm.M);
   const uint32_t sBw = smem_u32(sm.Bw), sX = smem_u32(sm.Xt), sH = smem_u32(sm.Hb);
   const uint32_t sMlo = smem_u32(sm.Mlo);
 
-  float Ht[kP];  // H^T[n = t][p], fp32 across the chunks
+  float Ht[kP / 2];  // H^T[n = r][p = 32 hf ..], fp32 across the chunks
 #pragma unroll
-  for (int q = 0; q < kP; ++q) Ht[q] = 0.0f;
+  for (int q = 0; q < kP / 2; ++q) Ht[q] = 0.0f;
   unsigned phase = 0;
   const int nch = (L + kQ - 1) / kQ;
-  const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+  ChunkIn in;
+  fetch(0, in);
 
 #pragma unroll 1
   for (int c = 0; c < nch; ++c) {
-    const int tok = c * kQ + t;
+    const int tok = c * kQ + r;
     const bool valid = tok < L;
-    // ---- this token: dt, document start, C and B rows, x row ----
+    // ---- this chunk's operands into shared memory ----
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      *reinterpret_cast<uint4*>(sm.C + tile_off(r, 8 * (8 * hf + k))) = in.c[k];
+      *reinterpret_cast<uint4*>(sm.Bm + tile_off(r, 8 * (8 * hf + k))) = in.b[k];
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      *reinterpret_cast<uint4*>(sm.Xt + tile_off_mn(8 * (4 * hf + k), r)) = in.x[k];
+    uint4 braw[8], xraw[4];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) braw[k] = in.b[k];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) xraw[k] = in.x[k];
     float dt = 0.0f;
-    bool start = false;
-    if (valid) {
-      const float v = __bfloat162float(dtg[((size_t)b * L + tok) * H + h]) + bias;
-      dt = p.softplus ? (v > 20.0f ? v : log1pf(expf(v))) : v;
-      if (seqb && tok > 0) start = __ldg(seqb + tok) != __ldg(seqb + tok - 1);
-    }
-    const uint4* crow = reinterpret_cast<const uint4*>(Cg + (((size_t)b * L + tok) * G + g) * kNs);
-    const uint4* brow = reinterpret_cast<const uint4*>(Bg + (((size_t)b * L + tok) * G + g) * kNs);
-    uint4 braw[16];
-#pragma unroll
-    for (int k8 = 0; k8 < 16; ++k8) {
-      *reinterpret_cast<uint4*>(sm.C + tile_off(t, 8 * k8)) = valid ? __ldg(crow + k8) : z4;
-      braw[k8] = valid ? __ldg(brow + k8) : z4;
-      *reinterpret_cast<uint4*>(sm.Bm + tile_off(t, 8 * k8)) = braw[k8];
-    }
-    const uint4* xrow = reinterpret_cast<const uint4*>(xg + (((size_t)b * L + tok) * H + h) * kP);
-    uint4 xraw[8];
-#pragma unroll
-    for (int k8 = 0; k8 < 8; ++k8) {
-      xraw[k8] = valid ? __ldg(xrow + k8) : z4;
-      *reinterpret_cast<uint4*>(sm.Xt + tile_off_mn(8 * k8, t)) = xraw[k8];  // p = 8 k8 .. 8 k8 + 7
-    }
-    // ---- chunk scans: lcs = inclusive sum of dt A, ls = last document start ----
+    if (valid) dt = p.softplus ? (in.dtv > 20.0f ? in.dtv : log1pf(expf(in.dtv))) : in.dtv;
+    const bool start = valid && seqb && tok > 0 && in.seq_cur != in.seq_prev;
+    // the next chunk's inputs are in flight while this one is computed
+    if (c + 1 < nch) fetch(c + 1, in);
+    // ---- chunk scans (warps 0-3): lcs = inclusive sum of dt A, ls = last document start ----
     float la = dt * Ah;
-    int st = start ? t : -1;
+    int st = start ? r : -1;
+    if (hf == 0) {
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const float lo = __shfl_up_sync(kFull, la, off);
-      const int so = __shfl_up_sync(kFull, st, off);
-      if (lane >= off) {
-        la += lo;
-        st = max(st, so);
+      for (int off = 1; off < 32; off <<= 1) {
+        const float lo = __shfl_up_sync(kFull, la, off);
+        const int so = __shfl_up_sync(kFull, st, off);
+        if (lane >= off) {
+          la += lo;
+          st = max(st, so);
+        }
+      }
+      if (lane == 31) {
+        sm.wsum[warp] = la;
+        sm.wmax[warp] = st;
       }
     }
-    if (lane == 31) {
-      sm.wsum[warp] = la;
-      sm.wmax[warp] = st;
+    __syncthreads();
+    if (hf == 0) {
+      for (int w = 0; w < warp; ++w) {
+        la += sm.wsum[w];
+        st = max(st, sm.wmax[w]);
+      }
+      sm.lcs[r] = la;
+      sm.dt[r] = dt;
+      sm.ls[r] = st;
     }
     __syncthreads();
-    for (int w = 0; w < warp; ++w) {
-      la += sm.wsum[w];
-      st = max(st, sm.wmax[w]);
-    }
-    sm.lcs[t] = la;
-    sm.dt[t] = dt;
-    sm.ls[t] = st;
-    __syncthreads();
+    la = sm.lcs[r];
+    st = sm.ls[r];
     const float lcsQ = sm.lcs[kQ - 1];
     const int lsQ = sm.ls[kQ - 1];
-    // ---- B scaled by w_t = dt_t exp(lcs_Q-1 - lcs_t) [t >= ls_Q-1], as [n][t] ----
-    const float wt = (t >= lsQ) ? dt * __expf(lcsQ - la) : 0.0f;
+    // ---- B scaled by w_r = dt_r exp(lcs_Q-1 - lcs_r) [r >= ls_Q-1], MN-major ----
+    const float wt = (r >= lsQ) ? dt * __expf(lcsQ - la) : 0.0f;
 #pragma unroll
-    for (int k8 = 0; k8 < 16; ++k8) {  // n = 8 k8 .. 8 k8 + 7 of token t
-      const uint4 q = braw[k8];
-      *reinterpret_cast<uint4*>(sm.Bw + tile_off_mn(8 * k8, t)) =
+    for (int k = 0; k < 8; ++k) {  // n = 8 (8 hf + k) .. of token r
+      const uint4 q = braw[k];
+      *reinterpret_cast<uint4*>(sm.Bw + tile_off_mn(8 * (8 * hf + k), r)) =
           make_uint4(pack_bf16(bf_lo(q.x) * wt, bf_hi(q.x) * wt), pack_bf16(bf_lo(q.y) * wt, bf_hi(q.y) * wt),
                      pack_bf16(bf_lo(q.z) * wt, bf_hi(q.z) * wt), pack_bf16(bf_lo(q.w) * wt, bf_hi(q.w) * wt));
     }
@@ -248,40 +279,38 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
     phase ^= 1u;
     if (!__syncthreads_and(ok)) break;
     tc_fence_after();
-    // ---- row t of M = (C B^T o L) dt, and row t of C' ----
-    {
-      const float lcs_i = la;
-      const int ls_i = st;
+    // ---- columns 64 hf .. 64 hf + 63 of row r of M = (C B^T o L) dt (pair hi / lo), row r of C' ----
 #pragma unroll 1
-      for (int j0 = 0; j0 < kQ; j0 += 32) {
-        float v[32];
-        tmem_ld32(lane_row + j0, v);
+    for (int j0 = 64 * hf; j0 < 64 * hf + 64; j0 += 32) {
+      float v[32];
+      tmem_ld32(lane_row + j0, v);
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          float m[8], r[8];
+      for (int e = 0; e < 32; e += 8) {
+        float m[8], rr[8];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int j = j0 + e + q;
-            m[q] = (j >= ls_i && j <= t) ? v[e + q] * __expf(lcs_i - sm.lcs[j]) * sm.dt[j] : 0.0f;
-          }
-          const uint4 hi = make_uint4(pack_bf16(m[0], m[1]), pack_bf16(m[2], m[3]), pack_bf16(m[4], m[5]),
-                                      pack_bf16(m[6], m[7]));
-          const uint32_t hw[4] = {hi.x, hi.y, hi.z, hi.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            r[2 * q] = m[2 * q] - bf_lo(hw[q]);
-            r[2 * q + 1] = m[2 * q + 1] - bf_hi(hw[q]);
-          }
-          *reinterpret_cast<uint4*>(sm.M + tile_off(t, j0 + e)) = hi;
-          *reinterpret_cast<uint4*>(sm.Mlo + tile_off(t, j0 + e)) =
-              make_uint4(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]), pack_bf16(r[4], r[5]),
-                         pack_bf16(r[6], r[7]));
+        for (int q = 0; q < 8; ++q) {
+          const int j = j0 + e + q;
+          m[q] = (j >= st && j <= r) ? v[e + q] * __expf(la - sm.lcs[j]) * sm.dt[j] : 0.0f;
         }
-      }
-      const float cs = ls_i < 0 ? __expf(lcs_i) : 0.0f;
+        const uint4 hi = make_uint4(pack_bf16(m[0], m[1]), pack_bf16(m[2], m[3]), pack_bf16(m[4], m[5]),
+                                    pack_bf16(m[6], m[7]));
+        const uint32_t hw[4] = {hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
-      for (int k8 = 0; k8 < 16; ++k8) {
-        uint4* q = reinterpret_cast<uint4*>(sm.C + tile_off(t, 8 * k8));
+        for (int q = 0; q < 4; ++q) {
+          rr[2 * q] = m[2 * q] - bf_lo(hw[q]);
+          rr[2 * q + 1] = m[2 * q + 1] - bf_hi(hw[q]);
+        }
+        *reinterpret_cast<uint4*>(sm.M + tile_off(r, j0 + e)) = hi;
+        *reinterpret_cast<uint4*>(sm.Mlo + tile_off(r, j0 + e)) =
+            make_uint4(pack_bf16(rr[0], rr[1]), pack_bf16(rr[2], rr[3]), pack_bf16(rr[4], rr[5]),
+                       pack_bf16(rr[6], rr[7]));
+      }
+    }
+    {
+      const float cs = st < 0 ? __expf(la) : 0.0f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        uint4* q = reinterpret_cast<uint4*>(sm.C + tile_off(r, 8 * (8 * hf + k)));
         const uint4 cv = *q;
         *q = make_uint4(pack_bf16(bf_lo(cv.x) * cs, bf_hi(cv.x) * cs), pack_bf16(bf_lo(cv.y) * cs, bf_hi(cv.y) * cs),
                         pack_bf16(bf_lo(cv.z) * cs, bf_hi(cv.z) * cs), pack_bf16(bf_lo(cv.w) * cs, bf_hi(cv.w) * cs));
@@ -303,42 +332,42 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
     phase ^= 1u;
     if (!__syncthreads_and(ok)) break;
     tc_fence_after();
-    // ---- y row t; the state row n = t ----
+    // ---- y row r (p = 32 hf ..); the state row n = r (p = 32 hf ..) ----
     {
-      float yv[kP];
-      tmem_ld32(lane_row + 128, yv);
-      tmem_ld32(lane_row + 160, yv + 32);
+      float yv[32];
+      tmem_ld32(lane_row + 128 + 32 * hf, yv);
       if (valid) {
-        uint4* yrow = reinterpret_cast<uint4*>(yg + (((size_t)b * L + tok) * H + h) * kP);
+        uint4* yrow = reinterpret_cast<uint4*>(yg + (((size_t)b * L + tok) * H + h) * kP) + 4 * hf;
 #pragma unroll
-        for (int k8 = 0; k8 < 8; ++k8) {
-          const uint32_t w4[4] = {xraw[k8].x, xraw[k8].y, xraw[k8].z, xraw[k8].w};
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t w4[4] = {xraw[k].x, xraw[k].y, xraw[k].z, xraw[k].w};
           uint32_t o[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int q = 8 * k8 + 2 * e;
+            const int q = 8 * k + 2 * e;
             o[e] = pack_bf16(fmaf(Dh, bf_lo(w4[e]), yv[q]), fmaf(Dh, bf_hi(w4[e]), yv[q + 1]));
           }
-          yrow[k8] = make_uint4(o[0], o[1], o[2], o[3]);
+          yrow[k] = make_uint4(o[0], o[1], o[2], o[3]);
         }
       }
-      float sv[kP];
-      tmem_ld32(lane_row + 192, sv);
-      tmem_ld32(lane_row + 224, sv + 32);
+      float sv[32];
+      tmem_ld32(lane_row + 192 + 32 * hf, sv);
       const float dec = lsQ < 0 ? __expf(lcsQ) : 0.0f;
 #pragma unroll
-      for (int q = 0; q < kP; ++q) Ht[q] = fmaf(dec, Ht[q], sv[q]);
+      for (int q = 0; q < kP / 2; ++q) Ht[q] = fmaf(dec, Ht[q], sv[q]);
 #pragma unroll
-      for (int k8 = 0; k8 < 8; ++k8)  // p = 8 k8 .. 8 k8 + 7 of state row n = t
-        *reinterpret_cast<uint4*>(sm.Hb + tile_off_mn(8 * k8, t)) =
-            make_uint4(pack_bf16(Ht[8 * k8], Ht[8 * k8 + 1]), pack_bf16(Ht[8 * k8 + 2], Ht[8 * k8 + 3]),
-                       pack_bf16(Ht[8 * k8 + 4], Ht[8 * k8 + 5]), pack_bf16(Ht[8 * k8 + 6], Ht[8 * k8 + 7]));
+      for (int k = 0; k < 4; ++k)  // p = 8 (4 hf + k) .. of state row n = r
+        *reinterpret_cast<uint4*>(sm.Hb + tile_off_mn(8 * (4 * hf + k), r)) =
+            make_uint4(pack_bf16(Ht[8 * k], Ht[8 * k + 1]), pack_bf16(Ht[8 * k + 2], Ht[8 * k + 3]),
+                       pack_bf16(Ht[8 * k + 4], Ht[8 * k + 5]), pack_bf16(Ht[8 * k + 6], Ht[8 * k + 7]));
     }
     tc_fence_before();
+    __syncthreads();  // every thread is done with this chunk's shared operands and TMEM
   }
   if (p.final_state) {
 #pragma unroll
-    for (int q = 0; q < kP; ++q) p.final_state[(((size_t)b * H + h) * kP + q) * kNs + t] = Ht[q];
+    for (int q = 0; q < kP / 2; ++q)
+      p.final_state[(((size_t)b * H + h) * kP + 32 * hf + q) * kNs + r] = Ht[q];
   }
   tc_fence_before();
   __syncthreads();

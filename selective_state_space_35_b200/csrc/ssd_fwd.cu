@@ -103,9 +103,9 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 32 consecutive fp32 columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld32(uint32_t addr, float v[32]) {
-  uint32_t r[32];
+// 32 consecutive fp32 columns of this thread's TMEM lane (the values are
+// valid after tmem_wait()).
+__device__ __forceinline__ void tmem_ld32(uint32_t addr, uint32_t r[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
       "%13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
@@ -115,10 +115,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t addr, float v[32]) {
         "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
         "=r"(r[30]), "=r"(r[31])
       : "r"(addr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 }
+__device__ __forceinline__ void tmem_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -280,17 +278,21 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
     if (!__syncthreads_and(ok)) break;
     tc_fence_after();
     // ---- columns 64 hf .. 64 hf + 63 of row r of M = (C B^T o L) dt (pair hi / lo), row r of C' ----
-#pragma unroll 1
-    for (int j0 = 64 * hf; j0 < 64 * hf + 64; j0 += 32) {
-      float v[32];
-      tmem_ld32(lane_row + j0, v);
+    uint32_t sraw[64];
+    tmem_ld32(lane_row + 64 * hf, sraw);
+    tmem_ld32(lane_row + 64 * hf + 32, sraw + 32);
+    tmem_wait();
+#pragma unroll
+    for (int jj = 0; jj < 64; jj += 32) {
+      const int j0 = 64 * hf + jj;
+      const uint32_t* v = sraw + jj;
 #pragma unroll
       for (int e = 0; e < 32; e += 8) {
         float m[8], rr[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
           const int j = j0 + e + q;
-          m[q] = (j >= st && j <= r) ? v[e + q] * __expf(la - sm.lcs[j]) * sm.dt[j] : 0.0f;
+          m[q] = (j >= st && j <= r) ? __uint_as_float(v[e + q]) * __expf(la - sm.lcs[j]) * sm.dt[j] : 0.0f;
         }
         const uint4 hi = make_uint4(pack_bf16(m[0], m[1]), pack_bf16(m[2], m[3]), pack_bf16(m[4], m[5]),
                                     pack_bf16(m[6], m[7]));
@@ -334,8 +336,10 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
     tc_fence_after();
     // ---- y row r (p = 32 hf ..); the state row n = r (p = 32 hf ..) ----
     {
-      float yv[32];
+      uint32_t yv[32], sv[32];
       tmem_ld32(lane_row + 128 + 32 * hf, yv);
+      tmem_ld32(lane_row + 192 + 32 * hf, sv);
+      tmem_wait();
       if (valid) {
         uint4* yrow = reinterpret_cast<uint4*>(yg + (((size_t)b * L + tok) * H + h) * kP) + 4 * hf;
 #pragma unroll
@@ -345,16 +349,15 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int q = 8 * k + 2 * e;
-            o[e] = pack_bf16(fmaf(Dh, bf_lo(w4[e]), yv[q]), fmaf(Dh, bf_hi(w4[e]), yv[q + 1]));
+            o[e] = pack_bf16(fmaf(Dh, bf_lo(w4[e]), __uint_as_float(yv[q])),
+                             fmaf(Dh, bf_hi(w4[e]), __uint_as_float(yv[q + 1])));
           }
           yrow[k] = make_uint4(o[0], o[1], o[2], o[3]);
         }
       }
-      float sv[32];
-      tmem_ld32(lane_row + 192 + 32 * hf, sv);
       const float dec = lsQ < 0 ? __expf(lcsQ) : 0.0f;
 #pragma unroll
-      for (int q = 0; q < kP / 2; ++q) Ht[q] = fmaf(dec, Ht[q], sv[q]);
+      for (int q = 0; q < kP / 2; ++q) Ht[q] = fmaf(dec, Ht[q], __uint_as_float(sv[q]));
 #pragma unroll
       for (int k = 0; k < 4; ++k)  // p = 8 (4 hf + k) .. of state row n = r
         *reinterpret_cast<uint4*>(sm.Hb + tile_off_mn(8 * (4 * hf + k), r)) =

@@ -309,3 +309,31 @@ def test_deterministic_backward_workspace(ssm):
     g.workspace, g.workspace_bytes = fake + (1 << 24) + 16, 1 << 30
     assert L.ssm_scan_bwd(ctypes.byref(p), ctypes.byref(g), None) == 1  # misaligned
     assert "aligned" in ssm.ssm_last_error()
+
+
+def test_ssd_param_validation(ssm):
+    """ssm_ssd_fwd rejects bad arguments before any launch: struct size, sizes,
+    groups that do not divide the heads, fp32 storage, P / N other than 64 /
+    128, NULL and misaligned pointers."""
+    from selective_state_space_35_b200 import _lib
+    L = _lib.load()
+    fake = 1 << 20
+
+    def params(**kw):
+        p = ssm.ssm_ssd_params()
+        p.struct_size = ctypes.sizeof(ssm.ssm_ssd_params)
+        p.B, p.L, p.H, p.P, p.G, p.N = 1, 256, 4, 64, 2, 128
+        p.dtype = 1
+        p.x, p.dt_raw, p.A, p.Bm, p.Cm, p.y = fake, fake + 4096, fake + 8192, fake + 12288, \
+            fake + 16384, fake + 20480
+        p.dt_softplus = 1
+        for k, v in kw.items():
+            setattr(p, k, v)
+        return p
+
+    for kw, status in [(dict(struct_size=3), 1), (dict(B=0), 1), (dict(G=3), 1), (dict(dtype=0), 2),
+                       (dict(P=32), 2), (dict(N=64), 2), (dict(x=None), 1), (dict(y=fake + 8), 1),
+                       (dict(A=fake + 2), 1)]:
+        p = params(**kw)
+        assert L.ssm_ssd_fwd(ctypes.byref(p), None) == status, kw
+        assert ssm.ssm_last_error()

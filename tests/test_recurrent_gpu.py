@@ -197,3 +197,56 @@ def test_decode_continues_gpu_prefill():
     assert rel_l2(got, full["out"][..., s:]) <= TOL_F32
     # the state was advanced in place through the last token
     assert rel_l2(host64(fs), full["final_state"]) <= TOL_F32
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_many_tiles_parity(dtype):
+    """B * D = 130 * 1000 rows: 1016 CTAs of 128 rows (the last one half
+    full), several waves on 148 SMs. 3 steps against the oracle."""
+    B, D, N, steps = 130, 1000, 16, 3
+    di = synth.decode_inputs(B, D, N, steps, dtype, 7350 + int(dtype == "bf16"))
+    go, gu, gcs, gh = _run_decode_gpu(di, B, D, N, steps)
+    wo, wu, wcs, wh = _run_decode_oracle(di, steps)
+    fp32 = dtype == "f32"
+    tol = TOL_F32 if fp32 else TOL_BF16_OUT
+    for t in range(steps):
+        w_o = wo[t] if fp32 else oracle.round_bf16(wo[t])
+        w_u = wu[t] if fp32 else oracle.round_bf16(wu[t])
+        assert rel_l2(go[t], w_o) <= tol, (t, rel_l2(go[t], w_o))
+        assert rel_l2(gu[t], w_u) <= tol
+    # every row's state, not only the whole-array norm
+    err = np.abs(gh - wh).max(axis=-1) / np.maximum(np.abs(wh).max(axis=-1), 1e-3)
+    assert err.max() <= (1e-5 if fp32 else 2e-3), err.max()
+    np.testing.assert_array_equal(gcs, wcs)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_vector_equals_scalar_access(dtype):
+    """N = 16 with the state 16-byte aligned takes the kernel's 16-byte
+    state accesses; the same state one float off that alignment takes its
+    scalar accesses. Both do the same operations per row in the same order:
+    outputs, conv window and state bitwise equal over 4 steps."""
+    import torch
+    ssm = _ssm()
+    B, D, N, steps = 7, 300, 16, 4
+    di = synth.decode_inputs(B, D, N, steps, dtype, 7360 + int(dtype == "bf16"))
+    dev = "cuda"
+    x, dl, z = to_dev(di.x, dev), to_dev(di.delta, dev), to_dev(di.z, dev)
+    Bm, Cm = to_dev(di.Bm, dev), to_dev(di.Cm, dev)
+    kw = dict(conv_bias=f32_dev(di.conv_b, dev), Dskip=f32_dev(di.Dskip, dev),
+              delta_bias=f32_dev(di.delta_bias, dev))
+    A, w = f32_dev(di.A, dev), f32_dev(di.conv_w, dev)
+    h0 = f32_dev(di.h0, dev)
+    runs = []
+    for off in (0, 1):
+        buf = torch.zeros(B * D * N + 4, dtype=torch.float32, device=dev)
+        st = buf[off:off + B * D * N].view(B, D, N)
+        st.copy_(h0)
+        assert (st.data_ptr() % 16 == 0) == (off == 0)
+        cs = to_dev(di.conv_state, dev).contiguous()
+        outs = [ssm.decode_step(x[t], cs, w, dl[t], A, Bm[t], Cm[t], st, z=z[t], **kw).clone()
+                for t in range(steps)]
+        torch.cuda.synchronize()
+        runs.append((torch.stack(outs), cs.clone(), st.clone()))
+    for a, b in zip(runs[0], runs[1]):
+        assert torch.equal(a, b)

@@ -79,7 +79,7 @@ typedef enum { SSM_DTYPE_F32 = 0, SSM_DTYPE_BF16 = 1 } ssm_dtype_t;
 const char* ssm_last_error(void);
 
 /* ABI version of this header (bumped on any incompatible change). */
-#define SSM_ABI_VERSION 6
+#define SSM_ABI_VERSION 7
 int ssm_abi_version(void);
 
 /* ---------------------------------------------------------------------------
@@ -428,6 +428,9 @@ ssm_status_t ssm_decode_step(const ssm_decode_params* p, ssm_stream_t stream);
  * Supported: dtype bf16, P = 64, N = 128, G >= 1 dividing H, any L >= 1
  * (else SSM_ERR_UNSUPPORTED); every pointer 16-byte aligned. One CTA per
  * (b, h); the chunks of a row run in order inside it.
+ * chunk_states (nullable; required by ssm_ssd_bwd): [B][H][nc][N][P] fp32
+ * with nc = ceil(L / 128), the state entering each chunk (S_{128c-1}
+ * stored [n][p]; zeros for chunk 0); caller-owned, written by this call.
  * ------------------------------------------------------------------------ */
 typedef struct {
     size_t struct_size;        /* = sizeof(ssm_ssd_params) */
@@ -446,9 +449,50 @@ typedef struct {
     float* final_state;
     int* status;               /* device int, nullable: SSM_ERR_TIMEOUT if a bounded wait for
                                   the tensor cores gave up (outputs then invalid) */
+    float* chunk_states;       /* [B][H][ceil(L/128)][N][P] fp32, nullable (see above) */
 } ssm_ssd_params;
 
 ssm_status_t ssm_ssd_fwd(const ssm_ssd_params* p, ssm_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * ssm_ssd_bwd — reverse mode of ssm_ssd_fwd (same section of "hung-phan
+ * ml-skills mamba"), given dy = dL/dy and the chunk_states the forward wrote
+ * for the same inputs (no gradient enters through the final state). With
+ * G_t[p][n] = dL/dS_t (G_t = dy_t[p] C_t[n] + a_{t+1} G_{t+1}):
+ *   dx[b][t][h][p] = D[h] dy_t[p] + dt_t sum_n G_t[p][n] B_t[n]
+ *   d dt_t = sum_{p,n} G_t[p][n] (x_t[p] B_t[n] + a_t A[h] S_{t-1}[p][n])
+ *   dA[h]  = sum over b, t of dt_t sum_{p,n} G_t[p][n] a_t S_{t-1}[p][n]
+ *   dB[b][t][g][n] = sum over the group's heads of dt_t sum_p G_t[p][n] x_t[p]
+ *   dC[b][t][g][n] = sum over the group's heads of sum_p dy_t[p] S_t[p][n]
+ *   dD[h] = sum dy x;  d dt_raw = d dt sigmoid(dt_raw + dt_bias) with the
+ *   softplus (else d dt);  d dt_bias[h] = sum over b, t of d dt_raw.
+ * Per chunk of 128 tokens, in reverse order, the transposed masked products
+ * (dy x^T, M^T dy, dS B, dS^T C, C^T dy, ...) run on the tensor cores with
+ * bf16 operands and fp32 accumulation; the state adjoint carried between
+ * chunks is fp32 and enters the products rounded to bf16.
+ *   p: the forward's parameters (y, final_state ignored), with chunk_states
+ *      non-NULL and as the forward wrote it.
+ *   dy, dx    [B][L][H][P] bf16        ddt_raw   [B][L][H] fp32
+ *   dB, dC    [B][L][G][N] fp32        dA        [H] fp32
+ *   dD, ddt_bias [H] fp32, nullable
+ * Outputs are overwritten (the call zeroes dA, dB, dC, dD, ddt_bias, then
+ * adds each head's share with fp32 atomics: not bitwise reproducible).
+ * Same support and alignment rules as ssm_ssd_fwd; dx, dy, dB, dC 16-byte
+ * aligned. Errors and the status word as for ssm_ssd_fwd.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    size_t struct_size;        /* = sizeof(ssm_ssd_grads) */
+    const void* dy;
+    void* dx;
+    float* ddt_raw;
+    float* dA;
+    float* dB;
+    float* dC;
+    float* dD;
+    float* ddt_bias;
+} ssm_ssd_grads;
+
+ssm_status_t ssm_ssd_bwd(const ssm_ssd_params* p, const ssm_ssd_grads* g, ssm_stream_t stream);
 
 #ifdef __cplusplus
 }

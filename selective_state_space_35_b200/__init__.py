@@ -22,14 +22,15 @@ from ._lib import (SsmError, ssm_abi_version, ssm_conv1d_bwd, ssm_conv1d_bwd_noa
                    ssm_probe_ex2_rate, ssm_scan_bwd, ssm_scan_status,
                    ssm_scan_fwd, ssm_scan_grads, ssm_scan_params, ssm_scan_workspace_size,
                    ssm_scan_bwd_workspace_size, ssm_ssd_params, ssm_ssd_fwd,
-                   ssm_scan_fwd_summary, ssm_scan_bwd_summary, ssm_state_carry,
+                   ssm_ssd_grads, ssm_ssd_bwd, ssm_scan_fwd_summary, ssm_scan_bwd_summary, ssm_state_carry,
                    ssm_conv1d_fwd_ctx, ssm_conv1d_bwd_ctx)
 
 __all__ = [
     "SsmError", "ssm_abi_version", "ssm_last_error", "ssm_conv1d_fwd", "ssm_conv1d_bwd",
     "ssm_conv1d_bwd_workspace_size", "ssm_conv1d_bwd_noalloc", "ssm_scan_workspace_size", "ssm_scan_fwd", "ssm_scan_bwd",
     "ssm_scan_params", "ssm_scan_grads", "ssm_scan_bwd_workspace_size", "ssm_ssd_params",
-    "ssm_ssd_fwd", "ssd_fwd", "ssm_probe_ex2_rate", "probe_ex2_rate", "ssm_scan_status",
+    "ssm_ssd_fwd", "ssd_fwd", "ssm_ssd_grads", "ssm_ssd_bwd", "ssd_bwd", "ssd_chunk_states_shape",
+    "ssm_probe_ex2_rate", "probe_ex2_rate", "ssm_scan_status",
     "scan_status", "conv1d_fwd", "conv1d_bwd", "scan_params",
     "scan_workspace_size", "scan_fwd", "scan_bwd", "load",
     "ssm_decode_params", "ssm_decode_step", "decode_step", "ssm_conv1d_scan_fwd",
@@ -465,13 +466,16 @@ def state_carry(decay, value, r, *, reverse=False, init=None, seq_prev=None, seq
     return out
 
 
-def ssd_fwd(x, dt_raw, A, Bm, Cm, *, D=None, dt_bias=None, softplus=True, seq_idx=None,
-            return_final_state=False, out=None, status=None, stream=None):
-    """Mamba-2 SSD forward on the tensor cores.
+SSD_CHUNK = 128  # tokens per chunk of the SSD kernels
 
-    x [B, L, H, 64] bf16; dt_raw [B, L, H] bf16; Bm, Cm [B, L, G, 128] bf16;
-    A, D, dt_bias [H] fp32; seq_idx [B, L] int32. Returns (y [B, L, H, 64]
-    bf16, final_state [B, H, 64, 128] fp32 or None)."""
+
+def ssd_chunk_states_shape(B, L, H, P=64, N=128):
+    """Shape of the per-chunk entering states the SSD forward saves for the
+    backward: [B, H, ceil(L / 128), N, P] fp32."""
+    return (B, H, (L + SSD_CHUNK - 1) // SSD_CHUNK, N, P)
+
+
+def _ssd_params(x, dt_raw, A, Bm, Cm, D, dt_bias, softplus, seq_idx, status, chunk_states):
     torch = _torch()
     B, L, H, P = x.shape
     G, N = Bm.shape[2], Bm.shape[3]
@@ -483,10 +487,7 @@ def ssd_fwd(x, dt_raw, A, Bm, Cm, *, D=None, dt_bias=None, softplus=True, seq_id
     _need(D, "D", torch.float32, (H,))
     _need(dt_bias, "dt_bias", torch.float32, (H,))
     _need(seq_idx, "seq_idx", torch.int32, (B, L))
-    y = torch.empty_like(x) if out is None else out
-    _need(y, "out", torch.bfloat16, (B, L, H, P))
-    fs = (torch.empty((B, H, P, N), dtype=torch.float32, device=x.device)
-          if return_final_state else None)
+    _need(chunk_states, "chunk_states", torch.float32, ssd_chunk_states_shape(B, L, H, P, N))
     p = ssm_ssd_params()
     p.struct_size = ctypes.sizeof(ssm_ssd_params)
     p.B, p.L, p.H, p.P, p.G, p.N = B, L, H, P, G, N
@@ -497,8 +498,58 @@ def ssd_fwd(x, dt_raw, A, Bm, Cm, *, D=None, dt_bias=None, softplus=True, seq_id
     p.dt_bias = dt_bias.data_ptr() if dt_bias is not None else None
     p.dt_softplus = 1 if softplus else 0
     p.seq_idx = seq_idx.data_ptr() if seq_idx is not None else None
+    p.status = status.data_ptr() if status is not None else None
+    p.chunk_states = chunk_states.data_ptr() if chunk_states is not None else None
+    return p
+
+
+def ssd_fwd(x, dt_raw, A, Bm, Cm, *, D=None, dt_bias=None, softplus=True, seq_idx=None,
+            return_final_state=False, chunk_states=None, out=None, status=None, stream=None):
+    """Mamba-2 SSD forward on the tensor cores.
+
+    x [B, L, H, 64] bf16; dt_raw [B, L, H] bf16; Bm, Cm [B, L, G, 128] bf16;
+    A, D, dt_bias [H] fp32; seq_idx [B, L] int32. chunk_states: a tensor of
+    ssd_chunk_states_shape(B, L, H) fp32 to receive the state entering each
+    chunk (what ssd_bwd needs), or None. Returns (y [B, L, H, 64] bf16,
+    final_state [B, H, 64, 128] fp32 or None)."""
+    torch = _torch()
+    B, L, H, P = x.shape
+    N = Bm.shape[3]
+    p = _ssd_params(x, dt_raw, A, Bm, Cm, D, dt_bias, softplus, seq_idx, status, chunk_states)
+    y = torch.empty_like(x) if out is None else out
+    _need(y, "out", torch.bfloat16, (B, L, H, P))
+    fs = (torch.empty((B, H, P, N), dtype=torch.float32, device=x.device)
+          if return_final_state else None)
     p.y = y.data_ptr()
     p.final_state = fs.data_ptr() if fs is not None else None
-    p.status = status.data_ptr() if status is not None else None
     _lib.check(ssm_ssd_fwd(p, _stream(stream, x.device)))
     return y, fs
+
+
+def ssd_bwd(x, dt_raw, A, Bm, Cm, dy, chunk_states, *, D=None, dt_bias=None, softplus=True,
+            seq_idx=None, status=None, stream=None):
+    """Backward of ssd_fwd from dy [B, L, H, 64] bf16 and the chunk_states the
+    forward saved for the same inputs. Returns dict(dx [B, L, H, 64] bf16,
+    ddt_raw [B, L, H] fp32, dA [H], dB, dC [B, L, G, 128] fp32, dD [H] or
+    None, ddt_bias [H] or None)."""
+    torch = _torch()
+    B, L, H, P = x.shape
+    G, N = Bm.shape[2], Bm.shape[3]
+    if chunk_states is None:
+        raise ValueError("ssd_bwd needs the chunk_states written by ssd_fwd")
+    p = _ssd_params(x, dt_raw, A, Bm, Cm, D, dt_bias, softplus, seq_idx, status, chunk_states)
+    _need(dy, "dy", torch.bfloat16, (B, L, H, P))
+    f32 = dict(dtype=torch.float32, device=x.device)
+    out = {"dx": torch.empty_like(x), "ddt_raw": torch.empty((B, L, H), **f32),
+           "dA": torch.empty((H,), **f32), "dB": torch.empty((B, L, G, N), **f32),
+           "dC": torch.empty((B, L, G, N), **f32),
+           "dD": torch.empty((H,), **f32) if D is not None else None,
+           "ddt_bias": torch.empty((H,), **f32) if dt_bias is not None else None}
+    g = ssm_ssd_grads()
+    g.struct_size = ctypes.sizeof(ssm_ssd_grads)
+    g.dy, g.dx, g.ddt_raw = dy.data_ptr(), out["dx"].data_ptr(), out["ddt_raw"].data_ptr()
+    g.dA, g.dB, g.dC = out["dA"].data_ptr(), out["dB"].data_ptr(), out["dC"].data_ptr()
+    g.dD = out["dD"].data_ptr() if out["dD"] is not None else None
+    g.ddt_bias = out["ddt_bias"].data_ptr() if out["ddt_bias"] is not None else None
+    _lib.check(ssm_ssd_bwd(p, g, _stream(stream, x.device)))
+    return out

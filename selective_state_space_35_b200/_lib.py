@@ -71,6 +71,15 @@ class ssm_ssd_params(ctypes.Structure):
         ("x", _vp), ("dt_raw", _vp), ("A", _vp), ("Bm", _vp), ("Cm", _vp),
         ("D", _vp), ("dt_bias", _vp), ("dt_softplus", _i), ("seq_idx", _vp),
         ("y", _vp), ("final_state", _vp), ("status", _vp),
+        ("chunk_states", _vp),
+    ]
+
+
+class ssm_ssd_grads(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", _sz),
+        ("dy", _vp), ("dx", _vp), ("ddt_raw", _vp), ("dA", _vp),
+        ("dB", _vp), ("dC", _vp), ("dD", _vp), ("ddt_bias", _vp),
     ]
 
 
@@ -93,7 +102,8 @@ EXPORTS = ("ssm_last_error", "ssm_abi_version", "ssm_conv1d_fwd", "ssm_conv1d_bw
            "ssm_conv1d_bwd", "ssm_conv1d_bwd_noalloc", "ssm_scan_workspace_size", "ssm_scan_fwd",
            "ssm_scan_bwd", "ssm_scan_bwd_workspace_size", "ssm_scan_status", "ssm_probe_ex2_rate", "ssm_decode_step",
            "ssm_conv1d_scan_fwd", "ssm_scan_fwd_summary", "ssm_scan_bwd_summary",
-           "ssm_state_carry", "ssm_conv1d_fwd_ctx", "ssm_conv1d_bwd_ctx", "ssm_ssd_fwd")
+           "ssm_state_carry", "ssm_conv1d_fwd_ctx", "ssm_conv1d_bwd_ctx", "ssm_ssd_fwd",
+           "ssm_ssd_bwd")
 
 
 def load(path: str | None = None):
@@ -140,6 +150,8 @@ def load(path: str | None = None):
     L.ssm_decode_step.argtypes = [ctypes.POINTER(ssm_decode_params), _vp]
     L.ssm_ssd_fwd.restype = _i
     L.ssm_ssd_fwd.argtypes = [ctypes.POINTER(ssm_ssd_params), _vp]
+    L.ssm_ssd_bwd.restype = _i
+    L.ssm_ssd_bwd.argtypes = [ctypes.POINTER(ssm_ssd_params), ctypes.POINTER(ssm_ssd_grads), _vp]
     L.ssm_scan_fwd_summary.restype = _i
     L.ssm_scan_fwd_summary.argtypes = [ctypes.POINTER(ssm_scan_params), _vp, _vp, _vp, _vp]
     L.ssm_scan_bwd_summary.restype = _i
@@ -255,3 +267,7 @@ def ssm_conv1d_bwd_ctx(*args) -> int:
 
 def ssm_ssd_fwd(params: ssm_ssd_params, stream) -> int:
     return load().ssm_ssd_fwd(ctypes.byref(params), stream)
+
+
+def ssm_ssd_bwd(params: ssm_ssd_params, grads: ssm_ssd_grads, stream) -> int:
+    return load().ssm_ssd_bwd(ctypes.byref(params), ctypes.byref(grads), stream)

@@ -730,8 +730,12 @@ ssm_status_t ssm_probe_ex2_rate(float* sink, size_t sink_floats, double* ex2_per
 
 
 // ---------------------------------------------------------------------------
-ssm_status_t ssm_ssd_fwd(const ssm_ssd_params* p, ssm_stream_t stream) {
-  if (injected("ssm_ssd_fwd")) return fail(SSM_ERR_INJECTED, "ssm_ssd_fwd: injected failure");
+}  // extern "C"
+
+namespace {
+// Checks shared by the SSD forward and backward: shapes, support, the
+// forward's pointers (y only when `need_y`), alignment.
+ssm_status_t ssd_check(const ssm_ssd_params* p, bool need_y) {
   if (!p) return fail(SSM_ERR_INVALID_ARG, "params is NULL");
   if (p->struct_size != sizeof(ssm_ssd_params))
     return fail(SSM_ERR_INVALID_ARG, "struct_size %zu != %zu", p->struct_size, sizeof(ssm_ssd_params));
@@ -741,16 +745,21 @@ ssm_status_t ssm_ssd_fwd(const ssm_ssd_params* p, ssm_stream_t stream) {
   if (p->dtype != SSM_DTYPE_BF16) return fail(SSM_ERR_UNSUPPORTED, "ssd: bf16 only");
   if (p->P != 64 || p->N != 128)
     return fail(SSM_ERR_UNSUPPORTED, "ssd: P=%d N=%d (supported: P=64, N=128)", p->P, p->N);
-  if (!p->x || !p->dt_raw || !p->A || !p->Bm || !p->Cm || !p->y)
+  if (!p->x || !p->dt_raw || !p->A || !p->Bm || !p->Cm || (need_y && !p->y))
     return fail(SSM_ERR_INVALID_ARG, "x, dt_raw, A, Bm, Cm and y must be non-NULL");
-  const void* v16[] = {p->x, p->Bm, p->Cm, p->y};
+  const void* v16[] = {p->x, p->Bm, p->Cm, need_y ? p->y : nullptr, p->chunk_states};
   for (const void* q : v16)
-    if (!aligned(q, 16)) return fail(SSM_ERR_INVALID_ARG, "ssd: x, Bm, Cm, y must be 16-byte aligned");
+    if (q && !aligned(q, 16))
+      return fail(SSM_ERR_INVALID_ARG, "ssd: x, Bm, Cm, y, chunk_states must be 16-byte aligned");
   const void* v4[] = {p->A, p->D, p->dt_bias, p->seq_idx, p->final_state, p->status};
   for (const void* q : v4)
     if (q && !aligned(q, 4)) return fail(SSM_ERR_INVALID_ARG, "ssd: fp32 / int32 pointer misaligned");
   if (!aligned(p->dt_raw, 2)) return fail(SSM_ERR_INVALID_ARG, "ssd: dt_raw misaligned");
-  ssm::SsdArgs a;
+  return SSM_OK;
+}
+
+ssm::SsdArgs ssd_args(const ssm_ssd_params* p) {
+  ssm::SsdArgs a{};
   a.x = p->x;
   a.dt_raw = p->dt_raw;
   a.A = p->A;
@@ -769,8 +778,48 @@ ssm_status_t ssm_ssd_fwd(const ssm_ssd_params* p, ssm_stream_t stream) {
   a.G = p->G;
   a.N = p->N;
   a.softplus = p->dt_softplus ? 1 : 0;
-  return cuda_status(ssm::launch_ssd_fwd(a, reinterpret_cast<cudaStream_t>(stream)),
+  a.chunk_states = p->chunk_states;
+  return a;
+}
+}  // namespace
+
+extern "C" {
+
+ssm_status_t ssm_ssd_fwd(const ssm_ssd_params* p, ssm_stream_t stream) {
+  if (injected("ssm_ssd_fwd")) return fail(SSM_ERR_INJECTED, "ssm_ssd_fwd: injected failure");
+  const ssm_status_t st = ssd_check(p, true);
+  if (st != SSM_OK) return st;
+  return cuda_status(ssm::launch_ssd_fwd(ssd_args(p), reinterpret_cast<cudaStream_t>(stream)),
                      "ssm_ssd_fwd launch");
+}
+
+ssm_status_t ssm_ssd_bwd(const ssm_ssd_params* p, const ssm_ssd_grads* g, ssm_stream_t stream) {
+  if (injected("ssm_ssd_bwd")) return fail(SSM_ERR_INJECTED, "ssm_ssd_bwd: injected failure");
+  const ssm_status_t st = ssd_check(p, false);
+  if (st != SSM_OK) return st;
+  if (!g) return fail(SSM_ERR_INVALID_ARG, "grads is NULL");
+  if (g->struct_size != sizeof(ssm_ssd_grads))
+    return fail(SSM_ERR_INVALID_ARG, "grads struct_size %zu != %zu", g->struct_size, sizeof(ssm_ssd_grads));
+  if (!p->chunk_states) return fail(SSM_ERR_INVALID_ARG, "ssd bwd: chunk_states (from the forward) is NULL");
+  if (!g->dy || !g->dx || !g->ddt_raw || !g->dA || !g->dB || !g->dC)
+    return fail(SSM_ERR_INVALID_ARG, "ssd bwd: dy, dx, ddt_raw, dA, dB and dC must be non-NULL");
+  const void* v16[] = {g->dy, g->dx, g->dB, g->dC};
+  for (const void* q : v16)
+    if (!aligned(q, 16)) return fail(SSM_ERR_INVALID_ARG, "ssd bwd: dy, dx, dB, dC must be 16-byte aligned");
+  const void* v4[] = {g->ddt_raw, g->dA, g->dD, g->ddt_bias};
+  for (const void* q : v4)
+    if (q && !aligned(q, 4)) return fail(SSM_ERR_INVALID_ARG, "ssd bwd: fp32 pointer misaligned");
+  ssm::SsdArgs a = ssd_args(p);
+  a.dy = g->dy;
+  a.dx = g->dx;
+  a.ddt_raw = g->ddt_raw;
+  a.dA = g->dA;
+  a.dB = g->dB;
+  a.dC = g->dC;
+  a.dD = g->dD;
+  a.ddt_bias = g->ddt_bias;
+  return cuda_status(ssm::launch_ssd_bwd(a, reinterpret_cast<cudaStream_t>(stream)),
+                     "ssm_ssd_bwd launch");
 }
 
 }  // extern "C"

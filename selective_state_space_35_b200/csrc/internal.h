@@ -190,10 +190,21 @@ struct SsdArgs {
   void* y;
   float* final_state;
   int* status;
+  float* chunk_states;  // [B][H][nc][N][P] fp32: the state entering each chunk
   int B, L, H, P, G, N;
   int softplus;
+  // backward only
+  const void* dy;
+  void* dx;
+  float* ddt_raw;
+  float* dA;
+  float* dB;
+  float* dC;
+  float* dD;
+  float* ddt_bias;
 };
 cudaError_t launch_ssd_fwd(const SsdArgs& a, cudaStream_t s);
+cudaError_t launch_ssd_bwd(const SsdArgs& a, cudaStream_t s);
 cudaError_t launch_cu_seqlens_to_seq(const int32_t* cu, int n_docs, int L, int32_t* seq,
                                      cudaStream_t s);
 

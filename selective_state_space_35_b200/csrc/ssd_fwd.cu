@@ -203,6 +203,12 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
   for (int c = 0; c < nch; ++c) {
     const int tok = c * kQ + r;
     const bool valid = tok < L;
+    if (p.chunk_states) {  // the state entering this chunk, for the backward
+      float4* cs = reinterpret_cast<float4*>(p.chunk_states +
+                                             ((((size_t)b * H + h) * nch + c) * kNs + r) * kP + 32 * hf);
+#pragma unroll
+      for (int q = 0; q < kP / 8; ++q) cs[q] = make_float4(Ht[4 * q], Ht[4 * q + 1], Ht[4 * q + 2], Ht[4 * q + 3]);
+    }
     // ---- this chunk's operands into shared memory ----
 #pragma unroll
     for (int k = 0; k < 8; ++k) {

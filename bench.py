@@ -529,9 +529,12 @@ def config_bench(cfg, device, pk, reps=5):
 
 
 def ssd_bench(device, pk, B=2, L=8192, H=64, P=64, G=1, N=128, reps=5):
-    """Mamba-2 SSD forward on the tensor cores at a d_inner = 4096 shape (64
-    heads of 64, one B / C group, state 128), B2 L8192 bf16: CUDA events over
-    `reps` calls after two warm-up calls (inputs 0.28 GB, larger than L2)."""
+    """Mamba-2 SSD forward and backward on the tensor cores at a d_inner =
+    4096 shape (64 heads of 64, one B / C group, state 128), B2 L8192 bf16:
+    CUDA events over `reps` calls after two warm-up calls (inputs 0.28 GB,
+    larger than L2). The forward is timed alone (inference: no saved states)
+    and as the training forward that saves the chunk states; the backward
+    from those states and a seeded dy."""
     import torch
     import selective_state_space_35_b200 as ssm
     si = synth.ssd_inputs(B, L, H, P, G, N, synth.seed_for(11))
@@ -544,29 +547,53 @@ def ssd_bench(device, pk, B=2, L=8192, H=64, P=64, G=1, N=128, reps=5):
 
     x, dtr, Bm, Cm = bf(si.x), bf(si.dt_raw), bf(si.Bm), bf(si.Cm)
     A, D, db = f32(si.A), f32(si.D), f32(si.dt_bias)
+    rng = np.random.Generator(np.random.PCG64(synth.seed_for(12)))
+    dy = torch.from_numpy(synth.f32_to_bf16_bits(rng.standard_normal((B, L, H, P)).astype(np.float32))
+                          .view(np.int16)).view(torch.bfloat16).to(device)
     y = torch.empty_like(x)
-    for _ in range(2):
-        ssm.ssd_fwd(x, dtr, A, Bm, Cm, D=D, dt_bias=db, out=y)
+    cs = torch.empty(ssm.ssd_chunk_states_shape(B, L, H, P, N), dtype=torch.float32, device=device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(reps):
-        ssm.ssd_fwd(x, dtr, A, Bm, Cm, D=D, dt_bias=db, out=y)
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / reps
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    ms = timed(lambda: ssm.ssd_fwd(x, dtr, A, Bm, Cm, D=D, dt_bias=db, out=y))
+    ms_train = timed(lambda: ssm.ssd_fwd(x, dtr, A, Bm, Cm, D=D, dt_bias=db, out=y, chunk_states=cs))
+    ms_bwd = timed(lambda: ssm.ssd_bwd(x, dtr, A, Bm, Cm, dy, cs, D=D, dt_bias=db))
     Q = 128
     chunks = B * H * (-(-L // Q))
     # per chunk: C B^T (2 Q Q N), Y_diag (2 Q P Q), Y_off (2 Q P N), chunk state (2 N P Q)
     flops = chunks * (2 * Q * Q * N + 2 * Q * P * Q + 2 * Q * P * N + 2 * N * P * Q)
     issued = flops + chunks * 2 * Q * P * Q  # the remainder product of the decay-masked C B^T
+    # backward per chunk: C B^T, dy x^T, B dH, C Hp, C^T dYs, M^T dy, dS B, dYs Hp^T, dS^T C, x dH^T
+    flops_bwd = chunks * 2 * (Q * Q * N + Q * Q * P + Q * P * N + Q * P * N + N * P * Q + Q * P * Q
+                              + Q * N * Q + Q * N * P + Q * N * Q + Q * N * P)
     nbytes = 2 * B * L * H * P * 2 + 2 * B * L * G * N * 2 + B * L * H * 2
+    cs_bytes = cs.numel() * 4
+    # backward: x, dy, dx, B, C, dt, ddt (fp32), dB / dC (fp32 atomics), chunk states read
+    nbytes_bwd = (3 * B * L * H * P * 2 + 2 * B * L * G * N * 2 + B * L * H * (2 + 4)
+                  + 2 * B * L * G * N * 4 + cs_bytes)
     tf = flops / (ms * 1e-3) / 1e12
-    return {"workload": f"Mamba-2 SSD forward, B{B} L{L} H{H} P{P} G{G} N{N} bf16, chunks of {Q}, "
-                        "tcgen05 bf16 products with fp32 TMEM accumulators",
+    tf_bwd = flops_bwd / (ms_bwd * 1e-3) / 1e12
+    return {"workload": f"Mamba-2 SSD forward and backward, B{B} L{L} H{H} P{P} G{G} N{N} bf16, "
+                        f"chunks of {Q}, tcgen05 bf16 products with fp32 TMEM accumulators",
             "ms": ms, "tokens_per_s": B * L / (ms * 1e-3), "tflops": tf,
             "tflops_issued": issued / (ms * 1e-3) / 1e12,
             "tensor_frac_of_peak": tf / pk["bf16_tflops"], "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
-            "flops_per_call": flops, "bytes_per_call": nbytes, "launches": reps + 2}
+            "flops_per_call": flops, "bytes_per_call": nbytes,
+            "fwd_saving_states_ms": ms_train, "chunk_states_bytes": cs_bytes,
+            "bwd_ms": ms_bwd, "bwd_tflops": tf_bwd, "bwd_tensor_frac_of_peak": tf_bwd / pk["bf16_tflops"],
+            "bwd_flops_per_call": flops_bwd, "bwd_hbm_gbs": nbytes_bwd / (ms_bwd * 1e-3) / 1e9,
+            "train_tokens_per_s": B * L / ((ms_train + ms_bwd) * 1e-3),
+            "launches": 3 * (reps + 2)}
 
 
 def deterministic_bench(ly, bwd_ms, reps=5):

@@ -142,10 +142,24 @@ __device__ __forceinline__ void unpack8(const uint4 q, float* v) {
 __device__ __forceinline__ uint4 pack8(const float* v) {
   return make_uint4(pk2(v[0], v[1]), pk2(v[2], v[3]), pk2(v[4], v[5]), pk2(v[6], v[7]));
 }
-__device__ __forceinline__ void red_add4(float* dst, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a), "f"(b), "f"(c), "f"(d)
+// dst[0 .. bytes/4) += src[...] (fp32), one bulk reduction from shared memory
+// (both 16-byte aligned, bytes a multiple of 16); completion of the read of
+// src is awaited with bulk_wait_read().
+__device__ __forceinline__ void bulk_add_f32(float* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes)
                : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+
+// dB / dC rows are staged in shared memory the chunk's products no longer
+// read (C, B, M, dS, x: free once the second group has completed), 528 bytes
+// apart (512 + 16: a warp's 16-byte stores of one column fall on distinct
+// banks), and added to global memory one 512-byte row at a time.
+constexpr uint32_t kStageRow = 528;
+constexpr uint32_t kStageB = 0, kStageC = kQ * kStageRow;
 
 // Sum of v over the 32 lanes of the warp for each of 32 columns: recursive
 // halving; lane l ends with column l.
@@ -165,6 +179,7 @@ __device__ __forceinline__ float colsum32(float v[32], int lane) {
 
 __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p) {
   static_assert(sizeof(SsdBwdSmem) <= 227 * 1024, "shared memory per CTA");
+  static_assert(kStageC + kQ * kStageRow <= offsetof(SsdBwdSmem, dY), "dB / dC staging overlaps live tiles");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   SsdBwdSmem& sm = *reinterpret_cast<SsdBwdSmem*>(smem_raw);
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -252,6 +267,14 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p) {
         for (int e = 0; e < 8; ++e) hdh = fmaf(dHc[8 * k + e], v[e], hdh);
         *reinterpret_cast<uint4*>(sm.Hp + toff(r, 8 * (4 * hf + k), kRs64)) = pack8(v);
       }
+    }
+    if (c > 0) {  // the previous chunk's rows into L2 while this one runs
+      const size_t xp = xo - (size_t)kQ * H * kP, bp = bo - (size_t)kQ * G * kNs;
+      prefetch_l2(Cg + bp);
+      prefetch_l2(Bg + bp);
+      prefetch_l2(xg + xp);
+      prefetch_l2(dyg + xp);
+      prefetch_l2(p.chunk_states + ((((size_t)b * H + h) * nch + c - 1) * kNs + r) * kP + 32 * hf);
     }
     const float dtv = valid ? __bfloat162float(dtg[((size_t)b * L + tok) * H + h]) + bias : 0.0f;
     float dt = 0.0f;
@@ -456,6 +479,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p) {
         }
       }
     }
+    float4* stB = reinterpret_cast<float4*>(smem_raw + kStageB + r * kStageRow);
+    float4* stC = reinterpret_cast<float4*>(smem_raw + kStageC + r * kStageRow);
 #pragma unroll 1
     for (int blk = 0; blk < 2; ++blk) {
       const int n0 = 64 * hf + 32 * blk;
@@ -464,21 +489,25 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p) {
       tm_ld32(lrow + 128 + n0, bv);
       tm_ld32(lrow + 384 + n0, tv);
       tm_wait();
-      if (valid) {
-        float* dC = p.dC + bo + 32 * blk;
-        float* dB = p.dB + bo + 32 * blk;
 #pragma unroll
-        for (int q = 0; q < 32; q += 4) {
-          red_add4(dC + q, cv[q], cv[q + 1], cv[q + 2], cv[q + 3]);
-          red_add4(dB + q, fmaf(w_r, tv[q], bv[q]), fmaf(w_r, tv[q + 1], bv[q + 1]),
-                   fmaf(w_r, tv[q + 2], bv[q + 2]), fmaf(w_r, tv[q + 3], bv[q + 3]));
-        }
+      for (int q = 0; q < 32; q += 4) {
+        stC[(n0 + q) / 4] = make_float4(cv[q], cv[q + 1], cv[q + 2], cv[q + 3]);
+        stB[(n0 + q) / 4] = make_float4(fmaf(w_r, tv[q], bv[q]), fmaf(w_r, tv[q + 1], bv[q + 1]),
+                                        fmaf(w_r, tv[q + 2], bv[q + 2]), fmaf(w_r, tv[q + 3], bv[q + 3]));
       }
     }
     // the carry for the chunk to the left, as the next products' operand
 #pragma unroll
     for (int k = 0; k < 4; ++k)
       *reinterpret_cast<uint4*>(sm.dH + toff(r, 8 * (4 * hf + k), kRs64)) = pack8(dHc + 8 * k);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    if (valid) {  // row r of dC (half 0) or dB (half 1), summed into global memory
+      const size_t ro = (((size_t)b * L + tok) * G + g) * kNs;
+      if (hf == 0) bulk_add_f32(p.dC + ro, stC, kNs * 4);
+      else bulk_add_f32(p.dB + ro, stB, kNs * 4);
+      bulk_wait_read();  // the staging rows are refilled by the next chunk
+    }
     tc_before();
     __syncthreads();  // every thread is done with this chunk's shared operands and TMEM
   }

@@ -337,3 +337,44 @@ def test_ssd_param_validation(ssm):
         p = params(**kw)
         assert L.ssm_ssd_fwd(ctypes.byref(p), None) == status, kw
         assert ssm.ssm_last_error()
+
+
+def test_ssd_bwd_param_validation(ssm):
+    """ssm_ssd_bwd rejects bad arguments before any launch: the forward's
+    checks, a missing chunk_states, grads struct size, NULL and misaligned
+    gradient pointers; and a misaligned chunk_states in the forward."""
+    from selective_state_space_35_b200 import _lib
+    L = _lib.load()
+    fake = 1 << 20
+
+    def params(**kw):
+        p = ssm.ssm_ssd_params()
+        p.struct_size = ctypes.sizeof(ssm.ssm_ssd_params)
+        p.B, p.L, p.H, p.P, p.G, p.N = 1, 256, 4, 64, 2, 128
+        p.dtype = 1
+        p.x, p.dt_raw, p.A, p.Bm, p.Cm = fake, fake + 4096, fake + 8192, fake + 12288, fake + 16384
+        p.chunk_states = fake + 65536
+        p.dt_softplus = 1
+        for k, v in kw.items():
+            setattr(p, k, v)
+        return p
+
+    def grads(**kw):
+        g = ssm.ssm_ssd_grads()
+        g.struct_size = ctypes.sizeof(ssm.ssm_ssd_grads)
+        g.dy, g.dx, g.ddt_raw, g.dA, g.dB, g.dC = (fake + 1024 * i for i in range(40, 46))
+        for k, v in kw.items():
+            setattr(g, k, v)
+        return g
+
+    cases = [(dict(), dict(struct_size=5), 1), (dict(), dict(dy=None), 1), (dict(), dict(dB=fake + 4), 1),
+             (dict(), dict(ddt_raw=fake + 2), 1), (dict(chunk_states=None), dict(), 1),
+             (dict(chunk_states=fake + 8), dict(), 1), (dict(P=32), dict(), 2), (dict(G=3), dict(), 1)]
+    for pkw, gkw, status in cases:
+        p, g = params(**pkw), grads(**gkw)
+        assert L.ssm_ssd_bwd(ctypes.byref(p), ctypes.byref(g), None) == status, (pkw, gkw)
+        assert ssm.ssm_last_error()
+    assert L.ssm_ssd_bwd(ctypes.byref(params()), None, None) == 1
+    p = params(y=fake + 20480, chunk_states=fake + 8)
+    assert L.ssm_ssd_fwd(ctypes.byref(p), None) == 1
+    assert "aligned" in ssm.ssm_last_error()

@@ -74,10 +74,14 @@ conv1d_fwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
 }
 
 // dx_s = sum_k w_k dc_{s+3-k} [same document], dc_t = du_t * silu'(c_t).
-// Each thread recomputes c_t for its 8 tokens plus the 3 after them, writes
-// dx for its 8 tokens, and adds its tokens' share of dw and dbias into a
-// per-CTA partial (reduced over (b, tile) by conv1d_wreduce_kernel).
-template <typename T, bool VEC, bool SEQ, bool HALO>
+// Each thread recomputes c_t for its kT tokens plus the 3 after them, writes
+// dx for its tokens, and adds its tokens' share of dw and dbias into a
+// per-CTA partial (reduced over (b, tile) by conv1d_wreduce_kernel). Without
+// document ids kT = 16: the 3-token halos, the recomputed c of the halo and
+// the warp reduction of the partials are paid once per 16 tokens (0.195 ->
+// 0.174 ms at B2 D1536 L32768 bf16); with them kT = 8, which keeps the
+// per-token segment ids within the registers of a full SM.
+template <typename T, bool VEC, bool SEQ, bool HALO, int kT>
 __global__ void __launch_bounds__(kConvThreads)
 conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
                   const float* __restrict__ bias, const int32_t* __restrict__ seq,
@@ -87,7 +91,7 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
                   const T* __restrict__ du_next, const int32_t* __restrict__ seq_next, int D,
                   int L, int silu) {
   const int d = blockIdx.y, b = blockIdx.z;
-  const int t0 = (blockIdx.x * kConvThreads + threadIdx.x) * 8;
+  const int t0 = (blockIdx.x * kConvThreads + threadIdx.x) * kT;
   const bool live = t0 < L;
   const size_t row = ((size_t)b * D + d) * L;
   const T* xr = x + row;
@@ -97,13 +101,13 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
   for (int k = 0; k < 4; ++k) wk[k] = __ldg(w + d * 4 + k);
   const float bs = bias ? __ldg(bias + d) : 0.0f;
 
-  float xv[14];   // x[t0-3 .. t0+10]
-  float duv[11];  // du[t0 .. t0+10]
-  int sg[14];     // seg[t0-3 .. t0+10]
+  float xv[kT + 6];   // x[t0-3 .. t0+kT+2]
+  float duv[kT + 3];  // du[t0 .. t0+kT+2]
+  int sg[kT + 6];     // seg[t0-3 .. t0+kT+2]
 #pragma unroll
-  for (int i = 0; i < 14; ++i) { xv[i] = 0.0f; sg[i] = 0; }
+  for (int i = 0; i < kT + 6; ++i) { xv[i] = 0.0f; sg[i] = 0; }
 #pragma unroll
-  for (int i = 0; i < 11; ++i) duv[i] = 0.0f;
+  for (int i = 0; i < kT + 3; ++i) duv[i] = 0.0f;
   // halos of a row cut out of a longer sequence: the 3 inputs before token 0,
   // and the 3 inputs and upstream gradients after token L-1
   const size_t hrow = ((size_t)b * D + d) * 3;
@@ -114,20 +118,23 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
       if (s >= 0) xv[i] = Io<T>::ld(xr + s);
       else if (HALO && x_prev) xv[i] = Io<T>::ld(x_prev + hrow + 3 + s);
     }
-    load_row8<T, VEC>(xr, t0, L, xv + 3);
-    load_row8<T, VEC>(dur, t0, L, duv);
+#pragma unroll
+    for (int k = 0; k < kT / 8; ++k) {
+      load_row8<T, VEC>(xr, t0 + 8 * k, L, xv + 3 + 8 * k);
+      load_row8<T, VEC>(dur, t0 + 8 * k, L, duv + 8 * k);
+    }
 #pragma unroll
     for (int i = 0; i < 3; ++i) {
-      const int s = t0 + 8 + i;
+      const int s = t0 + kT + i;
       if (s < L) {
-        xv[11 + i] = Io<T>::ld(xr + s);
-        duv[8 + i] = Io<T>::ld(dur + s);
+        xv[kT + 3 + i] = Io<T>::ld(xr + s);
+        duv[kT + i] = Io<T>::ld(dur + s);
       }
     }
-    if (HALO && x_next && t0 + 11 > L) {
+    if (HALO && x_next && t0 + kT + 3 > L) {
       // tokens L .. L+2 of the window come from the next piece
 #pragma unroll
-      for (int i = 3; i < 14; ++i) {
+      for (int i = 3; i < kT + 6; ++i) {
         const int s = t0 - 3 + i;
         if (s >= L && s < L + 3) {
           xv[i] = Io<T>::ld(x_next + hrow + (s - L));
@@ -138,7 +145,7 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
     if (SEQ) {
       const int32_t* sr = seq + (size_t)b * L;
 #pragma unroll
-      for (int i = 0; i < 14; ++i) {
+      for (int i = 0; i < kT + 6; ++i) {
         const int s = t0 - 3 + i;
         int v = 0;
         if (s >= 0 && s < L) v = __ldg(sr + s);
@@ -150,10 +157,10 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
     }
   }
 
-  // dc for tokens t0 .. t0+10 (token t0+j: x window xv[j..j+3], segment sg[j+3])
-  float dc[11];
+  // dc for tokens t0 .. t0+kT+2 (token t0+j: x window xv[j..j+3], segment sg[j+3])
+  float dc[kT + 3];
 #pragma unroll
-  for (int j = 0; j < 11; ++j) {
+  for (int j = 0; j < kT + 3; ++j) {
     float c = bs;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -170,24 +177,28 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
   }
 
   if (live) {
-    float o[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float acc = 0.0f;
+    for (int k8 = 0; k8 < kT / 8; ++k8) {
+      float o[8];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int j = i + 3 - k;  // output token t0+j uses x_{t0+i} through tap k
-        const bool ok = !SEQ || sg[j + 3] == sg[i + 3];
-        acc = fmaf(wk[k], ok ? dc[j] : 0.0f, acc);
+      for (int i = 0; i < 8; ++i) {
+        const int ii = 8 * k8 + i;
+        float acc = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int j = ii + 3 - k;  // output token t0+j uses x_{t0+ii} through tap k
+          const bool ok = !SEQ || sg[j + 3] == sg[ii + 3];
+          acc = fmaf(wk[k], ok ? dc[j] : 0.0f, acc);
+        }
+        o[i] = acc;
       }
-      o[i] = acc;
+      store_row8<T, VEC>(dx + row, t0 + 8 * k8, L, o);
     }
-    store_row8<T, VEC>(dx + row, t0, L, o);
   }
 
   float pw[5] = {0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < kT; ++i) {
     // this row's own tokens only (past L, dc is nonzero only with a next-piece halo)
     const float dci = (HALO && t0 + i >= L) ? 0.0f : dc[i];
 #pragma unroll
@@ -244,15 +255,17 @@ void conv_fwd_t(const ConvArgs& a, cudaStream_t s) {
 
 template <typename T, bool VEC, bool SEQ, bool HALO>
 void conv_bwd_h(const ConvArgs& a, cudaStream_t s) {
-  dim3 grid(conv_tiles(a.L), a.D, a.B);
-  conv1d_bwd_kernel<T, VEC, SEQ, HALO><<<grid, kConvThreads, 0, s>>>(
+  constexpr int kT = SEQ ? 8 : kConvBwdTok;
+  const int tiles = (a.L + kConvThreads * kT - 1) / (kConvThreads * kT);
+  dim3 grid(tiles, a.D, a.B);
+  conv1d_bwd_kernel<T, VEC, SEQ, HALO, kT><<<grid, kConvThreads, 0, s>>>(
       static_cast<const T*>(a.x), a.w, a.bias, a.seq, static_cast<const T*>(a.du),
       static_cast<T*>(a.out), a.partial, static_cast<const T*>(a.x_prev), a.seq_prev,
       static_cast<const T*>(a.x_next), static_cast<const T*>(a.du_next), a.seq_next, a.D, a.L,
       a.silu);
   const int n = a.D * 5;
   conv1d_wreduce_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.partial, a.dw, a.dbias, a.B,
-                                                        conv_tiles(a.L), a.D);
+                                                        tiles, a.D);
 }
 
 template <typename T, bool VEC, bool SEQ>

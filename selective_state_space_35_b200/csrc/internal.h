@@ -61,6 +61,10 @@ constexpr int kMaxScratchDevices = 64;
 cudaError_t conv_bwd_scratch(float** ptr);
 cudaError_t launch_conv1d_bwd(const ConvArgs& a, cudaStream_t s);
 inline int conv_tiles(int L) { return (L + kConvTile - 1) / kConvTile; }
+// The backward without document ids: kConvBwdTok tokens per thread (with
+// them 8, as the forward); its dw / dbias partials are per (b, tile, d), at
+// most conv_tiles(L) tiles, which sizes its scratch.
+constexpr int kConvBwdTok = 16;
 
 struct ScanArgs {
   // inputs

@@ -17,15 +17,16 @@ namespace ssm {
 namespace {
 
 // HALO: the row is a piece of a longer sequence (halo pointers may be set);
-// without it the halo code is compiled out of the common path.
-template <typename T, bool VEC, bool SEQ, bool HALO>
+// without it the halo code is compiled out of the common path. kT tokens per
+// thread (16 without document ids: the 3-token halo is read once per 16).
+template <typename T, bool VEC, bool SEQ, bool HALO, int kT>
 __global__ void __launch_bounds__(kConvThreads)
 conv1d_fwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
                   const float* __restrict__ bias, const int32_t* __restrict__ seq,
                   const T* __restrict__ x_prev, const int32_t* __restrict__ seq_prev,
                   T* __restrict__ u, int D, int L, int silu) {
   const int d = blockIdx.y, b = blockIdx.z;
-  const int t0 = (blockIdx.x * kConvThreads + threadIdx.x) * 8;
+  const int t0 = (blockIdx.x * kConvThreads + threadIdx.x) * kT;
   if (t0 >= L) return;
   const size_t row = ((size_t)b * D + d) * L;
   const T* xr = x + row;
@@ -34,43 +35,48 @@ conv1d_fwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
   for (int k = 0; k < 4; ++k) wk[k] = __ldg(w + d * 4 + k);
   const float bs = bias ? __ldg(bias + d) : 0.0f;
 
-  // x[t0-3 .. t0+7]; before token 0 the halo x_prev (the 3 preceding inputs)
-  // or 0
+  // x[t0-3 .. t0+kT-1]; before token 0 the halo x_prev (the 3 preceding
+  // inputs) or 0
   const T* xp = (HALO && x_prev) ? x_prev + ((size_t)b * D + d) * 3 : nullptr;
-  float xv[11];
+  float xv[kT + 3];
 #pragma unroll
   for (int i = 0; i < 3; ++i) {
     const int s = t0 - 3 + i;
     xv[i] = s >= 0 ? Io<T>::ld(xr + s) : (xp ? Io<T>::ld(xp + 3 + s) : 0.0f);
   }
-  load_row8<T, VEC>(xr, t0, L, xv + 3);
+#pragma unroll
+  for (int k = 0; k < kT / 8; ++k) load_row8<T, VEC>(xr, t0 + 8 * k, L, xv + 3 + 8 * k);
 
-  int sg[11];
+  int sg[kT + 3];
   if (SEQ) {
     const int32_t* sr = seq + (size_t)b * L;
 #pragma unroll
-    for (int i = 0; i < 11; ++i) {
+    for (int i = 0; i < kT + 3; ++i) {
       const int s = t0 - 3 + i;
       sg[i] = (s >= 0 && s < L) ? __ldg(sr + s)
                                 : ((HALO && s < 0 && seq_prev) ? __ldg(seq_prev + (size_t)b * 3 + 3 + s) : 0);
     }
   }
 
-  float out[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    float acc = bs;
+  for (int k8 = 0; k8 < kT / 8; ++k8) {
+    float out[8];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      // tap k of output t0+i reads x_{t0+i-3+k} = xv[i+k]; xv is 0 before t=0
-      const bool ok = !SEQ || sg[i + k] == sg[i + 3];
-      acc = fmaf(wk[k], ok ? xv[i + k] : 0.0f, acc);
+    for (int i = 0; i < 8; ++i) {
+      const int ii = 8 * k8 + i;
+      float acc = bs;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        // tap k of output t0+ii reads x_{t0+ii-3+k} = xv[ii+k]; xv is 0 before t=0
+        const bool ok = !SEQ || sg[ii + k] == sg[ii + 3];
+        acc = fmaf(wk[k], ok ? xv[ii + k] : 0.0f, acc);
+      }
+      // SiLU with the SFU sigmoid (the fused conv + scan forward computes the
+      // same expression, so both store identical u)
+      out[i] = silu ? acc * sigmoid_fast(acc) : acc;
     }
-    // SiLU with the SFU sigmoid (the fused conv + scan forward computes the
-    // same expression, so both store identical u)
-    out[i] = silu ? acc * sigmoid_fast(acc) : acc;
+    store_row8<T, VEC>(u + row, t0 + 8 * k8, L, out);
   }
-  store_row8<T, VEC>(u + row, t0, L, out);
 }
 
 // dx_s = sum_k w_k dc_{s+3-k} [same document], dc_t = du_t * silu'(c_t).
@@ -241,8 +247,9 @@ __global__ void conv1d_wreduce_kernel(const float* __restrict__ partial, float* 
 
 template <typename T, bool VEC, bool SEQ, bool HALO>
 void conv_fwd_h(const ConvArgs& a, cudaStream_t s) {
-  dim3 grid(conv_tiles(a.L), a.D, a.B);
-  conv1d_fwd_kernel<T, VEC, SEQ, HALO><<<grid, kConvThreads, 0, s>>>(
+  constexpr int kT = SEQ ? 8 : 16;
+  dim3 grid((a.L + kConvThreads * kT - 1) / (kConvThreads * kT), a.D, a.B);
+  conv1d_fwd_kernel<T, VEC, SEQ, HALO, kT><<<grid, kConvThreads, 0, s>>>(
       static_cast<const T*>(a.x), a.w, a.bias, a.seq, static_cast<const T*>(a.x_prev), a.seq_prev,
       static_cast<T*>(a.out), a.D, a.L, a.silu);
 }

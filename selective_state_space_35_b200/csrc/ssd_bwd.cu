@@ -153,6 +153,11 @@ __device__ __forceinline__ void bulk_add_f32(float* dst, const void* src, uint32
 }
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+// 16 bytes global -> shared without registers; nbytes 0 fills zeros (src unread)
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t nbytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(nbytes)
+               : "memory");
+}
 
 // dB / dC rows are staged in shared memory the chunk's products no longer
 // read (C, B, M, dS, x: free once the second group has completed), 528 bytes
@@ -232,27 +237,27 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p) {
     const bool valid = tok < L;
     const size_t xo = (((size_t)b * L + tok) * H + h) * kP + 32 * hf;  // x / dy / dx row half
     const size_t bo = (((size_t)b * L + tok) * G + g) * kNs + 64 * hf; // B / C / dB / dC row half
-    // ---- this chunk's rows into shared memory ----
-    float xr[32], dyr[32];
+    // ---- this chunk's rows straight into their tiles (cp.async, zero-filled
+    // past L): no registers held, one round trip ----
     {
-      const uint4* crow = reinterpret_cast<const uint4*>(Cg + bo);
-      const uint4* brow = reinterpret_cast<const uint4*>(Bg + bo);
+      const size_t bs = valid ? bo : (((size_t)b * L) * G + g) * kNs + 64 * hf;  // in bounds when !valid
+      const size_t xs = valid ? xo : (((size_t)b * L) * H + h) * kP + 32 * hf;
+      const uint32_t nb = valid ? 16u : 0u;
+      const uint4* crow = reinterpret_cast<const uint4*>(Cg + bs);
+      const uint4* brow = reinterpret_cast<const uint4*>(Bg + bs);
+      const uint4* xrow = reinterpret_cast<const uint4*>(xg + xs);
+      const uint4* dyrow = reinterpret_cast<const uint4*>(dyg + xs);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        *reinterpret_cast<uint4*>(sm.C + toff(r, 8 * (8 * hf + k), kRs128)) = valid ? __ldg(crow + k) : z4;
-        *reinterpret_cast<uint4*>(sm.Bm + toff(r, 8 * (8 * hf + k), kRs128)) = valid ? __ldg(brow + k) : z4;
+        cp_async16(sm.C + toff(r, 8 * (8 * hf + k), kRs128), crow + k, nb);
+        cp_async16(sm.Bm + toff(r, 8 * (8 * hf + k), kRs128), brow + k, nb);
       }
-      const uint4* xrow = reinterpret_cast<const uint4*>(xg + xo);
-      const uint4* dyrow = reinterpret_cast<const uint4*>(dyg + xo);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const uint4 xq = valid ? __ldg(xrow + k) : z4;
-        const uint4 yq = valid ? __ldg(dyrow + k) : z4;
-        *reinterpret_cast<uint4*>(sm.X + toff(r, 8 * (4 * hf + k), kRs64)) = xq;
-        *reinterpret_cast<uint4*>(sm.dY + toff(r, 8 * (4 * hf + k), kRs64)) = yq;
-        unpack8(xq, xr + 8 * k);
-        unpack8(yq, dyr + 8 * k);
+        cp_async16(sm.X + toff(r, 8 * (4 * hf + k), kRs64), xrow + k, nb);
+        cp_async16(sm.dY + toff(r, 8 * (4 * hf + k), kRs64), dyrow + k, nb);
       }
+      asm volatile("cp.async.commit_group;" ::: "memory");
     }
     // the state entering the chunk, row n = r: bf16 tile, and <dH, Hp> for d lcs_Q-1
     float hdh = 0.0f;
@@ -281,6 +286,14 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p) {
     if (valid) dt = p.softplus ? (dtv > 20.0f ? dtv : log1pf(expf(dtv))) : dtv;
     bool start = false;
     if (valid && seqb && tok > 0) start = __ldg(seqb + tok) != __ldg(seqb + tok - 1);
+    // this thread's x and dy values, from the tiles its own copies filled
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    float xr[32], dyr[32];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      unpack8(*reinterpret_cast<const uint4*>(sm.X + toff(r, 8 * (4 * hf + k), kRs64)), xr + 8 * k);
+      unpack8(*reinterpret_cast<const uint4*>(sm.dY + toff(r, 8 * (4 * hf + k), kRs64)), dyr + 8 * k);
+    }
     // ---- chunk scans (warps 0-3): lcs = inclusive sum of dt A, ls = last document start ----
     float la = dt * Ah;
     int st = start ? r : -1;

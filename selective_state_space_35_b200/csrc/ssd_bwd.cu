@@ -29,7 +29,10 @@
 // C^T dYs) and, once M and dS are in shared memory, (M^T dy, dS B + dYs Hp^T,
 // dS^T C, x dH^T); the second runs while the threads reduce the decay terms.
 // One CTA of 256 threads per (b, h); 512 TMEM columns.
+#include <cuda.h>  // CUtensorMap (the maps are encoded through the runtime's driver entry point)
+
 #include <atomic>
+#include <cstring>
 
 #include "scan_common.cuh"
 
@@ -63,7 +66,8 @@ struct SsdBwdSmem {
   float wsum[8];
   int wmax[4];
   float blk[2][8];
-  uint64_t bar;
+  uint64_t bar;   // tensor-core products
+  uint64_t tbar;  // tensor-map copies of a chunk's rows
   uint32_t tmem;
 };
 
@@ -153,6 +157,19 @@ __device__ __forceinline__ void bulk_add_f32(float* dst, const void* src, uint32
 }
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+// One operand tile (128 rows of a row-major [rows][groups][features] bf16
+// tensor) by one tensor-map copy: the map's five dimensions (feature_lo 8,
+// row_lo 8, feature_hi, group, row_hi) put the box in shared memory in the
+// tiles' core-matrix order; rows past the tensor are zero-filled.
+__device__ __forceinline__ void tma_tile(void* dst, const CUtensorMap* map, int group, int row_hi,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+      "%5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(0), "r"(0), "r"(0), "r"(group), "r"(row_hi), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // 16 bytes global -> shared without registers; nbytes 0 fills zeros (src unread)
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t nbytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(nbytes)
@@ -182,7 +199,15 @@ __device__ __forceinline__ float colsum32(float v[32], int lane) {
   return v[0];
 }
 
-__global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p) {
+// The four maps cover C, B ([B L][G][128]) and x, dy ([B L][H][64]); `tma`
+// false (L not a multiple of 8, or no map could be encoded) copies every
+// chunk's rows with cp.async instead, as the ragged last chunk always does.
+struct SsdMaps {
+  CUtensorMap C, B, X, dY;
+};
+
+__global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p, const __grid_constant__ SsdMaps maps,
+                                                              const int tma) {
   static_assert(sizeof(SsdBwdSmem) <= 227 * 1024, "shared memory per CTA");
   static_assert(kStageC + kQ * kStageRow <= offsetof(SsdBwdSmem, dY), "dB / dC staging overlaps live tiles");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -207,6 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p) {
 
   if (t == 0) {
     mbar_init(&sm.bar, 1);
+    mbar_init(&sm.tbar, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -229,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p) {
 #pragma unroll
   for (int q = 0; q < 32; ++q) dHc[q] = 0.0f;
   float dA_acc = 0.0f, dD_acc = 0.0f, ddb_acc = 0.0f;
-  unsigned phase = 0;
+  unsigned phase = 0, tphase = 0;
 
 #pragma unroll 1
   for (int c = nch - 1; c >= 0; --c) {
@@ -237,9 +263,20 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p) {
     const bool valid = tok < L;
     const size_t xo = (((size_t)b * L + tok) * H + h) * kP + 32 * hf;  // x / dy / dx row half
     const size_t bo = (((size_t)b * L + tok) * G + g) * kNs + 64 * hf; // B / C / dB / dC row half
-    // ---- this chunk's rows straight into their tiles (cp.async, zero-filled
-    // past L): no registers held, one round trip ----
-    {
+    // ---- this chunk's rows straight into their tiles: one tensor-map copy
+    // per tile for a whole chunk, else cp.async (zero-filled past L); no
+    // registers held ----
+    const bool by_map = tma && (c + 1) * kQ <= L;
+    if (by_map) {
+      if (t == 0) {
+        const int rh = (int)(((size_t)b * L + (size_t)c * kQ) / 8);
+        mbar_expect_tx(&sm.tbar, 2u * kQ * kNs * 2 + 2u * kQ * kP * 2);
+        tma_tile(sm.C, &maps.C, g, rh, &sm.tbar);
+        tma_tile(sm.Bm, &maps.B, g, rh, &sm.tbar);
+        tma_tile(sm.X, &maps.X, h, rh, &sm.tbar);
+        tma_tile(sm.dY, &maps.dY, h, rh, &sm.tbar);
+      }
+    } else {
       const size_t bs = valid ? bo : (((size_t)b * L) * G + g) * kNs + 64 * hf;  // in bounds when !valid
       const size_t xs = valid ? xo : (((size_t)b * L) * H + h) * kP + 32 * hf;
       const uint32_t nb = valid ? 16u : 0u;
@@ -286,8 +323,19 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p) {
     if (valid) dt = p.softplus ? (dtv > 20.0f ? dtv : log1pf(expf(dtv))) : dtv;
     bool start = false;
     if (valid && seqb && tok > 0) start = __ldg(seqb + tok) != __ldg(seqb + tok - 1);
-    // this thread's x and dy values, from the tiles its own copies filled
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    // this thread's x and dy values, from the filled tiles
+    if (by_map) {
+      const bool ok = mbar_wait_bounded(&sm.tbar, tphase, p.status);
+      tphase ^= 1u;
+      if (!__syncthreads_and(ok)) {
+        // the copies have not landed: wait once more (bounded) so that they
+        // do not land after the CTA has exited, then stop
+        if (t == 0) mbar_wait_bounded(&sm.tbar, tphase ^ 1u, nullptr);
+        break;
+      }
+    } else {
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    }
     float xr[32], dyr[32];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -521,6 +569,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p) {
       else bulk_add_f32(p.dB + ro, stB, kNs * 4);
       bulk_wait_read();  // the staging rows are refilled by the next chunk
     }
+    // generic accesses to the tiles before the next chunk's tensor-map writes
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_before();
     __syncthreads();  // every thread is done with this chunk's shared operands and TMEM
   }
@@ -545,6 +595,39 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p) {
 
 }  // namespace
 
+typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                      const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                      CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                      CUtensorMapFloatOOBfill);
+
+TensorMapEncodeFn tensor_map_encoder() {
+  static std::atomic<TensorMapEncodeFn> fn{nullptr};
+  TensorMapEncodeFn f = fn.load(std::memory_order_acquire);
+  if (!f) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      f = reinterpret_cast<TensorMapEncodeFn>(ptr);
+    fn.store(f, std::memory_order_release);
+  }
+  return f;
+}
+
+// A map over rows x groups x features (bf16, row-major) with 128-row boxes
+// in the tiles' core-matrix order (see tma_tile).
+bool encode_tile_map(TensorMapEncodeFn enc, CUtensorMap* m, const void* base, size_t rows, int groups,
+                     int features) {
+  const cuuint64_t dims[5] = {8, 8, (cuuint64_t)features / 8, (cuuint64_t)groups, (cuuint64_t)rows / 8};
+  const cuuint64_t strides[4] = {(cuuint64_t)groups * features * 2, 16, (cuuint64_t)features * 2,
+                                 (cuuint64_t)8 * groups * features * 2};
+  const cuuint32_t box[5] = {8, 8, (cuuint32_t)features / 8, 1, kQ / 8};
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_ssd_bwd(const SsdArgs& a, cudaStream_t s) {
   static std::atomic<unsigned long long> done{0};
   const int smem = (int)sizeof(SsdBwdSmem);
@@ -557,7 +640,16 @@ cudaError_t launch_ssd_bwd(const SsdArgs& a, cudaStream_t s) {
   if (a.dD && (e = cudaMemsetAsync(a.dD, 0, (size_t)a.H * sizeof(float), s)) != cudaSuccess) return e;
   if (a.ddt_bias && (e = cudaMemsetAsync(a.ddt_bias, 0, (size_t)a.H * sizeof(float), s)) != cudaSuccess)
     return e;
-  ssd_bwd_kernel<<<dim3(a.H, a.B), kThreads, smem, s>>>(a);
+  SsdMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  int tma = 0;
+  const TensorMapEncodeFn enc = a.L % 8 == 0 ? tensor_map_encoder() : nullptr;
+  if (enc) {
+    const size_t rows = (size_t)a.B * a.L;
+    tma = encode_tile_map(enc, &maps.C, a.Cm, rows, a.G, kNs) && encode_tile_map(enc, &maps.B, a.Bm, rows, a.G, kNs) &&
+          encode_tile_map(enc, &maps.X, a.x, rows, a.H, kP) && encode_tile_map(enc, &maps.dY, a.dy, rows, a.H, kP);
+  }
+  ssd_bwd_kernel<<<dim3(a.H, a.B), kThreads, smem, s>>>(a, maps, tma);
   return cudaGetLastError();
 }
 

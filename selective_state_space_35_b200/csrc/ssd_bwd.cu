@@ -29,12 +29,11 @@
 // C^T dYs) and, once M and dS are in shared memory, (M^T dy, dS B + dYs Hp^T,
 // dS^T C, x dH^T); the second runs while the threads reduce the decay terms.
 // One CTA of 256 threads per (b, h); 512 TMEM columns.
-#include <cuda.h>  // CUtensorMap (the maps are encoded through the runtime's driver entry point)
-
 #include <atomic>
 #include <cstring>
 
 #include "scan_common.cuh"
+#include "ssd_maps.cuh"
 
 namespace ssm {
 
@@ -595,39 +594,6 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p, c
 
 }  // namespace
 
-typedef CUresult (*TensorMapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                      const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
-                                      CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
-                                      CUtensorMapFloatOOBfill);
-
-TensorMapEncodeFn tensor_map_encoder() {
-  static std::atomic<TensorMapEncodeFn> fn{nullptr};
-  TensorMapEncodeFn f = fn.load(std::memory_order_acquire);
-  if (!f) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      f = reinterpret_cast<TensorMapEncodeFn>(ptr);
-    fn.store(f, std::memory_order_release);
-  }
-  return f;
-}
-
-// A map over rows x groups x features (bf16, row-major) with 128-row boxes
-// in the tiles' core-matrix order (see tma_tile).
-bool encode_tile_map(TensorMapEncodeFn enc, CUtensorMap* m, const void* base, size_t rows, int groups,
-                     int features) {
-  const cuuint64_t dims[5] = {8, 8, (cuuint64_t)features / 8, (cuuint64_t)groups, (cuuint64_t)rows / 8};
-  const cuuint64_t strides[4] = {(cuuint64_t)groups * features * 2, 16, (cuuint64_t)features * 2,
-                                 (cuuint64_t)8 * groups * features * 2};
-  const cuuint32_t box[5] = {8, 8, (cuuint32_t)features / 8, 1, kQ / 8};
-  const cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 cudaError_t launch_ssd_bwd(const SsdArgs& a, cudaStream_t s) {
   static std::atomic<unsigned long long> done{0};
   const int smem = (int)sizeof(SsdBwdSmem);
@@ -643,11 +609,11 @@ cudaError_t launch_ssd_bwd(const SsdArgs& a, cudaStream_t s) {
   SsdMaps maps;
   memset(&maps, 0, sizeof(maps));
   int tma = 0;
-  const TensorMapEncodeFn enc = a.L % 8 == 0 ? tensor_map_encoder() : nullptr;
+  const SsdTensorMapEncode enc = a.L % 8 == 0 ? ssd_tensor_map_encoder() : nullptr;
   if (enc) {
     const size_t rows = (size_t)a.B * a.L;
-    tma = encode_tile_map(enc, &maps.C, a.Cm, rows, a.G, kNs) && encode_tile_map(enc, &maps.B, a.Bm, rows, a.G, kNs) &&
-          encode_tile_map(enc, &maps.X, a.x, rows, a.H, kP) && encode_tile_map(enc, &maps.dY, a.dy, rows, a.H, kP);
+    tma = ssd_tile_map(enc, &maps.C, a.Cm, rows, a.G, kNs) && ssd_tile_map(enc, &maps.B, a.Bm, rows, a.G, kNs) &&
+          ssd_tile_map(enc, &maps.X, a.x, rows, a.H, kP) && ssd_tile_map(enc, &maps.dY, a.dy, rows, a.H, kP);
   }
   ssd_bwd_kernel<<<dim3(a.H, a.B), kThreads, smem, s>>>(a, maps, tma);
   return cudaGetLastError();

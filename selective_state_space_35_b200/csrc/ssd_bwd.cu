@@ -176,11 +176,26 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t 
 }
 
 // dB / dC rows are staged in shared memory the chunk's products no longer
-// read (C, B, M, dS, x: free once the second group has completed), 528 bytes
-// apart (512 + 16: a warp's 16-byte stores of one column fall on distinct
-// banks), and added to global memory one 512-byte row at a time.
+// read (C, B, M, dS, x: free once the second group has completed) and added
+// to global memory by bulk reductions. With tensor maps (tma bit 1): as four
+// boxes of 32 states x 128 tokens per matrix in the 128-byte swizzled order
+// (a row's 16-byte chunk k at chunk k ^ (row & 7): a warp's stores fall on
+// distinct banks), dC in C / B and dB in M / dS, eight tensor reductions per
+// chunk that undo the swizzle on the way out. Tokens past L carry exact
+// zeros (their dt, dy, x are 0), so a box that reaches past L adds nothing.
+// Otherwise rows 528 bytes apart (512 + 16), one 512-byte reduction per row.
 constexpr uint32_t kStageRow = 528;
 constexpr uint32_t kStageB = 0, kStageC = kQ * kStageRow;
+constexpr uint32_t kBoxBytes = kQ * 128;  // 32 fp32 states x 128 tokens
+
+// One staged box (32 states from n0, 128 tokens from row0, group g) added
+// into a [rows][G][128] fp32 tensor by a tensor-map bulk reduction.
+__device__ __forceinline__ void tma_add_box(const CUtensorMap* map, const void* src, int n0, int g, int row0) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(map),
+      "r"(n0), "r"(g), "r"(row0), "r"(smem_u32(src))
+      : "memory");
+}
 
 // Sum of v over the 32 lanes of the warp for each of 32 columns: recursive
 // halving; lane l ends with column l.
@@ -198,11 +213,12 @@ __device__ __forceinline__ float colsum32(float v[32], int lane) {
   return v[0];
 }
 
-// The four maps cover C, B ([B L][G][128]) and x, dy ([B L][H][64]); `tma`
-// false (L not a multiple of 8, or no map could be encoded) copies every
-// chunk's rows with cp.async instead, as the ragged last chunk always does.
+// tma bit 0: C, B ([B L][G][128]) and x, dy ([B L][H][64]) of whole chunks
+// by tensor map (L a multiple of 8); else every chunk's rows by cp.async, as
+// the ragged last chunk's always are. Bit 1: dB / dC by tensor reductions.
 struct SsdMaps {
-  CUtensorMap C, B, X, dY;
+  CUtensorMap C, B, X, dY;  // bit 0 of tma
+  CUtensorMap dB, dC;       // bit 1
 };
 
 __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p, const __grid_constant__ SsdMaps maps,
@@ -265,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p, c
     // ---- this chunk's rows straight into their tiles: one tensor-map copy
     // per tile for a whole chunk, else cp.async (zero-filled past L); no
     // registers held ----
-    const bool by_map = tma && (c + 1) * kQ <= L;
+    const bool by_map = (tma & 1) && (c + 1) * kQ <= L;
     if (by_map) {
       if (t == 0) {
         const int rh = (int)(((size_t)b * L + (size_t)c * kQ) / 8);
@@ -539,6 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p, c
         }
       }
     }
+    const bool boxes = (tma & 2) != 0;
     float4* stB = reinterpret_cast<float4*>(smem_raw + kStageB + r * kStageRow);
     float4* stC = reinterpret_cast<float4*>(smem_raw + kStageC + r * kStageRow);
 #pragma unroll 1
@@ -549,11 +566,22 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p, c
       tm_ld32(lrow + 128 + n0, bv);
       tm_ld32(lrow + 384 + n0, tv);
       tm_wait();
+      // box n0 / 32 of each matrix, row r: 16-byte chunk k at k ^ (r & 7)
+      unsigned char* bC = sm.C + (n0 / 32) * kBoxBytes + r * 128;
+      unsigned char* bB = sm.M + (n0 / 32) * kBoxBytes + r * 128;
 #pragma unroll
       for (int q = 0; q < 32; q += 4) {
-        stC[(n0 + q) / 4] = make_float4(cv[q], cv[q + 1], cv[q + 2], cv[q + 3]);
-        stB[(n0 + q) / 4] = make_float4(fmaf(w_r, tv[q], bv[q]), fmaf(w_r, tv[q + 1], bv[q + 1]),
-                                        fmaf(w_r, tv[q + 2], bv[q + 2]), fmaf(w_r, tv[q + 3], bv[q + 3]));
+        const float4 vc = make_float4(cv[q], cv[q + 1], cv[q + 2], cv[q + 3]);
+        const float4 vb = make_float4(fmaf(w_r, tv[q], bv[q]), fmaf(w_r, tv[q + 1], bv[q + 1]),
+                                      fmaf(w_r, tv[q + 2], bv[q + 2]), fmaf(w_r, tv[q + 3], bv[q + 3]));
+        if (boxes) {
+          const int ck = ((q / 4) ^ (r & 7)) * 16;
+          *reinterpret_cast<float4*>(bC + ck) = vc;
+          *reinterpret_cast<float4*>(bB + ck) = vb;
+        } else {
+          stC[(n0 + q) / 4] = vc;
+          stB[(n0 + q) / 4] = vb;
+        }
       }
     }
     // the carry for the chunk to the left, as the next products' operand
@@ -562,7 +590,18 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p, c
       *reinterpret_cast<uint4*>(sm.dH + toff(r, 8 * (4 * hf + k), kRs64)) = pack8(dHc + 8 * k);
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
-    if (valid) {  // row r of dC (half 0) or dB (half 1), summed into global memory
+    if (boxes) {  // eight tensor reductions: four boxes of dC, four of dB
+      if (t == 0) {
+        const int row0 = (int)((size_t)b * L + (size_t)c * kQ);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          tma_add_box(&maps.dC, sm.C + q * kBoxBytes, 32 * q, g, row0);
+          tma_add_box(&maps.dB, sm.M + q * kBoxBytes, 32 * q, g, row0);
+        }
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        bulk_wait_read();  // the staging is refilled by the next chunk
+      }
+    } else if (valid) {  // row r of dC (half 0) or dB (half 1), summed into global memory
       const size_t ro = (((size_t)b * L + tok) * G + g) * kNs;
       if (hf == 0) bulk_add_f32(p.dC + ro, stC, kNs * 4);
       else bulk_add_f32(p.dB + ro, stB, kNs * 4);
@@ -609,12 +648,13 @@ cudaError_t launch_ssd_bwd(const SsdArgs& a, cudaStream_t s) {
   SsdMaps maps;
   memset(&maps, 0, sizeof(maps));
   int tma = 0;
-  const SsdTensorMapEncode enc = a.L % 8 == 0 ? ssd_tensor_map_encoder() : nullptr;
-  if (enc) {
-    const size_t rows = (size_t)a.B * a.L;
-    tma = ssd_tile_map(enc, &maps.C, a.Cm, rows, a.G, kNs) && ssd_tile_map(enc, &maps.B, a.Bm, rows, a.G, kNs) &&
-          ssd_tile_map(enc, &maps.X, a.x, rows, a.H, kP) && ssd_tile_map(enc, &maps.dY, a.dy, rows, a.H, kP);
-  }
+  const SsdTensorMapEncode enc = ssd_tensor_map_encoder();
+  const size_t rows = (size_t)a.B * a.L;
+  if (enc && a.L % 8 == 0 && ssd_tile_map(enc, &maps.C, a.Cm, rows, a.G, kNs) &&
+      ssd_tile_map(enc, &maps.B, a.Bm, rows, a.G, kNs) && ssd_tile_map(enc, &maps.X, a.x, rows, a.H, kP) &&
+      ssd_tile_map(enc, &maps.dY, a.dy, rows, a.H, kP))
+    tma |= 1;
+  if (enc && ssd_sum_map(enc, &maps.dB, a.dB, rows, a.G) && ssd_sum_map(enc, &maps.dC, a.dC, rows, a.G)) tma |= 2;
   ssd_bwd_kernel<<<dim3(a.H, a.B), kThreads, smem, s>>>(a, maps, tma);
   return cudaGetLastError();
 }

@@ -1,4 +1,4 @@
-// Tensor maps for the SSD backward's operand tiles (host side). A map over a
+// Tensor maps for the SSD backward's operand tiles and dB / dC sums (host side). A map over a
 // row-major [rows][groups][features] bf16 tensor with five dimensions
 // (feature_lo 8, row_lo 8, feature_hi, group, row_hi) and a box of
 // (8, 8, features / 8, 1, 16) delivers 128 rows of one group into shared
@@ -47,6 +47,19 @@ inline bool ssd_tile_map(SsdTensorMapEncode enc, CUtensorMap* m, const void* bas
   const cuuint32_t es[5] = {1, 1, 1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A map over a [rows][groups][128] fp32 tensor for bulk reductions of boxes
+// of 32 states x 128 rows of one group, staged in shared memory in the
+// 128-byte swizzled order (16-byte chunk k of a box row r at k ^ (r & 7)).
+inline bool ssd_sum_map(SsdTensorMapEncode enc, CUtensorMap* m, void* base, size_t rows, int groups) {
+  const cuuint64_t dims[3] = {128, (cuuint64_t)groups, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {128 * 4, (cuuint64_t)groups * 128 * 4};
+  const cuuint32_t box[3] = {32, 1, 128};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 

@@ -71,6 +71,25 @@ __device__ __forceinline__ float2 cis(float theta) {
                      __uint_as_float(__float_as_uint(s) ^ ss));
 }
 
+// The same with sin and cos of the reduced angle on the special-function
+// unit (absolute error near 2^-21 on |r| <= pi/4): used with bf16 storage,
+// whose output rounding (2^-9) leaves that error far below the tolerance;
+// fp32 storage keeps the series above.
+__device__ __forceinline__ float2 cis_sfu(float theta) {
+  const float sh = fmaf(theta, 0.636619772f, 12582912.0f);  // theta 2/pi + 1.5 * 2^23
+  const int q = __float_as_int(sh);
+  const float k = sh - 12582912.0f;
+  float r = fmaf(-k, 1.57079637f, theta);                   // float(pi/2)
+  r = fmaf(-k, -4.37113883e-8f, r);                         // pi/2 - float(pi/2)
+  const float sn = __sinf(r), cs = __cosf(r);
+  const bool odd = q & 1;
+  const float c = odd ? sn : cs, s = odd ? cs : sn;
+  const unsigned sc = (unsigned)((q + 1) & 2) << 30;        // cos < 0 in quadrants 1, 2
+  const unsigned ss = (unsigned)(q & 2) << 30;              // sin < 0 in quadrants 2, 3
+  return make_float2(__uint_as_float(__float_as_uint(c) ^ sc),
+                     __uint_as_float(__float_as_uint(s) ^ ss));
+}
+
 // dt = softplus(v) with the accurate library exp / log1p: the phase dt Im A
 // magnifies dt's relative error by |Im A|, and dt is computed once per token
 // for all 16 states.
@@ -170,6 +189,8 @@ __device__ __forceinline__ unsigned block_resets(int sq, int sqp, int tok, int L
 
 // a_t = e^{dt Re A} e^{i dt Im A} for the block's 16 tokens (A's real part
 // pre-scaled by log2 e), 0 at a document start (rm: warp-uniform bit mask).
+// SFU: the angle's sin / cos on the special-function unit (bf16 storage).
+template <bool SFU>
 __device__ __forceinline__ void decays(const float4* dt4, float Ar2, float Ai, unsigned rm,
                                        float ar[kCB], float ai[kCB]) {
 #pragma unroll
@@ -179,7 +200,7 @@ __device__ __forceinline__ void decays(const float4* dt4, float Ar2, float Ai, u
     for (int j = 0; j < 4; ++j) {
       const float dt = comp(dq, j);
       const float mag = ex2_approx(dt * Ar2);
-      const float2 cs = cis(dt * Ai);
+      const float2 cs = SFU ? cis_sfu(dt * Ai) : cis(dt * Ai);
       ar[4 * q + j] = mag * cs.x;
       ai[4 * q + j] = mag * cs.y;
     }
@@ -286,7 +307,7 @@ cscan_fwd_kernel(const ScanArgs p) {
     if (nval) ck[(size_t)kb * kNMax] = make_float2(hr, hi);
     // the block's decays first (independent of h), then the serial chain
     float ar_[kCB], ai_[kCB];
-    decays(dt4, Ar2, Ai, rm, ar_, ai_);
+    decays<sizeof(T) == 2>(dt4, Ar2, Ai, rm, ar_, ai_);
 #pragma unroll
     for (int q = 0; q < kCB / 4; ++q) {
       const float4 xq = xu4[q], br = Br4[q], bi = Bi4[q], cr = Cr4[q], ci = Ci4[q];
@@ -464,7 +485,7 @@ cscan_bwd_kernel(const ScanArgs p) {
 
     // forward recompute of a_t and h_t over the block
     float Hr[kCB], Hi[kCB], Ar_[kCB], Ai_[kCB];
-    decays(dt4, Ar2, Ai, rm, Ar_, Ai_);
+    decays<sizeof(T) == 2>(dt4, Ar2, Ai, rm, Ar_, Ai_);
     {
       float hr = hck.x, hi = hck.y;
 #pragma unroll

@@ -8,7 +8,8 @@ import pytest
 
 import oracle
 import synth
-from pipeline import TOL_BF16_OUT, TOL_BF16_OUT_MAX, TOL_F32, TOL_GRAD, f32_dev, host64, max_abs, rel_l2, to_dev
+from pipeline import (TOL_BF16_OUT, TOL_BF16_OUT_MAX, TOL_F32, TOL_GRAD, bf16_out_max_abs_ok, f32_dev, host64,
+                      rel_l2, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -69,8 +70,9 @@ def _compare(ci, out, fs, gr, f, g, *, fp32, with_z, with_h0):
     want_out = f["out"] if fp32 else oracle.round_bf16(f["out"])
     errs["out"] = rel_l2(host64(out), want_out)
     assert errs["out"] <= (TOL_C32 if fp32 else TOL_BF16_OUT), errs
-    if not fp32:
-        assert max_abs(host64(out), want_out) <= TOL_BF16_OUT_MAX
+    if not fp32:  # one bf16 step allowed where |want| >= 4 (the same reading as the real scan's)
+        ok, worst = bf16_out_max_abs_ok(host64(out), want_out, TOL_BF16_OUT_MAX)
+        assert ok, worst
     errs["final_state"] = rel_l2(host64(fs), _pairs(f["final_state"]))
     assert errs["final_state"] <= (TOL_C32 if fp32 else TOL_GRAD), errs
     pairs = [("du", g["du"]), ("ddelta", g["ddelta"]), ("dA", _pairs(g["dA"])),

@@ -20,12 +20,17 @@
 // products): its own rounding would otherwise dominate the error of y.
 //
 // One CTA of 256 threads per (b, h): threads i and i + 128 own token i of
-// the chunk (and TMEM lane i), each for half of its columns; the next
-// chunk's global inputs are loaded into registers while the current one is
-// computed. No TMA multicast, no cluster.
+// the chunk (and TMEM lane i), each for half of its columns. The next
+// chunk's rows are fetched while the current one is computed: x into the
+// second of two x tiles at the chunk's start and B into the B tile once the
+// first product has released it, each by one tensor-map copy (cp.async for a
+// ragged last chunk or L not a multiple of 8), and C into registers. No TMA
+// multicast, no cluster.
 #include <atomic>
+#include <cstring>
 
 #include "scan_common.cuh"
+#include "ssd_maps.cuh"
 
 namespace ssm {
 
@@ -36,25 +41,27 @@ constexpr int kP = 64;   // head dimension
 constexpr int kNs = 128; // state size
 constexpr int kThreads = 256;  // two threads per token row
 
-// Shared memory: bf16 operands in the no-swizzle core-matrix layouts (every
-// operand has K = 128; core matrices 128 B apart along K, 2 KB apart along
-// M / N): K-major where a thread writes a row along K (C, B, the decay-masked
-// product), MN-major where it writes a row along M / N (x, the w-scaled B,
-// the state), so every thread stores 16-byte vectors.
+// Shared memory: bf16 operands in the no-swizzle core-matrix layouts (core
+// matrices 128 B apart along K, 2 KB apart along M / N): K-major where a row
+// runs along K (C, B, the decay-masked product), MN-major where a thread
+// writes a row along M / N (the w-scaled B, the state); x is stored by token
+// rows (8-row groups 1 KB apart, two buffers) and read MN-major by swapping
+// the descriptor's two strides.
 struct SsdSmem {
   unsigned char C[kQ * kNs * 2];    // C [i][n], then C' = C scaled by [ls_i < 0] exp(lcs_i)
   unsigned char Bm[kQ * kNs * 2];   // B [j][n]
   unsigned char M[kQ * kQ * 2];     // (C B^T o L) dt [i][j], rounded to bf16
   unsigned char Mlo[kQ * kQ * 2];   // its rounding remainder, rounded to bf16 (M = M + Mlo to ~2^-17)
   unsigned char Bw[kNs * kQ * 2];   // w_j B_j[n]: M = n, K = j, MN-major
-  unsigned char Xt[kP * kQ * 2];    // x_j[p]: N = p, K = j, MN-major
+  unsigned char X[2][kQ * kP * 2];  // x_j[p] of chunks c (buffer c & 1): rows j
   unsigned char Hb[kP * kNs * 2];   // H_prev[p][n]: N = p, K = n, MN-major
   float lcs[kQ];
   float dt[kQ];
   int ls[kQ];
   float wsum[4];
   int wmax[4];
-  uint64_t bar;
+  uint64_t bar;   // tensor-core products
+  uint64_t tbar;  // tensor-map copies of a chunk's B and x rows
   uint32_t tmem;
 };
 
@@ -80,20 +87,52 @@ __device__ __forceinline__ uint32_t umma_idesc(int n, int a_mn, int b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
          ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
 }
+// A descriptor with given leading (K-direction) and stride (M / N-direction)
+// byte offsets between core matrices.
+__device__ __forceinline__ uint64_t umma_desc2(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46);
+}
+// An x tile (token rows, 8-row groups 1 KB apart) read MN-major (N = p,
+// K = j): leading offset 1 KB, stride offset 128 B, 2 KB per K = 16 step.
+constexpr uint32_t kXRs = 1024;
+
 // D (+)= A B^T over K = 128 (eight K = 16 steps: two core matrices along K
-// each), A 128 x 128, B n x 128.
+// each), A 128 x 128, B n x 128; b_x: B is an x tile (MN-major view).
 __device__ __forceinline__ void umma_k128(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem, int n,
-                                          bool accumulate, int a_mn, int b_mn) {
+                                          bool accumulate, int a_mn, int b_mn, bool b_x = false) {
   const uint32_t idesc = umma_idesc(n, a_mn, b_mn);
 #pragma unroll
   for (int s = 0; s < 8; ++s) {
     const uint32_t acc = (accumulate || s > 0) ? 1u : 0u;
+    const uint64_t bd = b_x ? umma_desc2(b_smem + 2 * kXRs * s, kXRs, 128) : umma_desc(b_smem + 256 * s);
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(umma_desc(a_smem + 256 * s)), "l"(umma_desc(b_smem + 256 * s)), "r"(idesc), "r"(acc), "r"(0u),
-        "r"(0u), "r"(0u), "r"(0u));
+        "l"(umma_desc(a_smem + 256 * s)), "l"(bd), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
   }
+}
+
+// byte offset of (token j, feature p) in an x tile
+__device__ __forceinline__ uint32_t x_off(int j, int p) {
+  return (j >> 3) * kXRs + (p >> 3) * 128 + (j & 7) * 16 + (p & 7) * 2;
+}
+
+// One operand tile (128 rows of a row-major [rows][groups][features] bf16
+// tensor) by one tensor-map copy into the tiles' core-matrix order (see
+// ssd_maps.cuh); rows past the tensor are zero-filled.
+__device__ __forceinline__ void tma_tile(void* dst, const CUtensorMap* map, int group, int row_hi,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, "
+      "%5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(0), "r"(0), "r"(0), "r"(group), "r"(row_hi), "r"(smem_u32(bar))
+      : "memory");
+}
+// 16 bytes global -> shared without registers; nbytes 0 fills zeros (src unread)
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, uint32_t nbytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(nbytes)
+               : "memory");
 }
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -125,14 +164,21 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Global inputs of one chunk for one thread: half hf of token row r.
+// Register-fetched inputs of one chunk for one thread: half hf of token row r.
 struct ChunkIn {
-  uint4 c[8], b[8], x[4];  // C, B: n = 64 hf .. 64 hf + 63; x: p = 32 hf .. 32 hf + 31
-  float dtv;               // raw dt + bias (as read)
+  uint4 c[8];  // C: n = 64 hf .. 64 hf + 63
+  float dtv;   // raw dt + bias (as read)
   int seq_cur, seq_prev;
 };
 
-__global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
+struct SsdFwdMaps {
+  CUtensorMap B, X;
+};
+
+// maps: B ([B L][G][128]) and x ([B L][H][64]); tma false (L not a multiple
+// of 8, or no map could be encoded): B and x rows of every chunk by cp.async.
+__global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, const __grid_constant__ SsdFwdMaps maps,
+                                                              const int tma) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   SsdSmem& sm = *reinterpret_cast<SsdSmem*>(smem_raw);
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -155,22 +201,50 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
     const int tok = c * kQ + r;
     const bool valid = tok < L;
     const uint4* crow = reinterpret_cast<const uint4*>(Cg + (((size_t)b * L + tok) * G + g) * kNs) + 8 * hf;
-    const uint4* brow = reinterpret_cast<const uint4*>(Bg + (((size_t)b * L + tok) * G + g) * kNs) + 8 * hf;
-    const uint4* xrow = reinterpret_cast<const uint4*>(xg + (((size_t)b * L + tok) * H + h) * kP) + 4 * hf;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      in.c[k] = valid ? __ldg(crow + k) : z4;
-      in.b[k] = valid ? __ldg(brow + k) : z4;
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) in.x[k] = valid ? __ldg(xrow + k) : z4;
+    for (int k = 0; k < 8; ++k) in.c[k] = valid ? __ldg(crow + k) : z4;
     in.dtv = valid ? __bfloat162float(dtg[((size_t)b * L + tok) * H + h]) + bias : 0.0f;
     in.seq_cur = (seqb && valid) ? __ldg(seqb + tok) : 0;
     in.seq_prev = (seqb && valid && tok > 0) ? __ldg(seqb + tok - 1) : in.seq_cur;
   };
+  const int nch = (L + kQ - 1) / kQ;
+  auto by_map = [&](int cc) { return tma && (cc + 1) * kQ <= L; };
+  // chunk cc's x rows into x tile cc & 1 (the first of its two copies:
+  // arms the chunk's copy barrier for x and B together)
+  auto load_x = [&](int cc) {
+    unsigned char* xt = sm.X[cc & 1];
+    if (by_map(cc)) {
+      if (t == 0) {
+        mbar_expect_tx(&sm.tbar, (unsigned)(kQ * kNs * 2 + kQ * kP * 2));
+        tma_tile(xt, &maps.X, h, (int)(((size_t)b * L + (size_t)cc * kQ) / 8), &sm.tbar);
+      }
+    } else {
+      const int tk = cc * kQ + r;
+      const int tc = tk < L ? tk : 0;  // an in-bounds source when zero-filling
+      const uint4* xrow = reinterpret_cast<const uint4*>(xg + (((size_t)b * L + tc) * H + h) * kP) + 4 * hf;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) cp_async16(xt + x_off(r, 8 * (4 * hf + k)), xrow + k, tk < L ? 16u : 0u);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+  };
+  // chunk cc's B rows into the B tile
+  auto load_b = [&](int cc) {
+    if (by_map(cc)) {
+      if (t == 0) tma_tile(sm.Bm, &maps.B, g, (int)(((size_t)b * L + (size_t)cc * kQ) / 8), &sm.tbar);
+    } else {
+      const int tk = cc * kQ + r;
+      const int tc = tk < L ? tk : 0;
+      const uint4* brow = reinterpret_cast<const uint4*>(Bg + (((size_t)b * L + tc) * G + g) * kNs) + 8 * hf;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) cp_async16(sm.Bm + tile_off(r, 8 * (8 * hf + k)), brow + k, tk < L ? 16u : 0u);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+  };
+  unsigned tphase = 0;
 
   if (t == 0) {
     mbar_init(&sm.bar, 1);
+    mbar_init(&sm.tbar, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -188,16 +262,17 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
   const uint32_t lane_row = tmem + ((uint32_t)(32 * (warp & 3)) << 16);  // TMEM lane r
   // TMEM columns: S [0, 128), Y [128, 192), chunk state S_c^T [192, 256)
   const uint32_t sC = smem_u32(sm.C), sB = smem_u32(sm.Bm), sM = smem_u32(sm.M);
-  const uint32_t sBw = smem_u32(sm.Bw), sX = smem_u32(sm.Xt), sH = smem_u32(sm.Hb);
+  const uint32_t sBw = smem_u32(sm.Bw), sH = smem_u32(sm.Hb);
   const uint32_t sMlo = smem_u32(sm.Mlo);
 
   float Ht[kP / 2];  // H^T[n = r][p = 32 hf ..], fp32 across the chunks
 #pragma unroll
   for (int q = 0; q < kP / 2; ++q) Ht[q] = 0.0f;
   unsigned phase = 0;
-  const int nch = (L + kQ - 1) / kQ;
   ChunkIn in;
   fetch(0, in);
+  load_x(0);
+  load_b(0);
 
 #pragma unroll 1
   for (int c = 0; c < nch; ++c) {
@@ -209,20 +284,34 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
 #pragma unroll
       for (int q = 0; q < kP / 8; ++q) cs[q] = make_float4(Ht[4 * q], Ht[4 * q + 1], Ht[4 * q + 2], Ht[4 * q + 3]);
     }
-    // ---- this chunk's operands into shared memory ----
+    // ---- this chunk's operands: C from registers; B and x tile c & 1 copied
+    // during the previous chunk ----
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < 8; ++k)
       *reinterpret_cast<uint4*>(sm.C + tile_off(r, 8 * (8 * hf + k))) = in.c[k];
-      *reinterpret_cast<uint4*>(sm.Bm + tile_off(r, 8 * (8 * hf + k))) = in.b[k];
+    {
+      bool ok = true;
+      if (by_map(c)) {
+        ok = mbar_wait_bounded(&sm.tbar, tphase, p.status);
+        tphase ^= 1u;
+      } else {
+        asm volatile("cp.async.wait_all;" ::: "memory");
+      }
+      if (!__syncthreads_and(ok)) {
+        // the copies have not landed: wait once more (bounded) so that they
+        // do not land after the CTA has exited, then stop
+        if (t == 0) mbar_wait_bounded(&sm.tbar, tphase ^ 1u, nullptr);
+        break;
+      }
     }
+    const unsigned char* xt = sm.X[c & 1];
+    const uint32_t sX = smem_u32(xt);
+    uint4 xraw[4];  // x of token r, p = 32 hf .., for the D x term
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
-      *reinterpret_cast<uint4*>(sm.Xt + tile_off_mn(8 * (4 * hf + k), r)) = in.x[k];
-    uint4 braw[8], xraw[4];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) braw[k] = in.b[k];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) xraw[k] = in.x[k];
+    for (int k = 0; k < 4; ++k) xraw[k] = *reinterpret_cast<const uint4*>(xt + x_off(r, 8 * (4 * hf + k)));
+    // the next chunk's x into the other tile, now (its last readers were the
+    // previous chunk's products)
+    if (c + 1 < nch) load_x(c + 1);
     float dt = 0.0f;
     if (valid) dt = p.softplus ? (in.dtv > 20.0f ? in.dtv : log1pf(expf(in.dtv))) : in.dtv;
     const bool start = valid && seqb && tok > 0 && in.seq_cur != in.seq_prev;
@@ -265,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
     const float wt = (r >= lsQ) ? dt * __expf(lcsQ - la) : 0.0f;
 #pragma unroll
     for (int k = 0; k < 8; ++k) {  // n = 8 (8 hf + k) .. of token r
-      const uint4 q = braw[k];
+      const uint4 q = *reinterpret_cast<const uint4*>(sm.Bm + tile_off(r, 8 * (8 * hf + k)));
       *reinterpret_cast<uint4*>(sm.Bw + tile_off_mn(8 * (8 * hf + k), r)) =
           make_uint4(pack_bf16(bf_lo(q.x) * wt, bf_hi(q.x) * wt), pack_bf16(bf_lo(q.y) * wt, bf_hi(q.y) * wt),
                      pack_bf16(bf_lo(q.z) * wt, bf_hi(q.z) * wt), pack_bf16(bf_lo(q.w) * wt, bf_hi(q.w) * wt));
@@ -283,6 +372,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
     phase ^= 1u;
     if (!__syncthreads_and(ok)) break;
     tc_fence_after();
+    // the B tile is free: the next chunk's B rows into it
+    if (c + 1 < nch) load_b(c + 1);
     // ---- columns 64 hf .. 64 hf + 63 of row r of M = (C B^T o L) dt (pair hi / lo), row r of C' ----
     uint32_t sraw[64];
     tmem_ld32(lane_row + 64 * hf, sraw);
@@ -330,10 +421,10 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
     __syncthreads();
     tc_fence_after();
     if (t == 0) {
-      umma_k128(tmem + 128, sM, sX, kP, false, 0, 1);
-      umma_k128(tmem + 128, sMlo, sX, kP, true, 0, 1);
+      umma_k128(tmem + 128, sM, sX, kP, false, 0, 1, true);
+      umma_k128(tmem + 128, sMlo, sX, kP, true, 0, 1, true);
       umma_k128(tmem + 128, sC, sH, kP, true, 0, 1);
-      umma_k128(tmem + 192, sBw, sX, kP, false, 1, 1);
+      umma_k128(tmem + 192, sBw, sX, kP, false, 1, 1, true);
       umma_commit(&sm.bar);
     }
     ok = mbar_wait_bounded(&sm.bar, phase, p.status);
@@ -373,6 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p) {
     tc_fence_before();
     __syncthreads();  // every thread is done with this chunk's shared operands and TMEM
   }
+  asm volatile("cp.async.wait_all;" ::: "memory");  // no copy lands after the CTA has exited
   if (p.final_state) {
 #pragma unroll
     for (int q = 0; q < kP / 2; ++q)
@@ -392,7 +484,15 @@ cudaError_t launch_ssd_fwd(const SsdArgs& a, cudaStream_t s) {
   const int smem = (int)sizeof(SsdSmem);
   cudaError_t e = smem_attr(ssd_fwd_kernel, smem, &done);
   if (e != cudaSuccess) return e;
-  ssd_fwd_kernel<<<dim3(a.H, a.B), kThreads, smem, s>>>(a);
+  SsdFwdMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  int tma = 0;
+  const SsdTensorMapEncode enc = a.L % 8 == 0 ? ssd_tensor_map_encoder() : nullptr;
+  if (enc) {
+    const size_t rows = (size_t)a.B * a.L;
+    tma = ssd_tile_map(enc, &maps.B, a.Bm, rows, a.G, kNs) && ssd_tile_map(enc, &maps.X, a.x, rows, a.H, kP);
+  }
+  ssd_fwd_kernel<<<dim3(a.H, a.B), kThreads, smem, s>>>(a, maps, tma);
   return cudaGetLastError();
 }
 

@@ -1,4 +1,5 @@
-// Tensor maps for the SSD backward's operand tiles and dB / dC sums (host side). A map over a
+// Tensor maps for the SSD kernels' operand tiles and the backward's dB / dC
+// sums (host side). A map over a
 // row-major [rows][groups][features] bf16 tensor with five dimensions
 // (feature_lo 8, row_lo 8, feature_hi, group, row_hi) and a box of
 // (8, 8, features / 8, 1, 16) delivers 128 rows of one group into shared
@@ -6,7 +7,7 @@
 //   (row >> 3) * (features * 16) + (feature >> 3) * 128 + (row & 7) * 16 + (feature & 7) * 2,
 // rows past the tensor zero-filled. The encoder comes from the driver
 // through the runtime's entry-point query, so the library links no driver
-// library; without it the kernel copies rows with cp.async.
+// library; without it the kernels copy rows with cp.async.
 #pragma once
 
 #include <cuda.h>

@@ -15,9 +15,11 @@
 // mbarrier (bounded waits). Operands are written by the CTA's threads into
 // shared memory in the K-major, no-swizzle core-matrix layout; the state
 // H^T[n][p] stays in fp32 registers (thread n) across the chunks of a
-// sequence and enters the next chunk's product as bf16. The decay-masked
-// C B^T enters as a bf16 pair (rounded value and rounded remainder, two
-// products): its own rounding would otherwise dominate the error of y.
+// sequence. The decay-masked C B^T and the state entering the next chunk
+// each enter as a bf16 pair (rounded value and rounded remainder, two
+// products), and C H_prev^T takes its row scale in fp32 afterwards (C itself
+// is exact in bf16): single bf16 roundings there would dominate the error of
+// y, the state's wherever the off-chunk term is large against y.
 //
 // One CTA of 256 threads per (b, h): threads i and i + 128 own token i of
 // the chunk (and TMEM lane i), each for half of its columns. The next
@@ -48,13 +50,14 @@ constexpr int kThreads = 256;  // two threads per token row
 // rows (8-row groups 1 KB apart, two buffers) and read MN-major by swapping
 // the descriptor's two strides.
 struct SsdSmem {
-  unsigned char C[kQ * kNs * 2];    // C [i][n], then C' = C scaled by [ls_i < 0] exp(lcs_i)
+  unsigned char C[kQ * kNs * 2];    // C [i][n]
   unsigned char Bm[kQ * kNs * 2];   // B [j][n]
   unsigned char M[kQ * kQ * 2];     // (C B^T o L) dt [i][j], rounded to bf16
   unsigned char Mlo[kQ * kQ * 2];   // its rounding remainder, rounded to bf16 (M = M + Mlo to ~2^-17)
   unsigned char Bw[kNs * kQ * 2];   // w_j B_j[n]: M = n, K = j, MN-major
   unsigned char X[2][kQ * kP * 2];  // x_j[p] of chunks c (buffer c & 1): rows j
-  unsigned char Hb[kP * kNs * 2];   // H_prev[p][n]: N = p, K = n, MN-major
+  unsigned char Hb[kP * kNs * 2];   // H_prev[p][n]: N = p, K = n, MN-major, rounded to bf16
+  unsigned char Hlo[kP * kNs * 2];  // its rounding remainder, rounded to bf16 (H_prev to ~2^-17)
   float lcs[kQ];
   float dt[kQ];
   int ls[kQ];
@@ -179,6 +182,7 @@ struct SsdFwdMaps {
 // of 8, or no map could be encoded): B and x rows of every chunk by cp.async.
 __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, const __grid_constant__ SsdFwdMaps maps,
                                                               const int tma) {
+  static_assert(sizeof(SsdSmem) <= 227 * 1024, "shared memory per CTA");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   SsdSmem& sm = *reinterpret_cast<SsdSmem*>(smem_raw);
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -248,21 +252,22 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
     fence_mbar_init();
   }
   if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 256;" ::"r"(smem_u32(&sm.tmem))
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(&sm.tmem))
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   // H_prev = 0 before the first chunk
   for (int i = t; i < kP * kNs * 2 / 16; i += kThreads)
-    reinterpret_cast<uint4*>(sm.Hb)[i] = make_uint4(0u, 0u, 0u, 0u);
+    reinterpret_cast<uint4*>(sm.Hb)[i] = reinterpret_cast<uint4*>(sm.Hlo)[i] = make_uint4(0u, 0u, 0u, 0u);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem;
   const uint32_t lane_row = tmem + ((uint32_t)(32 * (warp & 3)) << 16);  // TMEM lane r
-  // TMEM columns: S [0, 128), Y [128, 192), chunk state S_c^T [192, 256)
+  // TMEM columns: S [0, 128), Y_diag [128, 192), chunk state S_c^T [192, 256),
+  // C H_prev^T [256, 320)
   const uint32_t sC = smem_u32(sm.C), sB = smem_u32(sm.Bm), sM = smem_u32(sm.M);
-  const uint32_t sBw = smem_u32(sm.Bw), sH = smem_u32(sm.Hb);
+  const uint32_t sBw = smem_u32(sm.Bw), sH = smem_u32(sm.Hb), sHlo = smem_u32(sm.Hlo);
   const uint32_t sMlo = smem_u32(sm.Mlo);
 
   float Ht[kP / 2];  // H^T[n = r][p = 32 hf ..], fp32 across the chunks
@@ -374,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
     tc_fence_after();
     // the B tile is free: the next chunk's B rows into it
     if (c + 1 < nch) load_b(c + 1);
-    // ---- columns 64 hf .. 64 hf + 63 of row r of M = (C B^T o L) dt (pair hi / lo), row r of C' ----
+    // ---- columns 64 hf .. 64 hf + 63 of row r of M = (C B^T o L) dt (pair hi / lo) ----
     uint32_t sraw[64];
     tmem_ld32(lane_row + 64 * hf, sraw);
     tmem_ld32(lane_row + 64 * hf + 32, sraw + 32);
@@ -405,17 +410,10 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
                        pack_bf16(rr[6], rr[7]));
       }
     }
-    {
-      const float cs = st < 0 ? __expf(la) : 0.0f;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        uint4* q = reinterpret_cast<uint4*>(sm.C + tile_off(r, 8 * (8 * hf + k)));
-        const uint4 cv = *q;
-        *q = make_uint4(pack_bf16(bf_lo(cv.x) * cs, bf_hi(cv.x) * cs), pack_bf16(bf_lo(cv.y) * cs, bf_hi(cv.y) * cs),
-                        pack_bf16(bf_lo(cv.z) * cs, bf_hi(cv.z) * cs), pack_bf16(bf_lo(cv.w) * cs, bf_hi(cv.w) * cs));
-      }
-    }
-    // ---- Y = M x + C' H_prev^T and S_c^T = (diag(w) B)^T x ----
+    // the off-chunk term's row scale, applied in fp32 in the epilogue (C enters
+    // the product as given: exact in bf16)
+    const float cs = st < 0 ? __expf(la) : 0.0f;
+    // ---- Y_diag = M x, C H_prev^T (H_prev as a bf16 pair) and S_c^T = (diag(w) B)^T x ----
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     __syncthreads();
@@ -423,7 +421,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
     if (t == 0) {
       umma_k128(tmem + 128, sM, sX, kP, false, 0, 1, true);
       umma_k128(tmem + 128, sMlo, sX, kP, true, 0, 1, true);
-      umma_k128(tmem + 128, sC, sH, kP, true, 0, 1);
+      umma_k128(tmem + 256, sC, sH, kP, false, 0, 1);
+      umma_k128(tmem + 256, sC, sHlo, kP, true, 0, 1);
       umma_k128(tmem + 192, sBw, sX, kP, false, 1, 1, true);
       umma_commit(&sm.bar);
     }
@@ -433,9 +432,10 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
     tc_fence_after();
     // ---- y row r (p = 32 hf ..); the state row n = r (p = 32 hf ..) ----
     {
-      uint32_t yv[32], sv[32];
+      uint32_t yv[32], sv[32], ov[32];
       tmem_ld32(lane_row + 128 + 32 * hf, yv);
       tmem_ld32(lane_row + 192 + 32 * hf, sv);
+      tmem_ld32(lane_row + 256 + 32 * hf, ov);
       tmem_wait();
       if (valid) {
         uint4* yrow = reinterpret_cast<uint4*>(yg + (((size_t)b * L + tok) * H + h) * kP) + 4 * hf;
@@ -446,8 +446,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int q = 8 * k + 2 * e;
-            o[e] = pack_bf16(fmaf(Dh, bf_lo(w4[e]), __uint_as_float(yv[q])),
-                             fmaf(Dh, bf_hi(w4[e]), __uint_as_float(yv[q + 1])));
+            o[e] = pack_bf16(fmaf(Dh, bf_lo(w4[e]), fmaf(cs, __uint_as_float(ov[q]), __uint_as_float(yv[q]))),
+                             fmaf(Dh, bf_hi(w4[e]), fmaf(cs, __uint_as_float(ov[q + 1]), __uint_as_float(yv[q + 1]))));
           }
           yrow[k] = make_uint4(o[0], o[1], o[2], o[3]);
         }
@@ -456,10 +456,20 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
 #pragma unroll
       for (int q = 0; q < kP / 2; ++q) Ht[q] = fmaf(dec, Ht[q], __uint_as_float(sv[q]));
 #pragma unroll
-      for (int k = 0; k < 4; ++k)  // p = 8 (4 hf + k) .. of state row n = r
-        *reinterpret_cast<uint4*>(sm.Hb + tile_off_mn(8 * (4 * hf + k), r)) =
-            make_uint4(pack_bf16(Ht[8 * k], Ht[8 * k + 1]), pack_bf16(Ht[8 * k + 2], Ht[8 * k + 3]),
-                       pack_bf16(Ht[8 * k + 4], Ht[8 * k + 5]), pack_bf16(Ht[8 * k + 6], Ht[8 * k + 7]));
+      for (int k = 0; k < 4; ++k) {  // p = 8 (4 hf + k) .. of state row n = r: rounded value and remainder
+        const uint4 hi = make_uint4(pack_bf16(Ht[8 * k], Ht[8 * k + 1]), pack_bf16(Ht[8 * k + 2], Ht[8 * k + 3]),
+                                    pack_bf16(Ht[8 * k + 4], Ht[8 * k + 5]), pack_bf16(Ht[8 * k + 6], Ht[8 * k + 7]));
+        const uint32_t hw[4] = {hi.x, hi.y, hi.z, hi.w};
+        float rr[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          rr[2 * e] = Ht[8 * k + 2 * e] - bf_lo(hw[e]);
+          rr[2 * e + 1] = Ht[8 * k + 2 * e + 1] - bf_hi(hw[e]);
+        }
+        *reinterpret_cast<uint4*>(sm.Hb + tile_off_mn(8 * (4 * hf + k), r)) = hi;
+        *reinterpret_cast<uint4*>(sm.Hlo + tile_off_mn(8 * (4 * hf + k), r)) =
+            make_uint4(pack_bf16(rr[0], rr[1]), pack_bf16(rr[2], rr[3]), pack_bf16(rr[4], rr[5]), pack_bf16(rr[6], rr[7]));
+      }
     }
     tc_fence_before();
     __syncthreads();  // every thread is done with this chunk's shared operands and TMEM
@@ -474,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
   __syncthreads();
   tc_fence_after();
   if (warp == 0)
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 256;" ::"r"(tmem) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
 }
 
 }  // namespace

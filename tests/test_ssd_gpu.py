@@ -50,7 +50,7 @@ def _check(y, fs, want):
 
 
 @pytest.mark.parametrize("B,L,H,G,nb", [(1, 128, 1, 1, 0), (1, 256, 2, 1, 0), (2, 300, 4, 2, 3),
-                                        (1, 1000, 3, 1, 6), (2, 77, 2, 2, 2)])
+                                        (1, 1000, 3, 1, 6), (2, 77, 2, 2, 2), (2, 520, 4, 2, 2)])
 def test_ssd_fwd_parity(B, L, H, G, nb):
     seed = 7100 + L + H
     seq = None
@@ -114,10 +114,13 @@ def _check_bwd(got, want):
 
 
 @pytest.mark.parametrize("B,L,H,G,nb", [(1, 128, 1, 1, 0), (1, 256, 2, 1, 0), (2, 300, 4, 2, 3),
-                                        (1, 1000, 3, 1, 6), (2, 77, 2, 2, 2)])
+                                        (1, 1000, 3, 1, 6), (2, 77, 2, 2, 2), (2, 520, 4, 2, 2)])
 def test_ssd_bwd_parity(B, L, H, G, nb):
     """Every gradient against the oracle: one chunk, several, a ragged tail,
-    two heads per B / C group (dB, dC summed over them), document starts."""
+    two heads per B / C group (dB, dC summed over them), document starts.
+    L a multiple of 8 takes the tensor-map copies for whole chunks (with two
+    batch entries at L = 520: rows offset by the batch, and the ragged last
+    chunk's dB / dC boxes reaching into the next entry's rows with zeros)."""
     seed = 7500 + L + H
     seq = None
     if nb:

@@ -28,6 +28,9 @@
 // copy. Two groups of products per chunk: (C B^T, dy x^T, B dH, C Hp,
 // C^T dYs) and, once M and dS are in shared memory, (M^T dy, dS B + dYs Hp^T,
 // dS^T C, x dH^T); the second runs while the threads reduce the decay terms.
+// A whole chunk's C, B, x, dy rows arrive by one tensor-map copy each (a
+// ragged last chunk, or L not a multiple of 8, by cp.async), and dB / dC
+// leave by tensor-map bulk reductions of staged boxes (see ssd_maps.cuh).
 // One CTA of 256 threads per (b, h); 512 TMEM columns.
 #include <atomic>
 #include <cstring>

@@ -79,7 +79,7 @@ typedef enum { SSM_DTYPE_F32 = 0, SSM_DTYPE_BF16 = 1 } ssm_dtype_t;
 const char* ssm_last_error(void);
 
 /* ABI version of this header (bumped on any incompatible change). */
-#define SSM_ABI_VERSION 7
+#define SSM_ABI_VERSION 8
 int ssm_abi_version(void);
 
 /* ---------------------------------------------------------------------------
@@ -493,6 +493,46 @@ typedef struct {
 } ssm_ssd_grads;
 
 ssm_status_t ssm_ssd_bwd(const ssm_ssd_params* p, const ssm_ssd_grads* g, ssm_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Debug build: device-side index checks (the library compiled with
+ * -DSSM_DEBUG; a release build carries no checks and both calls below return
+ * SSM_ERR_UNSUPPORTED without touching the device).
+ *
+ * In a debug build the kernels check the element offsets of their global
+ * accesses against the extents the call's shapes give their buffers: every
+ * activation and B / C row against [B][D][L] (or [B][L][H][P], [B][L][G][N]
+ * for the SSD), the tokens a thread touches against its row, the checkpoint
+ * and chunk-state arrays, the dB / dC sums and partials, the conv1d partials
+ * against the workspace they were sized in, the recurrent state. A failed check
+ * is counted, the first failure of each kernel source is kept, and the
+ * access is redirected to the first element of its range, so the kernel ends
+ * normally: no trap, no fault, no skipped barrier. Outputs of a call with a
+ * failed check are invalid. Checks are compiled in one library per build;
+ * there is no run-time switch.
+ *
+ * ssm_debug_report SYNCHRONISES the current device, then fills *out with
+ * the failures since the last reset (summed over kernel sources) and one
+ * kept failure (site id and name, offset, count, extent; site 0 "none" when
+ * there was none); reset != 0 clears the records. Records are per device.
+ *
+ * ssm_debug_selftest launches one thread that writes through offset n of
+ * `buf` (n >= 1 floats of device memory): its check fails, is recorded with
+ * offset n, count 1, extent n, and the write lands on buf[0]. It exists to
+ * show that a failing check is seen; it reads nothing of the layer's math.
+ * ------------------------------------------------------------------------ */
+typedef struct ssm_debug_info {
+  size_t struct_size;            /* = sizeof(ssm_debug_info) */
+  unsigned long long failures;   /* failed checks since the last reset */
+  int site;                      /* id of the kept failure (0: none) */
+  long long offset;              /* its element offset */
+  long long count;               /* elements the access touches from there */
+  long long extent;              /* extent the offset was held to */
+  char site_name[48];            /* printable name of the site */
+} ssm_debug_info;
+
+ssm_status_t ssm_debug_report(ssm_debug_info* out, int reset);
+ssm_status_t ssm_debug_selftest(float* buf, size_t n, ssm_stream_t stream);
 
 #ifdef __cplusplus
 }

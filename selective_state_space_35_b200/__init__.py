@@ -23,7 +23,8 @@ from ._lib import (SsmError, ssm_abi_version, ssm_conv1d_bwd, ssm_conv1d_bwd_noa
                    ssm_scan_fwd, ssm_scan_grads, ssm_scan_params, ssm_scan_workspace_size,
                    ssm_scan_bwd_workspace_size, ssm_ssd_params, ssm_ssd_fwd,
                    ssm_ssd_grads, ssm_ssd_bwd, ssm_scan_fwd_summary, ssm_scan_bwd_summary, ssm_state_carry,
-                   ssm_conv1d_fwd_ctx, ssm_conv1d_bwd_ctx)
+                   ssm_conv1d_fwd_ctx, ssm_conv1d_bwd_ctx, ssm_debug_info, ssm_debug_report,
+                   ssm_debug_selftest)
 
 __all__ = [
     "SsmError", "ssm_abi_version", "ssm_last_error", "ssm_conv1d_fwd", "ssm_conv1d_bwd",
@@ -36,7 +37,8 @@ __all__ = [
     "ssm_decode_params", "ssm_decode_step", "decode_step", "ssm_conv1d_scan_fwd",
     "conv1d_scan_fwd", "ssm_scan_fwd_summary", "ssm_scan_bwd_summary", "ssm_state_carry",
     "ssm_conv1d_fwd_ctx", "ssm_conv1d_bwd_ctx", "scan_fwd_summary", "scan_bwd_summary",
-    "state_carry",
+    "state_carry", "ssm_debug_info", "ssm_debug_report", "ssm_debug_selftest", "debug_report",
+    "debug_selftest",
 ]
 
 load = _lib.load
@@ -553,3 +555,26 @@ def ssd_bwd(x, dt_raw, A, Bm, Cm, dy, chunk_states, *, D=None, dt_bias=None, sof
     g.ddt_bias = out["ddt_bias"].data_ptr() if out["ddt_bias"] is not None else None
     _lib.check(ssm_ssd_bwd(p, g, _stream(stream, x.device)))
     return out
+
+
+def debug_report(reset: bool = False) -> dict:
+    """Failed device index checks of a debug build (SSM_LIBRARY naming the
+    library built with -DSSM_DEBUG): synchronises the device and returns
+    dict(failures, site, site_name, offset, count, extent) of the first kept
+    failure; reset clears the records. A release build raises SsmError
+    (SSM_ERR_UNSUPPORTED)."""
+    info = ssm_debug_info()
+    info.struct_size = ctypes.sizeof(ssm_debug_info)
+    _lib.check(ssm_debug_report(ctypes.byref(info), 1 if reset else 0))
+    return dict(failures=int(info.failures), site=int(info.site),
+                site_name=info.site_name.decode(errors="replace"), offset=int(info.offset),
+                count=int(info.count), extent=int(info.extent))
+
+
+def debug_selftest(buf, stream=None) -> None:
+    """Debug build only: one write through offset buf.numel() of the fp32
+    device tensor `buf`, which its check turns into a recorded failure and a
+    write to buf[0]."""
+    torch = _torch()
+    _need(buf, "buf", torch.float32)
+    _lib.check(ssm_debug_selftest(_ptr(buf), buf.numel(), _stream(stream, buf.device)))

@@ -96,6 +96,16 @@ class ssm_decode_params(ctypes.Structure):
     ]
 
 
+class ssm_debug_info(ctypes.Structure):
+    _fields_ = [
+        ("struct_size", _sz),
+        ("failures", ctypes.c_ulonglong),
+        ("site", _i),
+        ("offset", ctypes.c_longlong), ("count", ctypes.c_longlong), ("extent", ctypes.c_longlong),
+        ("site_name", ctypes.c_char * 48),
+    ]
+
+
 _lib = None
 
 EXPORTS = ("ssm_last_error", "ssm_abi_version", "ssm_conv1d_fwd", "ssm_conv1d_bwd_workspace_size",
@@ -103,7 +113,7 @@ EXPORTS = ("ssm_last_error", "ssm_abi_version", "ssm_conv1d_fwd", "ssm_conv1d_bw
            "ssm_scan_bwd", "ssm_scan_bwd_workspace_size", "ssm_scan_status", "ssm_probe_ex2_rate", "ssm_decode_step",
            "ssm_conv1d_scan_fwd", "ssm_scan_fwd_summary", "ssm_scan_bwd_summary",
            "ssm_state_carry", "ssm_conv1d_fwd_ctx", "ssm_conv1d_bwd_ctx", "ssm_ssd_fwd",
-           "ssm_ssd_bwd")
+           "ssm_ssd_bwd", "ssm_debug_report", "ssm_debug_selftest")
 
 
 def load(path: str | None = None):
@@ -163,6 +173,10 @@ def load(path: str | None = None):
     L.ssm_conv1d_bwd_ctx.restype = _i
     L.ssm_conv1d_bwd_ctx.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                      _vp, _i, _i, _i, _i, _i, _i, _vp, _sz, _vp]
+    L.ssm_debug_report.restype = _i
+    L.ssm_debug_report.argtypes = [ctypes.POINTER(ssm_debug_info), _i]
+    L.ssm_debug_selftest.restype = _i
+    L.ssm_debug_selftest.argtypes = [_vp, _sz, _vp]
     if path is None:
         _lib = L
     return L
@@ -271,3 +285,11 @@ def ssm_ssd_fwd(params: ssm_ssd_params, stream) -> int:
 
 def ssm_ssd_bwd(params: ssm_ssd_params, grads: ssm_ssd_grads, stream) -> int:
     return load().ssm_ssd_bwd(ctypes.byref(params), ctypes.byref(grads), stream)
+
+
+def ssm_debug_report(info, reset) -> int:
+    return load().ssm_debug_report(info, reset)
+
+
+def ssm_debug_selftest(buf, n, stream) -> int:
+    return load().ssm_debug_selftest(buf, n, stream)

@@ -13,6 +13,9 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libssmscan.so")
 OBJDIR = os.path.join(HERE, "_build")
+# the same sources with the device index checks compiled in (-DSSM_DEBUG)
+DEBUG_LIB = os.path.join(HERE, "libssmscan_debug.so")
+DEBUG_OBJDIR = os.path.join(HERE, "_build_debug")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE,
@@ -35,10 +38,10 @@ def _deps():
         os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(INCLUDE, "*.h")) + [__file__]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
@@ -49,6 +52,8 @@ def build(force: bool = False, verbose: bool = False, out: str | None = None,
     objdir = OBJDIR if out is None else out + ".objs"
     if out is None and not force and not defines and up_to_date():
         return LIB
+    if out == DEBUG_LIB:
+        objdir = DEBUG_OBJDIR
     os.makedirs(objdir, exist_ok=True)
     cc = nvcc()
     srcs = _sources()
@@ -76,6 +81,14 @@ def build(force: bool = False, verbose: bool = False, out: str | None = None,
     return lib
 
 
+def build_debug(force: bool = False) -> str:
+    """Compile the debug library (device index checks, -DSSM_DEBUG) in-tree;
+    select it at run time with SSM_LIBRARY=<its path>."""
+    if not force and up_to_date(DEBUG_LIB):
+        return DEBUG_LIB
+    return build(force=True, out=DEBUG_LIB, defines=("SSM_DEBUG",))
+
+
 if __name__ == "__main__":
     import argparse
     ap = argparse.ArgumentParser()
@@ -83,5 +96,9 @@ if __name__ == "__main__":
     ap.add_argument("-v", action="store_true")
     ap.add_argument("--out", default=None, help="write the library here instead of in-tree")
     ap.add_argument("-D", action="append", default=[], help="preprocessor define (repeatable)")
+    ap.add_argument("--debug", action="store_true", help="build the debug library (index checks)")
     a = ap.parse_args()
-    print(build(force=a.force, verbose=a.v, out=a.out, defines=tuple(a.D)))
+    if a.debug:
+        print(build_debug(force=a.force))
+    else:
+        print(build(force=a.force, verbose=a.v, out=a.out, defines=tuple(a.D)))

@@ -823,3 +823,75 @@ ssm_status_t ssm_ssd_bwd(const ssm_ssd_params* p, const ssm_ssd_grads* g, ssm_st
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Debug build (-DSSM_DEBUG): records of the device index checks (debug.cuh)
+// ---------------------------------------------------------------------------
+namespace ssm {
+#ifdef SSM_DEBUG
+namespace {
+// Writes through offset n of a buffer of n floats: the check fails, records
+// (kDbgSelftest, n, 1, n) and hands back offset 0, so buf[0] is written.
+__global__ void debug_selftest_kernel(float* buf, long long n) {
+  buf[SSM_DIDX(kDbgSelftest, n, 1, n)] = 1.0f;
+}
+}  // namespace
+
+cudaError_t launch_debug_selftest(float* buf, long long n, cudaStream_t s) {
+  debug_selftest_kernel<<<1, 1, 0, s>>>(buf, n);
+  return cudaGetLastError();
+}
+
+SSM_DEBUG_TU(abi)
+#endif
+}  // namespace ssm
+
+extern "C" {
+
+ssm_status_t ssm_debug_report(ssm_debug_info* out, int reset) {
+  if (!out) return fail(SSM_ERR_INVALID_ARG, "out is NULL");
+  if (out->struct_size != sizeof(ssm_debug_info))
+    return fail(SSM_ERR_INVALID_ARG, "struct_size %zu != %zu", out->struct_size, sizeof(ssm_debug_info));
+#ifndef SSM_DEBUG
+  (void)reset;
+  return fail(SSM_ERR_UNSUPPORTED, "ssm_debug_report: library built without SSM_DEBUG (no device checks)");
+#else
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_status(e, "ssm_debug_report: synchronize");
+  out->failures = 0;
+  out->site = 0;
+  out->offset = out->count = out->extent = 0;
+  ssm::DebugRecord r;
+#define SSM_DEBUG_READ(name)                                                      \
+  e = ssm::debug_take_##name(&r, reset != 0);                                     \
+  if (e != cudaSuccess) return cuda_status(e, "ssm_debug_report: record of " #name); \
+  if (r.failures) {                                                               \
+    if (!out->failures) {                                                         \
+      out->site = r.site;                                                         \
+      out->offset = r.offset;                                                     \
+      out->count = r.count;                                                       \
+      out->extent = r.extent;                                                     \
+    }                                                                             \
+    out->failures += r.failures;                                                  \
+  }
+  SSM_DEBUG_UNITS(SSM_DEBUG_READ)
+#undef SSM_DEBUG_READ
+  snprintf(out->site_name, sizeof(out->site_name), "%s", ssm::debug_site_name(out->site));
+  return ok();
+#endif
+}
+
+ssm_status_t ssm_debug_selftest(float* buf, size_t n, ssm_stream_t stream) {
+#ifndef SSM_DEBUG
+  (void)buf;
+  (void)n;
+  (void)stream;
+  return fail(SSM_ERR_UNSUPPORTED, "ssm_debug_selftest: library built without SSM_DEBUG");
+#else
+  if (!buf || n < 1) return fail(SSM_ERR_INVALID_ARG, "ssm_debug_selftest: buf NULL or n < 1");
+  return cuda_status(ssm::launch_debug_selftest(buf, (long long)n, reinterpret_cast<cudaStream_t>(stream)),
+                     "ssm_debug_selftest launch");
+#endif
+}
+
+}  // extern "C"

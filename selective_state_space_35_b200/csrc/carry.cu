@@ -83,4 +83,6 @@ cudaError_t launch_state_carry(const float* decay, const float* value, int R, in
   return cudaGetLastError();
 }
 
+SSM_DEBUG_TU(carry)
+
 }  // namespace ssm

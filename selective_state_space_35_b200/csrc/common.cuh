@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "debug.cuh"
+
 namespace ssm {
 
 constexpr unsigned kFull = 0xffffffffu;
@@ -143,7 +145,7 @@ template <typename T, bool VEC>
 __device__ __forceinline__ void load_row8(const T* row, int t, int L, float v[8]) {
   if (VEC) {
     if (t < L) {
-      Io<T>::ld8(row + t, v);
+      Io<T>::ld8(row + SSM_DIDX(kDbgRowVec, t, 8, L), v);
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[i] = 0.0f;
@@ -157,7 +159,7 @@ __device__ __forceinline__ void load_row8(const T* row, int t, int L, float v[8]
 template <typename T, bool VEC>
 __device__ __forceinline__ void store_row8(T* row, int t, int L, const float v[8]) {
   if (VEC) {
-    if (t < L) Io<T>::st8(row + t, v);
+    if (t < L) Io<T>::st8(row + SSM_DIDX(kDbgRowVec, t, 8, L), v);
   } else {
 #pragma unroll
     for (int i = 0; i < 8; ++i)

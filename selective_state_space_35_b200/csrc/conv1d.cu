@@ -28,7 +28,7 @@ conv1d_fwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
   const int d = blockIdx.y, b = blockIdx.z;
   const int t0 = (blockIdx.x * kConvThreads + threadIdx.x) * kT;
   if (t0 >= L) return;
-  const size_t row = ((size_t)b * D + d) * L;
+  const size_t row = SSM_DIDX(kDbgConvRow, (size_t)b * D + d, 1, (size_t)gridDim.z * D) * L;
   const T* xr = x + row;
   float wk[4];
 #pragma unroll
@@ -42,7 +42,7 @@ conv1d_fwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
 #pragma unroll
   for (int i = 0; i < 3; ++i) {
     const int s = t0 - 3 + i;
-    xv[i] = s >= 0 ? Io<T>::ld(xr + s) : (xp ? Io<T>::ld(xp + 3 + s) : 0.0f);
+    xv[i] = s >= 0 ? Io<T>::ld(xr + SSM_DIDX(kDbgConvTok, s, 1, L)) : (xp ? Io<T>::ld(xp + 3 + s) : 0.0f);
   }
 #pragma unroll
   for (int k = 0; k < kT / 8; ++k) load_row8<T, VEC>(xr, t0 + 8 * k, L, xv + 3 + 8 * k);
@@ -99,7 +99,7 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
   const int d = blockIdx.y, b = blockIdx.z;
   const int t0 = (blockIdx.x * kConvThreads + threadIdx.x) * kT;
   const bool live = t0 < L;
-  const size_t row = ((size_t)b * D + d) * L;
+  const size_t row = SSM_DIDX(kDbgConvRow, (size_t)b * D + d, live ? 1 : 0, (size_t)gridDim.z * D) * L;
   const T* xr = x + row;
   const T* dur = du + row;
   float wk[4];
@@ -121,7 +121,7 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
 #pragma unroll
     for (int i = 0; i < 3; ++i) {
       const int s = t0 - 3 + i;
-      if (s >= 0) xv[i] = Io<T>::ld(xr + s);
+      if (s >= 0) xv[i] = Io<T>::ld(xr + SSM_DIDX(kDbgConvTok, s, 1, L));
       else if (HALO && x_prev) xv[i] = Io<T>::ld(x_prev + hrow + 3 + s);
     }
 #pragma unroll
@@ -228,19 +228,26 @@ conv1d_bwd_kernel(const T* __restrict__ x, const float* __restrict__ w,
     float s = 0.0f;
 #pragma unroll
     for (int wi = 0; wi < kConvThreads / 32; ++wi) s += red[wi][threadIdx.x];
-    partial[(((size_t)b * gridDim.x + blockIdx.x) * D + d) * 5 + threadIdx.x] = s;
+    // the workspace holds conv_tiles(L) tiles per batch entry (1024-token
+    // tiles); this launch's tiles are at least as long
+    partial[SSM_DIDX(kDbgConvPartial, (((size_t)b * gridDim.x + blockIdx.x) * D + d) * 5 + threadIdx.x,
+                     1, (size_t)gridDim.z * conv_tiles(L) * D * 5)] = s;
   }
 }
 
 // dw[d][k] = sum over (b, tile) of partial[b][tile][d][k], fixed order.
+// ws_tiles: tiles per batch entry the partials buffer was sized for.
 __global__ void conv1d_wreduce_kernel(const float* __restrict__ partial, float* __restrict__ dw,
-                                      float* __restrict__ dbias, int B, int tiles, int D) {
+                                      float* __restrict__ dbias, int B, int tiles, int D,
+                                      int ws_tiles) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= D * 5) return;
   const int d = i / 5, k = i % 5;
   float s = 0.0f;
   for (int b = 0; b < B; ++b)
-    for (int t = 0; t < tiles; ++t) s += partial[(((size_t)b * tiles + t) * D + d) * 5 + k];
+    for (int t = 0; t < tiles; ++t)
+      s += partial[SSM_DIDX(kDbgConvReduce, (((size_t)b * tiles + t) * D + d) * 5 + k, 1,
+                            (size_t)B * ws_tiles * D * 5)];
   if (k < 4) dw[d * 4 + k] = s;
   else if (dbias) dbias[d] = s;
 }
@@ -272,7 +279,7 @@ void conv_bwd_h(const ConvArgs& a, cudaStream_t s) {
       a.silu);
   const int n = a.D * 5;
   conv1d_wreduce_kernel<<<(n + 255) / 256, 256, 0, s>>>(a.partial, a.dw, a.dbias, a.B,
-                                                        tiles, a.D);
+                                                        tiles, a.D, conv_tiles(a.L));
 }
 
 template <typename T, bool VEC, bool SEQ>
@@ -306,6 +313,8 @@ cudaError_t launch_conv1d_bwd(const ConvArgs& a, cudaStream_t s) {
   }
   return cudaGetLastError();
 }
+
+SSM_DEBUG_TU(conv1d)
 
 }  // namespace ssm
 

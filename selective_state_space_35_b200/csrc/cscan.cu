@@ -231,7 +231,7 @@ cscan_fwd_kernel(const ScanArgs p) {
   const int N = p.N, L = p.L;
   const bool nval = active && n < N;
   const size_t rowid = (size_t)b * p.D + (active ? d : 0);
-  const size_t row = rowid * L;
+  const size_t row = SSM_DIDX(kDbgCscanRow, rowid, active ? 1 : 0, (size_t)p.B * p.D) * L;
   const size_t nslot = (size_t)p.nchunks * (kChunk / kCB);  // checkpoint slots per row
   const bool has_z = p.z != nullptr;
 
@@ -298,7 +298,10 @@ cscan_fwd_kernel(const ScanArgs p) {
   const float4* Bi4 = reinterpret_cast<const float4*>(&sm.BC[1][n][0]);
   const float4* Cr4 = reinterpret_cast<const float4*>(&sm.BC[2][n][0]);
   const float4* Ci4 = reinterpret_cast<const float4*>(&sm.BC[3][n][0]);
-  float2* ck = reinterpret_cast<float2*>(p.ckpt) + rowid * nslot * kNMax + n;
+  // a row's slots: [nslot][kNMax] (re, im) pairs
+  float2* ck = reinterpret_cast<float2*>(p.ckpt) +
+               SSM_DIDX(kDbgCscanCkpt, rowid * nslot * kNMax + n, nval ? (nslot - 1) * kNMax + 1 : 0,
+                        (size_t)p.B * p.D * nslot * kNMax);
 
 #pragma unroll 1
   for (int kb = 0; kb < nb; ++kb) {
@@ -378,7 +381,7 @@ cscan_bwd_kernel(const ScanArgs p) {
   const int N = p.N, L = p.L;
   const bool nval = active && n < N;
   const size_t rowid = (size_t)b * p.D + (active ? d : 0);
-  const size_t row = rowid * L;
+  const size_t row = SSM_DIDX(kDbgCscanRow, rowid, active ? 1 : 0, (size_t)p.B * p.D) * L;
   const size_t nslot = (size_t)p.nchunks * (kChunk / kCB);
   const bool has_z = p.z != nullptr;
 
@@ -396,7 +399,9 @@ cscan_bwd_kernel(const ScanArgs p) {
   const float Ar2 = An.x * kLog2e, Ai = An.y;
   const float Dv = (active && p.Dskip) ? __ldg(p.Dskip + d) : 0.0f;
   const float bias = (active && p.delta_bias) ? __ldg(p.delta_bias + d) : 0.0f;
-  const float2* ckp = reinterpret_cast<const float2*>(p.ckpt) + rowid * nslot * kNMax + n;
+  const float2* ckp = reinterpret_cast<const float2*>(p.ckpt) +
+                      SSM_DIDX(kDbgCscanCkpt, rowid * nslot * kNMax + n,
+                               nval ? (nslot - 1) * kNMax + 1 : 0, (size_t)p.B * p.D * nslot * kNMax);
 
   float nx_dl = 0.0f, nx_u = 0.0f, nx_go = 0.0f, nx_z = 0.0f, nx_y = 0.0f;
   int nx_sq = 0, nx_sqp = 0;
@@ -698,5 +703,7 @@ cudaError_t launch_cscan_bwd(const ScanArgs& a, cudaStream_t s) {
   if (a.bf16) return a.vec ? cbwd_t<__nv_bfloat16, true>(a, s) : cbwd_t<__nv_bfloat16, false>(a, s);
   return a.vec ? cbwd_t<float, true>(a, s) : cbwd_t<float, false>(a, s);
 }
+
+SSM_DEBUG_TU(cscan)
 
 }  // namespace ssm

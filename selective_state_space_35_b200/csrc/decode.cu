@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(kDecThreads, sizeof(T) == 2 ? 8 : 6) decode_st
   for (int j = 0; j < kPerThr / 4; ++j) {  // groups of 4 states
     const int n0 = kPerThr * q + 4 * j;
     if (n0 < N) {
-      float* hp = a.state + g * N + n0;
+      float* hp = a.state + SSM_DIDX(kDbgDecodeState, g * N + n0, VEC ? 4 : 1, rows * N);
       const float* Ap = a.A + (size_t)d * N + n0;
       const float4 Bv = ld4<T, VEC>(static_cast<const T*>(a.Bm) + (size_t)b * N, n0, N);
       const float4 Cv = ld4<T, VEC>(static_cast<const T*>(a.Cm) + (size_t)b * N, n0, N);
@@ -149,5 +149,7 @@ cudaError_t launch_decode_step(const DecodeArgs& a, cudaStream_t s) {
   }
   return cudaGetLastError();
 }
+
+SSM_DEBUG_TU(decode)
 
 }  // namespace ssm

@@ -60,7 +60,7 @@ constexpr size_t kConvBwdScratchFloats = size_t(1) << 20;  // 4 MiB per device
 constexpr int kMaxScratchDevices = 64;
 cudaError_t conv_bwd_scratch(float** ptr);
 cudaError_t launch_conv1d_bwd(const ConvArgs& a, cudaStream_t s);
-inline int conv_tiles(int L) { return (L + kConvTile - 1) / kConvTile; }
+__host__ __device__ inline int conv_tiles(int L) { return (L + kConvTile - 1) / kConvTile; }
 // The backward without document ids: kConvBwdTok tokens per thread (with
 // them 8, as the forward); its dw / dbias partials are per (b, tile, d), at
 // most conv_tiles(L) tiles, which sizes its scratch.
@@ -211,5 +211,22 @@ cudaError_t launch_ssd_fwd(const SsdArgs& a, cudaStream_t s);
 cudaError_t launch_ssd_bwd(const SsdArgs& a, cudaStream_t s);
 cudaError_t launch_cu_seqlens_to_seq(const int32_t* cu, int n_docs, int L, int32_t* seq,
                                      cudaStream_t s);
+
+// First failed device index check of one translation unit (debug.cuh):
+// failures counts every failed check since the last reset.
+struct DebugRecord {
+  unsigned long long failures;
+  long long offset, count, extent;
+  int site, pad;
+};
+#ifdef SSM_DEBUG
+// The kernel sources that carry checks, each reading its own record.
+#define SSM_DEBUG_UNITS(X) \
+  X(conv1d) X(scan16_fwd) X(scan16_bwd) X(scan_fwd) X(scan_bwd) X(cscan) X(decode) X(ssd_fwd) X(ssd_bwd) X(carry) X(probe) X(abi)
+#define SSM_DEBUG_DECL(name) cudaError_t debug_take_##name(DebugRecord* out, bool reset);
+SSM_DEBUG_UNITS(SSM_DEBUG_DECL)
+#undef SSM_DEBUG_DECL
+cudaError_t launch_debug_selftest(float* buf, long long n, cudaStream_t s);
+#endif
 
 }  // namespace ssm

@@ -59,4 +59,6 @@ cudaError_t probe_ex2_rate(float* sink, size_t sink_floats, double* rate, cudaSt
   return cudaGetLastError();
 }
 
+SSM_DEBUG_TU(probe)
+
 }  // namespace ssm

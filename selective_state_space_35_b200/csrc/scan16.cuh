@@ -32,6 +32,11 @@ constexpr int kSegs = kCh / kSeg;
 __host__ __device__ __forceinline__ size_t ck_chunk(int b, int rp, int Dp, int nch, int c) {
   return ((((size_t)b * Dp + rp) * nch + c) * kN) * (2 * kSegs);
 }
+// Floats of the checkpoint array of a call from `at` to its end (the extent
+// the debug build's index checks hold checkpoint accesses to).
+__device__ __forceinline__ long long ck_left(const ScanArgs& p, const float* at) {
+  return (long long)ck_chunk(p.B, 0, p.Dp, p.nchunks, 0) - (long long)(at - p.ckpt);
+}
 
 // Forward B / C tiles, packed by pack_bc_fwd_kernel into [B][nchunks][mat][kN][64] float4:
 // float4 (k * 16 + jj) of a (mat, state) row holds tokens 16jj+2k, 16jj+8+2k,

@@ -121,7 +121,8 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_kernel(const
   const int L = p.L, nch = p.nchunks;
   const size_t rid0 = (size_t)b * p.D + (act0 ? d0 : 0);
   const size_t rid1 = (size_t)b * p.D + (act1 ? d0 + 1 : 0);
-  const size_t row0 = rid0 * L, row1 = rid1 * L;
+  const size_t row0 = SSM_DIDX(kDbgS16Row, rid0, act0 ? 1 : 0, (size_t)p.B * p.D) * L;
+  const size_t row1 = SSM_DIDX(kDbgS16Row, rid1, act1 ? 1 : 0, (size_t)p.B * p.D) * L;
   const T* Bm = static_cast<const T*>(p.Bm);
   const T* Cm = static_cast<const T*>(p.Cm);
   const bool has_z = p.z != nullptr;
@@ -183,6 +184,9 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_kernel(const
     const int tl = c * kCh + 8 * lane;
     const bool valid = tl < L;
     const bool ok0 = valid && act0, ok1 = valid && act1;
+    // the lane's 8 tokens of each row (L is a multiple of 8 on this path)
+    const int t0o = SSM_DIDX(kDbgS16Tok, tl, ok0 ? 8 : 0, L);
+    const int t1o = SSM_DIDX(kDbgS16Tok, tl, ok1 ? 8 : 0, L);
     const float* ckc = p.ckpt + ck_chunk(b, rp, p.Dp, nch, c) + lane;
     if (c >= 1) {  // the next chunk's lines into L2
       const int tn = tl - kCh;
@@ -204,19 +208,19 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_kernel(const
     float2 dd[8], xx[8], dy[8];
     {
       float dl0[8], dl1[8], u0[8], u1[8], g0[8], g1[8];
-      ld8<T, true>(static_cast<const T*>(p.delta) + row0 + tl, ok0, dl0);
-      ld8<T, true>(static_cast<const T*>(p.delta) + row1 + tl, ok1, dl1);
-      ld8<T, true>(static_cast<const T*>(p.u) + row0 + tl, ok0, u0);
-      ld8<T, true>(static_cast<const T*>(p.u) + row1 + tl, ok1, u1);
-      ld8<T, VG>(static_cast<const T*>(p.dout) + row0 + tl, ok0, g0);
-      ld8<T, VG>(static_cast<const T*>(p.dout) + row1 + tl, ok1, g1);
+      ld8<T, true>(static_cast<const T*>(p.delta) + row0 + t0o, ok0, dl0);
+      ld8<T, true>(static_cast<const T*>(p.delta) + row1 + t1o, ok1, dl1);
+      ld8<T, true>(static_cast<const T*>(p.u) + row0 + t0o, ok0, u0);
+      ld8<T, true>(static_cast<const T*>(p.u) + row1 + t1o, ok1, u1);
+      ld8<T, VG>(static_cast<const T*>(p.dout) + row0 + t0o, ok0, g0);
+      ld8<T, VG>(static_cast<const T*>(p.dout) + row1 + t1o, ok1, g1);
       float dz0[8], dz1[8];
       if (has_z) {
         float z0[8], z1[8], y0[8], y1[8];
-        ld8<T, true>(static_cast<const T*>(p.z) + row0 + tl, ok0, z0);
-        ld8<T, true>(static_cast<const T*>(p.z) + row1 + tl, ok1, z1);
-        ld8<T, true>(static_cast<const T*>(p.ysave) + row0 + tl, ok0, y0);
-        ld8<T, true>(static_cast<const T*>(p.ysave) + row1 + tl, ok1, y1);
+        ld8<T, true>(static_cast<const T*>(p.z) + row0 + t0o, ok0, z0);
+        ld8<T, true>(static_cast<const T*>(p.z) + row1 + t1o, ok1, z1);
+        ld8<T, true>(static_cast<const T*>(p.ysave) + row0 + t0o, ok0, y0);
+        ld8<T, true>(static_cast<const T*>(p.ysave) + row1 + t1o, ok1, y1);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const float s0 = sigmoid_fast(z0[i]), s1 = sigmoid_fast(z1[i]);
@@ -225,8 +229,8 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_kernel(const
           g0[i] *= z0[i] * s0;
           g1[i] *= z1[i] * s1;
         }
-        if (ok0) st8<T, VG>(static_cast<T*>(p.dz) + row0 + tl, dz0);
-        if (ok1) st8<T, VG>(static_cast<T*>(p.dz) + row1 + tl, dz1);
+        if (ok0) st8<T, VG>(static_cast<T*>(p.dz) + row0 + t0o, dz0);
+        if (ok1) st8<T, VG>(static_cast<T*>(p.dz) + row1 + t1o, dz1);
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -266,14 +270,17 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_kernel(const
 
     const T* tileB = &sm.tile[buf][0][0][0];
     const T* tileC = &sm.tile[buf][1][0][0];
-    float2 hck = make_float2(ok0 ? __ldg(ckc) : 0.0f, ok1 ? __ldg(ckc + kSegs) : 0.0f);
+    float2 hck = make_float2(ok0 ? __ldg(ckc + SSM_DIDX(kDbgS16Ckpt, 0, 1, ck_left(p, ckc))) : 0.0f,
+                             ok1 ? __ldg(ckc + SSM_DIDX(kDbgS16Ckpt, kSegs, 1, ck_left(p, ckc))) : 0.0f);
     auto states = [&](auto RS) {
 #pragma unroll 1
     for (int n = 0; n < kN; ++n) {
       const float2 hin = hck;
       if (n + 1 < kN)  // next state's checkpoint, one state ahead
-        hck = make_float2(ok0 ? __ldg(ckc + (n + 1) * 2 * kSegs) : 0.0f,
-                          ok1 ? __ldg(ckc + (n + 1) * 2 * kSegs + kSegs) : 0.0f);
+        hck = make_float2(
+            ok0 ? __ldg(ckc + SSM_DIDX(kDbgS16Ckpt, (n + 1) * 2 * kSegs, 1, ck_left(p, ckc))) : 0.0f,
+            ok1 ? __ldg(ckc + SSM_DIDX(kDbgS16Ckpt, (n + 1) * 2 * kSegs + kSegs, 1, ck_left(p, ckc)))
+                : 0.0f);
       const float4 Aq = sm.A[warp][n];
       const float2 a2 = make_float2(Aq.x, Aq.y), ap2 = make_float2(Aq.z, Aq.w);
       float Bt[8], Ct[8];
@@ -359,13 +366,19 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_kernel(const
         }
         const int t = c * kCh + 8 * (f & 31) + 4 * (f >> 5);
         if (t < L && p.dbc_part) {  // deterministic: this CTA's sum, added later in order
-          float* dst = p.dbc_part + ((size_t)blockIdx.x * 2 + mat) * p.dbc_bnl + ((size_t)b * kN + n) * L + t;
+          float* dst = p.dbc_part + SSM_DIDX(kDbgS16Part,
+                                             ((size_t)blockIdx.x * 2 + mat) * p.dbc_bnl +
+                                                 ((size_t)b * kN + n) * L + t,
+                                             4,
+                                             (size_t)((p.D + kBwdCtaRows16 - 1) / kBwdCtaRows16) * 2 *
+                                                 p.dbc_bnl);
           dst[0] = s.x;
           dst[1] = s.y;
           dst[2] = s.z;
           dst[3] = s.w;
         } else if (t < L) {
-          float* dst = (mat ? p.dC : p.dB) + ((size_t)b * kN + n) * L + t;
+          float* dst = (mat ? p.dC : p.dB) +
+                       SSM_DIDX(kDbgS16BC, ((size_t)b * kN + n) * L + t, 4, (size_t)p.B * kN * L);
           if (VG) {
             asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(s.x),
                          "f"(s.y), "f"(s.z), "f"(s.w)
@@ -398,12 +411,12 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_kernel(const
         if (valid) ddbp = fadd2(ddbp, ddr);
       }
       if (ok0) {
-        st8<T, VG>(static_cast<T*>(p.du) + row0 + tl, du0);
-        st8<T, VG>(static_cast<T*>(p.ddelta) + row0 + tl, dd0);
+        st8<T, VG>(static_cast<T*>(p.du) + row0 + t0o, du0);
+        st8<T, VG>(static_cast<T*>(p.ddelta) + row0 + t0o, dd0);
       }
       if (ok1) {
-        st8<T, VG>(static_cast<T*>(p.du) + row1 + tl, du1);
-        st8<T, VG>(static_cast<T*>(p.ddelta) + row1 + tl, dd1);
+        st8<T, VG>(static_cast<T*>(p.du) + row1 + t1o, du1);
+        st8<T, VG>(static_cast<T*>(p.ddelta) + row1 + t1o, dd1);
       }
     }
   }
@@ -425,8 +438,8 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_kernel(const
       const float2 v = sm.dA[warp][n][j];
       s += rr ? v.y : v.x;
     }
-    if (rr == 0 && act0) p.part_dA[rid0 * kN + n] = s;
-    if (rr == 1 && act1) p.part_dA[rid1 * kN + n] = s;
+    if (rr == 0 && act0) p.part_dA[SSM_DIDX(kDbgS16Param, rid0 * kN + n, 1, (size_t)p.B * p.D * kN)] = s;
+    if (rr == 1 && act1) p.part_dA[SSM_DIDX(kDbgS16Param, rid1 * kN + n, 1, (size_t)p.B * p.D * kN)] = s;
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
@@ -473,7 +486,8 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_summary_kern
   const int L = p.L, nch = p.nchunks;
   const size_t rid0 = (size_t)b * p.D + (act0 ? d0 : 0);
   const size_t rid1 = (size_t)b * p.D + (act1 ? d0 + 1 : 0);
-  const size_t row0 = rid0 * L, row1 = rid1 * L;
+  const size_t row0 = SSM_DIDX(kDbgS16Row, rid0, act0 ? 1 : 0, (size_t)p.B * p.D) * L;
+  const size_t row1 = SSM_DIDX(kDbgS16Row, rid1, act1 ? 1 : 0, (size_t)p.B * p.D) * L;
   const T* Cm = static_cast<const T*>(p.Cm);
   const bool has_z = p.z != nullptr;
   const int32_t* seqb = p.seq ? p.seq + (size_t)b * L : nullptr;
@@ -530,17 +544,20 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 2 : 1) scan16_bwd_summary_kern
     const int tl = c * kCh + 8 * lane;
     const bool valid = tl < L;
     const bool ok0 = valid && act0, ok1 = valid && act1;
+    // the lane's 8 tokens of each row (L is a multiple of 8 on this path)
+    const int t0o = SSM_DIDX(kDbgS16Tok, tl, ok0 ? 8 : 0, L);
+    const int t1o = SSM_DIDX(kDbgS16Tok, tl, ok1 ? 8 : 0, L);
     float2 dd[8], dy[8];
     {
       float dl0[8], dl1[8], g0[8], g1[8];
-      ld8<T, true>(static_cast<const T*>(p.delta) + row0 + tl, ok0, dl0);
-      ld8<T, true>(static_cast<const T*>(p.delta) + row1 + tl, ok1, dl1);
-      ld8<T, true>(static_cast<const T*>(p.dout) + row0 + tl, ok0, g0);
-      ld8<T, true>(static_cast<const T*>(p.dout) + row1 + tl, ok1, g1);
+      ld8<T, true>(static_cast<const T*>(p.delta) + row0 + t0o, ok0, dl0);
+      ld8<T, true>(static_cast<const T*>(p.delta) + row1 + t1o, ok1, dl1);
+      ld8<T, true>(static_cast<const T*>(p.dout) + row0 + t0o, ok0, g0);
+      ld8<T, true>(static_cast<const T*>(p.dout) + row1 + t1o, ok1, g1);
       if (has_z) {
         float z0[8], z1[8];
-        ld8<T, true>(static_cast<const T*>(p.z) + row0 + tl, ok0, z0);
-        ld8<T, true>(static_cast<const T*>(p.z) + row1 + tl, ok1, z1);
+        ld8<T, true>(static_cast<const T*>(p.z) + row0 + t0o, ok0, z0);
+        ld8<T, true>(static_cast<const T*>(p.z) + row1 + t1o, ok1, z1);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           g0[i] *= z0[i] * sigmoid_fast(z0[i]);
@@ -690,5 +707,7 @@ cudaError_t launch_scan16_bwd(const ScanArgs& a, cudaStream_t s) {
   return scan16_bwd_rows(a) == 2 * kBwdWarpsBig ? bwd16_dispatch<kBwdWarpsBig>(a, s)
                                                 : bwd16_dispatch<kBwdWarpsSmall>(a, s);
 }
+
+SSM_DEBUG_TU(scan16_bwd)
 
 }  // namespace ssm

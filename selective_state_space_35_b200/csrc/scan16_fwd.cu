@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
   const bool active = d < p.D;
   const int L = p.L, nch = p.nchunks;
   const size_t rowid = (size_t)b * p.D + (active ? d : 0);
-  const size_t row = rowid * L;
+  const size_t row = SSM_DIDX(kDbgS16Row, rowid, active ? 1 : 0, (size_t)p.B * p.D) * L;
   const T* u_in = static_cast<const T*>(CONV ? p.xconv : p.u) + row;
   const T* dl_in = static_cast<const T*>(p.delta) + row;
   const T* z_in = (p.z && !SUM) ? static_cast<const T*>(p.z) + row : nullptr;
@@ -153,11 +153,17 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
     if (threadIdx.x == 0 && c + 1 < nch) {
       fence_proxy_async_smem();
       mbar_expect_tx(&sm.bar[buf ^ 1], kTileBytes);
-      tma_load_1d(&sm.tile[buf ^ 1][0], pk + (size_t)(c + 1) * kFwdTileF4, kTileBytes,
+      tma_load_1d(&sm.tile[buf ^ 1][0],
+                  pk + SSM_DIDX(kDbgPackBC, (size_t)(c + 1) * kFwdTileF4, kFwdTileF4,
+                                (size_t)nch * kFwdTileF4),
+                  kTileBytes,
                   &sm.bar[buf ^ 1]);
     }
     const int tl = c * kCh + 16 * jj;
     const bool va = active && tl < L, vb = active && tl + 8 < L;
+    // the lane's two 8-token pieces (L is a multiple of 8 on this path)
+    const int ta = SSM_DIDX(kDbgS16Tok, tl, va ? 8 : 0, L);
+    const int tb = SSM_DIDX(kDbgS16Tok, tl + 8, vb ? 8 : 0, L);
     if (c + 1 < nch && (jj & 3) == 0 && active) {  // the next chunk's lines into L2
       const int tn = tl + kCh;
       if (tn < L) {
@@ -169,10 +175,10 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
 
     // per-token values: (sub-segment a, sub-segment b) pairs
     float ua[8], ub[8], da[8], db[8];
-    load8<T, (!CONV || XVEC)>(u_in + tl, va, ua);
-    load8<T, (!CONV || XVEC)>(u_in + tl + 8, vb, ub);
-    load8<T, true>(dl_in + tl, va, da);
-    load8<T, true>(dl_in + tl + 8, vb, db);
+    load8<T, (!CONV || XVEC)>(u_in + ta, va, ua);
+    load8<T, (!CONV || XVEC)>(u_in + tb, vb, ub);
+    load8<T, true>(dl_in + ta, va, da);
+    load8<T, true>(dl_in + tb, vb, db);
     // document starts among tokens tl .. tl+15 (bit i), ids tl-3 .. tl+15
     unsigned rm = 0u;
     int sg[19];
@@ -223,8 +229,8 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
         ua[i] = uo[i];
         ub[i] = uo[8 + i];
       }
-      if (va) store8<T>(u_out + tl, ua);
-      if (vb) store8<T>(u_out + tl + 8, ub);
+      if (va) store8<T>(u_out + ta, ua);
+      if (vb) store8<T>(u_out + tb, ub);
     }
     const bool any_reset = __any_sync(kFull, rm != 0u);
     if constexpr (SUM) any_start = any_start || any_reset;
@@ -299,7 +305,9 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
         if (jj == 15) sm.H[r][n] = end;
         if constexpr (SUM) continue;
         const float sb = fmaf(P[s].x, start, H[s].x);  // state entering sub-segment b
-        if (va) *reinterpret_cast<float2*>(ckc + n * 2 * kSegs) = make_float2(start, sb);
+        if (va)
+          *reinterpret_cast<float2*>(
+              ckc + SSM_DIDX(kDbgS16Ckpt, n * 2 * kSegs, 2, ck_left(p, ckc))) = make_float2(start, sb);
         h[s] = make_float2(start, sb);
       }
       if constexpr (!SUM) {
@@ -338,24 +346,24 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
       }
       if (z_in) {
         float za[8], zb[8];
-        load8<T, true>(z_in + tl, va, za);
-        load8<T, true>(z_in + tl + 8, vb, zb);
+        load8<T, true>(z_in + ta, va, za);
+        load8<T, true>(z_in + tb, vb, zb);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           oa[i] = ya[i] * (za[i] * sigmoid_fast(za[i]));
           ob[i] = yb[i] * (zb[i] * sigmoid_fast(zb[i]));
         }
         if (va) {
-          put(out + tl, oa);
-          store8<T>(ysv + tl, ya);
+          put(out + ta, oa);
+          store8<T>(ysv + ta, ya);
         }
         if (vb) {
-          put(out + tl + 8, ob);
-          store8<T>(ysv + tl + 8, yb);
+          put(out + tb, ob);
+          store8<T>(ysv + tb, yb);
         }
       } else {
-        if (va) put(out + tl, ya);
-        if (vb) put(out + tl + 8, yb);
+        if (va) put(out + ta, ya);
+        if (vb) put(out + tb, yb);
       }
     }
   }
@@ -366,11 +374,12 @@ __global__ void __launch_bounds__(W * 32, W < 8 ? 3 : 1) scan16_fwd_kernel(const
 #pragma unroll
     for (int off = 8; off > 0; off >>= 1) dt_sum += __shfl_xor_sync(kFull, dt_sum, off, 16);
     if (active) {
-      p.split_P[rowid * p.Npad + jj] = any_start ? 0.0f : ex2_approx(sm.A[r][jj].x * dt_sum);
-      p.split_H[rowid * p.Npad + jj] = sm.H[r][jj];
+      p.split_P[SSM_DIDX(kDbgS16State, rowid * p.Npad + jj, 1, (size_t)p.B * p.D * p.Npad)] =
+          any_start ? 0.0f : ex2_approx(sm.A[r][jj].x * dt_sum);
+      p.split_H[SSM_DIDX(kDbgS16State, rowid * p.Npad + jj, 1, (size_t)p.B * p.D * p.Npad)] = sm.H[r][jj];
     }
   } else if (active && p.final_state) {
-    p.final_state[rowid * kN + jj] = sm.H[r][jj];
+    p.final_state[SSM_DIDX(kDbgS16State, rowid * kN + jj, 1, (size_t)p.B * p.D * kN)] = sm.H[r][jj];
   }
 }
 
@@ -417,5 +426,7 @@ cudaError_t launch_scan16_fwd_summary(const ScanArgs& a, cudaStream_t s) {
   return big ? fwd16_t<float, false, true, kFwdWarpsBig, true>(a, s)
              : fwd16_t<float, false, true, kFwdWarpsSmall, true>(a, s);
 }
+
+SSM_DEBUG_TU(scan16_fwd)
 
 }  // namespace ssm

@@ -195,7 +195,7 @@ scan_bwd_kernel(const ScanArgs p) {
   const int t_begin = split * p.chunks_per_split * kChunk;
   const int t_end = min((split + 1) * p.chunks_per_split * kChunk, L);
   const size_t rowid = (size_t)b * p.D + (active ? d : 0);
-  const size_t row = rowid * L;
+  const size_t row = SSM_DIDX(kDbgScanRow, rowid, active ? 1 : 0, (size_t)p.B * p.D) * L;
   // the forward keeps the state entering every 16-token block; this kernel
   // starts from every other one
   constexpr int kCk = 16;
@@ -234,7 +234,9 @@ scan_bwd_kernel(const ScanArgs p) {
   auto prefetch = [&](int kb) {
     const int tb = t_begin + kb * kBlk;
     issue_block<T, VEC>(sm, Bm, Cm, rp, n_arrays, b, N, L, tb, r, n, active);
-    if (nval) ck_issued = __ldg(p.ckpt + (rowid * nblk + tb / kCk) * kNMax + n);
+    if (nval)
+      ck_issued = __ldg(p.ckpt + SSM_DIDX(kDbgScanCkpt, (rowid * nblk + tb / kCk) * kNMax + n, 1,
+                                          (size_t)p.B * p.D * nblk * kNMax));
     if (seqb) {
       const int t = tb + lane;
       sq_cur = t < L ? __ldg(seqb + t) : 0;
@@ -559,7 +561,7 @@ scan_bwd_summary_kernel(const ScanArgs p) {
   const int c_begin = split * p.chunks_per_split;
   const int c_end = min(c_begin + p.chunks_per_split, p.nchunks);
   const size_t rowid = (size_t)b * p.D + (active ? d : 0);
-  const size_t row = rowid * L;
+  const size_t row = SSM_DIDX(kDbgScanRow, rowid, active ? 1 : 0, (size_t)p.B * p.D) * L;
   const T* dl_row = static_cast<const T*>(p.delta) + row;
   const T* z_row = p.z ? static_cast<const T*>(p.z) + row : nullptr;
   const T* go_row = static_cast<const T*>(p.dout) + row;
@@ -741,5 +743,7 @@ cudaError_t launch_scan_bwd_summary(const ScanArgs& a, cudaStream_t s) {
   }
   return cudaGetLastError();
 }
+
+SSM_DEBUG_TU(scan_bwd)
 
 }  // namespace ssm

@@ -172,7 +172,7 @@ scan_fwd_kernel(const ScanArgs p) {
   const int c_begin = split * p.chunks_per_split;
   const int c_end = min(c_begin + p.chunks_per_split, p.nchunks);
   const size_t rowid = (size_t)b * p.D + (active ? d : 0);
-  const size_t row = rowid * L;
+  const size_t row = SSM_DIDX(kDbgScanRow, rowid, active ? 1 : 0, (size_t)p.B * p.D) * L;
 
   const T* Bm = static_cast<const T*>(p.Bm);
   const T* Cm = static_cast<const T*>(p.Cm);
@@ -282,7 +282,10 @@ scan_fwd_kernel(const ScanArgs p) {
     const bool any_reset = __any_sync(kFull, rmask != 0u);
 
     // 16-token checkpoints of this chunk: [row][c * 16 + k][kNMax] fp32 pairs
-    float2* ck16 = reinterpret_cast<float2*>(p.ckpt) + (rowid * p.nchunks + c) * 16 * (kNMax / 2);
+    float2* ck16 = reinterpret_cast<float2*>(p.ckpt) +
+                   SSM_DIDX(kDbgScanCkpt, (rowid * p.nchunks + c) * 16 * (kNMax / 2),
+                            active ? 16 * (kNMax / 2) : 0,
+                            (size_t)p.B * p.D * p.nchunks * 16 * (kNMax / 2));
 
     if (NT) {
       // compile-time state count: fully unrolled and software-pipelined (the
@@ -439,5 +442,7 @@ cudaError_t launch_cu_seqlens_to_seq(const int32_t* cu, int n_docs, int L, int32
   cu_seqlens_to_seq_kernel<<<(L + 255) / 256, 256, 0, s>>>(cu, n_docs, L, seq);
   return cudaGetLastError();
 }
+
+SSM_DEBUG_TU(scan_fwd)
 
 }  // namespace ssm

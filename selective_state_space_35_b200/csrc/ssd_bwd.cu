@@ -279,8 +279,11 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p, c
   for (int c = nch - 1; c >= 0; --c) {
     const int tok = c * kQ + r;
     const bool valid = tok < L;
-    const size_t xo = (((size_t)b * L + tok) * H + h) * kP + 32 * hf;  // x / dy / dx row half
-    const size_t bo = (((size_t)b * L + tok) * G + g) * kNs + 64 * hf; // B / C / dB / dC row half
+    // x / dy / dx row half; B / C / dB / dC row half (used only for valid rows)
+    const size_t xo = SSM_DIDX(kDbgSsdRow, (((size_t)b * L + tok) * H + h) * kP + 32 * hf, valid ? 32 : 0,
+                               (size_t)p.B * L * H * kP);
+    const size_t bo = SSM_DIDX(kDbgSsdRow, (((size_t)b * L + tok) * G + g) * kNs + 64 * hf, valid ? 64 : 0,
+                               (size_t)p.B * L * G * kNs);
     // ---- this chunk's rows straight into their tiles: one tensor-map copy
     // per tile for a whole chunk, else cp.async (zero-filled past L); no
     // registers held ----
@@ -318,7 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p, c
     float hdh = 0.0f;
     {
       const float4* hrow = reinterpret_cast<const float4*>(
-          p.chunk_states + ((((size_t)b * H + h) * nch + c) * kNs + r) * kP + 32 * hf);
+          p.chunk_states + SSM_DIDX(kDbgSsdChunkState, ((((size_t)b * H + h) * nch + c) * kNs + r) * kP + 32 * hf,
+                                    32, (size_t)p.B * H * nch * kNs * kP));
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const float4 a0 = __ldg(hrow + 2 * k), a1 = __ldg(hrow + 2 * k + 1);
@@ -336,7 +340,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p, c
       prefetch_l2(dyg + xp);
       prefetch_l2(p.chunk_states + ((((size_t)b * H + h) * nch + c - 1) * kNs + r) * kP + 32 * hf);
     }
-    const float dtv = valid ? __bfloat162float(dtg[((size_t)b * L + tok) * H + h]) + bias : 0.0f;
+    const float dtv = valid ? __bfloat162float(dtg[SSM_DIDX(kDbgSsdRow, ((size_t)b * L + tok) * H + h, 1,
+                                                             (size_t)p.B * L * H)]) + bias
+                            : 0.0f;
     float dt = 0.0f;
     if (valid) dt = p.softplus ? (dtv > 20.0f ? dtv : log1pf(expf(dtv))) : dtv;
     bool start = false;
@@ -530,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p, c
       dA_acc = fmaf(dt, dl, dA_acc);
       const float dv = p.softplus ? ddt * (1.0f / (1.0f + __expf(-dtv))) : ddt;
       if (valid) {
-        p.ddt_raw[((size_t)b * L + tok) * H + h] = dv;
+        p.ddt_raw[SSM_DIDX(kDbgSsdRow, ((size_t)b * L + tok) * H + h, 1, (size_t)p.B * L * H)] = dv;
         ddb_acc += dv;
       }
     }
@@ -605,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_bwd_kernel(const SsdArgs p, c
         bulk_wait_read();  // the staging is refilled by the next chunk
       }
     } else if (valid) {  // row r of dC (half 0) or dB (half 1), summed into global memory
-      const size_t ro = (((size_t)b * L + tok) * G + g) * kNs;
+      const size_t ro = SSM_DIDX(kDbgSsdRow, (((size_t)b * L + tok) * G + g) * kNs, kNs, (size_t)p.B * L * G * kNs);
       if (hf == 0) bulk_add_f32(p.dC + ro, stC, kNs * 4);
       else bulk_add_f32(p.dB + ro, stB, kNs * 4);
       bulk_wait_read();  // the staging rows are refilled by the next chunk
@@ -661,5 +667,7 @@ cudaError_t launch_ssd_bwd(const SsdArgs& a, cudaStream_t s) {
   ssd_bwd_kernel<<<dim3(a.H, a.B), kThreads, smem, s>>>(a, maps, tma);
   return cudaGetLastError();
 }
+
+SSM_DEBUG_TU(ssd_bwd)
 
 }  // namespace ssm

@@ -204,10 +204,15 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
   auto fetch = [&](int c, ChunkIn& in) {
     const int tok = c * kQ + r;
     const bool valid = tok < L;
-    const uint4* crow = reinterpret_cast<const uint4*>(Cg + (((size_t)b * L + tok) * G + g) * kNs) + 8 * hf;
+    const uint4* crow =
+        reinterpret_cast<const uint4*>(Cg + SSM_DIDX(kDbgSsdRow, (((size_t)b * L + tok) * G + g) * kNs,
+                                                     valid ? kNs : 0, (size_t)p.B * L * G * kNs)) +
+        8 * hf;
 #pragma unroll
     for (int k = 0; k < 8; ++k) in.c[k] = valid ? __ldg(crow + k) : z4;
-    in.dtv = valid ? __bfloat162float(dtg[((size_t)b * L + tok) * H + h]) + bias : 0.0f;
+    in.dtv = valid ? __bfloat162float(dtg[SSM_DIDX(kDbgSsdRow, ((size_t)b * L + tok) * H + h, 1,
+                                                    (size_t)p.B * L * H)]) + bias
+                   : 0.0f;
     in.seq_cur = (seqb && valid) ? __ldg(seqb + tok) : 0;
     in.seq_prev = (seqb && valid && tok > 0) ? __ldg(seqb + tok - 1) : in.seq_cur;
   };
@@ -225,7 +230,10 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
     } else {
       const int tk = cc * kQ + r;
       const int tc = tk < L ? tk : 0;  // an in-bounds source when zero-filling
-      const uint4* xrow = reinterpret_cast<const uint4*>(xg + (((size_t)b * L + tc) * H + h) * kP) + 4 * hf;
+      const uint4* xrow =
+          reinterpret_cast<const uint4*>(xg + SSM_DIDX(kDbgSsdRow, (((size_t)b * L + tc) * H + h) * kP,
+                                                       tk < L ? kP : 0, (size_t)p.B * L * H * kP)) +
+          4 * hf;
 #pragma unroll
       for (int k = 0; k < 4; ++k) cp_async16(xt + x_off(r, 8 * (4 * hf + k)), xrow + k, tk < L ? 16u : 0u);
       asm volatile("cp.async.commit_group;" ::: "memory");
@@ -238,7 +246,10 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
     } else {
       const int tk = cc * kQ + r;
       const int tc = tk < L ? tk : 0;
-      const uint4* brow = reinterpret_cast<const uint4*>(Bg + (((size_t)b * L + tc) * G + g) * kNs) + 8 * hf;
+      const uint4* brow =
+          reinterpret_cast<const uint4*>(Bg + SSM_DIDX(kDbgSsdRow, (((size_t)b * L + tc) * G + g) * kNs,
+                                                       tk < L ? kNs : 0, (size_t)p.B * L * G * kNs)) +
+          8 * hf;
 #pragma unroll
       for (int k = 0; k < 8; ++k) cp_async16(sm.Bm + tile_off(r, 8 * (8 * hf + k)), brow + k, tk < L ? 16u : 0u);
       asm volatile("cp.async.commit_group;" ::: "memory");
@@ -284,8 +295,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
     const int tok = c * kQ + r;
     const bool valid = tok < L;
     if (p.chunk_states) {  // the state entering this chunk, for the backward
-      float4* cs = reinterpret_cast<float4*>(p.chunk_states +
-                                             ((((size_t)b * H + h) * nch + c) * kNs + r) * kP + 32 * hf);
+      float4* cs = reinterpret_cast<float4*>(
+          p.chunk_states + SSM_DIDX(kDbgSsdChunkState, ((((size_t)b * H + h) * nch + c) * kNs + r) * kP + 32 * hf,
+                                    32, (size_t)p.B * H * nch * kNs * kP));
 #pragma unroll
       for (int q = 0; q < kP / 8; ++q) cs[q] = make_float4(Ht[4 * q], Ht[4 * q + 1], Ht[4 * q + 2], Ht[4 * q + 3]);
     }
@@ -438,7 +450,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
       tmem_ld32(lane_row + 256 + 32 * hf, ov);
       tmem_wait();
       if (valid) {
-        uint4* yrow = reinterpret_cast<uint4*>(yg + (((size_t)b * L + tok) * H + h) * kP) + 4 * hf;
+        uint4* yrow = reinterpret_cast<uint4*>(yg + SSM_DIDX(kDbgSsdRow, (((size_t)b * L + tok) * H + h) * kP,
+                                                             kP, (size_t)p.B * L * H * kP)) +
+                      4 * hf;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const uint32_t w4[4] = {xraw[k].x, xraw[k].y, xraw[k].z, xraw[k].w};
@@ -478,7 +492,8 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
   if (p.final_state) {
 #pragma unroll
     for (int q = 0; q < kP / 2; ++q)
-      p.final_state[(((size_t)b * H + h) * kP + 32 * hf + q) * kNs + r] = Ht[q];
+      p.final_state[SSM_DIDX(kDbgSsdState, (((size_t)b * H + h) * kP + 32 * hf + q) * kNs + r, 1,
+                             (size_t)p.B * H * kP * kNs)] = Ht[q];
   }
   tc_fence_before();
   __syncthreads();
@@ -505,5 +520,7 @@ cudaError_t launch_ssd_fwd(const SsdArgs& a, cudaStream_t s) {
   ssd_fwd_kernel<<<dim3(a.H, a.B), kThreads, smem, s>>>(a, maps, tma);
   return cudaGetLastError();
 }
+
+SSM_DEBUG_TU(ssd_fwd)
 
 }  // namespace ssm

@@ -24,3 +24,15 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _device_index_checks(request):
+    """SSM_DEBUG_CHECKS=1 (SSM_LIBRARY naming the -DSSM_DEBUG build): a GPU
+    test must leave no failed device index check behind."""
+    yield
+    if os.environ.get("SSM_DEBUG_CHECKS") != "1" or "gpu" not in request.keywords:
+        return
+    import selective_state_space_35_b200 as ssm
+    rep = ssm.debug_report(reset=True)
+    assert rep["failures"] == 0, f"device index check failed: {rep}"

@@ -378,3 +378,34 @@ def test_ssd_bwd_param_validation(ssm):
     p = params(y=fake + 20480, chunk_states=fake + 8)
     assert L.ssm_ssd_fwd(ctypes.byref(p), None) == 1
     assert "aligned" in ssm.ssm_last_error()
+
+
+def test_release_build_has_no_debug_checks(ssm):
+    # the release library answers both debug calls before touching the device
+    with pytest.raises(ssm.SsmError) as e:
+        ssm.debug_report()
+    assert e.value.status == 2  # SSM_ERR_UNSUPPORTED
+    assert ssm.ssm_debug_selftest(None, 1, None) == 2
+
+
+def test_debug_library_builds_with_every_symbol():
+    """The -DSSM_DEBUG build compiles, exports what the header declares and
+    carries the checks (its report asks the device instead of refusing)."""
+    from selective_state_space_35_b200 import build
+    try:
+        lib_path = build.build_debug()
+    except RuntimeError as err:  # no nvcc on this machine
+        pytest.skip(str(err))
+    lib = ctypes.CDLL(lib_path)
+    for n in _declared():
+        assert hasattr(lib, n), n
+    from selective_state_space_35_b200 import _lib
+    info = _lib.ssm_debug_info()
+    info.struct_size = ctypes.sizeof(_lib.ssm_debug_info)
+    lib.ssm_debug_report.restype = ctypes.c_int
+    lib.ssm_debug_report.argtypes = [ctypes.POINTER(_lib.ssm_debug_info), ctypes.c_int]
+    st = lib.ssm_debug_report(ctypes.byref(info), 0)
+    assert st in (0, 3), st  # 0 with a device, SSM_ERR_CUDA without one; never unsupported
+    bad = _lib.ssm_debug_info()
+    bad.struct_size = 1
+    assert lib.ssm_debug_report(ctypes.byref(bad), 0) == 1

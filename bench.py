@@ -320,6 +320,8 @@ def main():
     ap.add_argument("--no-deterministic", action="store_true",
                     help="skip the measurement of the deterministic backward")
     ap.add_argument("--no-ssd", action="store_true", help="skip the Mamba-2 SSD forward measurement")
+    ap.add_argument("--no-fused", action="store_true",
+                    help="skip the fused conv + scan forward measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -456,6 +458,8 @@ def main():
         line["deterministic_bwd"] = deterministic_bench(layers[0], avg["scan_bwd"])
     if not args.no_ssd:
         line["ssd"] = ssd_bench(device, pk)
+    if not args.no_fused:
+        line["fused_fwd"] = fused_fwd_bench(layers[0], avg["conv1d_fwd"] + avg["scan_fwd"])
     line["peaks"] = {k: pk[k] for k in ("hbm_gbs", "bf16_tflops", "sm_max_mhz", "source")}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -629,6 +633,33 @@ def deterministic_bench(ly, bwd_ms, reps=5):
     return {"ms_per_layer": ms, "atomic_ms_per_layer": bwd_ms, "cost": ms / bwd_ms - 1.0,
             "workspace_bytes": nbytes, "other_grads_bitwise_equal_to_atomic": same,
             "launches": (reps + 1) * 3}
+
+
+def fused_fwd_bench(ly, sep_ms, reps=5):
+    """The fused conv + SiLU + scan forward (ssm_conv1d_scan_fwd) on the bench
+    layer, timed with CUDA events over `reps` launches after one warm-up,
+    beside the separate conv1d + scan forward of the timed step, whose u and
+    out it must reproduce bitwise."""
+    import torch
+    import selective_state_space_35_b200 as ssm
+    u, out, ws = torch.empty_like(ly.u), torch.empty_like(ly.out), torch.empty_like(ly.ws)
+
+    def run():
+        ssm.conv1d_scan_fwd(ly.x, ly.w, ly.cb, ly.delta, ly.A, ly.Bm, ly.Cm, u=u, out=out,
+                            workspace=ws, return_final_state=ly.shape.final_state, **ly.kw)
+
+    run()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    same = bool(torch.equal(u, ly.u) and torch.equal(out, ly.out))
+    del u, out, ws
+    return {"ms_per_layer": ms, "separate_ms_per_layer": sep_ms, "gain": 1.0 - ms / sep_ms,
+            "u_out_bitwise_equal_to_separate": same, "launches": (reps + 1) * 2}
 
 
 def complex_bench(device, ly, pk, reps=5):

@@ -45,8 +45,8 @@ SFU_EX2_PER_CLK_PER_SM = 16  # MUFU ex2 results per SM per clock (ssm_probe_ex2_
 
 # DRAM bytes (read + write) per launch of the current N = 16 scan kernels at
 # the 32K bench workload (one layer B2 D1536 N16 L32768 bf16, 11-warp CTAs),
-# from one ncu capture (profiles/scan16_kernels_B2_D1536_L32768.md); a kernel
-# changed since its capture has no entry.
+# from one ncu capture of these kernels at that shape (its summary is kept with
+# the profiles); a kernel changed since its capture has no entry.
 NCU_TRAFFIC = {"scan_bwd": 1832.669e6 + 597.325e6, "scan_fwd": 612.897e6 + 1155.971e6}
 
 

@@ -60,6 +60,7 @@ struct SsdSmem {
   unsigned char Hlo[kP * kNs * 2];  // its rounding remainder, rounded to bf16 (H_prev to ~2^-17)
   float lcs[kQ];
   float dt[kQ];
+  float bt[kQ];     // dt_j e^(lcs_k - lcs_j), k = j | 15: the end of j's 16-column block
   int ls[kQ];
   float wsum[4];
   int wmax[4];
@@ -365,6 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
     __syncthreads();
     la = sm.lcs[r];
     st = sm.ls[r];
+    if (hf == 0) sm.bt[r] = dt * __expf(sm.lcs[r | 15] - la);  // read after the next barrier
     const float lcsQ = sm.lcs[kQ - 1];
     const int lsQ = sm.ls[kQ - 1];
     // ---- B scaled by w_r = dt_r exp(lcs_Q-1 - lcs_r) [r >= ls_Q-1], MN-major ----
@@ -392,6 +394,11 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
     // the B tile is free: the next chunk's B rows into it
     if (c + 1 < nch) load_b(c + 1);
     // ---- columns 64 hf .. 64 hf + 63 of row r of M = (C B^T o L) dt (pair hi / lo) ----
+    // For a column j whose 16-column block ends (token k = j | 15) at or
+    // before row r, e^(lcs_r - lcs_j) is taken as e^(lcs_r - lcs_k) times the
+    // column's e^(lcs_k - lcs_j), both at most 1 since lcs does not increase
+    // along the chunk: one exponential per row and block instead of one per
+    // element. The block holding the diagonal keeps the direct form.
     uint32_t sraw[64];
     tmem_ld32(lane_row + 64 * hf, sraw);
     tmem_ld32(lane_row + 64 * hf + 32, sraw + 32);
@@ -403,10 +410,21 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
 #pragma unroll
       for (int e = 0; e < 32; e += 8) {
         float m[8], rr[8];
+        const int jg = j0 + e, kb = jg | 15;
+        if (jg > r) {  // above the diagonal
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const int j = j0 + e + q;
-          m[q] = (j >= st && j <= r) ? __uint_as_float(v[e + q]) * __expf(la - sm.lcs[j]) * sm.dt[j] : 0.0f;
+          for (int q = 0; q < 8; ++q) m[q] = 0.0f;
+        } else if (kb <= r) {
+          const float a = __expf(la - sm.lcs[kb]);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            m[q] = (jg + q >= st) ? __uint_as_float(v[e + q]) * (a * sm.bt[jg + q]) : 0.0f;
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const int j = jg + q;
+            m[q] = (j >= st && j <= r) ? __uint_as_float(v[e + q]) * __expf(la - sm.lcs[j]) * sm.dt[j] : 0.0f;
+          }
         }
         const uint4 hi = make_uint4(pack_bf16(m[0], m[1]), pack_bf16(m[2], m[3]), pack_bf16(m[4], m[5]),
                                     pack_bf16(m[6], m[7]));

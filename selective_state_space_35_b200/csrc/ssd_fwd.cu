@@ -386,6 +386,12 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
     if (t == 0) {
       umma_k128(tmem, sC, sB, kQ, false, 0, 0);
       umma_commit(&sm.bar);
+      // the products that do not need M run while the threads build it: C
+      // H_prev^T (H_prev as a bf16 pair) and S_c^T = (diag(w) B)^T x (the
+      // commit after Y_diag covers them)
+      umma_k128(tmem + 256, sC, sH, kP, false, 0, 1);
+      umma_k128(tmem + 256, sC, sHlo, kP, true, 0, 1);
+      umma_k128(tmem + 192, sBw, sX, kP, false, 1, 1, true);
     }
     bool ok = mbar_wait_bounded(&sm.bar, phase, p.status);
     phase ^= 1u;
@@ -443,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
     // the off-chunk term's row scale, applied in fp32 in the epilogue (C enters
     // the product as given: exact in bf16)
     const float cs = st < 0 ? __expf(la) : 0.0f;
-    // ---- Y_diag = M x, C H_prev^T (H_prev as a bf16 pair) and S_c^T = (diag(w) B)^T x ----
+    // ---- Y_diag = M x (M as a bf16 pair) ----
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     __syncthreads();
@@ -451,9 +457,6 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_kernel(const SsdArgs p, c
     if (t == 0) {
       umma_k128(tmem + 128, sM, sX, kP, false, 0, 1, true);
       umma_k128(tmem + 128, sMlo, sX, kP, true, 0, 1, true);
-      umma_k128(tmem + 256, sC, sH, kP, false, 0, 1);
-      umma_k128(tmem + 256, sC, sHlo, kP, true, 0, 1);
-      umma_k128(tmem + 192, sBw, sX, kP, false, 1, 1, true);
       umma_commit(&sm.bar);
     }
     ok = mbar_wait_bounded(&sm.bar, phase, p.status);

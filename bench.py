@@ -228,7 +228,13 @@ def oracle_sample(inp, seconds: float, threads: int):
     D, L = sh.D, sh.L
     rows_per = max(1, threads)
     done, t_total, d0 = 0, 0.0, 0
-    f64 = lambda t, sl: synth.bf16_bits_to_f32(t.bits[sl]).astype(np.float64)  # noqa: E731
+    bf16 = sh.dtype == "bf16"
+
+    def f64(t, sl):
+        v = synth.bf16_bits_to_f32(t.bits[sl]) if t.bits is not None else t.f32[sl]
+        return v.astype(np.float64)
+
+    stored = oracle.round_bf16 if bf16 else (lambda a: a)  # the activation dtype's rounding
     while t_total < seconds and d0 < D:
         d1 = min(D, d0 + rows_per)
         sl = np.s_[0:1, d0:d1, :]
@@ -239,11 +245,11 @@ def oracle_sample(inp, seconds: float, threads: int):
         w, cb = inp.conv_w[d0:d1], inp.conv_b[d0:d1]
         t0 = time.perf_counter()
         _, u = oracle.conv1d_fwd(x, w, cb, seq)
-        u = oracle.round_bf16(u)
+        u = stored(u)
         kw = dict(z=z, Dskip=Dk, delta_bias=db, seq_idx=seq, nthreads=threads)
         oracle.scan_fwd(u, dl, A, Bm, Cm, **kw)
         g = oracle.scan_bwd(u, dl, A, Bm, Cm, go, **kw)
-        oracle.conv1d_bwd(x, w, cb, seq, oracle.round_bf16(g["du"]))
+        oracle.conv1d_bwd(x, w, cb, seq, stored(g["du"]))
         t_total += time.perf_counter() - t0
         done += d1 - d0
         d0 = d1
@@ -304,7 +310,8 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", type=int, default=3)
+    ap.add_argument("--config", type=int, default=3, choices=(2, 3, 4, 5),
+                    help="bench workload (the bf16 configs; 1 is a parity case only)")
     ap.add_argument("--n-splits", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0, help="limit the layer count (profiling)")
     ap.add_argument("--e2e-steps", type=int, default=10)
